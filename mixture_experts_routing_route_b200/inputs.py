@@ -1,0 +1,196 @@
+"""Seeded synthetic inputs for the MoE-layer forward.
+
+This module only draws random numbers and fixes tensor shapes. It holds none of
+the layer's arithmetic (no routing, no sorting, no FFN), so that the CPU oracle
+and the CUDA path can both be fed the very same bytes from here without sharing
+any computation.
+
+Workloads (all synthetic, no dataset is involved):
+
+* ``tiny_fp32``     T=256  d=64   E=4   k=1 F=128   GELU   fp32, cf 1.25
+* ``mixtral``       T=4096 d=4096 E=8   k=2 F=14336 SwiGLU bf16, dropless
+* ``fine_grained``  T=4096 d=4096 E=256 k=8 F=2048  SwiGLU bf16, dropless
+* ``capacity_skew`` T=16384 d=1024 E=64 k=2 F=4096  GELU   bf16, cf 1.0,
+  logit bias b_e = 1.5*ln(1/(e+1)) (Zipf-like skew)
+* ``long_skewed``   T=32768 d=4096 E=8  k=2 F=14336 SwiGLU bf16, logit bias
+  (beta, 0, ..., 0) so that expert 0 gets about 40% of the slots; dropless and
+  cf 1.25 variants.
+
+Distributions: x ~ N(0, 1); router and expert weights ~ N(0, 0.02) (tiny_fp32:
+N(0, 0.1)). Every tensor is drawn from torch's CPU generator, one generator per
+(seed, tensor, expert) so that slices can be drawn in parallel threads and any
+expert's weights can be regenerated alone. bf16 tensors are the fp32 draw
+rounded to nearest-even by ``Tensor.to(torch.bfloat16)``.
+"""
+from __future__ import annotations
+
+import math
+from concurrent.futures import ThreadPoolExecutor
+from dataclasses import dataclass, field, replace
+from typing import Optional
+
+import torch
+
+# Logit bias on expert 0 that gives it ~40% of the slots on the long_skewed
+# workload's seeded x and router weight. Found by bisection with the CPU oracle
+# (tests/golden/calibrate_long_skewed_bias.py); share at this value: see the
+# fixture tests/golden/long_skewed_bias.json.
+LONG_SKEWED_BETA = 2.15625
+
+ACT_GELU = "gelu"
+ACT_SWIGLU = "swiglu"
+
+
+@dataclass(frozen=True)
+class MoeShape:
+    """Shape and recipe of one MoE-layer workload."""
+
+    name: str
+    T: int
+    d: int
+    E: int
+    k: int
+    F: int
+    act: str = ACT_SWIGLU
+    dtype: str = "bf16"          # "bf16" or "f32"
+    cf: float = 0.0              # capacity factor; 0 means dropless
+    x_std: float = 1.0
+    w_std: float = 0.02
+    bias: str = "none"           # "none", "zipf" or "expert0"
+    seed: int = 1000
+
+    def with_(self, **kw) -> "MoeShape":
+        return replace(self, **kw)
+
+    @property
+    def slots(self) -> int:
+        return self.T * self.k
+
+
+CONFIGS = {
+    "tiny_fp32": MoeShape("tiny_fp32", T=256, d=64, E=4, k=1, F=128, act=ACT_GELU,
+                          dtype="f32", cf=1.25, w_std=0.1, seed=1001),
+    "mixtral": MoeShape("mixtral", T=4096, d=4096, E=8, k=2, F=14336, seed=1002),
+    "fine_grained": MoeShape("fine_grained", T=4096, d=4096, E=256, k=8, F=2048, seed=1003),
+    "capacity_skew": MoeShape("capacity_skew", T=16384, d=1024, E=64, k=2, F=4096,
+                              act=ACT_GELU, cf=1.0, bias="zipf", seed=1004),
+    "long_skewed": MoeShape("long_skewed", T=32768, d=4096, E=8, k=2, F=14336,
+                            bias="expert0", seed=1005),
+    "long_skewed_cf": MoeShape("long_skewed_cf", T=32768, d=4096, E=8, k=2, F=14336,
+                               cf=1.25, bias="expert0", seed=1005),
+}
+
+# Tensor ids inside one seed's stream family.
+_X, _WG, _W1, _W3, _W2 = 0, 1, 2, 3, 4
+
+
+def _gen(seed: int, tensor: int, part: int) -> torch.Generator:
+    return torch.Generator().manual_seed(seed * 1_000_003 + tensor * 10_007 + part)
+
+
+def _draw(shape, std, seed, tensor, part, dtype):
+    g = _gen(seed, tensor, part)
+    t = torch.randn(*shape, generator=g, dtype=torch.float32)
+    if std != 1.0:
+        t.mul_(std)
+    return t.to(dtype)
+
+
+def torch_dtype(name: str) -> torch.dtype:
+    return {"bf16": torch.bfloat16, "f32": torch.float32}[name]
+
+
+def bias_vector(shape: MoeShape) -> Optional[torch.Tensor]:
+    """fp32 logit bias [E] of the workload, or None."""
+    if shape.bias == "none":
+        return None
+    if shape.bias == "zipf":
+        return torch.tensor([1.5 * math.log(1.0 / (e + 1)) for e in range(shape.E)],
+                            dtype=torch.float32)
+    if shape.bias == "expert0":
+        b = torch.zeros(shape.E, dtype=torch.float32)
+        b[0] = LONG_SKEWED_BETA
+        return b
+    raise ValueError(shape.bias)
+
+
+@dataclass
+class MoeInputs:
+    shape: MoeShape
+    x: torch.Tensor            # [T, d]
+    wg: torch.Tensor           # [d, E]
+    bias: Optional[torch.Tensor]
+    w1: torch.Tensor           # [E, d, F]  (W_gate for SwiGLU, W1 for GELU)
+    w3: Optional[torch.Tensor] # [E, d, F]  (W_up for SwiGLU) or None
+    w2: torch.Tensor           # [E, F, d]  (W_down / W2)
+    extra: dict = field(default_factory=dict)
+
+
+def make_x(shape: MoeShape, threads: int = 8) -> torch.Tensor:
+    dt = torch_dtype(shape.dtype)
+    # x is drawn in row blocks of 1024 tokens so large T draws in parallel.
+    blocks = [(i, min(1024, shape.T - i)) for i in range(0, shape.T, 1024)]
+    with ThreadPoolExecutor(threads) as ex:
+        parts = list(ex.map(lambda b: _draw((b[1], shape.d), shape.x_std, shape.seed, _X, b[0], dt),
+                            blocks))
+    return torch.cat(parts, 0) if parts else torch.empty(0, shape.d, dtype=dt)
+
+
+def make_expert_weights(shape: MoeShape, tensor: int, rows: int, cols: int,
+                        threads: int = 8) -> torch.Tensor:
+    dt = torch_dtype(shape.dtype)
+    out = torch.empty(shape.E, rows, cols, dtype=dt)
+
+    def one(e):
+        out[e] = _draw((rows, cols), shape.w_std, shape.seed, tensor, e, dt)
+
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(one, range(shape.E)))
+    return out
+
+
+def make_inputs(shape: MoeShape, threads: int = 8, experts: bool = True) -> MoeInputs:
+    """Draw every input of ``shape`` on the host (CPU tensors)."""
+    dt = torch_dtype(shape.dtype)
+    x = make_x(shape, threads)
+    wg = _draw((shape.d, shape.E), shape.w_std, shape.seed, _WG, 0, dt)
+    bias = bias_vector(shape)
+    if experts:
+        w1 = make_expert_weights(shape, _W1, shape.d, shape.F, threads)
+        w3 = make_expert_weights(shape, _W3, shape.d, shape.F, threads) \
+            if shape.act == ACT_SWIGLU else None
+        w2 = make_expert_weights(shape, _W2, shape.F, shape.d, threads)
+    else:
+        w1 = w3 = w2 = None
+    return MoeInputs(shape, x, wg, bias, w1, w3, w2)
+
+
+def worked_example_a() -> MoeInputs:
+    """The 8-token / 4-expert / top-1 case whose per-expert counts are 3/0/4/1.
+
+    The page ("MegaBlocks: why MoE is hard", section 2) gives only the counts,
+    not which token goes where. The assignment used here is
+    ``[2, 0, 2, 3, 0, 2, 0, 2]``; it is forced through the router by d = 4,
+    W_g = I_4 and x_t = 5 * onehot(e_t), so that expert e_t has logit 5 and
+    every other expert logit 0.
+    """
+    ids = [2, 0, 2, 3, 0, 2, 0, 2]
+    T, E, d = 8, 4, 4
+    shape = MoeShape("worked_example_a", T=T, d=d, E=E, k=1, F=64, act=ACT_GELU,
+                     dtype="f32", cf=0.0, w_std=0.1, seed=1000)
+    x = torch.zeros(T, d, dtype=torch.float32)
+    for t, e in enumerate(ids):
+        x[t, e] = 5.0
+    wg = torch.eye(d, E, dtype=torch.float32)
+    w1 = make_expert_weights(shape, _W1, d, shape.F)
+    w2 = make_expert_weights(shape, _W2, shape.F, d)
+    return MoeInputs(shape, x, wg, None, w1, None, w2, extra={"ids": ids})
+
+
+def small_case(name: str, T: int, d: int, E: int, k: int, F: int, act: str,
+               dtype: str = "bf16", cf: float = 0.0, bias: str = "none",
+               seed: int = 7, w_std: float = 0.02) -> MoeInputs:
+    """A reduced-size workload with the same distributions, for parity tests."""
+    shape = MoeShape(name, T=T, d=d, E=E, k=k, F=F, act=act, dtype=dtype, cf=cf,
+                     bias=bias, seed=seed, w_std=w_std)
+    return make_inputs(shape)

@@ -1,0 +1,343 @@
+"""CPU oracle for the single-GPU MoE-layer forward (route, permute, gather,
+expert FFN, combine).
+
+TEST INFRASTRUCTURE. This module is the plain, slow, obviously correct
+reference that the CUDA path is checked against. Only the tests, the package's
+smoke check and the benchmark's CPU-baseline / reference arm may import it. The
+product path never calls it, and it shares no code with the CUDA kernels: it
+imports numpy and scipy only.
+
+Everything is float64 unless stated. Inputs are numpy arrays; bf16 inputs are
+passed already widened to float32 (the widening is exact).
+
+Sources (page title, then section):
+
+* "ops-transformer MoE operators" blog (aicoding.csdn.net), 原理 Steps 1-4 and
+  实现 (MoEGatingForward: softmax, top-k by selection, renormalise the K
+  weights to sum 1).
+* "MoE Router: who decides which expert a token goes to" (lpnh.cn): gate is
+  Linear(hidden, E, bias=False), softmax, top-k, renormalise; capacity
+  limit with dropped tokens taking the residual path.
+* "MegaBlocks 01 - why MoE is hard" (ai-reference-codex), section 1 (router
+  = bias-free linear + softmax + top-k), section 3 (capacity
+  C = cf * tokens * top_k / E, overflow dropped, dropped output zero), section
+  4.1 (sort by expert id, histogram, inclusive cumsum = bins; sort only the
+  low ceil(log2 E) key bits), section 4.2 (capacity formula with int()),
+  section 4.3 (gather into expert-contiguous rows, bmm -> activation -> bmm,
+  weights [E, hs, ffn], scatter multiplied by the router weight and summed
+  over top-k), section 4.5 (which rows get dropped), section 5 (top-k sum).
+* "Integrating MoE into your model with Colossal-AI" (blog.gitcode.com), step
+  2: gate logits cast to fp32 before routing; gated MLP option.
+
+Readings where the pages are silent or disagree (the same list is kept with
+the design notes):
+
+* No learned router bias. An optional fixed fp32 logit bias b[E] is added
+  before the softmax (it is how the skewed workloads are made).
+* Top-k selects on the fp32 logits (the precision the kernel routes in);
+  softmax is monotone, so this is the order the pages' top-k on softmax
+  scores gives, with exact ties broken toward the lower expert index.
+* Capacity C = int(cf * (k * T / E)) truncated toward zero; cf <= 0 means
+  dropless. Drop order is arrival order: flat slot s = t * k + j ascending.
+  A dropped slot contributes zero; the surviving weights are not
+  renormalised again.
+* Auxiliary loss aux = E * sum_i f_i * P_i, f_i = (slots routed to i before
+  any drop) / (T * k), P_i = mean over tokens of the full softmax p[t, i].
+* GELU is the exact erf form; SwiGLU is silu(x W_gate) * (x W_up), then
+  W_down; silu(z) = z / (1 + exp(-z)).
+* The router weight multiplies the expert output in the combine, in the
+  combine's own precision, summed over j = 0..k-1 in ascending order.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+from scipy.special import erf as _erf
+
+__all__ = [
+    "gate_logits", "softmax_rows", "topk_select", "renormalise", "aux_loss",
+    "near_tie_tokens", "route", "capacity", "sort_end_bit", "permute", "gather",
+    "activation", "expert_ffn", "combine", "forward", "forward_tokens",
+]
+
+
+# --------------------------------------------------------------------------
+# route
+# --------------------------------------------------------------------------
+
+def gate_logits(x, wg, bias=None):
+    """Router gate: logits[t, e] = sum_i x[t, i] * Wg[i, e] (+ b[e]).
+
+    "MoE Router" page: the gate is Linear(hidden, E) without bias; Colossal-AI
+    step 2: logits are taken to fp32 before routing. Returns float64 [T, E]
+    (exact dot products up to float64 rounding); callers round to float32.
+    """
+    l = np.asarray(x, dtype=np.float64) @ np.asarray(wg, dtype=np.float64)
+    if bias is not None:
+        l = l + np.asarray(bias, dtype=np.float64)[None, :]
+    return l
+
+
+def softmax_rows(logits):
+    """p[t, :] = softmax(logits[t, :]) over the E experts, float64.
+
+    ops-transformer blog, 实现 step 1 (softmax over num_experts).
+    """
+    l = np.asarray(logits, dtype=np.float64)
+    m = l.max(axis=1, keepdims=True)
+    e = np.exp(l - m)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def topk_select(logits32, k):
+    """Indices of the k largest logits per token, largest first.
+
+    ops-transformer blog, 实现 step 2 (top-K over the E scores). Equal values
+    are ordered by the lower expert index (a stable ordering of -logit). The
+    comparison is made on the float32 values given.
+    """
+    l = np.asarray(logits32, dtype=np.float32).astype(np.float64)
+    order = np.argsort(-l, axis=1, kind="stable")
+    return order[:, :k].astype(np.int32)
+
+
+def renormalise(probs, idx):
+    """w[t, j] = p[t, idx[t, j]] / sum_j' p[t, idx[t, j']].
+
+    ops-transformer blog, 实现 step 3; "MoE Router" page (the K chosen
+    weights are made to sum to 1). float64.
+    """
+    p = np.asarray(probs, dtype=np.float64)
+    sel = np.take_along_axis(p, np.asarray(idx, dtype=np.int64), axis=1)
+    return sel / sel.sum(axis=1, keepdims=True)
+
+
+def aux_loss(probs, idx, E):
+    """Load-balance loss E * sum_i f_i * P_i.
+
+    The pages name the loss (ops-transformer blog 坑1; CANN page 2.2; "MoE
+    Router": every expert should get about 1/E of the tokens) but print no
+    formula; the Switch/GShard form is used. f_i counts slots routed to expert
+    i before any capacity drop, over all T * k slots; P_i is the mean routing
+    probability of expert i over the T tokens.
+    """
+    p = np.asarray(probs, dtype=np.float64)
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    f = np.bincount(idx.reshape(-1), minlength=E).astype(np.float64) / (T * k)
+    P = p.mean(axis=0)
+    return float(E * np.sum(f * P))
+
+
+def near_tie_tokens(logits32, k, eps=1e-3):
+    """Tokens whose k-th and (k+1)-th largest logits are closer than eps.
+
+    Their top-k set can flip under a different (equally valid) float
+    summation order, so end-to-end index checks leave them out.
+    """
+    l = np.sort(np.asarray(logits32, dtype=np.float64), axis=1)[:, ::-1]
+    if k >= l.shape[1]:
+        return np.zeros(l.shape[0], dtype=bool)
+    return (l[:, k - 1] - l[:, k]) < eps
+
+
+def route(x, wg, bias, k):
+    """Router stage: logits, softmax, top-k, renormalised weights, aux loss."""
+    l64 = gate_logits(x, wg, bias)
+    logits32 = l64.astype(np.float32)
+    p64 = softmax_rows(l64)
+    idx = topk_select(logits32, k)
+    w64 = renormalise(p64, idx)
+    E = l64.shape[1]
+    return {
+        "logits": logits32,
+        "probs64": p64,
+        "probs": p64.astype(np.float32),
+        "topk_idx": idx,
+        "topk_w64": w64,
+        "topk_w": w64.astype(np.float32),
+        "aux": aux_loss(p64, idx, E),
+        "near_tie": near_tie_tokens(logits32, k),
+    }
+
+
+# --------------------------------------------------------------------------
+# permute
+# --------------------------------------------------------------------------
+
+def capacity(cf, k, T, E):
+    """Expert capacity C = int(cf * (k * T / E)), or None when dropless.
+
+    MegaBlocks page, sections 3 and 4.2 (world size 1). cf <= 0 means no
+    capacity limit.
+    """
+    if cf is None or cf <= 0:
+        return None
+    return int(cf * (k * T / E))
+
+
+def sort_end_bit(E):
+    """Number of low key bits the sort needs: max(ceil(log2 E), 1).
+
+    MegaBlocks page, section 4.1.
+    """
+    return max(int(math.ceil(math.log2(E))), 1) if E > 1 else 1
+
+
+def permute(idx, E, cap=None):
+    """Sorting metadata, capacity drop and the row map of the gathered layout.
+
+    MegaBlocks page, sections 4.1 (stable sort of the flat top-k expert ids,
+    histogram, inclusive cumsum = bins), 3/4.2 (capacity), 4.4/4.5 (an expert
+    keeps the first C of its slots in sorted order; the rest are dropped).
+
+    Layout of the gathered rows: the kept slots of expert 0, then of expert 1,
+    ... each expert's slots in ascending flat-slot order, no padding. So expert
+    e owns rows [seg_offsets[e], seg_offsets[e+1]).
+    """
+    idx = np.asarray(idx, dtype=np.int64)
+    T, k = idx.shape
+    S = T * k
+    flat = idx.reshape(-1)
+    if np.any((flat < 0) | (flat >= E)):
+        raise ValueError("expert id out of range")
+    mask = (1 << sort_end_bit(E)) - 1
+    key = flat & mask
+    counts = np.bincount(flat, minlength=E).astype(np.int64)
+    bins = np.cumsum(counts)
+    sorted_slot = np.argsort(key, kind="stable")
+    start = bins - counts                      # first sorted position of each expert
+    rank = np.empty(S, dtype=np.int64)
+    rank[sorted_slot] = np.arange(S) - start[flat[sorted_slot]]
+    if cap is None:
+        drop = np.zeros(S, dtype=bool)
+        kept = counts.copy()
+    else:
+        drop = rank >= cap
+        kept = np.minimum(counts, cap)
+    seg_offsets = np.concatenate([[0], np.cumsum(kept)])
+    slot_to_row = np.where(drop, -1, seg_offsets[flat] + rank)
+    R = int(seg_offsets[-1])
+    row_slot = np.empty(R, dtype=np.int64)
+    keep = ~drop
+    row_slot[slot_to_row[keep]] = np.nonzero(keep)[0]
+    return {
+        "counts": counts.astype(np.int32),
+        "bins": bins.astype(np.int32),
+        "sorted_slot": sorted_slot.astype(np.int32),
+        "rank": rank.astype(np.int32),
+        "drop": drop.astype(np.uint8),
+        "kept_counts": kept.astype(np.int32),
+        "seg_offsets": seg_offsets.astype(np.int32),
+        "slot_to_row": slot_to_row.astype(np.int32),
+        "row_slot": row_slot.astype(np.int32),
+        "rows": R,
+    }
+
+
+# --------------------------------------------------------------------------
+# gather / expert FFN / combine
+# --------------------------------------------------------------------------
+
+def gather(x, row_slot, k):
+    """x_perm[r] = x[row_slot[r] // k] (MegaBlocks page, section 4.3: the
+    token of flat slot s is s // top_k)."""
+    x = np.asarray(x)
+    return x[np.asarray(row_slot, dtype=np.int64) // k]
+
+
+def activation(z, act, z_up=None):
+    """GELU (exact erf form) or SwiGLU's silu(z_gate) * z_up, float64."""
+    z = np.asarray(z, dtype=np.float64)
+    if act == "gelu":
+        return 0.5 * z * (1.0 + _erf(z / math.sqrt(2.0)))
+    if act == "swiglu":
+        return (z / (1.0 + np.exp(-z))) * np.asarray(z_up, dtype=np.float64)
+    raise ValueError(act)
+
+
+def _expert_mlp(xe, e, w1, w3, w2, act):
+    xe = np.asarray(xe, dtype=np.float64)
+    z1 = xe @ np.asarray(w1[e], dtype=np.float64)
+    z3 = xe @ np.asarray(w3[e], dtype=np.float64) if act == "swiglu" else None
+    h = activation(z1, act, z3)
+    return h @ np.asarray(w2[e], dtype=np.float64)
+
+
+def expert_ffn(x_perm, seg_offsets, w1, w3, w2, act):
+    """Per-expert MLP over each expert's rows: bmm -> activation -> bmm.
+
+    MegaBlocks page, section 4.3 (weights [E, hs, ffn]); the gated (SwiGLU)
+    form follows the CANN operator list and Colossal-AI's gated-MLP option.
+    w1 is W1 (GELU) or W_gate (SwiGLU), w3 is W_up (SwiGLU only), w2 is
+    W2 / W_down. Returns float64 [R, d].
+    """
+    seg = np.asarray(seg_offsets, dtype=np.int64)
+    E = len(seg) - 1
+    y = np.zeros((int(seg[-1]), np.asarray(w2[0]).shape[1]), dtype=np.float64)
+    for e in range(E):
+        a, b = int(seg[e]), int(seg[e + 1])
+        if b > a:
+            y[a:b] = _expert_mlp(x_perm[a:b], e, w1, w3, w2, act)
+    return y
+
+
+def combine(y_perm, topk_w, slot_to_row, T, k):
+    """out[t] = sum over j = 0..k-1 of w[t, j] * y_perm[row(t, j)], dropped
+    slots skipped; a token with every slot dropped gets a zero row.
+
+    ops-transformer blog, 原理 step 4 (weighted sum); MegaBlocks page,
+    sections 4.3 and 5 (multiply by the router weight, sum over top-k).
+    """
+    y = np.asarray(y_perm, dtype=np.float64)
+    w = np.asarray(topk_w, dtype=np.float64).reshape(T, k)
+    rows = np.asarray(slot_to_row, dtype=np.int64).reshape(T, k)
+    out = np.zeros((T, y.shape[1]), dtype=np.float64)
+    for j in range(k):
+        r = rows[:, j]
+        m = r >= 0
+        out[m] += w[m, j, None] * y[r[m]]
+    return out
+
+
+# --------------------------------------------------------------------------
+# whole layer
+# --------------------------------------------------------------------------
+
+def forward(x, wg, bias, w1, w3, w2, k, act, cf=0.0, topk_idx=None, topk_w=None):
+    """The whole MoE-layer forward. If topk_idx (and topk_w) are given, the
+    permute/FFN/combine run on that routing instead of the oracle's own."""
+    x = np.asarray(x)
+    T = x.shape[0]
+    E = np.asarray(wg).shape[1]
+    r = route(x, wg, bias, k)
+    idx = r["topk_idx"] if topk_idx is None else np.asarray(topk_idx)
+    w = r["topk_w64"] if topk_w is None else np.asarray(topk_w, dtype=np.float64)
+    pm = permute(idx, E, capacity(cf, k, T, E))
+    xp = gather(x, pm["row_slot"], k)
+    y = expert_ffn(xp, pm["seg_offsets"], w1, w3, w2, act)
+    out = combine(y, w, pm["slot_to_row"], T, k)
+    return {"route": r, "permute": pm, "x_perm": xp, "y_perm": y, "out": out}
+
+
+def forward_tokens(x, tokens, topk_idx, topk_w, slot_to_row, w1, w3, w2, act):
+    """Layer output for a subset of tokens only, from a given routing and
+    drop map (slot_to_row < 0 marks a dropped slot). Used to check full-size
+    runs on sampled tokens: each sampled token's kept (token, expert) pairs
+    go through that expert's MLP. Returns float64 [len(tokens), d]."""
+    x = np.asarray(x)
+    T = x.shape[0]
+    idx = np.asarray(topk_idx).reshape(T, -1)
+    k = idx.shape[1]
+    w = np.asarray(topk_w, dtype=np.float64).reshape(T, k)
+    rows = np.asarray(slot_to_row).reshape(T, k)
+    tokens = np.asarray(tokens, dtype=np.int64)
+    out = np.zeros((len(tokens), np.asarray(w2[0]).shape[1]), dtype=np.float64)
+    pairs = [(i, int(t), j) for i, t in enumerate(tokens) for j in range(k) if rows[t, j] >= 0]
+    for e in sorted({int(idx[t, j]) for _, t, j in pairs}):
+        mine = [(i, t, j) for i, t, j in pairs if int(idx[t, j]) == e]
+        y = _expert_mlp(x[[t for _, t, _ in mine]], e, w1, w3, w2, act)
+        for (i, t, j), yr in zip(mine, y):
+            out[i] += w[t, j] * yr
+    return out

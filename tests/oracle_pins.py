@@ -1,0 +1,352 @@
+"""Pins for the CPU oracle: checks against facts the pages and mathematics
+fix, not against the oracle's own formulas.
+
+Each ``pin_*`` takes the oracle namespace ``o`` and raises AssertionError when
+the oracle is wrong. tests/test_oracle_pins.py runs every pin on the real
+oracle; tests/test_oracle_mutations.py plants mistakes in a copy of the oracle
+and checks that some pin fails for each of them.
+"""
+from __future__ import annotations
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import torch
+import torch.nn.functional as Fn
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ----------------------------------------------------------------------------
+# brute-force helpers (pure Python loops on tiny inputs)
+# ----------------------------------------------------------------------------
+
+def _bf_topk(row, k):
+    """k largest, largest first, ties to the lower index, by explicit selection."""
+    taken = []
+    for _ in range(k):
+        best = None
+        for e, v in enumerate(row):
+            if e in taken:
+                continue
+            if best is None or v > row[best]:
+                best = e
+        taken.append(best)
+    return taken
+
+
+def _bf_permute(flat, E, cap):
+    """Counting, ranks, drops and rows by walking the slots in arrival order."""
+    seen = [0] * E
+    rank = []
+    for e in flat:
+        rank.append(seen[e])
+        seen[e] += 1
+    counts = seen
+    bins = list(itertools.accumulate(counts))
+    buckets = [[] for _ in range(E)]
+    for s, e in enumerate(flat):
+        buckets[e].append(s)
+    sorted_slot = [s for b in buckets for s in b]
+    drop = [cap is not None and r >= cap for r in rank]
+    kept = [min(c, cap) if cap is not None else c for c in counts]
+    seg = [0]
+    for c in kept:
+        seg.append(seg[-1] + c)
+    slot_to_row = [-1 if drop[s] else seg[e] + rank[s] for s, e in enumerate(flat)]
+    return counts, bins, sorted_slot, rank, drop, kept, seg, slot_to_row
+
+
+# ----------------------------------------------------------------------------
+# pins
+# ----------------------------------------------------------------------------
+
+def pin_example_a(o):
+    """MegaBlocks page section 2: counts 3/0/4/1 from the forced routing."""
+    g = _golden("worked_example_a.json")
+    ids = [2, 0, 2, 3, 0, 2, 0, 2]
+    x = np.zeros((8, 4))
+    for t, e in enumerate(ids):
+        x[t, e] = 5.0
+    r = o.route(x, np.eye(4), None, 1)
+    assert r["topk_idx"][:, 0].tolist() == ids
+    assert np.all(r["topk_w"] == 1.0)
+    pm = o.permute(r["topk_idx"], 4, o.capacity(0.0, 1, 8, 4))
+    assert pm["counts"].tolist() == g["counts"]
+    assert pm["bins"].tolist() == list(itertools.accumulate(g["counts"]))
+    assert np.diff(pm["seg_offsets"]).tolist() == g["gemm_rows"]
+
+
+def pin_example_b(o):
+    """ops-transformer blog 原理: picks experts 0 and 6, weights softmax([0.9, 0.7])."""
+    g = _golden("worked_example_b.json")
+    a = 1.0 / (1.0 + math.exp(-(0.9 - 0.7)))    # closed form of softmax([0.9,0.7])[0]
+    for seed in range(20):
+        rng = _rng(seed)
+        s = rng.uniform(-3.0, g["filler_upper_bound"] - 1e-3, size=g["E"])
+        for e, v in g["known_scores"].items():
+            s[int(e)] = v
+        r = o.route(s[None, :], np.eye(g["E"]), None, g["k"])
+        assert r["topk_idx"][0].tolist() == g["selected"]
+        w = r["topk_w64"][0]
+        assert abs(w[0] - a) < 1e-12 and abs(w[1] - (1 - a)) < 1e-12
+    assert abs(a - 0.549834) < 5e-7
+
+
+def pin_topk_vs_torch(o):
+    """Top-k on tie-free inputs equals torch.topk (largest first)."""
+    rng = _rng(1)
+    for E, k in [(4, 1), (8, 2), (64, 2), (256, 8), (5, 5)]:
+        l = rng.standard_normal((50, E)).astype(np.float32)
+        ref = torch.topk(torch.from_numpy(l), k, dim=1).indices.numpy()
+        assert np.array_equal(o.topk_select(l, k), ref)
+
+
+def pin_topk_ties(o):
+    """Exact ties go to the lower expert index (brute-force selection)."""
+    rng = _rng(2)
+    for _ in range(200):
+        E = int(rng.integers(2, 9))
+        k = int(rng.integers(1, E + 1))
+        row = rng.integers(-2, 3, size=E).astype(np.float32)  # many exact ties
+        assert o.topk_select(row[None, :], k)[0].tolist() == _bf_topk(row.tolist(), k)
+    z = np.array([[0.0, -0.0, 0.0, -0.0]], dtype=np.float32)  # +0 and -0 compare equal
+    assert o.topk_select(z, 2)[0].tolist() == [0, 1]
+
+
+def pin_softmax_vs_torch(o):
+    rng = _rng(3)
+    l = rng.standard_normal((40, 16)) * 4
+    ref = torch.softmax(torch.from_numpy(l), dim=1).numpy()
+    assert np.allclose(o.softmax_rows(l), ref, rtol=1e-13, atol=0)
+    assert np.allclose(o.softmax_rows(l + 123.0), ref, rtol=1e-12, atol=0)
+
+
+def pin_renormalise(o):
+    rng = _rng(4)
+    x = rng.standard_normal((30, 16))
+    wg = rng.standard_normal((16, 8))
+    for k in (1, 2, 3, 8):
+        r = o.route(x, wg, None, k)
+        assert np.allclose(r["topk_w64"].sum(1), 1.0, rtol=0, atol=1e-14)
+        if k == 1:
+            assert np.all(r["topk_w"] == 1.0)
+        # weights are the selected probabilities scaled by one factor per token
+        sel = np.take_along_axis(torch.softmax(torch.from_numpy(x @ wg), 1).numpy(),
+                                 r["topk_idx"].astype(np.int64), 1)
+        assert np.allclose(r["topk_w64"], sel / sel.sum(1, keepdims=True), rtol=1e-12)
+    # changing an unselected logit changes nothing after renormalisation
+    l = np.array([[3.0, 1.0, 2.5, -1.0]])
+    l2 = l.copy()
+    l2[0, 3] = 0.9
+    w1 = o.renormalise(o.softmax_rows(l), [[0, 2]])
+    w2 = o.renormalise(o.softmax_rows(l2), [[0, 2]])
+    assert np.allclose(w1, w2, rtol=1e-14)
+
+
+def pin_aux(o):
+    """Balanced routing with uniform probabilities gives 1; collapse gives E;
+    small cases match a double loop."""
+    E, T, k = 4, 8, 2
+    probs = np.full((T, E), 1.0 / E)
+    idx = np.array([[t % E, (t + 1) % E] for t in range(T)])
+    assert abs(o.aux_loss(probs, idx, E) - 1.0) < 1e-15
+    onehot = np.zeros((T, E))
+    onehot[:, 2] = 1.0
+    assert abs(o.aux_loss(onehot, np.full((T, 1), 2), E) - E) < 1e-15
+    rng = _rng(5)
+    for _ in range(20):
+        E = int(rng.integers(2, 7))
+        T = int(rng.integers(1, 9))
+        k = int(rng.integers(1, E + 1))
+        p = rng.random((T, E))
+        p /= p.sum(1, keepdims=True)
+        idx = np.array([rng.permutation(E)[:k] for _ in range(T)])
+        tot = 0.0
+        for i in range(E):
+            f = sum(1 for t in range(T) for j in range(k) if idx[t][j] == i) / (T * k)
+            P = sum(p[t][i] for t in range(T)) / T
+            tot += f * P
+        assert abs(o.aux_loss(p, idx, E) - E * tot) < 1e-12
+
+
+def pin_capacity(o):
+    for c in _golden("capacity_values.json")["cases"]:
+        assert o.capacity(c["cf"], c["k"], c["T"], c["E"]) == c["C"], c
+    assert o.capacity(0.0, 2, 100, 4) is None
+    assert o.sort_end_bit(1) == 1 and o.sort_end_bit(2) == 1
+    assert o.sort_end_bit(8) == 3 and o.sort_end_bit(64) == 6
+    assert o.sort_end_bit(65) == 7 and o.sort_end_bit(256) == 8
+
+
+def pin_permute_bruteforce(o):
+    """Every capacity on tiny inputs matches the arrival-order walk."""
+    rng = _rng(6)
+    for _ in range(60):
+        T = int(rng.integers(1, 17))
+        E = int(rng.integers(1, 6))
+        k = int(rng.integers(1, min(3, E) + 1))
+        idx = np.array([rng.permutation(E)[:k] for _ in range(T)])
+        flat = idx.reshape(-1).tolist()
+        for cap in [None] + list(range(0, T * k + 1)):
+            pm = o.permute(idx, E, cap)
+            counts, bins, ss, rank, drop, kept, seg, s2r = _bf_permute(flat, E, cap)
+            assert pm["counts"].tolist() == counts
+            assert pm["bins"].tolist() == bins
+            assert pm["sorted_slot"].tolist() == ss
+            assert pm["rank"].tolist() == rank
+            assert pm["drop"].astype(bool).tolist() == drop
+            assert pm["kept_counts"].tolist() == kept
+            assert pm["seg_offsets"].tolist() == seg
+            assert pm["slot_to_row"].tolist() == s2r
+            for r, s in enumerate(pm["row_slot"].tolist()):
+                assert s2r[s] == r
+
+
+def pin_permute_vs_torch_sort(o):
+    """Stable sort order equals torch.sort(stable=True); a bijection; forced
+    uniform assignment (slot s -> expert s mod E) gives equal counts."""
+    rng = _rng(7)
+    for E in (3, 8, 64, 256):
+        idx = rng.integers(0, E, size=(500, 2))
+        pm = o.permute(idx, E, None)
+        ref = torch.sort(torch.from_numpy(idx.reshape(-1)), stable=True).indices.numpy()
+        assert np.array_equal(pm["sorted_slot"], ref)
+        assert np.array_equal(np.sort(pm["sorted_slot"]), np.arange(idx.size))
+    T, k, E = 64, 2, 8
+    forced = (np.arange(T * k) % E).reshape(T, k)   # MegaBlocks section 5 uniform assignment
+    pm = o.permute(forced, E, None)
+    assert pm["counts"].tolist() == [T * k // E] * E
+    assert pm["sorted_slot"][:T * k // E].tolist() == list(range(0, T * k, E))
+
+
+def pin_activations(o):
+    """Known values: GELU(z) = z * Phi(z); silu(z) = z * sigmoid(z)."""
+    z = np.array([-3.0, -1.0, 0.0, 0.5, 1.0, 2.0])
+    phi = np.array([0.0013498980316300946, 0.15865525393145707, 0.5,
+                    0.6914624612740131, 0.8413447460685429, 0.9772498680518208])
+    assert np.allclose(o.activation(z, "gelu"), z * phi, rtol=1e-14, atol=1e-16)
+    sig = np.array([0.04742587317756678, 0.2689414213699951, 0.5,
+                    0.6224593312018546, 0.7310585786300049, 0.8807970779778823])
+    up = np.array([2.0, -1.0, 3.0, 1.0, 1.0, 0.5])
+    assert np.allclose(o.activation(z, "swiglu", up), z * sig * up, rtol=1e-14, atol=1e-16)
+
+
+def pin_dense_mlp(o):
+    """One expert, top-1: the layer is a dense MLP (torch F.linear/F.gelu/F.silu, fp64)."""
+    rng = _rng(8)
+    T, d, F = 7, 12, 20
+    x = rng.standard_normal((T, d))
+    w1 = rng.standard_normal((1, d, F)) * 0.3
+    w3 = rng.standard_normal((1, d, F)) * 0.3
+    w2 = rng.standard_normal((1, F, d)) * 0.3
+    tx = torch.from_numpy(x)
+    t1, t3, t2 = (torch.from_numpy(w[0].T.copy()) for w in (w1, w3, w2))
+    ref_g = Fn.linear(Fn.gelu(Fn.linear(tx, t1), approximate="none"), t2).numpy()
+    ref_s = Fn.linear(Fn.silu(Fn.linear(tx, t1)) * Fn.linear(tx, t3), t2).numpy()
+    wg = rng.standard_normal((d, 1))
+    og = o.forward(x, wg, None, w1, None, w2, 1, "gelu")["out"]
+    os_ = o.forward(x, wg, None, w1, w3, w2, 1, "swiglu")["out"]
+    assert np.allclose(og, ref_g, rtol=1e-12, atol=1e-12)
+    assert np.allclose(os_, ref_s, rtol=1e-12, atol=1e-12)
+
+
+def _dense_dispatch_reference(x, idx, w, kept_mask, w1, w3, w2, act):
+    """The dispatch-mask / combine-weight formulation: every expert runs on
+    every token (torch fp64), and a dense [T, E] combine weight picks and
+    scales the outputs. No sort, no gather."""
+    T, k = idx.shape
+    E = w1.shape[0]
+    cw = torch.zeros(T, E, dtype=torch.float64)
+    for t in range(T):
+        for j in range(k):
+            if kept_mask[t, j]:
+                cw[t, idx[t, j]] += w[t, j]
+    tx = torch.from_numpy(np.asarray(x, dtype=np.float64))
+    out = torch.zeros(T, w2.shape[2], dtype=torch.float64)
+    for e in range(E):
+        z = tx @ torch.from_numpy(w1[e])
+        if act == "gelu":
+            h = Fn.gelu(z, approximate="none")
+        else:
+            h = Fn.silu(z) * (tx @ torch.from_numpy(w3[e]))
+        out += cw[:, e:e + 1] * (h @ torch.from_numpy(w2[e]))
+    return out.numpy()
+
+
+def pin_forward_dense_formulation(o):
+    """Sorted/gathered/combined output equals the dense dispatch-mask form,
+    with and without capacity drops."""
+    rng = _rng(9)
+    for act, cf, k, E in [("gelu", 0.0, 1, 4), ("swiglu", 0.0, 2, 5),
+                          ("swiglu", 0.75, 2, 4), ("gelu", 1.0, 3, 6)]:
+        T, d, F = 23, 8, 12
+        x = rng.standard_normal((T, d))
+        wg = rng.standard_normal((d, E))
+        w1 = rng.standard_normal((E, d, F)) * 0.4
+        w3 = rng.standard_normal((E, d, F)) * 0.4
+        w2 = rng.standard_normal((E, F, d)) * 0.4
+        res = o.forward(x, wg, None, w1, w3 if act == "swiglu" else None, w2, k, act, cf)
+        idx = res["route"]["topk_idx"]
+        # arrival-order capacity by brute force
+        cap = None if cf <= 0 else int(cf * (k * T / E))
+        seen = [0] * E
+        kept_mask = np.zeros((T, k), dtype=bool)
+        for t in range(T):
+            for j in range(k):
+                e = idx[t, j]
+                kept_mask[t, j] = cap is None or seen[e] < cap
+                seen[e] += 1
+        ref = _dense_dispatch_reference(x, idx, res["route"]["topk_w64"], kept_mask,
+                                        w1, w3, w2, act)
+        assert np.allclose(res["out"], ref, rtol=1e-11, atol=1e-11), (act, cf)
+        sub = [0, 5, 22]
+        ft = o.forward_tokens(x, sub, idx, res["route"]["topk_w64"],
+                              res["permute"]["slot_to_row"], w1,
+                              w3 if act == "swiglu" else None, w2, act)
+        assert np.allclose(ft, ref[sub], rtol=1e-11, atol=1e-11)
+
+
+def pin_all_dropped_token_is_zero(o):
+    """Capacity 0 drops every slot, so the output is all zeros."""
+    rng = _rng(10)
+    T, d, F, E = 6, 4, 8, 2
+    x = rng.standard_normal((T, d))
+    w1 = rng.standard_normal((E, d, F))
+    w2 = rng.standard_normal((E, F, d))
+    res = o.forward(x, rng.standard_normal((d, E)), None, w1, None, w2, 1, "gelu", cf=0.1)
+    assert res["permute"]["rows"] == 0 and np.all(res["out"] == 0.0)
+
+
+ALL_PINS = [
+    pin_example_a, pin_example_b, pin_topk_vs_torch, pin_topk_ties,
+    pin_softmax_vs_torch, pin_renormalise, pin_aux, pin_capacity,
+    pin_permute_bruteforce, pin_permute_vs_torch_sort, pin_activations,
+    pin_dense_mlp, pin_forward_dense_formulation, pin_all_dropped_token_is_zero,
+]
+
+
+def pin_bias(o):
+    """With a zero gate weight, every token's probabilities are softmax(b)
+    and its top-k is b's order (closed form)."""
+    b = np.array([0.3, -1.0, 2.0, 0.3, 1.5])
+    x = np.ones((3, 4))
+    r = o.route(x, np.zeros((4, 5)), b, 3)
+    e = np.exp(b - b.max())
+    assert np.allclose(r["probs64"], np.tile(e / e.sum(), (3, 1)), rtol=1e-14)
+    assert r["topk_idx"].tolist() == [[2, 4, 0]] * 3
+
+
+ALL_PINS.append(pin_bias)

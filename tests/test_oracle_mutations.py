@@ -1,0 +1,100 @@
+"""Plant plausible mistakes in the CPU oracle and check that the pins catch
+each one. The mistakes are planted in the oracle module only, on the CPU."""
+import math
+
+import numpy as np
+import pytest
+from scipy.special import erf
+
+from oracle import moe_oracle as O
+from tests.oracle_pins import ALL_PINS
+
+
+def _ties_to_higher(logits32, k):
+    l = np.asarray(logits32, dtype=np.float64)
+    E = l.shape[1]
+    order = E - 1 - np.argsort(-l[:, ::-1], axis=1, kind="stable")
+    return order[:, :k].astype(np.int32)
+
+
+def _no_renorm(probs, idx):
+    return np.take_along_axis(np.asarray(probs, float), np.asarray(idx, np.int64), 1)
+
+
+def _capacity_without_k(cf, k, T, E):
+    return None if cf is None or cf <= 0 else int(cf * (T / E))
+
+
+def _aux_over_tokens(probs, idx, E):
+    p = np.asarray(probs, float)
+    T, k = np.asarray(idx).shape
+    f = np.bincount(np.asarray(idx).reshape(-1), minlength=E) / T
+    return float(E * np.sum(f * p.mean(0)))
+
+
+def _gelu_tanh(z, act, z_up=None):
+    z = np.asarray(z, float)
+    if act == "gelu":
+        return 0.5 * z * (1 + np.tanh(math.sqrt(2 / math.pi) * (z + 0.044715 * z ** 3)))
+    return (z / (1 + np.exp(-z))) * z_up
+
+
+def _softmax_wrong_axis(l):
+    l = np.asarray(l, float)
+    e = np.exp(l - l.max(0, keepdims=True))
+    return e / e.sum(0, keepdims=True)
+
+
+def _gate_no_bias(x, wg, bias=None):
+    return np.asarray(x, float) @ np.asarray(wg, float)
+
+
+def _combine_swapped_weights(y_perm, topk_w, slot_to_row, T, k):
+    w = np.asarray(topk_w, float).reshape(T, k)[:, ::-1]
+    return _REAL["combine"](y_perm, w, slot_to_row, T, k)
+
+
+def _gather_mod(x, row_slot, k):
+    return np.asarray(x)[np.asarray(row_slot, np.int64) % np.asarray(x).shape[0]]
+
+
+def _ffn_wrong_expert(x_perm, seg_offsets, w1, w3, w2, act):
+    E = len(seg_offsets) - 1
+    perm = [(e + 1) % E for e in range(E)]
+    return _REAL["expert_ffn"](x_perm, seg_offsets, [w1[p] for p in perm],
+                               None if w3 is None else [w3[p] for p in perm], w2, act)
+
+
+def _permute_drop_gt(idx, E, cap=None):
+    r = _REAL["permute"](idx, E, None if cap is None else cap + 1)
+    return r
+
+
+_REAL = {n: getattr(O, n) for n in ("combine", "expert_ffn", "permute")}
+
+MUTATIONS = {
+    "topk_ties_to_higher_index": ("topk_select", _ties_to_higher),
+    "no_renormalisation": ("renormalise", _no_renorm),
+    "capacity_without_k": ("capacity", _capacity_without_k),
+    "aux_f_over_tokens": ("aux_loss", _aux_over_tokens),
+    "gelu_tanh_approximation": ("activation", _gelu_tanh),
+    "softmax_wrong_axis": ("softmax_rows", _softmax_wrong_axis),
+    "gate_drops_bias": ("gate_logits", _gate_no_bias),
+    "combine_swaps_weights": ("combine", _combine_swapped_weights),
+    "gather_wrong_token": ("gather", _gather_mod),
+    "ffn_wrong_expert": ("expert_ffn", _ffn_wrong_expert),
+    "drop_off_by_one": ("permute", _permute_drop_gt),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_mutation(name, monkeypatch):
+    attr, bad = MUTATIONS[name]
+    monkeypatch.setattr(O, attr, bad)
+    caught = []
+    for pin in ALL_PINS:
+        try:
+            pin(O)
+        except (AssertionError, ValueError, IndexError, TypeError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught the planted mistake {name}"
