@@ -1,0 +1,255 @@
+/*
+ * moe_b200.h -- C ABI of the single-GPU Mixture-of-Experts layer forward for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (sources: "ops-transformer MoE operators" blog, 原理 Steps 1-4 and
+ * 实现; "MoE Router: who decides which expert a token goes to"; "MegaBlocks 01 -
+ * why MoE is hard", sections 1-5; "Integrating MoE into your model with
+ * Colossal-AI", step 2):
+ *
+ *   route    logits = x Wg (+ b), p = softmax(logits), top-k (ties -> lower
+ *            expert index), w = p_sel / sum(p_sel), aux = E * sum_i f_i P_i
+ *   permute  histogram of the T*k slots per expert, inclusive scan (bins),
+ *            stable counting sort on the low max(ceil(log2 E),1) key bits,
+ *            capacity C = int(cf * k * T / E) with drop by arrival order
+ *   gather   x_perm[row] = x[slot / k] for every kept slot, expert-contiguous
+ *   ffn      per expert e over its rows: SwiGLU  h = silu(x W_gate[e]) * (x W_up[e])
+ *                                      GELU    h = gelu(x W1[e])          (exact erf)
+ *            then y = h W_down[e] (or h W2[e])
+ *   combine  out[t] = sum_{j<k, slot kept} w[t,j] * y[row(t,j)]   (zero if all dropped)
+ *
+ * Conventions for every entry point below:
+ *  - All tensor pointers are DEVICE pointers unless the name says host, and
+ *    are owned by the caller. The library never allocates or frees device
+ *    memory and never synchronises the stream, except moe_get_device_error.
+ *  - Layouts are row-major. A slot is s = t * k + j (token t, choice j).
+ *    Weights: Wg [d, E]; W1 / W_gate / W_up [E, d, F]; W2 / W_down [E, F, d]
+ *    (the [E, hs, ffn] layout of the MegaBlocks page, section 4.3).
+ *  - Gathered rows: the kept slots of expert 0 in ascending slot order, then
+ *    expert 1, ...; expert e owns rows [seg_offsets[e], seg_offsets[e+1]).
+ *  - dtype MOE_BF16: x, weights, x_perm, h, y_perm and out are bf16; router
+ *    logits/probabilities/weights, the bias and the aux loss are fp32 and all
+ *    accumulation is fp32. dtype MOE_F32: every tensor is fp32.
+ *  - Limits: 1 <= E <= 256, 1 <= k <= min(E, 8), T >= 0, T * k < 2^31.
+ *    bf16: d % 128 == 0 and F % 128 == 0. f32: d % 4 == 0 and F % 4 == 0.
+ *    Every device pointer 16-byte aligned.
+ *  - Host-checkable problems return a status synchronously and launch
+ *    nothing. Data-dependent problems found on the device (an expert id out of
+ *    range, a row index out of range, a bounded wait that timed out) set bits
+ *    in a device error word kept in the first bytes of the workspace; kernels
+ *    never trap and never write out of bounds; outputs of that call are then
+ *    unspecified. Read the word with moe_get_device_error.
+ *  - Workspace: every entry point takes (ws, ws_bytes). Its first 256 bytes
+ *    are a control block (error word and counters) that must be zeroed once
+ *    with moe_workspace_init before first use; the same workspace may then be
+ *    reused by any number of calls on one stream. Calls that share a
+ *    workspace must not run concurrently.
+ *  - stream: a cudaStream_t (NULL = legacy default stream).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* same object as cudaStream_t */
+typedef struct CUevent_st* moe_event_t;   /* same object as cudaEvent_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_NULL = 1,        /* a required pointer is NULL */
+  MOE_ERR_INVALID = 2,     /* a size or parameter is out of range */
+  MOE_ERR_UNSUPPORTED = 3, /* valid but outside this build's limits (divisibility) */
+  MOE_ERR_WORKSPACE = 4,   /* ws_bytes smaller than the matching *_workspace_size */
+  MOE_ERR_ALIGN = 5,       /* a pointer is not 16-byte aligned */
+  MOE_ERR_CUDA = 6,        /* a CUDA call or kernel launch failed */
+  MOE_ERR_DEVICE = 7       /* the device error word is non-zero */
+} moe_status_t;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
+typedef enum { MOE_ACT_GELU = 0, MOE_ACT_SWIGLU = 1 } moe_act_t;
+
+/* Bits of the device error word. */
+#define MOE_DEVERR_EXPERT_RANGE 0x1u /* a top-k expert id outside [0, E) */
+#define MOE_DEVERR_ROW_RANGE 0x2u    /* a slot/row index outside its buffer */
+#define MOE_DEVERR_TIMEOUT 0x4u      /* a bounded on-chip wait gave up */
+
+/* One MoE layer: shapes, activation, capacity and the weight pointers. */
+typedef struct {
+  int d;                    /* hidden size */
+  int E;                    /* number of experts */
+  int k;                    /* experts per token */
+  int F;                    /* expert FFN size */
+  moe_dtype_t dtype;
+  moe_act_t act;
+  double capacity_factor;   /* <= 0: dropless; else C = int(cf * (k * T / E)) */
+  const void* w_router;     /* Wg [d, E] */
+  const float* router_bias; /* fixed logit bias [E] (fp32) or NULL */
+  const void* w1;           /* W_gate (SwiGLU) or W1 (GELU), [E, d, F] */
+  const void* w3;           /* W_up [E, d, F] (SwiGLU), NULL for GELU */
+  const void* w2;           /* W_down / W2 [E, F, d] */
+} moe_layer_t;
+
+/* Device pointers into a moe_forward workspace where that call leaves its
+ * intermediate results (see moe_forward_views). */
+typedef struct {
+  int32_t* topk_idx;     /* [T, k] */
+  float* topk_w;         /* [T, k] */
+  float* aux_loss;       /* [1] */
+  int32_t* counts;       /* [E] */
+  int32_t* bins;         /* [E] */
+  int32_t* kept_counts;  /* [E] */
+  int32_t* seg_offsets;  /* [E + 1] */
+  int32_t* sorted_slot;  /* [T * k] */
+  int32_t* slot_to_row;  /* [T * k] */
+  int32_t* row_slot;     /* [rows_max] */
+  uint8_t* drop_mask;    /* [T * k] */
+  void* x_perm;          /* [rows_max, d] */
+  void* h;               /* [rows_max, F] */
+  void* y_perm;          /* [rows_max, d] */
+  int64_t rows_max;
+  int64_t capacity;      /* C, or -1 when dropless */
+} moe_views_t;
+
+/* Human-readable name of a status code (static string). */
+MOE_API const char* moe_status_string(moe_status_t status);
+
+/* Zero the control block (first 256 bytes) of a workspace, asynchronously
+ * on `stream`. Needed once per workspace before its first use. */
+MOE_API moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Read (synchronises `stream`) and optionally clear the device error word of
+ * a workspace into *host_bits. Returns MOE_ERR_DEVICE if it was non-zero. */
+MOE_API moe_status_t moe_get_device_error(void* ws, moe_stream_t stream, uint32_t* host_bits,
+                                  int clear);
+
+/* Capacity C = int(cf * (k * T / E)) evaluated in double, as the MegaBlocks
+ * page's expert_capacity (section 4.2, world size 1); -1 (dropless) when
+ * cf <= 0. */
+MOE_API int64_t moe_capacity(double capacity_factor, int T, int k, int E);
+
+/* Upper bound on gathered rows: T*k when capacity < 0 (dropless), else
+ * min(T*k, E*C). */
+MOE_API int64_t moe_rows_max(int T, int k, int E, int64_t capacity);
+
+/* ------------------------------------------------------------------ route
+ * Router gate Linear(d, E) without learned bias (+ optional fixed fp32 logit
+ * bias), softmax over E, top-k by selection with ties to the lower expert
+ * index (selection compares the fp32 logits), renormalisation of the k
+ * weights to sum 1, and the load-balance loss aux = E * sum_i f_i * P_i with
+ * f_i = (slots routed to i, before any capacity drop) / (T*k) and
+ * P_i = mean_t p[t,i]. ("ops-transformer MoE operators", 实现: softmax,
+ * top-K selection, NormalizeWeights; "MoE Router": gate without bias,
+ * softmax, topk, renormalise.)
+ *   x          [T, d] (dtype)          w_router [d, E] (dtype)
+ *   bias       [E] fp32 or NULL
+ *   topk_idx   out [T, k] int32        topk_w out [T, k] fp32
+ *   aux_loss   out [1] fp32 (device)
+ *   logits, probs  optional out [T, E] fp32 (NULL to skip)
+ *   ws         >= moe_route_workspace_size(T, d, E) bytes */
+MOE_API size_t moe_route_workspace_size(int T, int d, int E);
+MOE_API moe_status_t moe_route(const void* x, const void* w_router, const float* bias, moe_dtype_t dtype,
+                       int T, int d, int E, int k, int32_t* topk_idx, float* topk_w,
+                       float* aux_loss, float* logits, float* probs, void* ws, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/* ---------------------------------------------------------------- permute
+ * Sorting metadata of the T*k slots by expert id ("MegaBlocks", section 4.1:
+ * sort, histogram, inclusive cumsum; only max(ceil(log2 E),1) key bits are
+ * sorted), then capacity drop by arrival order (sections 3, 4.2, 4.5).
+ *   topk_idx     [T, k] int32, values in [0, E)
+ *   capacity     C >= 0 (0 drops every slot), or any negative value for dropless
+ *   counts       out [E]    slots per expert (before the drop)
+ *   bins         out [E]    inclusive prefix sum of counts
+ *   sorted_slot  out [T*k]  slots in stable order of expert id
+ *   slot_to_row  out [T*k]  gathered row of each slot, -1 if dropped
+ *   row_slot     out [moe_rows_max(...)]  slot of each gathered row (rows
+ *                past seg_offsets[E] are left untouched)
+ *   drop_mask    out [T*k]  1 if the slot is dropped (u8)
+ *   kept_counts  out [E]    min(counts, C)
+ *   seg_offsets  out [E+1]  exclusive prefix sum of kept_counts
+ *   ws           >= moe_permute_workspace_size(T, k, E) bytes */
+MOE_API size_t moe_permute_workspace_size(int T, int k, int E);
+MOE_API moe_status_t moe_permute(const int32_t* topk_idx, int T, int k, int E, int64_t capacity,
+                         int32_t* counts, int32_t* bins, int32_t* sorted_slot,
+                         int32_t* slot_to_row, int32_t* row_slot, uint8_t* drop_mask,
+                         int32_t* kept_counts, int32_t* seg_offsets, void* ws, size_t ws_bytes,
+                         moe_stream_t stream);
+
+/* ----------------------------------------------------------------- gather
+ * x_perm[r] = x[row_slot[r] / k] for r < seg_offsets[E] ("MegaBlocks",
+ * section 4.3, binned_gather in compact form), moved row by row with bulk
+ * (TMA) copies. rows_max bounds seg_offsets[E].
+ *   ws  >= 256 bytes (control block) */
+MOE_API moe_status_t moe_gather(const void* x, moe_dtype_t dtype, int T, int d, int k,
+                        const int32_t* row_slot, const int32_t* seg_offsets, int E,
+                        int64_t rows_max, void* x_perm, void* ws, size_t ws_bytes,
+                        moe_stream_t stream);
+
+/* ------------------------------------------------------------- expert FFN
+ * Grouped expert MLP over the expert-contiguous rows ("MegaBlocks", section
+ * 4.3: bmm -> activation -> bmm, weights [E, hs, ffn]). bf16 runs on the
+ * tcgen05 tensor cores (fp32 accumulation in tensor memory, SwiGLU/GELU in
+ * the up-projection epilogue, h rounded to bf16); f32 runs on CUDA cores.
+ * Experts with no rows read no weights.
+ *   x_perm  [rows_max, d]   h out [rows_max, F]   y_perm out [rows_max, d]
+ *   w1 W_gate/W1 [E, d, F], w3 W_up [E, d, F] (SwiGLU) or NULL, w2 [E, F, d]
+ *   seg_offsets [E+1] from moe_permute
+ *   ws  >= 256 bytes (control block) */
+MOE_API moe_status_t moe_expert_ffn(const void* x_perm, const void* w1, const void* w3, const void* w2,
+                            moe_dtype_t dtype, moe_act_t act, int64_t rows_max, int d, int F,
+                            int E, const int32_t* seg_offsets, void* h, void* y_perm, void* ws,
+                            size_t ws_bytes, moe_stream_t stream);
+
+/* ---------------------------------------------------------------- combine
+ * out[t] = sum_{j=0..k-1, slot_to_row[t*k+j] >= 0} topk_w[t,j] * y_perm[row]
+ * in fp32, j ascending; zero row when every slot of t is dropped
+ * ("ops-transformer", 原理 Step 4; "MegaBlocks", sections 4.3 and 5).
+ * Each output row is written by one thread group that gathers its k rows:
+ * no atomics, deterministic.
+ *   ws  >= 256 bytes (control block) */
+MOE_API moe_status_t moe_combine(const void* y_perm, const float* topk_w, const int32_t* slot_to_row,
+                         moe_dtype_t dtype, int T, int d, int k, int64_t rows_max, void* out,
+                         void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ---------------------------------------------------------------- forward
+ * The whole layer on one stream with no host synchronisation: route ->
+ * permute -> gather -> expert FFN (up, down) -> combine.
+ *   x [T, d], out [T, d] (dtype); aux_loss out [1] fp32 device or NULL.
+ *   events: NULL, or 7 cudaEvent_t recorded on `stream` before route and
+ *   after route, permute, gather, up-projection, down-projection, combine.
+ *   ws >= moe_forward_workspace_size(layer, T) bytes; it holds every
+ *   intermediate (see moe_forward_views). */
+MOE_API size_t moe_forward_workspace_size(const moe_layer_t* layer, int T);
+MOE_API moe_status_t moe_forward(const moe_layer_t* layer, const void* x, int T, void* out,
+                         float* aux_loss, void* ws, size_t ws_bytes, moe_stream_t stream,
+                         const moe_event_t* events);
+
+/* Where moe_forward(layer, ., T, ...) leaves its intermediates in `ws`. */
+MOE_API moe_status_t moe_forward_views(const moe_layer_t* layer, int T, void* ws, size_t ws_bytes,
+                               moe_views_t* views);
+
+/* moe_forward with HOST input and output: copies x_host (T*d elements,
+ * pinned host memory recommended) into the workspace, runs the forward,
+ * copies the output into out_host and the aux loss into *aux_host. All
+ * copies are asynchronous on `stream`; the host buffers must stay valid
+ * until the stream reaches this point. ws >= moe_forward_host_workspace_size. */
+MOE_API size_t moe_forward_host_workspace_size(const moe_layer_t* layer, int T);
+MOE_API moe_status_t moe_forward_host(const moe_layer_t* layer, const void* x_host, int T, void* out_host,
+                              float* aux_host, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

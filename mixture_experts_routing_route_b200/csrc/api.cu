@@ -1,0 +1,420 @@
+// The extern "C" entry points of libmoe_b200.so: argument checks, workspace
+// layout, and the stage launches on the caller's stream. Nothing here
+// allocates device memory or synchronises, except moe_get_device_error.
+#include "common.cuh"
+#include <climits>
+#include <cmath>
+
+namespace moe {
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t esize(moe_dtype_t dt) { return dt == MOE_BF16 ? 2 : 4; }
+
+moe_status_t check_dims(moe_dtype_t dt, int T, int d, int E, int k) {
+  if (dt != MOE_BF16 && dt != MOE_F32) return MOE_ERR_INVALID;
+  if (T < 0 || d <= 0 || E < 1 || E > 256 || k < 1 || k > 8 || k > E) return MOE_ERR_INVALID;
+  if (static_cast<long long>(T) * k >= INT_MAX) return MOE_ERR_INVALID;
+  if (dt == MOE_BF16 && d % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (dt == MOE_F32 && d % 4 != 0) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status_t check_ffn(moe_dtype_t dt, int F) {
+  if (F <= 0) return MOE_ERR_INVALID;
+  if (dt == MOE_BF16 && F % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (dt == MOE_F32 && F % 4 != 0) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_CHECK(expr)                      \
+  do {                                       \
+    const moe_status_t st_ = (expr);         \
+    if (st_ != MOE_OK) return st_;           \
+  } while (0)
+
+#define MOE_NEED(p)                                  \
+  do {                                               \
+    if ((p) == nullptr) return MOE_ERR_NULL;         \
+    if (!aligned16(p)) return MOE_ERR_ALIGN;         \
+  } while (0)
+
+#define MOE_OPT(p)                                   \
+  do {                                               \
+    if ((p) != nullptr && !aligned16(p)) return MOE_ERR_ALIGN; \
+  } while (0)
+
+// Bump allocator over a workspace, 256-byte aligned pieces.
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<uint8_t*>(b)) {}
+  void* take(size_t bytes) {
+    void* p = base ? base + off : nullptr;
+    off += align_up(bytes);
+    return p;
+  }
+};
+
+struct FwdLayout {
+  Control* ctl;
+  void* partials;
+  float* logits_scratch;
+  int32_t* idx;
+  float* w;
+  float* aux;
+  int32_t *counts, *bins, *kept, *seg;
+  int32_t *sorted_slot, *slot_to_row, *row_slot;
+  uint8_t* drop;
+  int32_t* rank;
+  void *x_perm, *h, *y_perm;
+  void *x_dev, *out_dev;  // host-buffer variant only
+  int64_t cap, rows_max;
+  size_t bytes;
+};
+
+FwdLayout fwd_layout(const moe_layer_t* L, int T, void* ws, bool host_io) {
+  FwdLayout f{};
+  Carver c(ws);
+  const size_t S = static_cast<size_t>(T) * L->k;
+  const size_t es = esize(L->dtype);
+  f.cap = moe_capacity(L->capacity_factor, T, L->k, L->E);
+  f.rows_max = moe_rows_max(T, L->k, L->E, f.cap);
+  const size_t R = static_cast<size_t>(f.rows_max);
+  f.ctl = static_cast<Control*>(c.take(sizeof(Control)));
+  f.partials = c.take(route_partials_bytes(T, L->E));
+  f.logits_scratch = static_cast<float*>(c.take(route_logits_scratch_bytes(T, L->d, L->E)));
+  f.idx = static_cast<int32_t*>(c.take(S * 4));
+  f.w = static_cast<float*>(c.take(S * 4));
+  f.aux = static_cast<float*>(c.take(4));
+  f.counts = static_cast<int32_t*>(c.take(L->E * 4));
+  f.bins = static_cast<int32_t*>(c.take(L->E * 4));
+  f.kept = static_cast<int32_t*>(c.take(L->E * 4));
+  f.seg = static_cast<int32_t*>(c.take((L->E + 1) * 4));
+  f.sorted_slot = static_cast<int32_t*>(c.take(S * 4));
+  f.slot_to_row = static_cast<int32_t*>(c.take(S * 4));
+  f.row_slot = static_cast<int32_t*>(c.take(R * 4));
+  f.drop = static_cast<uint8_t*>(c.take(S));
+  f.rank = static_cast<int32_t*>(c.take(permute_scratch_bytes(T, L->k, L->E)));
+  f.x_perm = c.take(R * L->d * es);
+  f.h = c.take(R * L->F * es);
+  f.y_perm = c.take(R * L->d * es);
+  if (host_io) {
+    f.x_dev = c.take(static_cast<size_t>(T) * L->d * es);
+    f.out_dev = c.take(static_cast<size_t>(T) * L->d * es);
+  }
+  f.bytes = c.off;
+  return f;
+}
+
+moe_status_t check_layer(const moe_layer_t* L, int T) {
+  if (L == nullptr) return MOE_ERR_NULL;
+  MOE_CHECK(check_dims(L->dtype, T, L->d, L->E, L->k));
+  MOE_CHECK(check_ffn(L->dtype, L->F));
+  if (L->act != MOE_ACT_GELU && L->act != MOE_ACT_SWIGLU) return MOE_ERR_INVALID;
+  if (!std::isfinite(L->capacity_factor)) return MOE_ERR_INVALID;
+  MOE_NEED(L->w_router);
+  MOE_NEED(L->w1);
+  MOE_NEED(L->w2);
+  if (L->act == MOE_ACT_SWIGLU) MOE_NEED(L->w3);
+  MOE_OPT(L->router_bias);
+  return MOE_OK;
+}
+
+moe_status_t run_forward(const moe_layer_t* L, const void* x, int T, void* out, float* aux_user,
+                         const FwdLayout& f, cudaStream_t s, const moe_event_t* ev) {
+  auto rec = [&](int i) {
+    if (ev != nullptr && ev[i] != nullptr) cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev[i]), s);
+  };
+  const size_t es = esize(L->dtype);
+  rec(0);
+  MOE_CHECK(from_cuda(launch_route(x, L->w_router, L->router_bias, L->dtype, T, L->d, L->E, L->k,
+                                   f.idx, f.w, f.aux, nullptr, nullptr, f.logits_scratch,
+                                   f.partials, f.ctl, s)));
+  rec(1);
+  MOE_CHECK(from_cuda(launch_permute(f.idx, T, L->k, L->E, f.cap, f.counts, f.bins, f.sorted_slot,
+                                     f.slot_to_row, f.row_slot, f.drop, f.kept, f.seg, f.rank,
+                                     f.ctl, s)));
+  rec(2);
+  MOE_CHECK(from_cuda(launch_gather(x, es, T, L->d, L->k, f.row_slot, f.seg, L->E, f.rows_max,
+                                    f.x_perm, f.ctl, s)));
+  rec(3);
+  cudaEvent_t after_up = (ev != nullptr) ? reinterpret_cast<cudaEvent_t>(ev[4]) : nullptr;
+  if (L->dtype == MOE_BF16)
+    MOE_CHECK(from_cuda(launch_ffn_bf16(f.x_perm, L->w1, L->w3, L->w2, L->act, f.rows_max, L->d,
+                                        L->F, L->E, f.seg, f.h, f.y_perm, f.ctl, s, after_up)));
+  else
+    MOE_CHECK(from_cuda(launch_ffn_f32(static_cast<const float*>(f.x_perm),
+                                       static_cast<const float*>(L->w1),
+                                       static_cast<const float*>(L->w3),
+                                       static_cast<const float*>(L->w2), L->act, f.rows_max, L->d,
+                                       L->F, L->E, f.seg, static_cast<float*>(f.h),
+                                       static_cast<float*>(f.y_perm), f.ctl, s, after_up)));
+  rec(5);
+  MOE_CHECK(from_cuda(launch_combine(f.y_perm, f.w, f.slot_to_row, es, T, L->d, L->k, f.rows_max,
+                                     out, f.ctl, s)));
+  rec(6);
+  if (aux_user != nullptr && aux_user != f.aux)
+    MOE_CHECK(from_cuda(cudaMemcpyAsync(aux_user, f.aux, 4, cudaMemcpyDeviceToDevice, s)));
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t st) {
+  switch (st) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_NULL: return "a required pointer is NULL";
+    case MOE_ERR_INVALID: return "a size or parameter is out of range";
+    case MOE_ERR_UNSUPPORTED: return "shape outside this build's limits";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case MOE_ERR_CUDA: return "CUDA call or kernel launch failed";
+    case MOE_ERR_DEVICE: return "device error word is set";
+  }
+  return "unknown status";
+}
+
+moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_NEED(ws);
+  if (ws_bytes < sizeof(Control)) return MOE_ERR_WORKSPACE;
+  return from_cuda(cudaMemsetAsync(ws, 0, sizeof(Control), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_get_device_error(void* ws, moe_stream_t stream, uint32_t* host_bits, int clear) {
+  MOE_NEED(ws);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, &static_cast<Control*>(ws)->err, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (clear && cudaMemsetAsync(&static_cast<Control*>(ws)->err, 0, 4, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (host_bits) *host_bits = v;
+  return v ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+int64_t moe_capacity(double cf, int T, int k, int E) {
+  if (!(cf > 0.0) || E <= 0) return -1;
+  const double c = cf * (static_cast<double>(k) * static_cast<double>(T) / static_cast<double>(E));
+  return static_cast<int64_t>(c);  // truncation toward zero, as int() does
+}
+
+int64_t moe_rows_max(int T, int k, int E, int64_t capacity) {
+  const int64_t S = static_cast<int64_t>(T) * k;
+  if (capacity < 0) return S;
+  const int64_t ec = static_cast<int64_t>(E) * capacity;
+  return ec < S ? ec : S;
+}
+
+size_t moe_route_workspace_size(int T, int d, int E) {
+  if (T < 0 || E < 1) return 0;
+  return align_up(sizeof(Control)) + route_partials_bytes(T, E) + route_logits_scratch_bytes(T, d, E);
+}
+
+moe_status_t moe_route(const void* x, const void* w_router, const float* bias, moe_dtype_t dtype,
+                       int T, int d, int E, int k, int32_t* topk_idx, float* topk_w, float* aux_loss,
+                       float* logits, float* probs, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_CHECK(check_dims(dtype, T, d, E, k));
+  MOE_NEED(x);
+  MOE_NEED(w_router);
+  MOE_NEED(topk_idx);
+  MOE_NEED(topk_w);
+  MOE_NEED(aux_loss);
+  MOE_NEED(ws);
+  MOE_OPT(bias);
+  MOE_OPT(logits);
+  MOE_OPT(probs);
+  if (ws_bytes < moe_route_workspace_size(T, d, E)) return MOE_ERR_WORKSPACE;
+  Carver c(ws);
+  Control* ctl = static_cast<Control*>(c.take(sizeof(Control)));
+  void* partials = c.take(route_partials_bytes(T, E));
+  float* scratch = static_cast<float*>(c.take(route_logits_scratch_bytes(T, d, E)));
+  return from_cuda(launch_route(x, w_router, bias, dtype, T, d, E, k, topk_idx, topk_w, aux_loss,
+                                logits, probs, scratch, partials, ctl,
+                                reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_permute_workspace_size(int T, int k, int E) {
+  if (T < 0 || k < 1) return 0;
+  return align_up(sizeof(Control)) + permute_scratch_bytes(T, k, E);
+}
+
+moe_status_t moe_permute(const int32_t* topk_idx, int T, int k, int E, int64_t capacity,
+                         int32_t* counts, int32_t* bins, int32_t* sorted_slot, int32_t* slot_to_row,
+                         int32_t* row_slot, uint8_t* drop_mask, int32_t* kept_counts,
+                         int32_t* seg_offsets, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (T < 0 || E < 1 || E > 256 || k < 1 || k > 8 || k > E) return MOE_ERR_INVALID;
+  if (static_cast<long long>(T) * k >= INT_MAX) return MOE_ERR_INVALID;
+  if (T > 0) {
+    MOE_NEED(topk_idx);
+    MOE_NEED(sorted_slot);
+    MOE_NEED(slot_to_row);
+    MOE_NEED(drop_mask);
+    if (moe_rows_max(T, k, E, capacity) > 0) MOE_NEED(row_slot);
+  }
+  MOE_NEED(counts);
+  MOE_NEED(bins);
+  MOE_NEED(kept_counts);
+  MOE_NEED(seg_offsets);
+  MOE_NEED(ws);
+  if (ws_bytes < moe_permute_workspace_size(T, k, E)) return MOE_ERR_WORKSPACE;
+  Carver c(ws);
+  Control* ctl = static_cast<Control*>(c.take(sizeof(Control)));
+  int32_t* rank = static_cast<int32_t*>(c.take(permute_scratch_bytes(T, k, E)));
+  return from_cuda(launch_permute(topk_idx, T, k, E, capacity, counts, bins, sorted_slot,
+                                  slot_to_row, row_slot, drop_mask, kept_counts, seg_offsets, rank,
+                                  ctl, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_gather(const void* x, moe_dtype_t dtype, int T, int d, int k,
+                        const int32_t* row_slot, const int32_t* seg_offsets, int E, int64_t rows_max,
+                        void* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_CHECK(check_dims(dtype, T, d, E, k));
+  if (rows_max < 0 || rows_max > static_cast<int64_t>(T) * k) return MOE_ERR_INVALID;
+  MOE_NEED(seg_offsets);
+  MOE_NEED(ws);
+  if (ws_bytes < sizeof(Control)) return MOE_ERR_WORKSPACE;
+  if (rows_max > 0 && T > 0) {
+    MOE_NEED(x);
+    MOE_NEED(row_slot);
+    MOE_NEED(x_perm);
+  }
+  return from_cuda(launch_gather(x, esize(dtype), T, d, k, row_slot, seg_offsets, E, rows_max,
+                                 x_perm, static_cast<Control*>(ws),
+                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_expert_ffn(const void* x_perm, const void* w1, const void* w3, const void* w2,
+                            moe_dtype_t dtype, moe_act_t act, int64_t rows_max, int d, int F, int E,
+                            const int32_t* seg_offsets, void* h, void* y_perm, void* ws,
+                            size_t ws_bytes, moe_stream_t stream) {
+  MOE_CHECK(check_dims(dtype, 0, d, E, 1));
+  MOE_CHECK(check_ffn(dtype, F));
+  if (act != MOE_ACT_GELU && act != MOE_ACT_SWIGLU) return MOE_ERR_INVALID;
+  if (rows_max < 0 || rows_max >= INT_MAX) return MOE_ERR_INVALID;
+  MOE_NEED(w1);
+  MOE_NEED(w2);
+  if (act == MOE_ACT_SWIGLU) MOE_NEED(w3);
+  MOE_NEED(seg_offsets);
+  MOE_NEED(ws);
+  if (ws_bytes < sizeof(Control)) return MOE_ERR_WORKSPACE;
+  if (rows_max > 0) {
+    MOE_NEED(x_perm);
+    MOE_NEED(h);
+    MOE_NEED(y_perm);
+  }
+  Control* ctl = static_cast<Control*>(ws);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == MOE_BF16)
+    return from_cuda(launch_ffn_bf16(x_perm, w1, w3, w2, act, rows_max, d, F, E, seg_offsets, h,
+                                     y_perm, ctl, s, nullptr));
+  return from_cuda(launch_ffn_f32(static_cast<const float*>(x_perm), static_cast<const float*>(w1),
+                                  static_cast<const float*>(w3), static_cast<const float*>(w2), act,
+                                  rows_max, d, F, E, seg_offsets, static_cast<float*>(h),
+                                  static_cast<float*>(y_perm), ctl, s, nullptr));
+}
+
+moe_status_t moe_combine(const void* y_perm, const float* topk_w, const int32_t* slot_to_row,
+                         moe_dtype_t dtype, int T, int d, int k, int64_t rows_max, void* out, void* ws,
+                         size_t ws_bytes, moe_stream_t stream) {
+  MOE_CHECK(check_dims(dtype, T, d, k, k));
+  if (rows_max < 0) return MOE_ERR_INVALID;
+  MOE_NEED(ws);
+  if (ws_bytes < sizeof(Control)) return MOE_ERR_WORKSPACE;
+  if (T > 0) {
+    MOE_NEED(topk_w);
+    MOE_NEED(slot_to_row);
+    MOE_NEED(out);
+    if (rows_max > 0) MOE_NEED(y_perm);
+  }
+  return from_cuda(launch_combine(y_perm, topk_w, slot_to_row, esize(dtype), T, d, k, rows_max, out,
+                                  static_cast<Control*>(ws), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_forward_workspace_size(const moe_layer_t* layer, int T) {
+  if (layer == nullptr || T < 0) return 0;
+  return fwd_layout(layer, T, nullptr, false).bytes;
+}
+
+size_t moe_forward_host_workspace_size(const moe_layer_t* layer, int T) {
+  if (layer == nullptr || T < 0) return 0;
+  return fwd_layout(layer, T, nullptr, true).bytes;
+}
+
+moe_status_t moe_forward_views(const moe_layer_t* layer, int T, void* ws, size_t ws_bytes,
+                               moe_views_t* v) {
+  MOE_CHECK(check_layer(layer, T));
+  MOE_NEED(ws);
+  if (v == nullptr) return MOE_ERR_NULL;
+  const FwdLayout f = fwd_layout(layer, T, ws, false);
+  if (ws_bytes < f.bytes) return MOE_ERR_WORKSPACE;
+  v->topk_idx = f.idx;
+  v->topk_w = f.w;
+  v->aux_loss = f.aux;
+  v->counts = f.counts;
+  v->bins = f.bins;
+  v->kept_counts = f.kept;
+  v->seg_offsets = f.seg;
+  v->sorted_slot = f.sorted_slot;
+  v->slot_to_row = f.slot_to_row;
+  v->row_slot = f.row_slot;
+  v->drop_mask = f.drop;
+  v->x_perm = f.x_perm;
+  v->h = f.h;
+  v->y_perm = f.y_perm;
+  v->rows_max = f.rows_max;
+  v->capacity = f.cap;
+  return MOE_OK;
+}
+
+moe_status_t moe_forward(const moe_layer_t* layer, const void* x, int T, void* out, float* aux_loss,
+                         void* ws, size_t ws_bytes, moe_stream_t stream, const moe_event_t* events) {
+  MOE_CHECK(check_layer(layer, T));
+  MOE_NEED(ws);
+  MOE_OPT(aux_loss);
+  if (T > 0) {
+    MOE_NEED(x);
+    MOE_NEED(out);
+  }
+  const FwdLayout f = fwd_layout(layer, T, ws, false);
+  if (ws_bytes < f.bytes) return MOE_ERR_WORKSPACE;
+  return run_forward(layer, x, T, out, aux_loss, f, reinterpret_cast<cudaStream_t>(stream), events);
+}
+
+moe_status_t moe_forward_host(const moe_layer_t* layer, const void* x_host, int T, void* out_host,
+                              float* aux_host, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_CHECK(check_layer(layer, T));
+  MOE_NEED(ws);
+  if (T > 0 && (x_host == nullptr || out_host == nullptr)) return MOE_ERR_NULL;
+  const FwdLayout f = fwd_layout(layer, T, ws, true);
+  if (ws_bytes < f.bytes) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(T) * layer->d * esize(layer->dtype);
+  if (bytes) MOE_CHECK(from_cuda(cudaMemcpyAsync(f.x_dev, x_host, bytes, cudaMemcpyHostToDevice, s)));
+  MOE_CHECK(run_forward(layer, f.x_dev, T, f.out_dev, nullptr, f, s, nullptr));
+  if (bytes) MOE_CHECK(from_cuda(cudaMemcpyAsync(out_host, f.out_dev, bytes, cudaMemcpyDeviceToHost, s)));
+  if (aux_host) MOE_CHECK(from_cuda(cudaMemcpyAsync(aux_host, f.aux, 4, cudaMemcpyDeviceToHost, s)));
+  return MOE_OK;
+}
+
+}  // extern "C"

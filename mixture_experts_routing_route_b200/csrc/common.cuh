@@ -1,0 +1,80 @@
+// Internal declarations shared by the kernels and the C-ABI layer.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+#include <cstddef>
+
+#include "../../include/moe_b200.h"
+
+namespace moe {
+
+// First 256 bytes of every workspace.
+struct Control {
+  uint32_t err;           // MOE_DEVERR_* bits, sticky until cleared
+  uint32_t route_ticket;  // blocks of the router that finished (reset by the last one)
+  uint32_t reserved[62];
+};
+static_assert(sizeof(Control) == 256, "control block is 256 bytes");
+
+constexpr size_t kAlign = 256;
+__host__ __device__ inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a; }
+
+__device__ __forceinline__ void set_error(Control* ctl, uint32_t bits) {
+  atomicOr(&ctl->err, bits);
+}
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t u) {
+  return __uint_as_float(static_cast<uint32_t>(u) << 16);
+}
+
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static __device__ __forceinline__ float to_f32(float v) { return v; }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+};
+
+// ------------------------------------------------------------------ launchers
+// Router. Tokens per router block (partials are per block).
+constexpr int kRouteFusedTokensPerBlock = 32;   // E <= 8 path: 8 warps x 4 tokens
+constexpr int kRouteSelectTokensPerBlock = 64;  // general path
+int route_num_blocks(int T, int E);
+size_t route_partials_bytes(int T, int E);
+cudaError_t launch_route(const void* x, const void* wg, const float* bias, moe_dtype_t dt, int T,
+                         int d, int E, int k, int32_t* idx, float* w, float* aux, float* logits,
+                         float* probs, float* logits_scratch, void* partials, Control* ctl,
+                         cudaStream_t s);
+size_t route_logits_scratch_bytes(int T, int d, int E);
+
+// Permute.
+size_t permute_scratch_bytes(int T, int k, int E);
+cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int64_t cap, int32_t* counts,
+                           int32_t* bins, int32_t* sorted_slot, int32_t* slot_to_row,
+                           int32_t* row_slot, uint8_t* drop, int32_t* kept, int32_t* seg,
+                           int32_t* rank_scratch, Control* ctl, cudaStream_t s);
+
+// Gather.
+cudaError_t launch_gather(const void* x, size_t elem, int T, int d, int k, const int32_t* row_slot,
+                          const int32_t* seg, int E, int64_t rows_max, void* x_perm, Control* ctl,
+                          cudaStream_t s);
+
+// Grouped GEMMs.
+cudaError_t launch_ffn_bf16(const void* x_perm, const void* w1, const void* w3, const void* w2,
+                            moe_act_t act, int64_t rows_max, int d, int F, int E,
+                            const int32_t* seg, void* h, void* y, Control* ctl, cudaStream_t s,
+                            cudaEvent_t after_up);
+cudaError_t launch_ffn_f32(const float* x_perm, const float* w1, const float* w3, const float* w2,
+                           moe_act_t act, int64_t rows_max, int d, int F, int E,
+                           const int32_t* seg, float* h, float* y, Control* ctl, cudaStream_t s,
+                           cudaEvent_t after_up);
+
+// Combine.
+cudaError_t launch_combine(const void* y, const float* w, const int32_t* slot_to_row, size_t elem,
+                           int T, int d, int k, int64_t rows_max, void* out, Control* ctl,
+                           cudaStream_t s);
+
+int num_sms();
+
+}  // namespace moe

@@ -1,0 +1,207 @@
+// Gather (x rows into expert-contiguous order) and the weighted combine.
+//
+// Gather: "MegaBlocks 01", section 4.3 (binned_gather reorders [tokens, hs]
+// by the sort; the token of flat slot s is s / top_k), here without padding.
+// Each warp's lane 0 drives a ring of shared-memory buffers with bulk (TMA)
+// copies: cp.async.bulk global->shared completing on an mbarrier, then
+// cp.async.bulk shared->global into the gathered row. No multicast.
+//
+// Combine: "ops-transformer MoE operators", 原理 Step 4 (weighted sum of the
+// chosen experts' outputs) and "MegaBlocks 01", sections 4.3 and 5 (multiply by
+// the router weight and sum over top-k; dropped slots contribute zero). The
+// kernel gathers each token's k rows instead of scattering: every output
+// element is written once, by one thread, in a fixed j order (no atomics).
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kGatherWarps = 4;
+constexpr int kGatherBufs = 4;
+constexpr int kGatherPiece = 8192;  // bytes per buffer
+
+__global__ void __launch_bounds__(kGatherWarps * 32)
+gather_bulk(const uint8_t* __restrict__ x, uint32_t row_bytes, int T, int k,
+            const int32_t* __restrict__ row_slot, const int32_t* __restrict__ seg, int E,
+            long long rows_max, uint8_t* __restrict__ x_perm, Control* ctl) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ __align__(8) uint64_t bars[kGatherWarps][kGatherBufs];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane != 0) return;
+
+  long long R = __ldg(seg + E);
+  if (R > rows_max || R < 0) {
+    set_error(ctl, MOE_DEVERR_ROW_RANGE);
+    R = R < 0 ? 0 : rows_max;
+  }
+  const long long S = static_cast<long long>(T) * k;
+  const uint32_t ppr = (row_bytes + kGatherPiece - 1) / kGatherPiece;  // pieces per row
+  const long long total = R * ppr;
+  const long long gw = static_cast<long long>(blockIdx.x) * kGatherWarps + warp;
+  const long long tw = static_cast<long long>(gridDim.x) * kGatherWarps;
+  if (gw >= total) return;
+  const long long mine = (total - gw + tw - 1) / tw;
+
+  uint8_t* buf0 = smem + static_cast<size_t>(warp) * kGatherBufs * kGatherPiece;
+  for (int b = 0; b < kGatherBufs; ++b) mbar_init(&bars[warp][b], 1);
+  fence_mbar_init();
+
+  // Source / destination / size of the i-th piece of this warp. A bad slot
+  // index is reported and the piece is skipped (size 0).
+  auto piece = [&](long long i, const uint8_t*& src, uint8_t*& dst, uint32_t& bytes) {
+    const long long p = gw + i * tw;
+    const long long row = p / ppr;
+    const uint32_t off = static_cast<uint32_t>(p % ppr) * kGatherPiece;
+    const int slot = __ldg(row_slot + row);
+    bytes = min(static_cast<uint32_t>(kGatherPiece), row_bytes - off);
+    if (slot < 0 || slot >= S) {
+      set_error(ctl, MOE_DEVERR_ROW_RANGE);
+      bytes = 0;
+      return;
+    }
+    src = x + static_cast<size_t>(slot / k) * row_bytes + off;
+    dst = x_perm + static_cast<size_t>(row) * row_bytes + off;
+  };
+
+  const uint8_t* srcs[kGatherBufs];
+  uint8_t* dsts[kGatherBufs];
+  uint32_t sizes[kGatherBufs];
+  uint32_t phase = 0;  // bit b: parity to wait for on buffer b
+  const long long pro = mine < kGatherBufs ? mine : kGatherBufs;
+  for (long long i = 0; i < pro; ++i) {
+    piece(i, srcs[i], dsts[i], sizes[i]);
+    if (sizes[i]) {
+      mbar_arrive_expect_tx(&bars[warp][i], sizes[i]);
+      bulk_load(buf0 + i * kGatherPiece, srcs[i], sizes[i], &bars[warp][i]);
+    }
+  }
+  bool ok = true;
+  for (long long i = 0; i < mine && ok; ++i) {
+    const int b = static_cast<int>(i % kGatherBufs);
+    if (sizes[b]) {
+      if (!mbar_wait_bounded(&bars[warp][b], (phase >> b) & 1u)) {
+        set_error(ctl, MOE_DEVERR_TIMEOUT);
+        ok = false;
+        break;
+      }
+      phase ^= 1u << b;
+      bulk_store(dsts[b], buf0 + b * kGatherPiece, sizes[b]);
+      bulk_commit();
+    }
+    const long long nxt = i + kGatherBufs;
+    if (nxt < mine) {
+      bulk_wait_read<0>();  // the store above has finished reading buffer b
+      piece(nxt, srcs[b], dsts[b], sizes[b]);
+      if (sizes[b]) {
+        mbar_arrive_expect_tx(&bars[warp][b], sizes[b]);
+        bulk_load(buf0 + b * kGatherPiece, srcs[b], sizes[b], &bars[warp][b]);
+      }
+    }
+  }
+  if (!ok) {
+    // Let every load still in flight land before the buffers go away.
+    for (int b = 0; b < kGatherBufs; ++b) (void)mbar_wait_bounded(&bars[warp][b], (phase >> b) & 1u);
+  }
+  bulk_wait<0>();
+}
+
+template <typename T>
+struct CombineVec;
+template <> struct CombineVec<__nv_bfloat16> {
+  static constexpr int kVec = 8;
+  static __device__ __forceinline__ void fma(const uint4& u, float w, float (&a)[8]) {
+    const uint32_t v[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      a[2 * i] = fmaf(w, __uint_as_float(v[i] << 16), a[2 * i]);
+      a[2 * i + 1] = fmaf(w, __uint_as_float(v[i] & 0xffff0000u), a[2 * i + 1]);
+    }
+  }
+  static __device__ __forceinline__ uint4 pack(const float (&a)[8]) {
+    uint32_t v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(a[2 * i], a[2 * i + 1]);
+      v[i] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    return make_uint4(v[0], v[1], v[2], v[3]);
+  }
+};
+template <> struct CombineVec<float> {
+  static constexpr int kVec = 4;
+  static __device__ __forceinline__ void fma(const uint4& u, float w, float (&a)[4]) {
+    a[0] = fmaf(w, __uint_as_float(u.x), a[0]);
+    a[1] = fmaf(w, __uint_as_float(u.y), a[1]);
+    a[2] = fmaf(w, __uint_as_float(u.z), a[2]);
+    a[3] = fmaf(w, __uint_as_float(u.w), a[3]);
+  }
+  static __device__ __forceinline__ uint4 pack(const float (&a)[4]) {
+    return make_uint4(__float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]),
+                      __float_as_uint(a[3]));
+  }
+};
+
+constexpr int kCombineThreads = 128;
+
+// grid.x = token, grid.y = column chunk of kCombineThreads * kVec elements.
+template <typename T>
+__global__ void __launch_bounds__(kCombineThreads)
+combine_gather(const T* __restrict__ y, const float* __restrict__ w,
+               const int32_t* __restrict__ slot_to_row, int d, int k, long long rows_max,
+               T* __restrict__ out, Control* ctl) {
+  constexpr int V = CombineVec<T>::kVec;
+  const int t = blockIdx.x;
+  const int col = (blockIdx.y * kCombineThreads + threadIdx.x) * V;
+  if (col >= d) return;
+  float acc[V];
+#pragma unroll
+  for (int i = 0; i < V; ++i) acc[i] = 0.f;
+  for (int j = 0; j < k; ++j) {
+    const int row = __ldg(slot_to_row + static_cast<size_t>(t) * k + j);
+    if (row < 0) continue;
+    if (row >= rows_max) {
+      if (col == 0) set_error(ctl, MOE_DEVERR_ROW_RANGE);
+      continue;
+    }
+    const float wj = __ldg(w + static_cast<size_t>(t) * k + j);
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(row) * d + col));
+    CombineVec<T>::fma(u, wj, acc);
+  }
+  *reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * d + col) = CombineVec<T>::pack(acc);
+}
+
+}  // namespace
+
+cudaError_t launch_gather(const void* x, size_t elem, int T, int d, int k, const int32_t* row_slot,
+                          const int32_t* seg, int E, int64_t rows_max, void* x_perm, Control* ctl,
+                          cudaStream_t s) {
+  if (rows_max <= 0 || T <= 0) return cudaSuccess;
+  const uint32_t row_bytes = static_cast<uint32_t>(static_cast<size_t>(d) * elem);
+  const size_t smem = static_cast<size_t>(kGatherWarps) * kGatherBufs * kGatherPiece;
+  cudaFuncSetAttribute(gather_bulk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  gather_bulk<<<num_sms(), kGatherWarps * 32, smem, s>>>(
+      static_cast<const uint8_t*>(x), row_bytes, T, k, row_slot, seg, E, rows_max,
+      static_cast<uint8_t*>(x_perm), ctl);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const void* y, const float* w, const int32_t* slot_to_row, size_t elem,
+                           int T, int d, int k, int64_t rows_max, void* out, Control* ctl,
+                           cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  const int vec = elem == 2 ? 8 : 4;
+  dim3 grid(T, (d + kCombineThreads * vec - 1) / (kCombineThreads * vec));
+  if (elem == 2)
+    combine_gather<__nv_bfloat16><<<grid, kCombineThreads, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(y), w, slot_to_row, d, k, rows_max,
+        static_cast<__nv_bfloat16*>(out), ctl);
+  else
+    combine_gather<float><<<grid, kCombineThreads, 0, s>>>(static_cast<const float*>(y), w,
+                                                          slot_to_row, d, k, rows_max,
+                                                          static_cast<float*>(out), ctl);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

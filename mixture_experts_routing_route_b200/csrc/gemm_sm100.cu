@@ -1,0 +1,412 @@
+// Grouped expert GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// "MegaBlocks 01 - why MoE is hard", section 2 (the per-expert GEMMs are
+// small, variable in M and skewed) and section 4.3 (bmm -> activation -> bmm
+// over weights [E, hs, ffn]). Instead of padding every expert to a fixed
+// capacity, the experts' rows are contiguous segments of one matrix and the
+// kernel walks a device-side list of 128-row tiles, so M varies per expert
+// with no host synchronisation and experts with no rows read no weights.
+//
+//   C[rows of e, n-tile] = epilogue( A[rows of e, :] . B[e][:, n-tile] )
+//   A: [rows_max, K] bf16 row-major (K-major operand)
+//   B: [E, K, N] bf16 row-major (MN-major operand; the pages' layout)
+//   epilogue: SwiGLU (two B matrices, W_gate and W_up, side by side in one
+//             N=256 MMA: silu(gate) * up), GELU (exact erf), or plain store;
+//             fp32 in registers, rounded once to bf16.
+//
+// CTA = 6 warps, one CTA per SM, persistent over tiles:
+//   warp 0   TMA producer: A tile 128x64 and B tile 64xN per stage, 128-byte
+//            swizzle, into a 4-stage shared-memory ring (mbarrier full/empty)
+//   warp 1   MMA issuer: one thread issues tcgen05.mma (M=128, N=256, K=16)
+//            into a double-buffered fp32 accumulator in tensor memory and
+//            frees ring slots / publishes accumulators with tcgen05.commit
+//   warps 2-5 epilogue: tcgen05.ld of their 32-lane quarter of the
+//            accumulator, activation, bf16 stores of valid rows only
+// Tiles are ordered expert-major, then N, with the M tile fastest, so CTAs
+// that run at the same time share one weight column block through L2.
+// Every wait is bounded; a time-out sets MOE_DEVERR_TIMEOUT and unwinds.
+#include "common.cuh"
+#include "ptx.cuh"
+#include <cudaTypedefs.h>
+#include <cmath>
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle row
+constexpr int STAGES = 4;
+constexpr int kThreads = 192;
+constexpr int kMaxE = 256;
+
+enum { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_STORE = 2 };
+
+template <int EPI, int NMMA>
+struct Cfg {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BK * NMMA * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int OUT_N = EPI == EPI_SWIGLU ? NMMA / 2 : NMMA;
+  static constexpr int B_BOXES = NMMA / 64;  // 64-column boxes of 8 KB
+  static constexpr int TMEM_COLS = 2 * NMMA;
+  static constexpr size_t SMEM = static_cast<size_t>(STAGES) * STAGE_BYTES + 1024;
+  static constexpr uint32_t IDESC = make_idesc_bf16(BM, NMMA);
+};
+
+struct GemmArgs {
+  const int32_t* seg;  // [E+1] row segment offsets
+  __nv_bfloat16* out;  // [rows_max, N]
+  int E;
+  int K;
+  int N;  // output columns
+  long long rows_max;
+  Control* ctl;
+};
+
+__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+__device__ __forceinline__ float gelu_erf(float z) {
+  return 0.5f * z * (1.0f + erff(z * 0.70710678118654752440f));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Tile -> (expert, row start, valid rows, n0).
+struct Tile {
+  int e, row0, rows, n0;
+};
+
+__device__ __forceinline__ Tile decode_tile(int tau, const int* tile_start, const int* seg, int E,
+                                            int ntn, int out_n) {
+  int lo = 0, hi = E - 1;  // last e with tile_start[e] <= tau
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tile_start[mid] <= tau) lo = mid; else hi = mid - 1;
+  }
+  const int e = lo;
+  const int m_e = seg[e + 1] - seg[e];
+  const int mt_e = (m_e + BM - 1) / BM;
+  const int local = tau - tile_start[e];
+  const int nt = local / mt_e, mt = local - nt * mt_e;
+  Tile t;
+  t.e = e;
+  t.row0 = seg[e] + mt * BM;
+  t.rows = min(BM, m_e - mt * BM);
+  t.n0 = nt * out_n;
+  (void)ntn;
+  return t;
+}
+
+template <int EPI, int NMMA>
+__global__ void __launch_bounds__(kThreads, 1)
+grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                const __grid_constant__ CUtensorMap tmB1, GemmArgs args) {
+  using C = Cfg<EPI, NMMA>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t tfull_bar[2], tempty_bar[2], drain_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int seg_s[kMaxE + 1];
+  __shared__ int tile_start_s[kMaxE + 1];
+  __shared__ volatile int abort_s;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = args.E;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+
+  // ---- schedule: per-expert tile counts and their prefix
+  for (int i = threadIdx.x; i <= E; i += kThreads) seg_s[i] = __ldg(args.seg + i);
+  if (threadIdx.x == 0) abort_s = 0;
+  __syncthreads();
+  const int ntn = args.N / C::OUT_N;
+  if (warp == 0) {
+    // lane l owns experts [8l, 8l+8)
+    int loc[8];
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane * 8 + i;
+      int m = 0;
+      if (e < E) {
+        m = seg_s[e + 1] - seg_s[e];
+        if (m < 0 || seg_s[e] < 0 || seg_s[e + 1] > args.rows_max) {
+          set_error(args.ctl, MOE_DEVERR_ROW_RANGE);
+          m = 0;
+        }
+      }
+      loc[i] = ((m + BM - 1) / BM) * ntn;
+      sum += loc[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += n;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane * 8 + i;
+      if (e < E) tile_start_s[e] = run;
+      run += loc[i];
+    }
+    // The lanes cover experts 0..255 only; the total goes to entry E (which
+    // is 256 when E = 256). Experts >= E contributed 0 tiles to the sum.
+    if (lane == 31) tile_start_s[E] = incl;
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&tfull_bar[b], 1); mbar_init(&tempty_bar[b], 4); }
+    mbar_init(&drain_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_s, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+  // A segment whose rows are out of range gets zero tiles; the true total is
+  // the prefix at E (entries past a bad segment were computed with m = 0).
+  const int total = tile_start_s[E];
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tmA);
+      prefetch_tmap(&tmB0);
+      prefetch_tmap(&tmB1);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0;  // stages that ever received a load
+      uint32_t last_parity = 0;  // parity of that stage's latest load
+      const int nkb = args.K / BK;
+      for (int tau = blockIdx.x; tau < total && !abort_s; tau += gridDim.x) {
+        const Tile t = decode_tile(tau, tile_start_s, seg_s, E, ntn, C::OUT_N);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u)) {
+            set_error(args.ctl, MOE_DEVERR_TIMEOUT);
+            abort_s = 1;
+            break;
+          }
+          uint8_t* sa = smem + stage * C::STAGE_BYTES;
+          uint8_t* sb = sa + C::A_BYTES;
+          mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
+          tma_load_2d(sa, &tmA, &full_bar[stage], kb * BK, t.row0);
+          const int brow = t.e * args.K + kb * BK;
+#pragma unroll
+          for (int j = 0; j < C::B_BOXES; ++j) {
+            if (EPI == EPI_SWIGLU) {
+              constexpr int H = C::B_BOXES / 2;
+              tma_load_2d(sb + j * 8192, j < H ? &tmB0 : &tmB1, &full_bar[stage],
+                          t.n0 + (j % H) * 64, brow);
+            } else {
+              tma_load_2d(sb + j * 8192, &tmB0, &full_bar[stage], t.n0 + j * 64, brow);
+            }
+          }
+          issued_mask |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // Every load issued must have landed before the CTA may exit.
+      for (int s = 0; s < STAGES; ++s)
+        if (issued_mask & (1u << s)) (void)mbar_wait_bounded(&full_bar[s], (last_parity >> s) & 1u);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      const int nkb = args.K / BK;
+      bool issued_any = false;
+      for (int tau = blockIdx.x; tau < total && !abort_s; tau += gridDim.x) {
+        if (!mbar_wait_bounded(&tempty_bar[acc], acc_phase ^ 1u)) {
+          set_error(args.ctl, MOE_DEVERR_TIMEOUT);
+          abort_s = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * NMMA;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&full_bar[stage], phase)) {
+            set_error(args.ctl, MOE_DEVERR_TIMEOUT);
+            abort_s = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t adesc = make_sw128_desc(a_addr + kk * 32, 16, 1024);
+            const uint64_t bdesc = make_sw128_desc(b_addr + kk * 2048, 8192, 1024);
+            umma_bf16(d_tmem, adesc, bdesc, C::IDESC, (kb | kk) != 0 ? 1u : 0u);
+          }
+          issued_any = true;
+          umma_commit(&empty_bar[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&tfull_bar[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (issued_any) {
+        // Tensor memory is freed below: wait until every MMA issued is done.
+        umma_commit(&drain_bar);
+        (void)mbar_wait_bounded(&drain_bar, 0);
+      }
+    }
+  } else {
+    // epilogue warps 2..5: TMEM lane quarter = warp % 4
+    const int q = warp & 3;
+    const int r_in_tile = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
+      // Lane 0 polls and decides for the whole warp, so the warp-wide
+      // tcgen05.ld below always runs converged.
+      int ok = 0;
+      if (lane == 0) {
+        ok = !abort_s && mbar_wait_bounded(&tfull_bar[acc], acc_phase);
+        if (!ok && !abort_s) {
+          set_error(args.ctl, MOE_DEVERR_TIMEOUT);
+          abort_s = 1;
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      const Tile t = decode_tile(tau, tile_start_s, seg_s, E, ntn, C::OUT_N);
+      tc_fence_after();
+      const bool valid = r_in_tile < t.rows;
+      __nv_bfloat16* orow = args.out + static_cast<size_t>(t.row0 + r_in_tile) * args.N + t.n0;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * NMMA;
+#pragma unroll 1
+      for (int c = 0; c < C::OUT_N; c += 32) {
+        uint32_t v[32];
+        uint32_t packed[16];
+        if (EPI == EPI_SWIGLU) {
+          uint32_t u[32];
+          tmem_ld_32x32b_x32(tbase + c, v);
+          tmem_ld_32x32b_x32(tbase + C::OUT_N + c, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float h0 = silu(__uint_as_float(v[2 * i])) * __uint_as_float(u[2 * i]);
+            const float h1 = silu(__uint_as_float(v[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+            packed[i] = pack_bf16(h0, h1);
+          }
+        } else {
+          tmem_ld_32x32b_x32(tbase + c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float a = __uint_as_float(v[2 * i]), b = __uint_as_float(v[2 * i + 1]);
+            if (EPI == EPI_GELU) { a = gelu_erf(a); b = gelu_erf(b); }
+            packed[i] = pack_bf16(a, b);
+          }
+        }
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ----------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 map over [rows, cols] row-major, box [box_rows, 64 cols], 128-B swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int EPI, int NMMA>
+cudaError_t run_gemm(const void* A, const void* B0, const void* B1, int64_t rows_max, int K, int N,
+                     int E, const int32_t* seg, void* out, Control* ctl, cudaStream_t s) {
+  using C = Cfg<EPI, NMMA>;
+  CUtensorMap ta, tb0, tb1;
+  if (!make_map(&ta, A, static_cast<uint64_t>(rows_max), K, BM)) return cudaErrorInvalidValue;
+  if (!make_map(&tb0, B0, static_cast<uint64_t>(E) * K, N, BK)) return cudaErrorInvalidValue;
+  if (!make_map(&tb1, B1 ? B1 : B0, static_cast<uint64_t>(E) * K, N, BK)) return cudaErrorInvalidValue;
+  GemmArgs a;
+  a.seg = seg;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.E = E;
+  a.K = K;
+  a.N = N;
+  a.rows_max = rows_max;
+  a.ctl = ctl;
+  auto kern = grouped_gemm_tc<EPI, NMMA>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM));
+  kern<<<num_sms(), kThreads, C::SMEM, s>>>(ta, tb0, tb1, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_ffn_bf16(const void* x_perm, const void* w1, const void* w3, const void* w2,
+                            moe_act_t act, int64_t rows_max, int d, int F, int E,
+                            const int32_t* seg, void* h, void* y, Control* ctl, cudaStream_t s,
+                            cudaEvent_t after_up) {
+  if (rows_max <= 0) {
+    if (after_up) cudaEventRecord(after_up, s);
+    return cudaSuccess;
+  }
+  cudaError_t err;
+  if (act == MOE_ACT_SWIGLU)
+    err = run_gemm<EPI_SWIGLU, 256>(x_perm, w1, w3, rows_max, d, F, E, seg, h, ctl, s);
+  else if (F % 256 == 0)
+    err = run_gemm<EPI_GELU, 256>(x_perm, w1, nullptr, rows_max, d, F, E, seg, h, ctl, s);
+  else
+    err = run_gemm<EPI_GELU, 128>(x_perm, w1, nullptr, rows_max, d, F, E, seg, h, ctl, s);
+  if (err != cudaSuccess) return err;
+  if (after_up) cudaEventRecord(after_up, s);
+  if (d % 256 == 0)
+    err = run_gemm<EPI_STORE, 256>(h, w2, nullptr, rows_max, F, d, E, seg, y, ctl, s);
+  else
+    err = run_gemm<EPI_STORE, 128>(h, w2, nullptr, rows_max, F, d, E, seg, y, ctl, s);
+  return err;
+}
+
+}  // namespace moe

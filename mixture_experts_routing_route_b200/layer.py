@@ -1,0 +1,99 @@
+"""MoeLayer: a user-facing handle around the C ABI's whole-layer forward.
+
+Holds the layer's device weights and a workspace (device memory allocated by
+torch: plumbing only), fills the C layer struct, and calls moe_forward /
+moe_forward_host. Intermediates of the last forward can be read as torch views
+of the workspace.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import _abi as abi
+
+
+class MoeLayer:
+    def __init__(self, w_router: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
+                 w3: Optional[torch.Tensor] = None, bias: Optional[torch.Tensor] = None,
+                 k: int = 2, act: str = "swiglu", capacity_factor: float = 0.0):
+        if not w1.is_cuda:
+            raise ValueError("weights must be CUDA tensors")
+        self.E, self.d, self.F = w1.shape
+        self.k = k
+        self.dtype = w1.dtype
+        self.act = abi.MOE_ACT_SWIGLU if act == "swiglu" else abi.MOE_ACT_GELU
+        self.cf = float(capacity_factor)
+        self.w_router = w_router.contiguous()
+        self.w1 = w1.contiguous()
+        self.w3 = None if w3 is None else w3.contiguous()
+        self.w2 = w2.contiguous()
+        self.bias = None if bias is None else bias.to(device=w1.device, dtype=torch.float32).contiguous()
+        self.c = abi.layer_struct(self.d, self.E, k, self.F, abi.dtype_code(self.dtype), self.act,
+                                  self.cf, self.w_router, self.bias, self.w1, self.w3, self.w2)
+        self._ws = {}
+
+    def workspace(self, T: int, host_io: bool = False, stream=None) -> torch.Tensor:
+        key = (T, host_io)
+        if key not in self._ws:
+            n = (abi.moe_forward_host_workspace_size(self.c, T) if host_io
+                 else abi.moe_forward_workspace_size(self.c, T))
+            ws = torch.empty(max(n, 256), dtype=torch.uint8, device=self.w1.device)
+            abi.moe_workspace_init(ws, stream)
+            self._ws[key] = ws
+        return self._ws[key]
+
+    def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None,
+                aux: Optional[torch.Tensor] = None, stream=None, events=None):
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty(T, self.d, dtype=self.dtype, device=x.device)
+        if aux is None:
+            aux = torch.empty(1, dtype=torch.float32, device=x.device)
+        ws = self.workspace(T, stream=stream)
+        abi.moe_forward(self.c, x, T, out, aux, ws, stream, events)
+        return out, aux
+
+    __call__ = forward
+
+    def forward_host(self, x_host: torch.Tensor, out_host: torch.Tensor, aux_host: torch.Tensor,
+                     stream=None):
+        T = x_host.shape[0]
+        ws = self.workspace(T, host_io=True, stream=stream)
+        abi.moe_forward_host(self.c, x_host, T, out_host, aux_host, ws, stream)
+
+    def device_error(self, T: int, stream=None) -> int:
+        return abi.moe_get_device_error(self.workspace(T, stream=stream), stream)
+
+    def views(self, T: int) -> dict:
+        """Torch views of the intermediates moe_forward left in the workspace."""
+        ws = self.workspace(T)
+        v = abi.moe_forward_views(self.c, T, ws)
+        base = ws.data_ptr()
+        R = v.rows_max
+        S = T * self.k
+
+        def view(ptr, n, dt, shape):
+            es = torch.empty(0, dtype=dt).element_size()
+            off = ptr - base
+            return ws[off:off + n * es].view(dt).view(*shape)
+
+        return {
+            "topk_idx": view(v.topk_idx, S, torch.int32, (T, self.k)),
+            "topk_w": view(v.topk_w, S, torch.float32, (T, self.k)),
+            "aux": view(v.aux_loss, 1, torch.float32, (1,)),
+            "counts": view(v.counts, self.E, torch.int32, (self.E,)),
+            "bins": view(v.bins, self.E, torch.int32, (self.E,)),
+            "kept_counts": view(v.kept_counts, self.E, torch.int32, (self.E,)),
+            "seg_offsets": view(v.seg_offsets, self.E + 1, torch.int32, (self.E + 1,)),
+            "sorted_slot": view(v.sorted_slot, S, torch.int32, (S,)),
+            "slot_to_row": view(v.slot_to_row, S, torch.int32, (S,)),
+            "row_slot": view(v.row_slot, R, torch.int32, (R,)),
+            "drop": view(v.drop_mask, S, torch.uint8, (S,)),
+            "x_perm": view(v.x_perm, R * self.d, self.dtype, (R, self.d)),
+            "h": view(v.h, R * self.F, self.dtype, (R, self.F)),
+            "y_perm": view(v.y_perm, R * self.d, self.dtype, (R, self.d)),
+            "rows_max": R,
+            "capacity": v.capacity,
+        }

@@ -1,0 +1,82 @@
+"""The C-ABI library without a GPU: it builds, loads, exports every function
+include/moe_b200.h declares, and its host-only logic (capacity, row bounds,
+workspace sizes, argument checks that return before any launch) is right."""
+import ctypes
+
+import pytest
+
+from mixture_experts_routing_route_b200 import build as build_mod
+
+
+@pytest.fixture(scope="module")
+def abi():
+    build_mod.build()
+    from mixture_experts_routing_route_b200 import _abi
+    return _abi
+
+
+def test_exports_every_declared_function(abi):
+    declared = abi.header_functions()
+    assert len(declared) >= 15
+    lib = ctypes.CDLL(abi.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_capacity_matches_oracle_formula(abi):
+    from oracle import moe_oracle as O
+    for cf, k, T, E in [(1.25, 1, 256, 4), (1.0, 2, 16384, 64), (1.25, 2, 32768, 8), (1.1, 3, 10, 4),
+                        (0.05, 1, 64, 4), (0.0, 2, 100, 8), (-1.0, 2, 5, 2), (2.5, 8, 4096, 256)]:
+        ref = O.capacity(cf, k, T, E)
+        assert abi.moe_capacity(cf, T, k, E) == (-1 if ref is None else ref)
+
+
+def test_rows_max(abi):
+    assert abi.moe_rows_max(100, 2, 8, -1) == 200
+    assert abi.moe_rows_max(100, 2, 8, 10) == 80
+    assert abi.moe_rows_max(100, 2, 8, 1000) == 200
+    assert abi.moe_rows_max(0, 2, 8, -1) == 0
+
+
+def test_workspace_sizes_grow(abi):
+    a = abi.moe_route_workspace_size(4096, 4096, 8)
+    b = abi.moe_route_workspace_size(32768, 4096, 8)
+    assert 256 < a < b
+    assert abi.moe_permute_workspace_size(4096, 2, 8) >= 256 + 4096 * 2 * 4
+    L = abi.MoeLayerC(4096, 8, 2, 14336, abi.MOE_BF16, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, 16, 16)
+    n = abi.moe_forward_workspace_size(L, 4096)
+    # x_perm + h + y_perm alone: 8192 rows of (4096 + 14336 + 4096) bf16
+    assert n >= 8192 * (4096 + 14336 + 4096) * 2
+    assert abi.moe_forward_host_workspace_size(L, 4096) >= n + 2 * 4096 * 4096 * 2
+
+
+def _call_route(abi, **over):
+    a = dict(x=16, wg=16, bias=None, dt=abi.MOE_BF16, T=8, d=128, E=8, k=2, idx=16, w=16, aux=16,
+             logits=None, probs=None, ws=16, ws_bytes=1 << 30)
+    a.update(over)
+    return abi._lib.moe_route(a["x"], a["wg"], a["bias"], a["dt"], a["T"], a["d"], a["E"], a["k"],
+                              a["idx"], a["w"], a["aux"], a["logits"], a["probs"], a["ws"],
+                              a["ws_bytes"], None)
+
+
+def test_argument_checks_return_before_launch(abi):
+    # every case here fails a host check, so nothing is launched
+    assert _call_route(abi, x=None) == 1                      # MOE_ERR_NULL
+    assert _call_route(abi, k=9) == 2                         # k > 8
+    assert _call_route(abi, E=4, k=5) == 2                    # k > E
+    assert _call_route(abi, E=257) == 2                       # E > 256
+    assert _call_route(abi, d=96) == 3                        # bf16 needs d % 128 == 0
+    assert _call_route(abi, x=24) == 5                        # misaligned pointer
+    assert _call_route(abi, ws_bytes=100) == 4                # workspace too small
+    assert _call_route(abi, T=-1) == 2
+    assert abi._lib.moe_workspace_init(None, 256, None) == 1
+    L = abi.MoeLayerC(4096, 8, 2, 100, abi.MOE_BF16, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, 16, 16)
+    assert abi._lib.moe_forward(ctypes.byref(L), 16, 4, 16, None, 16, 1 << 40, None, None) == 3
+    L2 = abi.MoeLayerC(4096, 8, 2, 128, abi.MOE_BF16, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, None, 16)
+    assert abi._lib.moe_forward(ctypes.byref(L2), 16, 4, 16, None, 16, 1 << 40, None, None) == 1
+    assert abi._lib.moe_permute(16, 4, 2, 0, -1, *([16] * 8), 16, 1 << 20, None) == 2
+
+
+def test_status_strings(abi):
+    for st in range(8):
+        assert abi.status_string(st)

@@ -1,0 +1,183 @@
+"""GPU parity of each C-ABI stage entry point on its own (moe_route,
+moe_permute, moe_gather, moe_expert_ffn, moe_combine), stage-chained against
+the CPU oracle, plus the permute's edge cases and its device error word."""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_routing_route_b200 import _abi as abi
+from mixture_experts_routing_route_b200.inputs import small_case
+from oracle import moe_oracle as O
+from tests.gpu_helpers import (TOL_AUX_REL, TOL_BF16_OUT, TOL_PROB_REL, ExpertWeights,
+                               max_err_ratio, new_ws, np32, npi, rel_err)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def route_on_gpu(x, wg, bias, T, d, E, k):
+    idx = torch.empty(T, k, dtype=torch.int32, device=DEV)
+    w = torch.empty(T, k, dtype=torch.float32, device=DEV)
+    aux = torch.empty(1, dtype=torch.float32, device=DEV)
+    logits = torch.empty(T, E, dtype=torch.float32, device=DEV)
+    probs = torch.empty(T, E, dtype=torch.float32, device=DEV)
+    ws = new_ws(abi.moe_route_workspace_size(T, d, E))
+    abi.moe_route(x, wg, bias, T, d, E, k, idx, w, aux, logits, probs, ws)
+    torch.cuda.synchronize()
+    assert abi.moe_get_device_error(ws) == 0
+    return idx, w, aux, logits, probs
+
+
+@pytest.mark.parametrize("T,d,E,k,dt,bias", [
+    (1000, 512, 8, 2, "bf16", "none"),     # fused E <= 8 path
+    (77, 4096, 8, 2, "bf16", "expert0"),   # fused, d = 4096, ragged quad
+    (300, 256, 5, 3, "bf16", "none"),      # fused with E < 8 (padded experts)
+    (513, 256, 64, 2, "bf16", "zipf"),     # tiled GEMM + select, 2 experts per lane
+    (129, 256, 256, 8, "bf16", "none"),    # 8 experts per lane, k = 8
+    (200, 64, 4, 1, "f32", "none"),        # fp32 fused
+    (90, 64, 40, 4, "f32", "none"),        # fp32 general
+])
+def test_route(T, d, E, k, dt, bias):
+    inp = small_case("r", T=T, d=d, E=E, k=k, F=128, act="gelu", dtype=dt, bias=bias, seed=T + E)
+    x, wg = inp.x.to(DEV), inp.wg.to(DEV)
+    b = None if inp.bias is None else inp.bias.to(DEV)
+    idx, w, aux, logits, probs = route_on_gpu(x, wg, b, T, d, E, k)
+    r = O.route(np32(inp.x), np32(inp.wg), None if inp.bias is None else inp.bias.numpy(), k)
+    g_logits = np32(logits)
+    # fp32 accumulation of the gate GEMM: close to the exact logits
+    assert np.max(np.abs(g_logits - r["logits"])) <= 1e-5 * max(1.0, np.max(np.abs(r["logits"])))
+    # top-k decided on the GPU's own fp32 logits: bit-exact with the oracle's selection of them
+    assert np.array_equal(npi(idx), O.topk_select(g_logits, k))
+    ok = ~r["near_tie"]
+    assert np.array_equal(npi(idx)[ok], r["topk_idx"][ok])
+    assert rel_err(np32(probs), r["probs64"]) <= TOL_PROB_REL
+    g_idx = npi(idx).astype(np.int64)
+    assert rel_err(np32(w), O.renormalise(r["probs64"], g_idx)) <= TOL_PROB_REL
+    aux_ref = O.aux_loss(r["probs64"], g_idx, E)
+    assert abs(float(aux.item()) - aux_ref) <= TOL_AUX_REL * aux_ref
+
+
+def test_route_exact_ties_lower_index():
+    """Hand-placed exact ties (integer-valued logits) go to the lower expert."""
+    T, d, E, k = 64, 128, 8, 3
+    rng = np.random.default_rng(5)
+    x = np.zeros((T, d), np.float32)
+    x[:, :E] = rng.integers(-2, 3, size=(T, E))
+    wg = np.zeros((d, E), np.float32)
+    wg[:E, :E] = np.eye(E)
+    for dt in (torch.bfloat16, torch.float32):
+        xt = torch.from_numpy(x).to(dt).to(DEV)
+        wt = torch.from_numpy(wg).to(dt).to(DEV)
+        idx, *_ = route_on_gpu(xt, wt, None, T, d, E, k)
+        assert np.array_equal(npi(idx), O.topk_select(x[:, :E], k))
+    E2 = 40
+    wg2 = np.zeros((d, E2), np.float32)
+    wg2[:E2, :E2] = np.eye(E2)
+    x2 = np.zeros((T, d), np.float32)
+    x2[:, :E2] = rng.integers(-1, 2, size=(T, E2))
+    idx, *_ = route_on_gpu(torch.from_numpy(x2).to(DEV), torch.from_numpy(wg2).to(DEV), None, T, d, E2, 5)
+    assert np.array_equal(npi(idx), O.topk_select(x2[:, :E2], 5))
+
+
+def permute_on_gpu(idx_np, E, cap):
+    T, k = idx_np.shape
+    S = T * k
+    R = abi.moe_rows_max(T, k, E, cap)
+    t = lambda n: torch.full((max(n, 1),), -7, dtype=torch.int32, device=DEV)
+    out = {"counts": t(E), "bins": t(E), "sorted_slot": t(S), "slot_to_row": t(S),
+           "row_slot": t(R), "kept_counts": t(E), "seg_offsets": t(E + 1)}
+    drop = torch.full((max(S, 1),), 7, dtype=torch.uint8, device=DEV)
+    ws = new_ws(abi.moe_permute_workspace_size(T, k, E))
+    idx = torch.from_numpy(np.ascontiguousarray(idx_np, dtype=np.int32)).to(DEV)
+    abi.moe_permute(idx, T, k, E, cap, out["counts"], out["bins"], out["sorted_slot"],
+                    out["slot_to_row"], out["row_slot"], drop, out["kept_counts"],
+                    out["seg_offsets"], ws)
+    torch.cuda.synchronize()
+    res = {kk: npi(vv) for kk, vv in out.items()}
+    res["drop"] = npi(drop)
+    res["err"] = abi.moe_get_device_error(ws)
+    return res
+
+
+def assert_permute_equal(g, ref, S, E):
+    assert g["err"] == 0
+    for key in ("counts", "bins", "kept_counts"):
+        assert np.array_equal(g[key][:E], ref[key]), key
+    assert np.array_equal(g["seg_offsets"][:E + 1], ref["seg_offsets"])
+    for key in ("sorted_slot", "slot_to_row"):
+        assert np.array_equal(g[key][:S], ref[key]), key
+    assert np.array_equal(g["drop"][:S], ref["drop"])
+    assert np.array_equal(g["row_slot"][:ref["rows"]], ref["row_slot"])
+
+
+@pytest.mark.parametrize("T,k,E", [(1, 1, 1), (5, 2, 3), (512, 2, 8), (1025, 1, 7), (3000, 8, 256),
+                                   (4096, 2, 64), (20000, 3, 17)])
+def test_permute_random(T, k, E):
+    rng = np.random.default_rng(T * 31 + E)
+    idx = np.array([rng.permutation(E)[:k] for _ in range(T)])
+    S = T * k
+    for cap in (-1, 0, 1, max(1, S // E), S):
+        g = permute_on_gpu(idx, E, cap)
+        ref = O.permute(idx, E, None if cap < 0 else cap)
+        assert_permute_equal(g, ref, S, E)
+
+
+def test_permute_skewed_and_forced():
+    """Skew (most slots on one expert) and the forced uniform assignment
+    (slot s -> expert s mod E, MegaBlocks section 5)."""
+    T, k, E = 3333, 2, 8
+    rng = np.random.default_rng(1)
+    idx = np.where(rng.random((T, k)) < 0.8, 0, rng.integers(1, E, size=(T, k)))
+    idx[:, 1] = np.where(idx[:, 1] == idx[:, 0], (idx[:, 0] + 1) % E, idx[:, 1])
+    for cap in (-1, 512, 2000):
+        assert_permute_equal(permute_on_gpu(idx, E, cap), O.permute(idx, E, None if cap < 0 else cap),
+                             T * k, E)
+    forced = (np.arange(T * k) % E).reshape(T, k)
+    assert_permute_equal(permute_on_gpu(forced, E, -1), O.permute(forced, E, None), T * k, E)
+
+
+def test_permute_bad_expert_id_sets_error_bit():
+    """An id outside [0, E) is reported in the device error word; the slot is
+    marked dropped and nothing is written out of bounds."""
+    idx = np.array([[0, 1], [2, 9], [3, 1]])
+    g = permute_on_gpu(idx, 4, -1)
+    assert g["err"] & abi.DEVERR_EXPERT_RANGE
+    assert g["slot_to_row"][3] == -1 and g["drop"][3] == 1
+
+
+def test_gather_ffn_combine_entry_points():
+    T, d, E, k, F = 400, 256, 8, 2, 256
+    inp = small_case("s", T=T, d=d, E=E, k=k, F=F, act="swiglu", seed=21)
+    x = inp.x.to(DEV)
+    idx, w, aux, logits, probs = route_on_gpu(x, inp.wg.to(DEV), None, T, d, E, k)
+    pm_ref = O.permute(npi(idx).astype(np.int64), E, None)
+    R = pm_ref["rows"]
+    row_slot = torch.from_numpy(pm_ref["row_slot"]).to(DEV)
+    seg = torch.from_numpy(pm_ref["seg_offsets"]).to(DEV)
+    s2r = torch.from_numpy(pm_ref["slot_to_row"]).to(DEV)
+    ws = new_ws(256)
+    x_perm = torch.empty(R, d, dtype=torch.bfloat16, device=DEV)
+    abi.moe_gather(x, T, d, k, row_slot, seg, E, R, x_perm, ws)
+    h = torch.empty(R, F, dtype=torch.bfloat16, device=DEV)
+    y = torch.empty(R, d, dtype=torch.bfloat16, device=DEV)
+    abi.moe_expert_ffn(x_perm, inp.w1.to(DEV), inp.w3.to(DEV), inp.w2.to(DEV), abi.MOE_ACT_SWIGLU,
+                       R, d, F, E, seg, h, y, ws)
+    out = torch.empty(T, d, dtype=torch.bfloat16, device=DEV)
+    abi.moe_combine(y, w, s2r, T, d, k, R, out, ws)
+    torch.cuda.synchronize()
+    assert abi.moe_get_device_error(ws) == 0
+    xp_ref = O.gather(np32(inp.x), pm_ref["row_slot"], k)
+    assert np.array_equal(np32(x_perm), xp_ref)
+    w1, w3, w2 = ExpertWeights(inp.w1), ExpertWeights(inp.w3), ExpertWeights(inp.w2)
+    # h: activation output before the down projection
+    h_ref = np.zeros((R, F))
+    for e in range(E):
+        a, b = pm_ref["seg_offsets"][e], pm_ref["seg_offsets"][e + 1]
+        if b > a:
+            h_ref[a:b] = O.activation(xp_ref[a:b] @ w1[e].astype(np.float64), "swiglu",
+                                      xp_ref[a:b] @ w3[e].astype(np.float64))
+    assert max_err_ratio(np32(h), h_ref) <= 1e-2
+    y_ref = O.expert_ffn(xp_ref, pm_ref["seg_offsets"], w1, w3, w2, "swiglu")
+    assert max_err_ratio(np32(y), y_ref) <= TOL_BF16_OUT
+    out_ref = O.combine(np32(y), np32(w), pm_ref["slot_to_row"], T, k)
+    assert max_err_ratio(np32(out), out_ref) <= 1e-2
