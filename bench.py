@@ -1,0 +1,454 @@
+"""Benchmark of the MoE-layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+
+One step = one whole-layer forward (route -> permute -> gather -> expert FFN
+up/down -> combine) over one batch of T tokens, through moe_forward with the
+inputs resident in HBM. The default workload is the Mixtral-shaped layer
+(T=4096, d=4096, E=8 experts, top-2, SwiGLU F=14336, bf16, dropless), synthetic
+and seeded. Prints one JSON line (rank 0).
+
+Timing: W untimed warm-up steps; then K steps bracketed by a barrier and a
+device synchronize; between steps a 256 MB buffer is written to flush L2
+(outside the timed events); every step is timed with CUDA events recorded on
+the launching stream by the library between its stages; the value is the
+whole-job token rate, max over ranks of the summed step time. N > 1 runs N
+independent replicas (one per GPU, each its own T tokens): the layer has no
+cross-GPU exchange step, so there is no data-path collective (weak scaling).
+
+--impl reference runs the CPU oracle (numpy float64) on the host cores as the
+reference arm, each step a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from mixture_experts_routing_route_b200.inputs import CONFIGS, make_inputs  # noqa: E402
+
+METRIC = "MoE-layer fwd tokens/s on 1 B200 (Mixtral 8e top-2 bf16)"
+UNIT = "tokens/s"
+STAGES = ["route", "permute", "gather", "ffn_up", "ffn_down", "combine"]
+FLUSH_BYTES = 256 << 20
+GEMM_SRC = os.path.join(ROOT, "mixture_experts_routing_route_b200", "csrc", "gemm_sm100.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.txt")
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--config", default="mixtral", choices=sorted(CONFIGS))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--T", type=int, default=None, help="override T (reduced case for profiling)")
+    p.add_argument("--E", type=int, default=None, help="override E (reduced case for profiling)")
+    return p.parse_args()
+
+
+def shape_of(args):
+    sh = CONFIGS[args.config]
+    if args.T is not None or args.E is not None:
+        sh = sh.with_(T=args.T or sh.T, E=args.E or sh.E,
+                      name=f"{sh.name}_T{args.T or sh.T}_E{args.E or sh.E}")
+    return sh
+
+
+def workload_config(sh):
+    return {"workload": f"{sh.name}: T={sh.T} d={sh.d} E={sh.E} top-{sh.k} {sh.act} F={sh.F} "
+                        f"{sh.dtype}" + (f" cf={sh.cf}" if sh.cf > 0 else " dropless")
+                        + ("" if sh.bias == "none" else f" bias={sh.bias}"),
+            "T": sh.T, "d": sh.d, "E": sh.E, "k": sh.k, "F": sh.F, "act": sh.act,
+            "capacity_factor": sh.cf, "global_batch_tokens": sh.T,
+            "l2": "256 MB buffer written between timed steps (outside the events)"}
+
+
+# ------------------------------------------------------------------ roofline
+def algorithmic(sh, counts_kept):
+    """Algorithmic flops and bytes per stage for one forward (no re-reads).
+
+    R = kept rows, E_act = experts with R_e > 0, b = element bytes.
+      route    bytes T*d*b + d*E*b + T*k*8 (x once, Wg once, idx + w out)
+      permute  bytes S*4 + S*(4+4+4+1) (idx in; sorted_slot, slot_to_row,
+               row_slot, drop out)
+      gather   bytes T_used*d*b + R*d*b (each token read once, rows written)
+      ffn_up   flops 2*R*d*F*(2 SwiGLU | 1 GELU); bytes weights of active
+               experts + R*d*b + R*F*b
+      ffn_down flops 2*R*F*d; bytes E_act*F*d*b + R*F*b + R*d*b
+      combine  bytes R*d*b + S*8 + T*d*b
+    """
+    b = 2 if sh.dtype == "bf16" else 4
+    T, d, E, k, F = sh.T, sh.d, sh.E, sh.k, sh.F
+    S = T * k
+    R = int(sum(counts_kept))
+    e_act = int(sum(1 for c in counts_kept if c > 0))
+    nup = 2 if sh.act == "swiglu" else 1
+    return {
+        "route": {"bytes": T * d * b + d * E * b + S * 8},
+        "permute": {"bytes": S * 4 + S * 13},
+        "gather": {"bytes": min(T, R) * d * b + R * d * b},
+        "ffn_up": {"flops": 2 * R * d * F * nup,
+                   "bytes": e_act * d * F * b * nup + R * d * b + R * F * b},
+        "ffn_down": {"flops": 2 * R * F * d, "bytes": e_act * F * d * b + R * F * b + R * d * b},
+        "combine": {"bytes": R * d * b + S * 8 + T * d * b},
+    }
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def file_hash(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def measured_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, or None when the
+    kernel source changed since that capture."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    cur = file_hash(GEMM_SRC)
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel \
+                    and parts[1] == workload and parts[3] == cur:
+                return float(parts[2])
+    return None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpus):
+        self.gpus = gpus
+        self.proc = None
+        self.path = os.path.join("/tmp", f"moe_bench_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", ",".join(str(g) for g in self.gpus)],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                c = [x.strip() for x in line.split(",")]
+                if len(c) < 9:
+                    continue
+                try:
+                    sm.append(float(c[1]))
+                    smax.append(float(c[2]))
+                    power.append(float(c[3]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, c[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        hi = max(sm)
+        load = [s for s, p in zip(sm, power) if p > 200.0] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm), "sm_mhz_peak_seen": hi}
+
+    @staticmethod
+    def rejected(c):
+        bad = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+        if any(r in bad for r in c.get("reasons", [])):
+            return True
+        if c.get("sm_mhz") and c.get("sm_max_mhz") and not c["reasons"] and \
+                c["sm_mhz"] < 0.6 * c["sm_max_mhz"]:
+            return True
+        return False
+
+
+# ------------------------------------------------------------------ distributed
+def dist_setup(n):
+    if n <= 1:
+        return 0, 1, 0
+    import torch.distributed as dist
+    from datetime import timedelta
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", n))
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def reduce_max(v, world):
+    if world <= 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_sample_run(inp, tokens, w64):
+    """One oracle forward over a sample of the workload's tokens."""
+    from oracle import moe_oracle as O
+    sh = inp.shape
+    x = inp.x[:tokens].float().numpy()
+    bias = None if inp.bias is None else inp.bias.numpy()
+    t0 = time.perf_counter()
+    O.forward(x, inp.wg.float().numpy(), bias, w64["w1"], w64["w3"], w64["w2"], sh.k, sh.act, sh.cf)
+    return time.perf_counter() - t0
+
+
+def weights_f64(inp):
+    cvt = lambda w: None if w is None else [w[e].to(torch.float64).numpy() for e in range(w.shape[0])]  # noqa: E731
+    return {"w1": cvt(inp.w1), "w3": cvt(inp.w3), "w2": cvt(inp.w2)}
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"), default=None)
+        if n:
+            return int(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", 0))
+    if rank != 0:
+        return 0
+    sh = shape_of(args)
+    inp = make_inputs(sh)
+    w64 = weights_f64(inp)
+    tokens = min(64, sh.T)
+    for _ in range(args.warmup):
+        oracle_sample_run(inp, tokens, w64)
+    tot = 0.0
+    for _ in range(args.steps):
+        tot += oracle_sample_run(inp, tokens, w64)
+    value = tokens * args.steps / tot
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)", "config": workload_config(sh),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                         "sample": f"{tokens} of the workload's {sh.T} tokens per step, whole "
+                                   f"layer (route, permute, gather, expert FFN, combine) in "
+                                   f"numpy float64"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def cpu_baseline(sh, inp):
+    w64 = weights_f64(inp)
+    tokens = min(256, sh.T)
+    oracle_sample_run(inp, min(16, sh.T), w64)  # first touch of the converted weights
+    t = oracle_sample_run(inp, tokens, w64)
+    return {"value": tokens / t, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"one oracle forward (numpy float64) of the first {tokens} of {sh.T} tokens "
+                      f"of the same workload, {t:.1f} s"}
+
+
+# ------------------------------------------------------------------ main
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    from mixture_experts_routing_route_b200 import MoeLayer
+    from mixture_experts_routing_route_b200 import _abi as abi
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    sh = shape_of(args)
+    # each replica draws its own tokens; the weights are the same everywhere
+    inp = make_inputs(sh.with_(seed=sh.seed)) if rank == 0 else None
+    if rank != 0:
+        base = make_inputs(sh)
+        from mixture_experts_routing_route_b200.inputs import make_x
+        base.x = make_x(sh.with_(seed=sh.seed + 7919 * rank))
+        inp = base
+    x = inp.x.to(dev)
+    layer = MoeLayer(inp.wg.to(dev), inp.w1.to(dev), inp.w2.to(dev),
+                     w3=None if inp.w3 is None else inp.w3.to(dev),
+                     bias=None if inp.bias is None else inp.bias.to(dev),
+                     k=sh.k, act=sh.act, capacity_factor=sh.cf)
+    out = torch.empty(sh.T, sh.d, dtype=x.dtype, device=dev)
+    aux = torch.empty(1, dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+
+    for _ in range(max(3, args.warmup)):
+        layer.forward(x, out, aux)
+    torch.cuda.synchronize()
+    if layer.device_error(sh.T) != 0:
+        raise RuntimeError("device error word set during warm-up")
+    v = layer.views(sh.T)
+    kept = v["kept_counts"].cpu().tolist()
+    launches_per_step = (1 if (sh.E <= 8) else 2) + 1 + (1 if sum(kept) > 0 else 0) + 2 + 1
+
+    def timed_region():
+        barrier(world)
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.fill_(i & 0xff)
+            layer.forward(x, out, aux, events=evs[i])
+        torch.cuda.synchronize()
+        barrier(world)
+        per = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(6)] for i in range(args.steps)]
+        return per
+
+    sampler = ClockSampler(list(range(world)) if rank == 0 else [])
+    if rank == 0:
+        sampler.start()
+    per = timed_region()
+    clocks = sampler.stop() if rank == 0 else {}
+    if rank == 0 and ClockSampler.rejected(clocks):
+        sampler = ClockSampler(list(range(world)))
+        sampler.start()
+        per = timed_region()
+        clocks = sampler.stop()
+        clocks["remeasured"] = True
+    step_ms = [sum(p) for p in per]
+    total_ms = reduce_max(sum(step_ms), world)
+    if layer.device_error(sh.T) != 0:
+        raise RuntimeError("device error word set during the timed steps")
+
+    stage_ms = {s: statistics.mean(p[j] for p in per) for j, s in enumerate(STAGES)}
+    alg = algorithmic(sh, kept)
+    peaks = load_peaks()
+    roof = {}
+    for s in STAGES:
+        t = stage_ms[s] * 1e-3
+        a = alg[s]
+        r = {"us": stage_ms[s] * 1e3, "GB_s": a["bytes"] / t / 1e9 if t > 0 else None}
+        r["hbm_frac"] = r["GB_s"] / peaks["hbm_gbs"] if r["GB_s"] else None
+        if "flops" in a:
+            r["TFLOP_s"] = a["flops"] / t / 1e12 if t > 0 else None
+            r["tensor_frac"] = r["TFLOP_s"] / peaks["bf16_tflops"] if r["TFLOP_s"] else None
+        roof[s] = r
+
+    dom = "ffn_up"
+    tf = roof[dom]["TFLOP_s"]
+    traffic = measured_traffic("grouped_gemm_tc_swiglu", sh.name)
+    roofline = {"kernel": "grouped_gemm_tc<SwiGLU> (expert up/gate projection)",
+                "bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"] if tf else None,
+                "traffic": traffic,
+                "peak_source": f"{peaks['source']} bf16 dense burst (kernel timed alone per step)",
+                "algorithmic_per_launch": f"2*R*d*2F = {alg[dom]['flops']:.4e} flop (R={sum(kept)} rows)"}
+
+    e2e = None
+    if not args.no_e2e:
+        x_host = inp.x.pin_memory()
+        out_host = torch.empty(sh.T, sh.d, dtype=x.dtype).pin_memory()
+        aux_host = torch.empty(1, dtype=torch.float32).pin_memory()
+        for _ in range(2):
+            layer.forward_host(x_host, out_host, aux_host)
+        torch.cuda.synchronize()
+        e_ms = []
+        barrier(world)
+        for i in range(args.steps):
+            flush.fill_(i & 0xff)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            layer.forward_host(x_host, out_host, aux_host)
+            b.record(stream)
+            b.synchronize()  # the host reads the result every step
+            e_ms.append(a.elapsed_time(b))
+        e_total = reduce_max(sum(e_ms), world)
+        elem = x.element_size()
+        e2e = {"value": world * sh.T * args.steps / (e_total * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": sh.T * sh.d * elem,
+               "d2h_bytes_per_step": sh.T * sh.d * elem + 4,
+               "api": "moe_forward_host (pinned host x/out, async copies on the stream)"}
+
+    if rank != 0:
+        _finish(world)
+        return 0
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(sh, inp)
+    value = world * sh.T * args.steps / (total_ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": sh.dtype,
+        "data": "synthetic (seeded; random-init weights of the layer's shape)",
+        "config": dict(workload_config(sh), parallelism=f"replicas x{world}" if world > 1 else "1 GPU"),
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "stages": roof,
+        "aux_loss": float(aux.item()),
+        "rows": int(sum(kept)), "experts_active": int(sum(1 for c in kept if c > 0)),
+        "imbalance_max_over_mean": (max(kept) / (sum(kept) / sh.E)) if sum(kept) else None,
+    }
+    print(json.dumps(line), flush=True)
+    _finish(world)
+    return 0
+
+
+def _finish(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

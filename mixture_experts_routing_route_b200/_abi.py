@@ -212,6 +212,11 @@ def moe_forward_host_workspace_size(layer: MoeLayerC, T: int) -> int:
 def moe_forward(layer: MoeLayerC, x, T, out, aux_loss, ws, stream=None, events=None):
     ev = None
     if events is not None:
+        # torch creates a CUDA event lazily, on its first record(): record once
+        # so that the handle exists (the library then re-records it in place).
+        for e in events:
+            if e is not None and e.cuda_event == 0:
+                e.record(torch.cuda.current_stream() if stream is None else stream)
         arr = (c_void_p * 7)(*[e.cuda_event if e is not None else None for e in events])
         ev = ctypes.cast(arr, c_void_p)
     _check("moe_forward", _lib.moe_forward(

@@ -126,11 +126,19 @@ router_fused_e8(const Tin* __restrict__ x, const Tin* __restrict__ wg, const flo
 
   // Stage Wg as [d][8] (zero for experts >= E).
   if constexpr (sizeof(Tin) == 2) {
-    uint16_t* ws = reinterpret_cast<uint16_t*>(smem_raw);
-    const uint16_t* wgu = reinterpret_cast<const uint16_t*>(wg);
-    for (int i = threadIdx.x; i < d * 8; i += blockDim.x) {
-      const int r = i >> 3, e = i & 7;
-      ws[wg_row_slot_bf16(r) * 8 + e] = e < E ? wgu[static_cast<size_t>(r) * E + e] : uint16_t(0);
+    if (E == 8) {
+      // one 16-byte row per load, rows in flight across the whole block
+      const uint4* src = reinterpret_cast<const uint4*>(wg);
+      uint4* dst = reinterpret_cast<uint4*>(smem_raw);
+#pragma unroll 8
+      for (int r = threadIdx.x; r < d; r += blockDim.x) dst[wg_row_slot_bf16(r)] = __ldg(src + r);
+    } else {
+      uint16_t* ws = reinterpret_cast<uint16_t*>(smem_raw);
+      const uint16_t* wgu = reinterpret_cast<const uint16_t*>(wg);
+      for (int i = threadIdx.x; i < d * 8; i += blockDim.x) {
+        const int r = i >> 3, e = i & 7;
+        ws[wg_row_slot_bf16(r) * 8 + e] = e < E ? wgu[static_cast<size_t>(r) * E + e] : uint16_t(0);
+      }
     }
   } else {
     float* ws = reinterpret_cast<float*>(smem_raw);
