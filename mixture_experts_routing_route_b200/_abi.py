@@ -35,7 +35,7 @@ class MoeError(RuntimeError):
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     if not os.path.exists(path):
         raise ImportError(f"libmoe_b200.so is not built ({path}); run "
-                          "`python -m mixture_experts_routing_route_b200.build`")
+                          "`python mixture_experts_routing_route_b200/build.py`")
     return ctypes.CDLL(path)
 
 

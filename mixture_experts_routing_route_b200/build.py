@@ -1,6 +1,7 @@
 """Build libmoe_b200.so in-tree with nvcc for sm_100a.
 
-Usage: python -m mixture_experts_routing_route_b200.build [--force]
+Usage: python mixture_experts_routing_route_b200/build.py [--force]
+(run it as a script: importing the package loads the library being built)
 """
 from __future__ import annotations
 

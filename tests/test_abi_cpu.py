@@ -5,12 +5,12 @@ import ctypes
 
 import pytest
 
-from mixture_experts_routing_route_b200 import build as build_mod
+import __graft_entry__
 
 
 @pytest.fixture(scope="module")
 def abi():
-    build_mod.build()
+    __graft_entry__.build()
     from mixture_experts_routing_route_b200 import _abi
     return _abi
 
