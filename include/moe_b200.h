@@ -186,6 +186,32 @@ MOE_API moe_status_t moe_permute(const int32_t* topk_idx, int T, int k, int E, i
                          int32_t* kept_counts, int32_t* seg_offsets, void* ws, size_t ws_bytes,
                          moe_stream_t stream);
 
+/* --------------------------------------------------- permute, no allocation
+ * The same permute for callers that cannot allocate device memory: code that
+ * runs where the CUDA allocator is not reachable or not allowed (a library
+ * handed only pre-allocated tensors, a runtime whose memory pool is fixed
+ * before the first call, a plugin in a process that forbids cudaMalloc after
+ * start-up). It takes no workspace and calls no allocating routine. The paper
+ * has no counterpart to this entry point; it exists for such callers only.
+ *   Outputs and their meaning are those of moe_permute.
+ *   device_error  out [1] u32 (device) or NULL: the call's device error bits.
+ *   Limit: T*k <= MOE_PERMUTE_NOALLOC_MAX_SLOTS; larger sizes return
+ *   MOE_ERR_WORKSPACE and launch nothing.
+ * Its scratch is one file-scope static device array (256 bytes of control
+ * block + 4 bytes per slot up to the limit, ~256 KB), which every GPU that
+ * loads this library holds until the process exits. The first call on a
+ * device looks up that array's device address (cudaGetSymbolAddress, with
+ * that device current); make that first call before any stream capture.
+ * Every call shares the array: calls that overlap on the GPU (other streams,
+ * other host threads) race and give wrong results. */
+#define MOE_PERMUTE_NOALLOC_MAX_SLOTS 65536
+MOE_API moe_status_t moe_permute_noalloc(const int32_t* topk_idx, int T, int k, int E,
+                                         int64_t capacity, int32_t* counts, int32_t* bins,
+                                         int32_t* sorted_slot, int32_t* slot_to_row,
+                                         int32_t* row_slot, uint8_t* drop_mask,
+                                         int32_t* kept_counts, int32_t* seg_offsets,
+                                         uint32_t* device_error, moe_stream_t stream);
+
 /* ----------------------------------------------------------------- gather
  * x_perm[r] = x[row_slot[r] / k] for r < seg_offsets[E] ("MegaBlocks",
  * section 4.3, binned_gather in compact form), moved row by row with bulk

@@ -71,6 +71,8 @@ _SIGS = {
     "moe_permute_workspace_size": (c_size_t, [c_int, c_int, c_int]),
     "moe_permute": (c_int, [c_void_p, c_int, c_int, c_int, c_int64] + [c_void_p] * 8
                     + [c_void_p, c_size_t, c_void_p]),
+    "moe_permute_noalloc": (c_int, [c_void_p, c_int, c_int, c_int, c_int64] + [c_void_p] * 9
+                            + [c_void_p]),
     "moe_gather": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_int,
                            c_int64, c_void_p, c_void_p, c_size_t, c_void_p]),
     "moe_expert_ffn": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int64,
@@ -175,6 +177,15 @@ def moe_permute(topk_idx, T, k, E, capacity, counts, bins, sorted_slot, slot_to_
         _ptr(topk_idx), T, k, E, int(capacity), _ptr(counts), _ptr(bins), _ptr(sorted_slot),
         _ptr(slot_to_row), _ptr(row_slot), _ptr(drop_mask), _ptr(kept_counts), _ptr(seg_offsets),
         _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_permute_noalloc(topk_idx, T, k, E, capacity, counts, bins, sorted_slot, slot_to_row,
+                        row_slot, drop_mask, kept_counts, seg_offsets, device_error=None,
+                        stream=None):
+    _check("moe_permute_noalloc", _lib.moe_permute_noalloc(
+        _ptr(topk_idx), T, k, E, int(capacity), _ptr(counts), _ptr(bins), _ptr(sorted_slot),
+        _ptr(slot_to_row), _ptr(row_slot), _ptr(drop_mask), _ptr(kept_counts), _ptr(seg_offsets),
+        _ptr(device_error), _stream(stream)))
 
 
 def moe_gather(x, T, d, k, row_slot, seg_offsets, E, rows_max, x_perm, ws, stream=None):
