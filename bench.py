@@ -57,14 +57,15 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--T", type=int, default=None, help="override T (reduced case for profiling)")
     p.add_argument("--E", type=int, default=None, help="override E (reduced case for profiling)")
+    p.add_argument("--F", type=int, default=None, help="override F (reduced case for profiling)")
     return p.parse_args()
 
 
 def shape_of(args):
     sh = CONFIGS[args.config]
-    if args.T is not None or args.E is not None:
-        sh = sh.with_(T=args.T or sh.T, E=args.E or sh.E,
-                      name=f"{sh.name}_T{args.T or sh.T}_E{args.E or sh.E}")
+    if args.T is not None or args.E is not None or args.F is not None:
+        sh = sh.with_(T=args.T or sh.T, E=args.E or sh.E, F=args.F or sh.F,
+                      name=f"{sh.name}_T{args.T or sh.T}_E{args.E or sh.E}_F{args.F or sh.F}")
     return sh
 
 
@@ -225,12 +226,25 @@ def barrier(world):
 
 
 def reduce_max(v, world):
+    """Max over ranks of a per-rank time (the job's time is the slowest rank's)."""
     if world <= 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_seed(sh, rank):
+    """Token seed of replica `rank`: rank 0 uses the workload's own seed, the
+    others draw their own tokens (the weights are the same on every rank)."""
+    return sh.seed if rank == 0 else sh.seed + 7919 * rank
+
+
+def job_value(tokens_per_rank, steps, world, total_ms_max):
+    """Whole-job token rate: all ranks' tokens over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (total_ms_max * 1e-3)
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -314,12 +328,10 @@ def main():
     torch.cuda.set_device(dev)
     sh = shape_of(args)
     # each replica draws its own tokens; the weights are the same everywhere
-    inp = make_inputs(sh.with_(seed=sh.seed)) if rank == 0 else None
+    inp = make_inputs(sh)
     if rank != 0:
-        base = make_inputs(sh)
         from mixture_experts_routing_route_b200.inputs import make_x
-        base.x = make_x(sh.with_(seed=sh.seed + 7919 * rank))
-        inp = base
+        inp.x = make_x(sh.with_(seed=replica_seed(sh, rank)))
     x = inp.x.to(dev)
     layer = MoeLayer(inp.wg.to(dev), inp.w1.to(dev), inp.w2.to(dev),
                      w3=None if inp.w3 is None else inp.w3.to(dev),
@@ -370,6 +382,13 @@ def main():
     stage_ms = {s: statistics.mean(p[j] for p in per) for j, s in enumerate(STAGES)}
     alg = algorithmic(sh, kept)
     peaks = load_peaks()
+    # A timed region long enough to hit the 1 kW power cap is compared with the
+    # sustained (power-capped) GEMM figure, a short one with the burst figure.
+    capped = rank == 0 and "sw_power_cap" in (clocks or {}).get("reasons", [])
+    if capped and peaks.get("bf16_tflops_sustained"):
+        tc_peak, tc_kind = peaks["bf16_tflops_sustained"], "sustained (sw_power_cap active while timed)"
+    else:
+        tc_peak, tc_kind = peaks["bf16_tflops"], "burst"
     roof = {}
     for s in STAGES:
         t = stage_ms[s] * 1e-3
@@ -378,17 +397,17 @@ def main():
         r["hbm_frac"] = r["GB_s"] / peaks["hbm_gbs"] if r["GB_s"] else None
         if "flops" in a:
             r["TFLOP_s"] = a["flops"] / t / 1e12 if t > 0 else None
-            r["tensor_frac"] = r["TFLOP_s"] / peaks["bf16_tflops"] if r["TFLOP_s"] else None
+            r["tensor_frac"] = r["TFLOP_s"] / tc_peak if r["TFLOP_s"] else None
         roof[s] = r
 
     dom = "ffn_up"
     tf = roof[dom]["TFLOP_s"]
     traffic = measured_traffic("grouped_gemm_tc_swiglu", sh.name)
     roofline = {"kernel": "grouped_gemm_tc<SwiGLU> (expert up/gate projection)",
-                "bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"] if tf else None,
+                "bound": "tensor", "achieved": tf, "peak": tc_peak,
+                "unit": "TFLOP/s", "frac": tf / tc_peak if tf else None,
                 "traffic": traffic,
-                "peak_source": f"{peaks['source']} bf16 dense burst (kernel timed alone per step)",
+                "peak_source": f"{peaks['source']} bf16 dense {tc_kind}",
                 "algorithmic_per_launch": f"2*R*d*2F = {alg[dom]['flops']:.4e} flop (R={sum(kept)} rows)"}
 
     e2e = None
@@ -412,7 +431,7 @@ def main():
             e_ms.append(a.elapsed_time(b))
         e_total = reduce_max(sum(e_ms), world)
         elem = x.element_size()
-        e2e = {"value": world * sh.T * args.steps / (e_total * 1e-3), "unit": UNIT,
+        e2e = {"value": job_value(sh.T, args.steps, world, e_total), "unit": UNIT,
                "h2d_bytes_per_step": sh.T * sh.d * elem,
                "d2h_bytes_per_step": sh.T * sh.d * elem + 4,
                "api": "moe_forward_host (pinned host x/out, async copies on the stream)"}
@@ -423,7 +442,7 @@ def main():
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(sh, inp)
-    value = world * sh.T * args.steps / (total_ms * 1e-3)
+    value = job_value(sh.T, args.steps, world, total_ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": total_ms / args.steps,

@@ -13,7 +13,9 @@ namespace moe {
 struct Control {
   uint32_t err;           // MOE_DEVERR_* bits, sticky until cleared
   uint32_t route_ticket;  // blocks of the router that finished (reset by the last one)
-  uint32_t reserved[62];
+  uint32_t bar_count;     // grid barrier: blocks arrived (reset by the last one)
+  uint32_t bar_gen;       // grid barrier: generation, bumped when all arrived
+  uint32_t reserved[60];
 };
 static_assert(sizeof(Control) == 256, "control block is 256 bytes");
 
@@ -37,10 +39,8 @@ template <> struct Elem<__nv_bfloat16> {
 };
 
 // ------------------------------------------------------------------ launchers
-// Router. Tokens per router block (partials are per block).
-constexpr int kRouteFusedTokensPerBlock = 32;   // E <= 8 path: 8 warps x 4 tokens
-constexpr int kRouteSelectTokensPerBlock = 64;  // general path
-int route_num_blocks(int T, int E);
+// Router. Tokens per block of the general path (partials are per block).
+constexpr int kRouteSelectTokensPerBlock = 64;
 size_t route_partials_bytes(int T, int E);
 cudaError_t launch_route(const void* x, const void* wg, const float* bias, moe_dtype_t dt, int T,
                          int d, int E, int k, int32_t* idx, float* w, float* aux, float* logits,
@@ -48,8 +48,15 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, moe_d
                          cudaStream_t s);
 size_t route_logits_scratch_bytes(int T, int d, int E);
 
-// Permute.
+// Permute. launch_permute picks the multi-CTA kernel when the slots fit its
+// per-CTA shared memory, else the single-CTA kernel; launch_permute_single
+// always runs the single-CTA kernel (needs only the rank scratch).
 size_t permute_scratch_bytes(int T, int k, int E);
+cudaError_t launch_permute_single(const int32_t* idx, int T, int k, int E, int64_t cap,
+                                  int32_t* counts, int32_t* bins, int32_t* sorted_slot,
+                                  int32_t* slot_to_row, int32_t* row_slot, uint8_t* drop,
+                                  int32_t* kept, int32_t* seg, int32_t* rank_scratch, Control* ctl,
+                                  cudaStream_t s);
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int64_t cap, int32_t* counts,
                            int32_t* bins, int32_t* sorted_slot, int32_t* slot_to_row,
                            int32_t* row_slot, uint8_t* drop, int32_t* kept, int32_t* seg,

@@ -145,31 +145,90 @@ template <> struct CombineVec<float> {
 
 constexpr int kCombineThreads = 128;
 
-// grid.x = token, grid.y = column chunk of kCombineThreads * kVec elements.
-template <typename T>
+// One block per token (grid.x) and column range (grid.y); each thread owns
+// up to two 16-byte column vectors and requests the K rows of both before it
+// accumulates. K is the compile-time top-k (0: runtime k, rows one by one).
+template <typename T, int K>
 __global__ void __launch_bounds__(kCombineThreads)
 combine_gather(const T* __restrict__ y, const float* __restrict__ w,
-               const int32_t* __restrict__ slot_to_row, int d, int k, long long rows_max,
+               const int32_t* __restrict__ slot_to_row, int d, int k_rt, long long rows_max,
                T* __restrict__ out, Control* ctl) {
   constexpr int V = CombineVec<T>::kVec;
+  constexpr int NV = 2;  // column vectors per thread
+  const int k = K > 0 ? K : k_rt;
   const int t = blockIdx.x;
-  const int col = (blockIdx.y * kCombineThreads + threadIdx.x) * V;
-  if (col >= d) return;
-  float acc[V];
+  const int col0 = (blockIdx.y * kCombineThreads * NV + threadIdx.x) * V;
+  if (col0 >= d) return;
+  int rows[K > 0 ? K : 1];
+  float wj[K > 0 ? K : 1];
+  float acc[NV][V];
 #pragma unroll
-  for (int i = 0; i < V; ++i) acc[i] = 0.f;
-  for (int j = 0; j < k; ++j) {
-    const int row = __ldg(slot_to_row + static_cast<size_t>(t) * k + j);
-    if (row < 0) continue;
-    if (row >= rows_max) {
-      if (col == 0) set_error(ctl, MOE_DEVERR_ROW_RANGE);
-      continue;
+  for (int c = 0; c < NV; ++c)
+#pragma unroll
+    for (int i = 0; i < V; ++i) acc[c][i] = 0.f;
+  if constexpr (K > 0) {
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+      rows[j] = __ldg(slot_to_row + static_cast<size_t>(t) * K + j);
+      wj[j] = __ldg(w + static_cast<size_t>(t) * K + j);
+      if (rows[j] >= rows_max) {
+        if (col0 == 0) set_error(ctl, MOE_DEVERR_ROW_RANGE);
+        rows[j] = -1;
+      }
     }
-    const float wj = __ldg(w + static_cast<size_t>(t) * k + j);
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(row) * d + col));
-    CombineVec<T>::fma(u, wj, acc);
+    uint4 u[K][NV];
+#pragma unroll
+    for (int j = 0; j < K; ++j)
+#pragma unroll
+      for (int c = 0; c < NV; ++c) {
+        const int col = col0 + c * kCombineThreads * V;
+        u[j][c] = make_uint4(0, 0, 0, 0);
+        if (rows[j] >= 0 && col < d)
+          u[j][c] = __ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(rows[j]) * d + col));
+      }
+#pragma unroll
+    for (int j = 0; j < K; ++j)
+      if (rows[j] >= 0)
+#pragma unroll
+        for (int c = 0; c < NV; ++c) CombineVec<T>::fma(u[j][c], wj[j], acc[c]);
+  } else {
+    for (int j = 0; j < k; ++j) {
+      const int row = __ldg(slot_to_row + static_cast<size_t>(t) * k + j);
+      if (row < 0) continue;
+      if (row >= rows_max) {
+        if (col0 == 0) set_error(ctl, MOE_DEVERR_ROW_RANGE);
+        continue;
+      }
+      const float wv = __ldg(w + static_cast<size_t>(t) * k + j);
+#pragma unroll
+      for (int c = 0; c < NV; ++c) {
+        const int col = col0 + c * kCombineThreads * V;
+        if (col < d)
+          CombineVec<T>::fma(__ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(row) * d + col)),
+                             wv, acc[c]);
+      }
+    }
   }
-  *reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * d + col) = CombineVec<T>::pack(acc);
+#pragma unroll
+  for (int c = 0; c < NV; ++c) {
+    const int col = col0 + c * kCombineThreads * V;
+    if (col < d)
+      *reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * d + col) = CombineVec<T>::pack(acc[c]);
+  }
+}
+
+template <typename T>
+void launch_combine_t(const T* y, const float* w, const int32_t* s2r, int T_, int d, int k,
+                      long long rows_max, T* out, Control* ctl, cudaStream_t s) {
+  constexpr int V = CombineVec<T>::kVec;
+  dim3 grid(T_, (d + kCombineThreads * V * 2 - 1) / (kCombineThreads * V * 2));
+  switch (k) {
+    case 1: combine_gather<T, 1><<<grid, kCombineThreads, 0, s>>>(y, w, s2r, d, k, rows_max, out, ctl); break;
+    case 2: combine_gather<T, 2><<<grid, kCombineThreads, 0, s>>>(y, w, s2r, d, k, rows_max, out, ctl); break;
+    case 4: combine_gather<T, 4><<<grid, kCombineThreads, 0, s>>>(y, w, s2r, d, k, rows_max, out, ctl); break;
+    case 8: combine_gather<T, 8><<<grid, kCombineThreads, 0, s>>>(y, w, s2r, d, k, rows_max, out, ctl); break;
+    default: combine_gather<T, 0><<<grid, kCombineThreads, 0, s>>>(y, w, s2r, d, k, rows_max, out, ctl); break;
+  }
 }
 
 }  // namespace
@@ -191,16 +250,12 @@ cudaError_t launch_combine(const void* y, const float* w, const int32_t* slot_to
                            int T, int d, int k, int64_t rows_max, void* out, Control* ctl,
                            cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  const int vec = elem == 2 ? 8 : 4;
-  dim3 grid(T, (d + kCombineThreads * vec - 1) / (kCombineThreads * vec));
   if (elem == 2)
-    combine_gather<__nv_bfloat16><<<grid, kCombineThreads, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(y), w, slot_to_row, d, k, rows_max,
-        static_cast<__nv_bfloat16*>(out), ctl);
+    launch_combine_t<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(y), w, slot_to_row, T, d, k,
+                                    rows_max, static_cast<__nv_bfloat16*>(out), ctl, s);
   else
-    combine_gather<float><<<grid, kCombineThreads, 0, s>>>(static_cast<const float*>(y), w,
-                                                          slot_to_row, d, k, rows_max,
-                                                          static_cast<float*>(out), ctl);
+    launch_combine_t<float>(static_cast<const float*>(y), w, slot_to_row, T, d, k, rows_max,
+                            static_cast<float*>(out), ctl, s);
   return cudaGetLastError();
 }
 

@@ -84,8 +84,9 @@ extern "C" moe_status_t moe_permute_noalloc(const int32_t* topk_idx, int T, int 
   Control* ctl = static_cast<Control*>(scratch);
   int32_t* rank = static_cast<int32_t*>(scratch) + kNoallocCtlWords;
   if (cudaMemsetAsync(ctl, 0, sizeof(Control), s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (launch_permute(topk_idx, T, k, E, capacity, counts, bins, sorted_slot, slot_to_row, row_slot,
-                     drop_mask, kept_counts, seg_offsets, rank, ctl, s) != cudaSuccess)
+  if (launch_permute_single(topk_idx, T, k, E, capacity, counts, bins, sorted_slot, slot_to_row,
+                            row_slot, drop_mask, kept_counts, seg_offsets, rank, ctl,
+                            s) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (device_error != nullptr &&
       cudaMemcpyAsync(device_error, &ctl->err, sizeof(uint32_t), cudaMemcpyDeviceToDevice, s) !=

@@ -32,26 +32,34 @@ __device__ __forceinline__ bool better(float va, int ea, float vb, int eb) {
   return va > vb || (va == vb && ea < eb);
 }
 
-// Reduce the aux partials of all blocks (fixed block order, float64), then
-// aux = E * sum_e f_e * P_e. Run by every thread of the last block.
+// Reduce the aux partials of all blocks, then aux = E * sum_e f_e * P_e, in
+// float64 and in a fixed order: expert e's partials are summed by one warp
+// (lane l takes blocks l, l+32, ...; a butterfly combines the lanes) and the
+// per-expert terms are added by a tree over 256 slots. The result does not
+// depend on the block size. Run by every thread of the last block.
 __device__ void finalize_aux(const float* part_p, const int32_t* part_c, int nblk, int E, int T,
                              int k, float* aux) {
   __shared__ double red[256];
-  double v = 0.0;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) red[i] = 0.0;
+  __syncthreads();
+  for (int e = warp; e < E; e += nw) {
     double ps = 0.0;
     long long cs = 0;
-    for (int b = 0; b < nblk; ++b) {
+    for (int b = lane; b < nblk; b += 32) {
       ps += static_cast<double>(__ldcg(part_p + static_cast<size_t>(b) * E + e));
       cs += __ldcg(part_c + static_cast<size_t>(b) * E + e);
     }
-    const double P = T > 0 ? ps / T : 0.0;
-    const double f = T > 0 ? static_cast<double>(cs) / (static_cast<double>(T) * k) : 0.0;
-    v += f * P;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      ps += __shfl_xor_sync(kFull, ps, off);
+      cs += __shfl_xor_sync(kFull, cs, off);
+    }
+    if (lane == 0 && T > 0)
+      red[e] = (static_cast<double>(cs) / (static_cast<double>(T) * k)) * (ps / T);
   }
-  red[threadIdx.x] = v;
   __syncthreads();
-  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+  for (int s = 128; s > 0; s >>= 1) {
     if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
     __syncthreads();
   }
@@ -105,171 +113,254 @@ template <> struct VecTraits<float> {
   }
 };
 
-// Shared-memory slot of Wg row i (8 experts, one 16-byte chunk per row for
-// bf16): XOR-swizzled so the 8 lanes of a quarter-warp, which read rows
-// 8l + j, hit 8 different bank groups.
-__device__ __forceinline__ int wg_row_slot_bf16(int i) { return i ^ ((i >> 3) & 7); }
+
+// Fused router for E <= 8.
+//
+// Block = 12 warps = 6 slices of d x 2 token quads: warp (slice, quad) takes 4
+// tokens and one sixth of d, so a block works on 8 tokens and each SM keeps
+// 12 warps' x loads in flight. Wg is staged once per block in shared memory as
+// fp32 pairs: for row pair p = (2p, 2p+1) and expert e the float2
+// (Wg[2p][e], Wg[2p+1][e]); a lane's 16-byte x slice (8 bf16 = 4 row pairs)
+// then meets 4 pair-rows of 64 bytes, read with an XOR swizzle so that the 8
+// lanes of a quarter-warp hit 8 different bank groups. Products use the packed
+// fma.rn.f32x2 (even rows in .x, odd rows in .y; the two halves are added at
+// the end). Each warp's partial logits are reduce-scattered (lane l: token l/8,
+// expert l%8), the slices are added in slice order through shared memory,
+// and the quads' 8-lane groups do softmax / top-k / renormalisation.
+constexpr int kFusedSlices = 6;
+constexpr int kFusedQuads = 2;
+constexpr int kFusedTokensPerGroup = 4 * kFusedQuads;
+constexpr int kFusedThreads = 32 * kFusedSlices * kFusedQuads;
+
+__device__ __forceinline__ void fma2(float2& acc, float2 a, float2 b) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(r)
+      : "l"(*reinterpret_cast<const unsigned long long*>(&a)),
+        "l"(*reinterpret_cast<const unsigned long long*>(&b)),
+        "l"(*reinterpret_cast<const unsigned long long*>(&acc)));
+  acc = *reinterpret_cast<const float2*>(&r);
+}
+
+// Byte offset of 16-byte chunk c (0..15) of the 256-byte block of 4 pair-rows
+// owned by slice position g (pair-rows 4g .. 4g+3).
+__device__ __forceinline__ uint32_t wg_chunk_off(uint32_t g, uint32_t c) {
+  return g * 256u + 16u * (c ^ (g & 7u));
+}
 
 template <typename Tin>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kFusedThreads, 1)
 router_fused_e8(const Tin* __restrict__ x, const Tin* __restrict__ wg, const float* __restrict__ bias,
                 int T, int d, int E, int k, int32_t* __restrict__ idx_out, float* __restrict__ w_out,
                 float* __restrict__ logits_out, float* __restrict__ probs_out,
                 float* __restrict__ part_p, int32_t* __restrict__ part_c, float* __restrict__ aux,
                 Control* ctl) {
-  constexpr int V = VecTraits<Tin>::kVec;
+  constexpr int V = VecTraits<Tin>::kVec;  // elements per 16-byte x load: 8 (bf16) or 4 (fp32)
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  __shared__ float blk_p[8][8];
-  __shared__ int32_t blk_c[8][8];
+  __shared__ float slice_part[kFusedSlices][kFusedQuads][32];
+  __shared__ float blk_p[kFusedQuads][8];
+  __shared__ int32_t blk_c[kFusedQuads][8];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
+  const int slice = warp / kFusedQuads, quad = warp % kFusedQuads;
 
-  // Stage Wg as [d][8] (zero for experts >= E).
-  if constexpr (sizeof(Tin) == 2) {
-    if (E == 8) {
-      // one 16-byte row per load, rows in flight across the whole block
-      const uint4* src = reinterpret_cast<const uint4*>(wg);
-      uint4* dst = reinterpret_cast<uint4*>(smem_raw);
-#pragma unroll 8
-      for (int r = threadIdx.x; r < d; r += blockDim.x) dst[wg_row_slot_bf16(r)] = __ldg(src + r);
-    } else {
-      uint16_t* ws = reinterpret_cast<uint16_t*>(smem_raw);
-      const uint16_t* wgu = reinterpret_cast<const uint16_t*>(wg);
-      for (int i = threadIdx.x; i < d * 8; i += blockDim.x) {
-        const int r = i >> 3, e = i & 7;
-        ws[wg_row_slot_bf16(r) * 8 + e] = e < E ? wgu[static_cast<size_t>(r) * E + e] : uint16_t(0);
+  // ---- stage Wg: row pairs (zero for experts >= E and for a missing odd row)
+  const int npairs = (d + 1) / 2;
+  if (sizeof(Tin) == 2 && E == 8) {
+    // two 16-byte rows per pair-row, all loads of a thread in flight together
+    const uint4* src = reinterpret_cast<const uint4*>(wg);
+#pragma unroll 4
+    for (int p = threadIdx.x; p < npairs; p += kFusedThreads) {
+      const uint4 r0 = __ldg(src + 2 * p), r1 = __ldg(src + 2 * p + 1);
+      const uint32_t a[4] = {r0.x, r0.y, r0.z, r0.w}, b[4] = {r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {  // experts 2c, 2c+1
+        const float4 v = make_float4(__uint_as_float(a[c] << 16), __uint_as_float(b[c] << 16),
+                                     __uint_as_float(a[c] & 0xffff0000u),
+                                     __uint_as_float(b[c] & 0xffff0000u));
+        *reinterpret_cast<float4*>(smem_raw + wg_chunk_off(p >> 2, ((p & 3) << 2) | c)) = v;
       }
     }
-  } else {
-    float* ws = reinterpret_cast<float*>(smem_raw);
-    for (int i = threadIdx.x; i < d * 8; i += blockDim.x) {
-      const int r = i >> 3, e = i & 7;
-      ws[i] = e < E ? static_cast<float>(wg[static_cast<size_t>(r) * E + e]) : 0.f;
+  } else
+  for (int i = threadIdx.x; i < npairs * 8; i += kFusedThreads) {
+    const int p = i >> 3, e = i & 7;
+    float w0 = 0.f, w1 = 0.f;
+    if (e < E) {
+      w0 = Elem<Tin>::to_f32(wg[static_cast<size_t>(2 * p) * E + e]);
+      if (2 * p + 1 < d) w1 = Elem<Tin>::to_f32(wg[static_cast<size_t>(2 * p + 1) * E + e]);
     }
+    // pair-row p, expert e: chunk (p % 4) * 4 + e / 2 of group p / 4, half e % 2
+    const uint32_t off = wg_chunk_off(p >> 2, ((p & 3) << 2) | (e >> 1)) + (e & 1) * 8;
+    *reinterpret_cast<float2*>(smem_raw + off) = make_float2(w0, w1);
   }
   __syncthreads();
 
-  // lane -> (token-in-quad tq, expert e) after the reduce-scatter
-  const int tq = lane >> 3;
+  const int tq = lane >> 3;  // token of the quad after the reduce-scatter
   const int e = lane & 7;
   const bool e_ok = e < E;
   const float b_e = (bias != nullptr && e_ok) ? bias[e] : 0.f;
   float psum = 0.f;
   int cnt = 0;
+  // this slice's share of d, cut at multiples of 8 elements (one 16-byte group of 4 pairs)
+  const int nvec8 = d / 8;  // whole 8-element vectors (d % 8 == 0 here, see use_fused)
+  const int per = (nvec8 + kFusedSlices - 1) / kFusedSlices;
+  const int v_lo = min(nvec8, slice * per), v_hi = min(nvec8, v_lo + per);
 
-  const int groups = (T + 31) / 32;
+  const int groups = (T + kFusedTokensPerGroup - 1) / kFusedTokensPerGroup;
   for (int g = blockIdx.x; g < groups; g += gridDim.x) {
-    const int t_base = g * 32 + warp * 4;
-    float acc[32];
+    const int t_base = g * kFusedTokensPerGroup + quad * 4;
+    float2 acc[4][8];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[q][j] = make_float2(0.f, 0.f);
 
-    for (int i0 = lane * V; i0 < d; i0 += 32 * V) {
-      float xv[4][V];
+    constexpr int kUnroll = 2;
+    for (int vb = v_lo + lane; vb < v_hi; vb += 32 * kUnroll) {
+      uint4 raw[kUnroll][4][8 / V];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int t = t_base + q;
-        uint4 u = make_uint4(0, 0, 0, 0);
-        if (t < T) u = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d + i0));
-        VecTraits<Tin>::unpack(u, xv[q]);
+      for (int u = 0; u < kUnroll; ++u) {
+        const int v = vb + 32 * u;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int t = t_base + q;
+#pragma unroll
+          for (int h = 0; h < 8 / V; ++h) {
+            raw[u][q][h] = make_uint4(0, 0, 0, 0);
+            if (t < T && v < v_hi)
+              raw[u][q][h] = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d +
+                                                                   static_cast<size_t>(v) * 8 + h * V));
+          }
+        }
       }
 #pragma unroll
-      for (int j = 0; j < V; ++j) {
-        float wr[8];
-        if constexpr (sizeof(Tin) == 2) {
-          const uint4 u = reinterpret_cast<const uint4*>(smem_raw)[wg_row_slot_bf16(i0 + j)];
-          VecTraits<__nv_bfloat16>::unpack(u, wr);
-        } else {
-          const float4* p = reinterpret_cast<const float4*>(smem_raw) + (i0 + j) * 2;
-          const float4 a = p[0], b = p[1];
-          wr[0] = a.x; wr[1] = a.y; wr[2] = a.z; wr[3] = a.w;
-          wr[4] = b.x; wr[5] = b.y; wr[6] = b.z; wr[7] = b.w;
+      for (int u = 0; u < kUnroll; ++u) {
+        const int v = vb + 32 * u;
+        if (v >= v_hi) break;
+        const uint32_t grp = static_cast<uint32_t>(v);  // pair-rows 4v .. 4v+3
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) {
+          // row pair pp of the 4 tokens' 8-element slices
+          float2 xq[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if constexpr (sizeof(Tin) == 2) {
+              const uint32_t wv = pp == 0 ? raw[u][q][0].x : pp == 1 ? raw[u][q][0].y
+                                : pp == 2 ? raw[u][q][0].z : raw[u][q][0].w;
+              xq[q] = make_float2(__uint_as_float(wv << 16), __uint_as_float(wv & 0xffff0000u));
+            } else {
+              const uint4& r4 = raw[u][q][pp >> 1];
+              xq[q] = (pp & 1) ? make_float2(__uint_as_float(r4.z), __uint_as_float(r4.w))
+                               : make_float2(__uint_as_float(r4.x), __uint_as_float(r4.y));
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {  // experts 2c, 2c+1
+            const float4 w = *reinterpret_cast<const float4*>(smem_raw + wg_chunk_off(grp, (pp << 2) | c));
+            const float2 wa = make_float2(w.x, w.y), wb = make_float2(w.z, w.w);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              fma2(acc[q][2 * c], xq[q], wa);
+              fma2(acc[q][2 * c + 1], xq[q], wb);
+            }
+          }
         }
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-          for (int ee = 0; ee < 8; ++ee) acc[q * 8 + ee] = fmaf(xv[q][j], wr[ee], acc[q * 8 + ee]);
       }
     }
-    // Reduce-scatter over the warp: afterwards lane l holds the full sum of acc[l].
+    // even + odd halves, then reduce-scatter: lane l holds the sum of value l
+    float a[32];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[q * 8 + j] = acc[q][j].x + acc[q][j].y;
 #pragma unroll
     for (int half = 16; half >= 1; half >>= 1) {
       const bool upper = (lane & half) != 0;
 #pragma unroll
       for (int i = 0; i < half; ++i) {
-        const float send = upper ? acc[i] : acc[i + half];
-        const float keep = upper ? acc[i + half] : acc[i];
-        acc[i] = keep + __shfl_xor_sync(kFull, send, half);
+        const float send = upper ? a[i] : a[i + half];
+        const float keep = upper ? a[i + half] : a[i];
+        a[i] = keep + __shfl_xor_sync(kFull, send, half);
       }
     }
-    const int t = t_base + tq;
-    const bool t_ok = t < T;
-    float v = e_ok ? acc[0] + b_e : -INFINITY;
-    if (logits_out != nullptr && t_ok && e_ok) logits_out[static_cast<size_t>(t) * E + e] = v;
+    slice_part[slice][quad][lane] = a[0];
+    __syncthreads();
+    if (slice == 0) {
+      const int t = t_base + tq;
+      const bool t_ok = t < T;
+      float lg = 0.f;
+#pragma unroll
+      for (int sl = 0; sl < kFusedSlices; ++sl) lg += slice_part[sl][quad][lane];
+      float v = e_ok ? lg + b_e : -INFINITY;
+      if (logits_out != nullptr && t_ok && e_ok) logits_out[static_cast<size_t>(t) * E + e] = v;
 
-    // softmax inside the 8-lane group of token t
-    float m = v;
+      // softmax inside the 8-lane group of token t
+      float m = v;
 #pragma unroll
-    for (int off = 4; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
-    const float ex = e_ok ? expf(v - m) : 0.f;
-    float s = ex;
+      for (int off = 4; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+      const float ex = e_ok ? expf(v - m) : 0.f;
+      float sm = ex;
 #pragma unroll
-    for (int off = 4; off >= 1; off >>= 1) s += __shfl_xor_sync(kFull, s, off);
-    const float p = ex / s;
-    if (probs_out != nullptr && t_ok && e_ok) probs_out[static_cast<size_t>(t) * E + e] = p;
-    if (t_ok && e_ok) psum += p;
+      for (int off = 4; off >= 1; off >>= 1) sm += __shfl_xor_sync(kFull, sm, off);
+      const float p = ex / sm;
+      if (probs_out != nullptr && t_ok && e_ok) probs_out[static_cast<size_t>(t) * E + e] = p;
+      if (t_ok && e_ok) psum += p;
 
-    // top-k by k rounds of a group arg-max
-    bool taken = !e_ok;
-    float wsum = 0.f;
-    int my_e = 0;
-    float my_p = 0.f;
+      // top-k by k rounds of a group arg-max
+      bool taken = !e_ok;
+      float wsum = 0.f;
+      int my_e = 0;
+      float my_p = 0.f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j < k) {
-        float bv = taken ? -INFINITY : v;
-        int be = taken ? 0x7fffffff : e;
+      for (int j = 0; j < 8; ++j) {
+        if (j < k) {
+          float bv = taken ? -INFINITY : v;
+          int be = taken ? 0x7fffffff : e;
 #pragma unroll
-        for (int off = 4; off >= 1; off >>= 1) {
-          const float ov = __shfl_xor_sync(kFull, bv, off);
-          const int oe = __shfl_xor_sync(kFull, be, off);
-          if (better(ov, oe, bv, be)) { bv = ov; be = oe; }
+          for (int off = 4; off >= 1; off >>= 1) {
+            const float ov = __shfl_xor_sync(kFull, bv, off);
+            const int oe = __shfl_xor_sync(kFull, be, off);
+            if (better(ov, oe, bv, be)) { bv = ov; be = oe; }
+          }
+          if (be >= E || be < 0) {
+            if (t_ok && e == 0) set_error(ctl, MOE_DEVERR_EXPERT_RANGE);
+            be = 0;
+          }
+          const float pb = __shfl_sync(kFull, p, (lane & ~7) | be);
+          if (e == be) {
+            taken = true;
+            if (t_ok) ++cnt;
+          }
+          wsum += pb;
+          if (e == j) { my_e = be; my_p = pb; }
         }
-        if (be >= E || be < 0) {
-          if (t_ok && e == 0) set_error(ctl, MOE_DEVERR_EXPERT_RANGE);
-          be = 0;
-        }
-        const float pb = __shfl_sync(kFull, p, (lane & ~7) | be);
-        if (e == be) {
-          taken = true;
-          if (t_ok) ++cnt;
-        }
-        wsum += pb;
-        if (e == j) { my_e = be; my_p = pb; }
+      }
+      if (t_ok && e < k) {
+        idx_out[static_cast<size_t>(t) * k + e] = my_e;
+        w_out[static_cast<size_t>(t) * k + e] = my_p / wsum;
       }
     }
-    if (t_ok && e < k) {
-      idx_out[static_cast<size_t>(t) * k + e] = my_e;
-      w_out[static_cast<size_t>(t) * k + e] = my_p / wsum;
-    }
+    __syncthreads();  // slice_part is rewritten by the next group
   }
   // Warp totals per expert: lanes e, e+8, e+16, e+24 hold the same expert.
-  psum += __shfl_xor_sync(kFull, psum, 8);
-  psum += __shfl_xor_sync(kFull, psum, 16);
-  cnt += __shfl_xor_sync(kFull, cnt, 8);
-  cnt += __shfl_xor_sync(kFull, cnt, 16);
-  if (lane < 8) {
-    blk_p[warp][lane] = psum;
-    blk_c[warp][lane] = cnt;
+  if (slice == 0) {
+    psum += __shfl_xor_sync(kFull, psum, 8);
+    psum += __shfl_xor_sync(kFull, psum, 16);
+    cnt += __shfl_xor_sync(kFull, cnt, 8);
+    cnt += __shfl_xor_sync(kFull, cnt, 16);
+    if (lane < 8) {
+      blk_p[quad][lane] = psum;
+      blk_c[quad][lane] = cnt;
+    }
   }
   __syncthreads();
   __shared__ float tot_p[8];
   __shared__ int32_t tot_c[8];
   if (threadIdx.x < 8) {
-    float a = 0.f;
+    float s = 0.f;
     int c = 0;
-    for (int w = 0; w < 8; ++w) { a += blk_p[w][threadIdx.x]; c += blk_c[w][threadIdx.x]; }
-    tot_p[threadIdx.x] = a;
+    for (int w = 0; w < kFusedQuads; ++w) { s += blk_p[w][threadIdx.x]; c += blk_c[w][threadIdx.x]; }
+    tot_p[threadIdx.x] = s;
     tot_c[threadIdx.x] = c;
   }
   __syncthreads();
@@ -441,18 +532,14 @@ router_select(const float* __restrict__ logits_in, const float* __restrict__ bia
 }
 
 bool use_fused(int d, int E, moe_dtype_t dt) {
-  const size_t bytes = static_cast<size_t>(d) * 8 * (dt == MOE_BF16 ? 2 : 4);
-  return E <= 8 && bytes <= 96 * 1024;
+  (void)dt;
+  const size_t bytes = static_cast<size_t>((d + 7) / 8) * 256;  // fp32 pairs, 256 B per 8 rows
+  return E <= 8 && d % 8 == 0 && bytes <= 160 * 1024;
 }
+
+size_t fused_smem_bytes(int d) { return static_cast<size_t>((d + 7) / 8) * 256; }
 
 }  // namespace
-
-int route_num_blocks(int T, int E) {
-  // Fused path: a persistent grid of at most two blocks per SM.
-  const int groups = (T + 31) / 32;
-  if (E <= 8) return std::max(1, std::min(groups, 2 * num_sms()));
-  return std::max(1, (T + kRouteSelectTokensPerBlock - 1) / kRouteSelectTokensPerBlock);
-}
 
 static int route_max_blocks(int T) {
   return std::max((T + kRouteSelectTokensPerBlock - 1) / kRouteSelectTokensPerBlock,
@@ -478,20 +565,21 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, moe_d
   int32_t* part_c = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(partials) +
                                                align_up(static_cast<size_t>(nb_max) * E * 4));
   if (use_fused(d, E, dt)) {
-    const int groups = (T + 31) / 32;
-    const int grid = std::max(1, std::min(groups, 2 * num_sms()));
-    const size_t smem = static_cast<size_t>(d) * 8 * (dt == MOE_BF16 ? 2 : 4);
+    const int groups = (T + kFusedTokensPerGroup - 1) / kFusedTokensPerGroup;
+    const int grid = std::max(1, std::min(groups, num_sms()));
+    const size_t smem = fused_smem_bytes(d);
     if (dt == MOE_BF16) {
       auto kern = router_fused_e8<__nv_bfloat16>;
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      kern<<<grid, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(x),
-                                   static_cast<const __nv_bfloat16*>(wg), bias, T, d, E, k, idx, w,
-                                   logits, probs, part_p, part_c, aux, ctl);
+      kern<<<grid, kFusedThreads, smem, s>>>(static_cast<const __nv_bfloat16*>(x),
+                                             static_cast<const __nv_bfloat16*>(wg), bias, T, d, E, k,
+                                             idx, w, logits, probs, part_p, part_c, aux, ctl);
     } else {
       auto kern = router_fused_e8<float>;
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      kern<<<grid, 256, smem, s>>>(static_cast<const float*>(x), static_cast<const float*>(wg), bias,
-                                   T, d, E, k, idx, w, logits, probs, part_p, part_c, aux, ctl);
+      kern<<<grid, kFusedThreads, smem, s>>>(static_cast<const float*>(x), static_cast<const float*>(wg),
+                                             bias, T, d, E, k, idx, w, logits, probs, part_p, part_c,
+                                             aux, ctl);
     }
     return cudaGetLastError();
   }

@@ -68,3 +68,21 @@ def new_ws(nbytes: int, dev="cuda") -> torch.Tensor:
     ws = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=dev)
     _abi.moe_workspace_init(ws)
     return ws
+
+
+def check_topk_end_to_end(g_idx, route_ref, eps=1e-3):
+    """End-to-end top-k check against the oracle's own routing.
+
+    On tokens the oracle does not flag as near-ties (k-th and (k+1)-th logits
+    at least eps apart) the selected SET must be the oracle's. Inside the set
+    the order may differ only where two selected logits are closer than eps
+    (another float summation order can swap them); the GPU's order must be
+    non-increasing in the oracle's logits up to eps. The exact order is
+    checked separately, stage-chained on the GPU's own logits."""
+    g = np.asarray(g_idx, dtype=np.int64)
+    ref = np.asarray(route_ref["topk_idx"], dtype=np.int64)
+    ok = ~np.asarray(route_ref["near_tie"])
+    assert np.array_equal(np.sort(g[ok], axis=1), np.sort(ref[ok], axis=1)), "top-k set differs"
+    lg = np.take_along_axis(np.asarray(route_ref["logits"], np.float64), g, axis=1)
+    assert np.all(lg[:, :-1] >= lg[:, 1:] - eps), "top-k order not descending"
+    return int(np.sum(np.any(g[ok] != ref[ok], axis=1)))
