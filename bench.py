@@ -9,8 +9,10 @@ inputs resident in HBM. The default workload is the Mixtral-shaped layer
 and seeded. Prints one JSON line (rank 0).
 
 Timing: W untimed warm-up steps; then K steps bracketed by a barrier and a
-device synchronize; between steps a 256 MB buffer is written to flush L2
-(outside the timed events); every step is timed with CUDA events recorded on
+device synchronize; between steps a 256 MB buffer is read to evict L2
+(outside the timed events; a read, so the next step does not pay for writing
+back the flush's own dirty lines), and each step streams ~2.8 GB of expert
+weights, far more than the 126 MB L2; every step is timed with CUDA events recorded on
 the launching stream by the library between its stages; the value is the
 whole-job token rate, max over ranks of the summed step time. N > 1 runs N
 independent replicas (one per GPU, each its own T tokens): the layer has no
@@ -75,7 +77,7 @@ def workload_config(sh):
                         + ("" if sh.bias == "none" else f" bias={sh.bias}"),
             "T": sh.T, "d": sh.d, "E": sh.E, "k": sh.k, "F": sh.F, "act": sh.act,
             "capacity_factor": sh.cf, "global_batch_tokens": sh.T,
-            "l2": "256 MB buffer written between timed steps (outside the events)"}
+            "l2": "256 MB buffer read between timed steps (outside the events); per-step working set > L2"}
 
 
 # ------------------------------------------------------------------ roofline
@@ -339,7 +341,11 @@ def main():
                      k=sh.k, act=sh.act, capacity_factor=sh.cf)
     out = torch.empty(sh.T, sh.d, dtype=x.dtype, device=dev)
     aux = torch.empty(1, dtype=torch.float32, device=dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush_sink = torch.zeros(1, dtype=torch.int64, device=dev)
+
+    def evict_l2():
+        torch.sum(flush, dim=0, dtype=torch.int64, out=flush_sink[0])
     stream = torch.cuda.current_stream()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
 
@@ -356,7 +362,7 @@ def main():
         barrier(world)
         torch.cuda.synchronize()
         for i in range(args.steps):
-            flush.fill_(i & 0xff)
+            evict_l2()
             layer.forward(x, out, aux, events=evs[i])
         torch.cuda.synchronize()
         barrier(world)
@@ -421,7 +427,7 @@ def main():
         e_ms = []
         barrier(world)
         for i in range(args.steps):
-            flush.fill_(i & 0xff)
+            evict_l2()
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)

@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 #include <cstddef>
+#include <cuda.h>
 
 #include "../../include/moe_b200.h"
 
@@ -83,5 +84,9 @@ cudaError_t launch_combine(const void* y, const float* w, const int32_t* slot_to
                            cudaStream_t s);
 
 int num_sms();
+
+// 2-D bf16 TMA map over [rows, cols] row-major, box [box_rows, 64 cols], 128-byte swizzle.
+bool make_tma_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                      uint32_t box_rows);
 
 }  // namespace moe

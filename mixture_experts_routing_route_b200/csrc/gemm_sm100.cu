@@ -335,6 +335,8 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 }
 
 // ----------------------------------------------------------------- host side
+}  // namespace
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (fn == nullptr) {
@@ -348,7 +350,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 2-D bf16 map over [rows, cols] row-major, box [box_rows, 64 cols], 128-B swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+bool make_tma_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                      uint32_t box_rows) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {cols, rows};
@@ -361,14 +364,16 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
   return r == CUDA_SUCCESS;
 }
 
+namespace {
+
 template <int EPI, int NMMA>
 cudaError_t run_gemm(const void* A, const void* B0, const void* B1, int64_t rows_max, int K, int N,
                      int E, const int32_t* seg, void* out, Control* ctl, cudaStream_t s) {
   using C = Cfg<EPI, NMMA>;
   CUtensorMap ta, tb0, tb1;
-  if (!make_map(&ta, A, static_cast<uint64_t>(rows_max), K, BM)) return cudaErrorInvalidValue;
-  if (!make_map(&tb0, B0, static_cast<uint64_t>(E) * K, N, BK)) return cudaErrorInvalidValue;
-  if (!make_map(&tb1, B1 ? B1 : B0, static_cast<uint64_t>(E) * K, N, BK)) return cudaErrorInvalidValue;
+  if (!make_tma_2d_bf16(&ta, A, static_cast<uint64_t>(rows_max), K, BM)) return cudaErrorInvalidValue;
+  if (!make_tma_2d_bf16(&tb0, B0, static_cast<uint64_t>(E) * K, N, BK)) return cudaErrorInvalidValue;
+  if (!make_tma_2d_bf16(&tb1, B1 ? B1 : B0, static_cast<uint64_t>(E) * K, N, BK)) return cudaErrorInvalidValue;
   GemmArgs a;
   a.seg = seg;
   a.out = static_cast<__nv_bfloat16*>(out);

@@ -7,17 +7,18 @@
 // "MoE Router" page (Linear(hidden, E, bias=False) -> softmax -> topk ->
 // renormalise); "MegaBlocks 01", section 1 (bias-free linear router).
 //
-// Two paths:
-//  * E <= 8 and Wg small enough for shared memory: one fused kernel. A warp
-//    owns 4 tokens at a time; each lane streams 16-byte slices of the 4 x rows
-//    and multiplies them with the staged Wg rows, a 31-shuffle reduce-scatter
-//    leaves lane l with logit (token l/8, expert l%8), and selection then runs
-//    inside 8-lane groups. x is read from HBM exactly once.
-//  * otherwise: a tiled fp32 GEMM writes the logits [T, E] to scratch, then a
-//    warp-per-token kernel does softmax / top-k / renormalisation.
-// Both end with per-block aux partials reduced in a fixed order by the last
-// block to finish (a ticket counter), so the loss is deterministic.
+// Paths:
+//  * bf16 with E a multiple of 8 (E <= 32) or of 64: the gate GEMM runs on the
+//    tcgen05 tensor cores (router_tc: x streamed once by TMA, fp32 split-K
+//    partial logits to an L2-resident scratch), then router_select (a warp per
+//    token) adds the partials in order and routes.
+//  * fp32 with E <= 8: one fused CUDA-core kernel (router_fused_e8).
+//  * otherwise: a tiled CUDA-core GEMM for the logits, then router_select.
+// Every path leaves per-block aux partials (expert-major); aux_reduce sums them
+// in a fixed order (one block per expert, then the last block over experts),
+// so the loss is deterministic.
 #include "common.cuh"
+#include "ptx.cuh"
 #include <cfloat>
 #include <cmath>
 #include <algorithm>
@@ -32,77 +33,67 @@ __device__ __forceinline__ bool better(float va, int ea, float vb, int eb) {
   return va > vb || (va == vb && ea < eb);
 }
 
-// Reduce the aux partials of all blocks, then aux = E * sum_e f_e * P_e, in
-// float64 and in a fixed order: expert e's partials are summed by one warp
-// (lane l takes blocks l, l+32, ...; a butterfly combines the lanes) and the
-// per-expert terms are added by a tree over 256 slots. The result does not
-// depend on the block size. Run by every thread of the last block.
-__device__ void finalize_aux(const float* part_p, const int32_t* part_c, int nblk, int E, int T,
-                             int k, float* aux) {
-  __shared__ double red[256];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) red[i] = 0.0;
-  __syncthreads();
-  for (int e = warp; e < E; e += nw) {
-    double ps = 0.0;
-    long long cs = 0;
-    for (int b = lane; b < nblk; b += 32) {
-      ps += static_cast<double>(__ldcg(part_p + static_cast<size_t>(b) * E + e));
-      cs += __ldcg(part_c + static_cast<size_t>(b) * E + e);
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      ps += __shfl_xor_sync(kFull, ps, off);
-      cs += __shfl_xor_sync(kFull, cs, off);
-    }
-    if (lane == 0 && T > 0)
-      red[e] = (static_cast<double>(cs) / (static_cast<double>(T) * k)) * (ps / T);
+// This block's aux partials (per-expert probability sums and slot counts),
+// expert-major: part[e * ldb + block]. ldb = the largest grid of any router
+// kernel (route_max_blocks), so every path shares one layout.
+__device__ __forceinline__ void block_write_partials(const float* blk_p, const int32_t* blk_c,
+                                                     float* part_p, int32_t* part_c, int ldb,
+                                                     int E) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    part_p[static_cast<size_t>(e) * ldb + blockIdx.x] = blk_p[e];
+    part_c[static_cast<size_t>(e) * ldb + blockIdx.x] = blk_c[e];
   }
-  __syncthreads();
-  for (int s = 128; s > 0; s >>= 1) {
-    if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
-    __syncthreads();
-  }
-  if (threadIdx.x == 0 && aux) *aux = static_cast<float>(E * red[0]);
 }
 
-// Write this block's partials, take a ticket, and let the last block reduce.
-__device__ void block_partials_and_ticket(const float* blk_p, const int32_t* blk_c, float* part_p,
-                                          int32_t* part_c, int E, int T, int k, float* aux,
-                                          Control* ctl) {
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    part_p[static_cast<size_t>(blockIdx.x) * E + e] = blk_p[e];
-    part_c[static_cast<size_t>(blockIdx.x) * E + e] = blk_c[e];
-  }
-  __threadfence();
-  __syncthreads();
+// aux = E * sum_e f_e * P_e with f_e = count_e / (T*k), P_e = (sum_t p_te) / T.
+// Block e sums expert e's nblk partials (thread i: blocks i, i+256, ... in
+// order, float64; then a fixed tree) and writes its term; the last block to
+// finish (ticket) adds the E terms with a fixed tree. Deterministic.
+constexpr int kAuxThreads = 256;
+
+__global__ void __launch_bounds__(kAuxThreads)
+aux_reduce(const float* __restrict__ part_p, const int32_t* __restrict__ part_c, int ldb, int nblk,
+           int E, int T, int k, double* __restrict__ terms, float* __restrict__ aux, Control* ctl) {
+  __shared__ double sp[kAuxThreads];
+  __shared__ long long sc[kAuxThreads];
   __shared__ bool is_last;
+  const int e = blockIdx.x;
+  double ps = 0.0;
+  long long cs = 0;
+  for (int b = threadIdx.x; b < nblk; b += kAuxThreads) {
+    ps += static_cast<double>(part_p[static_cast<size_t>(e) * ldb + b]);
+    cs += part_c[static_cast<size_t>(e) * ldb + b];
+  }
+  sp[threadIdx.x] = ps;
+  sc[threadIdx.x] = cs;
+  __syncthreads();
+  for (int s = kAuxThreads / 2; s > 0; s >>= 1) {
+    if (threadIdx.x < s) { sp[threadIdx.x] += sp[threadIdx.x + s]; sc[threadIdx.x] += sc[threadIdx.x + s]; }
+    __syncthreads();
+  }
   if (threadIdx.x == 0) {
-    const unsigned prev = atomicAdd(&ctl->route_ticket, 1u);
-    is_last = (prev == gridDim.x - 1);
+    terms[e] = T > 0 ? (static_cast<double>(sc[0]) / (static_cast<double>(T) * k)) * (sp[0] / T) : 0.0;
+    __threadfence();
+    is_last = atomicAdd(&ctl->route_ticket, 1u) == gridDim.x - 1;
   }
   __syncthreads();
-  if (is_last) {
-    __threadfence();
-    finalize_aux(part_p, part_c, gridDim.x, E, T, k, aux);
-    if (threadIdx.x == 0) ctl->route_ticket = 0u;
+  if (!is_last) return;
+  __threadfence();
+  sp[threadIdx.x] = threadIdx.x < E ? __ldcg(terms + threadIdx.x) : 0.0;
+  __syncthreads();
+  for (int s = kAuxThreads / 2; s > 0; s >>= 1) {
+    if (threadIdx.x < s) sp[threadIdx.x] += sp[threadIdx.x + s];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    *aux = static_cast<float>(E * sp[0]);
+    ctl->route_ticket = 0u;
   }
 }
 
 // ---------------------------------------------------------------- fused, E <= 8
 template <typename Tin>
 struct VecTraits;
-template <> struct VecTraits<__nv_bfloat16> {
-  static constexpr int kVec = 8;  // elements per 16-byte load
-  static __device__ __forceinline__ void unpack(const uint4& u, float (&f)[8]) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      f[2 * i] = __uint_as_float(w[i] << 16);
-      f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-    }
-  }
-};
 template <> struct VecTraits<float> {
   static constexpr int kVec = 4;
   static __device__ __forceinline__ void unpack(const uint4& u, float (&f)[4]) {
@@ -153,7 +144,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 router_fused_e8(const Tin* __restrict__ x, const Tin* __restrict__ wg, const float* __restrict__ bias,
                 int T, int d, int E, int k, int32_t* __restrict__ idx_out, float* __restrict__ w_out,
                 float* __restrict__ logits_out, float* __restrict__ probs_out,
-                float* __restrict__ part_p, int32_t* __restrict__ part_c, float* __restrict__ aux,
+                float* __restrict__ part_p, int32_t* __restrict__ part_c, int ldb,
                 Control* ctl) {
   constexpr int V = VecTraits<Tin>::kVec;  // elements per 16-byte x load: 8 (bf16) or 4 (fp32)
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -364,7 +355,7 @@ router_fused_e8(const Tin* __restrict__ x, const Tin* __restrict__ wg, const flo
     tot_c[threadIdx.x] = c;
   }
   __syncthreads();
-  block_partials_and_ticket(tot_p, tot_c, part_p, part_c, E, T, k, aux, ctl);
+  block_write_partials(tot_p, tot_c, part_p, part_c, ldb, E);
 }
 
 // ---------------------------------------------------------------- general path
@@ -414,16 +405,105 @@ router_gemm_tiled(const Tin* __restrict__ x, const Tin* __restrict__ wg, int T, 
   }
 }
 
-// Warp per token: lane l holds experts l + 32q, q < EPL.
+// One token's routing by one warp: lane l holds the logits (bias included) of
+// experts l + 32q, q < EPL (-inf for e >= E). Softmax over E, top-k by k
+// rounds of a warp arg-max (ties to the lower expert), renormalised weights;
+// accumulates the token's probabilities and choices into the lane's aux sums.
 template <int EPL>
-__global__ void __launch_bounds__(256)
-router_select(const float* __restrict__ logits_in, const float* __restrict__ bias, int T, int E,
-              int k, int32_t* __restrict__ idx_out, float* __restrict__ w_out,
+__device__ __forceinline__ void warp_route_token(const float (&v)[EPL], int E, int k, int lane,
+                                                 size_t t, int32_t* __restrict__ idx_out,
+                                                 float* __restrict__ w_out,
+                                                 float* __restrict__ logits_out,
+                                                 float* __restrict__ probs_out,
+                                                 float (&psum)[EPL], int (&cnt)[EPL],
+                                                 Control* ctl) {
+#pragma unroll
+  for (int q = 0; q < EPL; ++q) {
+    const int e = lane + 32 * q;
+    if (logits_out != nullptr && e < E) logits_out[t * E + e] = v[q];
+  }
+  float m = -INFINITY;
+#pragma unroll
+  for (int q = 0; q < EPL; ++q) m = fmaxf(m, v[q]);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+  float ex[EPL], s = 0.f;
+#pragma unroll
+  for (int q = 0; q < EPL; ++q) {
+    ex[q] = (lane + 32 * q < E) ? expf(v[q] - m) : 0.f;
+    s += ex[q];
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) s += __shfl_xor_sync(kFull, s, off);
+  float p[EPL];
+#pragma unroll
+  for (int q = 0; q < EPL; ++q) {
+    const int e = lane + 32 * q;
+    p[q] = ex[q] / s;
+    if (e < E) {
+      psum[q] += p[q];
+      if (probs_out != nullptr) probs_out[t * E + e] = p[q];
+    }
+  }
+  unsigned taken = 0;
+  float wsum = 0.f;
+  int my_e = 0;
+  float my_p = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j < k) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int q = 0; q < EPL; ++q) {
+        const int e = lane + 32 * q;
+        if (e < E && !((taken >> q) & 1u) && better(v[q], e, bv, be)) { bv = v[q]; be = e; }
+      }
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) {
+        const float ov = __shfl_xor_sync(kFull, bv, off);
+        const int oe = __shfl_xor_sync(kFull, be, off);
+        if (better(ov, oe, bv, be)) { bv = ov; be = oe; }
+      }
+      if (be >= E || be < 0) {
+        if (lane == 0) set_error(ctl, MOE_DEVERR_EXPERT_RANGE);
+        be = 0;
+      }
+      const int owner = be & 31, qq = be >> 5;
+      float pv = 0.f;
+#pragma unroll
+      for (int q = 0; q < EPL; ++q)
+        if (q == qq) pv = p[q];
+      pv = __shfl_sync(kFull, pv, owner);
+      if (lane == owner) {
+#pragma unroll
+        for (int q = 0; q < EPL; ++q)
+          if (q == qq) { taken |= 1u << q; ++cnt[q]; }
+      }
+      wsum += pv;
+      if (lane == j) { my_e = be; my_p = pv; }
+    }
+  }
+  if (lane < k) {
+    idx_out[t * k + lane] = my_e;
+    w_out[t * k + lane] = my_p / wsum;
+  }
+}
+
+// Warp per token: lane l holds experts l + 32q, q < EPL. The logits are the
+// sum of KS partial [T, E] buffers (stride T*E), added in order, plus the bias.
+constexpr int kSelectWarps = 8;
+constexpr int kSelectTokensPerWarp = 2;
+constexpr int kSelectTokensPerBlock = kSelectWarps * kSelectTokensPerWarp;
+
+template <int EPL>
+__global__ void __launch_bounds__(kSelectWarps * 32)
+router_select(const float* __restrict__ logits_in, int KS, const float* __restrict__ bias, int T,
+              int E, int k, int32_t* __restrict__ idx_out, float* __restrict__ w_out,
               float* __restrict__ logits_out, float* __restrict__ probs_out,
-              float* __restrict__ part_p, int32_t* __restrict__ part_c, float* __restrict__ aux,
-              Control* ctl) {
-  __shared__ float blk_p_w[8][256];
-  __shared__ int32_t blk_c_w[8][256];
+              float* __restrict__ part_p, int32_t* __restrict__ part_c, int ldb, Control* ctl) {
+  __shared__ float blk_p_w[kSelectWarps][256];
+  __shared__ int32_t blk_c_w[kSelectWarps][256];
   __shared__ float tot_p[256];
   __shared__ int32_t tot_c[256];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -437,82 +517,30 @@ router_select(const float* __restrict__ logits_in, const float* __restrict__ bia
     const int e = lane + 32 * q;
     bq[q] = (bias != nullptr && e < E) ? bias[e] : 0.f;
   }
-  const int t_begin = blockIdx.x * kRouteSelectTokensPerBlock;
-  const int t_end = min(T, t_begin + kRouteSelectTokensPerBlock);
-  for (int t = t_begin + warp; t < t_end; t += 8) {
+  const size_t plane = static_cast<size_t>(T) * E;
+  const int t_begin = blockIdx.x * kSelectTokensPerBlock;
+  const int t_end = min(T, t_begin + kSelectTokensPerBlock);
+  for (int t = t_begin + warp; t < t_end; t += kSelectWarps) {
+    float pv[8][EPL];
+#pragma unroll
+    for (int src = 0; src < 8; ++src)
+#pragma unroll
+      for (int q = 0; q < EPL; ++q) {
+        const int e = lane + 32 * q;
+        pv[src][q] = (src < KS && e < E)
+                         ? __ldcg(logits_in + src * plane + static_cast<size_t>(t) * E + e) : 0.f;
+      }
     float v[EPL];
 #pragma unroll
     for (int q = 0; q < EPL; ++q) {
-      const int e = lane + 32 * q;
-      v[q] = e < E ? logits_in[static_cast<size_t>(t) * E + e] + bq[q] : -INFINITY;
-      if (logits_out != nullptr && e < E) logits_out[static_cast<size_t>(t) * E + e] = v[q];
+      float acc = 0.f;
+#pragma unroll
+      for (int src = 0; src < 8; ++src)
+        if (src < KS) acc += pv[src][q];
+      v[q] = (lane + 32 * q < E) ? acc + bq[q] : -INFINITY;
     }
-    float m = -INFINITY;
-#pragma unroll
-    for (int q = 0; q < EPL; ++q) m = fmaxf(m, v[q]);
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
-    float ex[EPL], s = 0.f;
-#pragma unroll
-    for (int q = 0; q < EPL; ++q) {
-      ex[q] = (lane + 32 * q < E) ? expf(v[q] - m) : 0.f;
-      s += ex[q];
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) s += __shfl_xor_sync(kFull, s, off);
-    float p[EPL];
-#pragma unroll
-    for (int q = 0; q < EPL; ++q) {
-      const int e = lane + 32 * q;
-      p[q] = ex[q] / s;
-      if (e < E) {
-        psum[q] += p[q];
-        if (probs_out != nullptr) probs_out[static_cast<size_t>(t) * E + e] = p[q];
-      }
-    }
-    unsigned taken = 0;
-    float wsum = 0.f;
-    int my_e = 0;
-    float my_p = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j < k) {
-        float bv = -INFINITY;
-        int be = 0x7fffffff;
-#pragma unroll
-        for (int q = 0; q < EPL; ++q) {
-          const int e = lane + 32 * q;
-          if (e < E && !((taken >> q) & 1u) && better(v[q], e, bv, be)) { bv = v[q]; be = e; }
-        }
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) {
-          const float ov = __shfl_xor_sync(kFull, bv, off);
-          const int oe = __shfl_xor_sync(kFull, be, off);
-          if (better(ov, oe, bv, be)) { bv = ov; be = oe; }
-        }
-        if (be >= E || be < 0) {
-          if (lane == 0) set_error(ctl, MOE_DEVERR_EXPERT_RANGE);
-          be = 0;
-        }
-        const int owner = be & 31, qq = be >> 5;
-        float pv = 0.f;
-#pragma unroll
-        for (int q = 0; q < EPL; ++q)
-          if (q == qq) pv = p[q];
-        pv = __shfl_sync(kFull, pv, owner);
-        if (lane == owner) {
-#pragma unroll
-          for (int q = 0; q < EPL; ++q)
-            if (q == qq) { taken |= 1u << q; ++cnt[q]; }
-        }
-        wsum += pv;
-        if (lane == j) { my_e = be; my_p = pv; }
-      }
-    }
-    if (lane < k) {
-      idx_out[static_cast<size_t>(t) * k + lane] = my_e;
-      w_out[static_cast<size_t>(t) * k + lane] = my_p / wsum;
-    }
+    warp_route_token<EPL>(v, E, k, lane, static_cast<size_t>(t), idx_out, w_out, logits_out,
+                          probs_out, psum, cnt, ctl);
   }
 #pragma unroll
   for (int q = 0; q < EPL; ++q) {
@@ -523,87 +551,331 @@ router_select(const float* __restrict__ logits_in, const float* __restrict__ bia
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     float a = 0.f;
     int c = 0;
-    for (int w = 0; w < 8; ++w) { a += blk_p_w[w][e]; c += blk_c_w[w][e]; }
+    for (int w = 0; w < kSelectWarps; ++w) { a += blk_p_w[w][e]; c += blk_c_w[w][e]; }
     tot_p[e] = a;
     tot_c[e] = c;
   }
   __syncthreads();
-  block_partials_and_ticket(tot_p, tot_c, part_p, part_c, E, T, k, aux, ctl);
+  block_write_partials(tot_p, tot_c, part_p, part_c, ldb, E);
+}
+
+// ---------------------------------------------------------------- tensor cores
+// The gate GEMM on tcgen05 for bf16 layers. CTA (tile, ks) takes 128 tokens
+// and the d-range [ks*dk, (ks+1)*dk). Warp 0 streams the x tile (TMA, 128x64,
+// 128-byte swizzle) through a 4-stage ring; warp 1 issues M=128, N=Epad (E
+// rounded up to 16), K=16 MMAs into tensor memory. Wg is either TMA-streamed
+// beside x as the MN-major operand (E a multiple of 64, the expert GEMM's B
+// path) or, for E <= 32, transposed once into shared memory as a K-major
+// operand (the first ring stages are already loading meanwhile). The four
+// warps then copy their 32 accumulator rows to the fp32 partial buffer
+// logits[ks][t][e]; router_select adds the KS partials in ks order.
+constexpr int kTcStages = 4;
+constexpr int kTcThreads = 128;
+
+struct RouterTcArgs {
+  int T, d, E, Epad, KS, dk;
+  const __nv_bfloat16* wg;  // [d, E] (staged path)
+  float* partial;           // [KS][T][E]
+  Control* ctl;
+};
+
+template <bool kTmaB>
+__global__ void __launch_bounds__(kTcThreads, 1)
+router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+          RouterTcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[kTcStages], empty_bar[kTcStages], done_bar;
+  __shared__ uint32_t tmem_base_s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int tile = blockIdx.x / a.KS;
+  const int ks = blockIdx.x - tile * a.KS;
+  const int nkb = a.dk / 64;
+  const int b_boxes = kTmaB ? a.Epad / 64 : 0;
+  const uint32_t a_bytes = 128 * 128, stage_bytes = a_bytes + b_boxes * 8192;
+  uint8_t* ring = smem;
+  uint8_t* wgt = smem + kTcStages * stage_bytes;  // staged Wg^T (E <= 32)
+  const uint32_t wgt_kb_bytes = static_cast<uint32_t>(a.Epad) * 128;
+  // Accumulator slots: k-block kb accumulates into TMEM columns
+  // [(kb / G) * Epad, +Epad), G k-blocks per slot, as many slots as 512
+  // columns hold. The epilogue adds the slots in IEEE fp32, so a tensor-core
+  // accumulation chain is at most 4*G MMAs long.
+  const int nslot_cap = 512 / a.Epad;
+  const int G = (nkb + nslot_cap - 1) / nslot_cap;
+  const int nslot = (nkb + G - 1) / G;
+  uint32_t tcols = 32;
+  while (tcols < static_cast<uint32_t>(nslot * a.Epad)) tcols <<= 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTcStages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    mbar_init(&done_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_s, tcols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+
+  // The first ring stages are free: start their loads before anything else.
+  const int pre = nkb < kTcStages ? nkb : kTcStages;
+  auto issue = [&](int kb, int st) {
+    uint8_t* sa = ring + st * stage_bytes;
+    const int kx = ks * a.dk + kb * 64;
+    mbar_arrive_expect_tx(&full_bar[st], stage_bytes);
+    tma_load_2d(sa, &tmX, &full_bar[st], kx, tile * 128);
+    for (int j = 0; j < b_boxes; ++j) tma_load_2d(sa + a_bytes + j * 8192, &tmW, &full_bar[st], j * 64, kx);
+  };
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmX);
+    if (kTmaB) prefetch_tmap(&tmW);
+    for (int kb = 0; kb < pre; ++kb) issue(kb, kb);
+  }
+  if (!kTmaB) {
+    // Wg^T for this CTA's d-range as K-major 128-byte-swizzled rows: expert e,
+    // k-block kb -> row e of block kb, 16-byte chunk (kk/8) ^ (e%8). One Wg
+    // row (E % 8 == 0 experts) per group of 16-byte loads; experts E..Epad-1
+    // are zero.
+    const int k0 = ks * a.dk;
+    const int vecs = a.E / 8, vecs_pad = a.Epad / 8;
+#pragma unroll 4
+    for (int i = threadIdx.x; i < a.dk * vecs_pad; i += kTcThreads) {
+      const int kl = i / vecs_pad, vq = i - kl * vecs_pad;
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (vq < vecs)
+        u = __ldg(reinterpret_cast<const uint4*>(a.wg + static_cast<size_t>(k0 + kl) * a.E) + vq);
+      const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+      const int kb = kl >> 6, kk = kl & 63;
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        const int e = vq * 8 + h;
+        const uint32_t off = kb * wgt_kb_bytes + e * 128 + ((((kk >> 3) ^ (e & 7)) & 7) << 4) + (kk & 7) * 2;
+        *reinterpret_cast<uint16_t*>(wgt + off) =
+            static_cast<uint16_t>((h & 1) ? (wv[h >> 1] >> 16) : (wv[h >> 1] & 0xffffu));
+      }
+    }
+    fence_proxy_async_smem();  // generic-proxy writes, read by the tensor core
+    __syncthreads();
+  }
+
+  bool ok = true;
+  if (warp == 0 && lane == 0) {
+    uint32_t phase = 1;  // the prologue filled round 0
+    int st = pre % kTcStages;
+    if (pre < kTcStages) phase = 0;
+    for (int kb = pre; kb < nkb; ++kb) {
+      if (!mbar_wait_bounded(&empty_bar[st], phase ^ 1u)) { set_error(a.ctl, MOE_DEVERR_TIMEOUT); break; }
+      issue(kb, st);
+      if (++st == kTcStages) { st = 0; phase ^= 1u; }
+    }
+  } else if (warp == 1 && lane == 0) {
+    const uint32_t idesc = make_idesc_bf16(128, a.Epad, !kTmaB);
+    uint32_t phase = 0;
+    bool issued = false;
+    for (int kb = 0, st = 0; kb < nkb; ++kb) {
+      if (!mbar_wait_bounded(&full_bar[st], phase)) { set_error(a.ctl, MOE_DEVERR_TIMEOUT); break; }
+      tc_fence_after();
+      const uint32_t a_addr = smem_u32(ring + st * stage_bytes);
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>((kb / G) * a.Epad);
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t adesc = make_sw128_desc(a_addr + kk * 32, 16, 1024);
+        const uint64_t bdesc = kTmaB ? make_sw128_desc(a_addr + a_bytes + kk * 2048, 8192, 1024)
+                                     : make_sw128_desc(smem_u32(wgt) + kb * wgt_kb_bytes + kk * 32, 16, 1024);
+        umma_bf16(d_tmem, adesc, bdesc, idesc, ((kb % G) | kk) != 0 ? 1u : 0u);
+      }
+      issued = true;
+      umma_commit(&empty_bar[st]);
+      if (++st == kTcStages) { st = 0; phase ^= 1u; }
+    }
+    if (issued) umma_commit(&done_bar);
+    else mbar_arrive(&done_bar);
+  }
+  {
+    int d_ok = 0;
+    if (lane == 0) d_ok = mbar_wait_bounded(&done_bar, 0);
+    d_ok = __shfl_sync(kFull, d_ok, 0);
+    if (!d_ok) { if (lane == 0) set_error(a.ctl, MOE_DEVERR_TIMEOUT); ok = false; }
+  }
+  tc_fence_after();
+  // ---- accumulator rows -> partial logits [ks][t][e]
+  {
+    const int r = warp * 32 + lane;
+    const int t = tile * 128 + r;
+    float* dst = a.partial + static_cast<size_t>(ks) * a.T * a.E + static_cast<size_t>(t) * a.E;
+    const uint32_t trow = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+    for (int c0 = 0; c0 < a.Epad; c0 += 16) {
+      float sum[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) sum[i] = 0.f;
+      for (int sl = 0; sl < nslot; ++sl) {  // slot order
+        uint32_t u[16];
+        tmem_ld_32x32b_x16(trow + sl * a.Epad + c0, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sum[i] += __uint_as_float(u[i]);
+      }
+      uint32_t v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(sum[i]);
+      if (t < a.T && ok) {
+        if (c0 + 16 <= a.E) {
+#pragma unroll
+          for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4*>(dst + c0 + i) =
+                make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                            __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (c0 + i < a.E) dst[c0 + i] = __uint_as_float(v[i]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tcols);
+  }
 }
 
 bool use_fused(int d, int E, moe_dtype_t dt) {
-  (void)dt;
   const size_t bytes = static_cast<size_t>((d + 7) / 8) * 256;  // fp32 pairs, 256 B per 8 rows
-  return E <= 8 && d % 8 == 0 && bytes <= 160 * 1024;
+  return dt == MOE_F32 && E <= 8 && d % 8 == 0 && bytes <= 160 * 1024;
 }
 
 size_t fused_smem_bytes(int d) { return static_cast<size_t>((d + 7) / 8) * 256; }
 
+// Tensor-core router plan: split factor KS (a power of two <= 8 dividing the
+// d/64 k-blocks) grows while the grid stays within the SMs; the staged Wg^T
+// of one CTA must fit in 128 KB.
+constexpr int kMaxKS = 8;
+
+struct TcPlan {
+  bool use = false;
+  bool tma_b = false;
+  int Epad = 0, KS = 1, ntile = 0;
+  size_t smem = 0;
+};
+
+TcPlan plan_tc(int T, int d, int E, moe_dtype_t dt) {
+  TcPlan p;
+  if (dt != MOE_BF16 || T <= 0 || d % 64 != 0) return p;
+  if (E % 64 == 0) {
+    p.tma_b = true;
+    p.Epad = E;
+  } else if (E <= 32 && E % 8 == 0) {
+    p.Epad = (E + 15) / 16 * 16;
+  } else {
+    return p;
+  }
+  p.ntile = (T + 127) / 128;
+  const int nkb = d / 64;
+  int ks = 1;
+  while (ks < kMaxKS && p.ntile * ks * 2 <= num_sms() && nkb % (ks * 2) == 0) ks *= 2;
+  if (!p.tma_b)
+    while (static_cast<size_t>(d / ks) * p.Epad * 2 > 128 * 1024 && ks < kMaxKS && nkb % (ks * 2) == 0) ks *= 2;
+  if (!p.tma_b && static_cast<size_t>(d / ks) * p.Epad * 2 > 128 * 1024) return p;
+  p.KS = ks;
+  const size_t stage = 128 * 128 + (p.tma_b ? static_cast<size_t>(p.Epad / 64) * 8192 : 0);
+  p.smem = 1024 + kTcStages * stage + (p.tma_b ? 0 : static_cast<size_t>(d / ks) * p.Epad * 2);
+  p.use = true;
+  return p;
+}
+
 }  // namespace
 
 static int route_max_blocks(int T) {
-  return std::max((T + kRouteSelectTokensPerBlock - 1) / kRouteSelectTokensPerBlock,
-                  std::max(1, 2 * num_sms()));
+  return std::max(std::max(1, (T + kSelectTokensPerBlock - 1) / kSelectTokensPerBlock), num_sms());
 }
 
 size_t route_partials_bytes(int T, int E) {
-  // Sized for the larger of the two paths' grids: sums then counts.
-  return align_up(static_cast<size_t>(route_max_blocks(T)) * E * 4) * 2;
+  // per-block sums then counts (expert-major), then the per-expert terms
+  return align_up(static_cast<size_t>(route_max_blocks(T)) * E * 4) * 2 + align_up(256 * 8);
 }
 
 size_t route_logits_scratch_bytes(int T, int d, int E) {
   (void)d;
-  return align_up(static_cast<size_t>(T) * E * 4);
+  return align_up(static_cast<size_t>(kMaxKS) * T * E * 4);
 }
 
 cudaError_t launch_route(const void* x, const void* wg, const float* bias, moe_dtype_t dt, int T,
                          int d, int E, int k, int32_t* idx, float* w, float* aux, float* logits,
                          float* probs, float* logits_scratch, void* partials, Control* ctl,
                          cudaStream_t s) {
-  const int nb_max = route_max_blocks(T);
+  const int ldb = route_max_blocks(T);
   float* part_p = static_cast<float*>(partials);
   int32_t* part_c = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(partials) +
-                                               align_up(static_cast<size_t>(nb_max) * E * 4));
+                                               align_up(static_cast<size_t>(ldb) * E * 4));
+  double* terms = reinterpret_cast<double*>(static_cast<uint8_t*>(partials) +
+                                            2 * align_up(static_cast<size_t>(ldb) * E * 4));
+  int nblk = 0;
   if (use_fused(d, E, dt)) {
     const int groups = (T + kFusedTokensPerGroup - 1) / kFusedTokensPerGroup;
     const int grid = std::max(1, std::min(groups, num_sms()));
     const size_t smem = fused_smem_bytes(d);
-    if (dt == MOE_BF16) {
-      auto kern = router_fused_e8<__nv_bfloat16>;
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      kern<<<grid, kFusedThreads, smem, s>>>(static_cast<const __nv_bfloat16*>(x),
-                                             static_cast<const __nv_bfloat16*>(wg), bias, T, d, E, k,
-                                             idx, w, logits, probs, part_p, part_c, aux, ctl);
-    } else {
-      auto kern = router_fused_e8<float>;
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      kern<<<grid, kFusedThreads, smem, s>>>(static_cast<const float*>(x), static_cast<const float*>(wg),
-                                             bias, T, d, E, k, idx, w, logits, probs, part_p, part_c,
-                                             aux, ctl);
+    auto kern = router_fused_e8<float>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    kern<<<grid, kFusedThreads, smem, s>>>(static_cast<const float*>(x), static_cast<const float*>(wg),
+                                           bias, T, d, E, k, idx, w, logits, probs, part_p, part_c,
+                                           ldb, ctl);
+    nblk = grid;
+  } else {
+    int KS = 1;
+    const TcPlan tp = plan_tc(T, d, E, dt);
+    if (tp.use) {
+      CUtensorMap tx, tw;
+      if (!make_tma_2d_bf16(&tx, x, static_cast<uint64_t>(T), d, 128)) return cudaErrorInvalidValue;
+      if (tp.tma_b) {
+        if (!make_tma_2d_bf16(&tw, wg, static_cast<uint64_t>(d), E, 64)) return cudaErrorInvalidValue;
+      } else {
+        tw = tx;  // unused by the staged path
+      }
+      RouterTcArgs a;
+      a.T = T; a.d = d; a.E = E; a.Epad = tp.Epad; a.KS = tp.KS; a.dk = d / tp.KS;
+      a.wg = static_cast<const __nv_bfloat16*>(wg);
+      a.partial = logits_scratch;
+      a.ctl = ctl;
+      const dim3 grid(tp.ntile * tp.KS);
+      if (tp.tma_b) {
+        cudaFuncSetAttribute(router_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(tp.smem));
+        router_tc<true><<<grid, kTcThreads, tp.smem, s>>>(tx, tw, a);
+      } else {
+        cudaFuncSetAttribute(router_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(tp.smem));
+        router_tc<false><<<grid, kTcThreads, tp.smem, s>>>(tx, tw, a);
+      }
+      KS = tp.KS;
+    } else if (T > 0) {
+      dim3 g1((T + 63) / 64, (E + 63) / 64);
+      if (dt == MOE_BF16)
+        router_gemm_tiled<__nv_bfloat16><<<g1, 256, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(wg), T, d, E,
+            logits_scratch);
+      else
+        router_gemm_tiled<float><<<g1, 256, 0, s>>>(static_cast<const float*>(x),
+                                                    static_cast<const float*>(wg), T, d, E,
+                                                    logits_scratch);
     }
-    return cudaGetLastError();
-  }
-  if (T > 0) {
-    dim3 g1((T + 63) / 64, (E + 63) / 64);
-    if (dt == MOE_BF16)
-      router_gemm_tiled<__nv_bfloat16><<<g1, 256, 0, s>>>(
-          static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(wg), T, d, E,
-          logits_scratch);
-    else
-      router_gemm_tiled<float><<<g1, 256, 0, s>>>(static_cast<const float*>(x),
-                                                  static_cast<const float*>(wg), T, d, E,
-                                                  logits_scratch);
-  }
-  const int g2 = std::max(1, (T + kRouteSelectTokensPerBlock - 1) / kRouteSelectTokensPerBlock);
-  const int epl = (E + 31) / 32;
-#define MOE_SELECT(N)                                                                        \
-  router_select<N><<<g2, 256, 0, s>>>(logits_scratch, bias, T, E, k, idx, w, logits, probs, \
-                                      part_p, part_c, aux, ctl)
-  if (epl <= 1) MOE_SELECT(1);
-  else if (epl <= 2) MOE_SELECT(2);
-  else if (epl <= 4) MOE_SELECT(4);
-  else MOE_SELECT(8);
+    const int g2 = std::max(1, (T + kSelectTokensPerBlock - 1) / kSelectTokensPerBlock);
+    const int epl = (E + 31) / 32;
+#define MOE_SELECT(N)                                                                          \
+  router_select<N><<<g2, kSelectWarps * 32, 0, s>>>(logits_scratch, KS, bias, T, E, k, idx, w, \
+                                                    logits, probs, part_p, part_c, ldb, ctl)
+    if (epl <= 1) MOE_SELECT(1);
+    else if (epl <= 2) MOE_SELECT(2);
+    else if (epl <= 4) MOE_SELECT(4);
+    else MOE_SELECT(8);
 #undef MOE_SELECT
+    nblk = g2;
+  }
+  aux_reduce<<<E, kAuxThreads, 0, s>>>(part_p, part_c, ldb, nblk, E, T, k, terms, aux, ctl);
   return cudaGetLastError();
 }
 

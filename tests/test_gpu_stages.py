@@ -33,7 +33,12 @@ def route_on_gpu(x, wg, bias, T, d, E, k):
     (77, 4096, 8, 2, "bf16", "expert0"),   # fused, d = 4096, ragged quad
     (300, 256, 5, 3, "bf16", "none"),      # fused with E < 8 (padded experts)
     (513, 256, 64, 2, "bf16", "zipf"),     # tiled GEMM + select, 2 experts per lane
-    (129, 256, 256, 8, "bf16", "none"),    # 8 experts per lane, k = 8
+    (129, 256, 256, 8, "bf16", "none"),    # tensor cores, TMA Wg, 8 experts per lane, k = 8
+    (300, 512, 16, 2, "bf16", "zipf"),     # tensor cores, staged Wg^T (E <= 32)
+    (1000, 1024, 32, 4, "bf16", "none"),   # tensor cores, staged Wg^T, split over d
+    (2000, 1024, 64, 2, "bf16", "zipf"),   # tensor cores, TMA Wg, one tile per CTA
+    (97, 128, 128, 3, "bf16", "none"),     # tensor cores, 4 experts per lane
+    (10000, 4096, 8, 2, "bf16", "expert0"),  # tensor cores, no d split: 64 k-blocks in 32 slots
     (200, 64, 4, 1, "f32", "none"),        # fp32 fused
     (90, 64, 40, 4, "f32", "none"),        # fp32 general
 ])
@@ -69,13 +74,16 @@ def test_route_exact_ties_lower_index():
         wt = torch.from_numpy(wg).to(dt).to(DEV)
         idx, *_ = route_on_gpu(xt, wt, None, T, d, E, k)
         assert np.array_equal(npi(idx), O.topk_select(x[:, :E], k))
-    E2 = 40
-    wg2 = np.zeros((d, E2), np.float32)
-    wg2[:E2, :E2] = np.eye(E2)
-    x2 = np.zeros((T, d), np.float32)
-    x2[:, :E2] = rng.integers(-1, 2, size=(T, E2))
-    idx, *_ = route_on_gpu(torch.from_numpy(x2).to(DEV), torch.from_numpy(wg2).to(DEV), None, T, d, E2, 5)
-    assert np.array_equal(npi(idx), O.topk_select(x2[:, :E2], 5))
+    # E = 16, 32 (tensor cores, staged Wg^T), 40 (CUDA cores), 64 (tensor cores, TMA Wg)
+    for E2 in (16, 32, 40, 64):
+        wg2 = np.zeros((d, E2), np.float32)
+        wg2[:E2, :E2] = np.eye(E2)
+        x2 = np.zeros((T, d), np.float32)
+        x2[:, :E2] = rng.integers(-1, 2, size=(T, E2))
+        for dt in (torch.bfloat16, torch.float32):
+            idx, *_ = route_on_gpu(torch.from_numpy(x2).to(dt).to(DEV),
+                                   torch.from_numpy(wg2).to(dt).to(DEV), None, T, d, E2, 5)
+            assert np.array_equal(npi(idx), O.topk_select(x2[:, :E2], 5)), (E2, dt)
 
 
 def permute_on_gpu(idx_np, E, cap):
