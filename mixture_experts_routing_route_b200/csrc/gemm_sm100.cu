@@ -17,13 +17,15 @@
 // CTA = 6 warps, one CTA per SM, persistent over tiles:
 //   warp 0   TMA producer: A tile 128x64 and B tile 64xN per stage, 128-byte
 //            swizzle, into a 4-stage shared-memory ring (mbarrier full/empty)
-//   warp 1   MMA issuer: one thread issues tcgen05.mma (M=128, N=256, K=16)
-//            into a double-buffered fp32 accumulator in tensor memory and
-//            frees ring slots / publishes accumulators with tcgen05.commit
+//   warp 1   MMA issuer: one thread issues tcgen05.mma (M=128, N=256, K=16;
+//            M=64 for a tile of at most 64 valid rows) into a double-buffered
+//            fp32 accumulator in tensor memory and frees ring slots /
+//            publishes accumulators with tcgen05.commit
 //   warps 2-5 epilogue: tcgen05.ld of their 32-lane quarter of the
 //            accumulator, activation, bf16 stores of valid rows only
 // Tiles are ordered expert-major, then N, with the M tile fastest, so CTAs
-// that run at the same time share one weight column block through L2.
+// that run at the same time share one weight column block through L2; a
+// partial last wave is split into half-width tiles.
 // Every wait is bounded; a time-out sets MOE_DEVERR_TIMEOUT and unwinds.
 #include "common.cuh"
 #include "ptx.cuh"
@@ -34,25 +36,13 @@ namespace moe {
 
 namespace {
 
-constexpr int BM = 128;
-constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle row
-constexpr int STAGES = 4;
+constexpr int BM = 128;  // rows of A per CTA
+constexpr int BK = 64;   // 64 bf16 = one 128-byte swizzle row
 constexpr int kThreads = 192;
 constexpr int kMaxE = 256;
+constexpr int kBoxBytes = 64 * BK * 2;  // one 64-column B box: 8 KB
 
 enum { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_STORE = 2 };
-
-template <int EPI, int NMMA>
-struct Cfg {
-  static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BK * NMMA * 2;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int OUT_N = EPI == EPI_SWIGLU ? NMMA / 2 : NMMA;
-  static constexpr int B_BOXES = NMMA / 64;  // 64-column boxes of 8 KB
-  static constexpr int TMEM_COLS = 2 * NMMA;
-  static constexpr size_t SMEM = static_cast<size_t>(STAGES) * STAGE_BYTES + 1024;
-  static constexpr uint32_t IDESC = make_idesc_bf16(BM, NMMA);
-};
 
 struct GemmArgs {
   const int32_t* seg;  // [E+1] row segment offsets
@@ -74,13 +64,80 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Tile -> (expert, row start, valid rows, n0).
+// ------------------------------------------------------------------ schedule
+// Warp 0: copy the segment offsets, then tile_start[e] = exclusive prefix of
+// the per-expert unit counts ceil(m_e / TILE_M) * ntn; tile_start[E] = total.
+// Lane l owns experts [8l, 8l + 8). A segment whose rows are out of range is
+// reported and gets zero tiles.
+template <int TILE_M>
+__device__ __forceinline__ void build_schedule(const GemmArgs& args, int ntn, const int* seg_s,
+                                               int* tile_start_s, int lane) {
+  const int E = args.E;
+  int loc[8];
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane * 8 + i;
+    int m = 0;
+    if (e < E) {
+      m = seg_s[e + 1] - seg_s[e];
+      if (m < 0 || seg_s[e] < 0 || seg_s[e + 1] > args.rows_max) {
+        set_error(args.ctl, MOE_DEVERR_ROW_RANGE);
+        m = 0;
+      }
+    }
+    loc[i] = ((m + TILE_M - 1) / TILE_M) * ntn;
+    sum += loc[i];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += n;
+  }
+  int run = incl - sum;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane * 8 + i;
+    if (e < E) tile_start_s[e] = run;
+    run += loc[i];
+  }
+  // The lanes cover experts 0..255 only; the total goes to entry E (which is
+  // 256 when E = 256). Experts >= E contributed 0 tiles to the sum.
+  if (lane == 31) tile_start_s[E] = incl;
+}
+
+// Tile -> (expert, first row, valid rows, first output column, half width).
 struct Tile {
   int e, row0, rows, n0;
+  bool half;
 };
 
-__device__ __forceinline__ Tile decode_tile(int tau, const int* tile_start, const int* seg, int E,
-                                            int ntn, int out_n) {
+// Work units: tiles ordered expert-major, then N tile, M tile fastest, dealt
+// round-robin to W persistent workers. When the last wave would leave workers
+// idle (total % W = r tiles, 2r <= W), those r tiles become 2r half-width
+// units (N/2 columns each), so the tail takes half a tile's time.
+__device__ __forceinline__ bool split_tail(int total, int W) {
+  const int r = total % W;
+  return r != 0 && 2 * r <= W;
+}
+
+__device__ __forceinline__ int num_units(int total, int W) {
+  return split_tail(total, W) ? total + total % W : total;
+}
+
+template <int TILE_M, int OUT_N>
+__device__ __forceinline__ Tile decode_unit(int u, int total, int W, const int* tile_start,
+                                            const int* seg, int E) {
+  int tau = u, half = -1;
+  if (split_tail(total, W)) {
+    const int r = total % W;
+    if (u >= total - r) {
+      const int h = u - (total - r);
+      tau = total - r + (h >> 1);
+      half = h & 1;
+    }
+  }
   int lo = 0, hi = E - 1;  // last e with tile_start[e] <= tau
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -88,16 +145,91 @@ __device__ __forceinline__ Tile decode_tile(int tau, const int* tile_start, cons
   }
   const int e = lo;
   const int m_e = seg[e + 1] - seg[e];
-  const int mt_e = (m_e + BM - 1) / BM;
+  const int mt_e = (m_e + TILE_M - 1) / TILE_M;
   const int local = tau - tile_start[e];
   const int nt = local / mt_e, mt = local - nt * mt_e;
   Tile t;
   t.e = e;
-  t.row0 = seg[e] + mt * BM;
-  t.rows = min(BM, m_e - mt * BM);
-  t.n0 = nt * out_n;
-  (void)ntn;
+  t.row0 = seg[e] + mt * TILE_M;
+  t.rows = min(TILE_M, m_e - mt * TILE_M);
+  t.n0 = nt * OUT_N + (half > 0 ? OUT_N / 2 : 0);
+  t.half = half >= 0;
   return t;
+}
+
+// ------------------------------------------------------------------ epilogue
+// One thread = one accumulator row (its TMEM lane): OUTN output columns read
+// 32 at a time, activation in fp32, rounded once to bf16, stored if the row
+// is valid. SwiGLU: gate in columns [0, OUTN), up in [OUTN, 2 OUTN).
+template <int EPI, int OUTN>
+__device__ __forceinline__ void epilogue_row(uint32_t tbase, bool valid, __nv_bfloat16* orow) {
+#pragma unroll 1
+  for (int c = 0; c < OUTN; c += 32) {
+    uint32_t v[32];
+    uint32_t packed[16];
+    if constexpr (EPI == EPI_SWIGLU) {
+      uint32_t u[32];
+      tmem_ld_32x32b_x32(tbase + c, v);
+      tmem_ld_32x32b_x32(tbase + OUTN + c, u);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float h0 = silu(__uint_as_float(v[2 * i])) * __uint_as_float(u[2 * i]);
+        const float h1 = silu(__uint_as_float(v[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+        packed[i] = pack_bf16(h0, h1);
+      }
+    } else {
+      tmem_ld_32x32b_x32(tbase + c, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float a = __uint_as_float(v[2 * i]), b = __uint_as_float(v[2 * i + 1]);
+        if (EPI == EPI_GELU) { a = gelu_erf(a); b = gelu_erf(b); }
+        packed[i] = pack_bf16(a, b);
+      }
+    }
+    if (valid) {
+      uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+    }
+  }
+}
+
+// ==================================================================== kernel
+// Tile 128 x NMMA per CTA, 4-stage ring of 48 KB (NMMA = 256). A tile with
+// at most 64 valid rows (an expert's last) runs as an M = 64 MMA: half the
+// tensor work, the same operand loads. In tensor memory an M = 64 result
+// keeps rows 16 q .. 16 q + 15 in lanes 32 q .. 32 q + 15 (q = 0..3), so each
+// epilogue warp still owns one lane quarter, with 16 rows in it.
+constexpr int STAGES = 4;
+
+template <int EPI, int NMMA>
+struct Cfg {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BK * NMMA * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int OUT_N = EPI == EPI_SWIGLU ? NMMA / 2 : NMMA;
+  static constexpr int TMEM_COLS = 2 * NMMA;
+  static constexpr size_t SMEM = static_cast<size_t>(STAGES) * STAGE_BYTES + 1024;
+};
+
+// B boxes of one stage: SwiGLU puts NBOX/2 gate boxes then NBOX/2 up boxes
+// over the same output columns.
+template <int EPI, int NBOX>
+__device__ __forceinline__ void load_b_boxes(uint8_t* sb, const CUtensorMap* b0,
+                                             const CUtensorMap* b1, uint64_t* bar, int n0,
+                                             int brow) {
+#pragma unroll
+  for (int j = 0; j < NBOX; ++j) {
+    if constexpr (EPI == EPI_SWIGLU) {
+      constexpr int H = NBOX / 2;
+      tma_load_2d(sb + j * kBoxBytes, j < H ? b0 : b1, bar, n0 + (j % H) * 64, brow);
+    } else {
+      tma_load_2d(sb + j * kBoxBytes, b0, bar, n0 + j * 64, brow);
+    }
+  }
 }
 
 template <int EPI, int NMMA>
@@ -105,6 +237,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                 const __grid_constant__ CUtensorMap tmB1, GemmArgs args) {
   using C = Cfg<EPI, NMMA>;
+  // A half-width unit still loads whole 64-column boxes: gate and up halves
+  // need at least one box each under SwiGLU.
+  static_assert(EPI == EPI_SWIGLU ? NMMA >= 256 : NMMA >= 128, "half units need whole boxes");
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES];
   __shared__ __align__(8) uint64_t tfull_bar[2], tempty_bar[2], drain_bar;
@@ -118,46 +253,10 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
 
-  // ---- schedule: per-expert tile counts and their prefix
   for (int i = threadIdx.x; i <= E; i += kThreads) seg_s[i] = __ldg(args.seg + i);
   if (threadIdx.x == 0) abort_s = 0;
   __syncthreads();
-  const int ntn = args.N / C::OUT_N;
-  if (warp == 0) {
-    // lane l owns experts [8l, 8l+8)
-    int loc[8];
-    int sum = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane * 8 + i;
-      int m = 0;
-      if (e < E) {
-        m = seg_s[e + 1] - seg_s[e];
-        if (m < 0 || seg_s[e] < 0 || seg_s[e + 1] > args.rows_max) {
-          set_error(args.ctl, MOE_DEVERR_ROW_RANGE);
-          m = 0;
-        }
-      }
-      loc[i] = ((m + BM - 1) / BM) * ntn;
-      sum += loc[i];
-    }
-    int incl = sum;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += n;
-    }
-    int run = incl - sum;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane * 8 + i;
-      if (e < E) tile_start_s[e] = run;
-      run += loc[i];
-    }
-    // The lanes cover experts 0..255 only; the total goes to entry E (which
-    // is 256 when E = 256). Experts >= E contributed 0 tiles to the sum.
-    if (lane == 31) tile_start_s[E] = incl;
-  }
+  if (warp == 0) build_schedule<BM>(args, args.N / C::OUT_N, seg_s, tile_start_s, lane);
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(&tfull_bar[b], 1); mbar_init(&tempty_bar[b], 4); }
@@ -172,9 +271,10 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_s;
-  // A segment whose rows are out of range gets zero tiles; the true total is
-  // the prefix at E (entries past a bad segment were computed with m = 0).
-  const int total = tile_start_s[E];
+  const int total_tiles = tile_start_s[E];
+  const int W = gridDim.x;
+  const int total = num_units(total_tiles, W);
+  const int nkb = args.K / BK;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -185,9 +285,9 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       uint32_t phase = 0;
       uint32_t issued_mask = 0;  // stages that ever received a load
       uint32_t last_parity = 0;  // parity of that stage's latest load
-      const int nkb = args.K / BK;
-      for (int tau = blockIdx.x; tau < total && !abort_s; tau += gridDim.x) {
-        const Tile t = decode_tile(tau, tile_start_s, seg_s, E, ntn, C::OUT_N);
+      for (int u = blockIdx.x; u < total && !abort_s; u += W) {
+        const Tile t = decode_unit<BM, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, E);
+        const uint32_t tx = C::A_BYTES + (t.half ? C::B_BYTES / 2 : C::B_BYTES);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u)) {
             set_error(args.ctl, MOE_DEVERR_TIMEOUT);
@@ -196,19 +296,13 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           }
           uint8_t* sa = smem + stage * C::STAGE_BYTES;
           uint8_t* sb = sa + C::A_BYTES;
-          mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
+          mbar_arrive_expect_tx(&full_bar[stage], tx);
           tma_load_2d(sa, &tmA, &full_bar[stage], kb * BK, t.row0);
           const int brow = t.e * args.K + kb * BK;
-#pragma unroll
-          for (int j = 0; j < C::B_BOXES; ++j) {
-            if (EPI == EPI_SWIGLU) {
-              constexpr int H = C::B_BOXES / 2;
-              tma_load_2d(sb + j * 8192, j < H ? &tmB0 : &tmB1, &full_bar[stage],
-                          t.n0 + (j % H) * 64, brow);
-            } else {
-              tma_load_2d(sb + j * 8192, &tmB0, &full_bar[stage], t.n0 + j * 64, brow);
-            }
-          }
+          if (t.half)
+            load_b_boxes<EPI, NMMA / 128>(sb, &tmB0, &tmB1, &full_bar[stage], t.n0, brow);
+          else
+            load_b_boxes<EPI, NMMA / 64>(sb, &tmB0, &tmB1, &full_bar[stage], t.n0, brow);
           issued_mask |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -220,13 +314,19 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     }
   } else if (warp == 1) {
     if (lane == 0) {
+      constexpr uint32_t kIdescFull = make_idesc_bf16(BM, NMMA);
+      constexpr uint32_t kIdescHalf = make_idesc_bf16(BM, NMMA / 2);
+      constexpr uint32_t kIdescFull64 = make_idesc_bf16(64, NMMA);
+      constexpr uint32_t kIdescHalf64 = make_idesc_bf16(64, NMMA / 2);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      const int nkb = args.K / BK;
       bool issued_any = false;
-      for (int tau = blockIdx.x; tau < total && !abort_s; tau += gridDim.x) {
+      for (int u = blockIdx.x; u < total && !abort_s; u += W) {
+        const Tile t = decode_unit<BM, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, E);
+        const uint32_t idesc = t.rows <= 64 ? (t.half ? kIdescHalf64 : kIdescFull64)
+                                            : (t.half ? kIdescHalf : kIdescFull);
         if (!mbar_wait_bounded(&tempty_bar[acc], acc_phase ^ 1u)) {
           set_error(args.ctl, MOE_DEVERR_TIMEOUT);
           abort_s = 1;
@@ -248,8 +348,8 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t adesc = make_sw128_desc(a_addr + kk * 32, 16, 1024);
-            const uint64_t bdesc = make_sw128_desc(b_addr + kk * 2048, 8192, 1024);
-            umma_bf16(d_tmem, adesc, bdesc, C::IDESC, (kb | kk) != 0 ? 1u : 0u);
+            const uint64_t bdesc = make_sw128_desc(b_addr + kk * 2048, kBoxBytes, 1024);
+            umma_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           issued_any = true;
           umma_commit(&empty_bar[stage]);
@@ -268,10 +368,9 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   } else {
     // epilogue warps 2..5: TMEM lane quarter = warp % 4
     const int q = warp & 3;
-    const int r_in_tile = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
+    for (int u = blockIdx.x; u < total; u += W) {
       // Lane 0 polls and decides for the whole warp, so the warp-wide
       // tcgen05.ld below always runs converged.
       int ok = 0;
@@ -283,43 +382,17 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         }
       }
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      const Tile t = decode_tile(tau, tile_start_s, seg_s, E, ntn, C::OUT_N);
+      const Tile t = decode_unit<BM, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, E);
       tc_fence_after();
-      const bool valid = r_in_tile < t.rows;
+      const bool m64 = t.rows <= 64;
+      const int r_in_tile = m64 ? q * 16 + lane : q * 32 + lane;
+      const bool valid = (!m64 || lane < 16) && r_in_tile < t.rows;
       __nv_bfloat16* orow = args.out + static_cast<size_t>(t.row0 + r_in_tile) * args.N + t.n0;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * NMMA;
-#pragma unroll 1
-      for (int c = 0; c < C::OUT_N; c += 32) {
-        uint32_t v[32];
-        uint32_t packed[16];
-        if (EPI == EPI_SWIGLU) {
-          uint32_t u[32];
-          tmem_ld_32x32b_x32(tbase + c, v);
-          tmem_ld_32x32b_x32(tbase + C::OUT_N + c, u);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float h0 = silu(__uint_as_float(v[2 * i])) * __uint_as_float(u[2 * i]);
-            const float h1 = silu(__uint_as_float(v[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
-            packed[i] = pack_bf16(h0, h1);
-          }
-        } else {
-          tmem_ld_32x32b_x32(tbase + c, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float a = __uint_as_float(v[2 * i]), b = __uint_as_float(v[2 * i + 1]);
-            if (EPI == EPI_GELU) { a = gelu_erf(a); b = gelu_erf(b); }
-            packed[i] = pack_bf16(a, b);
-          }
-        }
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-        }
-      }
+      if (t.half)
+        epilogue_row<EPI, C::OUT_N / 2>(tbase, valid, orow);
+      else
+        epilogue_row<EPI, C::OUT_N>(tbase, valid, orow);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty_bar[acc]);

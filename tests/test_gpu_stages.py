@@ -188,3 +188,35 @@ def test_gather_ffn_combine_entry_points():
     assert max_err_ratio(np32(y), y_ref) <= TOL_BF16_OUT
     out_ref = O.combine(np32(y), np32(w), pm_ref["slot_to_row"], T, k)
     assert max_err_ratio(np32(out), out_ref) <= 1e-2
+
+
+@pytest.mark.parametrize("act,d,F", [("swiglu", 256, 256), ("gelu", 256, 512), ("gelu", 384, 384),
+                                     ("swiglu", 512, 128)])
+def test_expert_ffn_segment_boundaries(act, d, F):
+    """Segment sizes on both sides of the 64-row (M = 64 MMA) and 128-row
+    tiles, empty experts, and slack rows past the last segment; the rows
+    outside every segment are never written."""
+    m = [0, 1, 63, 64, 65, 127, 128, 129, 192, 193, 255, 256, 257, 300, 0, 513]
+    E = len(m)
+    seg = np.concatenate([[0], np.cumsum(m)]).astype(np.int32)
+    R = int(seg[-1]) + 77
+    g = torch.Generator().manual_seed(d + F)
+    x = torch.randn(R, d, generator=g).to(torch.bfloat16)
+    w1 = (torch.randn(E, d, F, generator=g) * 0.05).to(torch.bfloat16)
+    w3 = (torch.randn(E, d, F, generator=g) * 0.05).to(torch.bfloat16) if act == "swiglu" else None
+    w2 = (torch.randn(E, F, d, generator=g) * 0.05).to(torch.bfloat16)
+    sentinel = -3.0
+    h = torch.full((R, F), sentinel, dtype=torch.bfloat16, device=DEV)
+    y = torch.full((R, d), sentinel, dtype=torch.bfloat16, device=DEV)
+    ws = new_ws(256)
+    code = abi.MOE_ACT_SWIGLU if act == "swiglu" else abi.MOE_ACT_GELU
+    abi.moe_expert_ffn(x.to(DEV), w1.to(DEV), None if w3 is None else w3.to(DEV), w2.to(DEV), code,
+                       R, d, F, E, torch.from_numpy(seg).to(DEV), h, y, ws)
+    torch.cuda.synchronize()
+    assert abi.moe_get_device_error(ws) == 0
+    xs = np32(x)
+    W1, W2 = ExpertWeights(w1), ExpertWeights(w2)
+    W3 = ExpertWeights(w3) if w3 is not None else None
+    y_ref = O.expert_ffn(xs[:seg[-1]], seg, W1, W3, W2, act)
+    assert max_err_ratio(np32(y)[:seg[-1]], y_ref) <= TOL_BF16_OUT
+    assert np.all(np32(y)[seg[-1]:] == sentinel) and np.all(np32(h)[seg[-1]:] == sentinel)
