@@ -364,28 +364,28 @@ def main():
         raise RuntimeError("device error word set during warm-up")
     v = layer.views(sh.T)
     kept = v["kept_counts"].cpu().tolist()
-    launches_per_step = (1 if (sh.E <= 8) else 2) + 1 + (1 if sum(kept) > 0 else 0) + 2 + 1
-
     def timed_region():
         barrier(world)
         torch.cuda.synchronize()
+        n0 = abi.moe_kernel_launches()
         for i in range(args.steps):
             evict_l2()
             layer.forward(x, out, aux, events=evs[i])
+        n1 = abi.moe_kernel_launches()
         torch.cuda.synchronize()
         barrier(world)
         per = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(6)] for i in range(args.steps)]
-        return per
+        return per, n1 - n0
 
     sampler = ClockSampler(list(range(world)) if rank == 0 else [])
     if rank == 0:
         sampler.start()
-    per = timed_region()
+    per, launches = timed_region()
     clocks = sampler.stop() if rank == 0 else {}
     if rank == 0 and ClockSampler.rejected(clocks):
         sampler = ClockSampler(list(range(world)))
         sampler.start()
-        per = timed_region()
+        per, launches = timed_region()
         clocks = sampler.stop()
         clocks["remeasured"] = True
     step_ms = [sum(p) for p in per]
@@ -464,7 +464,7 @@ def main():
         "data": "synthetic (seeded; random-init weights of the layer's shape)",
         "config": dict(workload_config(sh), parallelism=f"replicas x{world}" if world > 1 else "1 GPU"),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": launches,
         "clocks": clocks,
         "stages": roof,
         "aux_loss": float(aux.item()),

@@ -128,6 +128,12 @@ MOE_API const char* moe_status_string(moe_status_t status);
  * on `stream`. Needed once per workspace before its first use. */
 MOE_API moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Number of CUDA kernels this library has launched in this process so far
+ * (all devices, all streams, every entry point), counted on the host at each
+ * launch. Read it before and after a region to count that region's launches.
+ * Never fails; needs no device. */
+MOE_API uint64_t moe_kernel_launches(void);
+
 /* Read (synchronises `stream`) and optionally clear the device error word of
  * a workspace into *host_bits. Returns MOE_ERR_DEVICE if it was non-zero. */
 MOE_API moe_status_t moe_get_device_error(void* ws, moe_stream_t stream, uint32_t* host_bits,

@@ -61,6 +61,7 @@ class MoeViewsC(ctypes.Structure):
 _SIGS = {
     "moe_status_string": (ctypes.c_char_p, [c_int]),
     "moe_workspace_init": (c_int, [c_void_p, c_size_t, c_void_p]),
+    "moe_kernel_launches": (ctypes.c_uint64, []),
     "moe_get_device_error": (c_int, [c_void_p, c_void_p, ctypes.POINTER(c_uint32), c_int]),
     "moe_capacity": (c_int64, [c_double, c_int, c_int, c_int]),
     "moe_rows_max": (c_int64, [c_int, c_int, c_int, c_int64]),
@@ -133,6 +134,11 @@ def dtype_code(t: torch.dtype) -> int:
 
 def status_string(st: int) -> str:
     return _lib.moe_status_string(st).decode()
+
+
+def moe_kernel_launches() -> int:
+    """Kernels the library has launched so far in this process."""
+    return int(_lib.moe_kernel_launches())
 
 
 def moe_capacity(cf: float, T: int, k: int, E: int) -> int:

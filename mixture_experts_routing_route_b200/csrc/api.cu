@@ -2,10 +2,17 @@
 // layout, and the stage launches on the caller's stream. Nothing here
 // allocates device memory or synchronises, except moe_get_device_error.
 #include "common.cuh"
+#include <atomic>
 #include <climits>
 #include <cmath>
 
 namespace moe {
+
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+}  // namespace
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 int num_sms() {
   static int n = 0;
@@ -193,6 +200,8 @@ const char* moe_status_string(moe_status_t st) {
   }
   return "unknown status";
 }
+
+uint64_t moe_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream) {
   MOE_NEED(ws);

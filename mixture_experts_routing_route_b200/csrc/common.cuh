@@ -85,6 +85,9 @@ cudaError_t launch_combine(const void* y, const float* w, const int32_t* slot_to
 
 int num_sms();
 
+// Counts every kernel this library launches (moe_kernel_launches reads it).
+void note_launch();
+
 // 2-D bf16 TMA map over [rows, cols] row-major, box [box_rows, 64 cols], 128-byte swizzle.
 bool make_tma_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
                       uint32_t box_rows);

@@ -229,6 +229,7 @@ void launch_combine_t(const T* y, const float* w, const int32_t* s2r, int T_, in
     case 8: combine_gather<T, 8><<<grid, kCombineThreads, 0, s>>>(y, w, s2r, d, k, rows_max, out, ctl); break;
     default: combine_gather<T, 0><<<grid, kCombineThreads, 0, s>>>(y, w, s2r, d, k, rows_max, out, ctl); break;
   }
+  note_launch();
 }
 
 }  // namespace
@@ -243,6 +244,7 @@ cudaError_t launch_gather(const void* x, size_t elem, int T, int d, int k, const
   gather_bulk<<<num_sms(), kGatherWarps * 32, smem, s>>>(
       static_cast<const uint8_t*>(x), row_bytes, T, k, row_slot, seg, E, rows_max,
       static_cast<uint8_t*>(x_perm), ctl);
+  note_launch();
   return cudaGetLastError();
 }
 

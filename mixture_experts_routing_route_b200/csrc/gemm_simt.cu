@@ -113,6 +113,7 @@ void run_f32(const float* A, const float* B0, const float* B1, int64_t rows_max,
   const long long mt_bound = (rows_max + TM - 1) / TM + E;
   dim3 grid((N + TN - 1) / TN, static_cast<unsigned>(mt_bound));
   grouped_gemm_f32<EPI><<<grid, 256, 0, s>>>(A, B0, B1, seg, E, K, N, rows_max, C, ctl);
+  note_launch();
 }
 
 }  // namespace

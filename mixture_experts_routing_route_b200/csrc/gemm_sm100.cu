@@ -458,6 +458,7 @@ cudaError_t run_gemm(const void* A, const void* B0, const void* B1, int64_t rows
   auto kern = grouped_gemm_tc<EPI, NMMA>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM));
   kern<<<num_sms(), kThreads, C::SMEM, s>>>(ta, tb0, tb1, a);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -358,6 +358,7 @@ cudaError_t launch_permute_single(const int32_t* idx, int T, int k, int E, int64
   const long long c = cap < 0 ? LLONG_MAX : static_cast<long long>(cap);
   permute_kernel<<<1, kThreads, 0, s>>>(idx, T * k, E, mask, c, counts, bins, sorted_slot,
                                         slot_to_row, row_slot, drop, kept, seg, rank_scratch, ctl);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -383,6 +384,7 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int64_t cap,
                   (void*)&counts, (void*)&bins, (void*)&sorted_slot, (void*)&slot_to_row,
                   (void*)&row_slot, (void*)&drop, (void*)&kept, (void*)&seg, (void*)&cta_counts,
                   (void*)&ctl};
+  note_launch();
   return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(permute_grid_kernel), dim3(g),
                                      dim3(kGThreads), args, 0, s);
 }

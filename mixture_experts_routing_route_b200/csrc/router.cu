@@ -824,6 +824,7 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, moe_d
     kern<<<grid, kFusedThreads, smem, s>>>(static_cast<const float*>(x), static_cast<const float*>(wg),
                                            bias, T, d, E, k, idx, w, logits, probs, part_p, part_c,
                                            ldb, ctl);
+    note_launch();
     nblk = grid;
   } else {
     int KS = 1;
@@ -846,10 +847,12 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, moe_d
         cudaFuncSetAttribute(router_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(tp.smem));
         router_tc<true><<<grid, kTcThreads, tp.smem, s>>>(tx, tw, a);
+        note_launch();
       } else {
         cudaFuncSetAttribute(router_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(tp.smem));
         router_tc<false><<<grid, kTcThreads, tp.smem, s>>>(tx, tw, a);
+        note_launch();
       }
       KS = tp.KS;
     } else if (T > 0) {
@@ -862,6 +865,7 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, moe_d
         router_gemm_tiled<float><<<g1, 256, 0, s>>>(static_cast<const float*>(x),
                                                     static_cast<const float*>(wg), T, d, E,
                                                     logits_scratch);
+      note_launch();
     }
     const int g2 = std::max(1, (T + kSelectTokensPerBlock - 1) / kSelectTokensPerBlock);
     const int epl = (E + 31) / 32;
@@ -873,9 +877,11 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, moe_d
     else if (epl <= 4) MOE_SELECT(4);
     else MOE_SELECT(8);
 #undef MOE_SELECT
+    note_launch();
     nblk = g2;
   }
   aux_reduce<<<E, kAuxThreads, 0, s>>>(part_p, part_c, ldb, nblk, E, T, k, terms, aux, ctl);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -61,6 +61,7 @@ def _call_route(abi, **over):
 
 def test_argument_checks_return_before_launch(abi):
     # every case here fails a host check, so nothing is launched
+    n0 = abi.moe_kernel_launches()
     assert _call_route(abi, x=None) == 1                      # MOE_ERR_NULL
     assert _call_route(abi, k=9) == 2                         # k > 8
     assert _call_route(abi, E=4, k=5) == 2                    # k > E
@@ -75,6 +76,7 @@ def test_argument_checks_return_before_launch(abi):
     L2 = abi.MoeLayerC(4096, 8, 2, 128, abi.MOE_BF16, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, None, 16)
     assert abi._lib.moe_forward(ctypes.byref(L2), 16, 4, 16, None, 16, 1 << 40, None, None) == 1
     assert abi._lib.moe_permute(16, 4, 2, 0, -1, *([16] * 8), 16, 1 << 20, None) == 2
+    assert abi.moe_kernel_launches() == n0
 
 
 def test_status_strings(abi):
