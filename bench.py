@@ -257,6 +257,60 @@ def job_value(tokens_per_rank, steps, world, total_ms_max):
     return world * tokens_per_rank * steps / (total_ms_max * 1e-3)
 
 
+# ------------------------------------------------------------------ end to end
+def measure_e2e(layer, inp, sh, args, world, elem):
+    """Tokens/s through the host-buffer entry point, as a serving loop runs
+    it: each step copies its x from pinned host memory, runs the layer and
+    copies out and aux back; two streams and two buffer sets alternate, so
+    step i+1's copies and launches overlap step i's compute, and the host
+    reads step i's result (aux) before it reuses that step's buffers. The
+    timed region (CUDA events) runs from the first step's input copy to the
+    last step's result copy. No L2 flush is needed: every step streams the
+    experts' weights (several GB) through the 126 MB L2."""
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    xs = [inp.x.pin_memory(), inp.x.clone().pin_memory()]
+    outs = [torch.empty(sh.T, sh.d, dtype=inp.x.dtype).pin_memory() for _ in range(2)]
+    auxs = [torch.empty(1, dtype=torch.float32).pin_memory() for _ in range(2)]
+    done = [None, None]
+
+    def step(i):
+        j = i % 2
+        if done[j] is not None:
+            done[j].synchronize()
+            if not (auxs[j].item() >= 0.0):  # the host reads the step's result
+                raise RuntimeError("aux loss not produced")
+        layer.forward_host(xs[j], outs[j], auxs[j], stream=streams[j], slot=j)
+        ev = torch.cuda.Event()
+        ev.record(streams[j])
+        done[j] = ev
+
+    for i in range(max(2, args.warmup)):
+        step(i)
+    torch.cuda.synchronize()
+    done[:] = [None, None]
+    barrier(world)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(streams[0])
+    streams[1].wait_event(start)
+    for i in range(args.steps):
+        step(i)
+    for j in range(2):
+        if done[j] is not None:
+            streams[0].wait_event(done[j])
+    end.record(streams[0])
+    end.synchronize()
+    from mixture_experts_routing_route_b200 import _abi as abi
+    for j in range(2):
+        if abi.moe_get_device_error(layer.workspace(sh.T, host_io=True, slot=j)) != 0:
+            raise RuntimeError("device error word set during the end-to-end steps")
+    e_total = reduce_max(start.elapsed_time(end), world)
+    return {"value": job_value(sh.T, args.steps, world, e_total), "unit": UNIT,
+            "h2d_bytes_per_step": sh.T * sh.d * elem,
+            "d2h_bytes_per_step": sh.T * sh.d * elem + 4,
+            "api": "MoeLayer.forward_host -> moe_forward_host (pinned host x/out/aux; two "
+                   "streams alternate, copies of one step overlap the compute of the next)"}
+
+
 # ------------------------------------------------------------------ CPU oracle
 def oracle_sample_run(inp, tokens, w64):
     """One oracle forward over a sample of the workload's tokens."""
@@ -355,7 +409,11 @@ def main():
     def evict_l2():
         torch.sum(flush, dim=0, dtype=torch.int64, out=flush_sink[0])
     stream = torch.cuda.current_stream()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    # Timed steps record 4 events: before route, around the up projection (the
+    # roofline's kernel) and after combine; the other stage boundaries carry
+    # no event, so consecutive kernels overlap their launches as in use.
+    evs = [[torch.cuda.Event(enable_timing=True) if j in (0, 3, 4, 6) else None for j in range(7)]
+           for _ in range(args.steps)]
 
     for _ in range(max(3, args.warmup)):
         layer.forward(x, out, aux)
@@ -374,7 +432,8 @@ def main():
         n1 = abi.moe_kernel_launches()
         torch.cuda.synchronize()
         barrier(world)
-        per = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(6)] for i in range(args.steps)]
+        per = [(evs[i][0].elapsed_time(evs[i][6]), evs[i][3].elapsed_time(evs[i][4]))
+               for i in range(args.steps)]
         return per, n1 - n0
 
     sampler = ClockSampler(list(range(world)) if rank == 0 else [])
@@ -388,12 +447,22 @@ def main():
         per, launches = timed_region()
         clocks = sampler.stop()
         clocks["remeasured"] = True
-    step_ms = [sum(p) for p in per]
+    step_ms = [p[0] for p in per]
     total_ms = reduce_max(sum(step_ms), world)
+    up_ms = statistics.mean(p[1] for p in per)
     if layer.device_error(sh.T) != 0:
         raise RuntimeError("device error word set during the timed steps")
 
-    stage_ms = {s: statistics.mean(p[j] for p in per) for j, s in enumerate(STAGES)}
+    # Stage breakdown: a separate, untimed pass with an event at every stage
+    # boundary (the events serialise the stages).
+    nb = min(args.steps, 20)
+    bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(nb)]
+    for i in range(nb):
+        evict_l2()
+        layer.forward(x, out, aux, events=bevs[i])
+    torch.cuda.synchronize()
+    stage_ms = {s: statistics.mean(bevs[i][j].elapsed_time(bevs[i][j + 1]) for i in range(nb))
+                for j, s in enumerate(STAGES)}
     alg = algorithmic(sh, kept)
     peaks = load_peaks()
     # A timed region long enough to hit the 1 kW power cap is compared with the
@@ -415,40 +484,20 @@ def main():
         roof[s] = r
 
     dom = "ffn_up"
-    tf = roof[dom]["TFLOP_s"]
+    tf = alg[dom]["flops"] / (up_ms * 1e-3) / 1e12 if up_ms > 0 else None
     traffic = measured_traffic("grouped_gemm_tc_swiglu", sh.name)
     roofline = {"kernel": "grouped_gemm_tc<SwiGLU> (expert up/gate projection)",
                 "bound": "tensor", "achieved": tf, "peak": tc_peak,
                 "unit": "TFLOP/s", "frac": tf / tc_peak if tf else None,
                 "traffic": traffic,
                 "peak_source": f"{peaks['source']} bf16 dense {tc_kind}",
-                "algorithmic_per_launch": f"2*R*d*2F = {alg[dom]['flops']:.4e} flop (R={sum(kept)} rows)"}
+                "algorithmic_per_launch": f"2*R*d*2F = {alg[dom]['flops']:.4e} flop (R={sum(kept)} rows)",
+                "launch_us": up_ms * 1e3,
+                "timing": "CUDA events on the launch stream around the up projection, every timed step"}
 
     e2e = None
     if not args.no_e2e:
-        x_host = inp.x.pin_memory()
-        out_host = torch.empty(sh.T, sh.d, dtype=x.dtype).pin_memory()
-        aux_host = torch.empty(1, dtype=torch.float32).pin_memory()
-        for _ in range(2):
-            layer.forward_host(x_host, out_host, aux_host)
-        torch.cuda.synchronize()
-        e_ms = []
-        barrier(world)
-        for i in range(args.steps):
-            evict_l2()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            layer.forward_host(x_host, out_host, aux_host)
-            b.record(stream)
-            b.synchronize()  # the host reads the result every step
-            e_ms.append(a.elapsed_time(b))
-        e_total = reduce_max(sum(e_ms), world)
-        elem = x.element_size()
-        e2e = {"value": job_value(sh.T, args.steps, world, e_total), "unit": UNIT,
-               "h2d_bytes_per_step": sh.T * sh.d * elem,
-               "d2h_bytes_per_step": sh.T * sh.d * elem + 4,
-               "api": "moe_forward_host (pinned host x/out, async copies on the stream)"}
+        e2e = measure_e2e(layer, inp, sh, args, world, x.element_size())
 
     if rank != 0:
         _finish(world)
@@ -467,6 +516,8 @@ def main():
         "gpu_launches": launches,
         "clocks": clocks,
         "stages": roof,
+        "stages_note": f"per-stage times from a separate pass of {nb} steps with an event at "
+                       f"every stage boundary (events serialise the stages)",
         "aux_loss": float(aux.item()),
         "rows": int(sum(kept)), "experts_active": int(sum(1 for c in kept if c > 0)),
         "imbalance_max_over_mean": (max(kept) / (sum(kept) / sh.E)) if sum(kept) else None,

@@ -39,6 +39,42 @@ template <> struct Elem<__nv_bfloat16> {
   static __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
 };
 
+// ------------------------------------------- programmatic dependent launch
+// Every kernel of the library is launched with programmatic stream
+// serialisation and starts with pdl_begin(): it waits there until the
+// previous kernel on the stream has finished and its writes are visible
+// (griddepcontrol.wait; a no-op when launched without the attribute), then
+// lets the next kernel be scheduled. The next kernel's launch and block
+// scheduling thus overlap this kernel's run instead of following its end.
+// A dependent grid is launched only after every block of this grid has
+// started, so its waiting blocks never hold resources this grid still needs.
+__device__ __forceinline__ void pdl_begin() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Counts every kernel this library launches (moe_kernel_launches reads it).
+void note_launch();
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       bool cooperative, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = cooperative ? 2 : 1;
+  note_launch();
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // ------------------------------------------------------------------ launchers
 // Router. Tokens per block of the general path (partials are per block).
 constexpr int kRouteSelectTokensPerBlock = 64;
@@ -84,9 +120,6 @@ cudaError_t launch_combine(const void* y, const float* w, const int32_t* slot_to
                            cudaStream_t s);
 
 int num_sms();
-
-// Counts every kernel this library launches (moe_kernel_launches reads it).
-void note_launch();
 
 // 2-D bf16 TMA map over [rows, cols] row-major, box [box_rows, 64 cols], 128-byte swizzle.
 bool make_tma_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,

@@ -26,6 +26,7 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
 gather_bulk(const uint8_t* __restrict__ x, uint32_t row_bytes, int T, int k,
             const int32_t* __restrict__ row_slot, const int32_t* __restrict__ seg, int E,
             long long rows_max, uint8_t* __restrict__ x_perm, Control* ctl) {
+  pdl_begin();
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t bars[kGatherWarps][kGatherBufs];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(kCombineThreads)
 combine_gather(const T* __restrict__ y, const float* __restrict__ w,
                const int32_t* __restrict__ slot_to_row, int d, int k_rt, long long rows_max,
                T* __restrict__ out, Control* ctl) {
+  pdl_begin();
   constexpr int V = CombineVec<T>::kVec;
   constexpr int NV = 2;  // column vectors per thread
   const int k = K > 0 ? K : k_rt;
@@ -218,18 +220,19 @@ combine_gather(const T* __restrict__ y, const float* __restrict__ w,
 }
 
 template <typename T>
-void launch_combine_t(const T* y, const float* w, const int32_t* s2r, int T_, int d, int k,
+cudaError_t launch_combine_t(const T* y, const float* w, const int32_t* s2r, int T_, int d, int k,
                       long long rows_max, T* out, Control* ctl, cudaStream_t s) {
   constexpr int V = CombineVec<T>::kVec;
   dim3 grid(T_, (d + kCombineThreads * V * 2 - 1) / (kCombineThreads * V * 2));
+  auto kern = combine_gather<T, 0>;
   switch (k) {
-    case 1: combine_gather<T, 1><<<grid, kCombineThreads, 0, s>>>(y, w, s2r, d, k, rows_max, out, ctl); break;
-    case 2: combine_gather<T, 2><<<grid, kCombineThreads, 0, s>>>(y, w, s2r, d, k, rows_max, out, ctl); break;
-    case 4: combine_gather<T, 4><<<grid, kCombineThreads, 0, s>>>(y, w, s2r, d, k, rows_max, out, ctl); break;
-    case 8: combine_gather<T, 8><<<grid, kCombineThreads, 0, s>>>(y, w, s2r, d, k, rows_max, out, ctl); break;
-    default: combine_gather<T, 0><<<grid, kCombineThreads, 0, s>>>(y, w, s2r, d, k, rows_max, out, ctl); break;
+    case 1: kern = combine_gather<T, 1>; break;
+    case 2: kern = combine_gather<T, 2>; break;
+    case 4: kern = combine_gather<T, 4>; break;
+    case 8: kern = combine_gather<T, 8>; break;
+    default: break;
   }
-  note_launch();
+  return launch_pdl(kern, grid, dim3(kCombineThreads), 0, s, false, y, w, s2r, d, k, rows_max, out, ctl);
 }
 
 }  // namespace
@@ -241,11 +244,9 @@ cudaError_t launch_gather(const void* x, size_t elem, int T, int d, int k, const
   const uint32_t row_bytes = static_cast<uint32_t>(static_cast<size_t>(d) * elem);
   const size_t smem = static_cast<size_t>(kGatherWarps) * kGatherBufs * kGatherPiece;
   cudaFuncSetAttribute(gather_bulk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  gather_bulk<<<num_sms(), kGatherWarps * 32, smem, s>>>(
-      static_cast<const uint8_t*>(x), row_bytes, T, k, row_slot, seg, E, rows_max,
-      static_cast<uint8_t*>(x_perm), ctl);
-  note_launch();
-  return cudaGetLastError();
+  return launch_pdl(gather_bulk, dim3(num_sms()), dim3(kGatherWarps * 32), smem, s, false,
+                    static_cast<const uint8_t*>(x), row_bytes, T, k, row_slot, seg, E, rows_max,
+                    static_cast<uint8_t*>(x_perm), ctl);
 }
 
 cudaError_t launch_combine(const void* y, const float* w, const int32_t* slot_to_row, size_t elem,
@@ -253,12 +254,10 @@ cudaError_t launch_combine(const void* y, const float* w, const int32_t* slot_to
                            cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   if (elem == 2)
-    launch_combine_t<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(y), w, slot_to_row, T, d, k,
-                                    rows_max, static_cast<__nv_bfloat16*>(out), ctl, s);
-  else
-    launch_combine_t<float>(static_cast<const float*>(y), w, slot_to_row, T, d, k, rows_max,
-                            static_cast<float*>(out), ctl, s);
-  return cudaGetLastError();
+    return launch_combine_t<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(y), w, slot_to_row, T,
+                                           d, k, rows_max, static_cast<__nv_bfloat16*>(out), ctl, s);
+  return launch_combine_t<float>(static_cast<const float*>(y), w, slot_to_row, T, d, k, rows_max,
+                                 static_cast<float*>(out), ctl, s);
 }
 
 }  // namespace moe

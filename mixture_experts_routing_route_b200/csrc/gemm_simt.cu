@@ -28,6 +28,7 @@ __global__ void __launch_bounds__(256)
 grouped_gemm_f32(const float* __restrict__ A, const float* __restrict__ B0,
                  const float* __restrict__ B1, const int32_t* __restrict__ seg, int E, int K, int N,
                  long long rows_max, float* __restrict__ Cout, Control* ctl) {
+  pdl_begin();
   __shared__ int mt_start[kMaxE + 1];
   __shared__ int seg_s[kMaxE + 1];
   __shared__ float As[TK][TM + 4];
@@ -108,12 +109,12 @@ grouped_gemm_f32(const float* __restrict__ A, const float* __restrict__ B0,
 }
 
 template <int EPI>
-void run_f32(const float* A, const float* B0, const float* B1, int64_t rows_max, int K, int N,
+cudaError_t run_f32(const float* A, const float* B0, const float* B1, int64_t rows_max, int K, int N,
              int E, const int32_t* seg, float* C, Control* ctl, cudaStream_t s) {
   const long long mt_bound = (rows_max + TM - 1) / TM + E;
   dim3 grid((N + TN - 1) / TN, static_cast<unsigned>(mt_bound));
-  grouped_gemm_f32<EPI><<<grid, 256, 0, s>>>(A, B0, B1, seg, E, K, N, rows_max, C, ctl);
-  note_launch();
+  return launch_pdl(grouped_gemm_f32<EPI>, grid, dim3(256), 0, s, false, A, B0, B1, seg, E, K, N,
+                    rows_max, C, ctl);
 }
 
 }  // namespace
@@ -122,15 +123,17 @@ cudaError_t launch_ffn_f32(const float* x_perm, const float* w1, const float* w3
                            moe_act_t act, int64_t rows_max, int d, int F, int E,
                            const int32_t* seg, float* h, float* y, Control* ctl, cudaStream_t s,
                            cudaEvent_t after_up) {
+  cudaError_t e = cudaSuccess;
   if (rows_max > 0) {
     if (act == MOE_ACT_SWIGLU)
-      run_f32<EPI_SWIGLU>(x_perm, w1, w3, rows_max, d, F, E, seg, h, ctl, s);
+      e = run_f32<EPI_SWIGLU>(x_perm, w1, w3, rows_max, d, F, E, seg, h, ctl, s);
     else
-      run_f32<EPI_GELU>(x_perm, w1, nullptr, rows_max, d, F, E, seg, h, ctl, s);
+      e = run_f32<EPI_GELU>(x_perm, w1, nullptr, rows_max, d, F, E, seg, h, ctl, s);
   }
+  if (e != cudaSuccess) return e;
   if (after_up) cudaEventRecord(after_up, s);
-  if (rows_max > 0) run_f32<EPI_STORE>(h, w2, nullptr, rows_max, F, d, E, seg, y, ctl, s);
-  return cudaGetLastError();
+  if (rows_max > 0) e = run_f32<EPI_STORE>(h, w2, nullptr, rows_max, F, d, E, seg, y, ctl, s);
+  return e;
 }
 
 }  // namespace moe

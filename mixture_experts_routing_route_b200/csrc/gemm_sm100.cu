@@ -236,6 +236,7 @@ template <int EPI, int NMMA>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                 const __grid_constant__ CUtensorMap tmB1, GemmArgs args) {
+  pdl_begin();
   using C = Cfg<EPI, NMMA>;
   // A half-width unit still loads whole 64-column boxes: gate and up halves
   // need at least one box each under SwiGLU.
@@ -457,9 +458,7 @@ cudaError_t run_gemm(const void* A, const void* B0, const void* B1, int64_t rows
   a.ctl = ctl;
   auto kern = grouped_gemm_tc<EPI, NMMA>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM));
-  kern<<<num_sms(), kThreads, C::SMEM, s>>>(ta, tb0, tb1, a);
-  note_launch();
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(num_sms()), dim3(kThreads), C::SMEM, s, false, ta, tb0, tb1, a);
 }
 
 }  // namespace

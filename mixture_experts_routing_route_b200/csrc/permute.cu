@@ -45,6 +45,7 @@ permute_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_mask,
                int32_t* __restrict__ row_slot, uint8_t* __restrict__ drop,
                int32_t* __restrict__ kept, int32_t* __restrict__ seg, int32_t* __restrict__ rank_g,
                Control* ctl) {
+  pdl_begin();
   __shared__ int hist[32][kMaxE + 1];
   __shared__ int running[kMaxE];
   __shared__ int start_s[kMaxE];
@@ -212,6 +213,7 @@ permute_grid_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_
                     int32_t* __restrict__ slot_to_row, int32_t* __restrict__ row_slot,
                     uint8_t* __restrict__ drop, int32_t* __restrict__ kept,
                     int32_t* __restrict__ seg, int32_t* __restrict__ cta_counts, Control* ctl) {
+  pdl_begin();
   __shared__ int s_e[kGMaxChunk];
   __shared__ int s_rank[kGMaxChunk];
   __shared__ int hist[8][kMaxE + 1];
@@ -356,10 +358,9 @@ cudaError_t launch_permute_single(const int32_t* idx, int T, int k, int E, int64
                                   cudaStream_t s) {
   const unsigned mask = static_cast<unsigned>(key_mask_of(E));
   const long long c = cap < 0 ? LLONG_MAX : static_cast<long long>(cap);
-  permute_kernel<<<1, kThreads, 0, s>>>(idx, T * k, E, mask, c, counts, bins, sorted_slot,
-                                        slot_to_row, row_slot, drop, kept, seg, rank_scratch, ctl);
-  note_launch();
-  return cudaGetLastError();
+  return launch_pdl(permute_kernel, dim3(1), dim3(kThreads), 0, s, false, idx, T * k, E, mask, c,
+                    counts, bins, sorted_slot, slot_to_row, row_slot, drop, kept, seg, rank_scratch,
+                    ctl);
 }
 
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int64_t cap, int32_t* counts,
@@ -379,14 +380,9 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int64_t cap,
                                                    align_up(static_cast<size_t>(S) * 4));
   unsigned mask = static_cast<unsigned>(key_mask_of(E));
   long long c = cap < 0 ? LLONG_MAX : static_cast<long long>(cap);
-  int S_ = S, E_ = E, chunk_ = chunk;
-  void* args[] = {(void*)&idx, (void*)&S_, (void*)&E_, (void*)&mask, (void*)&c, (void*)&chunk_,
-                  (void*)&counts, (void*)&bins, (void*)&sorted_slot, (void*)&slot_to_row,
-                  (void*)&row_slot, (void*)&drop, (void*)&kept, (void*)&seg, (void*)&cta_counts,
-                  (void*)&ctl};
-  note_launch();
-  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(permute_grid_kernel), dim3(g),
-                                     dim3(kGThreads), args, 0, s);
+  return launch_pdl(permute_grid_kernel, dim3(g), dim3(kGThreads), 0, s, true, idx, S, E, mask, c,
+                    chunk, counts, bins, sorted_slot, slot_to_row, row_slot, drop, kept, seg,
+                    cta_counts, ctl);
 }
 
 }  // namespace moe

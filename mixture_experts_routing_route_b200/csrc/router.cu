@@ -54,6 +54,7 @@ constexpr int kAuxThreads = 256;
 __global__ void __launch_bounds__(kAuxThreads)
 aux_reduce(const float* __restrict__ part_p, const int32_t* __restrict__ part_c, int ldb, int nblk,
            int E, int T, int k, double* __restrict__ terms, float* __restrict__ aux, Control* ctl) {
+  pdl_begin();
   __shared__ double sp[kAuxThreads];
   __shared__ long long sc[kAuxThreads];
   __shared__ bool is_last;
@@ -146,6 +147,7 @@ router_fused_e8(const Tin* __restrict__ x, const Tin* __restrict__ wg, const flo
                 float* __restrict__ logits_out, float* __restrict__ probs_out,
                 float* __restrict__ part_p, int32_t* __restrict__ part_c, int ldb,
                 Control* ctl) {
+  pdl_begin();
   constexpr int V = VecTraits<Tin>::kVec;  // elements per 16-byte x load: 8 (bf16) or 4 (fp32)
   extern __shared__ __align__(16) uint8_t smem_raw[];
   __shared__ float slice_part[kFusedSlices][kFusedQuads][32];
@@ -364,6 +366,7 @@ template <typename Tin>
 __global__ void __launch_bounds__(256)
 router_gemm_tiled(const Tin* __restrict__ x, const Tin* __restrict__ wg, int T, int d, int E,
                   float* __restrict__ out) {
+  pdl_begin();
   __shared__ float xs[32][64 + 4];
   __shared__ float ws[32][64 + 4];
   const int t0 = blockIdx.x * 64, e0 = blockIdx.y * 64;
@@ -502,6 +505,7 @@ router_select(const float* __restrict__ logits_in, int KS, const float* __restri
               int E, int k, int32_t* __restrict__ idx_out, float* __restrict__ w_out,
               float* __restrict__ logits_out, float* __restrict__ probs_out,
               float* __restrict__ part_p, int32_t* __restrict__ part_c, int ldb, Control* ctl) {
+  pdl_begin();
   __shared__ float blk_p_w[kSelectWarps][256];
   __shared__ int32_t blk_c_w[kSelectWarps][256];
   __shared__ float tot_p[256];
@@ -568,12 +572,13 @@ router_select(const float* __restrict__ logits_in, int KS, const float* __restri
 // path) or, for E <= 32, transposed once into shared memory as a K-major
 // operand (the first ring stages are already loading meanwhile). The four
 // warps then copy their 32 accumulator rows to the fp32 partial buffer
-// logits[ks][t][e]; router_select adds the KS partials in ks order.
-constexpr int kTcStages = 4;
+// logits[ks][t][e]; router_select adds the KS partials in ks order. The ring
+// has as many stages (up to kTcStages) as shared memory holds.
+constexpr int kTcStages = 8;
 constexpr int kTcThreads = 128;
 
 struct RouterTcArgs {
-  int T, d, E, Epad, KS, dk;
+  int T, d, E, Epad, KS, dk, stages;
   const __nv_bfloat16* wg;  // [d, E] (staged path)
   float* partial;           // [KS][T][E]
   Control* ctl;
@@ -583,6 +588,7 @@ template <bool kTmaB>
 __global__ void __launch_bounds__(kTcThreads, 1)
 router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
           RouterTcArgs a) {
+  pdl_begin();
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kTcStages], empty_bar[kTcStages], done_bar;
   __shared__ uint32_t tmem_base_s;
@@ -594,8 +600,9 @@ router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
   const int nkb = a.dk / 64;
   const int b_boxes = kTmaB ? a.Epad / 64 : 0;
   const uint32_t a_bytes = 128 * 128, stage_bytes = a_bytes + b_boxes * 8192;
+  const int nst = a.stages;
   uint8_t* ring = smem;
-  uint8_t* wgt = smem + kTcStages * stage_bytes;  // staged Wg^T (E <= 32)
+  uint8_t* wgt = smem + nst * stage_bytes;  // staged Wg^T (E <= 32)
   const uint32_t wgt_kb_bytes = static_cast<uint32_t>(a.Epad) * 128;
   // Accumulator slots: k-block kb accumulates into TMEM columns
   // [(kb / G) * Epad, +Epad), G k-blocks per slot, as many slots as 512
@@ -608,7 +615,7 @@ router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
   while (tcols < static_cast<uint32_t>(nslot * a.Epad)) tcols <<= 1;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kTcStages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    for (int s = 0; s < nst; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
     mbar_init(&done_bar, 1);
     fence_mbar_init();
   }
@@ -622,7 +629,7 @@ router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
   const uint32_t tmem_base = tmem_base_s;
 
   // The first ring stages are free: start their loads before anything else.
-  const int pre = nkb < kTcStages ? nkb : kTcStages;
+  const int pre = nkb < nst ? nkb : nst;
   auto issue = [&](int kb, int st) {
     uint8_t* sa = ring + st * stage_bytes;
     const int kx = ks * a.dk + kb * 64;
@@ -665,12 +672,12 @@ router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
   bool ok = true;
   if (warp == 0 && lane == 0) {
     uint32_t phase = 1;  // the prologue filled round 0
-    int st = pre % kTcStages;
-    if (pre < kTcStages) phase = 0;
+    int st = pre % nst;
+    if (pre < nst) phase = 0;
     for (int kb = pre; kb < nkb; ++kb) {
       if (!mbar_wait_bounded(&empty_bar[st], phase ^ 1u)) { set_error(a.ctl, MOE_DEVERR_TIMEOUT); break; }
       issue(kb, st);
-      if (++st == kTcStages) { st = 0; phase ^= 1u; }
+      if (++st == nst) { st = 0; phase ^= 1u; }
     }
   } else if (warp == 1 && lane == 0) {
     const uint32_t idesc = make_idesc_bf16(128, a.Epad, !kTmaB);
@@ -689,7 +696,7 @@ router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
       }
       issued = true;
       umma_commit(&empty_bar[st]);
-      if (++st == kTcStages) { st = 0; phase ^= 1u; }
+      if (++st == nst) { st = 0; phase ^= 1u; }
     }
     if (issued) umma_commit(&done_bar);
     else mbar_arrive(&done_bar);
@@ -753,13 +760,15 @@ size_t fused_smem_bytes(int d) { return static_cast<size_t>((d + 7) / 8) * 256; 
 
 // Tensor-core router plan: split factor KS (a power of two <= 8 dividing the
 // d/64 k-blocks) grows while the grid stays within the SMs; the staged Wg^T
-// of one CTA must fit in 128 KB.
+// of one CTA must fit in 128 KB; the ring takes what is left of 227 KB, up to
+// kTcStages stages.
 constexpr int kMaxKS = 8;
+constexpr int kTcFill = 1;  // grid of at most half the SMs (measured faster than filling them)
 
 struct TcPlan {
   bool use = false;
   bool tma_b = false;
-  int Epad = 0, KS = 1, ntile = 0;
+  int Epad = 0, KS = 1, ntile = 0, stages = 0;
   size_t smem = 0;
 };
 
@@ -777,13 +786,17 @@ TcPlan plan_tc(int T, int d, int E, moe_dtype_t dt) {
   p.ntile = (T + 127) / 128;
   const int nkb = d / 64;
   int ks = 1;
-  while (ks < kMaxKS && p.ntile * ks * 2 <= num_sms() && nkb % (ks * 2) == 0) ks *= 2;
+  while (ks < kMaxKS && p.ntile * ks * 2 <= num_sms() * kTcFill && nkb % (ks * 2) == 0) ks *= 2;
   if (!p.tma_b)
     while (static_cast<size_t>(d / ks) * p.Epad * 2 > 128 * 1024 && ks < kMaxKS && nkb % (ks * 2) == 0) ks *= 2;
   if (!p.tma_b && static_cast<size_t>(d / ks) * p.Epad * 2 > 128 * 1024) return p;
   p.KS = ks;
   const size_t stage = 128 * 128 + (p.tma_b ? static_cast<size_t>(p.Epad / 64) * 8192 : 0);
-  p.smem = 1024 + kTcStages * stage + (p.tma_b ? 0 : static_cast<size_t>(d / ks) * p.Epad * 2);
+  const size_t wgt = p.tma_b ? 0 : static_cast<size_t>(d / ks) * p.Epad * 2;
+  const size_t avail = 227 * 1024 - 1024 - wgt;
+  p.stages = static_cast<int>(std::min<size_t>(kTcStages, avail / stage));
+  if (p.stages < 2) return p;
+  p.smem = 1024 + p.stages * stage + wgt;
   p.use = true;
   return p;
 }
@@ -821,10 +834,11 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, moe_d
     const size_t smem = fused_smem_bytes(d);
     auto kern = router_fused_e8<float>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    kern<<<grid, kFusedThreads, smem, s>>>(static_cast<const float*>(x), static_cast<const float*>(wg),
-                                           bias, T, d, E, k, idx, w, logits, probs, part_p, part_c,
-                                           ldb, ctl);
-    note_launch();
+    const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kFusedThreads), smem, s, false,
+                                     static_cast<const float*>(x), static_cast<const float*>(wg),
+                                     bias, T, d, E, k, idx, w, logits, probs, part_p, part_c, ldb,
+                                     ctl);
+    if (e != cudaSuccess) return e;
     nblk = grid;
   } else {
     int KS = 1;
@@ -839,50 +853,44 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, moe_d
       }
       RouterTcArgs a;
       a.T = T; a.d = d; a.E = E; a.Epad = tp.Epad; a.KS = tp.KS; a.dk = d / tp.KS;
+      a.stages = tp.stages;
       a.wg = static_cast<const __nv_bfloat16*>(wg);
       a.partial = logits_scratch;
       a.ctl = ctl;
       const dim3 grid(tp.ntile * tp.KS);
-      if (tp.tma_b) {
-        cudaFuncSetAttribute(router_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(tp.smem));
-        router_tc<true><<<grid, kTcThreads, tp.smem, s>>>(tx, tw, a);
-        note_launch();
-      } else {
-        cudaFuncSetAttribute(router_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(tp.smem));
-        router_tc<false><<<grid, kTcThreads, tp.smem, s>>>(tx, tw, a);
-        note_launch();
-      }
+      auto kern = tp.tma_b ? router_tc<true> : router_tc<false>;
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(tp.smem));
+      const cudaError_t e = launch_pdl(kern, grid, dim3(kTcThreads), tp.smem, s, false, tx, tw, a);
+      if (e != cudaSuccess) return e;
       KS = tp.KS;
     } else if (T > 0) {
       dim3 g1((T + 63) / 64, (E + 63) / 64);
-      if (dt == MOE_BF16)
-        router_gemm_tiled<__nv_bfloat16><<<g1, 256, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(wg), T, d, E,
-            logits_scratch);
-      else
-        router_gemm_tiled<float><<<g1, 256, 0, s>>>(static_cast<const float*>(x),
-                                                    static_cast<const float*>(wg), T, d, E,
-                                                    logits_scratch);
-      note_launch();
+      const cudaError_t e =
+          dt == MOE_BF16
+              ? launch_pdl(router_gemm_tiled<__nv_bfloat16>, g1, dim3(256), 0, s, false,
+                           static_cast<const __nv_bfloat16*>(x),
+                           static_cast<const __nv_bfloat16*>(wg), T, d, E, logits_scratch)
+              : launch_pdl(router_gemm_tiled<float>, g1, dim3(256), 0, s, false,
+                           static_cast<const float*>(x), static_cast<const float*>(wg), T, d, E,
+                           logits_scratch);
+      if (e != cudaSuccess) return e;
     }
     const int g2 = std::max(1, (T + kSelectTokensPerBlock - 1) / kSelectTokensPerBlock);
     const int epl = (E + 31) / 32;
-#define MOE_SELECT(N)                                                                          \
-  router_select<N><<<g2, kSelectWarps * 32, 0, s>>>(logits_scratch, KS, bias, T, E, k, idx, w, \
-                                                    logits, probs, part_p, part_c, ldb, ctl)
-    if (epl <= 1) MOE_SELECT(1);
-    else if (epl <= 2) MOE_SELECT(2);
-    else if (epl <= 4) MOE_SELECT(4);
-    else MOE_SELECT(8);
-#undef MOE_SELECT
-    note_launch();
+    auto sel = epl <= 1 ? router_select<1>
+             : epl <= 2 ? router_select<2>
+             : epl <= 4 ? router_select<4>
+                        : router_select<8>;
+    const cudaError_t e = launch_pdl(sel, dim3(g2), dim3(kSelectWarps * 32), 0, s, false,
+                                     static_cast<const float*>(logits_scratch), KS, bias, T, E, k,
+                                     idx, w, logits, probs, part_p, part_c, ldb, ctl);
+    if (e != cudaSuccess) return e;
     nblk = g2;
   }
-  aux_reduce<<<E, kAuxThreads, 0, s>>>(part_p, part_c, ldb, nblk, E, T, k, terms, aux, ctl);
-  note_launch();
-  return cudaGetLastError();
+  return launch_pdl(aux_reduce, dim3(E), dim3(kAuxThreads), 0, s, false,
+                    static_cast<const float*>(part_p), static_cast<const int32_t*>(part_c), ldb,
+                    nblk, E, T, k, terms, aux, ctl);
 }
 
 }  // namespace moe

@@ -34,8 +34,10 @@ class MoeLayer:
                                   self.cf, self.w_router, self.bias, self.w1, self.w3, self.w2)
         self._ws = {}
 
-    def workspace(self, T: int, host_io: bool = False, stream=None) -> torch.Tensor:
-        key = (T, host_io)
+    def workspace(self, T: int, host_io: bool = False, stream=None, slot: int = 0) -> torch.Tensor:
+        """The device workspace for T tokens; `slot` keeps separate ones for
+        calls that may run at the same time on different streams."""
+        key = (T, host_io, slot)
         if key not in self._ws:
             n = (abi.moe_forward_host_workspace_size(self.c, T) if host_io
                  else abi.moe_forward_workspace_size(self.c, T))
@@ -58,9 +60,12 @@ class MoeLayer:
     __call__ = forward
 
     def forward_host(self, x_host: torch.Tensor, out_host: torch.Tensor, aux_host: torch.Tensor,
-                     stream=None):
+                     stream=None, slot: int = 0):
+        """Pinned host x in, pinned host out and aux back, all asynchronous on
+        `stream`. Calls that overlap (double-buffered serving on two streams)
+        pass different `slot`s so they use different workspaces."""
         T = x_host.shape[0]
-        ws = self.workspace(T, host_io=True, stream=stream)
+        ws = self.workspace(T, host_io=True, stream=stream, slot=slot)
         abi.moe_forward_host(self.c, x_host, T, out_host, aux_host, ws, stream)
 
     def device_error(self, T: int, stream=None) -> int:
