@@ -57,6 +57,9 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--gather-in-gemm", action="store_true",
+                   help="bf16: gather x rows inside the up projection (tile::gather4) instead of "
+                        "the gather kernel")
     p.add_argument("--T", type=int, default=None, help="override T (reduced case for profiling)")
     p.add_argument("--E", type=int, default=None, help="override E (reduced case for profiling)")
     p.add_argument("--F", type=int, default=None, help="override F (reduced case for profiling)")
@@ -88,9 +91,10 @@ def algorithmic(sh, counts_kept):
       route    bytes T*d*b + d*E*b + T*k*8 (x once, Wg once, idx + w out)
       permute  bytes S*4 + S*(4+4+4+1) (idx in; sorted_slot, slot_to_row,
                row_slot, drop out)
-      gather   bytes T_used*d*b + R*d*b (each token read once, rows written)
+      gather   bytes T_used*d*b + R*d*b (each token read once, rows written);
+               with --gather-in-gemm no separate stage
       ffn_up   flops 2*R*d*F*(2 SwiGLU | 1 GELU); bytes weights of active
-               experts + R*d*b + R*F*b
+               experts + R*d*b (A rows: x_perm, or x gathered) + R*F*b
       ffn_down flops 2*R*F*d; bytes E_act*F*d*b + R*F*b + R*d*b
       combine  bytes R*d*b + S*8 + T*d*b
     """
@@ -400,7 +404,7 @@ def main():
     layer = MoeLayer(inp.wg.to(dev), inp.w1.to(dev), inp.w2.to(dev),
                      w3=None if inp.w3 is None else inp.w3.to(dev),
                      bias=None if inp.bias is None else inp.bias.to(dev),
-                     k=sh.k, act=sh.act, capacity_factor=sh.cf)
+                     k=sh.k, act=sh.act, capacity_factor=sh.cf, gather_in_gemm=args.gather_in_gemm)
     out = torch.empty(sh.T, sh.d, dtype=x.dtype, device=dev)
     aux = torch.empty(1, dtype=torch.float32, device=dev)
     flush = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
@@ -476,6 +480,9 @@ def main():
     for s in STAGES:
         t = stage_ms[s] * 1e-3
         a = alg[s]
+        if s == "gather" and args.gather_in_gemm and sh.dtype == "bf16":
+            roof[s] = {"us": stage_ms[s] * 1e3, "fused_into": "ffn_up (tile::gather4 A loads)"}
+            continue
         r = {"us": stage_ms[s] * 1e3, "GB_s": a["bytes"] / t / 1e9 if t > 0 else None}
         r["hbm_frac"] = r["GB_s"] / peaks["hbm_gbs"] if r["GB_s"] else None
         if "flops" in a:
@@ -511,7 +518,8 @@ def main():
         "warmup": max(3, args.warmup), "ms_per_step": total_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": sh.dtype,
         "data": "synthetic (seeded; random-init weights of the layer's shape)",
-        "config": dict(workload_config(sh), parallelism=f"replicas x{world}" if world > 1 else "1 GPU"),
+        "config": dict(workload_config(sh), parallelism=f"replicas x{world}" if world > 1 else "1 GPU",
+                       **({"gather": "in the up projection (tile::gather4)"} if args.gather_in_gemm else {})),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks,

@@ -98,7 +98,15 @@ typedef struct {
   const void* w1;           /* W_gate (SwiGLU) or W1 (GELU), [E, d, F] */
   const void* w3;           /* W_up [E, d, F] (SwiGLU), NULL for GELU */
   const void* w2;           /* W_down / W2 [E, F, d] */
+  int flags;                /* MOE_LAYER_* bits, 0 for the default path */
 } moe_layer_t;
+
+/* moe_layer_t.flags. MOE_LAYER_GATHER_IN_GEMM (bf16 only): moe_forward skips
+ * the gather kernel and x_perm; the up projection loads its A rows straight
+ * from x with TMA tile::gather4 (row r = token row_slot[r] / k). Same results
+ * bit for bit; slower on every workload measured on B200 (each A tile is
+ * re-gathered for every output column block), so it is off by default. */
+#define MOE_LAYER_GATHER_IN_GEMM 1
 
 /* Device pointers into a moe_forward workspace where that call leaves its
  * intermediate results (see moe_forward_views). */
@@ -114,7 +122,7 @@ typedef struct {
   int32_t* slot_to_row;  /* [T * k] */
   int32_t* row_slot;     /* [rows_max] */
   uint8_t* drop_mask;    /* [T * k] */
-  void* x_perm;          /* [rows_max, d] */
+  void* x_perm;          /* [rows_max, d]; NULL with MOE_LAYER_GATHER_IN_GEMM */
   void* h;               /* [rows_max, F] */
   void* y_perm;          /* [rows_max, d] */
   int64_t rows_max;
@@ -256,7 +264,9 @@ MOE_API moe_status_t moe_combine(const void* y_perm, const float* topk_w, const 
 
 /* ---------------------------------------------------------------- forward
  * The whole layer on one stream with no host synchronisation: route ->
- * permute -> gather -> expert FFN (up, down) -> combine.
+ * permute -> gather -> expert FFN (up, down) -> combine. With
+ * MOE_LAYER_GATHER_IN_GEMM the gather is part of the up projection and the
+ * "gather" events bracket no work.
  *   x [T, d], out [T, d] (dtype); aux_loss out [1] fp32 device or NULL.
  *   events: NULL, or 7 cudaEvent_t recorded on `stream` before route and
  *   after route, permute, gather, up-projection, down-projection, combine.

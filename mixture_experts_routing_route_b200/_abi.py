@@ -23,6 +23,7 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_NULL", 2: "MOE_ERR_INVALID", 3: "MOE_ERR_UNSU
           4: "MOE_ERR_WORKSPACE", 5: "MOE_ERR_ALIGN", 6: "MOE_ERR_CUDA", 7: "MOE_ERR_DEVICE"}
 MOE_F32, MOE_BF16 = 0, 1
 MOE_ACT_GELU, MOE_ACT_SWIGLU = 0, 1
+MOE_LAYER_GATHER_IN_GEMM = 1
 DEVERR_EXPERT_RANGE, DEVERR_ROW_RANGE, DEVERR_TIMEOUT = 1, 2, 4
 
 
@@ -48,7 +49,8 @@ c_double, c_uint32 = ctypes.c_double, ctypes.c_uint32
 class MoeLayerC(ctypes.Structure):
     _fields_ = [("d", c_int), ("E", c_int), ("k", c_int), ("F", c_int), ("dtype", c_int),
                 ("act", c_int), ("capacity_factor", c_double), ("w_router", c_void_p),
-                ("router_bias", c_void_p), ("w1", c_void_p), ("w3", c_void_p), ("w2", c_void_p)]
+                ("router_bias", c_void_p), ("w1", c_void_p), ("w3", c_void_p), ("w2", c_void_p),
+                ("flags", c_int)]
 
 
 class MoeViewsC(ctypes.Structure):
@@ -213,9 +215,9 @@ def moe_combine(y_perm, topk_w, slot_to_row, T, d, k, rows_max, out, ws, stream=
         int(rows_max), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
 
 
-def layer_struct(d, E, k, F, dtype, act, cf, w_router, bias, w1, w3, w2) -> MoeLayerC:
+def layer_struct(d, E, k, F, dtype, act, cf, w_router, bias, w1, w3, w2, flags=0) -> MoeLayerC:
     return MoeLayerC(d, E, k, F, dtype, act, float(cf), _ptr(w_router), _ptr(bias), _ptr(w1),
-                     _ptr(w3), _ptr(w2))
+                     _ptr(w3), _ptr(w2), int(flags))
 
 
 def moe_forward_workspace_size(layer: MoeLayerC, T: int) -> int:

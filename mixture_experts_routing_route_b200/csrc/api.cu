@@ -94,6 +94,10 @@ struct FwdLayout {
   size_t bytes;
 };
 
+bool gather_in_gemm(const moe_layer_t* L) {
+  return L->dtype == MOE_BF16 && (L->flags & MOE_LAYER_GATHER_IN_GEMM) != 0;
+}
+
 FwdLayout fwd_layout(const moe_layer_t* L, int T, void* ws, bool host_io) {
   FwdLayout f{};
   Carver c(ws);
@@ -117,7 +121,9 @@ FwdLayout fwd_layout(const moe_layer_t* L, int T, void* ws, bool host_io) {
   f.row_slot = static_cast<int32_t*>(c.take(R * 4));
   f.drop = static_cast<uint8_t*>(c.take(S));
   f.rank = static_cast<int32_t*>(c.take(permute_scratch_bytes(T, L->k, L->E)));
-  f.x_perm = c.take(R * L->d * es);
+  // With MOE_LAYER_GATHER_IN_GEMM the up projection gathers the token rows
+  // itself and there is no x_perm.
+  f.x_perm = gather_in_gemm(L) ? nullptr : c.take(R * L->d * es);
   f.h = c.take(R * L->F * es);
   f.y_perm = c.take(R * L->d * es);
   if (host_io) {
@@ -134,6 +140,8 @@ moe_status_t check_layer(const moe_layer_t* L, int T) {
   MOE_CHECK(check_ffn(L->dtype, L->F));
   if (L->act != MOE_ACT_GELU && L->act != MOE_ACT_SWIGLU) return MOE_ERR_INVALID;
   if (!std::isfinite(L->capacity_factor)) return MOE_ERR_INVALID;
+  if ((L->flags & ~MOE_LAYER_GATHER_IN_GEMM) != 0) return MOE_ERR_INVALID;
+  if ((L->flags & MOE_LAYER_GATHER_IN_GEMM) && L->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   MOE_NEED(L->w_router);
   MOE_NEED(L->w1);
   MOE_NEED(L->w2);
@@ -157,20 +165,25 @@ moe_status_t run_forward(const moe_layer_t* L, const void* x, int T, void* out, 
                                      f.slot_to_row, f.row_slot, f.drop, f.kept, f.seg, f.rank,
                                      f.ctl, s)));
   rec(2);
-  MOE_CHECK(from_cuda(launch_gather(x, es, T, L->d, L->k, f.row_slot, f.seg, L->E, f.rows_max,
-                                    f.x_perm, f.ctl, s)));
+  if (!gather_in_gemm(L))
+    MOE_CHECK(from_cuda(launch_gather(x, es, T, L->d, L->k, f.row_slot, f.seg, L->E, f.rows_max,
+                                      f.x_perm, f.ctl, s)));
   rec(3);
   cudaEvent_t after_up = (ev != nullptr) ? reinterpret_cast<cudaEvent_t>(ev[4]) : nullptr;
-  if (L->dtype == MOE_BF16)
-    MOE_CHECK(from_cuda(launch_ffn_bf16(f.x_perm, L->w1, L->w3, L->w2, L->act, f.rows_max, L->d,
-                                        L->F, L->E, f.seg, f.h, f.y_perm, f.ctl, s, after_up)));
-  else
+  if (L->dtype == MOE_BF16) {
+    const bool g = gather_in_gemm(L);
+    MOE_CHECK(from_cuda(launch_ffn_bf16(g ? x : f.x_perm, g ? T : f.rows_max,
+                                        g ? f.row_slot : nullptr, L->k, L->w1, L->w3, L->w2,
+                                        L->act, f.rows_max, L->d, L->F, L->E, f.seg, f.h,
+                                        f.y_perm, f.ctl, s, after_up)));
+  } else {
     MOE_CHECK(from_cuda(launch_ffn_f32(static_cast<const float*>(f.x_perm),
                                        static_cast<const float*>(L->w1),
                                        static_cast<const float*>(L->w3),
                                        static_cast<const float*>(L->w2), L->act, f.rows_max, L->d,
                                        L->F, L->E, f.seg, static_cast<float*>(f.h),
                                        static_cast<float*>(f.y_perm), f.ctl, s, after_up)));
+  }
   rec(5);
   MOE_CHECK(from_cuda(launch_combine(f.y_perm, f.w, f.slot_to_row, es, T, L->d, L->k, f.rows_max,
                                      out, f.ctl, s)));
@@ -335,8 +348,8 @@ moe_status_t moe_expert_ffn(const void* x_perm, const void* w1, const void* w3, 
   Control* ctl = static_cast<Control*>(ws);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == MOE_BF16)
-    return from_cuda(launch_ffn_bf16(x_perm, w1, w3, w2, act, rows_max, d, F, E, seg_offsets, h,
-                                     y_perm, ctl, s, nullptr));
+    return from_cuda(launch_ffn_bf16(x_perm, rows_max, nullptr, 1, w1, w3, w2, act, rows_max, d, F,
+                                     E, seg_offsets, h, y_perm, ctl, s, nullptr));
   return from_cuda(launch_ffn_f32(static_cast<const float*>(x_perm), static_cast<const float*>(w1),
                                   static_cast<const float*>(w3), static_cast<const float*>(w2), act,
                                   rows_max, d, F, E, seg_offsets, static_cast<float*>(h),

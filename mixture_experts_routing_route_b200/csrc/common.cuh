@@ -104,11 +104,13 @@ cudaError_t launch_gather(const void* x, size_t elem, int T, int d, int k, const
                           const int32_t* seg, int E, int64_t rows_max, void* x_perm, Control* ctl,
                           cudaStream_t s);
 
-// Grouped GEMMs.
-cudaError_t launch_ffn_bf16(const void* x_perm, const void* w1, const void* w3, const void* w2,
-                            moe_act_t act, int64_t rows_max, int d, int F, int E,
-                            const int32_t* seg, void* h, void* y, Control* ctl, cudaStream_t s,
-                            cudaEvent_t after_up);
+// Grouped GEMMs. bf16: A is x_perm [rows_max, d] when row_slot is NULL, else
+// the token rows x [a_rows = T, d], gathered by the up projection itself
+// (row r reads token row_slot[r] / k).
+cudaError_t launch_ffn_bf16(const void* a, int64_t a_rows, const int32_t* row_slot, int k,
+                            const void* w1, const void* w3, const void* w2, moe_act_t act,
+                            int64_t rows_max, int d, int F, int E, const int32_t* seg, void* h,
+                            void* y, Control* ctl, cudaStream_t s, cudaEvent_t after_up);
 cudaError_t launch_ffn_f32(const float* x_perm, const float* w1, const float* w3, const float* w2,
                            moe_act_t act, int64_t rows_max, int d, int F, int E,
                            const int32_t* seg, float* h, float* y, Control* ctl, cudaStream_t s,

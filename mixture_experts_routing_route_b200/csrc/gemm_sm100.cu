@@ -45,8 +45,10 @@ constexpr int kBoxBytes = 64 * BK * 2;  // one 64-column B box: 8 KB
 enum { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_STORE = 2 };
 
 struct GemmArgs {
-  const int32_t* seg;  // [E+1] row segment offsets
-  __nv_bfloat16* out;  // [rows_max, N]
+  const int32_t* seg;       // [E+1] row segment offsets
+  __nv_bfloat16* out;       // [rows_max, N]
+  const int32_t* row_slot;  // gathering A: slot of each row (token = slot / k)
+  int k;
   int E;
   int K;
   int N;  // output columns
@@ -232,12 +234,18 @@ __device__ __forceinline__ void load_b_boxes(uint8_t* sb, const CUtensorMap* b0,
   }
 }
 
-template <int EPI, int NMMA>
+// GATHER: A is not a gathered copy but the token rows themselves: the
+// producer warp loads each stage's 128 A rows with 32 tile::gather4 loads
+// (lane l: rows 4l..4l+3, token row_slot[row] / k, one-row boxes), so the
+// up projection reads x directly and x_perm is never written. Rows past the
+// expert's segment load token 0 and are never stored.
+template <int EPI, int NMMA, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                 const __grid_constant__ CUtensorMap tmB1, GemmArgs args) {
   pdl_begin();
   using C = Cfg<EPI, NMMA>;
+  static_assert(!GATHER || EPI != EPI_STORE, "only the up projection gathers");
   // A half-width unit still loads whole 64-column boxes: gate and up halves
   // need at least one box each under SwiGLU.
   static_assert(EPI == EPI_SWIGLU ? NMMA >= 256 : NMMA >= 128, "half units need whole boxes");
@@ -277,7 +285,8 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   const int total = num_units(total_tiles, W);
   const int nkb = args.K / BK;
 
-  if (warp == 0) {
+  if (warp == 0 && !GATHER) {
+    // One thread waits for each ring slot, arms it and issues its loads.
     if (lane == 0) {
       prefetch_tmap(&tmA);
       prefetch_tmap(&tmB0);
@@ -313,6 +322,60 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       for (int s = 0; s < STAGES; ++s)
         if (issued_mask & (1u << s)) (void)mbar_wait_bounded(&full_bar[s], (last_parity >> s) & 1u);
     }
+  } else if (warp == 0) {
+    // GATHER: lane 0 waits for each ring slot and arms it, then the whole
+    // warp issues its 32 gather4 loads (lane 0 also the B boxes).
+    if (lane == 0) {
+      prefetch_tmap(&tmA);
+      prefetch_tmap(&tmB0);
+      prefetch_tmap(&tmB1);
+    }
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued_mask = 0;
+    uint32_t last_parity = 0;
+    bool go = true;
+    for (int u = blockIdx.x; u < total && go; u += W) {
+      const Tile t = decode_unit<BM, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, E);
+      const uint32_t tx = C::A_BYTES + (t.half ? C::B_BYTES / 2 : C::B_BYTES);
+      int tok[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = lane * 4 + i;
+        if (r < t.rows) tok[i] = __ldg(args.row_slot + t.row0 + r) / args.k;
+      }
+      for (int kb = 0; kb < nkb; ++kb) {
+        int ok = 0;
+        if (lane == 0) {
+          ok = !abort_s && mbar_wait_bounded(&empty_bar[stage], phase ^ 1u);
+          if (!ok && !abort_s) {
+            set_error(args.ctl, MOE_DEVERR_TIMEOUT);
+            abort_s = 1;
+          }
+          if (ok) mbar_arrive_expect_tx(&full_bar[stage], tx);
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+          go = false;
+          break;
+        }
+        uint8_t* sa = smem + stage * C::STAGE_BYTES;
+        uint8_t* sb = sa + C::A_BYTES;
+        tma_gather4(sa + lane * 512, &tmA, &full_bar[stage], kb * BK, tok[0], tok[1], tok[2], tok[3]);
+        if (lane == 0) {
+          const int brow = t.e * args.K + kb * BK;
+          if (t.half)
+            load_b_boxes<EPI, NMMA / 128>(sb, &tmB0, &tmB1, &full_bar[stage], t.n0, brow);
+          else
+            load_b_boxes<EPI, NMMA / 64>(sb, &tmB0, &tmB1, &full_bar[stage], t.n0, brow);
+        }
+        issued_mask |= 1u << stage;
+        last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (lane == 0)
+      for (int s = 0; s < STAGES; ++s)
+        if (issued_mask & (1u << s)) (void)mbar_wait_bounded(&full_bar[s], (last_parity >> s) & 1u);
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t kIdescFull = make_idesc_bf16(BM, NMMA);
@@ -440,50 +503,69 @@ bool make_tma_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t 
 
 namespace {
 
-template <int EPI, int NMMA>
-cudaError_t run_gemm(const void* A, const void* B0, const void* B1, int64_t rows_max, int K, int N,
-                     int E, const int32_t* seg, void* out, Control* ctl, cudaStream_t s) {
+// A: [a_rows, K] row-major; a_rows = rows_max, or T when gathering (then
+// row_slot / k pick each row's token).
+template <int EPI, int NMMA, bool GATHER>
+cudaError_t run_gemm(const void* A, int64_t a_rows, const int32_t* row_slot, int k, const void* B0,
+                     const void* B1, int64_t rows_max, int K, int N, int E, const int32_t* seg,
+                     void* out, Control* ctl, cudaStream_t s) {
   using C = Cfg<EPI, NMMA>;
   CUtensorMap ta, tb0, tb1;
-  if (!make_tma_2d_bf16(&ta, A, static_cast<uint64_t>(rows_max), K, BM)) return cudaErrorInvalidValue;
+  if (!make_tma_2d_bf16(&ta, A, static_cast<uint64_t>(a_rows), K, GATHER ? 1 : BM))
+    return cudaErrorInvalidValue;
   if (!make_tma_2d_bf16(&tb0, B0, static_cast<uint64_t>(E) * K, N, BK)) return cudaErrorInvalidValue;
   if (!make_tma_2d_bf16(&tb1, B1 ? B1 : B0, static_cast<uint64_t>(E) * K, N, BK)) return cudaErrorInvalidValue;
   GemmArgs a;
   a.seg = seg;
   a.out = static_cast<__nv_bfloat16*>(out);
+  a.row_slot = row_slot;
+  a.k = k;
   a.E = E;
   a.K = K;
   a.N = N;
   a.rows_max = rows_max;
   a.ctl = ctl;
-  auto kern = grouped_gemm_tc<EPI, NMMA>;
+  auto kern = grouped_gemm_tc<EPI, NMMA, GATHER>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM));
   return launch_pdl(kern, dim3(num_sms()), dim3(kThreads), C::SMEM, s, false, ta, tb0, tb1, a);
 }
 
+template <bool GATHER>
+cudaError_t run_up(const void* a, int64_t a_rows, const int32_t* row_slot, int k, const void* w1,
+                   const void* w3, moe_act_t act, int64_t rows_max, int d, int F, int E,
+                   const int32_t* seg, void* h, Control* ctl, cudaStream_t s) {
+  if (act == MOE_ACT_SWIGLU)
+    return run_gemm<EPI_SWIGLU, 256, GATHER>(a, a_rows, row_slot, k, w1, w3, rows_max, d, F, E, seg,
+                                             h, ctl, s);
+  if (F % 256 == 0)
+    return run_gemm<EPI_GELU, 256, GATHER>(a, a_rows, row_slot, k, w1, nullptr, rows_max, d, F, E,
+                                           seg, h, ctl, s);
+  return run_gemm<EPI_GELU, 128, GATHER>(a, a_rows, row_slot, k, w1, nullptr, rows_max, d, F, E, seg,
+                                         h, ctl, s);
+}
+
 }  // namespace
 
-cudaError_t launch_ffn_bf16(const void* x_perm, const void* w1, const void* w3, const void* w2,
-                            moe_act_t act, int64_t rows_max, int d, int F, int E,
-                            const int32_t* seg, void* h, void* y, Control* ctl, cudaStream_t s,
-                            cudaEvent_t after_up) {
+cudaError_t launch_ffn_bf16(const void* a, int64_t a_rows, const int32_t* row_slot, int k,
+                            const void* w1, const void* w3, const void* w2, moe_act_t act,
+                            int64_t rows_max, int d, int F, int E, const int32_t* seg, void* h,
+                            void* y, Control* ctl, cudaStream_t s, cudaEvent_t after_up) {
   if (rows_max <= 0) {
     if (after_up) cudaEventRecord(after_up, s);
     return cudaSuccess;
   }
-  cudaError_t err;
-  if (act == MOE_ACT_SWIGLU)
-    err = run_gemm<EPI_SWIGLU, 256>(x_perm, w1, w3, rows_max, d, F, E, seg, h, ctl, s);
-  else if (F % 256 == 0)
-    err = run_gemm<EPI_GELU, 256>(x_perm, w1, nullptr, rows_max, d, F, E, seg, h, ctl, s);
-  else
-    err = run_gemm<EPI_GELU, 128>(x_perm, w1, nullptr, rows_max, d, F, E, seg, h, ctl, s);
+  cudaError_t err =
+      row_slot != nullptr
+          ? run_up<true>(a, a_rows, row_slot, k, w1, w3, act, rows_max, d, F, E, seg, h, ctl, s)
+          : run_up<false>(a, rows_max, nullptr, 1, w1, w3, act, rows_max, d, F, E, seg, h, ctl, s);
   if (err != cudaSuccess) return err;
   if (after_up) cudaEventRecord(after_up, s);
   if (d % 256 == 0)
-    err = run_gemm<EPI_STORE, 256>(h, w2, nullptr, rows_max, F, d, E, seg, y, ctl, s);
+    err = run_gemm<EPI_STORE, 256, false>(h, rows_max, nullptr, 1, w2, nullptr, rows_max, F, d, E,
+                                          seg, y, ctl, s);
   else
-    err = run_gemm<EPI_STORE, 128>(h, w2, nullptr, rows_max, F, d, E, seg, y, ctl, s);
+    err = run_gemm<EPI_STORE, 128, false>(h, rows_max, nullptr, 1, w2, nullptr, rows_max, F, d, E,
+                                          seg, y, ctl, s);
   return err;
 }
 

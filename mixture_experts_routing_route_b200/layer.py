@@ -17,7 +17,8 @@ from . import _abi as abi
 class MoeLayer:
     def __init__(self, w_router: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
                  w3: Optional[torch.Tensor] = None, bias: Optional[torch.Tensor] = None,
-                 k: int = 2, act: str = "swiglu", capacity_factor: float = 0.0):
+                 k: int = 2, act: str = "swiglu", capacity_factor: float = 0.0,
+                 gather_in_gemm: bool = False):
         if not w1.is_cuda:
             raise ValueError("weights must be CUDA tensors")
         self.E, self.d, self.F = w1.shape
@@ -30,8 +31,12 @@ class MoeLayer:
         self.w3 = None if w3 is None else w3.contiguous()
         self.w2 = w2.contiguous()
         self.bias = None if bias is None else bias.to(device=w1.device, dtype=torch.float32).contiguous()
+        # gather_in_gemm: the up projection gathers x rows itself (bf16; see
+        # MOE_LAYER_GATHER_IN_GEMM in include/moe_b200.h)
+        flags = abi.MOE_LAYER_GATHER_IN_GEMM if gather_in_gemm else 0
         self.c = abi.layer_struct(self.d, self.E, k, self.F, abi.dtype_code(self.dtype), self.act,
-                                  self.cf, self.w_router, self.bias, self.w1, self.w3, self.w2)
+                                  self.cf, self.w_router, self.bias, self.w1, self.w3, self.w2,
+                                  flags)
         self._ws = {}
 
     def workspace(self, T: int, host_io: bool = False, stream=None, slot: int = 0) -> torch.Tensor:
@@ -96,7 +101,8 @@ class MoeLayer:
             "slot_to_row": view(v.slot_to_row, S, torch.int32, (S,)),
             "row_slot": view(v.row_slot, R, torch.int32, (R,)),
             "drop": view(v.drop_mask, S, torch.uint8, (S,)),
-            "x_perm": view(v.x_perm, R * self.d, self.dtype, (R, self.d)),
+            # no x_perm when the up projection gathers x rows itself
+            "x_perm": view(v.x_perm, R * self.d, self.dtype, (R, self.d)) if v.x_perm else None,
             "h": view(v.h, R * self.F, self.dtype, (R, self.F)),
             "y_perm": view(v.y_perm, R * self.d, self.dtype, (R, self.d)),
             "rows_max": R,

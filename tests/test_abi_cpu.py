@@ -47,6 +47,10 @@ def test_workspace_sizes_grow(abi):
     n = abi.moe_forward_workspace_size(L, 4096)
     # x_perm + h + y_perm alone: 8192 rows of (4096 + 14336 + 4096) bf16
     assert n >= 8192 * (4096 + 14336 + 4096) * 2
+    # gathering inside the up projection drops x_perm
+    Lg = abi.MoeLayerC(4096, 8, 2, 14336, abi.MOE_BF16, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, 16, 16,
+                       abi.MOE_LAYER_GATHER_IN_GEMM)
+    assert abi.moe_forward_workspace_size(Lg, 4096) == n - 8192 * 4096 * 2
     assert abi.moe_forward_host_workspace_size(L, 4096) >= n + 2 * 4096 * 4096 * 2
 
 

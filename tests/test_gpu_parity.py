@@ -78,9 +78,11 @@ def check_layer(inp, n_sample=None):
     R = pm["rows"]
     assert np.array_equal(npi(v["row_slot"])[:R], pm["row_slot"])
 
-    # ---- gather: bit-exact copy of rows
-    xp = np32(v["x_perm"])[:R]
-    assert np.array_equal(xp, O.gather(x, pm["row_slot"], k))
+    # ---- gather: bit-exact copy of rows (fp32 writes x_perm; bf16 gathers
+    # inside the up projection, checked through y below)
+    xp = O.gather(x, pm["row_slot"], k)
+    if v["x_perm"] is not None:
+        assert np.array_equal(np32(v["x_perm"])[:R], xp)
 
     # ---- expert FFN on the GPU's gathered rows
     w1, w2 = ExpertWeights(inp.w1), ExpertWeights(inp.w2)

@@ -220,3 +220,41 @@ def test_expert_ffn_segment_boundaries(act, d, F):
     y_ref = O.expert_ffn(xs[:seg[-1]], seg, W1, W3, W2, act)
     assert max_err_ratio(np32(y)[:seg[-1]], y_ref) <= TOL_BF16_OUT
     assert np.all(np32(y)[seg[-1]:] == sentinel) and np.all(np32(h)[seg[-1]:] == sentinel)
+
+
+@pytest.mark.parametrize("act,T,d,E,k,F,cf", [("swiglu", 700, 256, 8, 2, 512, 0.0),
+                                             ("gelu", 555, 384, 16, 2, 384, 1.0),
+                                             ("swiglu", 300, 256, 64, 8, 256, 0.0)])
+def test_fused_gather_equals_gather_then_ffn(act, T, d, E, k, F, cf):
+    """With MOE_LAYER_GATHER_IN_GEMM, moe_forward's up projection gathers x
+    rows itself (tile::gather4). Its h and y must equal, bit for bit,
+    moe_gather followed by moe_expert_ffn on the same permutation: the same
+    products in the same order, only the A rows' source differs."""
+    from mixture_experts_routing_route_b200 import MoeLayer
+    inp = small_case("fused", T=T, d=d, E=E, k=k, F=F, act=act, cf=cf, seed=T + d)
+    dv = {n: (None if t is None else t.to(DEV)) for n, t in
+          (("x", inp.x), ("wg", inp.wg), ("w1", inp.w1), ("w3", inp.w3), ("w2", inp.w2), ("bias", inp.bias))}
+    layer = MoeLayer(dv["wg"], dv["w1"], dv["w2"], w3=dv["w3"], bias=dv["bias"], k=k, act=act,
+                     capacity_factor=cf, gather_in_gemm=True)
+    out, _ = layer.forward(dv["x"])
+    plain = MoeLayer(dv["wg"], dv["w1"], dv["w2"], w3=dv["w3"], bias=dv["bias"], k=k, act=act,
+                     capacity_factor=cf)
+    out_plain, _ = plain.forward(dv["x"])
+    torch.cuda.synchronize()
+    assert layer.device_error(T) == 0
+    v = layer.views(T)
+    assert v["x_perm"] is None
+    R = int(v["seg_offsets"][-1].item())
+    Rm = v["rows_max"]
+    ws = new_ws(256)
+    x_perm = torch.empty(Rm, d, dtype=torch.bfloat16, device=DEV)
+    abi.moe_gather(dv["x"], T, d, k, v["row_slot"], v["seg_offsets"], E, Rm, x_perm, ws)
+    h = torch.empty(Rm, F, dtype=torch.bfloat16, device=DEV)
+    y = torch.empty(Rm, d, dtype=torch.bfloat16, device=DEV)
+    code = abi.MOE_ACT_SWIGLU if act == "swiglu" else abi.MOE_ACT_GELU
+    abi.moe_expert_ffn(x_perm, dv["w1"], dv["w3"], dv["w2"], code, Rm, d, F, E, v["seg_offsets"], h, y, ws)
+    torch.cuda.synchronize()
+    assert abi.moe_get_device_error(ws) == 0
+    assert torch.equal(h[:R], v["h"][:R])
+    assert torch.equal(y[:R], v["y_perm"][:R])
+    assert torch.equal(out, out_plain)
