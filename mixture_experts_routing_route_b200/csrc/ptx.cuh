@@ -221,6 +221,14 @@ __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
   return v;
 }
 
+// 16-byte load from distributed shared memory (addr 16-byte aligned).
+__device__ __forceinline__ float4 ld_shared_cluster_f32x4(uint32_t addr) {
+  float4 v;
+  asm("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+      : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
+
 // Shared-memory matrix descriptor (tcgen05 / UMMA), 128-byte swizzle.
 //   bits [0,14)  start address >> 4
 //   bits [16,30) leading-dimension byte offset >> 4

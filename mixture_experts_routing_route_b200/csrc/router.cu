@@ -580,11 +580,224 @@ constexpr int kTcThreads = 128;
 struct RouterTcArgs {
   int T, d, E, Epad, KS, dk, stages;
   const __nv_bfloat16* wg;  // [d, E] (staged path)
-  float* partial;           // [KS][T][E]
+  float* partial;           // [KS][T][E] (unfused)
   Control* ctl;
+  // fused selection (kFuseE != 0): the router's outputs and aux partials
+  const float* bias;
+  int k, ntile, ldb;
+  int32_t* idx;
+  float *w, *logits, *probs, *part_p, *aux;
+  int32_t* part_c;
 };
 
-template <bool kTmaB>
+// Fused selection, E <= 32. The KS CTAs of one 128-token tile run as a
+// cluster: CTA ks > 0 leaves its partial logits in its own shared memory and
+// the leader (ks = 0) adds them in ks order through distributed shared memory,
+// then the bias (the order router_select uses, so the logits are the same).
+// Leader thread r owns token tile*128 + r: softmax, k rounds of arg-max (ties
+// to the lower expert), renormalisation. The tile's aux partials
+// (probability sums and selection counts per expert) go to part[e][tile];
+// the last tile to finish (ticket) adds them in tile order and writes the
+// loss. EW (8, 16 or 32) is E rounded up: the per-token loops are that wide.
+constexpr int kFuseMaxE = 32;
+
+template <int EW>
+struct FuseCfg {
+  static constexpr int kStride = EW + 4;            // floats per shared row (16-byte aligned)
+  static constexpr int kParts = kTcThreads / EW;    // threads per expert in the reductions
+  static constexpr size_t kScratch = 2 * 128 * kStride * 4 + 128 * 4 + kTcThreads * 8;
+};
+
+// Thread r of each CTA: the sum over accumulator slots (in slot order) of
+// its row's columns, then the fused selection. Every thread of every CTA of
+// the cluster reaches both cluster barriers.
+template <int EW>
+__device__ __forceinline__ void fused_select_epilogue(const RouterTcArgs& a, uint32_t tmem_base,
+                                                      int nslot, int tile, int ks, bool ok,
+                                                      uint8_t* smem, int warp, int lane) {
+  using F = FuseCfg<EW>;
+  const int E = a.E;
+  const int r = warp * 32 + lane;
+  const int t = tile * 128 + r;
+  const uint32_t trow = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+  float v[EW];
+#pragma unroll
+  for (int h = 0; h < (EW + 15) / 16; ++h) {
+    float sum[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) sum[i] = 0.f;
+    for (int sl = 0; sl < nslot; ++sl) {
+      uint32_t u[16];
+      tmem_ld_32x32b_x16(trow + sl * a.Epad + h * 16, u);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) sum[i] += __uint_as_float(u[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (h * 16 + i < EW) v[h * 16 + i] = sum[i];
+  }
+  // The ring is idle (every MMA has completed): reuse it for row buffers.
+  float* red = reinterpret_cast<float*>(smem);                   // [128][kStride]
+  float* pm = red + 128 * F::kStride;                            // [128][kStride]
+  uint32_t* selm = reinterpret_cast<uint32_t*>(pm + 128 * F::kStride);  // [128]
+  float* part_ps = reinterpret_cast<float*>(selm + 128);         // [kTcThreads]
+  int* part_cs = reinterpret_cast<int*>(part_ps + kTcThreads);   // [kTcThreads]
+  __shared__ int last_s;
+  if (a.KS > 1) {
+    if (ks != 0) {
+#pragma unroll
+      for (int e = 0; e < EW; e += 4)
+        *reinterpret_cast<float4*>(red + r * F::kStride + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+    }
+    cluster_sync();
+    if (ks == 0) {
+      for (int src = 1; src < a.KS; ++src) {
+        const uint32_t base = mapa_shared(smem_u32(red + r * F::kStride), static_cast<uint32_t>(src));
+        float4 q[EW / 4];
+#pragma unroll
+        for (int e = 0; e < EW / 4; ++e) q[e] = ld_shared_cluster_f32x4(base + 16u * e);
+#pragma unroll
+        for (int e = 0; e < EW / 4; ++e) {
+          v[4 * e] += q[e].x;
+          v[4 * e + 1] += q[e].y;
+          v[4 * e + 2] += q[e].z;
+          v[4 * e + 3] += q[e].w;
+        }
+      }
+    }
+    cluster_sync();  // the other CTAs keep their buffers until the leader has read them
+  }
+  if (ks != 0) return;
+
+  const bool valid = ok && t < a.T;
+  float lg[EW], p[EW];
+  float m = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < EW; ++e) {
+    lg[e] = e < E ? v[e] + (a.bias != nullptr ? __ldg(a.bias + e) : 0.f) : -INFINITY;
+    m = fmaxf(m, lg[e]);
+  }
+  float ssum = 0.f;
+#pragma unroll
+  for (int e = 0; e < EW; ++e) {
+    p[e] = e < E ? expf(lg[e] - m) : 0.f;
+    ssum += p[e];
+  }
+#pragma unroll
+  for (int e = 0; e < EW; ++e) p[e] = p[e] / ssum;
+  if (valid) {
+#pragma unroll
+    for (int e = 0; e < EW; ++e) {
+      if (e < E && a.logits != nullptr) a.logits[static_cast<size_t>(t) * E + e] = lg[e];
+      if (e < E && a.probs != nullptr) a.probs[static_cast<size_t>(t) * E + e] = p[e];
+    }
+  }
+  uint32_t taken = 0;
+  int sel_e[8];
+  float sel_p[8];
+  float wsum = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    sel_e[j] = 0;
+    sel_p[j] = 0.f;
+    if (j < a.k) {
+      float bv = -INFINITY, bp = 0.f;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int e = 0; e < EW; ++e)
+        if (e < E && !((taken >> e) & 1u) && better(lg[e], e, bv, be)) { bv = lg[e]; be = e; bp = p[e]; }
+      if (be >= E) {  // no finite logit left
+        if (valid) set_error(a.ctl, MOE_DEVERR_EXPERT_RANGE);
+        be = 0;
+        bp = p[0];
+      }
+      taken |= 1u << be;
+      sel_e[j] = be;
+      sel_p[j] = bp;
+      wsum += bp;
+    }
+  }
+  if (valid) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (j < a.k) {
+        a.idx[static_cast<size_t>(t) * a.k + j] = sel_e[j];
+        a.w[static_cast<size_t>(t) * a.k + j] = sel_p[j] / wsum;
+      }
+  }
+  // ---- aux partials of this tile: thread (e, part) adds rows part, part +
+  // kParts, ... of expert e; then the kParts sums are added in part order.
+#pragma unroll
+  for (int e = 0; e < EW; ++e) pm[r * F::kStride + e] = valid ? p[e] : 0.f;
+  selm[r] = valid ? taken : 0u;
+  __syncthreads();
+  {
+    const int e = r % EW, part = r / EW;
+    float ps = 0.f;
+    int cs = 0;
+    for (int q = part; q < 128; q += F::kParts) {
+      ps += pm[q * F::kStride + e];
+      cs += (selm[q] >> e) & 1u;
+    }
+    part_ps[r] = ps;
+    part_cs[r] = cs;
+  }
+  __syncthreads();
+  if (r < E) {
+    float ps = 0.f;
+    int cs = 0;
+    for (int q = 0; q < F::kParts; ++q) {
+      ps += part_ps[q * EW + r];
+      cs += part_cs[q * EW + r];
+    }
+    a.part_p[static_cast<size_t>(r) * a.ldb + tile] = ps;
+    a.part_c[static_cast<size_t>(r) * a.ldb + tile] = cs;
+  }
+  __syncthreads();
+  if (r == 0) {
+    __threadfence();
+    last_s = atomicAdd(&a.ctl->route_ticket, 1u) == static_cast<unsigned>(a.ntile - 1);
+  }
+  __syncthreads();
+  if (!last_s) return;
+  __threadfence();
+  // ---- last tile: thread (e, part) adds tiles part, part + kParts, ... in
+  // float64, then thread e adds the kParts sums in part order.
+  double* dps = reinterpret_cast<double*>(red);              // [kTcThreads]
+  long long* dcs = reinterpret_cast<long long*>(dps + kTcThreads);  // [kTcThreads]
+  {
+    const int e = r % EW, part = r / EW;
+    double ps = 0.0;
+    long long cs = 0;
+    if (e < E)
+      for (int b = part; b < a.ntile; b += F::kParts) {
+        ps += static_cast<double>(__ldcg(a.part_p + static_cast<size_t>(e) * a.ldb + b));
+        cs += __ldcg(a.part_c + static_cast<size_t>(e) * a.ldb + b);
+      }
+    dps[r] = ps;
+    dcs[r] = cs;
+  }
+  __syncthreads();
+  if (r == 0) {
+    double tot = 0.0;
+    for (int e = 0; e < E; ++e) {
+      double ps = 0.0;
+      long long cs = 0;
+      for (int q = 0; q < F::kParts; ++q) {
+        ps += dps[q * EW + e];
+        cs += dcs[q * EW + e];
+      }
+      tot += (static_cast<double>(cs) / (static_cast<double>(a.T) * a.k)) * (ps / a.T);
+    }
+    *a.aux = static_cast<float>(E * tot);
+    a.ctl->route_ticket = 0u;
+  }
+}
+
+// kFuseE = 0: partial logits out (router_select follows); 8, 16 or 32: the
+// fused selection above with that width.
+template <bool kTmaB, int kFuseE>
 __global__ void __launch_bounds__(kTcThreads, 1)
 router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
           RouterTcArgs a) {
@@ -708,40 +921,44 @@ router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
     if (!d_ok) { if (lane == 0) set_error(a.ctl, MOE_DEVERR_TIMEOUT); ok = false; }
   }
   tc_fence_after();
-  // ---- accumulator rows -> partial logits [ks][t][e]
-  {
-    const int r = warp * 32 + lane;
-    const int t = tile * 128 + r;
-    float* dst = a.partial + static_cast<size_t>(ks) * a.T * a.E + static_cast<size_t>(t) * a.E;
-    const uint32_t trow = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
-    for (int c0 = 0; c0 < a.Epad; c0 += 16) {
-      float sum[16];
+  if constexpr (kFuseE == 0) {
+    // ---- accumulator rows -> partial logits [ks][t][e]
+    {
+      const int r = warp * 32 + lane;
+      const int t = tile * 128 + r;
+      float* dst = a.partial + static_cast<size_t>(ks) * a.T * a.E + static_cast<size_t>(t) * a.E;
+      const uint32_t trow = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+      for (int c0 = 0; c0 < a.Epad; c0 += 16) {
+        float sum[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) sum[i] = 0.f;
-      for (int sl = 0; sl < nslot; ++sl) {  // slot order
-        uint32_t u[16];
-        tmem_ld_32x32b_x16(trow + sl * a.Epad + c0, u);
-        tmem_ld_wait();
+        for (int i = 0; i < 16; ++i) sum[i] = 0.f;
+        for (int sl = 0; sl < nslot; ++sl) {  // slot order
+          uint32_t u[16];
+          tmem_ld_32x32b_x16(trow + sl * a.Epad + c0, u);
+          tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) sum[i] += __uint_as_float(u[i]);
-      }
-      uint32_t v[16];
+          for (int i = 0; i < 16; ++i) sum[i] += __uint_as_float(u[i]);
+        }
+        uint32_t v[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(sum[i]);
-      if (t < a.T && ok) {
-        if (c0 + 16 <= a.E) {
+        for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(sum[i]);
+        if (t < a.T && ok) {
+          if (c0 + 16 <= a.E) {
 #pragma unroll
-          for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4*>(dst + c0 + i) =
-                make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
-                            __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
-        } else {
+            for (int i = 0; i < 16; i += 4)
+              *reinterpret_cast<float4*>(dst + c0 + i) =
+                  make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                              __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+          } else {
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (c0 + i < a.E) dst[c0 + i] = __uint_as_float(v[i]);
+            for (int i = 0; i < 16; ++i)
+              if (c0 + i < a.E) dst[c0 + i] = __uint_as_float(v[i]);
+          }
         }
       }
     }
+  } else {
+    fused_select_epilogue<kFuseE>(a, tmem_base, nslot, tile, ks, ok, smem, warp, lane);
   }
   tc_fence_before();
   __syncthreads();
@@ -768,6 +985,7 @@ constexpr int kTcFill = 1;  // grid of at most half the SMs (measured faster tha
 struct TcPlan {
   bool use = false;
   bool tma_b = false;
+  int fuse_e = 0;  // 8, 16 or 32: router_tc<false, fuse_e> selects and reduces the aux loss too
   int Epad = 0, KS = 1, ntile = 0, stages = 0;
   size_t smem = 0;
 };
@@ -798,6 +1016,13 @@ TcPlan plan_tc(int T, int d, int E, moe_dtype_t dt) {
   if (p.stages < 2) return p;
   p.smem = 1024 + p.stages * stage + wgt;
   p.use = true;
+  // The fused selection reuses the ring for its row buffers.
+  if (!p.tma_b && E <= kFuseMaxE) {
+    const int ew = E <= 8 ? 8 : (E <= 16 ? 16 : 32);
+    const size_t scratch = ew == 8 ? FuseCfg<8>::kScratch
+                         : ew == 16 ? FuseCfg<16>::kScratch : FuseCfg<32>::kScratch;
+    if (p.stages * stage >= scratch) p.fuse_e = ew;
+  }
   return p;
 }
 
@@ -851,14 +1076,25 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, moe_d
       } else {
         tw = tx;  // unused by the staged path
       }
-      RouterTcArgs a;
+      RouterTcArgs a = {};
       a.T = T; a.d = d; a.E = E; a.Epad = tp.Epad; a.KS = tp.KS; a.dk = d / tp.KS;
       a.stages = tp.stages;
       a.wg = static_cast<const __nv_bfloat16*>(wg);
       a.partial = logits_scratch;
       a.ctl = ctl;
       const dim3 grid(tp.ntile * tp.KS);
-      auto kern = tp.tma_b ? router_tc<true> : router_tc<false>;
+      if (tp.fuse_e != 0) {
+        // one kernel: gate GEMM, cluster reduction over d, selection, aux loss
+        a.bias = bias; a.k = k; a.ntile = tp.ntile; a.ldb = ldb;
+        a.idx = idx; a.w = w; a.logits = logits; a.probs = probs;
+        a.part_p = part_p; a.part_c = part_c; a.aux = aux;
+        auto kern = tp.fuse_e == 8 ? router_tc<false, 8>
+                  : tp.fuse_e == 16 ? router_tc<false, 16> : router_tc<false, 32>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(tp.smem));
+        return launch_pdl_cluster(kern, grid, dim3(kTcThreads), tp.smem, s, tp.KS, tx, tw, a);
+      }
+      auto kern = tp.tma_b ? router_tc<true, 0> : router_tc<false, 0>;
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(tp.smem));
       const cudaError_t e = launch_pdl(kern, grid, dim3(kTcThreads), tp.smem, s, false, tx, tw, a);
