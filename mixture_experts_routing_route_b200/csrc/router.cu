@@ -841,7 +841,49 @@ router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_s;
 
-  // The first ring stages are free: start their loads before anything else.
+  // Wg^T for this CTA's d-range (staged path) as K-major 128-byte-swizzled
+  // rows: expert e, k-block kb -> row e of block kb, 16-byte chunk
+  // (kk/8) ^ (e%8). A task is 8 consecutive d-rows x 8 experts: eight 16-byte
+  // loads (one Wg row slice each), an 8x8 transpose of bf16 pairs with byte
+  // permutes, eight 16-byte stores (one expert's 8 k-values each). Tasks of
+  // the real experts come first; experts E..Epad-1 are zero. Each thread's
+  // first loads go out before the x tiles' TMA loads, so they do not queue
+  // behind them.
+  const int k0 = ks * a.dk;
+  const int nchunk = a.dk / 8, groups = a.E / 8;
+  const int ntask = kTmaB ? 0 : nchunk * (a.Epad / 8);
+  auto load_task = [&](int i, uint32_t (&in)[8][4]) {
+    const int g = i / nchunk, ch = i - g * nchunk;
+#pragma unroll
+    for (int rr = 0; rr < 8; ++rr) {
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (g < groups)
+        u = __ldg(reinterpret_cast<const uint4*>(a.wg + static_cast<size_t>(k0 + ch * 8 + rr) * a.E) + g);
+      in[rr][0] = u.x;
+      in[rr][1] = u.y;
+      in[rr][2] = u.z;
+      in[rr][3] = u.w;
+    }
+  };
+  auto store_task = [&](int i, const uint32_t (&in)[8][4]) {
+    const int g = i / nchunk, ch = i - g * nchunk;
+    const int kb = ch >> 3, c = ch & 7;
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const int e = g * 8 + jj;
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)  // k-values 2q (low half) and 2q+1 (high half)
+        o[q] = __byte_perm(in[2 * q][jj >> 1], in[2 * q + 1][jj >> 1], (jj & 1) ? 0x7632 : 0x5410);
+      const uint32_t off = kb * wgt_kb_bytes + e * 128 + (((c ^ e) & 7) << 4);
+      *reinterpret_cast<uint4*>(wgt + off) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  };
+  uint32_t in0[8][4];
+  const bool has0 = static_cast<int>(threadIdx.x) < ntask;
+  if (has0) load_task(threadIdx.x, in0);
+
+  // The first ring stages are free: start their loads now.
   const int pre = nkb < nst ? nkb : nst;
   auto issue = [&](int kb, int st) {
     uint8_t* sa = ring + st * stage_bytes;
@@ -856,27 +898,11 @@ router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
     for (int kb = 0; kb < pre; ++kb) issue(kb, kb);
   }
   if (!kTmaB) {
-    // Wg^T for this CTA's d-range as K-major 128-byte-swizzled rows: expert e,
-    // k-block kb -> row e of block kb, 16-byte chunk (kk/8) ^ (e%8). One Wg
-    // row (E % 8 == 0 experts) per group of 16-byte loads; experts E..Epad-1
-    // are zero.
-    const int k0 = ks * a.dk;
-    const int vecs = a.E / 8, vecs_pad = a.Epad / 8;
-#pragma unroll 4
-    for (int i = threadIdx.x; i < a.dk * vecs_pad; i += kTcThreads) {
-      const int kl = i / vecs_pad, vq = i - kl * vecs_pad;
-      uint4 u = make_uint4(0, 0, 0, 0);
-      if (vq < vecs)
-        u = __ldg(reinterpret_cast<const uint4*>(a.wg + static_cast<size_t>(k0 + kl) * a.E) + vq);
-      const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
-      const int kb = kl >> 6, kk = kl & 63;
-#pragma unroll
-      for (int h = 0; h < 8; ++h) {
-        const int e = vq * 8 + h;
-        const uint32_t off = kb * wgt_kb_bytes + e * 128 + ((((kk >> 3) ^ (e & 7)) & 7) << 4) + (kk & 7) * 2;
-        *reinterpret_cast<uint16_t*>(wgt + off) =
-            static_cast<uint16_t>((h & 1) ? (wv[h >> 1] >> 16) : (wv[h >> 1] & 0xffffu));
-      }
+    if (has0) store_task(threadIdx.x, in0);
+    for (int i = threadIdx.x + kTcThreads; i < ntask; i += kTcThreads) {
+      uint32_t in[8][4];
+      load_task(i, in);
+      store_task(i, in);
     }
     fence_proxy_async_smem();  // generic-proxy writes, read by the tensor core
     __syncthreads();
@@ -980,7 +1006,13 @@ size_t fused_smem_bytes(int d) { return static_cast<size_t>((d + 7) / 8) * 256; 
 // of one CTA must fit in 128 KB; the ring takes what is left of 227 KB, up to
 // kTcStages stages.
 constexpr int kMaxKS = 8;
-constexpr int kTcFill = 1;  // grid of at most half the SMs (measured faster than filling them)
+// Split over d: the grid may reach kTcFill x (SMs / 2) CTAs. The unfused
+// path keeps it at half the SMs (more splits cost router_select more partial
+// traffic than they save); the fused path, whose split is reduced on chip,
+// goes to two CTAs per SM with a 4-stage ring each (measured fastest).
+constexpr int kTcFill = 1;
+constexpr int kTcFillFused = 2;
+constexpr int kTcStagesFused = 4;
 
 struct TcPlan {
   bool use = false;
@@ -1003,8 +1035,10 @@ TcPlan plan_tc(int T, int d, int E, moe_dtype_t dt) {
   }
   p.ntile = (T + 127) / 128;
   const int nkb = d / 64;
+  const bool fusable = !p.tma_b && E <= kFuseMaxE;
+  const int fill = fusable ? kTcFillFused : kTcFill;
   int ks = 1;
-  while (ks < kMaxKS && p.ntile * ks * 2 <= num_sms() * kTcFill && nkb % (ks * 2) == 0) ks *= 2;
+  while (ks < kMaxKS && p.ntile * ks * 2 <= num_sms() * fill && nkb % (ks * 2) == 0) ks *= 2;
   if (!p.tma_b)
     while (static_cast<size_t>(d / ks) * p.Epad * 2 > 128 * 1024 && ks < kMaxKS && nkb % (ks * 2) == 0) ks *= 2;
   if (!p.tma_b && static_cast<size_t>(d / ks) * p.Epad * 2 > 128 * 1024) return p;
@@ -1012,12 +1046,12 @@ TcPlan plan_tc(int T, int d, int E, moe_dtype_t dt) {
   const size_t stage = 128 * 128 + (p.tma_b ? static_cast<size_t>(p.Epad / 64) * 8192 : 0);
   const size_t wgt = p.tma_b ? 0 : static_cast<size_t>(d / ks) * p.Epad * 2;
   const size_t avail = 227 * 1024 - 1024 - wgt;
-  p.stages = static_cast<int>(std::min<size_t>(kTcStages, avail / stage));
+  p.stages = static_cast<int>(std::min<size_t>(fusable ? kTcStagesFused : kTcStages, avail / stage));
   if (p.stages < 2) return p;
   p.smem = 1024 + p.stages * stage + wgt;
   p.use = true;
   // The fused selection reuses the ring for its row buffers.
-  if (!p.tma_b && E <= kFuseMaxE) {
+  if (fusable) {
     const int ew = E <= 8 ? 8 : (E <= 16 ? 16 : 32);
     const size_t scratch = ew == 8 ? FuseCfg<8>::kScratch
                          : ew == 16 ? FuseCfg<16>::kScratch : FuseCfg<32>::kScratch;
