@@ -22,7 +22,8 @@
 //            fp32 accumulator in tensor memory and frees ring slots /
 //            publishes accumulators with tcgen05.commit
 //   warps 2-5 epilogue: tcgen05.ld of their 32-lane quarter of the
-//            accumulator, activation, bf16 stores of valid rows only
+//            accumulator, activation, bf16 rows staged in shared memory and
+//            stored as whole 128-byte segments, valid rows only
 // Tiles are ordered expert-major, then N, with the M tile fastest, so CTAs
 // that run at the same time share one weight column block through L2; a
 // partial last wave is split into half-width tiles.
@@ -199,6 +200,66 @@ __device__ __forceinline__ void epilogue_row(uint32_t tbase, bool valid, __nv_bf
   }
 }
 
+// Epilogue of one warp through shared memory: for each 64-column group the
+// warp writes its rows (thread = row, 2 x 64 bytes) into a padded staging
+// buffer, then stores them back as whole 128-byte row segments, 8 lanes per
+// row, 4 rows per store instruction. Only rows [0, nrows) of the warp are
+// stored (rows past the expert's segment never are).
+constexpr bool kStagedStores = true;
+constexpr int kStageRow = 128 + 16;            // bytes per staged row (16 B pad: no bank conflicts)
+constexpr int kStageWarpBytes = 32 * kStageRow;
+
+template <int EPI, int OUTN>
+__device__ __forceinline__ void epilogue_staged(uint32_t tbase, uint8_t* buf, __nv_bfloat16* out,
+                                                long long row_base, int nrows, int N, int n0,
+                                                int lane) {
+#pragma unroll 1
+  for (int g = 0; g < OUTN; g += 64) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = g + 32 * h;
+      uint32_t v[32];
+      uint32_t packed[16];
+      if constexpr (EPI == EPI_SWIGLU) {
+        uint32_t u[32];
+        tmem_ld_32x32b_x32(tbase + c, v);
+        tmem_ld_32x32b_x32(tbase + OUTN + c, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float h0 = silu(__uint_as_float(v[2 * i])) * __uint_as_float(u[2 * i]);
+          const float h1 = silu(__uint_as_float(v[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+          packed[i] = pack_bf16(h0, h1);
+        }
+      } else {
+        tmem_ld_32x32b_x32(tbase + c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float a = __uint_as_float(v[2 * i]), b = __uint_as_float(v[2 * i + 1]);
+          if (EPI == EPI_GELU) { a = gelu_erf(a); b = gelu_erf(b); }
+          packed[i] = pack_bf16(a, b);
+        }
+      }
+      uint4* sp = reinterpret_cast<uint4*>(buf + lane * kStageRow + 64 * h);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        sp[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+    }
+    __syncwarp();
+    const int cq = lane & 7, rsub = lane >> 3;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int rr = it * 4 + rsub;
+      if (rr < nrows) {
+        const uint4 val = *reinterpret_cast<const uint4*>(buf + rr * kStageRow + cq * 16);
+        *reinterpret_cast<uint4*>(out + static_cast<size_t>(row_base + rr) * N + n0 + g + cq * 8) = val;
+      }
+    }
+    __syncwarp();
+  }
+}
+
 // ==================================================================== kernel
 // Tile 128 x NMMA per CTA, 4-stage ring of 48 KB (NMMA = 256). A tile with
 // at most 64 valid rows (an expert's last) runs as an M = 64 MMA: half the
@@ -214,7 +275,8 @@ struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int OUT_N = EPI == EPI_SWIGLU ? NMMA / 2 : NMMA;
   static constexpr int TMEM_COLS = 2 * NMMA;
-  static constexpr size_t SMEM = static_cast<size_t>(STAGES) * STAGE_BYTES + 1024;
+  static constexpr size_t STAGING = kStagedStores ? 4 * kStageWarpBytes : 0;
+  static constexpr size_t SMEM = static_cast<size_t>(STAGES) * STAGE_BYTES + STAGING + 1024;
 };
 
 // B boxes of one stage: SwiGLU puts NBOX/2 gate boxes then NBOX/2 up boxes
@@ -449,14 +511,24 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       const Tile t = decode_unit<BM, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, E);
       tc_fence_after();
       const bool m64 = t.rows <= 64;
-      const int r_in_tile = m64 ? q * 16 + lane : q * 32 + lane;
-      const bool valid = (!m64 || lane < 16) && r_in_tile < t.rows;
-      __nv_bfloat16* orow = args.out + static_cast<size_t>(t.row0 + r_in_tile) * args.N + t.n0;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * NMMA;
-      if (t.half)
-        epilogue_row<EPI, C::OUT_N / 2>(tbase, valid, orow);
-      else
-        epilogue_row<EPI, C::OUT_N>(tbase, valid, orow);
+      if constexpr (kStagedStores) {
+        uint8_t* buf = smem + STAGES * C::STAGE_BYTES + q * kStageWarpBytes;
+        const int wrow = m64 ? q * 16 : q * 32;
+        const int nrows = max(0, min(m64 ? 16 : 32, t.rows - wrow));
+        if (t.half)
+          epilogue_staged<EPI, C::OUT_N / 2>(tbase, buf, args.out, t.row0 + wrow, nrows, args.N, t.n0, lane);
+        else
+          epilogue_staged<EPI, C::OUT_N>(tbase, buf, args.out, t.row0 + wrow, nrows, args.N, t.n0, lane);
+      } else {
+        const int r_in_tile = m64 ? q * 16 + lane : q * 32 + lane;
+        const bool valid = (!m64 || lane < 16) && r_in_tile < t.rows;
+        __nv_bfloat16* orow = args.out + static_cast<size_t>(t.row0 + r_in_tile) * args.N + t.n0;
+        if (t.half)
+          epilogue_row<EPI, C::OUT_N / 2>(tbase, valid, orow);
+        else
+          epilogue_row<EPI, C::OUT_N>(tbase, valid, orow);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty_bar[acc]);
