@@ -236,6 +236,71 @@ def permute(idx, E, cap=None):
     }
 
 
+def permute_binned(idx, E, cap=None):
+    """The padded-binned layout of the pages' standard MoE path: expert e owns
+    the C rows [e*C, (e+1)*C) of an [E, C, hs] bucket; its slot of rank r (in
+    the stable expert order) sits in row e*C + r when r < C and is dropped
+    otherwise; rows past an expert's kept slots are padding (row_slot -1,
+    zero rows after the gather).
+
+    MegaBlocks page, sections 4.3 (binned_gather into [E, C, hs]), 4.4 (the
+    illustration's bucket[e, :len(rows)] = x[rows[:C]]), 4.5 (a short bin
+    keeps zeros; slots of rank >= C have no row: dropped), 4.6 (capacity 0:
+    C = the largest token count of the step, so nothing is dropped).
+
+    cap None means that dynamic capacity. Everything but the rows is the
+    permute() result for the same capacity; "bin" is C.
+    """
+    idx = np.asarray(idx, dtype=np.int64)
+    dense = permute(idx, E, cap)
+    counts = dense["counts"].astype(np.int64)
+    C = int(counts.max()) if cap is None else int(cap)
+    flat = idx.reshape(-1)
+    rank = dense["rank"].astype(np.int64)
+    drop = dense["drop"].astype(bool)
+    kept = np.minimum(counts, C)
+    seg_offsets = np.arange(E + 1, dtype=np.int64) * C
+    slot_to_row = np.where(drop, -1, flat * C + rank)
+    row_slot = np.full(E * C, -1, dtype=np.int64)
+    keep = ~drop
+    row_slot[slot_to_row[keep]] = np.nonzero(keep)[0]
+    out = dict(dense)
+    out.update({
+        "kept_counts": kept.astype(np.int32),
+        "seg_offsets": seg_offsets.astype(np.int32),
+        "slot_to_row": slot_to_row.astype(np.int32),
+        "row_slot": row_slot.astype(np.int32),
+        "rows": E * C,
+        "bin": C,
+    })
+    return out
+
+
+def gather_binned(x, row_slot, k):
+    """Bucket rows: x[row_slot[r] // k], or zeros where row_slot[r] < 0
+    (padding; MegaBlocks page, section 4.5)."""
+    x = np.asarray(x)
+    rs = np.asarray(row_slot, dtype=np.int64)
+    out = np.zeros((len(rs),) + x.shape[1:], dtype=x.dtype)
+    live = rs >= 0
+    out[live] = x[rs[live] // k]
+    return out
+
+
+def expert_ffn_binned(x_perm, kept_counts, bin_rows, w1, w3, w2, act):
+    """The expert MLP of each bin's kept rows; padding rows stay zero (an
+    expert applied to a zero row gives zero for both activations here, so
+    this equals running it over the whole bucket, as the pages' bmm does)."""
+    kept = np.asarray(kept_counts, dtype=np.int64)
+    E = len(kept)
+    y = np.zeros((E * bin_rows, np.asarray(w2[0]).shape[1]), dtype=np.float64)
+    for e in range(E):
+        a = e * bin_rows
+        if kept[e] > 0:
+            y[a:a + kept[e]] = _expert_mlp(x_perm[a:a + kept[e]], e, w1, w3, w2, act)
+    return y
+
+
 # --------------------------------------------------------------------------
 # gather / expert FFN / combine
 # --------------------------------------------------------------------------

@@ -350,3 +350,83 @@ def pin_bias(o):
 
 
 ALL_PINS.append(pin_bias)
+
+
+def pin_binned_example_a(o):
+    """The worked example in the [E, C, hs] bucket layout (MegaBlocks page,
+    sections 2 and 4.3-4.6), dynamic capacity and C = 2; padding rows of the
+    gathered bucket are zero."""
+    g = _golden("worked_example_a_binned.json")
+    ids = np.array(g["ids"]).reshape(-1, 1)
+    for c in g["cases"]:
+        b = o.permute_binned(ids, g["E"], c["capacity"])
+        assert b["bin"] == c["bin"]
+        for key in ("seg_offsets", "kept_counts", "slot_to_row", "row_slot", "drop"):
+            assert np.array_equal(np.asarray(b[key]), np.asarray(c[key])), (c["capacity"], key)
+        x = np.arange(1, 9, dtype=np.float64)[:, None] * np.ones((1, 3))
+        xb = o.gather_binned(x, b["row_slot"], 1)
+        assert np.array_equal(xb[:, 0], [0.0 if r < 0 else float(r + 1) for r in c["row_slot"]])
+
+
+def pin_binned_bruteforce(o):
+    """Tiny random routings: walking each expert's slots in ascending order,
+    the i-th lands in row e*C + i when i < C; C defaults to the largest count
+    (no drops)."""
+    rng = _rng(21)
+    for trial in range(60):
+        E = int(rng.integers(1, 6))
+        k = int(rng.integers(1, min(E, 3) + 1))
+        T = int(rng.integers(1, 9))
+        idx = np.array([rng.permutation(E)[:k] for _ in range(T)])
+        flat = idx.reshape(-1)
+        counts = [int(np.sum(flat == e)) for e in range(E)]
+        for cap in (None, 0, 1, 2, 5):
+            C = max(counts) if cap is None else cap
+            rows = [-1] * len(flat)
+            row_slot = [-1] * (E * C)
+            for e in range(E):
+                i = 0
+                for s in range(len(flat)):
+                    if flat[s] == e:
+                        if i < C:
+                            rows[s] = e * C + i
+                            row_slot[e * C + i] = s
+                        i += 1
+            b = o.permute_binned(idx, E, cap)
+            assert b["bin"] == C and b["rows"] == E * C
+            assert list(b["slot_to_row"]) == rows, (trial, cap)
+            assert list(b["row_slot"]) == row_slot, (trial, cap)
+            assert list(b["drop"]) == [1 if r < 0 else 0 for r in rows]
+            assert list(b["kept_counts"]) == [min(c, C) for c in counts]
+            assert list(b["seg_offsets"]) == [e * C for e in range(E + 1)]
+
+
+def pin_binned_forward_equals_dense(o):
+    """The bucket layout changes where rows live, not the layer: gathered,
+    expert MLP and combined output are the same as the dense layout's, for a
+    fixed capacity (same drops) and for capacity 0 (dynamic, nothing dropped,
+    equal to dropless)."""
+    rng = _rng(22)
+    T, d, E, k, F = 20, 6, 4, 2, 5
+    x = rng.standard_normal((T, d))
+    idx = np.array([rng.permutation(E)[:k] for _ in range(T)])
+    w = rng.random((T, k))
+    w1 = [rng.standard_normal((d, F)) for _ in range(E)]
+    w3 = [rng.standard_normal((d, F)) for _ in range(E)]
+    w2 = [rng.standard_normal((F, d)) for _ in range(E)]
+    for cap in (None, 3, 7):
+        dn = o.permute(idx, E, cap)
+        bn = o.permute_binned(idx, E, cap)
+        y_d = o.expert_ffn(o.gather(x, dn["row_slot"], k), dn["seg_offsets"], w1, w3, w2, "swiglu")
+        xb = o.gather_binned(x, bn["row_slot"], k)
+        y_b = o.expert_ffn_binned(xb, bn["kept_counts"], bn["bin"], w1, w3, w2, "swiglu")
+        keep = dn["slot_to_row"] >= 0
+        assert np.array_equal(y_d[dn["slot_to_row"][keep]], y_b[bn["slot_to_row"][keep]])
+        assert np.all(xb[bn["row_slot"] < 0] == 0) and np.all(y_b[bn["row_slot"] < 0] == 0)
+        out_d = o.combine(y_d, w, dn["slot_to_row"], T, k)
+        out_b = o.combine(y_b, w, bn["slot_to_row"], T, k)
+        assert np.array_equal(out_d, out_b), cap
+
+
+ALL_PINS.extend([pin_binned_example_a, pin_binned_bruteforce, pin_binned_forward_equals_dense])
+

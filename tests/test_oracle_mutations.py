@@ -70,7 +70,19 @@ def _permute_drop_gt(idx, E, cap=None):
     return r
 
 
-_REAL = {n: getattr(O, n) for n in ("combine", "expert_ffn", "permute")}
+def _binned_bin_is_mean(idx, E, cap=None):
+    if cap is None:
+        flat = np.asarray(idx).reshape(-1)
+        cap = int(math.ceil(len(flat) / E))
+    return _REAL["permute_binned"](idx, E, cap)
+
+
+def _binned_padding_repeats_row(x, row_slot, k):
+    x = np.asarray(x)
+    return x[np.abs(np.asarray(row_slot, np.int64)) // k]
+
+
+_REAL = {n: getattr(O, n) for n in ("combine", "expert_ffn", "permute", "permute_binned")}
 
 MUTATIONS = {
     "topk_ties_to_higher_index": ("topk_select", _ties_to_higher),
@@ -84,6 +96,8 @@ MUTATIONS = {
     "gather_wrong_token": ("gather", _gather_mod),
     "ffn_wrong_expert": ("expert_ffn", _ffn_wrong_expert),
     "drop_off_by_one": ("permute", _permute_drop_gt),
+    "binned_dynamic_bin_is_mean_count": ("permute_binned", _binned_bin_is_mean),
+    "binned_padding_not_zero": ("gather_binned", _binned_padding_repeats_row),
 }
 
 
