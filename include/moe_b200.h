@@ -107,6 +107,17 @@ typedef struct {
  * bit for bit; slower on every workload measured on B200 (each A tile is
  * re-gathered for every output column block), so it is off by default. */
 #define MOE_LAYER_GATHER_IN_GEMM 1
+/* MOE_LAYER_BINNED: the padded-binned [E, C, hs] layout of the pages'
+ * standard MoE path ("MegaBlocks", sections 4.3-4.6; see moe_permute_binned):
+ * expert e's rows are [e*C, e*C + kept_counts[e]) of a bucket of E*C rows
+ * (gathered padding rows are zero). capacity_factor > 0 fixes C =
+ * int(cf * k * T / E); capacity_factor <= 0 means dynamic capacity, C = the
+ * largest per-expert count of the call (nothing dropped), computed on the
+ * device, and the workspace is sized for the worst case C = T*k. The layer's
+ * output is the same as the default layout's; only the intermediates'
+ * layout differs. The expert FFN (bf16) skips the padding rows: h and y_perm
+ * rows past kept_counts[e] in each bin are not written. */
+#define MOE_LAYER_BINNED 2
 
 /* Device pointers into a moe_forward workspace where that call leaves its
  * intermediate results (see moe_forward_views). */
@@ -199,6 +210,27 @@ MOE_API moe_status_t moe_permute(const int32_t* topk_idx, int T, int k, int E, i
                          int32_t* slot_to_row, int32_t* row_slot, uint8_t* drop_mask,
                          int32_t* kept_counts, int32_t* seg_offsets, void* ws, size_t ws_bytes,
                          moe_stream_t stream);
+
+/* moe_permute into the padded-binned [E, C] layout ("MegaBlocks", sections
+ * 4.3 binned_gather into [E, C, hs], 4.5 short bins zero-padded and ranks >= C
+ * dropped, 4.6 capacity 0 = the largest per-expert count):
+ *   capacity     C >= 0, or negative for dynamic capacity: C = max(counts),
+ *                computed on the device (no slot dropped)
+ *   slot_to_row  out [T*k]  e*C + (rank of the slot within expert e), -1 if dropped
+ *   row_slot     out [moe_rows_max_binned(...)]  slot of each bucket row; -1
+ *                for padding rows; rows past seg_offsets[E] = E*C untouched
+ *   kept_counts  out [E]    min(counts, C)
+ *   seg_offsets  out [E+1]  e*C (so seg_offsets[1] is C)
+ * counts, bins, sorted_slot and drop_mask as moe_permute. */
+MOE_API moe_status_t moe_permute_binned(const int32_t* topk_idx, int T, int k, int E,
+                                int64_t capacity, int32_t* counts, int32_t* bins,
+                                int32_t* sorted_slot, int32_t* slot_to_row, int32_t* row_slot,
+                                uint8_t* drop_mask, int32_t* kept_counts, int32_t* seg_offsets,
+                                void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Rows of the binned bucket: E*C for capacity C >= 0, E*T*k (the worst case
+ * of dynamic capacity) for capacity < 0. */
+MOE_API int64_t moe_rows_max_binned(int T, int k, int E, int64_t capacity);
 
 /* --------------------------------------------------- permute, no allocation
  * The same permute for callers that cannot allocate device memory: code that

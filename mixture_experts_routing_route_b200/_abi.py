@@ -23,7 +23,7 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_NULL", 2: "MOE_ERR_INVALID", 3: "MOE_ERR_UNSU
           4: "MOE_ERR_WORKSPACE", 5: "MOE_ERR_ALIGN", 6: "MOE_ERR_CUDA", 7: "MOE_ERR_DEVICE"}
 MOE_F32, MOE_BF16 = 0, 1
 MOE_ACT_GELU, MOE_ACT_SWIGLU = 0, 1
-MOE_LAYER_GATHER_IN_GEMM = 1
+MOE_LAYER_GATHER_IN_GEMM, MOE_LAYER_BINNED = 1, 2
 DEVERR_EXPERT_RANGE, DEVERR_ROW_RANGE, DEVERR_TIMEOUT = 1, 2, 4
 
 
@@ -76,6 +76,9 @@ _SIGS = {
                     + [c_void_p, c_size_t, c_void_p]),
     "moe_permute_noalloc": (c_int, [c_void_p, c_int, c_int, c_int, c_int64] + [c_void_p] * 9
                             + [c_void_p]),
+    "moe_permute_binned": (c_int, [c_void_p, c_int, c_int, c_int, c_int64] + [c_void_p] * 8
+                           + [c_void_p, c_size_t, c_void_p]),
+    "moe_rows_max_binned": (c_int64, [c_int, c_int, c_int, c_int64]),
     "moe_gather": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_int,
                            c_int64, c_void_p, c_void_p, c_size_t, c_void_p]),
     "moe_expert_ffn": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int64,
@@ -151,6 +154,10 @@ def moe_rows_max(T: int, k: int, E: int, capacity: int) -> int:
     return _lib.moe_rows_max(T, k, E, capacity)
 
 
+def moe_rows_max_binned(T: int, k: int, E: int, capacity: int) -> int:
+    return _lib.moe_rows_max_binned(T, k, E, capacity)
+
+
 def moe_route_workspace_size(T, d, E) -> int:
     return _lib.moe_route_workspace_size(T, d, E)
 
@@ -182,6 +189,14 @@ def moe_route(x, w_router, bias, T, d, E, k, topk_idx, topk_w, aux_loss, logits,
 def moe_permute(topk_idx, T, k, E, capacity, counts, bins, sorted_slot, slot_to_row, row_slot,
                 drop_mask, kept_counts, seg_offsets, ws, stream=None):
     _check("moe_permute", _lib.moe_permute(
+        _ptr(topk_idx), T, k, E, int(capacity), _ptr(counts), _ptr(bins), _ptr(sorted_slot),
+        _ptr(slot_to_row), _ptr(row_slot), _ptr(drop_mask), _ptr(kept_counts), _ptr(seg_offsets),
+        _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_permute_binned(topk_idx, T, k, E, capacity, counts, bins, sorted_slot, slot_to_row,
+                       row_slot, drop_mask, kept_counts, seg_offsets, ws, stream=None):
+    _check("moe_permute_binned", _lib.moe_permute_binned(
         _ptr(topk_idx), T, k, E, int(capacity), _ptr(counts), _ptr(bins), _ptr(sorted_slot),
         _ptr(slot_to_row), _ptr(row_slot), _ptr(drop_mask), _ptr(kept_counts), _ptr(seg_offsets),
         _ptr(ws), ws.numel(), _stream(stream)))

@@ -94,6 +94,8 @@ struct FwdLayout {
   size_t bytes;
 };
 
+bool binned(const moe_layer_t* L) { return (L->flags & MOE_LAYER_BINNED) != 0; }
+
 bool gather_in_gemm(const moe_layer_t* L) {
   return L->dtype == MOE_BF16 && (L->flags & MOE_LAYER_GATHER_IN_GEMM) != 0;
 }
@@ -104,7 +106,8 @@ FwdLayout fwd_layout(const moe_layer_t* L, int T, void* ws, bool host_io) {
   const size_t S = static_cast<size_t>(T) * L->k;
   const size_t es = esize(L->dtype);
   f.cap = moe_capacity(L->capacity_factor, T, L->k, L->E);
-  f.rows_max = moe_rows_max(T, L->k, L->E, f.cap);
+  f.rows_max = binned(L) ? moe_rows_max_binned(T, L->k, L->E, f.cap)
+                         : moe_rows_max(T, L->k, L->E, f.cap);
   const size_t R = static_cast<size_t>(f.rows_max);
   f.ctl = static_cast<Control*>(c.take(sizeof(Control)));
   f.partials = c.take(route_partials_bytes(T, L->E));
@@ -140,7 +143,7 @@ moe_status_t check_layer(const moe_layer_t* L, int T) {
   MOE_CHECK(check_ffn(L->dtype, L->F));
   if (L->act != MOE_ACT_GELU && L->act != MOE_ACT_SWIGLU) return MOE_ERR_INVALID;
   if (!std::isfinite(L->capacity_factor)) return MOE_ERR_INVALID;
-  if ((L->flags & ~MOE_LAYER_GATHER_IN_GEMM) != 0) return MOE_ERR_INVALID;
+  if ((L->flags & ~(MOE_LAYER_GATHER_IN_GEMM | MOE_LAYER_BINNED)) != 0) return MOE_ERR_INVALID;
   if ((L->flags & MOE_LAYER_GATHER_IN_GEMM) && L->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   MOE_NEED(L->w_router);
   MOE_NEED(L->w1);
@@ -163,19 +166,20 @@ moe_status_t run_forward(const moe_layer_t* L, const void* x, int T, void* out, 
   rec(1);
   MOE_CHECK(from_cuda(launch_permute(f.idx, T, L->k, L->E, f.cap, f.counts, f.bins, f.sorted_slot,
                                      f.slot_to_row, f.row_slot, f.drop, f.kept, f.seg, f.rank,
-                                     f.ctl, s)));
+                                     f.ctl, s, binned(L))));
   rec(2);
   if (!gather_in_gemm(L))
     MOE_CHECK(from_cuda(launch_gather(x, es, T, L->d, L->k, f.row_slot, f.seg, L->E, f.rows_max,
-                                      f.x_perm, f.ctl, s)));
+                                      f.x_perm, f.ctl, s, binned(L))));
   rec(3);
   cudaEvent_t after_up = (ev != nullptr) ? reinterpret_cast<cudaEvent_t>(ev[4]) : nullptr;
   if (L->dtype == MOE_BF16) {
     const bool g = gather_in_gemm(L);
     MOE_CHECK(from_cuda(launch_ffn_bf16(g ? x : f.x_perm, g ? T : f.rows_max,
                                         g ? f.row_slot : nullptr, L->k, L->w1, L->w3, L->w2,
-                                        L->act, f.rows_max, L->d, L->F, L->E, f.seg, f.h,
-                                        f.y_perm, f.ctl, s, after_up)));
+                                        L->act, f.rows_max, L->d, L->F, L->E, f.seg,
+                                        binned(L) ? f.kept : nullptr, f.h, f.y_perm, f.ctl, s,
+                                        after_up)));
   } else {
     MOE_CHECK(from_cuda(launch_ffn_f32(static_cast<const float*>(f.x_perm),
                                        static_cast<const float*>(L->w1),
@@ -241,6 +245,11 @@ int64_t moe_capacity(double cf, int T, int k, int E) {
   return static_cast<int64_t>(c);  // truncation toward zero, as int() does
 }
 
+int64_t moe_rows_max_binned(int T, int k, int E, int64_t capacity) {
+  const int64_t S = static_cast<int64_t>(T) * k;
+  return static_cast<int64_t>(E) * (capacity < 0 ? S : capacity);
+}
+
 int64_t moe_rows_max(int T, int k, int E, int64_t capacity) {
   const int64_t S = static_cast<int64_t>(T) * k;
   if (capacity < 0) return S;
@@ -281,18 +290,21 @@ size_t moe_permute_workspace_size(int T, int k, int E) {
   return align_up(sizeof(Control)) + permute_scratch_bytes(T, k, E);
 }
 
-moe_status_t moe_permute(const int32_t* topk_idx, int T, int k, int E, int64_t capacity,
-                         int32_t* counts, int32_t* bins, int32_t* sorted_slot, int32_t* slot_to_row,
-                         int32_t* row_slot, uint8_t* drop_mask, int32_t* kept_counts,
-                         int32_t* seg_offsets, void* ws, size_t ws_bytes, moe_stream_t stream) {
+static moe_status_t permute_impl(const int32_t* topk_idx, int T, int k, int E, int64_t capacity,
+                                 int32_t* counts, int32_t* bins, int32_t* sorted_slot,
+                                 int32_t* slot_to_row, int32_t* row_slot, uint8_t* drop_mask,
+                                 int32_t* kept_counts, int32_t* seg_offsets, void* ws,
+                                 size_t ws_bytes, moe_stream_t stream, bool bin) {
   if (T < 0 || E < 1 || E > 256 || k < 1 || k > 8 || k > E) return MOE_ERR_INVALID;
   if (static_cast<long long>(T) * k >= INT_MAX) return MOE_ERR_INVALID;
+  const int64_t rows = bin ? moe_rows_max_binned(T, k, E, capacity) : moe_rows_max(T, k, E, capacity);
+  if (rows >= INT_MAX) return MOE_ERR_INVALID;
   if (T > 0) {
     MOE_NEED(topk_idx);
     MOE_NEED(sorted_slot);
     MOE_NEED(slot_to_row);
     MOE_NEED(drop_mask);
-    if (moe_rows_max(T, k, E, capacity) > 0) MOE_NEED(row_slot);
+    if (rows > 0) MOE_NEED(row_slot);
   }
   MOE_NEED(counts);
   MOE_NEED(bins);
@@ -305,7 +317,24 @@ moe_status_t moe_permute(const int32_t* topk_idx, int T, int k, int E, int64_t c
   int32_t* rank = static_cast<int32_t*>(c.take(permute_scratch_bytes(T, k, E)));
   return from_cuda(launch_permute(topk_idx, T, k, E, capacity, counts, bins, sorted_slot,
                                   slot_to_row, row_slot, drop_mask, kept_counts, seg_offsets, rank,
-                                  ctl, reinterpret_cast<cudaStream_t>(stream)));
+                                  ctl, reinterpret_cast<cudaStream_t>(stream), bin));
+}
+
+moe_status_t moe_permute(const int32_t* topk_idx, int T, int k, int E, int64_t capacity,
+                         int32_t* counts, int32_t* bins, int32_t* sorted_slot, int32_t* slot_to_row,
+                         int32_t* row_slot, uint8_t* drop_mask, int32_t* kept_counts,
+                         int32_t* seg_offsets, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  return permute_impl(topk_idx, T, k, E, capacity, counts, bins, sorted_slot, slot_to_row, row_slot,
+                      drop_mask, kept_counts, seg_offsets, ws, ws_bytes, stream, false);
+}
+
+moe_status_t moe_permute_binned(const int32_t* topk_idx, int T, int k, int E, int64_t capacity,
+                                int32_t* counts, int32_t* bins, int32_t* sorted_slot,
+                                int32_t* slot_to_row, int32_t* row_slot, uint8_t* drop_mask,
+                                int32_t* kept_counts, int32_t* seg_offsets, void* ws,
+                                size_t ws_bytes, moe_stream_t stream) {
+  return permute_impl(topk_idx, T, k, E, capacity, counts, bins, sorted_slot, slot_to_row, row_slot,
+                      drop_mask, kept_counts, seg_offsets, ws, ws_bytes, stream, true);
 }
 
 moe_status_t moe_gather(const void* x, moe_dtype_t dtype, int T, int d, int k,
@@ -349,7 +378,7 @@ moe_status_t moe_expert_ffn(const void* x_perm, const void* w1, const void* w3, 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == MOE_BF16)
     return from_cuda(launch_ffn_bf16(x_perm, rows_max, nullptr, 1, w1, w3, w2, act, rows_max, d, F,
-                                     E, seg_offsets, h, y_perm, ctl, s, nullptr));
+                                     E, seg_offsets, nullptr, h, y_perm, ctl, s, nullptr));
   return from_cuda(launch_ffn_f32(static_cast<const float*>(x_perm), static_cast<const float*>(w1),
                                   static_cast<const float*>(w3), static_cast<const float*>(w2), act,
                                   rows_max, d, F, E, seg_offsets, static_cast<float*>(h),

@@ -110,30 +110,35 @@ size_t route_logits_scratch_bytes(int T, int d, int E);
 
 // Permute. launch_permute picks the multi-CTA kernel when the slots fit its
 // per-CTA shared memory, else the single-CTA kernel; launch_permute_single
-// always runs the single-CTA kernel (needs only the rank scratch).
+// always runs the single-CTA kernel (needs only the rank scratch). binned:
+// the [E, C] bucket layout (row e*C + rank; C = cap, or the largest count
+// when cap < 0; padding rows get row_slot -1).
 size_t permute_scratch_bytes(int T, int k, int E);
 cudaError_t launch_permute_single(const int32_t* idx, int T, int k, int E, int64_t cap,
                                   int32_t* counts, int32_t* bins, int32_t* sorted_slot,
                                   int32_t* slot_to_row, int32_t* row_slot, uint8_t* drop,
                                   int32_t* kept, int32_t* seg, int32_t* rank_scratch, Control* ctl,
-                                  cudaStream_t s);
+                                  cudaStream_t s, bool binned = false);
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int64_t cap, int32_t* counts,
                            int32_t* bins, int32_t* sorted_slot, int32_t* slot_to_row,
                            int32_t* row_slot, uint8_t* drop, int32_t* kept, int32_t* seg,
-                           int32_t* rank_scratch, Control* ctl, cudaStream_t s);
+                           int32_t* rank_scratch, Control* ctl, cudaStream_t s,
+                           bool binned = false);
 
-// Gather.
+// Gather. binned: rows with row_slot -1 are padding and are written as zeros.
 cudaError_t launch_gather(const void* x, size_t elem, int T, int d, int k, const int32_t* row_slot,
                           const int32_t* seg, int E, int64_t rows_max, void* x_perm, Control* ctl,
-                          cudaStream_t s);
+                          cudaStream_t s, bool binned = false);
 
 // Grouped GEMMs. bf16: A is x_perm [rows_max, d] when row_slot is NULL, else
 // the token rows x [a_rows = T, d], gathered by the up projection itself
-// (row r reads token row_slot[r] / k).
+// (row r reads token row_slot[r] / k). Expert e's rows start at seg[e]; there
+// are kept[e] of them (binned layout), or seg[e + 1] - seg[e] when kept is NULL.
 cudaError_t launch_ffn_bf16(const void* a, int64_t a_rows, const int32_t* row_slot, int k,
                             const void* w1, const void* w3, const void* w2, moe_act_t act,
-                            int64_t rows_max, int d, int F, int E, const int32_t* seg, void* h,
-                            void* y, Control* ctl, cudaStream_t s, cudaEvent_t after_up);
+                            int64_t rows_max, int d, int F, int E, const int32_t* seg,
+                            const int32_t* kept, void* h, void* y, Control* ctl, cudaStream_t s,
+                            cudaEvent_t after_up);
 cudaError_t launch_ffn_f32(const float* x_perm, const float* w1, const float* w3, const float* w2,
                            moe_act_t act, int64_t rows_max, int d, int F, int E,
                            const int32_t* seg, float* h, float* y, Control* ctl, cudaStream_t s,

@@ -25,11 +25,19 @@ constexpr int kGatherPiece = 8192;  // bytes per buffer
 __global__ void __launch_bounds__(kGatherWarps * 32)
 gather_bulk(const uint8_t* __restrict__ x, uint32_t row_bytes, int T, int k,
             const int32_t* __restrict__ row_slot, const int32_t* __restrict__ seg, int E,
-            long long rows_max, uint8_t* __restrict__ x_perm, Control* ctl) {
+            long long rows_max, int binned, uint8_t* __restrict__ x_perm, Control* ctl) {
   pdl_begin();
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t bars[kGatherWarps][kGatherBufs];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // Binned layout: a padding row (row_slot -1) is stored from a zero piece.
+  uint8_t* zero = smem + static_cast<size_t>(kGatherWarps) * kGatherBufs * kGatherPiece;
+  if (binned) {
+    for (int i = threadIdx.x; i < kGatherPiece / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(zero)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();  // generic writes, read by the bulk stores
+  }
+  __syncthreads();
   if (lane != 0) return;
 
   long long R = __ldg(seg + E);
@@ -49,14 +57,20 @@ gather_bulk(const uint8_t* __restrict__ x, uint32_t row_bytes, int T, int k,
   for (int b = 0; b < kGatherBufs; ++b) mbar_init(&bars[warp][b], 1);
   fence_mbar_init();
 
-  // Source / destination / size of the i-th piece of this warp. A bad slot
-  // index is reported and the piece is skipped (size 0).
+  // Source / destination / size of the i-th piece of this warp. A padding
+  // row of the binned layout has no source (src null: stored from zero); any
+  // other bad slot index is reported and the piece is skipped (size 0).
   auto piece = [&](long long i, const uint8_t*& src, uint8_t*& dst, uint32_t& bytes) {
     const long long p = gw + i * tw;
     const long long row = p / ppr;
     const uint32_t off = static_cast<uint32_t>(p % ppr) * kGatherPiece;
     const int slot = __ldg(row_slot + row);
     bytes = min(static_cast<uint32_t>(kGatherPiece), row_bytes - off);
+    if (binned && slot == -1) {
+      src = nullptr;
+      dst = x_perm + static_cast<size_t>(row) * row_bytes + off;
+      return;
+    }
     if (slot < 0 || slot >= S) {
       set_error(ctl, MOE_DEVERR_ROW_RANGE);
       bytes = 0;
@@ -73,7 +87,7 @@ gather_bulk(const uint8_t* __restrict__ x, uint32_t row_bytes, int T, int k,
   const long long pro = mine < kGatherBufs ? mine : kGatherBufs;
   for (long long i = 0; i < pro; ++i) {
     piece(i, srcs[i], dsts[i], sizes[i]);
-    if (sizes[i]) {
+    if (sizes[i] && srcs[i]) {
       mbar_arrive_expect_tx(&bars[warp][i], sizes[i]);
       bulk_load(buf0 + i * kGatherPiece, srcs[i], sizes[i], &bars[warp][i]);
     }
@@ -81,7 +95,10 @@ gather_bulk(const uint8_t* __restrict__ x, uint32_t row_bytes, int T, int k,
   bool ok = true;
   for (long long i = 0; i < mine && ok; ++i) {
     const int b = static_cast<int>(i % kGatherBufs);
-    if (sizes[b]) {
+    if (sizes[b] && srcs[b] == nullptr) {
+      bulk_store(dsts[b], zero, sizes[b]);
+      bulk_commit();
+    } else if (sizes[b]) {
       if (!mbar_wait_bounded(&bars[warp][b], (phase >> b) & 1u)) {
         set_error(ctl, MOE_DEVERR_TIMEOUT);
         ok = false;
@@ -95,7 +112,7 @@ gather_bulk(const uint8_t* __restrict__ x, uint32_t row_bytes, int T, int k,
     if (nxt < mine) {
       bulk_wait_read<0>();  // the store above has finished reading buffer b
       piece(nxt, srcs[b], dsts[b], sizes[b]);
-      if (sizes[b]) {
+      if (sizes[b] && srcs[b]) {
         mbar_arrive_expect_tx(&bars[warp][b], sizes[b]);
         bulk_load(buf0 + b * kGatherPiece, srcs[b], sizes[b], &bars[warp][b]);
       }
@@ -239,14 +256,15 @@ cudaError_t launch_combine_t(const T* y, const float* w, const int32_t* s2r, int
 
 cudaError_t launch_gather(const void* x, size_t elem, int T, int d, int k, const int32_t* row_slot,
                           const int32_t* seg, int E, int64_t rows_max, void* x_perm, Control* ctl,
-                          cudaStream_t s) {
+                          cudaStream_t s, bool binned) {
   if (rows_max <= 0 || T <= 0) return cudaSuccess;
   const uint32_t row_bytes = static_cast<uint32_t>(static_cast<size_t>(d) * elem);
-  const size_t smem = static_cast<size_t>(kGatherWarps) * kGatherBufs * kGatherPiece;
+  // the ring of every warp, then one zero piece (binned padding rows)
+  const size_t smem = static_cast<size_t>(kGatherWarps) * kGatherBufs * kGatherPiece + kGatherPiece;
   cudaFuncSetAttribute(gather_bulk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   return launch_pdl(gather_bulk, dim3(num_sms()), dim3(kGatherWarps * 32), smem, s, false,
                     static_cast<const uint8_t*>(x), row_bytes, T, k, row_slot, seg, E, rows_max,
-                    static_cast<uint8_t*>(x_perm), ctl);
+                    binned ? 1 : 0, static_cast<uint8_t*>(x_perm), ctl);
 }
 
 cudaError_t launch_combine(const void* y, const float* w, const int32_t* slot_to_row, size_t elem,

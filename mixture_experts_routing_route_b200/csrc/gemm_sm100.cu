@@ -49,6 +49,8 @@ struct GemmArgs {
   const int32_t* seg;       // [E+1] row segment offsets
   __nv_bfloat16* out;       // [rows_max, N]
   const int32_t* row_slot;  // gathering A: slot of each row (token = slot / k)
+  const int32_t* kept;      // [E] rows of each expert from seg[e] (binned layout), or null:
+                            // seg[e + 1] - seg[e]
   int k;
   int E;
   int K;
@@ -68,13 +70,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 }
 
 // ------------------------------------------------------------------ schedule
-// Warp 0: copy the segment offsets, then tile_start[e] = exclusive prefix of
-// the per-expert unit counts ceil(m_e / TILE_M) * ntn; tile_start[E] = total.
-// Lane l owns experts [8l, 8l + 8). A segment whose rows are out of range is
-// reported and gets zero tiles.
+// Warp 0: tile_start[e] = exclusive prefix of the per-expert unit counts
+// ceil(m_e / TILE_M) * ntn (m_e = cnt[e] rows from seg[e]); tile_start[E] =
+// total. Lane l owns experts [8l, 8l + 8). A segment whose rows are out of
+// range is reported and gets zero tiles.
 template <int TILE_M>
 __device__ __forceinline__ void build_schedule(const GemmArgs& args, int ntn, const int* seg_s,
-                                               int* tile_start_s, int lane) {
+                                               const int* cnt_s, int* tile_start_s, int lane) {
   const int E = args.E;
   int loc[8];
   int sum = 0;
@@ -83,8 +85,9 @@ __device__ __forceinline__ void build_schedule(const GemmArgs& args, int ntn, co
     const int e = lane * 8 + i;
     int m = 0;
     if (e < E) {
-      m = seg_s[e + 1] - seg_s[e];
-      if (m < 0 || seg_s[e] < 0 || seg_s[e + 1] > args.rows_max) {
+      m = cnt_s[e];
+      if (m < 0 || seg_s[e] < 0 || static_cast<long long>(seg_s[e]) + m > args.rows_max ||
+          seg_s[e] + m > seg_s[e + 1]) {
         set_error(args.ctl, MOE_DEVERR_ROW_RANGE);
         m = 0;
       }
@@ -131,7 +134,7 @@ __device__ __forceinline__ int num_units(int total, int W) {
 
 template <int TILE_M, int OUT_N>
 __device__ __forceinline__ Tile decode_unit(int u, int total, int W, const int* tile_start,
-                                            const int* seg, int E) {
+                                            const int* seg, const int* cnt, int E) {
   int tau = u, half = -1;
   if (split_tail(total, W)) {
     const int r = total % W;
@@ -147,7 +150,7 @@ __device__ __forceinline__ Tile decode_unit(int u, int total, int W, const int* 
     if (tile_start[mid] <= tau) lo = mid; else hi = mid - 1;
   }
   const int e = lo;
-  const int m_e = seg[e + 1] - seg[e];
+  const int m_e = cnt[e];
   const int mt_e = (m_e + TILE_M - 1) / TILE_M;
   const int local = tau - tile_start[e];
   const int nt = local / mt_e, mt = local - nt * mt_e;
@@ -316,6 +319,7 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   __shared__ __align__(8) uint64_t tfull_bar[2], tempty_bar[2], drain_bar;
   __shared__ uint32_t tmem_base_s;
   __shared__ int seg_s[kMaxE + 1];
+  __shared__ int cnt_s[kMaxE];
   __shared__ int tile_start_s[kMaxE + 1];
   __shared__ volatile int abort_s;
 
@@ -324,10 +328,14 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
 
-  for (int i = threadIdx.x; i <= E; i += kThreads) seg_s[i] = __ldg(args.seg + i);
+  for (int i = threadIdx.x; i <= E; i += kThreads) {
+    seg_s[i] = __ldg(args.seg + i);
+    if (i < E)
+      cnt_s[i] = args.kept != nullptr ? __ldg(args.kept + i) : __ldg(args.seg + i + 1) - __ldg(args.seg + i);
+  }
   if (threadIdx.x == 0) abort_s = 0;
   __syncthreads();
-  if (warp == 0) build_schedule<BM>(args, args.N / C::OUT_N, seg_s, tile_start_s, lane);
+  if (warp == 0) build_schedule<BM>(args, args.N / C::OUT_N, seg_s, cnt_s, tile_start_s, lane);
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(&tfull_bar[b], 1); mbar_init(&tempty_bar[b], 4); }
@@ -358,7 +366,7 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       uint32_t issued_mask = 0;  // stages that ever received a load
       uint32_t last_parity = 0;  // parity of that stage's latest load
       for (int u = blockIdx.x; u < total && !abort_s; u += W) {
-        const Tile t = decode_unit<BM, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, E);
+        const Tile t = decode_unit<BM, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, cnt_s, E);
         const uint32_t tx = C::A_BYTES + (t.half ? C::B_BYTES / 2 : C::B_BYTES);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u)) {
@@ -398,7 +406,7 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     uint32_t last_parity = 0;
     bool go = true;
     for (int u = blockIdx.x; u < total && go; u += W) {
-      const Tile t = decode_unit<BM, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, E);
+      const Tile t = decode_unit<BM, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, cnt_s, E);
       const uint32_t tx = C::A_BYTES + (t.half ? C::B_BYTES / 2 : C::B_BYTES);
       int tok[4] = {0, 0, 0, 0};
 #pragma unroll
@@ -450,7 +458,7 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       uint32_t acc_phase = 0;
       bool issued_any = false;
       for (int u = blockIdx.x; u < total && !abort_s; u += W) {
-        const Tile t = decode_unit<BM, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, E);
+        const Tile t = decode_unit<BM, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, cnt_s, E);
         const uint32_t idesc = t.rows <= 64 ? (t.half ? kIdescHalf64 : kIdescFull64)
                                             : (t.half ? kIdescHalf : kIdescFull);
         if (!mbar_wait_bounded(&tempty_bar[acc], acc_phase ^ 1u)) {
@@ -508,7 +516,7 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         }
       }
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      const Tile t = decode_unit<BM, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, E);
+      const Tile t = decode_unit<BM, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, cnt_s, E);
       tc_fence_after();
       const bool m64 = t.rows <= 64;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * NMMA;
@@ -580,7 +588,7 @@ namespace {
 template <int EPI, int NMMA, bool GATHER>
 cudaError_t run_gemm(const void* A, int64_t a_rows, const int32_t* row_slot, int k, const void* B0,
                      const void* B1, int64_t rows_max, int K, int N, int E, const int32_t* seg,
-                     void* out, Control* ctl, cudaStream_t s) {
+                     const int32_t* kept, void* out, Control* ctl, cudaStream_t s) {
   using C = Cfg<EPI, NMMA>;
   CUtensorMap ta, tb0, tb1;
   if (!make_tma_2d_bf16(&ta, A, static_cast<uint64_t>(a_rows), K, GATHER ? 1 : BM))
@@ -591,6 +599,7 @@ cudaError_t run_gemm(const void* A, int64_t a_rows, const int32_t* row_slot, int
   a.seg = seg;
   a.out = static_cast<__nv_bfloat16*>(out);
   a.row_slot = row_slot;
+  a.kept = kept;
   a.k = k;
   a.E = E;
   a.K = K;
@@ -605,39 +614,42 @@ cudaError_t run_gemm(const void* A, int64_t a_rows, const int32_t* row_slot, int
 template <bool GATHER>
 cudaError_t run_up(const void* a, int64_t a_rows, const int32_t* row_slot, int k, const void* w1,
                    const void* w3, moe_act_t act, int64_t rows_max, int d, int F, int E,
-                   const int32_t* seg, void* h, Control* ctl, cudaStream_t s) {
+                   const int32_t* seg, const int32_t* kept, void* h, Control* ctl,
+                   cudaStream_t s) {
   if (act == MOE_ACT_SWIGLU)
     return run_gemm<EPI_SWIGLU, 256, GATHER>(a, a_rows, row_slot, k, w1, w3, rows_max, d, F, E, seg,
-                                             h, ctl, s);
+                                             kept, h, ctl, s);
   if (F % 256 == 0)
     return run_gemm<EPI_GELU, 256, GATHER>(a, a_rows, row_slot, k, w1, nullptr, rows_max, d, F, E,
-                                           seg, h, ctl, s);
+                                           seg, kept, h, ctl, s);
   return run_gemm<EPI_GELU, 128, GATHER>(a, a_rows, row_slot, k, w1, nullptr, rows_max, d, F, E, seg,
-                                         h, ctl, s);
+                                         kept, h, ctl, s);
 }
 
 }  // namespace
 
 cudaError_t launch_ffn_bf16(const void* a, int64_t a_rows, const int32_t* row_slot, int k,
                             const void* w1, const void* w3, const void* w2, moe_act_t act,
-                            int64_t rows_max, int d, int F, int E, const int32_t* seg, void* h,
-                            void* y, Control* ctl, cudaStream_t s, cudaEvent_t after_up) {
+                            int64_t rows_max, int d, int F, int E, const int32_t* seg,
+                            const int32_t* kept, void* h, void* y, Control* ctl, cudaStream_t s,
+                            cudaEvent_t after_up) {
   if (rows_max <= 0) {
     if (after_up) cudaEventRecord(after_up, s);
     return cudaSuccess;
   }
   cudaError_t err =
       row_slot != nullptr
-          ? run_up<true>(a, a_rows, row_slot, k, w1, w3, act, rows_max, d, F, E, seg, h, ctl, s)
-          : run_up<false>(a, rows_max, nullptr, 1, w1, w3, act, rows_max, d, F, E, seg, h, ctl, s);
+          ? run_up<true>(a, a_rows, row_slot, k, w1, w3, act, rows_max, d, F, E, seg, kept, h, ctl, s)
+          : run_up<false>(a, rows_max, nullptr, 1, w1, w3, act, rows_max, d, F, E, seg, kept, h, ctl,
+                          s);
   if (err != cudaSuccess) return err;
   if (after_up) cudaEventRecord(after_up, s);
   if (d % 256 == 0)
     err = run_gemm<EPI_STORE, 256, false>(h, rows_max, nullptr, 1, w2, nullptr, rows_max, F, d, E,
-                                          seg, y, ctl, s);
+                                          seg, kept, y, ctl, s);
   else
     err = run_gemm<EPI_STORE, 128, false>(h, rows_max, nullptr, 1, w2, nullptr, rows_max, F, d, E,
-                                          seg, y, ctl, s);
+                                          seg, kept, y, ctl, s);
   return err;
 }
 

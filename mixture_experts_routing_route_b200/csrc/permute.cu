@@ -40,7 +40,7 @@ constexpr int kMaxE = 256;
 
 __global__ void __launch_bounds__(kThreads)
 permute_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_mask, long long cap,
-               int32_t* __restrict__ counts, int32_t* __restrict__ bins,
+               int binned, int32_t* __restrict__ counts, int32_t* __restrict__ bins,
                int32_t* __restrict__ sorted_slot, int32_t* __restrict__ slot_to_row,
                int32_t* __restrict__ row_slot, uint8_t* __restrict__ drop,
                int32_t* __restrict__ kept, int32_t* __restrict__ seg, int32_t* __restrict__ rank_g,
@@ -50,13 +50,16 @@ permute_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_mask,
   __shared__ int running[kMaxE];
   __shared__ int start_s[kMaxE];
   __shared__ int seg_s[kMaxE + 1];
+  __shared__ int kept_s[kMaxE];
   __shared__ int wtot_c[8], wtot_k[8];
+  __shared__ int maxc_s;
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const unsigned lt_mask = (1u << lane) - 1u;
 
   for (int i = tid; i < 32 * (kMaxE + 1); i += kThreads) (&hist[0][0])[i] = 0;
   for (int i = tid; i < kMaxE; i += kThreads) running[i] = 0;
+  if (tid == 0) maxc_s = 0;
   __syncthreads();
 
   // ---- pass 1: stable rank of every slot within its expert
@@ -98,10 +101,15 @@ permute_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_mask,
   }
 
   // ---- counts, bins (inclusive), kept = min(count, C), seg (exclusive) over E <= 256
+  // Binned layout: bin size C = cap, or the largest count when cap is none.
+  if (binned && cap == LLONG_MAX && tid < E) atomicMax(&maxc_s, running[tid]);
+  __syncthreads();
+  const long long bin = binned ? (cap == LLONG_MAX ? static_cast<long long>(maxc_s) : cap) : 0;
   int c = 0, kp = 0, ci = 0, ki = 0;
   if (tid < 256) {
     c = tid < E ? running[tid] : 0;
-    kp = static_cast<int>(c < cap ? c : cap);
+    const long long lim = binned ? bin : cap;
+    kp = static_cast<int>(c < lim ? c : lim);
     ci = c;
     ki = kp;
 #pragma unroll
@@ -119,16 +127,28 @@ permute_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_mask,
     ci += pc;
     ki += pk;
     if (tid < E) {
+      const int sg = binned ? static_cast<int>(tid * bin) : ki - kp;
       counts[tid] = c;
       bins[tid] = ci;
       kept[tid] = kp;
-      seg[tid] = ki - kp;
+      seg[tid] = sg;
       start_s[tid] = ci - c;
-      seg_s[tid] = ki - kp;
+      seg_s[tid] = sg;
+      kept_s[tid] = kp;
     }
-    if (tid == E - 1) { seg[E] = ki; seg_s[E] = ki; }
+    if (tid == E - 1) {
+      const int end = binned ? static_cast<int>(E * bin) : ki;
+      seg[E] = end;
+      seg_s[E] = end;
+    }
   }
   __syncthreads();
+  // binned: the padding rows of every bin
+  if (binned)
+    for (long long i = tid; i < E * bin; i += kThreads) {
+      const int e = static_cast<int>(i / bin), r = static_cast<int>(i - e * bin);
+      if (r >= kept_s[e]) row_slot[i] = -1;
+    }
 
   // ---- pass 2: counting-sort scatter, drop mask and the row maps; the loads
   // of 4 slots are issued before any of them is used.
@@ -153,7 +173,7 @@ permute_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_mask,
       }
       const int r = rv[u];
       sorted_slot[start_s[e] + r] = s;
-      const bool dr = r >= cap;
+      const bool dr = r >= (binned ? bin : cap);
       drop[s] = dr ? 1 : 0;
       const int row = dr ? -1 : seg_s[e] + r;
       slot_to_row[s] = row;
@@ -208,7 +228,7 @@ __device__ bool grid_barrier(Control* ctl, unsigned nblocks) {
 
 __global__ void __launch_bounds__(kGThreads)
 permute_grid_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_mask,
-                    long long cap, int chunk, int32_t* __restrict__ counts,
+                    long long cap, int binned, int chunk, int32_t* __restrict__ counts,
                     int32_t* __restrict__ bins, int32_t* __restrict__ sorted_slot,
                     int32_t* __restrict__ slot_to_row, int32_t* __restrict__ row_slot,
                     uint8_t* __restrict__ drop, int32_t* __restrict__ kept,
@@ -222,7 +242,9 @@ permute_grid_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_
   __shared__ int tot[kMaxE];
   __shared__ int start_s[kMaxE];
   __shared__ int seg_s[kMaxE + 1];
+  __shared__ int kept_s[kMaxE];
   __shared__ int wtot_c[8], wtot_k[8];
+  __shared__ int maxc_s;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned lt_mask = (1u << lane) - 1u;
   const int lo = blockIdx.x * chunk;
@@ -230,6 +252,7 @@ permute_grid_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_
 
   for (int i = tid; i < 8 * (kMaxE + 1); i += kGThreads) (&hist[0][0])[i] = 0;
   for (int i = tid; i < kMaxE; i += kGThreads) { running[i] = 0; pre[i] = 0; tot[i] = 0; }
+  if (tid == 0) maxc_s = 0;
   __syncthreads();
 
   // ---- local stable ranks of this CTA's slots
@@ -280,10 +303,15 @@ permute_grid_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_
     if (b < static_cast<int>(blockIdx.x)) atomicAdd(&pre[e], c);
   }
   __syncthreads();
-  // counts, bins (inclusive), kept = min(count, C), seg (exclusive) over E <= 256
+  // counts, bins (inclusive), kept = min(count, C), seg (exclusive) over E <= 256;
+  // binned layout: bin size C = cap, or the largest count when cap is none
+  if (binned && cap == LLONG_MAX && tid < E) atomicMax(&maxc_s, tot[tid]);
+  __syncthreads();
+  const long long bin = binned ? (cap == LLONG_MAX ? static_cast<long long>(maxc_s) : cap) : 0;
+  const long long lim = binned ? bin : cap;
   int c = 0, kp = 0, ci = 0, ki = 0;
   c = tid < E ? tot[tid] : 0;
-  kp = static_cast<int>(c < cap ? c : cap);
+  kp = static_cast<int>(c < lim ? c : lim);
   ci = c;
   ki = kp;
 #pragma unroll
@@ -299,21 +327,31 @@ permute_grid_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_
   ci += pc;
   ki += pk;
   if (tid < E) {
+    const int sg = binned ? static_cast<int>(tid * bin) : ki - kp;
     if (blockIdx.x == 0) {
       counts[tid] = c;
       bins[tid] = ci;
       kept[tid] = kp;
-      seg[tid] = ki - kp;
+      seg[tid] = sg;
     }
     start_s[tid] = ci - c;
-    seg_s[tid] = ki - kp;
+    seg_s[tid] = sg;
+    kept_s[tid] = kp;
   }
   if (tid == E - 1) {
-    if (blockIdx.x == 0) seg[E] = ki;
-    seg_s[E] = ki;
+    const int end = binned ? static_cast<int>(E * bin) : ki;
+    if (blockIdx.x == 0) seg[E] = end;
+    seg_s[E] = end;
   }
   __syncthreads();
   if (!ok) return;  // a timed-out barrier leaves the offsets unknown: write nothing
+  // binned: this CTA's share of the padding rows of every bin
+  if (binned)
+    for (long long i = static_cast<long long>(blockIdx.x) * kGThreads + tid; i < E * bin;
+         i += static_cast<long long>(gridDim.x) * kGThreads) {
+      const int e = static_cast<int>(i / bin), r = static_cast<int>(i - e * bin);
+      if (r >= kept_s[e]) row_slot[i] = -1;
+    }
 
   // ---- counting-sort scatter, drop mask and the row maps
   for (int s = lo + tid; s < hi; s += kGThreads) {
@@ -330,7 +368,7 @@ permute_grid_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_
       continue;
     }
     sorted_slot[pos] = s;
-    const bool dr = r >= cap;
+    const bool dr = r >= lim;
     drop[s] = dr ? 1 : 0;
     const int row = dr ? -1 : seg_s[e] + r;
     slot_to_row[s] = row;
@@ -355,18 +393,18 @@ cudaError_t launch_permute_single(const int32_t* idx, int T, int k, int E, int64
                                   int32_t* counts, int32_t* bins, int32_t* sorted_slot,
                                   int32_t* slot_to_row, int32_t* row_slot, uint8_t* drop,
                                   int32_t* kept, int32_t* seg, int32_t* rank_scratch, Control* ctl,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, bool binned) {
   const unsigned mask = static_cast<unsigned>(key_mask_of(E));
   const long long c = cap < 0 ? LLONG_MAX : static_cast<long long>(cap);
   return launch_pdl(permute_kernel, dim3(1), dim3(kThreads), 0, s, false, idx, T * k, E, mask, c,
-                    counts, bins, sorted_slot, slot_to_row, row_slot, drop, kept, seg, rank_scratch,
+                    binned ? 1 : 0, counts, bins, sorted_slot, slot_to_row, row_slot, drop, kept, seg, rank_scratch,
                     ctl);
 }
 
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int64_t cap, int32_t* counts,
                            int32_t* bins, int32_t* sorted_slot, int32_t* slot_to_row,
                            int32_t* row_slot, uint8_t* drop, int32_t* kept, int32_t* seg,
-                           int32_t* scratch, Control* ctl, cudaStream_t s) {
+                           int32_t* scratch, Control* ctl, cudaStream_t s, bool binned) {
   const int S = T * k;
   const int sms = num_sms();
   // enough CTAs that each chunk fits shared memory, at most one per SM, and
@@ -375,13 +413,13 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int64_t cap,
   const int chunk = S > 0 ? (S + g - 1) / g : 0;
   if (S == 0 || chunk > kGMaxChunk || g < 2)
     return launch_permute_single(idx, T, k, E, cap, counts, bins, sorted_slot, slot_to_row,
-                                 row_slot, drop, kept, seg, scratch, ctl, s);
+                                 row_slot, drop, kept, seg, scratch, ctl, s, binned);
   int32_t* cta_counts = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(scratch) +
                                                    align_up(static_cast<size_t>(S) * 4));
   unsigned mask = static_cast<unsigned>(key_mask_of(E));
   long long c = cap < 0 ? LLONG_MAX : static_cast<long long>(cap);
   return launch_pdl(permute_grid_kernel, dim3(g), dim3(kGThreads), 0, s, true, idx, S, E, mask, c,
-                    chunk, counts, bins, sorted_slot, slot_to_row, row_slot, drop, kept, seg,
+                    binned ? 1 : 0, chunk, counts, bins, sorted_slot, slot_to_row, row_slot, drop, kept, seg,
                     cta_counts, ctl);
 }
 

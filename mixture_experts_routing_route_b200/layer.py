@@ -18,7 +18,7 @@ class MoeLayer:
     def __init__(self, w_router: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
                  w3: Optional[torch.Tensor] = None, bias: Optional[torch.Tensor] = None,
                  k: int = 2, act: str = "swiglu", capacity_factor: float = 0.0,
-                 gather_in_gemm: bool = False):
+                 gather_in_gemm: bool = False, binned: bool = False):
         if not w1.is_cuda:
             raise ValueError("weights must be CUDA tensors")
         self.E, self.d, self.F = w1.shape
@@ -33,7 +33,10 @@ class MoeLayer:
         self.bias = None if bias is None else bias.to(device=w1.device, dtype=torch.float32).contiguous()
         # gather_in_gemm: the up projection gathers x rows itself (bf16; see
         # MOE_LAYER_GATHER_IN_GEMM in include/moe_b200.h)
-        flags = abi.MOE_LAYER_GATHER_IN_GEMM if gather_in_gemm else 0
+        # binned: the [E, C, hs] bucket layout (MOE_LAYER_BINNED); with
+        # capacity_factor <= 0 the bin size is the call's largest expert count
+        flags = (abi.MOE_LAYER_GATHER_IN_GEMM if gather_in_gemm else 0) | \
+            (abi.MOE_LAYER_BINNED if binned else 0)
         self.c = abi.layer_struct(self.d, self.E, k, self.F, abi.dtype_code(self.dtype), self.act,
                                   self.cf, self.w_router, self.bias, self.w1, self.w3, self.w2,
                                   flags)

@@ -31,6 +31,16 @@ def test_capacity_matches_oracle_formula(abi):
         assert abi.moe_capacity(cf, T, k, E) == (-1 if ref is None else ref)
 
 
+def test_rows_max_binned(abi):
+    assert abi.moe_rows_max_binned(100, 2, 8, 10) == 80
+    assert abi.moe_rows_max_binned(100, 2, 8, -1) == 8 * 200   # dynamic: worst case C = T*k
+    assert abi.moe_rows_max_binned(100, 2, 8, 0) == 0
+    L = abi.MoeLayerC(4096, 8, 2, 14336, abi.MOE_BF16, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, 16, 16,
+                      abi.MOE_LAYER_BINNED)
+    Ld = abi.MoeLayerC(4096, 8, 2, 14336, abi.MOE_BF16, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, 16, 16)
+    assert abi.moe_forward_workspace_size(L, 4096) > abi.moe_forward_workspace_size(Ld, 4096)
+
+
 def test_rows_max(abi):
     assert abi.moe_rows_max(100, 2, 8, -1) == 200
     assert abi.moe_rows_max(100, 2, 8, 10) == 80
@@ -80,6 +90,11 @@ def test_argument_checks_return_before_launch(abi):
     L2 = abi.MoeLayerC(4096, 8, 2, 128, abi.MOE_BF16, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, None, 16)
     assert abi._lib.moe_forward(ctypes.byref(L2), 16, 4, 16, None, 16, 1 << 40, None, None) == 1
     assert abi._lib.moe_permute(16, 4, 2, 0, -1, *([16] * 8), 16, 1 << 20, None) == 2
+    L3 = abi.MoeLayerC(4096, 8, 2, 128, abi.MOE_BF16, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, 16, 16, 8)
+    assert abi._lib.moe_forward(ctypes.byref(L3), 16, 4, 16, None, 16, 1 << 40, None, None) == 2
+    L4 = abi.MoeLayerC(4096, 8, 2, 128, abi.MOE_F32, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, 16, 16,
+                       abi.MOE_LAYER_GATHER_IN_GEMM)
+    assert abi._lib.moe_forward(ctypes.byref(L4), 16, 4, 16, None, 16, 1 << 40, None, None) == 3
     assert abi.moe_kernel_launches() == n0
 
 

@@ -152,3 +152,43 @@ def test_repeat_is_deterministic():
     _, out1, aux1, _, _ = run_layer(inp)
     _, out2, aux2, _, _ = run_layer(inp)
     assert torch.equal(out1, out2) and torch.equal(aux1, aux2)
+
+
+@pytest.mark.parametrize("T,d,E,k,F,act,dt,cf,bias", [
+    (700, 256, 8, 2, 512, "swiglu", "bf16", 0.0, "none"),      # dynamic capacity (no drop)
+    (900, 256, 8, 2, 256, "swiglu", "bf16", 0.0, "expert0"),   # dynamic, skewed: big padding
+    (1000, 256, 16, 2, 512, "gelu", "bf16", 1.0, "zipf"),      # fixed capacity with drops
+    (256, 64, 4, 1, 128, "gelu", "f32", 1.25, "none"),         # fp32, fixed capacity
+    (200, 64, 6, 2, 96, "swiglu", "f32", 0.0, "none"),         # fp32, dynamic
+])
+def test_layer_binned(T, d, E, k, F, act, dt, cf, bias):
+    """The [E, C, hs] bucket layout (MOE_LAYER_BINNED): the same output as the
+    default layout, bit for bit; the bucket's rows (zero padding included) and
+    the expert outputs of the kept rows match the oracle's binned stages."""
+    from mixture_experts_routing_route_b200 import MoeLayer
+    inp = small_case("binned", T=T, d=d, E=E, k=k, F=F, act=act, dtype=dt, cf=cf, bias=bias,
+                     seed=T + E)
+    dv = device_inputs(inp)
+    mk = lambda b: MoeLayer(dv["wg"], dv["w1"], dv["w2"], w3=dv["w3"], bias=dv["bias"], k=k,
+                            act=act, capacity_factor=cf, binned=b)
+    lb, ld = mk(True), mk(False)
+    out_b, aux_b = lb.forward(dv["x"])
+    out_d, aux_d = ld.forward(dv["x"])
+    torch.cuda.synchronize()
+    assert lb.device_error(T) == 0 and ld.device_error(T) == 0
+    assert torch.equal(out_b, out_d) and torch.equal(aux_b, aux_d)
+    v = lb.views(T)
+    g_idx = npi(v["topk_idx"]).astype(np.int64)
+    cap = O.capacity(cf, k, T, E)
+    bn = O.permute_binned(g_idx, E, cap)
+    assert int(v["seg_offsets"][1].item()) == bn["bin"]
+    assert np.array_equal(npi(v["row_slot"])[:bn["rows"]], bn["row_slot"])
+    assert np.array_equal(npi(v["slot_to_row"]), bn["slot_to_row"])
+    xb = O.gather_binned(np32(inp.x), bn["row_slot"], k)
+    assert np.array_equal(np32(v["x_perm"])[:bn["rows"]], xb)
+    w1, w2 = ExpertWeights(inp.w1), ExpertWeights(inp.w2)
+    w3 = None if inp.w3 is None else ExpertWeights(inp.w3)
+    y_ref = O.expert_ffn_binned(xb, bn["kept_counts"], bn["bin"], w1, w3, w2, act)
+    live = bn["row_slot"] >= 0
+    tol = TOL_BF16_OUT if dt == "bf16" else TOL_F32_OUT
+    assert max_err_ratio(np32(v["y_perm"])[:bn["rows"]][live], y_ref[live]) <= tol

@@ -258,3 +258,58 @@ def test_fused_gather_equals_gather_then_ffn(act, T, d, E, k, F, cf):
     assert torch.equal(h[:R], v["h"][:R])
     assert torch.equal(y[:R], v["y_perm"][:R])
     assert torch.equal(out, out_plain)
+
+
+def permute_binned_on_gpu(idx_np, E, cap):
+    T, k = idx_np.shape
+    S = T * k
+    R = abi.moe_rows_max_binned(T, k, E, cap)
+    t = lambda n: torch.full((max(n, 1),), -7, dtype=torch.int32, device=DEV)
+    out = {"counts": t(E), "bins": t(E), "sorted_slot": t(S), "slot_to_row": t(S),
+           "row_slot": t(R), "kept_counts": t(E), "seg_offsets": t(E + 1)}
+    drop = torch.full((max(S, 1),), 7, dtype=torch.uint8, device=DEV)
+    ws = new_ws(abi.moe_permute_workspace_size(T, k, E))
+    idx = torch.from_numpy(np.ascontiguousarray(idx_np, dtype=np.int32)).to(DEV)
+    abi.moe_permute_binned(idx, T, k, E, cap, out["counts"], out["bins"], out["sorted_slot"],
+                           out["slot_to_row"], out["row_slot"], drop, out["kept_counts"],
+                           out["seg_offsets"], ws)
+    torch.cuda.synchronize()
+    res = {kk: npi(vv) for kk, vv in out.items()}
+    res["drop"] = npi(drop)
+    res["err"] = abi.moe_get_device_error(ws)
+    return res
+
+
+@pytest.mark.parametrize("T,k,E", [(5, 2, 3), (512, 2, 8), (1025, 1, 7), (3000, 8, 256), (20000, 3, 17)])
+def test_permute_binned(T, k, E):
+    """[E, C] bucket layout (MegaBlocks page, sections 4.3-4.6): bit-exact with
+    the oracle for fixed capacities and for dynamic capacity (C = the largest
+    count), single- and multi-CTA permute."""
+    rng = np.random.default_rng(T * 7 + E)
+    idx = np.array([rng.permutation(E)[:k] for _ in range(T)])
+    S = T * k
+    for cap in (-1, 0, 1, max(1, S // E), S):
+        g = permute_binned_on_gpu(idx, E, cap)
+        ref = O.permute_binned(idx, E, None if cap < 0 else cap)
+        assert g["err"] == 0
+        for key in ("counts", "bins", "kept_counts"):
+            assert np.array_equal(g[key][:E], ref[key]), (cap, key)
+        assert np.array_equal(g["seg_offsets"][:E + 1], ref["seg_offsets"]), cap
+        for key in ("sorted_slot", "slot_to_row"):
+            assert np.array_equal(g[key][:S], ref[key]), (cap, key)
+        assert np.array_equal(g["drop"][:S], ref["drop"]), cap
+        assert np.array_equal(g["row_slot"][:ref["rows"]], ref["row_slot"]), cap
+
+
+def test_permute_binned_skewed_dynamic():
+    """80% of the slots on expert 0: the dynamic bin is expert 0's count and
+    the other bins are mostly padding."""
+    T, k, E = 3333, 2, 8
+    rng = np.random.default_rng(1)
+    idx = np.where(rng.random((T, k)) < 0.8, 0, rng.integers(1, E, size=(T, k)))
+    idx[:, 1] = np.where(idx[:, 1] == idx[:, 0], (idx[:, 0] + 1) % E, idx[:, 1])
+    g = permute_binned_on_gpu(idx, E, -1)
+    ref = O.permute_binned(idx, E, None)
+    assert g["err"] == 0 and g["seg_offsets"][1] == ref["bin"] == ref["counts"].max()
+    assert np.array_equal(g["row_slot"][:ref["rows"]], ref["row_slot"])
+    assert np.array_equal(g["slot_to_row"][:T * k], ref["slot_to_row"])
