@@ -57,6 +57,8 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--binned", action="store_true",
+                   help="padded-binned [E, C, hs] layout (capacity_factor 0: C = the largest count)")
     p.add_argument("--gather-in-gemm", action="store_true",
                    help="bf16: gather x rows inside the up projection (tile::gather4) instead of "
                         "the gather kernel")
@@ -84,7 +86,7 @@ def workload_config(sh):
 
 
 # ------------------------------------------------------------------ roofline
-def algorithmic(sh, counts_kept):
+def algorithmic(sh, counts_kept, bucket_rows=None):
     """Algorithmic flops and bytes per stage for one forward (no re-reads).
 
     R = kept rows, E_act = experts with R_e > 0, b = element bytes.
@@ -92,7 +94,8 @@ def algorithmic(sh, counts_kept):
       permute  bytes S*4 + S*(4+4+4+1) (idx in; sorted_slot, slot_to_row,
                row_slot, drop out)
       gather   bytes T_used*d*b + R*d*b (each token read once, rows written);
-               with --gather-in-gemm no separate stage
+               binned: + the bucket's padding rows written as zeros (E*C rows
+               in all); with --gather-in-gemm no separate stage
       ffn_up   flops 2*R*d*F*(2 SwiGLU | 1 GELU); bytes weights of active
                experts + R*d*b (A rows: x_perm, or x gathered) + R*F*b
       ffn_down flops 2*R*F*d; bytes E_act*F*d*b + R*F*b + R*d*b
@@ -107,7 +110,7 @@ def algorithmic(sh, counts_kept):
     return {
         "route": {"bytes": T * d * b + d * E * b + S * 8},
         "permute": {"bytes": S * 4 + S * 13},
-        "gather": {"bytes": min(T, R) * d * b + R * d * b},
+        "gather": {"bytes": min(T, R) * d * b + (bucket_rows if bucket_rows is not None else R) * d * b},
         "ffn_up": {"flops": 2 * R * d * F * nup,
                    "bytes": e_act * d * F * b * nup + R * d * b + R * F * b},
         "ffn_down": {"flops": 2 * R * F * d, "bytes": e_act * F * d * b + R * F * b + R * d * b},
@@ -404,7 +407,8 @@ def main():
     layer = MoeLayer(inp.wg.to(dev), inp.w1.to(dev), inp.w2.to(dev),
                      w3=None if inp.w3 is None else inp.w3.to(dev),
                      bias=None if inp.bias is None else inp.bias.to(dev),
-                     k=sh.k, act=sh.act, capacity_factor=sh.cf, gather_in_gemm=args.gather_in_gemm)
+                     k=sh.k, act=sh.act, capacity_factor=sh.cf, gather_in_gemm=args.gather_in_gemm,
+                     binned=args.binned)
     out = torch.empty(sh.T, sh.d, dtype=x.dtype, device=dev)
     aux = torch.empty(1, dtype=torch.float32, device=dev)
     flush = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
@@ -426,6 +430,7 @@ def main():
         raise RuntimeError("device error word set during warm-up")
     v = layer.views(sh.T)
     kept = v["kept_counts"].cpu().tolist()
+    bucket_rows = int(v["seg_offsets"][-1].item()) if args.binned else None
     def timed_region():
         barrier(world)
         torch.cuda.synchronize()
@@ -467,7 +472,7 @@ def main():
     torch.cuda.synchronize()
     stage_ms = {s: statistics.mean(bevs[i][j].elapsed_time(bevs[i][j + 1]) for i in range(nb))
                 for j, s in enumerate(STAGES)}
-    alg = algorithmic(sh, kept)
+    alg = algorithmic(sh, kept, bucket_rows)
     peaks = load_peaks()
     # A timed region long enough to hit the 1 kW power cap is compared with the
     # sustained (power-capped) GEMM figure, a short one with the burst figure.
@@ -519,7 +524,9 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": sh.dtype,
         "data": "synthetic (seeded; random-init weights of the layer's shape)",
         "config": dict(workload_config(sh), parallelism=f"replicas x{world}" if world > 1 else "1 GPU",
-                       **({"gather": "in the up projection (tile::gather4)"} if args.gather_in_gemm else {})),
+                       **({"gather": "in the up projection (tile::gather4)"} if args.gather_in_gemm else {}),
+                       **({"layout": f"binned [E, C, d], C = {bucket_rows // sh.E if sh.E else 0}"}
+                          if args.binned else {})),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks,
