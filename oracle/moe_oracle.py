@@ -59,6 +59,8 @@ __all__ = [
     "gate_logits", "softmax_rows", "topk_select", "renormalise", "aux_loss",
     "near_tie_tokens", "route", "capacity", "sort_end_bit", "permute", "gather",
     "activation", "expert_ffn", "combine", "forward", "forward_tokens",
+    "permute_binned", "gather_binned", "expert_ffn_binned",
+    "philox4x32_10", "jitter_multipliers", "apply_jitter", "bf16_round", "logit_noise", "z_loss",
 ]
 
 
@@ -142,9 +144,13 @@ def near_tie_tokens(logits32, k, eps=1e-3):
     return (l[:, k - 1] - l[:, k]) < eps
 
 
-def route(x, wg, bias, k):
-    """Router stage: logits, softmax, top-k, renormalised weights, aux loss."""
+def route(x, wg, bias, k, noise=None):
+    """Router stage: logits, softmax, top-k, renormalised weights, aux loss,
+    z-loss. noise: optional [T, E] values added to the logits (the training
+    variant's Gaussian noise)."""
     l64 = gate_logits(x, wg, bias)
+    if noise is not None:
+        l64 = l64 + np.asarray(noise, dtype=np.float64)
     logits32 = l64.astype(np.float32)
     p64 = softmax_rows(l64)
     idx = topk_select(logits32, k)
@@ -158,8 +164,119 @@ def route(x, wg, bias, k):
         "topk_w64": w64,
         "topk_w": w64.astype(np.float32),
         "aux": aux_loss(p64, idx, E),
+        "z": z_loss(l64),
         "near_tie": near_tie_tokens(logits32, k),
     }
+
+
+# --------------------------------------------------------------------------
+# router variants (training): jitter, logit noise, z-loss
+# --------------------------------------------------------------------------
+#
+# The random numbers come from Philox4x32-10, the counter-based generator of
+# Salmon, Moraes, Dror and Shaw, "Parallel random numbers: as easy as 1, 2,
+# 3" (SC 2011), written here from that definition: a 4 x 32-bit counter
+# and a 2 x 32-bit key; each of the 10 rounds multiplies counter words 0 and
+# 2 by fixed odd constants, keeps the high and low halves, and mixes them
+# with words 1 and 3 and the key; the key advances by two Weyl constants
+# between rounds.
+
+_PHILOX_M = (0xD2511F53, 0xCD9E8D57)
+_PHILOX_W = (0x9E3779B9, 0xBB67AE85)
+_U32 = np.uint64(0xFFFFFFFF)
+
+
+def philox4x32_10(ctr, key):
+    """ctr: integer array [..., 4] of 32-bit words; key: (k0, k1).
+    Returns uint32 [..., 4]."""
+    c = np.asarray(ctr, dtype=np.uint64) & _U32
+    c0, c1, c2, c3 = (c[..., i] for i in range(4))
+    k0, k1 = np.uint64(key[0]) & _U32, np.uint64(key[1]) & _U32
+    m0, m1 = np.uint64(_PHILOX_M[0]), np.uint64(_PHILOX_M[1])
+    for _ in range(10):
+        p0 = c0 * m0
+        p1 = c2 * m1
+        hi0, lo0 = p0 >> np.uint64(32), p0 & _U32
+        hi1, lo1 = p1 >> np.uint64(32), p1 & _U32
+        c0, c1, c2, c3 = (hi1 ^ c1 ^ k0) & _U32, lo1, (hi0 ^ c3 ^ k1) & _U32, lo0
+        k0 = (k0 + np.uint64(_PHILOX_W[0])) & _U32
+        k1 = (k1 + np.uint64(_PHILOX_W[1])) & _U32
+    return np.stack([c0, c1, c2, c3], axis=-1).astype(np.uint32)
+
+
+def _philox_words(n, stream, seed, per_call):
+    """Word (n mod per_call) of Philox call floor(n / per_call) on counter
+    (call low 32 bits, call high 32 bits, stream, 0), key (seed low, seed
+    high), for every n in the integer array n; per_call is 4 or 2 (then the
+    pair 2*(n mod 2), 2*(n mod 2)+1 is returned as two arrays)."""
+    n = np.asarray(n, dtype=np.uint64)
+    call = n // np.uint64(per_call)
+    ctr = np.stack([call & _U32, call >> np.uint64(32), np.full_like(call, stream),
+                    np.zeros_like(call)], axis=-1)
+    out = philox4x32_10(ctr, (int(seed) & 0xFFFFFFFF, (int(seed) >> 32) & 0xFFFFFFFF))
+    j = (n % np.uint64(per_call)).astype(np.int64)
+    if per_call == 4:
+        return np.take_along_axis(out, j[..., None], axis=-1)[..., 0]
+    a = np.take_along_axis(out, (2 * j)[..., None], axis=-1)[..., 0]
+    b = np.take_along_axis(out, (2 * j + 1)[..., None], axis=-1)[..., 0]
+    return a, b
+
+
+def jitter_multipliers(T, d, eps, seed):
+    """Per-element router-input multipliers, uniform in [1 - eps, 1 + eps)
+    (MegaBlocks page, section 5: the router input is multiplied by uniform
+    noise in 1 +- eps during training). Element (t, i) = n = t*d + i uses
+    Philox stream 0, word n mod 4 of call n / 4: u = (word >> 8) / 2^24, and
+    m = (1 - eps) + (2 eps) * u, every operation in fp32 (returned fp32)."""
+    n = np.arange(T * d, dtype=np.uint64)
+    w = _philox_words(n, 0, seed, 4)
+    u = ((w >> np.uint32(8)).astype(np.float64) * 2.0 ** -24).astype(np.float32)
+    e32 = np.float32(eps)
+    a = np.float32(1.0) - e32
+    b = np.float32(2.0) * e32
+    return (a + b * u).astype(np.float32).reshape(T, d)
+
+
+def bf16_round(a32):
+    """Round fp32 values to the nearest bf16 (ties to even), returned as fp32."""
+    bits = np.asarray(a32, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    rounded = ((bits + np.uint64(0x7FFF) + ((bits >> np.uint64(16)) & np.uint64(1))) >> np.uint64(16)) << np.uint64(16)
+    return rounded.astype(np.uint32).view(np.float32)
+
+
+def apply_jitter(x32, mult, bf16):
+    """The router's input x * m, in fp32, rounded to bf16 for a bf16 layer
+    (the router then reads a tensor of the layer's dtype)."""
+    y = np.asarray(x32, dtype=np.float32) * np.asarray(mult, dtype=np.float32)
+    return bf16_round(y) if bf16 else y
+
+
+def logit_noise(T, E, std, seed):
+    """Gaussian noise added to the router logits ("Integrating MoE into your
+    model with Colossal-AI", step 2: NormalNoiseGenerator adds noise scaled by
+    the number of experts; the scale is the std argument, 1/E in that
+    reading). Logit (t, e) = n = t*E + e uses Philox stream 1, words
+    2*(n mod 2) and 2*(n mod 2)+1 of call n / 2: u1 = ((w0 >> 8) + 1) / 2^24
+    in (0, 1], u2 = (w1 >> 8) / 2^24, z = sqrt(-2 ln u1) cos(2 pi u2)
+    (Box and Muller, 1958). Returned float64 [T, E]."""
+    n = np.arange(T * E, dtype=np.uint64)
+    w0, w1 = _philox_words(n, 1, seed, 2)
+    u1 = ((w0 >> np.uint32(8)).astype(np.float64) + 1.0) * 2.0 ** -24
+    u2 = (w1 >> np.uint32(8)).astype(np.float64) * 2.0 ** -24
+    z = np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)
+    return (std * z).reshape(T, E)
+
+
+def z_loss(logits):
+    """Router z-loss: mean over tokens of the squared log-sum-exp of the
+    logits the softmax sees (bias and noise included). The pages name the
+    loss only (Colossal-AI's router_z_loss); this is the usual definition."""
+    l = np.asarray(logits, dtype=np.float64)
+    if l.shape[0] == 0:
+        return 0.0
+    m = l.max(axis=1, keepdims=True)
+    lse = m[:, 0] + np.log(np.exp(l - m).sum(axis=1))
+    return float(np.mean(lse ** 2))
 
 
 # --------------------------------------------------------------------------

@@ -430,3 +430,67 @@ def pin_binned_forward_equals_dense(o):
 
 ALL_PINS.extend([pin_binned_example_a, pin_binned_bruteforce, pin_binned_forward_equals_dense])
 
+
+def pin_philox_kat(o):
+    """Philox4x32-10 reproduces the generator's published known-answer vectors."""
+    for c in _golden("philox_kat.json")["cases"]:
+        got = o.philox4x32_10([int(v, 16) for v in c["ctr"]], tuple(int(v, 16) for v in c["key"]))
+        assert [int(v) for v in got] == [int(v, 16) for v in c["out"]], c
+
+
+def pin_jitter(o):
+    """Multipliers lie in [1 - eps, 1 + eps) with the uniform's mean and
+    variance (eps^2 / 3); eps = 0 gives exactly 1; seeds give different
+    streams; bf16 rounding of x * m is round-to-nearest-even."""
+    m = o.jitter_multipliers(256, 256, 0.01, 7).astype(np.float64)
+    assert m.min() >= 1 - 0.01 - 1e-7 and m.max() < 1 + 0.01 + 1e-7
+    assert abs(m.mean() - 1.0) < 2e-4
+    assert abs(m.var() - 0.01 ** 2 / 3) < 0.05 * 0.01 ** 2 / 3
+    assert np.all(o.jitter_multipliers(4, 8, 0.0, 7) == 1.0)
+    assert not np.array_equal(o.jitter_multipliers(4, 8, 0.1, 7), o.jitter_multipliers(4, 8, 0.1, 8))
+    # bf16 spacing at 1 is 2^-7: 1 + 2^-8 is a tie (to even: 1); 1 + 3*2^-8 is a
+    # tie between 1 + 2^-7 (odd) and 1 + 2^-6 (even); 1 + 2^-7 + 2^-9 is below
+    # the tie and rounds down to 1 + 2^-7
+    x = np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, 1.0 + 2.0 ** -7 + 2.0 ** -9], dtype=np.float32)
+    assert list(o.bf16_round(x)) == [1.0, 1.0 + 2.0 ** -6, 1.0 + 2.0 ** -7]
+
+
+def pin_logit_noise(o):
+    """Box-Muller normals: mean 0, standard deviation std, 68.3% within one
+    std; std = 0 gives zeros."""
+    z = o.logit_noise(512, 256, 0.5, 11)
+    assert abs(z.mean()) < 0.01 and abs(z.std() - 0.5) < 0.01
+    assert abs(np.mean(np.abs(z) < 0.5) - 0.6827) < 0.01
+    assert np.all(o.logit_noise(3, 4, 0.0, 11) == 0.0)
+
+
+def pin_z_loss(o):
+    """Equal logits c: (c + ln E)^2; a dominant logit L: close to L^2; small
+    random cases: a direct double loop."""
+    E = 8
+    assert abs(o.z_loss(np.full((5, E), 2.0)) - (2.0 + math.log(E)) ** 2) < 1e-12
+    l = np.zeros((3, E))
+    l[:, 3] = 40.0
+    assert abs(o.z_loss(l) - 40.0 ** 2) < 1e-6
+    rng = _rng(30)
+    l = rng.standard_normal((6, 5)) * 3
+    ref = sum(math.log(sum(math.exp(v) for v in row)) ** 2 for row in l) / 6
+    assert abs(o.z_loss(l) - ref) < 1e-12
+
+
+def pin_route_noise(o):
+    """Noise enters as a per-token additive logit term: routing with noise n
+    equals routing the gate logits plus n (closed form with a zero gate)."""
+    rng = _rng(31)
+    T, d, E, k = 12, 4, 6, 2
+    n = rng.standard_normal((T, E))
+    r = o.route(np.zeros((T, d)), np.zeros((d, E)), None, k, noise=n)
+    assert np.array_equal(r["topk_idx"], o.topk_select(n.astype(np.float32), k))
+    p = np.exp(n - n.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    assert np.allclose(r["probs64"], p, rtol=0, atol=1e-15)
+    assert abs(r["z"] - o.z_loss(n)) < 1e-12
+
+
+ALL_PINS.extend([pin_philox_kat, pin_jitter, pin_logit_noise, pin_z_loss, pin_route_noise])
+

@@ -82,7 +82,32 @@ def _binned_padding_repeats_row(x, row_slot, k):
     return x[np.abs(np.asarray(row_slot, np.int64)) // k]
 
 
-_REAL = {n: getattr(O, n) for n in ("combine", "expert_ffn", "permute", "permute_binned")}
+def _philox_nine_rounds(ctr, key):
+    c = np.asarray(ctr, dtype=np.uint64) & np.uint64(0xFFFFFFFF)
+    c0, c1, c2, c3 = (c[..., i] for i in range(4))
+    k0, k1 = np.uint64(key[0]), np.uint64(key[1])
+    for _ in range(9):
+        p0 = c0 * np.uint64(0xD2511F53)
+        p1 = c2 * np.uint64(0xCD9E8D57)
+        c0, c1, c2, c3 = ((p1 >> np.uint64(32)) ^ c1 ^ k0) & np.uint64(0xFFFFFFFF), p1 & np.uint64(0xFFFFFFFF), \
+            ((p0 >> np.uint64(32)) ^ c3 ^ k1) & np.uint64(0xFFFFFFFF), p0 & np.uint64(0xFFFFFFFF)
+        k0 = (k0 + np.uint64(0x9E3779B9)) & np.uint64(0xFFFFFFFF)
+        k1 = (k1 + np.uint64(0xBB67AE85)) & np.uint64(0xFFFFFFFF)
+    return np.stack([c0, c1, c2, c3], axis=-1).astype(np.uint32)
+
+
+def _z_loss_no_square(logits):
+    l = np.asarray(logits, dtype=np.float64)
+    m = l.max(axis=1, keepdims=True)
+    return float(np.mean(m[:, 0] + np.log(np.exp(l - m).sum(axis=1))))
+
+
+def _jitter_half_width(T, d, eps, seed):
+    return _REAL["jitter_multipliers"](T, d, eps / 2, seed)
+
+
+_REAL = {n: getattr(O, n) for n in ("combine", "expert_ffn", "permute", "permute_binned",
+                                    "jitter_multipliers")}
 
 MUTATIONS = {
     "topk_ties_to_higher_index": ("topk_select", _ties_to_higher),
@@ -98,6 +123,9 @@ MUTATIONS = {
     "drop_off_by_one": ("permute", _permute_drop_gt),
     "binned_dynamic_bin_is_mean_count": ("permute_binned", _binned_bin_is_mean),
     "binned_padding_not_zero": ("gather_binned", _binned_padding_repeats_row),
+    "philox_nine_rounds": ("philox4x32_10", _philox_nine_rounds),
+    "z_loss_without_square": ("z_loss", _z_loss_no_square),
+    "jitter_half_width": ("jitter_multipliers", _jitter_half_width),
 }
 
 
