@@ -99,6 +99,13 @@ typedef struct {
   const void* w3;           /* W_up [E, d, F] (SwiGLU), NULL for GELU */
   const void* w2;           /* W_down / W2 [E, F, d] */
   int flags;                /* MOE_LAYER_* bits, 0 for the default path */
+  /* Training-side router inputs (NULL for inference):
+   *   x_router     the router's input [T, d] (dtype) in place of x, e.g. x
+   *                jittered by moe_router_jitter; the experts still read x
+   *   logit_noise  [T, E] fp32 added to the gate logits after the bias,
+   *                e.g. from moe_router_noise */
+  const void* x_router;
+  const float* logit_noise;
 } moe_layer_t;
 
 /* moe_layer_t.flags. MOE_LAYER_GATHER_IN_GEMM (bf16 only): moe_forward skips
@@ -118,6 +125,9 @@ typedef struct {
  * layout differs. The expert FFN (bf16) skips the padding rows: h and y_perm
  * rows past kept_counts[e] in each bin are not written. */
 #define MOE_LAYER_BINNED 2
+/* MOE_LAYER_Z_LOSS: moe_forward also computes the router z-loss (see
+ * moe_route_train) into the workspace (moe_views_t.z_loss). */
+#define MOE_LAYER_Z_LOSS 4
 
 /* Device pointers into a moe_forward workspace where that call leaves its
  * intermediate results (see moe_forward_views). */
@@ -125,6 +135,7 @@ typedef struct {
   int32_t* topk_idx;     /* [T, k] */
   float* topk_w;         /* [T, k] */
   float* aux_loss;       /* [1] */
+  float* z_loss;         /* [1], written with MOE_LAYER_Z_LOSS */
   int32_t* counts;       /* [E] */
   int32_t* bins;         /* [E] */
   int32_t* kept_counts;  /* [E] */
@@ -187,6 +198,43 @@ MOE_API moe_status_t moe_route(const void* x, const void* w_router, const float*
                        int T, int d, int E, int k, int32_t* topk_idx, float* topk_w,
                        float* aux_loss, float* logits, float* probs, void* ws, size_t ws_bytes,
                        moe_stream_t stream);
+
+/* moe_route with the training-side variants:
+ *   logit_noise  [T, E] fp32 added to each logit after the bias, or NULL
+ *                ("Integrating MoE into your model with Colossal-AI", step 2:
+ *                NormalNoiseGenerator adds Gaussian noise to the gate logits;
+ *                see moe_router_noise)
+ *   z_loss       out [1] fp32 or NULL: mean over tokens of the squared
+ *                log-sum-exp of the logits the softmax sees (bias and noise
+ *                included). The pages name the loss only (router_z_loss);
+ *                this is its usual definition. Deterministic (fixed-order
+ *                reductions).
+ * Probabilities, top-k, weights and the aux loss are those of the noisy
+ * logits. For jitter, pass the jittered x (moe_router_jitter) as x. */
+MOE_API moe_status_t moe_route_train(const void* x, const void* w_router, const float* bias,
+                             const float* logit_noise, moe_dtype_t dtype, int T, int d, int E,
+                             int k, int32_t* topk_idx, float* topk_w, float* aux_loss,
+                             float* z_loss, float* logits, float* probs, void* ws,
+                             size_t ws_bytes, moe_stream_t stream);
+
+/* Router jitter ("MegaBlocks", section 5: the router input is multiplied by
+ * uniform noise in [1 - eps, 1 + eps] during training): x_out = x * m with
+ * m uniform in [1 - eps, 1 + eps) per element, from the counter-based
+ * generator Philox4x32-10 (Salmon et al., SC 2011) keyed by seed. Element n =
+ * t*d + i uses word n % 4 of the generator's call n / 4 on counter
+ * (lo32, hi32, 0, 0): u = (word >> 8) * 2^-24, m = (1 - eps) + (2 eps) u in
+ * fp32, x * m in fp32 (rounded to bf16 for bf16). 0 <= eps < 1. x and x_out
+ * [T, d] (dtype), device; they may not overlap. */
+MOE_API moe_status_t moe_router_jitter(const void* x, moe_dtype_t dtype, int T, int d, float eps,
+                               uint64_t seed, void* x_out, moe_stream_t stream);
+
+/* Gaussian logit noise noise_out [T, E] fp32 (device) = std_dev * N(0, 1), by
+ * Box-Muller from Philox4x32-10: value n = t*E + e uses words 2(n % 2) and
+ * 2(n % 2) + 1 of call n / 2 on counter (lo32, hi32, 1, 0). The Colossal-AI
+ * page scales the noise by the number of experts: std_dev = 1/E in that
+ * reading. */
+MOE_API moe_status_t moe_router_noise(int T, int E, float std_dev, uint64_t seed, float* noise_out,
+                              moe_stream_t stream);
 
 /* ---------------------------------------------------------------- permute
  * Sorting metadata of the T*k slots by expert id ("MegaBlocks", section 4.1:

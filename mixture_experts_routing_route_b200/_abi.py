@@ -23,7 +23,7 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_NULL", 2: "MOE_ERR_INVALID", 3: "MOE_ERR_UNSU
           4: "MOE_ERR_WORKSPACE", 5: "MOE_ERR_ALIGN", 6: "MOE_ERR_CUDA", 7: "MOE_ERR_DEVICE"}
 MOE_F32, MOE_BF16 = 0, 1
 MOE_ACT_GELU, MOE_ACT_SWIGLU = 0, 1
-MOE_LAYER_GATHER_IN_GEMM, MOE_LAYER_BINNED = 1, 2
+MOE_LAYER_GATHER_IN_GEMM, MOE_LAYER_BINNED, MOE_LAYER_Z_LOSS = 1, 2, 4
 DEVERR_EXPERT_RANGE, DEVERR_ROW_RANGE, DEVERR_TIMEOUT = 1, 2, 4
 
 
@@ -50,11 +50,11 @@ class MoeLayerC(ctypes.Structure):
     _fields_ = [("d", c_int), ("E", c_int), ("k", c_int), ("F", c_int), ("dtype", c_int),
                 ("act", c_int), ("capacity_factor", c_double), ("w_router", c_void_p),
                 ("router_bias", c_void_p), ("w1", c_void_p), ("w3", c_void_p), ("w2", c_void_p),
-                ("flags", c_int)]
+                ("flags", c_int), ("x_router", c_void_p), ("logit_noise", c_void_p)]
 
 
 class MoeViewsC(ctypes.Structure):
-    _fields_ = [(n, c_void_p) for n in ("topk_idx", "topk_w", "aux_loss", "counts", "bins",
+    _fields_ = [(n, c_void_p) for n in ("topk_idx", "topk_w", "aux_loss", "z_loss", "counts", "bins",
                                         "kept_counts", "seg_offsets", "sorted_slot",
                                         "slot_to_row", "row_slot", "drop_mask", "x_perm", "h",
                                         "y_perm")] + [("rows_max", c_int64), ("capacity", c_int64)]
@@ -76,6 +76,12 @@ _SIGS = {
                     + [c_void_p, c_size_t, c_void_p]),
     "moe_permute_noalloc": (c_int, [c_void_p, c_int, c_int, c_int, c_int64] + [c_void_p] * 9
                             + [c_void_p]),
+    "moe_route_train": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int,
+                                c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                c_void_p, c_size_t, c_void_p]),
+    "moe_router_jitter": (c_int, [c_void_p, c_int, c_int, c_int, ctypes.c_float, ctypes.c_uint64,
+                                  c_void_p, c_void_p]),
+    "moe_router_noise": (c_int, [c_int, c_int, ctypes.c_float, ctypes.c_uint64, c_void_p, c_void_p]),
     "moe_permute_binned": (c_int, [c_void_p, c_int, c_int, c_int, c_int64] + [c_void_p] * 8
                            + [c_void_p, c_size_t, c_void_p]),
     "moe_rows_max_binned": (c_int64, [c_int, c_int, c_int, c_int64]),
@@ -184,6 +190,24 @@ def moe_route(x, w_router, bias, T, d, E, k, topk_idx, topk_w, aux_loss, logits,
         _ptr(x), _ptr(w_router), _ptr(bias), dtype_code(x.dtype), T, d, E, k, _ptr(topk_idx),
         _ptr(topk_w), _ptr(aux_loss), _ptr(logits), _ptr(probs), _ptr(ws), ws.numel(),
         _stream(stream)))
+
+
+def moe_route_train(x, w_router, bias, logit_noise, T, d, E, k, topk_idx, topk_w, aux_loss, z_loss,
+                    logits, probs, ws, stream=None):
+    _check("moe_route_train", _lib.moe_route_train(
+        _ptr(x), _ptr(w_router), _ptr(bias), _ptr(logit_noise), dtype_code(x.dtype), T, d, E, k,
+        _ptr(topk_idx), _ptr(topk_w), _ptr(aux_loss), _ptr(z_loss), _ptr(logits), _ptr(probs),
+        _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_router_jitter(x, T, d, eps, seed, x_out, stream=None):
+    _check("moe_router_jitter", _lib.moe_router_jitter(
+        _ptr(x), dtype_code(x.dtype), T, d, float(eps), int(seed), _ptr(x_out), _stream(stream)))
+
+
+def moe_router_noise(T, E, std, seed, noise_out, stream=None):
+    _check("moe_router_noise", _lib.moe_router_noise(T, E, float(std), int(seed), _ptr(noise_out),
+                                                     _stream(stream)))
 
 
 def moe_permute(topk_idx, T, k, E, capacity, counts, bins, sorted_slot, slot_to_row, row_slot,

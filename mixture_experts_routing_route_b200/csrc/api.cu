@@ -84,6 +84,7 @@ struct FwdLayout {
   int32_t* idx;
   float* w;
   float* aux;
+  float* z;  // z-loss (MOE_LAYER_Z_LOSS)
   int32_t *counts, *bins, *kept, *seg;
   int32_t *sorted_slot, *slot_to_row, *row_slot;
   uint8_t* drop;
@@ -115,6 +116,7 @@ FwdLayout fwd_layout(const moe_layer_t* L, int T, void* ws, bool host_io) {
   f.idx = static_cast<int32_t*>(c.take(S * 4));
   f.w = static_cast<float*>(c.take(S * 4));
   f.aux = static_cast<float*>(c.take(4));
+  f.z = static_cast<float*>(c.take(4));
   f.counts = static_cast<int32_t*>(c.take(L->E * 4));
   f.bins = static_cast<int32_t*>(c.take(L->E * 4));
   f.kept = static_cast<int32_t*>(c.take(L->E * 4));
@@ -143,7 +145,10 @@ moe_status_t check_layer(const moe_layer_t* L, int T) {
   MOE_CHECK(check_ffn(L->dtype, L->F));
   if (L->act != MOE_ACT_GELU && L->act != MOE_ACT_SWIGLU) return MOE_ERR_INVALID;
   if (!std::isfinite(L->capacity_factor)) return MOE_ERR_INVALID;
-  if ((L->flags & ~(MOE_LAYER_GATHER_IN_GEMM | MOE_LAYER_BINNED)) != 0) return MOE_ERR_INVALID;
+  if ((L->flags & ~(MOE_LAYER_GATHER_IN_GEMM | MOE_LAYER_BINNED | MOE_LAYER_Z_LOSS)) != 0)
+    return MOE_ERR_INVALID;
+  MOE_OPT(L->x_router);
+  MOE_OPT(L->logit_noise);
   if ((L->flags & MOE_LAYER_GATHER_IN_GEMM) && L->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   MOE_NEED(L->w_router);
   MOE_NEED(L->w1);
@@ -160,9 +165,11 @@ moe_status_t run_forward(const moe_layer_t* L, const void* x, int T, void* out, 
   };
   const size_t es = esize(L->dtype);
   rec(0);
-  MOE_CHECK(from_cuda(launch_route(x, L->w_router, L->router_bias, L->dtype, T, L->d, L->E, L->k,
-                                   f.idx, f.w, f.aux, nullptr, nullptr, f.logits_scratch,
-                                   f.partials, f.ctl, s)));
+  // the router may read its own input (a jittered x) and add logit noise
+  MOE_CHECK(from_cuda(launch_route(L->x_router != nullptr ? L->x_router : x, L->w_router,
+                                   L->router_bias, L->logit_noise, L->dtype, T, L->d, L->E, L->k,
+                                   f.idx, f.w, f.aux, (L->flags & MOE_LAYER_Z_LOSS) ? f.z : nullptr,
+                                   nullptr, nullptr, f.logits_scratch, f.partials, f.ctl, s)));
   rec(1);
   MOE_CHECK(from_cuda(launch_permute(f.idx, T, L->k, L->E, f.cap, f.counts, f.bins, f.sorted_slot,
                                      f.slot_to_row, f.row_slot, f.drop, f.kept, f.seg, f.rank,
@@ -262,9 +269,11 @@ size_t moe_route_workspace_size(int T, int d, int E) {
   return align_up(sizeof(Control)) + route_partials_bytes(T, E) + route_logits_scratch_bytes(T, d, E);
 }
 
-moe_status_t moe_route(const void* x, const void* w_router, const float* bias, moe_dtype_t dtype,
-                       int T, int d, int E, int k, int32_t* topk_idx, float* topk_w, float* aux_loss,
-                       float* logits, float* probs, void* ws, size_t ws_bytes, moe_stream_t stream) {
+static moe_status_t route_impl(const void* x, const void* w_router, const float* bias,
+                               const float* logit_noise, moe_dtype_t dtype, int T, int d, int E,
+                               int k, int32_t* topk_idx, float* topk_w, float* aux_loss,
+                               float* z_loss, float* logits, float* probs, void* ws,
+                               size_t ws_bytes, moe_stream_t stream) {
   MOE_CHECK(check_dims(dtype, T, d, E, k));
   MOE_NEED(x);
   MOE_NEED(w_router);
@@ -273,6 +282,8 @@ moe_status_t moe_route(const void* x, const void* w_router, const float* bias, m
   MOE_NEED(aux_loss);
   MOE_NEED(ws);
   MOE_OPT(bias);
+  MOE_OPT(logit_noise);
+  MOE_OPT(z_loss);
   MOE_OPT(logits);
   MOE_OPT(probs);
   if (ws_bytes < moe_route_workspace_size(T, d, E)) return MOE_ERR_WORKSPACE;
@@ -280,9 +291,45 @@ moe_status_t moe_route(const void* x, const void* w_router, const float* bias, m
   Control* ctl = static_cast<Control*>(c.take(sizeof(Control)));
   void* partials = c.take(route_partials_bytes(T, E));
   float* scratch = static_cast<float*>(c.take(route_logits_scratch_bytes(T, d, E)));
-  return from_cuda(launch_route(x, w_router, bias, dtype, T, d, E, k, topk_idx, topk_w, aux_loss,
-                                logits, probs, scratch, partials, ctl,
+  return from_cuda(launch_route(x, w_router, bias, logit_noise, dtype, T, d, E, k, topk_idx, topk_w,
+                                aux_loss, z_loss, logits, probs, scratch, partials, ctl,
                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_route(const void* x, const void* w_router, const float* bias, moe_dtype_t dtype,
+                       int T, int d, int E, int k, int32_t* topk_idx, float* topk_w, float* aux_loss,
+                       float* logits, float* probs, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  return route_impl(x, w_router, bias, nullptr, dtype, T, d, E, k, topk_idx, topk_w, aux_loss,
+                    nullptr, logits, probs, ws, ws_bytes, stream);
+}
+
+moe_status_t moe_route_train(const void* x, const void* w_router, const float* bias,
+                             const float* logit_noise, moe_dtype_t dtype, int T, int d, int E, int k,
+                             int32_t* topk_idx, float* topk_w, float* aux_loss, float* z_loss,
+                             float* logits, float* probs, void* ws, size_t ws_bytes,
+                             moe_stream_t stream) {
+  return route_impl(x, w_router, bias, logit_noise, dtype, T, d, E, k, topk_idx, topk_w, aux_loss,
+                    z_loss, logits, probs, ws, ws_bytes, stream);
+}
+
+moe_status_t moe_router_jitter(const void* x, moe_dtype_t dtype, int T, int d, float eps,
+                               uint64_t seed, void* x_out, moe_stream_t stream) {
+  if (dtype != MOE_BF16 && dtype != MOE_F32) return MOE_ERR_INVALID;
+  if (T < 0 || d <= 0 || !(eps >= 0.0f && eps < 1.0f)) return MOE_ERR_INVALID;
+  if (T > 0) {
+    MOE_NEED(x);
+    MOE_NEED(x_out);
+  }
+  return from_cuda(launch_jitter(x, dtype, static_cast<long long>(T) * d, eps, seed, x_out,
+                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_router_noise(int T, int E, float std_dev, uint64_t seed, float* noise_out,
+                              moe_stream_t stream) {
+  if (T < 0 || E < 1 || !(std_dev >= 0.0f) || !std::isfinite(std_dev)) return MOE_ERR_INVALID;
+  if (T > 0) MOE_NEED(noise_out);
+  return from_cuda(launch_logit_noise(static_cast<long long>(T) * E, std_dev, seed, noise_out,
+                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t moe_permute_workspace_size(int T, int k, int E) {
@@ -422,6 +469,7 @@ moe_status_t moe_forward_views(const moe_layer_t* layer, int T, void* ws, size_t
   v->topk_idx = f.idx;
   v->topk_w = f.w;
   v->aux_loss = f.aux;
+  v->z_loss = f.z;
   v->counts = f.counts;
   v->bins = f.bins;
   v->kept_counts = f.kept;

@@ -102,10 +102,12 @@ cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, si
 // Router. Tokens per block of the general path (partials are per block).
 constexpr int kRouteSelectTokensPerBlock = 64;
 size_t route_partials_bytes(int T, int E);
-cudaError_t launch_route(const void* x, const void* wg, const float* bias, moe_dtype_t dt, int T,
-                         int d, int E, int k, int32_t* idx, float* w, float* aux, float* logits,
-                         float* probs, float* logits_scratch, void* partials, Control* ctl,
-                         cudaStream_t s);
+// noise: optional [T, E] fp32 added to the logits after the bias; z_out:
+// optional z-loss output (mean over tokens of the squared log-sum-exp).
+cudaError_t launch_route(const void* x, const void* wg, const float* bias, const float* noise,
+                         moe_dtype_t dt, int T, int d, int E, int k, int32_t* idx, float* w,
+                         float* aux, float* z_out, float* logits, float* probs,
+                         float* logits_scratch, void* partials, Control* ctl, cudaStream_t s);
 size_t route_logits_scratch_bytes(int T, int d, int E);
 
 // Permute. launch_permute picks the multi-CTA kernel when the slots fit its
@@ -124,6 +126,13 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int64_t cap,
                            int32_t* row_slot, uint8_t* drop, int32_t* kept, int32_t* seg,
                            int32_t* rank_scratch, Control* ctl, cudaStream_t s,
                            bool binned = false);
+
+// Router training inputs (noise.cu): x' = x * uniform(1 - eps, 1 + eps)
+// elementwise (n elements, dtype dt), and std * N(0, 1) logit noise (n
+// values, fp32), both from Philox4x32-10 keyed by seed.
+cudaError_t launch_jitter(const void* x, moe_dtype_t dt, long long n, float eps, uint64_t seed,
+                          void* out, cudaStream_t s);
+cudaError_t launch_logit_noise(long long n, float std, uint64_t seed, float* out, cudaStream_t s);
 
 // Gather. binned: rows with row_slot -1 are padding and are written as zeros.
 cudaError_t launch_gather(const void* x, size_t elem, int T, int d, int k, const int32_t* row_slot,

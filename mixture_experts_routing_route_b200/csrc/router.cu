@@ -52,8 +52,10 @@ __device__ __forceinline__ void block_write_partials(const float* blk_p, const i
 constexpr int kAuxThreads = 256;
 
 __global__ void __launch_bounds__(kAuxThreads)
-aux_reduce(const float* __restrict__ part_p, const int32_t* __restrict__ part_c, int ldb, int nblk,
-           int E, int T, int k, double* __restrict__ terms, float* __restrict__ aux, Control* ctl) {
+aux_reduce(const float* __restrict__ part_p, const int32_t* __restrict__ part_c,
+           const float* __restrict__ part_z, int ldb, int nblk, int E, int T, int k,
+           double* __restrict__ terms, float* __restrict__ aux, float* __restrict__ z_out,
+           Control* ctl) {
   pdl_begin();
   __shared__ double sp[kAuxThreads];
   __shared__ long long sc[kAuxThreads];
@@ -86,10 +88,20 @@ aux_reduce(const float* __restrict__ part_p, const int32_t* __restrict__ part_c,
     if (threadIdx.x < s) sp[threadIdx.x] += sp[threadIdx.x + s];
     __syncthreads();
   }
-  if (threadIdx.x == 0) {
-    *aux = static_cast<float>(E * sp[0]);
-    ctl->route_ticket = 0u;
+  if (threadIdx.x == 0) *aux = static_cast<float>(E * sp[0]);
+  if (z_out != nullptr) {  // z-loss: the blocks' partials in a fixed order, then / T
+    __syncthreads();
+    double zs = 0.0;
+    for (int b = threadIdx.x; b < nblk; b += kAuxThreads) zs += static_cast<double>(__ldcg(part_z + b));
+    sp[threadIdx.x] = zs;
+    __syncthreads();
+    for (int s = kAuxThreads / 2; s > 0; s >>= 1) {
+      if (threadIdx.x < s) sp[threadIdx.x] += sp[threadIdx.x + s];
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) *z_out = T > 0 ? static_cast<float>(sp[0] / T) : 0.f;
   }
+  if (threadIdx.x == 0) ctl->route_ticket = 0u;
 }
 
 // ---------------------------------------------------------------- fused, E <= 8
@@ -413,7 +425,7 @@ router_gemm_tiled(const Tin* __restrict__ x, const Tin* __restrict__ wg, int T, 
 // rounds of a warp arg-max (ties to the lower expert), renormalised weights;
 // accumulates the token's probabilities and choices into the lane's aux sums.
 template <int EPL>
-__device__ __forceinline__ void warp_route_token(const float (&v)[EPL], int E, int k, int lane,
+__device__ __forceinline__ float warp_route_token(const float (&v)[EPL], int E, int k, int lane,
                                                  size_t t, int32_t* __restrict__ idx_out,
                                                  float* __restrict__ w_out,
                                                  float* __restrict__ logits_out,
@@ -491,6 +503,7 @@ __device__ __forceinline__ void warp_route_token(const float (&v)[EPL], int E, i
     idx_out[t * k + lane] = my_e;
     w_out[t * k + lane] = my_p / wsum;
   }
+  return m + logf(s);  // log-sum-exp of the logits (the z-loss term), same in every lane
 }
 
 // Warp per token: lane l holds experts l + 32q, q < EPL. The logits are the
@@ -501,11 +514,13 @@ constexpr int kSelectTokensPerBlock = kSelectWarps * kSelectTokensPerWarp;
 
 template <int EPL>
 __global__ void __launch_bounds__(kSelectWarps * 32)
-router_select(const float* __restrict__ logits_in, int KS, const float* __restrict__ bias, int T,
-              int E, int k, int32_t* __restrict__ idx_out, float* __restrict__ w_out,
-              float* __restrict__ logits_out, float* __restrict__ probs_out,
-              float* __restrict__ part_p, int32_t* __restrict__ part_c, int ldb, Control* ctl) {
+router_select(const float* __restrict__ logits_in, int KS, const float* __restrict__ bias,
+              const float* __restrict__ noise, int T, int E, int k, int32_t* __restrict__ idx_out,
+              float* __restrict__ w_out, float* __restrict__ logits_out,
+              float* __restrict__ probs_out, float* __restrict__ part_p,
+              int32_t* __restrict__ part_c, float* __restrict__ part_z, int ldb, Control* ctl) {
   pdl_begin();
+  __shared__ float zw[kSelectWarps];
   __shared__ float blk_p_w[kSelectWarps][256];
   __shared__ int32_t blk_c_w[kSelectWarps][256];
   __shared__ float tot_p[256];
@@ -522,6 +537,7 @@ router_select(const float* __restrict__ logits_in, int KS, const float* __restri
     bq[q] = (bias != nullptr && e < E) ? bias[e] : 0.f;
   }
   const size_t plane = static_cast<size_t>(T) * E;
+  float zacc = 0.f;  // this warp's sum of squared log-sum-exp (z-loss)
   const int t_begin = blockIdx.x * kSelectTokensPerBlock;
   const int t_end = min(T, t_begin + kSelectTokensPerBlock);
   for (int t = t_begin + warp; t < t_end; t += kSelectWarps) {
@@ -541,11 +557,15 @@ router_select(const float* __restrict__ logits_in, int KS, const float* __restri
 #pragma unroll
       for (int src = 0; src < 8; ++src)
         if (src < KS) acc += pv[src][q];
-      v[q] = (lane + 32 * q < E) ? acc + bq[q] : -INFINITY;
+      const int e = lane + 32 * q;
+      v[q] = e < E ? acc + bq[q] : -INFINITY;
+      if (noise != nullptr && e < E) v[q] += __ldg(noise + static_cast<size_t>(t) * E + e);
     }
-    warp_route_token<EPL>(v, E, k, lane, static_cast<size_t>(t), idx_out, w_out, logits_out,
-                          probs_out, psum, cnt, ctl);
+    const float lse = warp_route_token<EPL>(v, E, k, lane, static_cast<size_t>(t), idx_out, w_out,
+                                            logits_out, probs_out, psum, cnt, ctl);
+    zacc += lse * lse;
   }
+  if (lane == 0) zw[warp] = zacc;
 #pragma unroll
   for (int q = 0; q < EPL; ++q) {
     const int e = lane + 32 * q;
@@ -561,6 +581,11 @@ router_select(const float* __restrict__ logits_in, int KS, const float* __restri
   }
   __syncthreads();
   block_write_partials(tot_p, tot_c, part_p, part_c, ldb, E);
+  if (part_z != nullptr && threadIdx.x == 0) {
+    float z = 0.f;
+    for (int w = 0; w < kSelectWarps; ++w) z += zw[w];
+    part_z[blockIdx.x] = z;
+  }
 }
 
 // ---------------------------------------------------------------- tensor cores
@@ -588,6 +613,9 @@ struct RouterTcArgs {
   int32_t* idx;
   float *w, *logits, *probs, *part_p, *aux;
   int32_t* part_c;
+  const float* noise;  // [T, E] added to the logits, or null
+  float* part_z;       // per-tile z-loss partials, or null (no z-loss)
+  float* z_out;        // the z-loss, or null
 };
 
 // Fused selection, E <= 32. The KS CTAs of one 128-token tile run as a
@@ -676,6 +704,7 @@ __device__ __forceinline__ void fused_select_epilogue(const RouterTcArgs& a, uin
 #pragma unroll
   for (int e = 0; e < EW; ++e) {
     lg[e] = e < E ? v[e] + (a.bias != nullptr ? __ldg(a.bias + e) : 0.f) : -INFINITY;
+    if (a.noise != nullptr && e < E && t < a.T) lg[e] += __ldg(a.noise + static_cast<size_t>(t) * E + e);
     m = fmaxf(m, lg[e]);
   }
   float ssum = 0.f;
@@ -726,6 +755,17 @@ __device__ __forceinline__ void fused_select_epilogue(const RouterTcArgs& a, uin
         a.w[static_cast<size_t>(t) * a.k + j] = sel_p[j] / wsum;
       }
   }
+  // ---- z-loss partial of this tile: lse^2 per token, a fixed butterfly per
+  // warp, then the 4 warps in order.
+  __shared__ float zw_s[kTcThreads / 32];
+  __shared__ double zd_s[kTcThreads];
+  if (a.part_z != nullptr) {
+    const float lse = m + logf(ssum);
+    float zt = valid ? lse * lse : 0.f;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) zt += __shfl_xor_sync(kFull, zt, off);
+    if (lane == 0) zw_s[warp] = zt;
+  }
   // ---- aux partials of this tile: thread (e, part) adds rows part, part +
   // kParts, ... of expert e; then the kParts sums are added in part order.
 #pragma unroll
@@ -754,6 +794,8 @@ __device__ __forceinline__ void fused_select_epilogue(const RouterTcArgs& a, uin
     a.part_p[static_cast<size_t>(r) * a.ldb + tile] = ps;
     a.part_c[static_cast<size_t>(r) * a.ldb + tile] = cs;
   }
+  if (a.part_z != nullptr && r == 0)
+    a.part_z[tile] = ((zw_s[0] + zw_s[1]) + zw_s[2]) + zw_s[3];
   __syncthreads();
   if (r == 0) {
     __threadfence();
@@ -791,8 +833,19 @@ __device__ __forceinline__ void fused_select_epilogue(const RouterTcArgs& a, uin
       tot += (static_cast<double>(cs) / (static_cast<double>(a.T) * a.k)) * (ps / a.T);
     }
     *a.aux = static_cast<float>(E * tot);
-    a.ctl->route_ticket = 0u;
   }
+  if (a.part_z != nullptr) {  // z-loss: tiles r, r + 128, ... then a fixed tree, / T
+    double zs = 0.0;
+    for (int b = r; b < a.ntile; b += kTcThreads) zs += static_cast<double>(__ldcg(a.part_z + b));
+    zd_s[r] = zs;
+    __syncthreads();
+    for (int st = kTcThreads / 2; st > 0; st >>= 1) {
+      if (r < st) zd_s[r] += zd_s[r + st];
+      __syncthreads();
+    }
+    if (r == 0) *a.z_out = static_cast<float>(zd_s[0] / a.T);
+  }
+  if (r == 0) a.ctl->route_ticket = 0u;
 }
 
 // kFuseE = 0: partial logits out (router_select follows); 8, 16 or 32: the
@@ -1067,8 +1120,10 @@ static int route_max_blocks(int T) {
 }
 
 size_t route_partials_bytes(int T, int E) {
-  // per-block sums then counts (expert-major), then the per-expert terms
-  return align_up(static_cast<size_t>(route_max_blocks(T)) * E * 4) * 2 + align_up(256 * 8);
+  // per-block sums then counts (expert-major), the per-expert terms, the
+  // per-block z-loss sums
+  return align_up(static_cast<size_t>(route_max_blocks(T)) * E * 4) * 2 + align_up(256 * 8) +
+         align_up(static_cast<size_t>(route_max_blocks(T)) * 4);  // z-loss partials
 }
 
 size_t route_logits_scratch_bytes(int T, int d, int E) {
@@ -1076,18 +1131,22 @@ size_t route_logits_scratch_bytes(int T, int d, int E) {
   return align_up(static_cast<size_t>(kMaxKS) * T * E * 4);
 }
 
-cudaError_t launch_route(const void* x, const void* wg, const float* bias, moe_dtype_t dt, int T,
-                         int d, int E, int k, int32_t* idx, float* w, float* aux, float* logits,
-                         float* probs, float* logits_scratch, void* partials, Control* ctl,
-                         cudaStream_t s) {
+cudaError_t launch_route(const void* x, const void* wg, const float* bias, const float* noise,
+                         moe_dtype_t dt, int T, int d, int E, int k, int32_t* idx, float* w,
+                         float* aux, float* z_out, float* logits, float* probs,
+                         float* logits_scratch, void* partials, Control* ctl, cudaStream_t s) {
   const int ldb = route_max_blocks(T);
   float* part_p = static_cast<float*>(partials);
   int32_t* part_c = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(partials) +
                                                align_up(static_cast<size_t>(ldb) * E * 4));
   double* terms = reinterpret_cast<double*>(static_cast<uint8_t*>(partials) +
                                             2 * align_up(static_cast<size_t>(ldb) * E * 4));
+  float* part_z = z_out == nullptr ? nullptr
+                                   : reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(terms) +
+                                                              align_up(256 * 8));
   int nblk = 0;
-  if (use_fused(d, E, dt)) {
+  // The fp32 E <= 8 kernel has neither the noise input nor the z-loss.
+  if (use_fused(d, E, dt) && noise == nullptr && z_out == nullptr) {
     const int groups = (T + kFusedTokensPerGroup - 1) / kFusedTokensPerGroup;
     const int grid = std::max(1, std::min(groups, num_sms()));
     const size_t smem = fused_smem_bytes(d);
@@ -1122,6 +1181,7 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, moe_d
         a.bias = bias; a.k = k; a.ntile = tp.ntile; a.ldb = ldb;
         a.idx = idx; a.w = w; a.logits = logits; a.probs = probs;
         a.part_p = part_p; a.part_c = part_c; a.aux = aux;
+        a.noise = noise; a.part_z = part_z; a.z_out = z_out;
         auto kern = tp.fuse_e == 8 ? router_tc<false, 8>
                   : tp.fuse_e == 16 ? router_tc<false, 16> : router_tc<false, 32>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1153,14 +1213,14 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, moe_d
              : epl <= 4 ? router_select<4>
                         : router_select<8>;
     const cudaError_t e = launch_pdl(sel, dim3(g2), dim3(kSelectWarps * 32), 0, s, false,
-                                     static_cast<const float*>(logits_scratch), KS, bias, T, E, k,
-                                     idx, w, logits, probs, part_p, part_c, ldb, ctl);
+                                     static_cast<const float*>(logits_scratch), KS, bias, noise, T,
+                                     E, k, idx, w, logits, probs, part_p, part_c, part_z, ldb, ctl);
     if (e != cudaSuccess) return e;
     nblk = g2;
   }
   return launch_pdl(aux_reduce, dim3(E), dim3(kAuxThreads), 0, s, false,
-                    static_cast<const float*>(part_p), static_cast<const int32_t*>(part_c), ldb,
-                    nblk, E, T, k, terms, aux, ctl);
+                    static_cast<const float*>(part_p), static_cast<const int32_t*>(part_c),
+                    static_cast<const float*>(part_z), ldb, nblk, E, T, k, terms, aux, z_out, ctl);
 }
 
 }  // namespace moe

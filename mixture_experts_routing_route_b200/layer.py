@@ -18,7 +18,7 @@ class MoeLayer:
     def __init__(self, w_router: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
                  w3: Optional[torch.Tensor] = None, bias: Optional[torch.Tensor] = None,
                  k: int = 2, act: str = "swiglu", capacity_factor: float = 0.0,
-                 gather_in_gemm: bool = False, binned: bool = False):
+                 gather_in_gemm: bool = False, binned: bool = False, z_loss: bool = False):
         if not w1.is_cuda:
             raise ValueError("weights must be CUDA tensors")
         self.E, self.d, self.F = w1.shape
@@ -36,7 +36,7 @@ class MoeLayer:
         # binned: the [E, C, hs] bucket layout (MOE_LAYER_BINNED); with
         # capacity_factor <= 0 the bin size is the call's largest expert count
         flags = (abi.MOE_LAYER_GATHER_IN_GEMM if gather_in_gemm else 0) | \
-            (abi.MOE_LAYER_BINNED if binned else 0)
+            (abi.MOE_LAYER_BINNED if binned else 0) | (abi.MOE_LAYER_Z_LOSS if z_loss else 0)
         self.c = abi.layer_struct(self.d, self.E, k, self.F, abi.dtype_code(self.dtype), self.act,
                                   self.cf, self.w_router, self.bias, self.w1, self.w3, self.w2,
                                   flags)
@@ -55,8 +55,14 @@ class MoeLayer:
         return self._ws[key]
 
     def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None,
-                aux: Optional[torch.Tensor] = None, stream=None, events=None):
+                aux: Optional[torch.Tensor] = None, stream=None, events=None,
+                x_router: Optional[torch.Tensor] = None,
+                logit_noise: Optional[torch.Tensor] = None):
+        """x_router: the router's own input (e.g. moe_router_jitter of x);
+        logit_noise: [T, E] fp32 added to the gate logits (training variants)."""
         T = x.shape[0]
+        self.c.x_router = None if x_router is None else x_router.data_ptr()
+        self.c.logit_noise = None if logit_noise is None else logit_noise.data_ptr()
         if out is None:
             out = torch.empty(T, self.d, dtype=self.dtype, device=x.device)
         if aux is None:
@@ -73,6 +79,8 @@ class MoeLayer:
         `stream`. Calls that overlap (double-buffered serving on two streams)
         pass different `slot`s so they use different workspaces."""
         T = x_host.shape[0]
+        self.c.x_router = None
+        self.c.logit_noise = None
         ws = self.workspace(T, host_io=True, stream=stream, slot=slot)
         abi.moe_forward_host(self.c, x_host, T, out_host, aux_host, ws, stream)
 
@@ -96,6 +104,7 @@ class MoeLayer:
             "topk_idx": view(v.topk_idx, S, torch.int32, (T, self.k)),
             "topk_w": view(v.topk_w, S, torch.float32, (T, self.k)),
             "aux": view(v.aux_loss, 1, torch.float32, (1,)),
+            "z_loss": view(v.z_loss, 1, torch.float32, (1,)),
             "counts": view(v.counts, self.E, torch.int32, (self.E,)),
             "bins": view(v.bins, self.E, torch.int32, (self.E,)),
             "kept_counts": view(v.kept_counts, self.E, torch.int32, (self.E,)),

@@ -192,3 +192,35 @@ def test_layer_binned(T, d, E, k, F, act, dt, cf, bias):
     live = bn["row_slot"] >= 0
     tol = TOL_BF16_OUT if dt == "bf16" else TOL_F32_OUT
     assert max_err_ratio(np32(v["y_perm"])[:bn["rows"]][live], y_ref[live]) <= tol
+
+
+def test_layer_training_router_inputs():
+    """The router reads jittered x and adds logit noise while the experts read
+    x; the z-loss comes back through the views."""
+    from mixture_experts_routing_route_b200 import MoeLayer, _abi as abi
+    T, d, E, k, F = 700, 256, 8, 2, 256
+    inp = small_case("train", T=T, d=d, E=E, k=k, F=F, act="swiglu", seed=77)
+    dv = device_inputs(inp)
+    xj = torch.empty_like(dv["x"])
+    abi.moe_router_jitter(dv["x"], T, d, 0.01, 5, xj)
+    noise = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    abi.moe_router_noise(T, E, 1.0 / E, 6, noise)
+    layer = MoeLayer(dv["wg"], dv["w1"], dv["w2"], w3=dv["w3"], k=k, act="swiglu", z_loss=True)
+    out, aux = layer.forward(dv["x"], x_router=xj, logit_noise=noise)
+    torch.cuda.synchronize()
+    assert layer.device_error(T) == 0
+    v = layer.views(T)
+    xj_ref = O.apply_jitter(np32(inp.x), O.jitter_multipliers(T, d, 0.01, 5), True)
+    assert np.array_equal(np32(xj), xj_ref)
+    r = O.route(xj_ref, np32(inp.wg), None, k, noise=np32(noise).astype(np.float64))
+    g_idx = npi(v["topk_idx"]).astype(np.int64)
+    check_topk_end_to_end(g_idx, r)
+    w_ref = O.renormalise(r["probs64"], g_idx)
+    assert rel_err(np32(v["topk_w"]), w_ref) <= TOL_PROB_REL
+    assert abs(float(v["z_loss"].item()) - r["z"]) <= TOL_AUX_REL * r["z"]
+    pm = O.permute(g_idx, E, None)
+    xp = O.gather(np32(inp.x), pm["row_slot"], k)      # the experts see x, not the jittered x
+    y_ref = O.expert_ffn(xp, pm["seg_offsets"], ExpertWeights(inp.w1), ExpertWeights(inp.w3),
+                         ExpertWeights(inp.w2), "swiglu")
+    out_ref = O.combine(y_ref, w_ref, pm["slot_to_row"], T, k)
+    assert max_err_ratio(np32(out), out_ref) <= TOL_BF16_OUT

@@ -313,3 +313,68 @@ def test_permute_binned_skewed_dynamic():
     assert g["err"] == 0 and g["seg_offsets"][1] == ref["bin"] == ref["counts"].max()
     assert np.array_equal(g["row_slot"][:ref["rows"]], ref["row_slot"])
     assert np.array_equal(g["slot_to_row"][:T * k], ref["slot_to_row"])
+
+
+@pytest.mark.parametrize("T,d,dt", [(37, 128, "bf16"), (1000, 512, "f32"), (4096, 4096, "bf16")])
+def test_router_jitter_matches_oracle(T, d, dt):
+    """Philox4x32-10 multipliers and x * m (MegaBlocks page, section 5), bit
+    for bit: the same generator and the same fp32 operations on both sides."""
+    g = torch.Generator().manual_seed(T)
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float32
+    x = torch.randn(T, d, generator=g).to(tdt)
+    out = torch.empty(T, d, dtype=tdt, device=DEV)
+    seed = 0x1234_5678_9ABC + T
+    abi.moe_router_jitter(x.to(DEV), T, d, 0.01, seed, out)
+    torch.cuda.synchronize()
+    m = O.jitter_multipliers(T, d, 0.01, seed)
+    ref = O.apply_jitter(np32(x), m, dt == "bf16")
+    assert np.array_equal(np32(out), ref)
+
+
+@pytest.mark.parametrize("T,E", [(33, 8), (4096, 64), (999, 7)])
+def test_router_noise_matches_oracle(T, E):
+    """Box-Muller normals from the same Philox words: fp32 on the GPU, float64
+    in the oracle."""
+    out = torch.empty(T, E, dtype=torch.float32, device=DEV)
+    abi.moe_router_noise(T, E, 1.0 / E, 99 + T, out)
+    torch.cuda.synchronize()
+    ref = O.logit_noise(T, E, 1.0 / E, 99 + T)
+    g = np32(out).astype(np.float64)
+    assert np.all(np.abs(g - ref) <= 2e-6 * (1.0 + np.abs(ref) * E))
+
+
+@pytest.mark.parametrize("T,d,E,k,dt", [
+    (1000, 1024, 8, 2, "bf16"),    # fused tensor-core router, KS split in a cluster
+    (300, 512, 32, 4, "bf16"),     # fused, E = 32
+    (513, 256, 64, 2, "bf16"),     # tensor cores (TMA Wg) + router_select + aux_reduce
+    (90, 64, 40, 4, "f32"),        # CUDA-core gate + router_select
+    (200, 64, 4, 1, "f32"),        # fp32 E <= 8: the general path when noise / z-loss are asked
+])
+def test_route_train(T, d, E, k, dt):
+    """moe_route_train: logits = x Wg + b + noise; top-k, weights, aux loss and
+    the z-loss of those logits, against the oracle."""
+    inp = small_case("rt", T=T, d=d, E=E, k=k, F=128, act="gelu", dtype=dt, bias="zipf", seed=T + E)
+    noise = torch.empty(T, E, dtype=torch.float32, device=DEV)
+    abi.moe_router_noise(T, E, 1.0 / E, 7, noise)
+    idx = torch.empty(T, k, dtype=torch.int32, device=DEV)
+    w = torch.empty(T, k, dtype=torch.float32, device=DEV)
+    aux = torch.empty(1, dtype=torch.float32, device=DEV)
+    z = torch.empty(1, dtype=torch.float32, device=DEV)
+    logits = torch.empty(T, E, dtype=torch.float32, device=DEV)
+    probs = torch.empty(T, E, dtype=torch.float32, device=DEV)
+    ws = new_ws(abi.moe_route_workspace_size(T, d, E))
+    abi.moe_route_train(inp.x.to(DEV), inp.wg.to(DEV), inp.bias.to(DEV), noise, T, d, E, k, idx, w,
+                        aux, z, logits, probs, ws)
+    torch.cuda.synchronize()
+    assert abi.moe_get_device_error(ws) == 0
+    n64 = np32(noise).astype(np.float64)
+    r = O.route(np32(inp.x), np32(inp.wg), inp.bias.numpy(), k, noise=n64)
+    g_logits = np32(logits)
+    assert np.max(np.abs(g_logits - r["logits"])) <= 1e-5 * max(1.0, np.max(np.abs(r["logits"])))
+    assert np.array_equal(npi(idx), O.topk_select(g_logits, k))
+    assert rel_err(np32(probs), r["probs64"]) <= TOL_PROB_REL
+    g_idx = npi(idx).astype(np.int64)
+    assert rel_err(np32(w), O.renormalise(r["probs64"], g_idx)) <= TOL_PROB_REL
+    aux_ref = O.aux_loss(r["probs64"], g_idx, E)
+    assert abs(float(aux.item()) - aux_ref) <= TOL_AUX_REL * aux_ref
+    assert abs(float(z.item()) - r["z"]) <= TOL_AUX_REL * r["z"]
