@@ -2,9 +2,11 @@
 //
 // Gather: "MegaBlocks 01", section 4.3 (binned_gather reorders [tokens, hs]
 // by the sort; the token of flat slot s is s / top_k), here without padding.
-// Each warp's lane 0 drives a ring of shared-memory buffers with bulk (TMA)
+// Each warp's lane 0 drives a ring of 6 shared-memory buffers with bulk (TMA)
 // copies: cp.async.bulk global->shared completing on an mbarrier, then
-// cp.async.bulk shared->global into the gathered row. No multicast.
+// cp.async.bulk shared->global into the gathered row. A buffer is refilled one
+// iteration after its store was issued, so loads and a store are always in
+// flight together. No multicast.
 //
 // Combine: "ops-transformer MoE operators", 原理 Step 4 (weighted sum of the
 // chosen experts' outputs) and "MegaBlocks 01", sections 4.3 and 5 (multiply by
@@ -19,7 +21,7 @@ namespace moe {
 namespace {
 
 constexpr int kGatherWarps = 4;
-constexpr int kGatherBufs = 4;
+constexpr int kGatherBufs = 6;
 constexpr int kGatherPiece = 8192;  // bytes per buffer
 
 __global__ void __launch_bounds__(kGatherWarps * 32)
@@ -95,6 +97,7 @@ gather_bulk(const uint8_t* __restrict__ x, uint32_t row_bytes, int T, int k,
   bool ok = true;
   for (long long i = 0; i < mine && ok; ++i) {
     const int b = static_cast<int>(i % kGatherBufs);
+    bool committed = sizes[b] != 0;  // this iteration issues a store group
     if (sizes[b] && srcs[b] == nullptr) {
       bulk_store(dsts[b], zero, sizes[b]);
       bulk_commit();
@@ -108,13 +111,19 @@ gather_bulk(const uint8_t* __restrict__ x, uint32_t row_bytes, int T, int k,
       bulk_store(dsts[b], buf0 + b * kGatherPiece, sizes[b]);
       bulk_commit();
     }
-    const long long nxt = i + kGatherBufs;
-    if (nxt < mine) {
-      bulk_wait_read<0>();  // the store above has finished reading buffer b
-      piece(nxt, srcs[b], dsts[b], sizes[b]);
-      if (sizes[b] && srcs[b]) {
-        mbar_arrive_expect_tx(&bars[warp][b], sizes[b]);
-        bulk_load(buf0 + b * kGatherPiece, srcs[b], sizes[b], &bars[warp][b]);
+    // Refill the buffer of the previous piece (its store is one group older
+    // than the one just issued), so a store and the loads overlap.
+    const long long nxt = i - 1 + kGatherBufs;
+    if (i >= 1 && nxt < mine) {
+      const int pb = static_cast<int>((i - 1) % kGatherBufs);
+      // the previous piece's store group must have read its buffer: when this
+      // iteration issued a group, that is every group but the newest
+      if (committed) bulk_wait_read<1>();
+      else bulk_wait_read<0>();
+      piece(nxt, srcs[pb], dsts[pb], sizes[pb]);
+      if (sizes[pb] && srcs[pb]) {
+        mbar_arrive_expect_tx(&bars[warp][pb], sizes[pb]);
+        bulk_load(buf0 + pb * kGatherPiece, srcs[pb], sizes[pb], &bars[warp][pb]);
       }
     }
   }
