@@ -68,3 +68,32 @@ def test_full_size(name):
                            ExpertWeights(inp.w2), sh.act)
     err = max_err_ratio(got[sample], ref)
     assert err <= TOL_BF16_OUT, err
+
+
+@pytest.mark.parametrize("name", ["mixtral", "long_skewed_cf"])
+def test_full_size_layout_variants_equal(name):
+    """The padded-binned layout (dynamic or fixed capacity) and the gather
+    inside the up projection change where rows live or where they are read
+    from, not what is computed: at full size the layer output and aux loss
+    are bit-identical to the default layout's."""
+    from mixture_experts_routing_route_b200 import MoeLayer
+    sh = CONFIGS[name]
+    inp = make_inputs(sh)
+    dv = device_inputs(inp)
+
+    def run(**kw):
+        layer = MoeLayer(dv["wg"], dv["w1"], dv["w2"], w3=dv["w3"], bias=dv["bias"], k=sh.k,
+                         act=sh.act, capacity_factor=sh.cf, **kw)
+        out, aux = layer.forward(dv["x"])
+        torch.cuda.synchronize()
+        assert layer.device_error(sh.T) == 0
+        res = (out.clone(), aux.clone())
+        del layer
+        torch.cuda.empty_cache()
+        return res
+
+    out0, aux0 = run()
+    for kw in ({"binned": True}, {"gather_in_gemm": True}):
+        out1, aux1 = run(**kw)
+        assert torch.equal(out1, out0), kw
+        assert torch.equal(aux1, aux0), kw
