@@ -44,6 +44,8 @@ METRIC = "MoE-layer fwd tokens/s on 1 B200 (Mixtral 8e top-2 bf16)"
 UNIT = "tokens/s"
 STAGES = ["route", "permute", "gather", "ffn_up", "ffn_down", "combine"]
 FLUSH_BYTES = 256 << 20
+SPEC_HBM_GBS = 8000.0       # nominal B200 HBM3e, for the spec-relative fractions
+SPEC_BF16_TFLOPS = 2250.0   # nominal dense bf16
 GEMM_SRC = os.path.join(ROOT, "mixture_experts_routing_route_b200", "csrc", "gemm_sm100.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.txt")
 
@@ -335,6 +337,17 @@ def weights_f64(inp):
     return {"w1": cvt(inp.w1), "w3": cvt(inp.w3), "w2": cvt(inp.w2)}
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def cpu_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -366,7 +379,8 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded)", "config": workload_config(sh),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "cpu_model": cpu_model(),
+                         "kind": "oracle",
                          "sample": f"{tokens} of the workload's {sh.T} tokens per step, whole "
                                    f"layer (route, permute, gather, expert FFN, combine) in "
                                    f"numpy float64"},
@@ -381,7 +395,8 @@ def cpu_baseline(sh, inp):
     tokens = min(256, sh.T)
     oracle_sample_run(inp, min(16, sh.T), w64)  # first touch of the converted weights
     t = oracle_sample_run(inp, tokens, w64)
-    return {"value": tokens / t, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+    return {"value": tokens / t, "unit": UNIT, "cores": cpu_threads(), "cpu_model": cpu_model(),
+            "kind": "oracle",
             "sample": f"one oracle forward (numpy float64) of the first {tokens} of {sh.T} tokens "
                       f"of the same workload, {t:.1f} s"}
 
@@ -490,9 +505,11 @@ def main():
             continue
         r = {"us": stage_ms[s] * 1e3, "GB_s": a["bytes"] / t / 1e9 if t > 0 else None}
         r["hbm_frac"] = r["GB_s"] / peaks["hbm_gbs"] if r["GB_s"] else None
+        r["hbm_frac_spec"] = r["GB_s"] / SPEC_HBM_GBS if r["GB_s"] else None
         if "flops" in a:
             r["TFLOP_s"] = a["flops"] / t / 1e12 if t > 0 else None
             r["tensor_frac"] = r["TFLOP_s"] / tc_peak if r["TFLOP_s"] else None
+            r["tensor_frac_spec"] = r["TFLOP_s"] / SPEC_BF16_TFLOPS if r["TFLOP_s"] else None
         roof[s] = r
 
     dom = "ffn_up"
@@ -505,7 +522,15 @@ def main():
                 "peak_source": f"{peaks['source']} bf16 dense {tc_kind}",
                 "algorithmic_per_launch": f"2*R*d*2F = {alg[dom]['flops']:.4e} flop (R={sum(kept)} rows)",
                 "launch_us": up_ms * 1e3,
-                "timing": "CUDA events on the launch stream around the up projection, every timed step"}
+                "timing": "CUDA events on the launch stream around the up projection, every timed step",
+                "peak_spec": SPEC_BF16_TFLOPS, "frac_spec": tf / SPEC_BF16_TFLOPS if tf else None}
+    # Route + permute + gather judged as one span against its bytes (the
+    # permute alone moves < 1 MB and is latency-bound).
+    span_us = sum(stage_ms[s_] for s_ in ("route", "permute", "gather")) * 1e3
+    span_bytes = sum(alg[s_]["bytes"] for s_ in ("route", "permute", "gather"))
+    dispatch_span = {"us": span_us, "bytes": span_bytes,
+                     "hbm_frac": span_bytes / (span_us * 1e-6) / 1e9 / peaks["hbm_gbs"] if span_us > 0 else None,
+                     "hbm_frac_spec": span_bytes / (span_us * 1e-6) / 1e9 / SPEC_HBM_GBS if span_us > 0 else None}
 
     e2e = None
     if not args.no_e2e:
@@ -531,6 +556,7 @@ def main():
         "gpu_launches": launches,
         "clocks": clocks,
         "stages": roof,
+        "dispatch_span": dispatch_span,
         "stages_note": f"per-stage times from a separate pass of {nb} steps with an event at "
                        f"every stage boundary (events serialise the stages)",
         "aux_loss": float(aux.item()),
