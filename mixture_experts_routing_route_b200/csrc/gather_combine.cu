@@ -172,21 +172,36 @@ template <> struct CombineVec<float> {
 
 constexpr int kCombineThreads = 128;
 
-// One block per token (grid.x) and column range (grid.y); each thread owns
-// up to two 16-byte column vectors and requests the K rows of both before it
-// accumulates. K is the compile-time top-k (0: runtime k, rows one by one).
+// Each thread owns up to two 16-byte column vectors of one token and requests
+// the K rows of both before it accumulates. A token needs tpt threads (its
+// d/V vectors, two per thread). When tpt <= the block, a block takes
+// 128/tpt whole tokens (grid.x = token groups); otherwise one token spreads
+// over grid.y blocks. K is the compile-time top-k (0: runtime k, rows one by
+// one).
 template <typename T, int K>
 __global__ void __launch_bounds__(kCombineThreads)
 combine_gather(const T* __restrict__ y, const float* __restrict__ w,
-               const int32_t* __restrict__ slot_to_row, int d, int k_rt, long long rows_max,
-               T* __restrict__ out, Control* ctl) {
+               const int32_t* __restrict__ slot_to_row, int T_, int d, int k_rt, int tpt,
+               long long rows_max, T* __restrict__ out, Control* ctl) {
   pdl_begin();
   constexpr int V = CombineVec<T>::kVec;
   constexpr int NV = 2;  // column vectors per thread
   const int k = K > 0 ? K : k_rt;
-  const int t = blockIdx.x;
-  const int col0 = (blockIdx.y * kCombineThreads * NV + threadIdx.x) * V;
-  if (col0 >= d) return;
+  int t, v0, vstride;
+  if (tpt <= kCombineThreads) {
+    const int tpb = kCombineThreads / tpt;
+    const int local = threadIdx.x / tpt;
+    if (local >= tpb) return;
+    t = blockIdx.x * tpb + local;
+    v0 = threadIdx.x - local * tpt;
+    vstride = tpt;
+  } else {
+    t = blockIdx.x;
+    v0 = blockIdx.y * kCombineThreads * NV + threadIdx.x;
+    vstride = kCombineThreads;
+  }
+  const int col0 = v0 * V;
+  if (t >= T_ || col0 >= d) return;
   int rows[K > 0 ? K : 1];
   float wj[K > 0 ? K : 1];
   float acc[NV][V];
@@ -209,7 +224,7 @@ combine_gather(const T* __restrict__ y, const float* __restrict__ w,
     for (int j = 0; j < K; ++j)
 #pragma unroll
       for (int c = 0; c < NV; ++c) {
-        const int col = col0 + c * kCombineThreads * V;
+        const int col = (v0 + c * vstride) * V;
         u[j][c] = make_uint4(0, 0, 0, 0);
         if (rows[j] >= 0 && col < d)
           u[j][c] = __ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(rows[j]) * d + col));
@@ -230,7 +245,7 @@ combine_gather(const T* __restrict__ y, const float* __restrict__ w,
       const float wv = __ldg(w + static_cast<size_t>(t) * k + j);
 #pragma unroll
       for (int c = 0; c < NV; ++c) {
-        const int col = col0 + c * kCombineThreads * V;
+        const int col = (v0 + c * vstride) * V;
         if (col < d)
           CombineVec<T>::fma(__ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(row) * d + col)),
                              wv, acc[c]);
@@ -239,7 +254,7 @@ combine_gather(const T* __restrict__ y, const float* __restrict__ w,
   }
 #pragma unroll
   for (int c = 0; c < NV; ++c) {
-    const int col = col0 + c * kCombineThreads * V;
+    const int col = (v0 + c * vstride) * V;
     if (col < d)
       *reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * d + col) = CombineVec<T>::pack(acc[c]);
   }
@@ -249,7 +264,11 @@ template <typename T>
 cudaError_t launch_combine_t(const T* y, const float* w, const int32_t* s2r, int T_, int d, int k,
                       long long rows_max, T* out, Control* ctl, cudaStream_t s) {
   constexpr int V = CombineVec<T>::kVec;
-  dim3 grid(T_, (d + kCombineThreads * V * 2 - 1) / (kCombineThreads * V * 2));
+  const int nvec = (d + V - 1) / V;
+  const int tpt = (nvec + 1) / 2;  // threads per token, two vectors each
+  const dim3 grid = tpt <= kCombineThreads
+                        ? dim3((T_ + kCombineThreads / tpt - 1) / (kCombineThreads / tpt), 1)
+                        : dim3(T_, (d + kCombineThreads * V * 2 - 1) / (kCombineThreads * V * 2));
   auto kern = combine_gather<T, 0>;
   switch (k) {
     case 1: kern = combine_gather<T, 1>; break;
@@ -258,7 +277,8 @@ cudaError_t launch_combine_t(const T* y, const float* w, const int32_t* s2r, int
     case 8: kern = combine_gather<T, 8>; break;
     default: break;
   }
-  return launch_pdl(kern, grid, dim3(kCombineThreads), 0, s, false, y, w, s2r, d, k, rows_max, out, ctl);
+  return launch_pdl(kern, grid, dim3(kCombineThreads), 0, s, false, y, w, s2r, T_, d, k, tpt,
+                    rows_max, out, ctl);
 }
 
 }  // namespace
