@@ -99,8 +99,7 @@ cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, si
 }
 
 // ------------------------------------------------------------------ launchers
-// Router. Tokens per block of the general path (partials are per block).
-constexpr int kRouteSelectTokensPerBlock = 64;
+// Router.
 size_t route_partials_bytes(int T, int E);
 // noise: optional [T, E] fp32 added to the logits after the bias; z_out:
 // optional z-loss output (mean over tokens of the squared log-sum-exp).

@@ -164,51 +164,11 @@ __device__ __forceinline__ Tile decode_unit(int u, int total, int W, const int* 
 }
 
 // ------------------------------------------------------------------ epilogue
-// One thread = one accumulator row (its TMEM lane): OUTN output columns read
-// 32 at a time, activation in fp32, rounded once to bf16, stored if the row
-// is valid. SwiGLU: gate in columns [0, OUTN), up in [OUTN, 2 OUTN).
-template <int EPI, int OUTN>
-__device__ __forceinline__ void epilogue_row(uint32_t tbase, bool valid, __nv_bfloat16* orow) {
-#pragma unroll 1
-  for (int c = 0; c < OUTN; c += 32) {
-    uint32_t v[32];
-    uint32_t packed[16];
-    if constexpr (EPI == EPI_SWIGLU) {
-      uint32_t u[32];
-      tmem_ld_32x32b_x32(tbase + c, v);
-      tmem_ld_32x32b_x32(tbase + OUTN + c, u);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float h0 = silu(__uint_as_float(v[2 * i])) * __uint_as_float(u[2 * i]);
-        const float h1 = silu(__uint_as_float(v[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
-        packed[i] = pack_bf16(h0, h1);
-      }
-    } else {
-      tmem_ld_32x32b_x32(tbase + c, v);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float a = __uint_as_float(v[2 * i]), b = __uint_as_float(v[2 * i + 1]);
-        if (EPI == EPI_GELU) { a = gelu_erf(a); b = gelu_erf(b); }
-        packed[i] = pack_bf16(a, b);
-      }
-    }
-    if (valid) {
-      uint4* dst = reinterpret_cast<uint4*>(orow + c);
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-    }
-  }
-}
-
 // Epilogue of one warp through shared memory: for each 64-column group the
 // warp writes its rows (thread = row, 2 x 64 bytes) into a padded staging
 // buffer, then stores them back as whole 128-byte row segments, 8 lanes per
 // row, 4 rows per store instruction. Only rows [0, nrows) of the warp are
 // stored (rows past the expert's segment never are).
-constexpr bool kStagedStores = true;
 constexpr int kStageRow = 128 + 16;            // bytes per staged row (16 B pad: no bank conflicts)
 constexpr int kStageWarpBytes = 32 * kStageRow;
 
@@ -278,7 +238,7 @@ struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int OUT_N = EPI == EPI_SWIGLU ? NMMA / 2 : NMMA;
   static constexpr int TMEM_COLS = 2 * NMMA;
-  static constexpr size_t STAGING = kStagedStores ? 4 * kStageWarpBytes : 0;
+  static constexpr size_t STAGING = 4 * kStageWarpBytes;  // epilogue staging, one per warp
   static constexpr size_t SMEM = static_cast<size_t>(STAGES) * STAGE_BYTES + STAGING + 1024;
 };
 
@@ -520,7 +480,7 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       tc_fence_after();
       const bool m64 = t.rows <= 64;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * NMMA;
-      if constexpr (kStagedStores) {
+      {
         uint8_t* buf = smem + STAGES * C::STAGE_BYTES + q * kStageWarpBytes;
         const int wrow = m64 ? q * 16 : q * 32;
         const int nrows = max(0, min(m64 ? 16 : 32, t.rows - wrow));
@@ -528,14 +488,6 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           epilogue_staged<EPI, C::OUT_N / 2>(tbase, buf, args.out, t.row0 + wrow, nrows, args.N, t.n0, lane);
         else
           epilogue_staged<EPI, C::OUT_N>(tbase, buf, args.out, t.row0 + wrow, nrows, args.N, t.n0, lane);
-      } else {
-        const int r_in_tile = m64 ? q * 16 + lane : q * 32 + lane;
-        const bool valid = (!m64 || lane < 16) && r_in_tile < t.rows;
-        __nv_bfloat16* orow = args.out + static_cast<size_t>(t.row0 + r_in_tile) * args.N + t.n0;
-        if (t.half)
-          epilogue_row<EPI, C::OUT_N / 2>(tbase, valid, orow);
-        else
-          epilogue_row<EPI, C::OUT_N>(tbase, valid, orow);
       }
       tc_fence_before();
       __syncwarp();

@@ -212,16 +212,9 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   return r;
 }
 
-// Load from distributed shared memory. Not volatile: the loads of one row can
-// be issued back to back; callers order them against writes with a cluster
-// barrier.
-__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
-  float v;
-  asm("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-  return v;
-}
-
-// 16-byte load from distributed shared memory (addr 16-byte aligned).
+// 16-byte load from distributed shared memory (addr 16-byte aligned). Not
+// volatile, so the loads of one row can be issued back to back; callers
+// order them against the writes with a cluster barrier.
 __device__ __forceinline__ float4 ld_shared_cluster_f32x4(uint32_t addr) {
   float4 v;
   asm("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
