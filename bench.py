@@ -391,8 +391,10 @@ def run_reference(args):
 
 
 def cpu_baseline(sh, inp):
+    """The oracle's whole layer over up to 4096 of the workload's tokens (all
+    of the Mixtral workload's; ~5-15 s on the host's cores)."""
     w64 = weights_f64(inp)
-    tokens = min(256, sh.T)
+    tokens = min(4096, sh.T)
     oracle_sample_run(inp, min(16, sh.T), w64)  # first touch of the converted weights
     t = oracle_sample_run(inp, tokens, w64)
     return {"value": tokens / t, "unit": UNIT, "cores": cpu_threads(), "cpu_model": cpu_model(),
