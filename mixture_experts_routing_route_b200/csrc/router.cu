@@ -601,9 +601,12 @@ router_select(const float* __restrict__ logits_in, int KS, const float* __restri
 // has as many stages (up to kTcStages) as shared memory holds.
 constexpr int kTcStages = 8;
 constexpr int kTcThreads = 128;
+constexpr int kMaxKS = 8;  // largest split of d over the CTAs of one token tile
 
 struct RouterTcArgs {
   int T, d, E, Epad, KS, dk, stages;
+  int tmem_cap;             // tensor-memory columns one CTA may take (512 / CTAs per SM)
+  int sub;                  // persistent kernel: k-blocks per ring stage, loaded together
   const __nv_bfloat16* wg;  // [d, E] (staged path)
   float* partial;           // [KS][T][E] (unfused)
   Control* ctl;
@@ -636,19 +639,10 @@ struct FuseCfg {
   static constexpr size_t kScratch = 2 * 128 * kStride * 4 + 128 * 4 + kTcThreads * 8;
 };
 
-// Thread r of each CTA: the sum over accumulator slots (in slot order) of
-// its row's columns, then the fused selection. Every thread of every CTA of
-// the cluster reaches both cluster barriers.
+// Thread r: the sum over accumulator slots (in slot order) of the first EW
+// columns of its row (trow = the row's tensor-memory address).
 template <int EW>
-__device__ __forceinline__ void fused_select_epilogue(const RouterTcArgs& a, uint32_t tmem_base,
-                                                      int nslot, int tile, int ks, bool ok,
-                                                      uint8_t* smem, int warp, int lane) {
-  using F = FuseCfg<EW>;
-  const int E = a.E;
-  const int r = warp * 32 + lane;
-  const int t = tile * 128 + r;
-  const uint32_t trow = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
-  float v[EW];
+__device__ __forceinline__ void slot_sums(uint32_t trow, int nslot, int Epad, float (&v)[EW]) {
 #pragma unroll
   for (int h = 0; h < (EW + 15) / 16; ++h) {
     float sum[16];
@@ -656,7 +650,7 @@ __device__ __forceinline__ void fused_select_epilogue(const RouterTcArgs& a, uin
     for (int i = 0; i < 16; ++i) sum[i] = 0.f;
     for (int sl = 0; sl < nslot; ++sl) {
       uint32_t u[16];
-      tmem_ld_32x32b_x16(trow + sl * a.Epad + h * 16, u);
+      tmem_ld_32x32b_x16(trow + sl * Epad + h * 16, u);
       tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 16; ++i) sum[i] += __uint_as_float(u[i]);
@@ -665,23 +659,47 @@ __device__ __forceinline__ void fused_select_epilogue(const RouterTcArgs& a, uin
     for (int i = 0; i < 16; ++i)
       if (h * 16 + i < EW) v[h * 16 + i] = sum[i];
   }
-  // The ring is idle (every MMA has completed): reuse it for row buffers.
-  float* red = reinterpret_cast<float*>(smem);                   // [128][kStride]
-  float* pm = red + 128 * F::kStride;                            // [128][kStride]
-  uint32_t* selm = reinterpret_cast<uint32_t*>(pm + 128 * F::kStride);  // [128]
-  float* part_ps = reinterpret_cast<float*>(selm + 128);         // [kTcThreads]
-  int* part_cs = reinterpret_cast<int*>(part_ps + kTcThreads);   // [kTcThreads]
-  __shared__ int last_s;
-  if (a.KS > 1) {
-    if (ks != 0) {
+}
+
+// The split over d (KS > 1): CTA ks > 0 leaves its row sums in its own shared
+// memory (red) and the leader (ks = 0) adds them in ks order through
+// distributed shared memory. Every thread of every CTA of the cluster reaches
+// both cluster barriers.
+template <int EW>
+__device__ __forceinline__ void cluster_row_sums(int KS, int ks, int r, float* red, float (&v)[EW]) {
+  using F = FuseCfg<EW>;
+  if (ks != 0) {
 #pragma unroll
-      for (int e = 0; e < EW; e += 4)
-        *reinterpret_cast<float4*>(red + r * F::kStride + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-    }
-    cluster_sync();
-    if (ks == 0) {
-      for (int src = 1; src < a.KS; ++src) {
-        const uint32_t base = mapa_shared(smem_u32(red + r * F::kStride), static_cast<uint32_t>(src));
+    for (int e = 0; e < EW; e += 4)
+      *reinterpret_cast<float4*>(red + r * F::kStride + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+  }
+  cluster_sync();
+  if (ks == 0) {
+    const uint32_t own = smem_u32(red + r * F::kStride);
+    if constexpr (EW == 8) {
+      // all peers' rows requested at once (one round trip), added in ks order
+      float4 q[kMaxKS - 1][2];
+#pragma unroll
+      for (int src = 1; src < kMaxKS; ++src)
+        if (src < KS) {
+          const uint32_t base = mapa_shared(own, static_cast<uint32_t>(src));
+          q[src - 1][0] = ld_shared_cluster_f32x4(base);
+          q[src - 1][1] = ld_shared_cluster_f32x4(base + 16u);
+        }
+#pragma unroll
+      for (int src = 1; src < kMaxKS; ++src)
+        if (src < KS) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            v[4 * h] += q[src - 1][h].x;
+            v[4 * h + 1] += q[src - 1][h].y;
+            v[4 * h + 2] += q[src - 1][h].z;
+            v[4 * h + 3] += q[src - 1][h].w;
+          }
+        }
+    } else {
+      for (int src = 1; src < KS; ++src) {
+        const uint32_t base = mapa_shared(own, static_cast<uint32_t>(src));
         float4 q[EW / 4];
 #pragma unroll
         for (int e = 0; e < EW / 4; ++e) q[e] = ld_shared_cluster_f32x4(base + 16u * e);
@@ -694,17 +712,37 @@ __device__ __forceinline__ void fused_select_epilogue(const RouterTcArgs& a, uin
         }
       }
     }
-    cluster_sync();  // the other CTAs keep their buffers until the leader has read them
   }
-  if (ks != 0) return;
+  cluster_sync();  // the other CTAs keep their buffers until the leader has read them
+}
 
+// Selection and aux partials of one 128-token tile, run by the 128 threads
+// that own its rows (thread r = token tile*128 + r, lane = r % 32); sync()
+// is a barrier over exactly those threads. scratch holds FuseCfg<EW>::kScratch
+// bytes. v = the row's logits before the bias; bias_r and noise_r are the
+// additive terms already fetched.
+template <int EW, class Sync>
+__device__ __forceinline__ void select_and_aux(const RouterTcArgs& a, const float (&v)[EW],
+                                               const float (&bias_r)[EW],
+                                               const float (&noise_r)[EW], int tile, bool ok,
+                                               int r, uint8_t* scratch, Sync sync) {
+  using F = FuseCfg<EW>;
+  const int E = a.E;
+  const int lane = r & 31, wq = r >> 5;
+  const int t = tile * 128 + r;
+  float* red = reinterpret_cast<float*>(scratch);                // [128][kStride]
+  float* pm = red + 128 * F::kStride;                            // [128][kStride]
+  uint32_t* selm = reinterpret_cast<uint32_t*>(pm + 128 * F::kStride);  // [128]
+  float* part_ps = reinterpret_cast<float*>(selm + 128);         // [kTcThreads]
+  int* part_cs = reinterpret_cast<int*>(part_ps + kTcThreads);   // [kTcThreads]
+  __shared__ int last_s;
   const bool valid = ok && t < a.T;
   float lg[EW], p[EW];
   float m = -INFINITY;
 #pragma unroll
   for (int e = 0; e < EW; ++e) {
-    lg[e] = e < E ? v[e] + (a.bias != nullptr ? __ldg(a.bias + e) : 0.f) : -INFINITY;
-    if (a.noise != nullptr && e < E && t < a.T) lg[e] += __ldg(a.noise + static_cast<size_t>(t) * E + e);
+    lg[e] = e < E ? v[e] + bias_r[e] : -INFINITY;
+    if (a.noise != nullptr && e < E && t < a.T) lg[e] += noise_r[e];
     m = fmaxf(m, lg[e]);
   }
   float ssum = 0.f;
@@ -764,14 +802,14 @@ __device__ __forceinline__ void fused_select_epilogue(const RouterTcArgs& a, uin
     float zt = valid ? lse * lse : 0.f;
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) zt += __shfl_xor_sync(kFull, zt, off);
-    if (lane == 0) zw_s[warp] = zt;
+    if (lane == 0) zw_s[wq] = zt;
   }
   // ---- aux partials of this tile: thread (e, part) adds rows part, part +
   // kParts, ... of expert e; then the kParts sums are added in part order.
 #pragma unroll
   for (int e = 0; e < EW; ++e) pm[r * F::kStride + e] = valid ? p[e] : 0.f;
   selm[r] = valid ? taken : 0u;
-  __syncthreads();
+  sync();
   {
     const int e = r % EW, part = r / EW;
     float ps = 0.f;
@@ -783,7 +821,7 @@ __device__ __forceinline__ void fused_select_epilogue(const RouterTcArgs& a, uin
     part_ps[r] = ps;
     part_cs[r] = cs;
   }
-  __syncthreads();
+  sync();
   if (r < E) {
     float ps = 0.f;
     int cs = 0;
@@ -796,12 +834,12 @@ __device__ __forceinline__ void fused_select_epilogue(const RouterTcArgs& a, uin
   }
   if (a.part_z != nullptr && r == 0)
     a.part_z[tile] = ((zw_s[0] + zw_s[1]) + zw_s[2]) + zw_s[3];
-  __syncthreads();
+  sync();
   if (r == 0) {
     __threadfence();
     last_s = atomicAdd(&a.ctl->route_ticket, 1u) == static_cast<unsigned>(a.ntile - 1);
   }
-  __syncthreads();
+  sync();
   if (!last_s) return;
   __threadfence();
   // ---- last tile: thread (e, part) adds tiles part, part + kParts, ... in
@@ -820,28 +858,32 @@ __device__ __forceinline__ void fused_select_epilogue(const RouterTcArgs& a, uin
     dps[r] = ps;
     dcs[r] = cs;
   }
-  __syncthreads();
+  sync();
+  // thread e: its expert's term f_e * P_e; thread 0 adds the terms in expert order
+  __shared__ double term_s[kFuseMaxE];
+  if (r < E) {
+    double ps = 0.0;
+    long long cs = 0;
+    for (int q = 0; q < F::kParts; ++q) {
+      ps += dps[q * EW + r];
+      cs += dcs[q * EW + r];
+    }
+    term_s[r] = (static_cast<double>(cs) / (static_cast<double>(a.T) * a.k)) * (ps / a.T);
+  }
+  sync();
   if (r == 0) {
     double tot = 0.0;
-    for (int e = 0; e < E; ++e) {
-      double ps = 0.0;
-      long long cs = 0;
-      for (int q = 0; q < F::kParts; ++q) {
-        ps += dps[q * EW + e];
-        cs += dcs[q * EW + e];
-      }
-      tot += (static_cast<double>(cs) / (static_cast<double>(a.T) * a.k)) * (ps / a.T);
-    }
+    for (int e = 0; e < E; ++e) tot += term_s[e];
     *a.aux = static_cast<float>(E * tot);
   }
   if (a.part_z != nullptr) {  // z-loss: tiles r, r + 128, ... then a fixed tree, / T
     double zs = 0.0;
     for (int b = r; b < a.ntile; b += kTcThreads) zs += static_cast<double>(__ldcg(a.part_z + b));
     zd_s[r] = zs;
-    __syncthreads();
+    sync();
     for (int st = kTcThreads / 2; st > 0; st >>= 1) {
       if (r < st) zd_s[r] += zd_s[r + st];
-      __syncthreads();
+      sync();
     }
     if (r == 0) *a.z_out = static_cast<float>(zd_s[0] / a.T);
   }
@@ -869,12 +911,17 @@ router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
   const int nst = a.stages;
   uint8_t* ring = smem;
   uint8_t* wgt = smem + nst * stage_bytes;  // staged Wg^T (E <= 32)
-  const uint32_t wgt_kb_bytes = static_cast<uint32_t>(a.Epad) * 128;
+  // k-block kb's E real rows start at kb * E * 128 bytes (E is a multiple of
+  // 8, so every block starts on a 1024-byte swizzle atom). The MMA's N = Epad
+  // also reads rows E..Epad-1 (at most one 8-row atom): the next block's first
+  // rows, or the 1 KB of slack after the last block. They land only in
+  // accumulator columns E..Epad-1, which nothing reads.
+  const uint32_t wgt_kb_bytes = static_cast<uint32_t>(a.E) * 128;
   // Accumulator slots: k-block kb accumulates into TMEM columns
   // [(kb / G) * Epad, +Epad), G k-blocks per slot, as many slots as 512
   // columns hold. The epilogue adds the slots in IEEE fp32, so a tensor-core
   // accumulation chain is at most 4*G MMAs long.
-  const int nslot_cap = 512 / a.Epad;
+  const int nslot_cap = a.tmem_cap / a.Epad;
   const int G = (nkb + nslot_cap - 1) / nslot_cap;
   const int nslot = (nkb + G - 1) / G;
   uint32_t tcols = 32;
@@ -901,17 +948,15 @@ router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
   // permutes, eight 16-byte stores (one expert's 8 k-values each). Tasks of
   // the real experts come first; experts E..Epad-1 are zero. Each thread's
   // first loads go out before the x tiles' TMA loads, so they do not queue
-  // behind them.
+  // behind them. Only the real experts' rows are staged (see wgt_kb_bytes).
   const int k0 = ks * a.dk;
   const int nchunk = a.dk / 8, groups = a.E / 8;
-  const int ntask = kTmaB ? 0 : nchunk * (a.Epad / 8);
+  const int ntask = kTmaB ? 0 : nchunk * groups;
   auto load_task = [&](int i, uint32_t (&in)[8][4]) {
     const int g = i / nchunk, ch = i - g * nchunk;
 #pragma unroll
     for (int rr = 0; rr < 8; ++rr) {
-      uint4 u = make_uint4(0, 0, 0, 0);
-      if (g < groups)
-        u = __ldg(reinterpret_cast<const uint4*>(a.wg + static_cast<size_t>(k0 + ch * 8 + rr) * a.E) + g);
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(a.wg + static_cast<size_t>(k0 + ch * 8 + rr) * a.E) + g);
       in[rr][0] = u.x;
       in[rr][1] = u.y;
       in[rr][2] = u.z;
@@ -933,8 +978,7 @@ router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
     }
   };
   uint32_t in0[8][4];
-  const bool has0 = static_cast<int>(threadIdx.x) < ntask;
-  if (has0) load_task(threadIdx.x, in0);
+  if (static_cast<int>(threadIdx.x) < ntask) load_task(threadIdx.x, in0);
 
   // The first ring stages are free: start their loads now.
   const int pre = nkb < nst ? nkb : nst;
@@ -951,16 +995,41 @@ router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
     for (int kb = 0; kb < pre; ++kb) issue(kb, kb);
   }
   if (!kTmaB) {
-    if (has0) store_task(threadIdx.x, in0);
-    for (int i = threadIdx.x + kTcThreads; i < ntask; i += kTcThreads) {
-      uint32_t in[8][4];
-      load_task(i, in);
-      store_task(i, in);
+    // the next task's loads go out before this task's stores
+    for (int i = threadIdx.x; i < ntask; i += kTcThreads) {
+      uint32_t nxt[8][4];
+      const bool more = i + kTcThreads < ntask;
+      if (more) load_task(i + kTcThreads, nxt);
+      store_task(i, in0);
+      if (more) {
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) in0[rr][q] = nxt[rr][q];
+      }
     }
     fence_proxy_async_smem();  // generic-proxy writes, read by the tensor core
     __syncthreads();
   }
 
+  // The fused selection's additive terms, fetched while the MMAs run.
+  constexpr int kEW = kFuseE > 0 ? kFuseE : 1;
+  float bias_r[kEW], noise_r[kEW];
+#pragma unroll
+  for (int e = 0; e < kEW; ++e) {
+    bias_r[e] = 0.f;
+    noise_r[e] = 0.f;
+  }
+  if constexpr (kFuseE != 0) {
+    const int t = tile * 128 + warp * 32 + lane;
+    if (ks == 0) {
+#pragma unroll
+      for (int e = 0; e < kEW; ++e) {
+        if (e < a.E && a.bias != nullptr) bias_r[e] = __ldg(a.bias + e);
+        if (e < a.E && a.noise != nullptr && t < a.T) noise_r[e] = __ldg(a.noise + static_cast<size_t>(t) * a.E + e);
+      }
+    }
+  }
   bool ok = true;
   if (warp == 0 && lane == 0) {
     uint32_t phase = 1;  // the prologue filled round 0
@@ -1037,13 +1106,228 @@ router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
       }
     }
   } else {
-    fused_select_epilogue<kFuseE>(a, tmem_base, nslot, tile, ks, ok, smem, warp, lane);
+    // The ring is idle (every MMA has completed): it holds the row buffers.
+    const int r = warp * 32 + lane;
+    float v[kEW];
+    slot_sums<kEW>(tmem_base + (static_cast<uint32_t>(warp * 32) << 16), nslot, a.Epad, v);
+    if (a.KS > 1) cluster_row_sums<kEW>(a.KS, ks, r, reinterpret_cast<float*>(smem), v);
+    if (ks == 0) select_and_aux<kEW>(a, v, bias_r, noise_r, tile, ok, r, smem, [] { __syncthreads(); });
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem_base, tcols);
+  }
+}
+
+// Persistent fused router, d unsplit (KS = 1), for more token tiles than
+// SMs: one CTA per SM stages Wg^T once and walks the tiles blockIdx.x,
+// blockIdx.x + gridDim.x, ... Six warps: warp 0 (one thread) streams x
+// k-blocks of all its tiles through the ring, warp 1 (one thread) issues the
+// MMAs of tile j into accumulator j % 2 (two of 256 tensor-memory columns),
+// warps 2-5 (thread = token row; warp w reads lane quarter w % 4) run the
+// selection and aux partials of tile j while tile j + 1 loads and multiplies.
+// Same arithmetic as router_tc's fused path with KS = 1.
+constexpr int kPersistThreads = 192;
+constexpr int kPersistAccCols = 256;
+
+__device__ __forceinline__ void epi_bar_sync() {  // the four selection warps
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+template <int EW>
+__global__ void __launch_bounds__(kPersistThreads, 1)
+router_tc_persist(const __grid_constant__ CUtensorMap tmX, RouterTcArgs a) {
+  pdl_begin();
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[kTcStages], empty_bar[kTcStages];
+  __shared__ __align__(8) uint64_t tfull_bar[2], tempty_bar[2], done_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int okw_s[4];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int nkb = a.d / 64;
+  constexpr uint32_t kBoxBytes = 128 * 128;  // one k-block of 128 token rows
+  const int sub = a.sub;                     // k-blocks per stage (divides nkb)
+  const int nkg = nkb / sub;                 // stage loads per tile
+  const uint32_t stage_bytes = kBoxBytes * sub;
+  const int nst = a.stages;
+  uint8_t* ring = smem;
+  uint8_t* wgt = smem + nst * stage_bytes;
+  // k-block kb's E rows at kb * E * 128 bytes; the padding rows E..Epad-1 the
+  // MMA also reads are the next block's (or the 1 KB slack), as in router_tc.
+  const uint32_t wgt_kb_bytes = static_cast<uint32_t>(a.E) * 128;
+  uint8_t* scratch = wgt + static_cast<size_t>(a.d) * a.E * 2 + 1024;
+  const int nslot_cap = kPersistAccCols / a.Epad;
+  const int G = (nkb + nslot_cap - 1) / nslot_cap;  // k-blocks per accumulator slot
+  const int nslot = (nkb + G - 1) / G;
+  const int my_tiles = static_cast<int>(blockIdx.x) < a.ntile
+                           ? (a.ntile - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                           : 0;
+  const int total = my_tiles * nkg;  // ring loads of this CTA
+  const int pre = total < nst ? total : nst;
+
+  // load i: tile i / nkg, k-blocks sub * (i % nkg) + [0, sub), stage i % nst;
+  // the sub boxes of a row's consecutive 128-byte pieces go out together
+  auto issue = [&](int i) {
+    const int j = i / nkg, kg = i - j * nkg, st = i % nst;
+    const int tile = static_cast<int>(blockIdx.x) + j * static_cast<int>(gridDim.x);
+    mbar_arrive_expect_tx(&full_bar[st], stage_bytes);
+    for (int u = 0; u < sub; ++u)
+      tma_load_2d(ring + st * stage_bytes + u * kBoxBytes, &tmX, &full_bar[st], (kg * sub + u) * 64,
+                  tile * 128);
+  };
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < nst; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&tfull_bar[b], 1); mbar_init(&tempty_bar[b], 4); }
+    mbar_init(&done_bar, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tmX);
+    for (int i = 0; i < pre; ++i) issue(i);  // the ring's first round, before the staging
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_s, 2 * kPersistAccCols);
+    tmem_relinquish();
+  }
+  // Wg^T staging by all threads: task = 8 d-rows x 8 experts, transposed with
+  // byte permutes into the K-major 128-byte-swizzled rows (see router_tc).
+  {
+    const int nchunk = a.d / 8, groups = a.E / 8, ntask = nchunk * groups;
+    for (int i = threadIdx.x; i < ntask; i += kPersistThreads) {
+      const int g = i / nchunk, ch = i - g * nchunk;
+      uint32_t in[8][4];
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(a.wg + static_cast<size_t>(ch * 8 + rr) * a.E) + g);
+        in[rr][0] = u.x;
+        in[rr][1] = u.y;
+        in[rr][2] = u.z;
+        in[rr][3] = u.w;
+      }
+      const int kb = ch >> 3, c = ch & 7;
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const int e = g * 8 + jj;
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          o[q] = __byte_perm(in[2 * q][jj >> 1], in[2 * q + 1][jj >> 1], (jj & 1) ? 0x7632 : 0x5410);
+        const uint32_t off = kb * wgt_kb_bytes + e * 128 + (((c ^ e) & 7) << 4);
+        *reinterpret_cast<uint4*>(wgt + off) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+  }
+  fence_proxy_async_smem();  // generic-proxy writes, read by the tensor core
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int i = pre;
+      for (; i < total; ++i) {
+        const int st = i % nst, round = i / nst;
+        if (!mbar_wait_bounded(&empty_bar[st], (round & 1) ^ 1u)) {
+          set_error(a.ctl, MOE_DEVERR_TIMEOUT);
+          break;
+        }
+        issue(i);
+      }
+      // wait (bounded) for the last load issued into each stage to land
+      for (int st = 0; st < nst && st < i; ++st) {
+        const int last = st + ((i - 1 - st) / nst) * nst;
+        mbar_wait_bounded(&full_bar[st], static_cast<uint32_t>(last / nst) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc_bf16(128, a.Epad, true);  // staged Wg^T is K-major
+      bool issued = false, ok = true;
+      int i = 0;
+      for (int j = 0; j < my_tiles && ok; ++j) {
+        const int acc = j & 1;
+        if (!mbar_wait_bounded(&tempty_bar[acc], static_cast<uint32_t>((j >> 1) & 1) ^ 1u)) {
+          set_error(a.ctl, MOE_DEVERR_TIMEOUT);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dbase = tmem_base + static_cast<uint32_t>(acc * kPersistAccCols);
+        for (int kg = 0; kg < nkg; ++kg, ++i) {
+          const int st = i % nst;
+          if (!mbar_wait_bounded(&full_bar[st], static_cast<uint32_t>(i / nst) & 1u)) {
+            set_error(a.ctl, MOE_DEVERR_TIMEOUT);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          for (int u = 0; u < sub; ++u) {
+            const int kb = kg * sub + u;
+            const uint32_t a_addr = smem_u32(ring + st * stage_bytes + u * kBoxBytes);
+            const uint32_t d_tmem = dbase + static_cast<uint32_t>((kb / G) * a.Epad);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t adesc = make_sw128_desc(a_addr + kk * 32, 16, 1024);
+              const uint64_t bdesc = make_sw128_desc(smem_u32(wgt) + kb * wgt_kb_bytes + kk * 32, 16, 1024);
+              umma_bf16(d_tmem, adesc, bdesc, idesc, ((kb % G) | kk) != 0 ? 1u : 0u);
+            }
+          }
+          issued = true;
+          umma_commit(&empty_bar[st]);
+        }
+        if (ok) umma_commit(&tfull_bar[acc]);
+      }
+      // every MMA issued has completed before the tensor memory is freed
+      if (issued) {
+        umma_commit(&done_bar);
+        mbar_wait_bounded(&done_bar, 0);
+      }
+    }
+  } else {
+    const int q = warp & 3;  // the lane quarter this warp may read
+    const int r = q * 32 + lane;
+    float bias_r[EW], noise_r[EW];
+#pragma unroll
+    for (int e = 0; e < EW; ++e) {
+      bias_r[e] = (e < a.E && a.bias != nullptr) ? __ldg(a.bias + e) : 0.f;
+      noise_r[e] = 0.f;
+    }
+    for (int j = 0; j < my_tiles; ++j) {
+      const int acc = j & 1;
+      const int tile = static_cast<int>(blockIdx.x) + j * static_cast<int>(gridDim.x);
+      const int t = tile * 128 + r;
+      if (a.noise != nullptr && t < a.T) {
+#pragma unroll
+        for (int e = 0; e < EW; ++e)
+          if (e < a.E) noise_r[e] = __ldg(a.noise + static_cast<size_t>(t) * a.E + e);
+      }
+      int okw = 1;
+      if (lane == 0) okw = mbar_wait_bounded(&tfull_bar[acc], static_cast<uint32_t>(j >> 1) & 1u);
+      okw = __shfl_sync(kFull, okw, 0);
+      if (lane == 0) okw_s[q] = okw;
+      epi_bar_sync();
+      if (!(okw_s[0] && okw_s[1] && okw_s[2] && okw_s[3])) {  // the four warps leave together
+        if (r == 0) set_error(a.ctl, MOE_DEVERR_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      float v[EW];
+      slot_sums<EW>(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                        static_cast<uint32_t>(acc * kPersistAccCols),
+                    nslot, a.Epad, v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty_bar[acc]);  // accumulator free for tile j + 2
+      select_and_aux<EW>(a, v, bias_r, noise_r, tile, true, r, scratch, [] { epi_bar_sync(); });
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * kPersistAccCols);
   }
 }
 
@@ -1058,7 +1342,6 @@ size_t fused_smem_bytes(int d) { return static_cast<size_t>((d + 7) / 8) * 256; 
 // d/64 k-blocks) grows while the grid stays within the SMs; the staged Wg^T
 // of one CTA must fit in 128 KB; the ring takes what is left of 227 KB, up to
 // kTcStages stages.
-constexpr int kMaxKS = 8;
 // Split over d: the grid may reach kTcFill x (SMs / 2) CTAs. The unfused
 // path keeps it at half the SMs (more splits cost router_select more partial
 // traffic than they save); the fused path, whose split is reduced on chip,
@@ -1073,6 +1356,7 @@ struct TcPlan {
   int fuse_e = 0;  // 8, 16 or 32: router_tc<false, fuse_e> selects and reduces the aux loss too
   int Epad = 0, KS = 1, ntile = 0, stages = 0;
   size_t smem = 0;
+  size_t stage = 0, scratch = 0;  // bytes of one ring stage; the fused selection's row buffers
 };
 
 TcPlan plan_tc(int T, int d, int E, moe_dtype_t dt) {
@@ -1093,22 +1377,27 @@ TcPlan plan_tc(int T, int d, int E, moe_dtype_t dt) {
   int ks = 1;
   while (ks < kMaxKS && p.ntile * ks * 2 <= num_sms() * fill && nkb % (ks * 2) == 0) ks *= 2;
   if (!p.tma_b)
-    while (static_cast<size_t>(d / ks) * p.Epad * 2 > 128 * 1024 && ks < kMaxKS && nkb % (ks * 2) == 0) ks *= 2;
-  if (!p.tma_b && static_cast<size_t>(d / ks) * p.Epad * 2 > 128 * 1024) return p;
+    while (static_cast<size_t>(d / ks) * E * 2 > 128 * 1024 && ks < kMaxKS && nkb % (ks * 2) == 0) ks *= 2;
+  if (!p.tma_b && static_cast<size_t>(d / ks) * E * 2 > 128 * 1024) return p;
   p.KS = ks;
   const size_t stage = 128 * 128 + (p.tma_b ? static_cast<size_t>(p.Epad / 64) * 8192 : 0);
-  const size_t wgt = p.tma_b ? 0 : static_cast<size_t>(d / ks) * p.Epad * 2;
+  // staged Wg^T: the real rows, plus one atom of slack read as padding rows
+  const size_t wgt = p.tma_b ? 0 : static_cast<size_t>(d / ks) * E * 2 + (p.Epad != E ? 1024 : 0);
   const size_t avail = 227 * 1024 - 1024 - wgt;
   p.stages = static_cast<int>(std::min<size_t>(fusable ? kTcStagesFused : kTcStages, avail / stage));
   if (p.stages < 2) return p;
   p.smem = 1024 + p.stages * stage + wgt;
+  p.stage = stage;
   p.use = true;
   // The fused selection reuses the ring for its row buffers.
   if (fusable) {
     const int ew = E <= 8 ? 8 : (E <= 16 ? 16 : 32);
     const size_t scratch = ew == 8 ? FuseCfg<8>::kScratch
                          : ew == 16 ? FuseCfg<16>::kScratch : FuseCfg<32>::kScratch;
-    if (p.stages * stage >= scratch) p.fuse_e = ew;
+    if (p.stages * stage >= scratch) {
+      p.fuse_e = ew;
+      p.scratch = scratch;
+    }
   }
   return p;
 }
@@ -1172,6 +1461,7 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, const
       RouterTcArgs a = {};
       a.T = T; a.d = d; a.E = E; a.Epad = tp.Epad; a.KS = tp.KS; a.dk = d / tp.KS;
       a.stages = tp.stages;
+      a.tmem_cap = 512;
       a.wg = static_cast<const __nv_bfloat16*>(wg);
       a.partial = logits_scratch;
       a.ctl = ctl;
@@ -1182,11 +1472,62 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, const
         a.idx = idx; a.w = w; a.logits = logits; a.probs = probs;
         a.part_p = part_p; a.part_c = part_c; a.aux = aux;
         a.noise = noise; a.part_z = part_z; a.z_out = z_out;
+        if (tp.KS == 1 && tp.ntile > num_sms()) {
+          // persistent: one CTA per SM stages Wg^T once and walks the tiles
+          const size_t fixed = 1024 + static_cast<size_t>(d) * E * 2 + 1024 + tp.scratch;
+          const size_t budget = 227 * 1024 - 2048;  // dynamic shared memory next to the static
+          // k-blocks per stage: 4 (each token row's 512 consecutive bytes requested
+          // together, measured 14-20% faster than one k-block per stage at T =
+          // 32768-65536), fewer if two such stages do not fit
+          int sub = 4;
+          while (sub > 1 && ((d / 64) % sub != 0 || fixed + 2 * 16384 * static_cast<size_t>(sub) > budget)) sub >>= 1;
+          const size_t sbytes = 16384 * static_cast<size_t>(sub);
+          const int st = fixed + 2 * sbytes <= budget
+                             ? static_cast<int>(std::min<size_t>(kTcStages, (budget - fixed) / sbytes))
+                             : 0;
+          if (st >= 2) {
+            // at least 120 KB, so that no two CTAs share an SM (each takes all
+            // 512 tensor-memory columns)
+            const size_t smem = std::max<size_t>(fixed + static_cast<size_t>(st) * sbytes, 120 * 1024);
+            a.stages = st;
+            a.sub = sub;
+            auto pk = tp.fuse_e == 8 ? router_tc_persist<8>
+                    : tp.fuse_e == 16 ? router_tc_persist<16> : router_tc_persist<32>;
+            cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+            return launch_pdl(pk, dim3(std::min(tp.ntile, num_sms())), dim3(kPersistThreads), smem, s,
+                              false, tx, a);
+          }
+        }
         auto kern = tp.fuse_e == 8 ? router_tc<false, 8>
                   : tp.fuse_e == 16 ? router_tc<false, 16> : router_tc<false, 32>;
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(tp.smem));
-        return launch_pdl_cluster(kern, grid, dim3(kTcThreads), tp.smem, s, tp.KS, tx, tw, a);
+        // More CTAs than SMs: take ring stages away while that lets the whole
+        // grid be resident at once (each CTA stages Wg^T once, no second wave).
+        size_t smem = tp.smem;
+        const long long G = grid.x, sms = num_sms();
+        int nb = 1;
+        if (G > sms) {
+          for (int st = tp.stages; st >= 2 && static_cast<size_t>(st) * tp.stage >= tp.scratch; --st) {
+            const size_t sm = tp.smem - static_cast<size_t>(tp.stages - st) * tp.stage;
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
+            int n = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kTcThreads, sm) != cudaSuccess) {
+              cudaGetLastError();
+              break;
+            }
+            if (st == tp.stages) nb = std::max(n, 1);
+            if (static_cast<long long>(n) * sms >= G) {
+              a.stages = st;
+              smem = sm;
+              nb = n;
+              break;
+            }
+          }
+        }
+        // CTAs that share an SM split its 512 tensor-memory columns.
+        const long long per_sm = std::min<long long>(nb, (G + sms - 1) / sms);
+        while (a.tmem_cap > tp.Epad && a.tmem_cap * per_sm > 512) a.tmem_cap >>= 1;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        return launch_pdl_cluster(kern, grid, dim3(kTcThreads), smem, s, tp.KS, tx, tw, a);
       }
       auto kern = tp.tma_b ? router_tc<true, 0> : router_tc<false, 0>;
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
