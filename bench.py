@@ -64,6 +64,10 @@ def parse():
     p.add_argument("--gather-in-gemm", action="store_true",
                    help="bf16: gather x rows inside the up projection (tile::gather4) instead of "
                         "the gather kernel")
+    p.add_argument("--combine-in-gemm", action="store_true",
+                   help="bf16, k = 1: the combine in the down projection's epilogue (no combine "
+                        "kernel, no y_perm)")
+    p.add_argument("--k", type=int, default=None, help="override top-k (e.g. 1 for --combine-in-gemm)")
     p.add_argument("--T", type=int, default=None, help="override T (reduced case for profiling)")
     p.add_argument("--E", type=int, default=None, help="override E (reduced case for profiling)")
     p.add_argument("--F", type=int, default=None, help="override F (reduced case for profiling)")
@@ -75,6 +79,8 @@ def shape_of(args):
     if args.T is not None or args.E is not None or args.F is not None:
         sh = sh.with_(T=args.T or sh.T, E=args.E or sh.E, F=args.F or sh.F,
                       name=f"{sh.name}_T{args.T or sh.T}_E{args.E or sh.E}_F{args.F or sh.F}")
+    if args.k is not None and args.k != sh.k:
+        sh = sh.with_(k=args.k, name=f"{sh.name}_k{args.k}")
     return sh
 
 
@@ -88,7 +94,7 @@ def workload_config(sh):
 
 
 # ------------------------------------------------------------------ roofline
-def algorithmic(sh, counts_kept, bucket_rows=None):
+def algorithmic(sh, counts_kept, bucket_rows=None, combine_in_gemm=False):
     """Algorithmic flops and bytes per stage for one forward (no re-reads).
 
     R = kept rows, E_act = experts with R_e > 0, b = element bytes.
@@ -101,7 +107,9 @@ def algorithmic(sh, counts_kept, bucket_rows=None):
       ffn_up   flops 2*R*d*F*(2 SwiGLU | 1 GELU); bytes weights of active
                experts + R*d*b (A rows: x_perm, or x gathered) + R*F*b
       ffn_down flops 2*R*F*d; bytes E_act*F*d*b + R*F*b + R*d*b
-      combine  bytes R*d*b + S*8 + T*d*b
+      combine  bytes R*d*b + S*8 + T*d*b; with --combine-in-gemm no separate
+               stage (the down projection writes its R rows to out; the
+               gather kernel also zeroes the T - R rows of dropped tokens, k = 1)
     """
     b = 2 if sh.dtype == "bf16" else 4
     T, d, E, k, F = sh.T, sh.d, sh.E, sh.k, sh.F
@@ -109,10 +117,12 @@ def algorithmic(sh, counts_kept, bucket_rows=None):
     R = int(sum(counts_kept))
     e_act = int(sum(1 for c in counts_kept if c > 0))
     nup = 2 if sh.act == "swiglu" else 1
+    zeroed = (T - R) if combine_in_gemm else 0
     return {
         "route": {"bytes": T * d * b + d * E * b + S * 8},
         "permute": {"bytes": S * 4 + S * 13},
-        "gather": {"bytes": min(T, R) * d * b + (bucket_rows if bucket_rows is not None else R) * d * b},
+        "gather": {"bytes": min(T, R) * d * b + (bucket_rows if bucket_rows is not None else R) * d * b
+                   + zeroed * d * b},
         "ffn_up": {"flops": 2 * R * d * F * nup,
                    "bytes": e_act * d * F * b * nup + R * d * b + R * F * b},
         "ffn_down": {"flops": 2 * R * F * d, "bytes": e_act * F * d * b + R * F * b + R * d * b},
@@ -425,7 +435,7 @@ def main():
                      w3=None if inp.w3 is None else inp.w3.to(dev),
                      bias=None if inp.bias is None else inp.bias.to(dev),
                      k=sh.k, act=sh.act, capacity_factor=sh.cf, gather_in_gemm=args.gather_in_gemm,
-                     binned=args.binned)
+                     binned=args.binned, combine_in_gemm=args.combine_in_gemm)
     out = torch.empty(sh.T, sh.d, dtype=x.dtype, device=dev)
     aux = torch.empty(1, dtype=torch.float32, device=dev)
     flush = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
@@ -491,7 +501,7 @@ def main():
     # events also span the host's enqueue of each launch.
     stage_ms = {s: statistics.median(bevs[i][j].elapsed_time(bevs[i][j + 1]) for i in range(nb))
                 for j, s in enumerate(STAGES)}
-    alg = algorithmic(sh, kept, bucket_rows)
+    alg = algorithmic(sh, kept, bucket_rows, combine_in_gemm=args.combine_in_gemm)
     peaks = load_peaks()
     # A timed region long enough to hit the 1 kW power cap is compared with the
     # sustained (power-capped) GEMM figure, a short one with the burst figure.
@@ -504,8 +514,11 @@ def main():
     for s in STAGES:
         t = stage_ms[s] * 1e-3
         a = alg[s]
-        if s == "gather" and args.gather_in_gemm and sh.dtype == "bf16":
+        if s == "gather" and args.gather_in_gemm and sh.dtype == "bf16" and not args.combine_in_gemm:
             roof[s] = {"us": stage_ms[s] * 1e3, "fused_into": "ffn_up (tile::gather4 A loads)"}
+            continue
+        if s == "combine" and args.combine_in_gemm:
+            roof[s] = {"us": stage_ms[s] * 1e3, "fused_into": "ffn_down (epilogue)"}
             continue
         r = {"us": stage_ms[s] * 1e3, "GB_s": a["bytes"] / t / 1e9 if t > 0 else None}
         r["hbm_frac"] = r["GB_s"] / peaks["hbm_gbs"] if r["GB_s"] else None
@@ -555,7 +568,8 @@ def main():
         "config": dict(workload_config(sh), parallelism=f"replicas x{world}" if world > 1 else "1 GPU",
                        **({"gather": "in the up projection (tile::gather4)"} if args.gather_in_gemm else {}),
                        **({"layout": f"binned [E, C, d], C = {bucket_rows // sh.E if sh.E else 0}"}
-                          if args.binned else {})),
+                          if args.binned else {}),
+                       **({"combine": "in the down projection's epilogue"} if args.combine_in_gemm else {})),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks,

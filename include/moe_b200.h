@@ -128,6 +128,15 @@ typedef struct {
 /* MOE_LAYER_Z_LOSS: moe_forward also computes the router z-loss (see
  * moe_route_train) into the workspace (moe_views_t.z_loss). */
 #define MOE_LAYER_Z_LOSS 4
+/* MOE_LAYER_COMBINE_IN_GEMM (bf16, k = 1 only; MOE_ERR_UNSUPPORTED
+ * otherwise): the combine runs in the down projection's epilogue ("MegaBlocks"
+ * section 4.3 multiplies each expert output by its gate weight as it is
+ * scattered back to the token). Each row's output, rounded to bf16 as y_perm
+ * would hold it, is multiplied by its slot's weight in fp32 and written
+ * straight to its token's row of out; the gather kernel zeroes the rows of
+ * tokens whose slot was dropped. No combine kernel and no y_perm; out is the
+ * same as the default path's bit for bit. */
+#define MOE_LAYER_COMBINE_IN_GEMM 8
 
 /* Device pointers into a moe_forward workspace where that call leaves its
  * intermediate results (see moe_forward_views). */
@@ -146,7 +155,7 @@ typedef struct {
   uint8_t* drop_mask;    /* [T * k] */
   void* x_perm;          /* [rows_max, d]; NULL with MOE_LAYER_GATHER_IN_GEMM */
   void* h;               /* [rows_max, F] */
-  void* y_perm;          /* [rows_max, d] */
+  void* y_perm;          /* [rows_max, d]; NULL with MOE_LAYER_COMBINE_IN_GEMM */
   int64_t rows_max;
   int64_t capacity;      /* C, or -1 when dropless */
 } moe_views_t;
@@ -346,7 +355,10 @@ MOE_API moe_status_t moe_combine(const void* y_perm, const float* topk_w, const 
  * The whole layer on one stream with no host synchronisation: route ->
  * permute -> gather -> expert FFN (up, down) -> combine. With
  * MOE_LAYER_GATHER_IN_GEMM the gather is part of the up projection and the
- * "gather" events bracket no work.
+ * "gather" events bracket only the zeroing of dropped tokens' rows (with
+ * MOE_LAYER_COMBINE_IN_GEMM) or no work; with MOE_LAYER_COMBINE_IN_GEMM the
+ * combine is part of the down projection and the "combine" events bracket
+ * no work.
  *   x [T, d], out [T, d] (dtype); aux_loss out [1] fp32 device or NULL.
  *   events: NULL, or 7 cudaEvent_t recorded on `stream` before route and
  *   after route, permute, gather, up-projection, down-projection, combine.

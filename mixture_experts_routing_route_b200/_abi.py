@@ -23,7 +23,7 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_NULL", 2: "MOE_ERR_INVALID", 3: "MOE_ERR_UNSU
           4: "MOE_ERR_WORKSPACE", 5: "MOE_ERR_ALIGN", 6: "MOE_ERR_CUDA", 7: "MOE_ERR_DEVICE"}
 MOE_F32, MOE_BF16 = 0, 1
 MOE_ACT_GELU, MOE_ACT_SWIGLU = 0, 1
-MOE_LAYER_GATHER_IN_GEMM, MOE_LAYER_BINNED, MOE_LAYER_Z_LOSS = 1, 2, 4
+MOE_LAYER_GATHER_IN_GEMM, MOE_LAYER_BINNED, MOE_LAYER_Z_LOSS, MOE_LAYER_COMBINE_IN_GEMM = 1, 2, 4, 8
 DEVERR_EXPERT_RANGE, DEVERR_ROW_RANGE, DEVERR_TIMEOUT = 1, 2, 4
 
 

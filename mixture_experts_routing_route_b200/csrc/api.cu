@@ -101,6 +101,10 @@ bool gather_in_gemm(const moe_layer_t* L) {
   return L->dtype == MOE_BF16 && (L->flags & MOE_LAYER_GATHER_IN_GEMM) != 0;
 }
 
+bool combine_in_gemm(const moe_layer_t* L) {
+  return L->dtype == MOE_BF16 && L->k == 1 && (L->flags & MOE_LAYER_COMBINE_IN_GEMM) != 0;
+}
+
 FwdLayout fwd_layout(const moe_layer_t* L, int T, void* ws, bool host_io) {
   FwdLayout f{};
   Carver c(ws);
@@ -130,7 +134,8 @@ FwdLayout fwd_layout(const moe_layer_t* L, int T, void* ws, bool host_io) {
   // itself and there is no x_perm.
   f.x_perm = gather_in_gemm(L) ? nullptr : c.take(R * L->d * es);
   f.h = c.take(R * L->F * es);
-  f.y_perm = c.take(R * L->d * es);
+  // With MOE_LAYER_COMBINE_IN_GEMM the down projection writes out itself.
+  f.y_perm = combine_in_gemm(L) ? nullptr : c.take(R * L->d * es);
   if (host_io) {
     f.x_dev = c.take(static_cast<size_t>(T) * L->d * es);
     f.out_dev = c.take(static_cast<size_t>(T) * L->d * es);
@@ -145,11 +150,14 @@ moe_status_t check_layer(const moe_layer_t* L, int T) {
   MOE_CHECK(check_ffn(L->dtype, L->F));
   if (L->act != MOE_ACT_GELU && L->act != MOE_ACT_SWIGLU) return MOE_ERR_INVALID;
   if (!std::isfinite(L->capacity_factor)) return MOE_ERR_INVALID;
-  if ((L->flags & ~(MOE_LAYER_GATHER_IN_GEMM | MOE_LAYER_BINNED | MOE_LAYER_Z_LOSS)) != 0)
+  if ((L->flags & ~(MOE_LAYER_GATHER_IN_GEMM | MOE_LAYER_BINNED | MOE_LAYER_Z_LOSS |
+                    MOE_LAYER_COMBINE_IN_GEMM)) != 0)
     return MOE_ERR_INVALID;
   MOE_OPT(L->x_router);
   MOE_OPT(L->logit_noise);
   if ((L->flags & MOE_LAYER_GATHER_IN_GEMM) && L->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if ((L->flags & MOE_LAYER_COMBINE_IN_GEMM) && (L->dtype != MOE_BF16 || L->k != 1))
+    return MOE_ERR_UNSUPPORTED;
   MOE_NEED(L->w_router);
   MOE_NEED(L->w1);
   MOE_NEED(L->w2);
@@ -175,18 +183,23 @@ moe_status_t run_forward(const moe_layer_t* L, const void* x, int T, void* out, 
                                      f.slot_to_row, f.row_slot, f.drop, f.kept, f.seg, f.rank,
                                      f.ctl, s, binned(L))));
   rec(2);
-  if (!gather_in_gemm(L))
+  const bool cig = combine_in_gemm(L);
+  // the gather kernel also zeroes the output rows of fully dropped tokens
+  // when the down projection writes out
+  if (!gather_in_gemm(L) || cig)
     MOE_CHECK(from_cuda(launch_gather(x, es, T, L->d, L->k, f.row_slot, f.seg, L->E, f.rows_max,
-                                      f.x_perm, f.ctl, s, binned(L))));
+                                      f.x_perm, f.ctl, s, binned(L), cig ? f.slot_to_row : nullptr,
+                                      cig ? out : nullptr)));
   rec(3);
   cudaEvent_t after_up = (ev != nullptr) ? reinterpret_cast<cudaEvent_t>(ev[4]) : nullptr;
   if (L->dtype == MOE_BF16) {
     const bool g = gather_in_gemm(L);
+    const CombineOut co{f.row_slot, f.w, out, T};
     MOE_CHECK(from_cuda(launch_ffn_bf16(g ? x : f.x_perm, g ? T : f.rows_max,
                                         g ? f.row_slot : nullptr, L->k, L->w1, L->w3, L->w2,
                                         L->act, f.rows_max, L->d, L->F, L->E, f.seg,
                                         binned(L) ? f.kept : nullptr, f.h, f.y_perm, f.ctl, s,
-                                        after_up)));
+                                        after_up, cig ? &co : nullptr)));
   } else {
     MOE_CHECK(from_cuda(launch_ffn_f32(static_cast<const float*>(f.x_perm),
                                        static_cast<const float*>(L->w1),
@@ -196,8 +209,9 @@ moe_status_t run_forward(const moe_layer_t* L, const void* x, int T, void* out, 
                                        static_cast<float*>(f.y_perm), f.ctl, s, after_up)));
   }
   rec(5);
-  MOE_CHECK(from_cuda(launch_combine(f.y_perm, f.w, f.slot_to_row, es, T, L->d, L->k, f.rows_max,
-                                     out, f.ctl, s)));
+  if (!cig)
+    MOE_CHECK(from_cuda(launch_combine(f.y_perm, f.w, f.slot_to_row, es, T, L->d, L->k, f.rows_max,
+                                       out, f.ctl, s)));
   rec(6);
   if (aux_user != nullptr && aux_user != f.aux)
     MOE_CHECK(from_cuda(cudaMemcpyAsync(aux_user, f.aux, 4, cudaMemcpyDeviceToDevice, s)));

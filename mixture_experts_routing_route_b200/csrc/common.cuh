@@ -134,19 +134,31 @@ cudaError_t launch_jitter(const void* x, moe_dtype_t dt, long long n, float eps,
 cudaError_t launch_logit_noise(long long n, float std, uint64_t seed, float* out, cudaStream_t s);
 
 // Gather. binned: rows with row_slot -1 are padding and are written as zeros.
+// zero_out (with slot_to_row [T, k]): also zero the [T, d] output rows of
+// tokens none of whose slots was kept (the combine runs in the down
+// projection). x_perm NULL: only that zeroing.
 cudaError_t launch_gather(const void* x, size_t elem, int T, int d, int k, const int32_t* row_slot,
                           const int32_t* seg, int E, int64_t rows_max, void* x_perm, Control* ctl,
-                          cudaStream_t s, bool binned = false);
+                          cudaStream_t s, bool binned = false, const int32_t* slot_to_row = nullptr,
+                          void* zero_out = nullptr);
 
 // Grouped GEMMs. bf16: A is x_perm [rows_max, d] when row_slot is NULL, else
 // the token rows x [a_rows = T, d], gathered by the up projection itself
 // (row r reads token row_slot[r] / k). Expert e's rows start at seg[e]; there
 // are kept[e] of them (binned layout), or seg[e + 1] - seg[e] when kept is NULL.
+// The combine folded into the down projection (k = 1): each row's output,
+// scaled by w[slot], goes to out[slot / k]; y is not written.
+struct CombineOut {
+  const int32_t* row_slot;  // [rows_max] slot of each row (-1: binned padding)
+  const float* w;           // [T * k] top-k weights
+  void* out;                // [T, d] layer output
+  int T;
+};
 cudaError_t launch_ffn_bf16(const void* a, int64_t a_rows, const int32_t* row_slot, int k,
                             const void* w1, const void* w3, const void* w2, moe_act_t act,
                             int64_t rows_max, int d, int F, int E, const int32_t* seg,
                             const int32_t* kept, void* h, void* y, Control* ctl, cudaStream_t s,
-                            cudaEvent_t after_up);
+                            cudaEvent_t after_up, const CombineOut* comb = nullptr);
 cudaError_t launch_ffn_f32(const float* x_perm, const float* w1, const float* w3, const float* w2,
                            moe_act_t act, int64_t rows_max, int d, int F, int E,
                            const int32_t* seg, float* h, float* y, Control* ctl, cudaStream_t s,

@@ -27,14 +27,17 @@ constexpr int kGatherPiece = 8192;  // bytes per buffer
 __global__ void __launch_bounds__(kGatherWarps * 32)
 gather_bulk(const uint8_t* __restrict__ x, uint32_t row_bytes, int T, int k,
             const int32_t* __restrict__ row_slot, const int32_t* __restrict__ seg, int E,
-            long long rows_max, int binned, uint8_t* __restrict__ x_perm, Control* ctl) {
+            long long rows_max, int binned, uint8_t* __restrict__ x_perm,
+            const int32_t* __restrict__ slot_to_row, uint8_t* __restrict__ zero_out, Control* ctl) {
   pdl_begin();
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t bars[kGatherWarps][kGatherBufs];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  // Binned layout: a padding row (row_slot -1) is stored from a zero piece.
+  // Binned layout: a padding row (row_slot -1) is stored from a zero piece;
+  // so is the layer output row of a token whose every slot was dropped, when
+  // the combine runs in the down projection (zero_out = the output).
   uint8_t* zero = smem + static_cast<size_t>(kGatherWarps) * kGatherBufs * kGatherPiece;
-  if (binned) {
+  if (binned || zero_out != nullptr) {
     for (int i = threadIdx.x; i < kGatherPiece / 16; i += blockDim.x)
       reinterpret_cast<uint4*>(zero)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();  // generic writes, read by the bulk stores
@@ -47,9 +50,11 @@ gather_bulk(const uint8_t* __restrict__ x, uint32_t row_bytes, int T, int k,
     set_error(ctl, MOE_DEVERR_ROW_RANGE);
     R = R < 0 ? 0 : rows_max;
   }
+  if (x_perm == nullptr) R = 0;  // the up projection gathers: output zeroing only
   const long long S = static_cast<long long>(T) * k;
   const uint32_t ppr = (row_bytes + kGatherPiece - 1) / kGatherPiece;  // pieces per row
-  const long long total = R * ppr;
+  const long long rowp = R * ppr;  // pieces of gathered rows, then of output rows
+  const long long total = rowp + (zero_out != nullptr ? static_cast<long long>(T) * ppr : 0);
   const long long gw = static_cast<long long>(blockIdx.x) * kGatherWarps + warp;
   const long long tw = static_cast<long long>(gridDim.x) * kGatherWarps;
   if (gw >= total) return;
@@ -64,6 +69,16 @@ gather_bulk(const uint8_t* __restrict__ x, uint32_t row_bytes, int T, int k,
   // other bad slot index is reported and the piece is skipped (size 0).
   auto piece = [&](long long i, const uint8_t*& src, uint8_t*& dst, uint32_t& bytes) {
     const long long p = gw + i * tw;
+    if (p >= rowp) {  // output row of token t: zero when none of its k slots was kept
+      const long long q = p - rowp, t = q / ppr;
+      const uint32_t off = static_cast<uint32_t>(q % ppr) * kGatherPiece;
+      bool kept = false;
+      for (int j = 0; j < k; ++j) kept |= __ldg(slot_to_row + t * k + j) >= 0;
+      bytes = kept ? 0u : min(static_cast<uint32_t>(kGatherPiece), row_bytes - off);
+      src = nullptr;
+      dst = zero_out + static_cast<size_t>(t) * row_bytes + off;
+      return;
+    }
     const long long row = p / ppr;
     const uint32_t off = static_cast<uint32_t>(p % ppr) * kGatherPiece;
     const int slot = __ldg(row_slot + row);
@@ -285,15 +300,16 @@ cudaError_t launch_combine_t(const T* y, const float* w, const int32_t* s2r, int
 
 cudaError_t launch_gather(const void* x, size_t elem, int T, int d, int k, const int32_t* row_slot,
                           const int32_t* seg, int E, int64_t rows_max, void* x_perm, Control* ctl,
-                          cudaStream_t s, bool binned) {
-  if (rows_max <= 0 || T <= 0) return cudaSuccess;
+                          cudaStream_t s, bool binned, const int32_t* slot_to_row, void* zero_out) {
+  if (T <= 0 || (rows_max <= 0 && zero_out == nullptr)) return cudaSuccess;
   const uint32_t row_bytes = static_cast<uint32_t>(static_cast<size_t>(d) * elem);
   // the ring of every warp, then one zero piece (binned padding rows)
   const size_t smem = static_cast<size_t>(kGatherWarps) * kGatherBufs * kGatherPiece + kGatherPiece;
   cudaFuncSetAttribute(gather_bulk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   return launch_pdl(gather_bulk, dim3(num_sms()), dim3(kGatherWarps * 32), smem, s, false,
                     static_cast<const uint8_t*>(x), row_bytes, T, k, row_slot, seg, E, rows_max,
-                    binned ? 1 : 0, static_cast<uint8_t*>(x_perm), ctl);
+                    binned ? 1 : 0, static_cast<uint8_t*>(x_perm), slot_to_row,
+                    static_cast<uint8_t*>(zero_out), ctl);
 }
 
 cudaError_t launch_combine(const void* y, const float* w, const int32_t* slot_to_row, size_t elem,

@@ -43,12 +43,17 @@ constexpr int kThreads = 192;
 constexpr int kMaxE = 256;
 constexpr int kBoxBytes = 64 * BK * 2;  // one 64-column B box: 8 KB
 
-enum { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_STORE = 2 };
+// EPI_COMBINE (down projection, k = 1): each row, rounded to bf16 as
+// EPI_STORE would store it, is scaled by its slot's top-k weight in fp32
+// (fmaf(w, y, 0), the combine's own arithmetic for one slot), rounded again
+// and stored at its token's row of the layer output.
+enum { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_STORE = 2, EPI_COMBINE = 3 };
 
 struct GemmArgs {
   const int32_t* seg;       // [E+1] row segment offsets
   __nv_bfloat16* out;       // [rows_max, N]
-  const int32_t* row_slot;  // gathering A: slot of each row (token = slot / k)
+  const int32_t* row_slot;  // gathering A, or EPI_COMBINE: slot of each row (token = slot / k)
+  const float* comb_w;      // EPI_COMBINE: top-k weight of each slot
   const int32_t* kept;      // [E] rows of each expert from seg[e] (binned layout), or null:
                             // seg[e + 1] - seg[e]
   int k;
@@ -56,6 +61,7 @@ struct GemmArgs {
   int K;
   int N;  // output columns
   long long rows_max;
+  long long slots;  // EPI_COMBINE: T * k (slot indices are checked against it)
   Control* ctl;
 };
 
@@ -173,9 +179,24 @@ constexpr int kStageRow = 128 + 16;            // bytes per staged row (16 B pad
 constexpr int kStageWarpBytes = 32 * kStageRow;
 
 template <int EPI, int OUTN>
-__device__ __forceinline__ void epilogue_staged(uint32_t tbase, uint8_t* buf, __nv_bfloat16* out,
+__device__ __forceinline__ void epilogue_staged(uint32_t tbase, uint8_t* buf, const GemmArgs& args,
                                                 long long row_base, int nrows, int N, int n0,
                                                 int lane) {
+  __nv_bfloat16* out = args.out;
+  // EPI_COMBINE: this lane's row -> (token, weight); -1: nothing to store
+  int tok = -1;
+  float wgt = 0.f;
+  if constexpr (EPI == EPI_COMBINE) {
+    if (lane < nrows) {
+      const int slot = __ldg(args.row_slot + row_base + lane);
+      if (slot >= 0 && slot < args.slots) {
+        tok = slot / args.k;
+        wgt = __ldg(args.comb_w + slot);
+      } else if (slot >= args.slots) {
+        set_error(args.ctl, MOE_DEVERR_ROW_RANGE);
+      }
+    }
+  }
 #pragma unroll 1
   for (int g = 0; g < OUTN; g += 64) {
 #pragma unroll
@@ -201,6 +222,10 @@ __device__ __forceinline__ void epilogue_staged(uint32_t tbase, uint8_t* buf, __
         for (int i = 0; i < 16; ++i) {
           float a = __uint_as_float(v[2 * i]), b = __uint_as_float(v[2 * i + 1]);
           if (EPI == EPI_GELU) { a = gelu_erf(a); b = gelu_erf(b); }
+          if (EPI == EPI_COMBINE) {
+            a = fmaf(wgt, __bfloat162float(__float2bfloat16_rn(a)), 0.f);
+            b = fmaf(wgt, __bfloat162float(__float2bfloat16_rn(b)), 0.f);
+          }
           packed[i] = pack_bf16(a, b);
         }
       }
@@ -214,9 +239,11 @@ __device__ __forceinline__ void epilogue_staged(uint32_t tbase, uint8_t* buf, __
 #pragma unroll
     for (int it = 0; it < 8; ++it) {
       const int rr = it * 4 + rsub;
-      if (rr < nrows) {
+      long long dst = row_base + rr;
+      if constexpr (EPI == EPI_COMBINE) dst = __shfl_sync(0xffffffffu, tok, rr);
+      if (rr < nrows && dst >= 0) {
         const uint4 val = *reinterpret_cast<const uint4*>(buf + rr * kStageRow + cq * 16);
-        *reinterpret_cast<uint4*>(out + static_cast<size_t>(row_base + rr) * N + n0 + g + cq * 8) = val;
+        *reinterpret_cast<uint4*>(out + static_cast<size_t>(dst) * N + n0 + g + cq * 8) = val;
       }
     }
     __syncwarp();
@@ -270,7 +297,7 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 const __grid_constant__ CUtensorMap tmB1, GemmArgs args) {
   pdl_begin();
   using C = Cfg<EPI, NMMA>;
-  static_assert(!GATHER || EPI != EPI_STORE, "only the up projection gathers");
+  static_assert(!GATHER || (EPI != EPI_STORE && EPI != EPI_COMBINE), "only the up projection gathers");
   // A half-width unit still loads whole 64-column boxes: gate and up halves
   // need at least one box each under SwiGLU.
   static_assert(EPI == EPI_SWIGLU ? NMMA >= 256 : NMMA >= 128, "half units need whole boxes");
@@ -485,9 +512,9 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         const int wrow = m64 ? q * 16 : q * 32;
         const int nrows = max(0, min(m64 ? 16 : 32, t.rows - wrow));
         if (t.half)
-          epilogue_staged<EPI, C::OUT_N / 2>(tbase, buf, args.out, t.row0 + wrow, nrows, args.N, t.n0, lane);
+          epilogue_staged<EPI, C::OUT_N / 2>(tbase, buf, args, t.row0 + wrow, nrows, args.N, t.n0, lane);
         else
-          epilogue_staged<EPI, C::OUT_N>(tbase, buf, args.out, t.row0 + wrow, nrows, args.N, t.n0, lane);
+          epilogue_staged<EPI, C::OUT_N>(tbase, buf, args, t.row0 + wrow, nrows, args.N, t.n0, lane);
       }
       tc_fence_before();
       __syncwarp();
@@ -540,7 +567,8 @@ namespace {
 template <int EPI, int NMMA, bool GATHER>
 cudaError_t run_gemm(const void* A, int64_t a_rows, const int32_t* row_slot, int k, const void* B0,
                      const void* B1, int64_t rows_max, int K, int N, int E, const int32_t* seg,
-                     const int32_t* kept, void* out, Control* ctl, cudaStream_t s) {
+                     const int32_t* kept, void* out, Control* ctl, cudaStream_t s,
+                     const float* comb_w = nullptr, long long slots = 0) {
   using C = Cfg<EPI, NMMA>;
   CUtensorMap ta, tb0, tb1;
   if (!make_tma_2d_bf16(&ta, A, static_cast<uint64_t>(a_rows), K, GATHER ? 1 : BM))
@@ -557,6 +585,8 @@ cudaError_t run_gemm(const void* A, int64_t a_rows, const int32_t* row_slot, int
   a.K = K;
   a.N = N;
   a.rows_max = rows_max;
+  a.comb_w = comb_w;
+  a.slots = slots;
   a.ctl = ctl;
   auto kern = grouped_gemm_tc<EPI, NMMA, GATHER>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM));
@@ -584,7 +614,7 @@ cudaError_t launch_ffn_bf16(const void* a, int64_t a_rows, const int32_t* row_sl
                             const void* w1, const void* w3, const void* w2, moe_act_t act,
                             int64_t rows_max, int d, int F, int E, const int32_t* seg,
                             const int32_t* kept, void* h, void* y, Control* ctl, cudaStream_t s,
-                            cudaEvent_t after_up) {
+                            cudaEvent_t after_up, const CombineOut* comb) {
   if (rows_max <= 0) {
     if (after_up) cudaEventRecord(after_up, s);
     return cudaSuccess;
@@ -596,6 +626,14 @@ cudaError_t launch_ffn_bf16(const void* a, int64_t a_rows, const int32_t* row_sl
                           s);
   if (err != cudaSuccess) return err;
   if (after_up) cudaEventRecord(after_up, s);
+  if (comb != nullptr) {  // k = 1: the combine in the down projection's epilogue
+    const long long slots = static_cast<long long>(comb->T) * k;
+    if (d % 256 == 0)
+      return run_gemm<EPI_COMBINE, 256, false>(h, rows_max, comb->row_slot, k, w2, nullptr, rows_max, F,
+                                               d, E, seg, kept, comb->out, ctl, s, comb->w, slots);
+    return run_gemm<EPI_COMBINE, 128, false>(h, rows_max, comb->row_slot, k, w2, nullptr, rows_max, F,
+                                             d, E, seg, kept, comb->out, ctl, s, comb->w, slots);
+  }
   if (d % 256 == 0)
     err = run_gemm<EPI_STORE, 256, false>(h, rows_max, nullptr, 1, w2, nullptr, rows_max, F, d, E,
                                           seg, kept, y, ctl, s);

@@ -18,7 +18,8 @@ class MoeLayer:
     def __init__(self, w_router: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
                  w3: Optional[torch.Tensor] = None, bias: Optional[torch.Tensor] = None,
                  k: int = 2, act: str = "swiglu", capacity_factor: float = 0.0,
-                 gather_in_gemm: bool = False, binned: bool = False, z_loss: bool = False):
+                 gather_in_gemm: bool = False, binned: bool = False, z_loss: bool = False,
+                 combine_in_gemm: bool = False):
         if not w1.is_cuda:
             raise ValueError("weights must be CUDA tensors")
         self.E, self.d, self.F = w1.shape
@@ -35,8 +36,11 @@ class MoeLayer:
         # MOE_LAYER_GATHER_IN_GEMM in include/moe_b200.h)
         # binned: the [E, C, hs] bucket layout (MOE_LAYER_BINNED); with
         # capacity_factor <= 0 the bin size is the call's largest expert count
+        # combine_in_gemm: k = 1, bf16: the down projection scales its rows by
+        # the top-k weight and writes out (MOE_LAYER_COMBINE_IN_GEMM)
         flags = (abi.MOE_LAYER_GATHER_IN_GEMM if gather_in_gemm else 0) | \
-            (abi.MOE_LAYER_BINNED if binned else 0) | (abi.MOE_LAYER_Z_LOSS if z_loss else 0)
+            (abi.MOE_LAYER_BINNED if binned else 0) | (abi.MOE_LAYER_Z_LOSS if z_loss else 0) | \
+            (abi.MOE_LAYER_COMBINE_IN_GEMM if combine_in_gemm else 0)
         self.c = abi.layer_struct(self.d, self.E, k, self.F, abi.dtype_code(self.dtype), self.act,
                                   self.cf, self.w_router, self.bias, self.w1, self.w3, self.w2,
                                   flags)
@@ -116,7 +120,8 @@ class MoeLayer:
             # no x_perm when the up projection gathers x rows itself
             "x_perm": view(v.x_perm, R * self.d, self.dtype, (R, self.d)) if v.x_perm else None,
             "h": view(v.h, R * self.F, self.dtype, (R, self.F)),
-            "y_perm": view(v.y_perm, R * self.d, self.dtype, (R, self.d)),
+            # no y_perm when the down projection writes the output itself
+            "y_perm": view(v.y_perm, R * self.d, self.dtype, (R, self.d)) if v.y_perm else None,
             "rows_max": R,
             "capacity": v.capacity,
         }

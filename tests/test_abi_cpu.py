@@ -61,6 +61,11 @@ def test_workspace_sizes_grow(abi):
     Lg = abi.MoeLayerC(4096, 8, 2, 14336, abi.MOE_BF16, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, 16, 16,
                        abi.MOE_LAYER_GATHER_IN_GEMM)
     assert abi.moe_forward_workspace_size(Lg, 4096) == n - 8192 * 4096 * 2
+    # the combine inside the down projection (k = 1) drops y_perm
+    L1 = abi.MoeLayerC(4096, 8, 1, 14336, abi.MOE_BF16, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, 16, 16)
+    Lc = abi.MoeLayerC(4096, 8, 1, 14336, abi.MOE_BF16, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, 16, 16,
+                       abi.MOE_LAYER_COMBINE_IN_GEMM)
+    assert abi.moe_forward_workspace_size(Lc, 4096) == abi.moe_forward_workspace_size(L1, 4096) - 4096 * 4096 * 2
     assert abi.moe_forward_host_workspace_size(L, 4096) >= n + 2 * 4096 * 4096 * 2
 
 
@@ -90,8 +95,15 @@ def test_argument_checks_return_before_launch(abi):
     L2 = abi.MoeLayerC(4096, 8, 2, 128, abi.MOE_BF16, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, None, 16)
     assert abi._lib.moe_forward(ctypes.byref(L2), 16, 4, 16, None, 16, 1 << 40, None, None) == 1
     assert abi._lib.moe_permute(16, 4, 2, 0, -1, *([16] * 8), 16, 1 << 20, None) == 2
-    L3 = abi.MoeLayerC(4096, 8, 2, 128, abi.MOE_BF16, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, 16, 16, 8)
+    L3 = abi.MoeLayerC(4096, 8, 2, 128, abi.MOE_BF16, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, 16, 16, 16)
     assert abi._lib.moe_forward(ctypes.byref(L3), 16, 4, 16, None, 16, 1 << 40, None, None) == 2
+    # the combine in the down projection: bf16 and k = 1 only
+    L5 = abi.MoeLayerC(4096, 8, 2, 128, abi.MOE_BF16, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, 16, 16,
+                       abi.MOE_LAYER_COMBINE_IN_GEMM)
+    assert abi._lib.moe_forward(ctypes.byref(L5), 16, 4, 16, None, 16, 1 << 40, None, None) == 3
+    L6 = abi.MoeLayerC(4096, 8, 1, 128, abi.MOE_F32, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, 16, 16,
+                       abi.MOE_LAYER_COMBINE_IN_GEMM)
+    assert abi._lib.moe_forward(ctypes.byref(L6), 16, 4, 16, None, 16, 1 << 40, None, None) == 3
     L4 = abi.MoeLayerC(4096, 8, 2, 128, abi.MOE_F32, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, 16, 16,
                        abi.MOE_LAYER_GATHER_IN_GEMM)
     assert abi._lib.moe_forward(ctypes.byref(L4), 16, 4, 16, None, 16, 1 << 40, None, None) == 3

@@ -194,6 +194,50 @@ def test_layer_binned(T, d, E, k, F, act, dt, cf, bias):
     assert max_err_ratio(np32(v["y_perm"])[:bn["rows"]][live], y_ref[live]) <= tol
 
 
+@pytest.mark.parametrize("T,d,E,F,act,cf,bias,binned,gig", [
+    (700, 256, 8, 512, "swiglu", 0.0, "none", False, False),      # dropless
+    (1000, 256, 16, 512, "gelu", 1.0, "zipf", False, False),      # capacity drops: zeroed rows
+    (900, 256, 8, 256, "swiglu", 1.25, "expert0", True, False),   # bucket layout
+    (1000, 256, 16, 512, "gelu", 1.0, "zipf", False, True),       # gather in the up projection too
+    (333, 384, 8, 384, "gelu", 0.0, "none", False, False),        # d % 256 != 0: 128-column tiles
+    (300, 256, 8, 256, "swiglu", 0.02, "none", False, False),     # C = 0: every token dropped
+])
+def test_layer_combine_in_gemm(T, d, E, F, act, cf, bias, binned, gig):
+    """k = 1: the combine in the down projection's epilogue
+    (MOE_LAYER_COMBINE_IN_GEMM) writes every output row, the default path's
+    output bit for bit, zero for dropped tokens, within the bf16 tolerance
+    of the oracle."""
+    from mixture_experts_routing_route_b200 import MoeLayer
+    inp = small_case("comb", T=T, d=d, E=E, k=1, F=F, act=act, dtype="bf16", cf=cf, bias=bias,
+                     seed=T + E)
+    dv = device_inputs(inp)
+    mk = lambda c: MoeLayer(dv["wg"], dv["w1"], dv["w2"], w3=dv["w3"], bias=dv["bias"], k=1, act=act,
+                            capacity_factor=cf, binned=binned and c, gather_in_gemm=gig and c,
+                            combine_in_gemm=c)
+    lc, ld = mk(True), mk(False)
+    out_c = torch.full((T, d), float("nan"), dtype=torch.bfloat16, device="cuda")  # rows left unwritten stay NaN
+    lc.forward(dv["x"], out_c)
+    out_d, aux_d = ld.forward(dv["x"])
+    torch.cuda.synchronize()
+    assert lc.device_error(T) == 0 and ld.device_error(T) == 0
+    assert torch.equal(out_c, out_d)
+    v = lc.views(T)
+    assert v["y_perm"] is None
+    # against the oracle, from the GPU's routing
+    g_idx = npi(v["topk_idx"]).astype(np.int64)
+    r = O.route(np32(inp.x), np32(inp.wg), None if inp.bias is None else inp.bias.numpy(), 1)
+    w_ref = O.renormalise(r["probs64"], g_idx)
+    pm = O.permute(g_idx, E, O.capacity(cf, 1, T, E))
+    xp = O.gather(np32(inp.x), pm["row_slot"], 1)
+    w1, w2 = ExpertWeights(inp.w1), ExpertWeights(inp.w2)
+    w3 = None if inp.w3 is None else ExpertWeights(inp.w3)
+    y_ref = O.expert_ffn(xp, pm["seg_offsets"], w1, w3, w2, act)
+    out_ref = O.combine(y_ref, w_ref, pm["slot_to_row"], T, 1)
+    assert max_err_ratio(np32(out_c), out_ref) <= TOL_BF16_OUT
+    dropped = pm["drop"].reshape(T, 1).all(axis=1)
+    assert np.all(np32(out_c)[dropped] == 0.0)
+
+
 def test_layer_training_router_inputs():
     """The router reads jittered x and adds logit noise while the experts read
     x; the z-loss comes back through the views."""
