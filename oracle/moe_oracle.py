@@ -144,15 +144,33 @@ def near_tie_tokens(logits32, k, eps=1e-3):
     return (l[:, k - 1] - l[:, k]) < eps
 
 
-def route(x, wg, bias, k, noise=None):
+def tempered_logits(logits, temperature):
+    """What the router's softmax sees under a temperature tau > 0: l / tau.
+
+    ops-transformer blog, 坑3 (numerical stability): instead of a hard top-K
+    the router takes a softmax with a temperature, so experts that are not
+    picked keep a little probability. The page gives no formula; the plain
+    reading is softmax(l / tau): tau > 1 flattens the probabilities, tau < 1
+    sharpens them, tau = 1 is the plain router. The top-k pick is unchanged
+    (l / tau is increasing in l); the renormalised weights, the aux loss's
+    P_i and the z-loss see l / tau.
+    """
+    if not temperature > 0:
+        raise ValueError("temperature must be > 0")
+    return np.asarray(logits, dtype=np.float64) / float(temperature)
+
+
+def route(x, wg, bias, k, noise=None, temperature=1.0):
     """Router stage: logits, softmax, top-k, renormalised weights, aux loss,
     z-loss. noise: optional [T, E] values added to the logits (the training
-    variant's Gaussian noise)."""
+    variant's Gaussian noise); temperature: the softmax's tau (see
+    tempered_logits)."""
     l64 = gate_logits(x, wg, bias)
     if noise is not None:
         l64 = l64 + np.asarray(noise, dtype=np.float64)
     logits32 = l64.astype(np.float32)
-    p64 = softmax_rows(l64)
+    lt = tempered_logits(l64, temperature)
+    p64 = softmax_rows(lt)
     idx = topk_select(logits32, k)
     w64 = renormalise(p64, idx)
     E = l64.shape[1]
@@ -164,7 +182,7 @@ def route(x, wg, bias, k, noise=None):
         "topk_w64": w64,
         "topk_w": w64.astype(np.float32),
         "aux": aux_loss(p64, idx, E),
-        "z": z_loss(l64),
+        "z": z_loss(lt),
         "near_tie": near_tie_tokens(logits32, k),
     }
 

@@ -492,5 +492,35 @@ def pin_route_noise(o):
     assert abs(r["z"] - o.z_loss(n)) < 1e-12
 
 
-ALL_PINS.extend([pin_philox_kat, pin_jitter, pin_logit_noise, pin_z_loss, pin_route_noise])
+def pin_temperature(o):
+    """Router temperature: two experts give the logistic closed form
+    1 / (1 + exp((b - a) / tau)); the pick does not move; tau = 1 is the
+    plain router; a huge tau gives uniform probabilities, hence aux = 1 for
+    any routing; the z-loss of equal logits c is (c / tau + ln E)^2."""
+    T, d, k = 7, 3, 1
+    x, wg = np.zeros((T, d)), np.zeros((d, 2))
+    a, b = 0.9, 0.2
+    for tau in (0.25, 0.5, 2.0, 10.0):
+        r = o.route(x, wg, np.array([a, b]), k, temperature=tau)
+        assert np.allclose(r["probs64"][:, 0], 1.0 / (1.0 + math.exp((b - a) / tau)), rtol=0, atol=1e-15)
+        assert np.all(r["topk_idx"][:, 0] == 0)
+    rng = _rng(32)
+    T, d, E, k = 40, 16, 8, 2
+    x, wg = rng.standard_normal((T, d)), rng.standard_normal((d, E))
+    base = o.route(x, wg, None, k)
+    same = o.route(x, wg, None, k, temperature=1.0)
+    for key in ("probs64", "topk_w64", "topk_idx"):
+        assert np.array_equal(base[key], same[key])
+    assert base["aux"] == same["aux"] and base["z"] == same["z"]
+    for tau in (0.3, 3.0):
+        assert np.array_equal(o.route(x, wg, None, k, temperature=tau)["topk_idx"], base["topk_idx"])
+    flat = o.route(x, wg, None, k, temperature=1e9)
+    assert np.allclose(flat["probs64"], 1.0 / E, rtol=0, atol=1e-8)
+    assert abs(flat["aux"] - 1.0) < 1e-7
+    c, tau = 2.0, 4.0
+    assert abs(o.z_loss(o.tempered_logits(np.full((3, E), c), tau)) - (c / tau + math.log(E)) ** 2) < 1e-12
+
+
+ALL_PINS.extend([pin_philox_kat, pin_jitter, pin_logit_noise, pin_z_loss, pin_route_noise,
+                 pin_temperature])
 

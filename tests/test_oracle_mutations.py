@@ -102,6 +102,10 @@ def _z_loss_no_square(logits):
     return float(np.mean(m[:, 0] + np.log(np.exp(l - m).sum(axis=1))))
 
 
+def _temperature_ignored(logits, temperature):
+    return np.asarray(logits, dtype=np.float64)
+
+
 def _jitter_half_width(T, d, eps, seed):
     return _REAL["jitter_multipliers"](T, d, eps / 2, seed)
 
@@ -126,6 +130,7 @@ MUTATIONS = {
     "philox_nine_rounds": ("philox4x32_10", _philox_nine_rounds),
     "z_loss_without_square": ("z_loss", _z_loss_no_square),
     "jitter_half_width": ("jitter_multipliers", _jitter_half_width),
+    "temperature_ignored": ("tempered_logits", _temperature_ignored),
 }
 
 
