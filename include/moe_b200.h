@@ -103,9 +103,11 @@ typedef struct {
    *   x_router     the router's input [T, d] (dtype) in place of x, e.g. x
    *                jittered by moe_router_jitter; the experts still read x
    *   logit_noise  [T, E] fp32 added to the gate logits after the bias,
-   *                e.g. from moe_router_noise */
+   *                e.g. from moe_router_noise
+   *   router_temperature  the softmax's tau (see moe_route_train); 0 means 1 */
   const void* x_router;
   const float* logit_noise;
+  float router_temperature;
 } moe_layer_t;
 
 /* moe_layer_t.flags. MOE_LAYER_GATHER_IN_GEMM (bf16 only): moe_forward skips
@@ -218,12 +220,19 @@ MOE_API moe_status_t moe_route(const void* x, const void* w_router, const float*
  *                included). The pages name the loss only (router_z_loss);
  *                this is its usual definition. Deterministic (fixed-order
  *                reductions).
+ *   temperature  tau > 0 (MOE_ERR_INVALID otherwise): the softmax sees
+ *                logits / tau ("ops-transformer MoE operators", 坑3: soft
+ *                top-K, a softmax with a temperature so that experts not
+ *                picked keep some probability; no formula is given, this is
+ *                the plain reading). The pick is unchanged; probabilities,
+ *                weights, the aux loss's P_i and the z-loss use l / tau.
+ *                tau = 1 gives moe_route's results bit for bit.
  * Probabilities, top-k, weights and the aux loss are those of the noisy
  * logits. For jitter, pass the jittered x (moe_router_jitter) as x. */
 MOE_API moe_status_t moe_route_train(const void* x, const void* w_router, const float* bias,
-                             const float* logit_noise, moe_dtype_t dtype, int T, int d, int E,
-                             int k, int32_t* topk_idx, float* topk_w, float* aux_loss,
-                             float* z_loss, float* logits, float* probs, void* ws,
+                             const float* logit_noise, float temperature, moe_dtype_t dtype, int T,
+                             int d, int E, int k, int32_t* topk_idx, float* topk_w,
+                             float* aux_loss, float* z_loss, float* logits, float* probs, void* ws,
                              size_t ws_bytes, moe_stream_t stream);
 
 /* Router jitter ("MegaBlocks", section 5: the router input is multiplied by

@@ -50,7 +50,8 @@ class MoeLayerC(ctypes.Structure):
     _fields_ = [("d", c_int), ("E", c_int), ("k", c_int), ("F", c_int), ("dtype", c_int),
                 ("act", c_int), ("capacity_factor", c_double), ("w_router", c_void_p),
                 ("router_bias", c_void_p), ("w1", c_void_p), ("w3", c_void_p), ("w2", c_void_p),
-                ("flags", c_int), ("x_router", c_void_p), ("logit_noise", c_void_p)]
+                ("flags", c_int), ("x_router", c_void_p), ("logit_noise", c_void_p),
+                ("router_temperature", ctypes.c_float)]
 
 
 class MoeViewsC(ctypes.Structure):
@@ -76,9 +77,9 @@ _SIGS = {
                     + [c_void_p, c_size_t, c_void_p]),
     "moe_permute_noalloc": (c_int, [c_void_p, c_int, c_int, c_int, c_int64] + [c_void_p] * 9
                             + [c_void_p]),
-    "moe_route_train": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int,
-                                c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
-                                c_void_p, c_size_t, c_void_p]),
+    "moe_route_train": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, ctypes.c_float, c_int, c_int,
+                                c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
+                                c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "moe_router_jitter": (c_int, [c_void_p, c_int, c_int, c_int, ctypes.c_float, ctypes.c_uint64,
                                   c_void_p, c_void_p]),
     "moe_router_noise": (c_int, [c_int, c_int, ctypes.c_float, ctypes.c_uint64, c_void_p, c_void_p]),
@@ -193,9 +194,10 @@ def moe_route(x, w_router, bias, T, d, E, k, topk_idx, topk_w, aux_loss, logits,
 
 
 def moe_route_train(x, w_router, bias, logit_noise, T, d, E, k, topk_idx, topk_w, aux_loss, z_loss,
-                    logits, probs, ws, stream=None):
+                    logits, probs, ws, stream=None, temperature=1.0):
     _check("moe_route_train", _lib.moe_route_train(
-        _ptr(x), _ptr(w_router), _ptr(bias), _ptr(logit_noise), dtype_code(x.dtype), T, d, E, k,
+        _ptr(x), _ptr(w_router), _ptr(bias), _ptr(logit_noise), float(temperature),
+        dtype_code(x.dtype), T, d, E, k,
         _ptr(topk_idx), _ptr(topk_w), _ptr(aux_loss), _ptr(z_loss), _ptr(logits), _ptr(probs),
         _ptr(ws), ws.numel(), _stream(stream)))
 
@@ -254,9 +256,10 @@ def moe_combine(y_perm, topk_w, slot_to_row, T, d, k, rows_max, out, ws, stream=
         int(rows_max), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
 
 
-def layer_struct(d, E, k, F, dtype, act, cf, w_router, bias, w1, w3, w2, flags=0) -> MoeLayerC:
+def layer_struct(d, E, k, F, dtype, act, cf, w_router, bias, w1, w3, w2, flags=0,
+                 router_temperature=1.0) -> MoeLayerC:
     return MoeLayerC(d, E, k, F, dtype, act, float(cf), _ptr(w_router), _ptr(bias), _ptr(w1),
-                     _ptr(w3), _ptr(w2), int(flags))
+                     _ptr(w3), _ptr(w2), int(flags), None, None, float(router_temperature))
 
 
 def moe_forward_workspace_size(layer: MoeLayerC, T: int) -> int:

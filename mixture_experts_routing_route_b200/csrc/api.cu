@@ -150,6 +150,7 @@ moe_status_t check_layer(const moe_layer_t* L, int T) {
   MOE_CHECK(check_ffn(L->dtype, L->F));
   if (L->act != MOE_ACT_GELU && L->act != MOE_ACT_SWIGLU) return MOE_ERR_INVALID;
   if (!std::isfinite(L->capacity_factor)) return MOE_ERR_INVALID;
+  if (!(L->router_temperature >= 0.0f) || !std::isfinite(L->router_temperature)) return MOE_ERR_INVALID;
   if ((L->flags & ~(MOE_LAYER_GATHER_IN_GEMM | MOE_LAYER_BINNED | MOE_LAYER_Z_LOSS |
                     MOE_LAYER_COMBINE_IN_GEMM)) != 0)
     return MOE_ERR_INVALID;
@@ -177,7 +178,8 @@ moe_status_t run_forward(const moe_layer_t* L, const void* x, int T, void* out, 
   MOE_CHECK(from_cuda(launch_route(L->x_router != nullptr ? L->x_router : x, L->w_router,
                                    L->router_bias, L->logit_noise, L->dtype, T, L->d, L->E, L->k,
                                    f.idx, f.w, f.aux, (L->flags & MOE_LAYER_Z_LOSS) ? f.z : nullptr,
-                                   nullptr, nullptr, f.logits_scratch, f.partials, f.ctl, s)));
+                                   nullptr, nullptr, f.logits_scratch, f.partials, f.ctl, s,
+                                   L->router_temperature > 0.0f ? L->router_temperature : 1.0f)));
   rec(1);
   MOE_CHECK(from_cuda(launch_permute(f.idx, T, L->k, L->E, f.cap, f.counts, f.bins, f.sorted_slot,
                                      f.slot_to_row, f.row_slot, f.drop, f.kept, f.seg, f.rank,
@@ -284,11 +286,12 @@ size_t moe_route_workspace_size(int T, int d, int E) {
 }
 
 static moe_status_t route_impl(const void* x, const void* w_router, const float* bias,
-                               const float* logit_noise, moe_dtype_t dtype, int T, int d, int E,
-                               int k, int32_t* topk_idx, float* topk_w, float* aux_loss,
-                               float* z_loss, float* logits, float* probs, void* ws,
-                               size_t ws_bytes, moe_stream_t stream) {
+                               const float* logit_noise, float temperature, moe_dtype_t dtype,
+                               int T, int d, int E, int k, int32_t* topk_idx, float* topk_w,
+                               float* aux_loss, float* z_loss, float* logits, float* probs,
+                               void* ws, size_t ws_bytes, moe_stream_t stream) {
   MOE_CHECK(check_dims(dtype, T, d, E, k));
+  if (!(temperature > 0.0f) || !std::isfinite(temperature)) return MOE_ERR_INVALID;
   MOE_NEED(x);
   MOE_NEED(w_router);
   MOE_NEED(topk_idx);
@@ -307,23 +310,23 @@ static moe_status_t route_impl(const void* x, const void* w_router, const float*
   float* scratch = static_cast<float*>(c.take(route_logits_scratch_bytes(T, d, E)));
   return from_cuda(launch_route(x, w_router, bias, logit_noise, dtype, T, d, E, k, topk_idx, topk_w,
                                 aux_loss, z_loss, logits, probs, scratch, partials, ctl,
-                                reinterpret_cast<cudaStream_t>(stream)));
+                                reinterpret_cast<cudaStream_t>(stream), temperature));
 }
 
 moe_status_t moe_route(const void* x, const void* w_router, const float* bias, moe_dtype_t dtype,
                        int T, int d, int E, int k, int32_t* topk_idx, float* topk_w, float* aux_loss,
                        float* logits, float* probs, void* ws, size_t ws_bytes, moe_stream_t stream) {
-  return route_impl(x, w_router, bias, nullptr, dtype, T, d, E, k, topk_idx, topk_w, aux_loss,
+  return route_impl(x, w_router, bias, nullptr, 1.0f, dtype, T, d, E, k, topk_idx, topk_w, aux_loss,
                     nullptr, logits, probs, ws, ws_bytes, stream);
 }
 
 moe_status_t moe_route_train(const void* x, const void* w_router, const float* bias,
-                             const float* logit_noise, moe_dtype_t dtype, int T, int d, int E, int k,
-                             int32_t* topk_idx, float* topk_w, float* aux_loss, float* z_loss,
-                             float* logits, float* probs, void* ws, size_t ws_bytes,
-                             moe_stream_t stream) {
-  return route_impl(x, w_router, bias, logit_noise, dtype, T, d, E, k, topk_idx, topk_w, aux_loss,
-                    z_loss, logits, probs, ws, ws_bytes, stream);
+                             const float* logit_noise, float temperature, moe_dtype_t dtype, int T,
+                             int d, int E, int k, int32_t* topk_idx, float* topk_w,
+                             float* aux_loss, float* z_loss, float* logits, float* probs, void* ws,
+                             size_t ws_bytes, moe_stream_t stream) {
+  return route_impl(x, w_router, bias, logit_noise, temperature, dtype, T, d, E, k, topk_idx, topk_w,
+                    aux_loss, z_loss, logits, probs, ws, ws_bytes, stream);
 }
 
 moe_status_t moe_router_jitter(const void* x, moe_dtype_t dtype, int T, int d, float eps,

@@ -102,11 +102,13 @@ cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, si
 // Router.
 size_t route_partials_bytes(int T, int E);
 // noise: optional [T, E] fp32 added to the logits after the bias; z_out:
-// optional z-loss output (mean over tokens of the squared log-sum-exp).
+// optional z-loss output (mean over tokens of the squared log-sum-exp);
+// temperature: the softmax sees logits / temperature (> 0; 1 = plain).
 cudaError_t launch_route(const void* x, const void* wg, const float* bias, const float* noise,
                          moe_dtype_t dt, int T, int d, int E, int k, int32_t* idx, float* w,
                          float* aux, float* z_out, float* logits, float* probs,
-                         float* logits_scratch, void* partials, Control* ctl, cudaStream_t s);
+                         float* logits_scratch, void* partials, Control* ctl, cudaStream_t s,
+                         float temperature = 1.0f);
 size_t route_logits_scratch_bytes(int T, int d, int E);
 
 // Permute. launch_permute picks the multi-CTA kernel when the slots fit its

@@ -431,7 +431,7 @@ __device__ __forceinline__ float warp_route_token(const float (&v)[EPL], int E, 
                                                  float* __restrict__ logits_out,
                                                  float* __restrict__ probs_out,
                                                  float (&psum)[EPL], int (&cnt)[EPL],
-                                                 Control* ctl) {
+                                                 float inv_tau, Control* ctl) {
 #pragma unroll
   for (int q = 0; q < EPL; ++q) {
     const int e = lane + 32 * q;
@@ -445,7 +445,7 @@ __device__ __forceinline__ float warp_route_token(const float (&v)[EPL], int E, 
   float ex[EPL], s = 0.f;
 #pragma unroll
   for (int q = 0; q < EPL; ++q) {
-    ex[q] = (lane + 32 * q < E) ? expf(v[q] - m) : 0.f;
+    ex[q] = (lane + 32 * q < E) ? expf((v[q] - m) * inv_tau) : 0.f;
     s += ex[q];
   }
 #pragma unroll
@@ -503,7 +503,9 @@ __device__ __forceinline__ float warp_route_token(const float (&v)[EPL], int E, 
     idx_out[t * k + lane] = my_e;
     w_out[t * k + lane] = my_p / wsum;
   }
-  return m + logf(s);  // log-sum-exp of the logits (the z-loss term), same in every lane
+  // log-sum-exp of the logits the softmax sees (l / tau; the z-loss term),
+  // the same in every lane
+  return m * inv_tau + logf(s);
 }
 
 // Warp per token: lane l holds experts l + 32q, q < EPL. The logits are the
@@ -518,7 +520,8 @@ router_select(const float* __restrict__ logits_in, int KS, const float* __restri
               const float* __restrict__ noise, int T, int E, int k, int32_t* __restrict__ idx_out,
               float* __restrict__ w_out, float* __restrict__ logits_out,
               float* __restrict__ probs_out, float* __restrict__ part_p,
-              int32_t* __restrict__ part_c, float* __restrict__ part_z, int ldb, Control* ctl) {
+              int32_t* __restrict__ part_c, float* __restrict__ part_z, int ldb, float inv_tau,
+              Control* ctl) {
   pdl_begin();
   __shared__ float zw[kSelectWarps];
   __shared__ float blk_p_w[kSelectWarps][256];
@@ -562,7 +565,7 @@ router_select(const float* __restrict__ logits_in, int KS, const float* __restri
       if (noise != nullptr && e < E) v[q] += __ldg(noise + static_cast<size_t>(t) * E + e);
     }
     const float lse = warp_route_token<EPL>(v, E, k, lane, static_cast<size_t>(t), idx_out, w_out,
-                                            logits_out, probs_out, psum, cnt, ctl);
+                                            logits_out, probs_out, psum, cnt, inv_tau, ctl);
     zacc += lse * lse;
   }
   if (lane == 0) zw[warp] = zacc;
@@ -619,6 +622,7 @@ struct RouterTcArgs {
   const float* noise;  // [T, E] added to the logits, or null
   float* part_z;       // per-tile z-loss partials, or null (no z-loss)
   float* z_out;        // the z-loss, or null
+  float inv_tau;       // 1 / the softmax temperature (1: the plain router)
 };
 
 // Fused selection, E <= 32. The KS CTAs of one 128-token tile run as a
@@ -748,7 +752,7 @@ __device__ __forceinline__ void select_and_aux(const RouterTcArgs& a, const floa
   float ssum = 0.f;
 #pragma unroll
   for (int e = 0; e < EW; ++e) {
-    p[e] = e < E ? expf(lg[e] - m) : 0.f;
+    p[e] = e < E ? expf((lg[e] - m) * a.inv_tau) : 0.f;
     ssum += p[e];
   }
 #pragma unroll
@@ -798,7 +802,7 @@ __device__ __forceinline__ void select_and_aux(const RouterTcArgs& a, const floa
   __shared__ float zw_s[kTcThreads / 32];
   __shared__ double zd_s[kTcThreads];
   if (a.part_z != nullptr) {
-    const float lse = m + logf(ssum);
+    const float lse = m * a.inv_tau + logf(ssum);  // of the logits the softmax sees, l / tau
     float zt = valid ? lse * lse : 0.f;
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) zt += __shfl_xor_sync(kFull, zt, off);
@@ -1423,7 +1427,9 @@ size_t route_logits_scratch_bytes(int T, int d, int E) {
 cudaError_t launch_route(const void* x, const void* wg, const float* bias, const float* noise,
                          moe_dtype_t dt, int T, int d, int E, int k, int32_t* idx, float* w,
                          float* aux, float* z_out, float* logits, float* probs,
-                         float* logits_scratch, void* partials, Control* ctl, cudaStream_t s) {
+                         float* logits_scratch, void* partials, Control* ctl, cudaStream_t s,
+                         float temperature) {
+  const float inv_tau = 1.0f / temperature;
   const int ldb = route_max_blocks(T);
   float* part_p = static_cast<float*>(partials);
   int32_t* part_c = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(partials) +
@@ -1434,8 +1440,8 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, const
                                    : reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(terms) +
                                                               align_up(256 * 8));
   int nblk = 0;
-  // The fp32 E <= 8 kernel has neither the noise input nor the z-loss.
-  if (use_fused(d, E, dt) && noise == nullptr && z_out == nullptr) {
+  // The fp32 E <= 8 kernel has neither the noise input, the z-loss nor a temperature.
+  if (use_fused(d, E, dt) && noise == nullptr && z_out == nullptr && inv_tau == 1.0f) {
     const int groups = (T + kFusedTokensPerGroup - 1) / kFusedTokensPerGroup;
     const int grid = std::max(1, std::min(groups, num_sms()));
     const size_t smem = fused_smem_bytes(d);
@@ -1462,6 +1468,7 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, const
       a.T = T; a.d = d; a.E = E; a.Epad = tp.Epad; a.KS = tp.KS; a.dk = d / tp.KS;
       a.stages = tp.stages;
       a.tmem_cap = 512;
+      a.inv_tau = inv_tau;
       a.wg = static_cast<const __nv_bfloat16*>(wg);
       a.partial = logits_scratch;
       a.ctl = ctl;
@@ -1555,7 +1562,8 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, const
                         : router_select<8>;
     const cudaError_t e = launch_pdl(sel, dim3(g2), dim3(kSelectWarps * 32), 0, s, false,
                                      static_cast<const float*>(logits_scratch), KS, bias, noise, T,
-                                     E, k, idx, w, logits, probs, part_p, part_c, part_z, ldb, ctl);
+                                     E, k, idx, w, logits, probs, part_p, part_c, part_z, ldb, inv_tau,
+                                     ctl);
     if (e != cudaSuccess) return e;
     nblk = g2;
   }

@@ -19,7 +19,7 @@ class MoeLayer:
                  w3: Optional[torch.Tensor] = None, bias: Optional[torch.Tensor] = None,
                  k: int = 2, act: str = "swiglu", capacity_factor: float = 0.0,
                  gather_in_gemm: bool = False, binned: bool = False, z_loss: bool = False,
-                 combine_in_gemm: bool = False):
+                 combine_in_gemm: bool = False, router_temperature: float = 1.0):
         if not w1.is_cuda:
             raise ValueError("weights must be CUDA tensors")
         self.E, self.d, self.F = w1.shape
@@ -41,9 +41,11 @@ class MoeLayer:
         flags = (abi.MOE_LAYER_GATHER_IN_GEMM if gather_in_gemm else 0) | \
             (abi.MOE_LAYER_BINNED if binned else 0) | (abi.MOE_LAYER_Z_LOSS if z_loss else 0) | \
             (abi.MOE_LAYER_COMBINE_IN_GEMM if combine_in_gemm else 0)
+        # router_temperature: the router softmax sees logits / tau (training
+        # variant; moe_route_train in include/moe_b200.h)
         self.c = abi.layer_struct(self.d, self.E, k, self.F, abi.dtype_code(self.dtype), self.act,
                                   self.cf, self.w_router, self.bias, self.w1, self.w3, self.w2,
-                                  flags)
+                                  flags, router_temperature)
         self._ws = {}
 
     def workspace(self, T: int, host_io: bool = False, stream=None, slot: int = 0) -> torch.Tensor:

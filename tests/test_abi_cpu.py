@@ -107,6 +107,12 @@ def test_argument_checks_return_before_launch(abi):
     L4 = abi.MoeLayerC(4096, 8, 2, 128, abi.MOE_F32, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, 16, 16,
                        abi.MOE_LAYER_GATHER_IN_GEMM)
     assert abi._lib.moe_forward(ctypes.byref(L4), 16, 4, 16, None, 16, 1 << 40, None, None) == 3
+    # the router temperature must be > 0 (moe_route_train) or >= 0 (layer, 0 = 1)
+    assert abi._lib.moe_route_train(16, 16, None, None, 0.0, abi.MOE_BF16, 8, 128, 8, 2, 16, 16, 16,
+                                    None, None, None, 16, 1 << 30, None) == 2
+    L7 = abi.MoeLayerC(4096, 8, 2, 128, abi.MOE_BF16, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, 16, 16,
+                       0, None, None, -1.0)
+    assert abi._lib.moe_forward(ctypes.byref(L7), 16, 4, 16, None, 16, 1 << 40, None, None) == 2
     assert abi.moe_kernel_launches() == n0
 
 

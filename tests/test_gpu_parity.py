@@ -238,9 +238,11 @@ def test_layer_combine_in_gemm(T, d, E, F, act, cf, bias, binned, gig):
     assert np.all(np32(out_c)[dropped] == 0.0)
 
 
-def test_layer_training_router_inputs():
-    """The router reads jittered x and adds logit noise while the experts read
-    x; the z-loss comes back through the views."""
+@pytest.mark.parametrize("tau", [1.0, 1.7])
+def test_layer_training_router_inputs(tau):
+    """The router reads jittered x and adds logit noise (and, tau != 1, runs
+    its softmax at that temperature) while the experts read x; the z-loss
+    comes back through the views."""
     from mixture_experts_routing_route_b200 import MoeLayer, _abi as abi
     T, d, E, k, F = 700, 256, 8, 2, 256
     inp = small_case("train", T=T, d=d, E=E, k=k, F=F, act="swiglu", seed=77)
@@ -249,14 +251,15 @@ def test_layer_training_router_inputs():
     abi.moe_router_jitter(dv["x"], T, d, 0.01, 5, xj)
     noise = torch.empty(T, E, dtype=torch.float32, device="cuda")
     abi.moe_router_noise(T, E, 1.0 / E, 6, noise)
-    layer = MoeLayer(dv["wg"], dv["w1"], dv["w2"], w3=dv["w3"], k=k, act="swiglu", z_loss=True)
+    layer = MoeLayer(dv["wg"], dv["w1"], dv["w2"], w3=dv["w3"], k=k, act="swiglu", z_loss=True,
+                     router_temperature=tau)
     out, aux = layer.forward(dv["x"], x_router=xj, logit_noise=noise)
     torch.cuda.synchronize()
     assert layer.device_error(T) == 0
     v = layer.views(T)
     xj_ref = O.apply_jitter(np32(inp.x), O.jitter_multipliers(T, d, 0.01, 5), True)
     assert np.array_equal(np32(xj), xj_ref)
-    r = O.route(xj_ref, np32(inp.wg), None, k, noise=np32(noise).astype(np.float64))
+    r = O.route(xj_ref, np32(inp.wg), None, k, noise=np32(noise).astype(np.float64), temperature=tau)
     g_idx = npi(v["topk_idx"]).astype(np.int64)
     check_topk_end_to_end(g_idx, r)
     w_ref = O.renormalise(r["probs64"], g_idx)

@@ -347,17 +347,21 @@ def test_router_noise_matches_oracle(T, E):
     assert np.all(np.abs(g - ref) <= 2e-6 * (1.0 + np.abs(ref) * E))
 
 
-@pytest.mark.parametrize("T,d,E,k,dt", [
-    (1000, 1024, 8, 2, "bf16"),    # fused tensor-core router, KS split in a cluster
-    (19500, 512, 8, 2, "bf16"),    # persistent fused router (more tiles than SMs)
-    (300, 512, 32, 4, "bf16"),     # fused, E = 32
-    (513, 256, 64, 2, "bf16"),     # tensor cores (TMA Wg) + router_select + aux_reduce
-    (90, 64, 40, 4, "f32"),        # CUDA-core gate + router_select
-    (200, 64, 4, 1, "f32"),        # fp32 E <= 8: the general path when noise / z-loss are asked
+@pytest.mark.parametrize("T,d,E,k,dt,tau", [
+    (1000, 1024, 8, 2, "bf16", 1.0),    # fused tensor-core router, KS split in a cluster
+    (1000, 1024, 8, 2, "bf16", 0.6),    # ... at a temperature
+    (19500, 512, 8, 2, "bf16", 2.0),    # persistent fused router (more tiles than SMs)
+    (300, 512, 32, 4, "bf16", 1.0),     # fused, E = 32
+    (300, 512, 32, 4, "bf16", 3.0),
+    (513, 256, 64, 2, "bf16", 1.0),     # tensor cores (TMA Wg) + router_select + aux_reduce
+    (513, 256, 64, 2, "bf16", 0.5),
+    (90, 64, 40, 4, "f32", 1.5),        # CUDA-core gate + router_select
+    (200, 64, 4, 1, "f32", 1.0),        # fp32 E <= 8: the general path when noise / z-loss are asked
+    (200, 64, 4, 1, "f32", 2.5),
 ])
-def test_route_train(T, d, E, k, dt):
-    """moe_route_train: logits = x Wg + b + noise; top-k, weights, aux loss and
-    the z-loss of those logits, against the oracle."""
+def test_route_train(T, d, E, k, dt, tau):
+    """moe_route_train: logits = x Wg + b + noise, softmax of logits / tau;
+    top-k, weights, aux loss and the z-loss, against the oracle."""
     inp = small_case("rt", T=T, d=d, E=E, k=k, F=128, act="gelu", dtype=dt, bias="zipf", seed=T + E)
     noise = torch.empty(T, E, dtype=torch.float32, device=DEV)
     abi.moe_router_noise(T, E, 1.0 / E, 7, noise)
@@ -369,11 +373,11 @@ def test_route_train(T, d, E, k, dt):
     probs = torch.empty(T, E, dtype=torch.float32, device=DEV)
     ws = new_ws(abi.moe_route_workspace_size(T, d, E))
     abi.moe_route_train(inp.x.to(DEV), inp.wg.to(DEV), inp.bias.to(DEV), noise, T, d, E, k, idx, w,
-                        aux, z, logits, probs, ws)
+                        aux, z, logits, probs, ws, temperature=tau)
     torch.cuda.synchronize()
     assert abi.moe_get_device_error(ws) == 0
     n64 = np32(noise).astype(np.float64)
-    r = O.route(np32(inp.x), np32(inp.wg), inp.bias.numpy(), k, noise=n64)
+    r = O.route(np32(inp.x), np32(inp.wg), inp.bias.numpy(), k, noise=n64, temperature=tau)
     g_logits = np32(logits)
     assert np.max(np.abs(g_logits - r["logits"])) <= 1e-5 * max(1.0, np.max(np.abs(r["logits"])))
     assert np.array_equal(npi(idx), O.topk_select(g_logits, k))
@@ -383,3 +387,24 @@ def test_route_train(T, d, E, k, dt):
     aux_ref = O.aux_loss(r["probs64"], g_idx, E)
     assert abs(float(aux.item()) - aux_ref) <= TOL_AUX_REL * aux_ref
     assert abs(float(z.item()) - r["z"]) <= TOL_AUX_REL * r["z"]
+
+
+@pytest.mark.parametrize("T,d,E,k,dt", [(1000, 1024, 8, 2, "bf16"), (513, 256, 64, 2, "bf16"),
+                                        (200, 64, 4, 1, "f32")])
+def test_route_train_at_unit_temperature_is_route(T, d, E, k, dt):
+    """moe_route_train with no noise, no z-loss and tau = 1 gives moe_route's
+    outputs bit for bit (the temperature multiplies by exactly 1)."""
+    inp = small_case("rt1", T=T, d=d, E=E, k=k, F=128, act="gelu", dtype=dt, bias="zipf", seed=T + 3)
+    x, wg, b = inp.x.to(DEV), inp.wg.to(DEV), inp.bias.to(DEV)
+    ref = route_on_gpu(x, wg, b, T, d, E, k)
+    idx = torch.empty(T, k, dtype=torch.int32, device=DEV)
+    w = torch.empty(T, k, dtype=torch.float32, device=DEV)
+    aux = torch.empty(1, dtype=torch.float32, device=DEV)
+    logits = torch.empty(T, E, dtype=torch.float32, device=DEV)
+    probs = torch.empty(T, E, dtype=torch.float32, device=DEV)
+    ws = new_ws(abi.moe_route_workspace_size(T, d, E))
+    abi.moe_route_train(x, wg, b, None, T, d, E, k, idx, w, aux, None, logits, probs, ws, temperature=1.0)
+    torch.cuda.synchronize()
+    assert abi.moe_get_device_error(ws) == 0
+    for g, r in zip((idx, w, aux, logits, probs), ref):
+        assert torch.equal(g, r)
