@@ -187,6 +187,57 @@ def route(x, wg, bias, k, noise=None, temperature=1.0):
     }
 
 
+def route_backward(x, wg, bias, k, d_w=None, d_aux=0.0, d_z=0.0, noise=None, temperature=1.0):
+    """Gradients of the router's losses, through the gate.
+
+    "ops-transformer MoE operators" blog, 实现 (the gating operator carries
+    the router's forward and its backward) and 坑3 (gradients reach the
+    experts through the softmax). The pages print no backward; this is the
+    chain rule of the forward in route(), for the scalar
+
+        L = sum_{t,j} d_w[t, j] * w[t, j] + d_aux * aux + d_z * z
+
+    (d_w: the upstream gradient of the renormalised top-k weights; aux, z:
+    the load-balance loss and the z-loss). The top-k pick and the counts f_i
+    are piecewise constant and pass no gradient; the fixed bias and the
+    noise are inputs. Returns float64 d_logits [T, E] (the gradient with
+    respect to the logits before the temperature), dx [T, d] and dwg [d, E].
+
+      w_j = p_{i_j} / s, s = sum_j p_{i_j}:
+          dL/dp_{i_j} = (d_w[t, j] - sum_m d_w[t, m] w_m) / s
+      aux = E sum_i f_i P_i, P_i = mean_t p[t, i]:  dL/dp[t, i] += d_aux E f_i / T
+      p = softmax(l / tau):  dL/dl = p (dL/dp - sum_e p_e dL/dp_e) / tau
+      z = mean_t lse_t^2, lse_t = logsumexp(l_t / tau):
+          dL/dl[t, e] += d_z (2 / T) lse_t p[t, e] / tau
+      l = x Wg + b (+ noise):  dx = dL/dl Wg^T, dWg = x^T dL/dl
+    """
+    r = route(x, wg, bias, k, noise=noise, temperature=temperature)
+    p = r["probs64"]
+    idx = r["topk_idx"]
+    w = r["topk_w64"]
+    T, E = p.shape
+    dp = np.zeros((T, E))
+    if d_w is not None:
+        g = np.asarray(d_w, dtype=np.float64)
+        s = np.take_along_axis(p, idx, axis=1).sum(axis=1)
+        gw = (g * w).sum(axis=1)
+        for j in range(k):
+            dp[np.arange(T), idx[:, j]] += (g[:, j] - gw) / s
+    if d_aux != 0.0:
+        f = np.bincount(idx.reshape(-1), minlength=E).astype(np.float64) / (T * k)
+        dp += d_aux * E * f[None, :] / T
+    tau = float(temperature)
+    dl = p * (dp - (p * dp).sum(axis=1, keepdims=True)) / tau
+    if d_z != 0.0:
+        lt = tempered_logits(gate_logits(x, wg, bias) + (0.0 if noise is None else np.asarray(noise, dtype=np.float64)), tau)
+        m = lt.max(axis=1, keepdims=True)
+        lse = m[:, 0] + np.log(np.exp(lt - m).sum(axis=1))
+        dl += d_z * (2.0 / T) * lse[:, None] * p / tau
+    x64 = np.asarray(x, dtype=np.float64)
+    wg64 = np.asarray(wg, dtype=np.float64)
+    return {"d_logits": dl, "dx": dl @ wg64.T, "dwg": x64.T @ dl, "route": r}
+
+
 # --------------------------------------------------------------------------
 # router variants (training): jitter, logit noise, z-loss
 # --------------------------------------------------------------------------

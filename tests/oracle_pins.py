@@ -521,6 +521,63 @@ def pin_temperature(o):
     assert abs(o.z_loss(o.tempered_logits(np.full((3, E), c), tau)) - (c / tau + math.log(E)) ** 2) < 1e-12
 
 
+def _router_loss(o, x, wg, bias, k, g, d_aux, d_z, noise, tau):
+    r = o.route(x, wg, bias, k, noise=noise, temperature=tau)
+    return float((g * r["topk_w64"]).sum() + d_aux * r["aux"] + d_z * r["z"])
+
+
+def pin_route_backward_finite_differences(o):
+    """The router backward against central differences of the forward's own
+    loss sum(d_w * w) + d_aux * aux + d_z * z (float64, step 1e-6; inputs
+    drawn without near-ties, so the pick does not move): d_logits through the
+    additive noise input, dx and dWg through x and Wg, at tau = 1 and 0.7,
+    with a bias and noise."""
+    rng = _rng(33)
+    T, d, E, k = 6, 5, 6, 2
+    h = 1e-6
+    for tau in (1.0, 0.7):
+        x, wg = rng.standard_normal((T, d)), rng.standard_normal((d, E))
+        bias, noise = rng.standard_normal(E), 0.3 * rng.standard_normal((T, E))
+        g = rng.standard_normal((T, k))
+        d_aux, d_z = 0.8, 0.35
+        b = o.route_backward(x, wg, bias, k, d_w=g, d_aux=d_aux, d_z=d_z, noise=noise, temperature=tau)
+        loss = lambda x_, wg_, n_: _router_loss(o, x_, wg_, bias, k, g, d_aux, d_z, n_, tau)
+        fd = np.zeros((T, E))
+        for t in range(T):
+            for e in range(E):
+                up, dn = noise.copy(), noise.copy()
+                up[t, e] += h
+                dn[t, e] -= h
+                fd[t, e] = (loss(x, wg, up) - loss(x, wg, dn)) / (2 * h)
+        assert np.max(np.abs(fd - b["d_logits"])) < 1e-7
+        for (t, i) in ((0, 0), (2, 3), (5, 4)):
+            up, dn = x.copy(), x.copy()
+            up[t, i] += h
+            dn[t, i] -= h
+            assert abs((loss(up, wg, noise) - loss(dn, wg, noise)) / (2 * h) - b["dx"][t, i]) < 1e-7
+        for (i, e) in ((0, 0), (1, 5), (4, 2)):
+            up, dn = wg.copy(), wg.copy()
+            up[i, e] += h
+            dn[i, e] -= h
+            assert abs((loss(x, up, noise) - loss(x, dn, noise)) / (2 * h) - b["dwg"][i, e]) < 1e-7
+
+
+def pin_route_backward_identities(o):
+    """Renormalised weights sum to 1, so a constant d_w passes no gradient;
+    without the z-loss every row of d_logits sums to 0 (softmax); with k = 1
+    the single weight is 1 whatever the logits."""
+    rng = _rng(34)
+    T, d, E = 9, 4, 5
+    x, wg = rng.standard_normal((T, d)), rng.standard_normal((d, E))
+    b = o.route_backward(x, wg, None, 2, d_w=np.full((T, 2), 1.7))
+    assert np.max(np.abs(b["d_logits"])) < 1e-13
+    b = o.route_backward(x, wg, None, 2, d_w=rng.standard_normal((T, 2)), d_aux=0.5, temperature=1.9)
+    assert np.max(np.abs(b["d_logits"].sum(axis=1))) < 1e-13
+    b = o.route_backward(x, wg, None, 1, d_w=rng.standard_normal((T, 1)))
+    assert np.max(np.abs(b["d_logits"])) < 1e-13
+
+
 ALL_PINS.extend([pin_philox_kat, pin_jitter, pin_logit_noise, pin_z_loss, pin_route_noise,
-                 pin_temperature])
+                 pin_temperature, pin_route_backward_finite_differences,
+                 pin_route_backward_identities])
 

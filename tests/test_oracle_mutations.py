@@ -110,8 +110,19 @@ def _jitter_half_width(T, d, eps, seed):
     return _REAL["jitter_multipliers"](T, d, eps / 2, seed)
 
 
+def _backward_ignores_temperature(x, wg, bias, k, d_w=None, d_aux=0.0, d_z=0.0, noise=None,
+                                  temperature=1.0):
+    r = _REAL["route_backward"](x, wg, bias, k, d_w, d_aux, d_z, noise, temperature)
+    return dict(r, d_logits=r["d_logits"] * temperature, dx=r["dx"] * temperature,
+                dwg=r["dwg"] * temperature)
+
+
+def _backward_drops_z(x, wg, bias, k, d_w=None, d_aux=0.0, d_z=0.0, noise=None, temperature=1.0):
+    return _REAL["route_backward"](x, wg, bias, k, d_w, d_aux, 0.0, noise, temperature)
+
+
 _REAL = {n: getattr(O, n) for n in ("combine", "expert_ffn", "permute", "permute_binned",
-                                    "jitter_multipliers")}
+                                    "jitter_multipliers", "route_backward")}
 
 MUTATIONS = {
     "topk_ties_to_higher_index": ("topk_select", _ties_to_higher),
@@ -131,6 +142,8 @@ MUTATIONS = {
     "z_loss_without_square": ("z_loss", _z_loss_no_square),
     "jitter_half_width": ("jitter_multipliers", _jitter_half_width),
     "temperature_ignored": ("tempered_logits", _temperature_ignored),
+    "backward_ignores_temperature": ("route_backward", _backward_ignores_temperature),
+    "backward_drops_z_loss": ("route_backward", _backward_drops_z),
 }
 
 
