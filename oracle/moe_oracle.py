@@ -212,10 +212,24 @@ def route_backward(x, wg, bias, k, d_w=None, d_aux=0.0, d_z=0.0, noise=None, tem
       l = x Wg + b (+ noise):  dx = dL/dl Wg^T, dWg = x^T dL/dl
     """
     r = route(x, wg, bias, k, noise=noise, temperature=temperature)
-    p = r["probs64"]
-    idx = r["topk_idx"]
-    w = r["topk_w64"]
+    l64 = gate_logits(x, wg, bias)
+    if noise is not None:
+        l64 = l64 + np.asarray(noise, dtype=np.float64)
+    out = route_backward_from(r["probs64"], r["topk_idx"], r["topk_w64"], l64, x, wg, d_w=d_w,
+                              d_aux=d_aux, d_z=d_z, temperature=temperature)
+    out["route"] = r
+    return out
+
+
+def route_backward_from(p, idx, w, logits, x, wg, d_w=None, d_aux=0.0, d_z=0.0, temperature=1.0):
+    """route_backward's chain rule from a given forward: probabilities p
+    [T, E], picks idx [T, k], renormalised weights w [T, k] and the logits
+    before the temperature (used by the z-loss term only)."""
+    p = np.asarray(p, dtype=np.float64)
+    idx = np.asarray(idx)
+    w = np.asarray(w, dtype=np.float64)
     T, E = p.shape
+    k = idx.shape[1]
     dp = np.zeros((T, E))
     if d_w is not None:
         g = np.asarray(d_w, dtype=np.float64)
@@ -229,13 +243,13 @@ def route_backward(x, wg, bias, k, d_w=None, d_aux=0.0, d_z=0.0, noise=None, tem
     tau = float(temperature)
     dl = p * (dp - (p * dp).sum(axis=1, keepdims=True)) / tau
     if d_z != 0.0:
-        lt = tempered_logits(gate_logits(x, wg, bias) + (0.0 if noise is None else np.asarray(noise, dtype=np.float64)), tau)
+        lt = tempered_logits(logits, tau)
         m = lt.max(axis=1, keepdims=True)
         lse = m[:, 0] + np.log(np.exp(lt - m).sum(axis=1))
         dl += d_z * (2.0 / T) * lse[:, None] * p / tau
     x64 = np.asarray(x, dtype=np.float64)
     wg64 = np.asarray(wg, dtype=np.float64)
-    return {"d_logits": dl, "dx": dl @ wg64.T, "dwg": x64.T @ dl, "route": r}
+    return {"d_logits": dl, "dx": dl @ wg64.T, "dwg": x64.T @ dl}
 
 
 # --------------------------------------------------------------------------
