@@ -235,6 +235,42 @@ MOE_API moe_status_t moe_route_train(const void* x, const void* w_router, const 
                              float* aux_loss, float* z_loss, float* logits, float* probs, void* ws,
                              size_t ws_bytes, moe_stream_t stream);
 
+/* Router backward: the gradients of
+ *     L = sum_{t,j} d_topk_w[t,j] * topk_w[t,j] + d_aux * aux + d_z * z_loss
+ * through the tempered softmax and the gate, with the pick and the aux
+ * loss's counts held fixed ("ops-transformer MoE operators", 实现: the gating
+ * operator has a forward and a backward; 坑3: gradients reach the experts
+ * through the softmax; the pages print no formula, this is the chain rule of
+ * moe_route_train's forward):
+ *     dL/dp_{i_j} = (d_topk_w[t,j] - sum_m d_topk_w[t,m] topk_w[t,m]) / sum_j p_{i_j}
+ *     dL/dp[t,e] += d_aux * E * f_e / T     (f_e = picks of e / (T*k))
+ *     d_logits    = p * (dL/dp - sum_e p_e dL/dp_e) / tau
+ *                   + d_z * (2/T) * lse(l_t / tau) * p / tau
+ *     dx = d_logits Wg^T,  d_wg = x^T d_logits
+ * The fixed bias and the logit noise take no gradient (d_logits is also
+ * theirs, if a caller wants them).
+ *   x, w_router   the forward's inputs, [T, d] and [d, E] (dtype)
+ *   probs         [T, E] fp32, the forward's probabilities (at tau)
+ *   logits        [T, E] fp32, the forward's logits before tau; read only
+ *                 when d_z != 0 (NULL otherwise)
+ *   topk_idx, topk_w  the forward's picks and renormalised weights [T, k]
+ *   d_topk_w      [T, k] fp32 upstream gradient of topk_w, or NULL (zero)
+ *   d_aux, d_z    upstream gradients of the two losses (host scalars)
+ *   temperature   tau > 0, as in the forward
+ *   d_logits      out [T, E] fp32, or NULL
+ *   dx            out [T, d] (dtype, rounded once), or NULL
+ *   d_wg          out [d, E] fp32, or NULL
+ *   ws            >= moe_route_backward_workspace_size(T, d, E) bytes
+ * fp32 arithmetic on CUDA cores; d_wg adds per-token-split partials in a
+ * fixed order (deterministic). */
+MOE_API size_t moe_route_backward_workspace_size(int T, int d, int E);
+MOE_API moe_status_t moe_route_backward(const void* x, const void* w_router, moe_dtype_t dtype,
+                                int T, int d, int E, int k, const float* probs,
+                                const float* logits, const int32_t* topk_idx,
+                                const float* topk_w, const float* d_topk_w, float d_aux,
+                                float d_z, float temperature, float* d_logits, void* dx,
+                                float* d_wg, void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Router jitter ("MegaBlocks", section 5: the router input is multiplied by
  * uniform noise in [1 - eps, 1 + eps] during training): x_out = x * m with
  * m uniform in [1 - eps, 1 + eps) per element, from the counter-based

@@ -80,6 +80,9 @@ _SIGS = {
     "moe_route_train": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, ctypes.c_float, c_int, c_int,
                                 c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
                                 c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "moe_route_backward_workspace_size": (c_size_t, [c_int, c_int, c_int]),
+    "moe_route_backward": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int] + [c_void_p] * 5
+                           + [ctypes.c_float] * 3 + [c_void_p] * 4 + [c_size_t, c_void_p]),
     "moe_router_jitter": (c_int, [c_void_p, c_int, c_int, c_int, ctypes.c_float, ctypes.c_uint64,
                                   c_void_p, c_void_p]),
     "moe_router_noise": (c_int, [c_int, c_int, ctypes.c_float, ctypes.c_uint64, c_void_p, c_void_p]),
@@ -200,6 +203,19 @@ def moe_route_train(x, w_router, bias, logit_noise, T, d, E, k, topk_idx, topk_w
         dtype_code(x.dtype), T, d, E, k,
         _ptr(topk_idx), _ptr(topk_w), _ptr(aux_loss), _ptr(z_loss), _ptr(logits), _ptr(probs),
         _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_route_backward_workspace_size(T, d, E) -> int:
+    return _lib.moe_route_backward_workspace_size(T, d, E)
+
+
+def moe_route_backward(x, w_router, T, d, E, k, probs, logits, topk_idx, topk_w, d_topk_w, d_aux, d_z,
+                       temperature, d_logits, dx, d_wg, ws, stream=None, dtype=None):
+    dt = dtype_code(x.dtype) if x is not None else dtype
+    _check("moe_route_backward", _lib.moe_route_backward(
+        _ptr(x), _ptr(w_router), dt, T, d, E, k, _ptr(probs), _ptr(logits), _ptr(topk_idx),
+        _ptr(topk_w), _ptr(d_topk_w), float(d_aux), float(d_z), float(temperature), _ptr(d_logits),
+        _ptr(dx), _ptr(d_wg), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def moe_router_jitter(x, T, d, eps, seed, x_out, stream=None):

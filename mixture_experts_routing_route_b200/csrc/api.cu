@@ -329,6 +329,44 @@ moe_status_t moe_route_train(const void* x, const void* w_router, const float* b
                     aux_loss, z_loss, logits, probs, ws, ws_bytes, stream);
 }
 
+size_t moe_route_backward_workspace_size(int T, int d, int E) {
+  if (T < 0 || d < 1 || E < 1) return 0;
+  return align_up(sizeof(Control)) + route_backward_scratch_bytes(T, d, E);
+}
+
+moe_status_t moe_route_backward(const void* x, const void* w_router, moe_dtype_t dtype, int T,
+                                int d, int E, int k, const float* probs, const float* logits,
+                                const int32_t* topk_idx, const float* topk_w,
+                                const float* d_topk_w, float d_aux, float d_z, float temperature,
+                                float* d_logits, void* dx, float* d_wg, void* ws, size_t ws_bytes,
+                                moe_stream_t stream) {
+  MOE_CHECK(check_dims(dtype, T, d, E, k));
+  if (!(temperature > 0.0f) || !std::isfinite(temperature) || !std::isfinite(d_aux) ||
+      !std::isfinite(d_z))
+    return MOE_ERR_INVALID;
+  MOE_NEED(ws);
+  MOE_OPT(logits);
+  MOE_OPT(d_topk_w);
+  MOE_OPT(d_logits);
+  MOE_OPT(dx);
+  MOE_OPT(d_wg);
+  if (T > 0) {
+    MOE_NEED(probs);
+    MOE_NEED(topk_idx);
+    if (d_topk_w != nullptr) MOE_NEED(topk_w);
+    if (d_z != 0.0f) MOE_NEED(logits);
+    if (dx != nullptr || d_wg != nullptr) MOE_NEED(w_router);
+    if (d_wg != nullptr) MOE_NEED(x);
+  }
+  if (ws_bytes < moe_route_backward_workspace_size(T, d, E)) return MOE_ERR_WORKSPACE;
+  Carver c(ws);
+  Control* ctl = static_cast<Control*>(c.take(sizeof(Control)));
+  void* scratch = c.take(route_backward_scratch_bytes(T, d, E));
+  return from_cuda(launch_route_backward(x, w_router, dtype, T, d, E, k, probs, logits, topk_idx,
+                                         topk_w, d_topk_w, d_aux, d_z, temperature, d_logits, dx,
+                                         d_wg, scratch, ctl, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_router_jitter(const void* x, moe_dtype_t dtype, int T, int d, float eps,
                                uint64_t seed, void* x_out, moe_stream_t stream) {
   if (dtype != MOE_BF16 && dtype != MOE_F32) return MOE_ERR_INVALID;

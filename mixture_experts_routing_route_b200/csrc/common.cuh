@@ -110,6 +110,17 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, const
                          float* logits_scratch, void* partials, Control* ctl, cudaStream_t s,
                          float temperature = 1.0f);
 size_t route_logits_scratch_bytes(int T, int d, int E);
+// Router backward (see router_backward.cu): d_logits [T, E] fp32 (or NULL:
+// kept in scratch), dx [T, d] (dtype) or NULL, d_wg [d, E] fp32 or NULL.
+// logits (before the temperature) are read only when d_z != 0; counts of the
+// picks are taken on the device when d_aux != 0.
+size_t route_backward_scratch_bytes(int T, int d, int E);
+cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt, int T, int d,
+                                  int E, int k, const float* probs, const float* logits,
+                                  const int32_t* idx, const float* w, const float* d_w,
+                                  float d_aux, float d_z, float temperature, float* d_logits,
+                                  void* dx, float* d_wg, void* scratch, Control* ctl,
+                                  cudaStream_t s);
 
 // Permute. launch_permute picks the multi-CTA kernel when the slots fit its
 // per-CTA shared memory, else the single-CTA kernel; launch_permute_single

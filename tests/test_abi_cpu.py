@@ -113,6 +113,16 @@ def test_argument_checks_return_before_launch(abi):
     L7 = abi.MoeLayerC(4096, 8, 2, 128, abi.MOE_BF16, abi.MOE_ACT_SWIGLU, 0.0, 16, None, 16, 16, 16,
                        0, None, None, -1.0)
     assert abi._lib.moe_forward(ctypes.byref(L7), 16, 4, 16, None, 16, 1 << 40, None, None) == 2
+    # router backward: tau > 0, a workspace, probs when T > 0
+    assert abi._lib.moe_route_backward(16, 16, abi.MOE_BF16, 8, 128, 8, 2, 16, None, 16, 16, None, 0.0,
+                                       0.0, 0.0, None, None, None, 16, 1 << 30, None) == 2
+    assert abi._lib.moe_route_backward(16, 16, abi.MOE_BF16, 8, 128, 8, 2, None, None, 16, 16, None,
+                                       0.0, 0.0, 1.0, None, None, None, 16, 1 << 30, None) == 1
+    assert abi._lib.moe_route_backward(16, 16, abi.MOE_BF16, 8, 128, 8, 2, 16, None, 16, 16, None, 0.0,
+                                       1.0, 1.0, None, None, None, 16, 1 << 30, None) == 1  # d_z needs logits
+    assert abi._lib.moe_route_backward(16, 16, abi.MOE_BF16, 8, 128, 8, 2, 16, None, 16, 16, None, 0.0,
+                                       0.0, 1.0, None, None, None, 16, 16, None) == 4
+    assert abi.moe_route_backward_workspace_size(4096, 4096, 8) >= 4096 * 8 * 4
     assert abi.moe_kernel_launches() == n0
 
 

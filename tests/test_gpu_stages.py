@@ -408,3 +408,47 @@ def test_route_train_at_unit_temperature_is_route(T, d, E, k, dt):
     assert abi.moe_get_device_error(ws) == 0
     for g, r in zip((idx, w, aux, logits, probs), ref):
         assert torch.equal(g, r)
+
+
+@pytest.mark.parametrize("T,d,E,k,dt,tau,d_aux,d_z", [
+    (1000, 1024, 8, 2, "bf16", 1.0, 0.01, 0.001),   # Mixtral's router shape at a reduced T
+    (777, 512, 8, 2, "bf16", 0.7, 0.5, 0.0),        # temperature, no z-loss term
+    (513, 256, 64, 2, "bf16", 1.3, 0.1, 0.02),      # two 32-expert chunks
+    (129, 256, 256, 8, "bf16", 1.0, 0.05, 0.01),    # E = 256, k = 8
+    (300, 512, 24, 3, "bf16", 2.0, 0.0, 0.1),       # E not a multiple of 32, no aux term
+    (200, 64, 40, 4, "f32", 1.0, 0.3, 0.05),        # fp32 (dx in fp32)
+])
+def test_route_backward(T, d, E, k, dt, tau, d_aux, d_z):
+    """moe_route_backward from the GPU's own forward (moe_route_train at tau)
+    against the oracle's chain rule of that forward: d_logits, dx and d_wg;
+    two runs give the same bits."""
+    inp = small_case("rb", T=T, d=d, E=E, k=k, F=128, act="gelu", dtype=dt, bias="zipf", seed=T + E)
+    x, wg, b = inp.x.to(DEV), inp.wg.to(DEV), inp.bias.to(DEV)
+    idx = torch.empty(T, k, dtype=torch.int32, device=DEV)
+    w = torch.empty(T, k, dtype=torch.float32, device=DEV)
+    aux = torch.empty(1, dtype=torch.float32, device=DEV)
+    logits = torch.empty(T, E, dtype=torch.float32, device=DEV)
+    probs = torch.empty(T, E, dtype=torch.float32, device=DEV)
+    ws = new_ws(abi.moe_route_workspace_size(T, d, E))
+    abi.moe_route_train(x, wg, b, None, T, d, E, k, idx, w, aux, None, logits, probs, ws, temperature=tau)
+    g = torch.from_numpy(np.random.default_rng(T).standard_normal((T, k)).astype(np.float32)).to(DEV)
+    bws = new_ws(abi.moe_route_backward_workspace_size(T, d, E))
+    outs = []
+    for _ in range(2):
+        d_logits = torch.empty(T, E, dtype=torch.float32, device=DEV)
+        dx = torch.empty(T, d, dtype=x.dtype, device=DEV)
+        d_wg = torch.empty(d, E, dtype=torch.float32, device=DEV)
+        abi.moe_route_backward(x, wg, T, d, E, k, probs, logits if d_z else None, idx, w, g, d_aux, d_z,
+                               tau, d_logits, dx, d_wg, bws)
+        torch.cuda.synchronize()
+        assert abi.moe_get_device_error(bws) == 0
+        outs.append((d_logits, dx, d_wg))
+    for a, c in zip(*outs):
+        assert torch.equal(a, c)
+    d_logits, dx, d_wg = outs[0]
+    ref = O.route_backward_from(np32(probs).astype(np.float64), npi(idx), np32(w).astype(np.float64),
+                                np32(logits).astype(np.float64), np32(inp.x), np32(inp.wg),
+                                d_w=np32(g).astype(np.float64), d_aux=d_aux, d_z=d_z, temperature=tau)
+    assert max_err_ratio(np32(d_logits), ref["d_logits"]) <= 1e-5
+    assert max_err_ratio(np32(d_wg), ref["dwg"]) <= 1e-4
+    assert max_err_ratio(np32(dx), ref["dx"]) <= (TOL_BF16_OUT if dt == "bf16" else 1e-5)
