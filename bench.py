@@ -68,6 +68,9 @@ def parse():
                    help="bf16, k = 1: the combine in the down projection's epilogue (no combine "
                         "kernel, no y_perm)")
     p.add_argument("--k", type=int, default=None, help="override top-k (e.g. 1 for --combine-in-gemm)")
+    p.add_argument("--router-backward", action="store_true",
+                   help="time the router backward (moe_route_backward: d_logits, dx, dWg) on the "
+                        "workload's router instead of the layer forward; one GPU")
     p.add_argument("--T", type=int, default=None, help="override T (reduced case for profiling)")
     p.add_argument("--E", type=int, default=None, help="override E (reduced case for profiling)")
     p.add_argument("--F", type=int, default=None, help="override F (reduced case for profiling)")
@@ -414,10 +417,84 @@ def cpu_baseline(sh, inp):
 
 
 # ------------------------------------------------------------------ main
+def run_router_backward(args):
+    """The router backward on the workload's router (x [T, d], Wg [d, E]):
+    inputs from one forward (moe_route_train), upstream gradients drawn from
+    a seed (d_w ~ N(0, 1), d_aux = 0.01, d_z = 0.001), L2 evicted between
+    steps. Algorithmic bytes per step: probs, logits, picks, weights and d_w
+    read, d_logits written; x read once for dWg, dx written once, Wg read and
+    dWg written (T*E*4*3 + T*k*12 + 2*T*d*b + d*E*(b+4))."""
+    from mixture_experts_routing_route_b200 import _abi as abi
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    sh = shape_of(args)
+    inp = make_inputs(sh)
+    T, d, E, k = sh.T, sh.d, sh.E, sh.k
+    x, wg = inp.x.to(dev), inp.wg.to(dev)
+    bias = None if inp.bias is None else inp.bias.to(dev)
+    idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+    w = torch.empty(T, k, dtype=torch.float32, device=dev)
+    aux = torch.empty(1, dtype=torch.float32, device=dev)
+    logits = torch.empty(T, E, dtype=torch.float32, device=dev)
+    probs = torch.empty(T, E, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(abi.moe_route_workspace_size(T, d, E), 256), dtype=torch.uint8, device=dev)
+    abi.moe_workspace_init(ws)
+    abi.moe_route_train(x, wg, bias, None, T, d, E, k, idx, w, aux, None, logits, probs, ws)
+    g = torch.from_numpy(np.random.default_rng(7).standard_normal((T, k)).astype(np.float32)).to(dev)
+    d_logits = torch.empty(T, E, dtype=torch.float32, device=dev)
+    dx = torch.empty(T, d, dtype=x.dtype, device=dev)
+    d_wg = torch.empty(d, E, dtype=torch.float32, device=dev)
+    bws = torch.empty(max(abi.moe_route_backward_workspace_size(T, d, E), 256), dtype=torch.uint8,
+                      device=dev)
+    abi.moe_workspace_init(bws)
+    flush = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    sink = torch.zeros(1, dtype=torch.int64, device=dev)
+    step = lambda: abi.moe_route_backward(x, wg, T, d, E, k, probs, logits, idx, w, g, 0.01, 0.001, 1.0,
+                                          d_logits, dx, d_wg, bws)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if abi.moe_get_device_error(bws) != 0:
+        raise RuntimeError("device error word set during warm-up")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    n0 = abi.moe_kernel_launches()
+    # a spin on the GPU first, so that the host enqueues every step before the
+    # GPU reaches it: the events then bracket device time only
+    torch.cuda._sleep(int(2e5) * args.steps)
+    for a, b in evs:
+        torch.sum(flush, dim=0, dtype=torch.int64, out=sink[0])
+        a.record()
+        step()
+        b.record()
+    n1 = abi.moe_kernel_launches()
+    torch.cuda.synchronize()
+    times = sorted(a.elapsed_time(b) for a, b in evs)
+    ms = statistics.median(times)
+    eb = x.element_size()
+    byts = T * E * 4 * 3 + T * k * 12 + 2 * T * d * eb + d * E * (eb + 4)
+    peaks = load_peaks()
+    gbs = byts / (ms * 1e-3) / 1e9
+    line = {"metric": "router backward tokens/s (d_logits, dx, dWg)", "value": T / (ms * 1e-3),
+            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "dtype": sh.dtype,
+            "data": "synthetic (seeded)", "config": workload_config(sh),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                         "algorithmic_per_step": byts,
+                         "timing": "median of CUDA events around each call (all calls enqueued "
+                                   "behind a GPU spin), L2 evicted between"},
+            "gpu_launches": n1 - n0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.router_backward:
+        return run_router_backward(args)
     from mixture_experts_routing_route_b200 import MoeLayer
     from mixture_experts_routing_route_b200 import _abi as abi
 

@@ -261,8 +261,9 @@ MOE_API moe_status_t moe_route_train(const void* x, const void* w_router, const 
  *   dx            out [T, d] (dtype, rounded once), or NULL
  *   d_wg          out [d, E] fp32, or NULL
  *   ws            >= moe_route_backward_workspace_size(T, d, E) bytes
- * fp32 arithmetic on CUDA cores; d_wg adds per-token-split partials in a
- * fixed order (deterministic). */
+ * d must be a multiple of 4 (MOE_ERR_UNSUPPORTED otherwise). fp32
+ * arithmetic on CUDA cores; d_wg adds per-token-split partials in a fixed
+ * order (deterministic). */
 MOE_API size_t moe_route_backward_workspace_size(int T, int d, int E);
 MOE_API moe_status_t moe_route_backward(const void* x, const void* w_router, moe_dtype_t dtype,
                                 int T, int d, int E, int k, const float* probs,

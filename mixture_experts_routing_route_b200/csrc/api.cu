@@ -341,6 +341,7 @@ moe_status_t moe_route_backward(const void* x, const void* w_router, moe_dtype_t
                                 float* d_logits, void* dx, float* d_wg, void* ws, size_t ws_bytes,
                                 moe_stream_t stream) {
   MOE_CHECK(check_dims(dtype, T, d, E, k));
+  if (d % 4 != 0) return MOE_ERR_UNSUPPORTED;  // 4 columns per vector access
   if (!(temperature > 0.0f) || !std::isfinite(temperature) || !std::isfinite(d_aux) ||
       !std::isfinite(d_z))
     return MOE_ERR_INVALID;

@@ -35,14 +35,20 @@ bwd_hist(const int32_t* __restrict__ idx, long long S, int E, int32_t* __restric
   __shared__ int h[256];  // E <= 256
   for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
   __syncthreads();
-  for (long long s = threadIdx.x; s < S; s += blockDim.x) {
-    const int e = __ldg(idx + s);
-    if (e < 0 || e >= E) {
-      set_error(ctl, MOE_DEVERR_EXPERT_RANGE);
-      continue;
-    }
-    atomicAdd(&h[e], 1);
+  auto add = [&](int e) {
+    if (e < 0 || e >= E) set_error(ctl, MOE_DEVERR_EXPERT_RANGE);
+    else atomicAdd(&h[e], 1);
+  };
+  // four picks per 16-byte load (idx is 16-byte aligned), then the tail
+  const long long S4 = S / 4;
+  for (long long q = threadIdx.x; q < S4; q += blockDim.x) {
+    const int4 v = __ldg(reinterpret_cast<const int4*>(idx) + q);
+    add(v.x);
+    add(v.y);
+    add(v.z);
+    add(v.w);
   }
+  for (long long s = S4 * 4 + threadIdx.x; s < S; s += blockDim.x) add(__ldg(idx + s));
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) counts[e] = h[e];
 }
@@ -157,103 +163,185 @@ template <> struct Io<__nv_bfloat16> {
   static __device__ __forceinline__ void st(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 };
 
-constexpr int kCols = 256;   // columns of d per block (a thread each)
-constexpr int kTok = 32;     // tokens per tile
-constexpr int kEChunk = 32;  // experts staged at a time
+// Vector access to CPT consecutive elements of a row (16-byte aligned for
+// fp32 x 4, 8-byte for bf16 x 4; d is a multiple of 4, which the row stride
+// and the column offsets keep).
+template <typename T, int CPT>
+struct Vec;
+template <> struct Vec<float, 4> {
+  static __device__ __forceinline__ void ld(const float* p, float (&v)[4]) {
+    const float4 u = __ldg(reinterpret_cast<const float4*>(p));
+    v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+  }
+  static __device__ __forceinline__ void st(float* p, const float (&v)[4]) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+};
+template <> struct Vec<__nv_bfloat16, 4> {
+  static __device__ __forceinline__ void ld(const __nv_bfloat16* p, float (&v)[4]) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    v[0] = __uint_as_float(u.x << 16); v[1] = __uint_as_float(u.x & 0xffff0000u);
+    v[2] = __uint_as_float(u.y << 16); v[3] = __uint_as_float(u.y & 0xffff0000u);
+  }
+  static __device__ __forceinline__ void st(__nv_bfloat16* p, const float (&v)[4]) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
+    *reinterpret_cast<uint2*>(p) = make_uint2(*reinterpret_cast<const uint32_t*>(&a),
+                                              *reinterpret_cast<const uint32_t*>(&b));
+  }
+};
+template <> struct Vec<float, 2> {
+  static __device__ __forceinline__ void ld(const float* p, float (&v)[2]) {
+    const float2 u = __ldg(reinterpret_cast<const float2*>(p));
+    v[0] = u.x; v[1] = u.y;
+  }
+};
+template <> struct Vec<__nv_bfloat16, 2> {
+  static __device__ __forceinline__ void ld(const __nv_bfloat16* p, float (&v)[2]) {
+    const uint32_t u = __ldg(reinterpret_cast<const unsigned int*>(p));
+    v[0] = __uint_as_float(u << 16); v[1] = __uint_as_float(u & 0xffff0000u);
+  }
+};
+template <typename T> struct Vec<T, 1> {
+  static __device__ __forceinline__ void ld(const T* p, float (&v)[1]) { v[0] = Io<T>::ld(p); }
+};
 
-// dx[t, c] = sum_e dl[t, e] Wg[c, e], e in increasing order. Block: 256
-// columns x 32 tokens; Wg's columns and dl's rows are staged per 32-expert
-// chunk, transposed so that a thread reads its column (conflict-free) and a
-// token quadruple (one 16-byte broadcast).
+// dx[t, c] = sum_e dl[t, e] Wg[c, e], e in increasing order. Block: 128
+// threads x 4 columns = 512 columns, 8 tiles of 16 tokens. Wg's columns are
+// staged transposed per 16-expert chunk (once per block when E <= 16), so a
+// thread reads its 4 columns in one conflict-free 16-byte load; each tile's
+// dl rows are staged transposed (four 16-byte broadcasts per expert); Wg is
+// read along its rows. With E > 16 every tile re-stages Wg, so a block then
+// takes one tile (tiles = 1) and the grid is 8 times taller.
+constexpr int kDxThreads = 128;
+constexpr int kDxCols = 4 * kDxThreads;
+constexpr int kDxTok = 16;
+constexpr int kDxE = 16;
+constexpr int kDxTiles = 8;
+
 template <typename T>
-__global__ void __launch_bounds__(kCols, 2)
-bwd_dx(const float* __restrict__ dl, const T* __restrict__ wg, int Tn, int d, int E,
+__global__ void __launch_bounds__(kDxThreads)
+bwd_dx(const float* __restrict__ dl, const T* __restrict__ wg, int Tn, int d, int E, int tiles,
        T* __restrict__ dx) {
   pdl_begin();
-  __shared__ float wg_s[kEChunk][kCols];
-  __shared__ __align__(16) float dl_s[kEChunk][kTok];
-  const int c = blockIdx.x * kCols + threadIdx.x;
-  const int t0 = blockIdx.y * kTok;
-  float acc[kTok];
-#pragma unroll
-  for (int i = 0; i < kTok; ++i) acc[i] = 0.f;
-  for (int e0 = 0; e0 < E; e0 += kEChunk) {
-    const int ne = min(kEChunk, E - e0);
-    __syncthreads();
-    for (int i = threadIdx.x; i < kEChunk * kCols; i += kCols) {
-      const int e = i / kCols, cc = i - e * kCols;
-      const int col = blockIdx.x * kCols + cc;
-      wg_s[e][cc] = (e < ne && col < d) ? Io<T>::ld(wg + static_cast<size_t>(col) * E + e0 + e) : 0.f;
+  __shared__ __align__(16) float wg_s[kDxE][kDxCols + 4];  // +4: the transposing stores spread over banks
+  __shared__ __align__(16) float dl_s[kDxE][kDxTok];
+  const int c = blockIdx.x * kDxCols + 4 * threadIdx.x;
+  const bool one_chunk = E <= kDxE;
+  auto stage_wg = [&](int e0, int ne) {
+    for (int i = threadIdx.x; i < ne * kDxCols; i += kDxThreads) {
+      const int cc = i / ne, e = i - cc * ne;
+      const int col = blockIdx.x * kDxCols + cc;
+      wg_s[e][cc] = col < d ? Io<T>::ld(wg + static_cast<size_t>(col) * E + e0 + e) : 0.f;
     }
-    for (int i = threadIdx.x; i < kEChunk * kTok; i += kCols) {
-      const int tt = i / kEChunk, e = i - tt * kEChunk;
-      const int t = t0 + tt;
-      dl_s[e][tt] = (e < ne && t < Tn) ? __ldg(dl + static_cast<size_t>(t) * E + e0 + e) : 0.f;
-    }
-    __syncthreads();
-    for (int e = 0; e < ne; ++e) {
-      const float wv = wg_s[e][threadIdx.x];
+  };
+  if (one_chunk) stage_wg(0, E);  // read after the first tile's barrier
+  for (int tile = 0; tile < tiles; ++tile) {
+    const int t0 = (blockIdx.y * tiles + tile) * kDxTok;
+    if (t0 >= Tn) break;  // the same for every thread of the block
+    float acc[kDxTok][4];
 #pragma unroll
-      for (int i = 0; i < kTok; i += 4) {
-        const float4 g = *reinterpret_cast<const float4*>(&dl_s[e][i]);
-        acc[i] = fmaf(g.x, wv, acc[i]);
-        acc[i + 1] = fmaf(g.y, wv, acc[i + 1]);
-        acc[i + 2] = fmaf(g.z, wv, acc[i + 2]);
-        acc[i + 3] = fmaf(g.w, wv, acc[i + 3]);
+    for (int i = 0; i < kDxTok; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int e0 = 0; e0 < E; e0 += kDxE) {
+      const int ne = min(kDxE, E - e0);
+      __syncthreads();  // the previous readers of the staged rows are done
+      if (!one_chunk) stage_wg(e0, ne);
+      for (int i = threadIdx.x; i < kDxE * kDxTok; i += kDxThreads) {
+        const int tt = i / kDxE, e = i - tt * kDxE;
+        const int t = t0 + tt;
+        dl_s[e][tt] = (e < ne && t < Tn) ? __ldg(dl + static_cast<size_t>(t) * E + e0 + e) : 0.f;
+      }
+      __syncthreads();
+      for (int e = 0; e < ne; ++e) {
+        const float4 wv = *reinterpret_cast<const float4*>(&wg_s[e][4 * threadIdx.x]);
+#pragma unroll
+        for (int i = 0; i < kDxTok; i += 4) {
+          const float4 g = *reinterpret_cast<const float4*>(&dl_s[e][i]);
+          const float gi[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            acc[i + u][0] = fmaf(gi[u], wv.x, acc[i + u][0]);
+            acc[i + u][1] = fmaf(gi[u], wv.y, acc[i + u][1]);
+            acc[i + u][2] = fmaf(gi[u], wv.z, acc[i + u][2]);
+            acc[i + u][3] = fmaf(gi[u], wv.w, acc[i + u][3]);
+          }
+        }
       }
     }
-  }
-  if (c < d) {
+    if (c < d) {
 #pragma unroll
-    for (int i = 0; i < kTok; ++i)
-      if (t0 + i < Tn) Io<T>::st(dx + static_cast<size_t>(t0 + i) * d + c, acc[i]);
+      for (int i = 0; i < kDxTok; ++i)
+        if (t0 + i < Tn) Vec<T, 4>::st(dx + static_cast<size_t>(t0 + i) * d + c, acc[i]);
+    }
   }
 }
 
 // dWg partial of token split s: part[s][c][e] = sum over the split's tokens
-// (increasing) of x[t, c] dl[t, e], for one 32-expert chunk (blockIdx.z).
-template <typename T>
-__global__ void __launch_bounds__(kCols)
+// (increasing) of x[t, c] dl[t, e], for one EC-expert chunk (blockIdx.z;
+// EC = 8, 16 or 32, the smallest that covers E up to 32). A thread owns
+// CPT = 32 / EC consecutive columns (one vector load of x per token) and
+// EC x CPT = 32 accumulators.
+constexpr int kDwgThreads = 128;
+constexpr int kDwgTok = 16;
+
+template <typename T, int EC>
+__global__ void __launch_bounds__(kDwgThreads)
 bwd_dwg_part(const T* __restrict__ x, const float* __restrict__ dl, int Tn, int d, int E,
              int tok_per_split, float* __restrict__ part) {
   pdl_begin();
-  __shared__ __align__(16) float dl_s[kTok][kEChunk];
-  const int c = blockIdx.x * kCols + threadIdx.x;
-  const int s = blockIdx.y, e0 = blockIdx.z * kEChunk;
-  const int ne = min(kEChunk, E - e0);
+  constexpr int CPT = 32 / EC;
+  __shared__ __align__(16) float dl_s[kDwgTok][EC];
+  const int c = (blockIdx.x * kDwgThreads + threadIdx.x) * CPT;
+  const int s = blockIdx.y, e0 = blockIdx.z * EC;
+  const int ne = min(EC, E - e0);
   const int tb = s * tok_per_split, te = min(Tn, tb + tok_per_split);
-  float acc[kEChunk];
+  float acc[EC][CPT];
 #pragma unroll
-  for (int i = 0; i < kEChunk; ++i) acc[i] = 0.f;
-  for (int t0 = tb; t0 < te; t0 += kTok) {
+  for (int e = 0; e < EC; ++e)
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) acc[e][j] = 0.f;
+  for (int t0 = tb; t0 < te; t0 += kDwgTok) {
     __syncthreads();
-    for (int i = threadIdx.x; i < kTok * kEChunk; i += kCols) {
-      const int tt = i / kEChunk, e = i - tt * kEChunk;
+    for (int i = threadIdx.x; i < kDwgTok * EC; i += kDwgThreads) {
+      const int tt = i / EC, e = i - tt * EC;
       const int t = t0 + tt;
       dl_s[tt][e] = (e < ne && t < te) ? __ldg(dl + static_cast<size_t>(t) * E + e0 + e) : 0.f;
     }
     __syncthreads();
-    float xv[kTok];
+    float xv[kDwgTok][CPT];
 #pragma unroll
-    for (int i = 0; i < kTok; ++i)
-      xv[i] = (c < d && t0 + i < te) ? Io<T>::ld(x + static_cast<size_t>(t0 + i) * d + c) : 0.f;
+    for (int i = 0; i < kDwgTok; ++i) {
+      if (c < d && t0 + i < te) {
+        Vec<T, CPT>::ld(x + static_cast<size_t>(t0 + i) * d + c, xv[i]);
+      } else {
 #pragma unroll
-    for (int i = 0; i < kTok; ++i) {
+        for (int j = 0; j < CPT; ++j) xv[i][j] = 0.f;
+      }
+    }
 #pragma unroll
-      for (int e = 0; e < kEChunk; e += 4) {
+    for (int i = 0; i < kDwgTok; ++i) {
+#pragma unroll
+      for (int e = 0; e < EC; e += 4) {
         const float4 g = *reinterpret_cast<const float4*>(&dl_s[i][e]);
-        acc[e] = fmaf(xv[i], g.x, acc[e]);
-        acc[e + 1] = fmaf(xv[i], g.y, acc[e + 1]);
-        acc[e + 2] = fmaf(xv[i], g.z, acc[e + 2]);
-        acc[e + 3] = fmaf(xv[i], g.w, acc[e + 3]);
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+          acc[e][j] = fmaf(xv[i][j], g.x, acc[e][j]);
+          acc[e + 1][j] = fmaf(xv[i][j], g.y, acc[e + 1][j]);
+          acc[e + 2][j] = fmaf(xv[i][j], g.z, acc[e + 2][j]);
+          acc[e + 3][j] = fmaf(xv[i][j], g.w, acc[e + 3][j]);
+        }
       }
     }
   }
   if (c < d) {
-    float* dst = part + (static_cast<size_t>(s) * d + c) * E + e0;
 #pragma unroll
-    for (int e = 0; e < kEChunk; ++e)
-      if (e < ne) dst[e] = acc[e];
+    for (int j = 0; j < CPT; ++j) {
+      float* dst = part + (static_cast<size_t>(s) * d + c + j) * E + e0;
+#pragma unroll
+      for (int e = 0; e < EC; ++e)
+        if (e < ne) dst[e] = acc[e][j];
+    }
   }
 }
 
@@ -269,16 +357,21 @@ bwd_dwg_reduce(const float* __restrict__ part, int nsplit, long long n, float* _
   }
 }
 
-int dwg_splits(int T) {
-  const int s = (T + 127) / 128;  // about 128 tokens per split
-  return s < 1 ? 1 : (s > 32 ? 32 : s);
+// Token splits of the dWg partials: at least 64 tokens each, at most 64, and
+// at most 32 MB of partials (d * E * 4 bytes per split).
+int dwg_splits(int T, int d, int E) {
+  int s = (T + 63) / 64;
+  const long long cap = (8LL << 20) / (static_cast<long long>(d) * E);
+  if (s > 64) s = 64;
+  if (s > cap) s = static_cast<int>(cap);
+  return s < 1 ? 1 : s;
 }
 
 }  // namespace
 
 size_t route_backward_scratch_bytes(int T, int d, int E) {
   return align_up(static_cast<size_t>(E) * 4) + align_up(static_cast<size_t>(T) * E * 4) +
-         align_up(static_cast<size_t>(dwg_splits(T)) * d * E * 4);
+         align_up(static_cast<size_t>(dwg_splits(T, d, E)) * d * E * 4);
 }
 
 cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt, int T, int d,
@@ -311,26 +404,40 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
                      d_z, inv_tau, T, E, k, dl, ctl);
     if (err != cudaSuccess) return err;
     if (dx != nullptr) {
-      const dim3 g((d + kCols - 1) / kCols, (T + kTok - 1) / kTok);
+      const int tiles = E <= kDxE ? kDxTiles : 1;
+      const dim3 g((d + kDxCols - 1) / kDxCols, (T + kDxTok * tiles - 1) / (kDxTok * tiles));
       err = dt == MOE_BF16
-                ? launch_pdl(bwd_dx<__nv_bfloat16>, g, dim3(kCols), 0, s, false, dl,
-                             static_cast<const __nv_bfloat16*>(wg), T, d, E, static_cast<__nv_bfloat16*>(dx))
-                : launch_pdl(bwd_dx<float>, g, dim3(kCols), 0, s, false, dl,
-                             static_cast<const float*>(wg), T, d, E, static_cast<float*>(dx));
+                ? launch_pdl(bwd_dx<__nv_bfloat16>, g, dim3(kDxThreads), 0, s, false, dl,
+                             static_cast<const __nv_bfloat16*>(wg), T, d, E, tiles,
+                             static_cast<__nv_bfloat16*>(dx))
+                : launch_pdl(bwd_dx<float>, g, dim3(kDxThreads), 0, s, false, dl,
+                             static_cast<const float*>(wg), T, d, E, tiles, static_cast<float*>(dx));
       if (err != cudaSuccess) return err;
     }
   }
   if (d_wg != nullptr) {
-    const int ns = dwg_splits(T);
+    const int ns = dwg_splits(T, d, E);
     const int tps = T > 0 ? (T + ns - 1) / ns : 0;
-    const dim3 g((d + kCols - 1) / kCols, ns, (E + kEChunk - 1) / kEChunk);
-    err = dt == MOE_BF16
-              ? launch_pdl(bwd_dwg_part<__nv_bfloat16>, g, dim3(kCols), 0, s, false,
-                           static_cast<const __nv_bfloat16*>(x), static_cast<const float*>(dl), T, d, E,
-                           tps, part)
-              : launch_pdl(bwd_dwg_part<float>, g, dim3(kCols), 0, s, false,
-                           static_cast<const float*>(x), static_cast<const float*>(dl), T, d, E, tps,
-                           part);
+    const int ec = E <= 8 ? 8 : (E <= 16 ? 16 : 32);
+    const int cols = kDwgThreads * (32 / ec);  // columns per block
+    const dim3 g((d + cols - 1) / cols, ns, (E + ec - 1) / ec);
+    if (dt == MOE_BF16) {
+      const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+      err = ec == 8    ? launch_pdl(bwd_dwg_part<__nv_bfloat16, 8>, g, dim3(kDwgThreads), 0, s, false, xb,
+                                    static_cast<const float*>(dl), T, d, E, tps, part)
+            : ec == 16 ? launch_pdl(bwd_dwg_part<__nv_bfloat16, 16>, g, dim3(kDwgThreads), 0, s, false, xb,
+                                    static_cast<const float*>(dl), T, d, E, tps, part)
+                       : launch_pdl(bwd_dwg_part<__nv_bfloat16, 32>, g, dim3(kDwgThreads), 0, s, false, xb,
+                                    static_cast<const float*>(dl), T, d, E, tps, part);
+    } else {
+      const float* xf = static_cast<const float*>(x);
+      err = ec == 8    ? launch_pdl(bwd_dwg_part<float, 8>, g, dim3(kDwgThreads), 0, s, false, xf,
+                                    static_cast<const float*>(dl), T, d, E, tps, part)
+            : ec == 16 ? launch_pdl(bwd_dwg_part<float, 16>, g, dim3(kDwgThreads), 0, s, false, xf,
+                                    static_cast<const float*>(dl), T, d, E, tps, part)
+                       : launch_pdl(bwd_dwg_part<float, 32>, g, dim3(kDwgThreads), 0, s, false, xf,
+                                    static_cast<const float*>(dl), T, d, E, tps, part);
+    }
     if (err != cudaSuccess) return err;
     const long long n = static_cast<long long>(d) * E;
     const int rg = static_cast<int>(std::min<long long>((n + 255) / 256, 8LL * num_sms()));
