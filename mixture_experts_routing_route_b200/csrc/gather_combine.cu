@@ -100,13 +100,15 @@ gather_bulk(const uint8_t* __restrict__ x, uint32_t row_bytes, int T, int k,
   const uint8_t* srcs[kGatherBufs];
   uint8_t* dsts[kGatherBufs];
   uint32_t sizes[kGatherBufs];
-  uint32_t phase = 0;  // bit b: parity to wait for on buffer b
+  uint32_t phase = 0;     // bit b: parity to wait for on buffer b
+  uint32_t inflight = 0;  // bit b: buffer b has a load not yet waited for
   const long long pro = mine < kGatherBufs ? mine : kGatherBufs;
   for (long long i = 0; i < pro; ++i) {
     piece(i, srcs[i], dsts[i], sizes[i]);
     if (sizes[i] && srcs[i]) {
       mbar_arrive_expect_tx(&bars[warp][i], sizes[i]);
       bulk_load(buf0 + i * kGatherPiece, srcs[i], sizes[i], &bars[warp][i]);
+      inflight |= 1u << i;
     }
   }
   bool ok = true;
@@ -123,6 +125,7 @@ gather_bulk(const uint8_t* __restrict__ x, uint32_t row_bytes, int T, int k,
         break;
       }
       phase ^= 1u << b;
+      inflight &= ~(1u << b);
       bulk_store(dsts[b], buf0 + b * kGatherPiece, sizes[b]);
       bulk_commit();
     }
@@ -139,12 +142,14 @@ gather_bulk(const uint8_t* __restrict__ x, uint32_t row_bytes, int T, int k,
       if (sizes[pb] && srcs[pb]) {
         mbar_arrive_expect_tx(&bars[warp][pb], sizes[pb]);
         bulk_load(buf0 + pb * kGatherPiece, srcs[pb], sizes[pb], &bars[warp][pb]);
+        inflight |= 1u << pb;
       }
     }
   }
   if (!ok) {
-    // Let every load still in flight land before the buffers go away.
-    for (int b = 0; b < kGatherBufs; ++b) (void)mbar_wait_bounded(&bars[warp][b], (phase >> b) & 1u);
+    // Let every load still in flight land (bounded) before the buffers go away.
+    for (int b = 0; b < kGatherBufs; ++b)
+      if ((inflight >> b) & 1u) (void)mbar_wait_bounded(&bars[warp][b], (phase >> b) & 1u);
   }
   bulk_wait<0>();
 }

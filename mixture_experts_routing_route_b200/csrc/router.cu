@@ -1039,10 +1039,19 @@ router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
     uint32_t phase = 1;  // the prologue filled round 0
     int st = pre % nst;
     if (pre < nst) phase = 0;
-    for (int kb = pre; kb < nkb; ++kb) {
+    int kb = pre;
+    for (; kb < nkb; ++kb) {
       if (!mbar_wait_bounded(&empty_bar[st], phase ^ 1u)) { set_error(a.ctl, MOE_DEVERR_TIMEOUT); break; }
       issue(kb, st);
       if (++st == nst) { st = 0; phase ^= 1u; }
+    }
+    if (kb < nkb) {
+      // stopped early: wait (bounded) for the last load issued into each
+      // stage, so that none lands after the block has gone
+      for (int s2 = 0; s2 < nst && s2 < kb; ++s2) {
+        const int last = s2 + ((kb - 1 - s2) / nst) * nst;
+        (void)mbar_wait_bounded(&full_bar[s2], static_cast<uint32_t>(last / nst) & 1u);
+      }
     }
   } else if (warp == 1 && lane == 0) {
     const uint32_t idesc = make_idesc_bf16(128, a.Epad, !kTmaB);
