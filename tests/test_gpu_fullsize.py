@@ -97,3 +97,61 @@ def test_full_size_layout_variants_equal(name):
         out1, aux1 = run(**kw)
         assert torch.equal(out1, out0), kw
         assert torch.equal(aux1, aux0), kw
+
+
+def test_full_size_combine_in_gemm_k1():
+    """The Mixtral-shaped layer at top-1 (dropless, and with capacity 1.25):
+    the combine in the down projection's epilogue gives the default path's
+    output bit for bit at full size."""
+    from mixture_experts_routing_route_b200 import MoeLayer
+    sh = CONFIGS["mixtral"].with_(k=1)
+    inp = make_inputs(sh)
+    dv = device_inputs(inp)
+    for cf in (0.0, 1.25):
+        outs = []
+        for comb in (False, True):
+            layer = MoeLayer(dv["wg"], dv["w1"], dv["w2"], w3=dv["w3"], bias=dv["bias"], k=1,
+                             act=sh.act, capacity_factor=cf, combine_in_gemm=comb)
+            out = torch.full((sh.T, sh.d), float("nan"), dtype=dv["x"].dtype, device="cuda")
+            layer.forward(dv["x"], out)
+            torch.cuda.synchronize()
+            assert layer.device_error(sh.T) == 0
+            outs.append(out)
+            del layer
+        assert torch.equal(outs[0], outs[1]), cf
+        torch.cuda.empty_cache()
+
+
+def test_full_size_router_backward():
+    """The router backward on the Mixtral router at full size (T = 4096,
+    d = 4096, E = 8, k = 2) from the GPU's own forward, against the oracle's
+    chain rule: d_logits, dx and dWg."""
+    from mixture_experts_routing_route_b200 import _abi as abi
+    sh = CONFIGS["mixtral"]
+    inp = make_inputs(sh)
+    T, d, E, k = sh.T, sh.d, sh.E, sh.k
+    x, wg = inp.x.to("cuda"), inp.wg.to("cuda")
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    aux = torch.empty(1, dtype=torch.float32, device="cuda")
+    logits = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    probs = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    ws = torch.empty(abi.moe_route_workspace_size(T, d, E), dtype=torch.uint8, device="cuda")
+    abi.moe_workspace_init(ws)
+    abi.moe_route_train(x, wg, None, None, T, d, E, k, idx, w, aux, None, logits, probs, ws)
+    g = torch.from_numpy(np.random.default_rng(5).standard_normal((T, k)).astype(np.float32)).to("cuda")
+    d_logits = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    dx = torch.empty(T, d, dtype=x.dtype, device="cuda")
+    d_wg = torch.empty(d, E, dtype=torch.float32, device="cuda")
+    bws = torch.empty(abi.moe_route_backward_workspace_size(T, d, E), dtype=torch.uint8, device="cuda")
+    abi.moe_workspace_init(bws)
+    abi.moe_route_backward(x, wg, T, d, E, k, probs, logits, idx, w, g, 0.01, 0.001, 1.0, d_logits, dx,
+                           d_wg, bws)
+    torch.cuda.synchronize()
+    assert abi.moe_get_device_error(bws) == 0
+    ref = O.route_backward_from(np32(probs).astype(np.float64), npi(idx), np32(w).astype(np.float64),
+                                np32(logits).astype(np.float64), np32(inp.x), np32(inp.wg),
+                                d_w=np32(g).astype(np.float64), d_aux=0.01, d_z=0.001)
+    assert max_err_ratio(np32(d_logits), ref["d_logits"]) <= 1e-5
+    assert max_err_ratio(np32(d_wg), ref["dwg"]) <= 1e-4
+    assert max_err_ratio(np32(dx), ref["dx"]) <= TOL_BF16_OUT
