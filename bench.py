@@ -38,7 +38,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from mixture_experts_routing_route_b200.inputs import CONFIGS, make_inputs  # noqa: E402
+from workloads import CONFIGS, make_inputs  # noqa: E402
 
 METRIC = "MoE-layer fwd tokens/s on 1 B200 (Mixtral 8e top-2 bf16)"
 UNIT = "tokens/s"
@@ -509,7 +509,7 @@ def main():
     # each replica draws its own tokens; the weights are the same everywhere
     inp = make_inputs(sh)
     if rank != 0:
-        from mixture_experts_routing_route_b200.inputs import make_x
+        from workloads import make_x
         inp.x = make_x(sh.with_(seed=replica_seed(sh, rank)))
     x = inp.x.to(dev)
     layer = MoeLayer(inp.wg.to(dev), inp.w1.to(dev), inp.w2.to(dev),

@@ -136,7 +136,9 @@ def near_tie_tokens(logits32, k, eps=1e-3):
     """Tokens whose k-th and (k+1)-th largest logits are closer than eps.
 
     Their top-k set can flip under a different (equally valid) float
-    summation order, so end-to-end index checks leave them out.
+    summation order, so end-to-end index checks leave them out. "Within eps"
+    is read as a strict gap < eps (a gap of exactly eps is not a near tie);
+    with k = E there is no (k+1)-th logit and no token is flagged.
     """
     l = np.sort(np.asarray(logits32, dtype=np.float64), axis=1)[:, ::-1]
     if k >= l.shape[1]:

@@ -17,7 +17,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
 sys.path.insert(0, ROOT)
 
-from mixture_experts_routing_route_b200.inputs import CONFIGS, make_inputs  # noqa: E402
+from workloads import CONFIGS, make_inputs  # noqa: E402
 from oracle import moe_oracle as O  # noqa: E402
 
 

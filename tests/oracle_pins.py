@@ -577,7 +577,53 @@ def pin_route_backward_identities(o):
     assert np.max(np.abs(b["d_logits"])) < 1e-13
 
 
+def _bf_near_tie(row, k, eps):
+    """Gap between the k-th and (k+1)-th largest values of one row, by an
+    explicit descending walk; no (k+1)-th value (k = E) means no near tie."""
+    s = sorted((float(v) for v in row), reverse=True)
+    if k >= len(s):
+        return False
+    return s[k - 1] - s[k] < eps
+
+
+def pin_near_tie(o):
+    """Which tokens the end-to-end top-k checks leave out: those whose k-th
+    and (k+1)-th largest logits are less than 1e-3 apart (the acceptance
+    rule's "within 1e-3", read as strictly less; an exact gap of eps is not a
+    near tie). Hand-built rows put gaps of 0.999e-3 and 1.001e-3 at the k /
+    k+1 boundary, a small gap one position earlier, unsorted rows, exact ties
+    and k = E; a gap that is exactly eps pins the strict comparison; random
+    rows on a 2^-10 grid (gaps of 0, ~0.98e-3 and ~1.95e-3) are checked
+    against the explicit walk for every k."""
+    eps = 1e-3
+    rows = np.array([
+        [3.0, 2.0, 2.0 - 0.999e-3, -1.0],      # k = 2 boundary gap just below eps
+        [3.0, 2.0, 2.0 - 1.001e-3, -1.0],      # just above eps
+        [2.0, 2.0 - 0.5e-3, 0.5, 0.0],         # small gap between 1st and 2nd only
+        [-1.0, 2.0 - 0.999e-3, 3.0, 2.0],      # first row, unsorted
+        [1.0, 1.0, 1.0, 0.0],                  # exact tie across the boundary
+        [0.0, 1.0, 1.0 + 1.001e-3, 5.0],       # 2nd/3rd gap above eps, unsorted
+    ], dtype=np.float32)
+    assert o.near_tie_tokens(rows, 2, eps).tolist() == [True, False, False, True, True, False]
+    assert o.near_tie_tokens(rows, 1, eps).tolist() == [False, False, True, False, True, False]
+    assert o.near_tie_tokens(rows, 4, eps).tolist() == [False] * len(rows)  # k = E
+    exact = np.array([[1.0, 0.5, 0.25, 0.0]], dtype=np.float32)  # gaps are exact in binary
+    assert o.near_tie_tokens(exact, 1, 0.5).tolist() == [False]
+    assert o.near_tie_tokens(exact, 1, 0.5 + 2.0 ** -20).tolist() == [True]
+    assert o.near_tie_tokens(exact, 2, 0.25).tolist() == [False]
+    rng = _rng(41)
+    grid = (rng.integers(0, 40, size=(300, 8)) * 2.0 ** -10).astype(np.float32)
+    for k in range(1, 9):
+        want = [_bf_near_tie(r, k, eps) for r in grid.tolist()]
+        assert o.near_tie_tokens(grid, k, eps).tolist() == want, k
+    # the flags route() reports are these, on its own fp32 logits
+    x, wg = rng.standard_normal((64, 6)), rng.standard_normal((6, 8))
+    r = o.route(x, wg, None, 3)
+    want = [_bf_near_tie(row, 3, eps) for row in r["logits"].tolist()]
+    assert r["near_tie"].tolist() == want
+
+
 ALL_PINS.extend([pin_philox_kat, pin_jitter, pin_logit_noise, pin_z_loss, pin_route_noise,
                  pin_temperature, pin_route_backward_finite_differences,
-                 pin_route_backward_identities])
+                 pin_route_backward_identities, pin_near_tie])
 

@@ -6,7 +6,7 @@ import os
 import sys
 
 import bench
-from mixture_experts_routing_route_b200.inputs import CONFIGS
+from workloads import CONFIGS
 
 
 def _args(**kw):

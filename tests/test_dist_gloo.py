@@ -22,7 +22,7 @@ def _worker(rank, world, port, out):
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         import bench
-        from mixture_experts_routing_route_b200.inputs import make_x, small_case
+        from workloads import make_x, small_case
         sh = small_case("dist", T=8, d=128, E=4, k=2, F=128, act="swiglu").shape
         x = make_x(sh.with_(seed=bench.replica_seed(sh, rank)))
         t_ms = 10.0 + 5.0 * rank  # a per-rank time; rank 1 is the slowest

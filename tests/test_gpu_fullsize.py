@@ -7,7 +7,7 @@ import numpy as np
 import pytest
 import torch
 
-from mixture_experts_routing_route_b200.inputs import CONFIGS, make_inputs
+from workloads import CONFIGS, make_inputs
 from oracle import moe_oracle as O
 from tests.gpu_helpers import (check_topk_end_to_end, TOL_AUX_REL, TOL_BF16_OUT, TOL_PROB_REL, ExpertWeights,
                                device_inputs, max_err_ratio, np32, npi, rel_err)

@@ -6,7 +6,7 @@ import pytest
 import torch
 
 from mixture_experts_routing_route_b200 import _abi as abi
-from mixture_experts_routing_route_b200.inputs import small_case
+from workloads import small_case
 from oracle import moe_oracle as O
 from tests.gpu_helpers import (check_topk_end_to_end, TOL_AUX_REL, TOL_BF16_OUT, TOL_PROB_REL, ExpertWeights,
                                max_err_ratio, new_ws, np32, npi, rel_err)

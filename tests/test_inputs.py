@@ -6,8 +6,8 @@ import os
 
 import torch
 
-from mixture_experts_routing_route_b200.inputs import (CONFIGS, LONG_SKEWED_BETA, bias_vector,
-                                                        make_inputs, small_case, worked_example_a)
+from workloads import (CONFIGS, LONG_SKEWED_BETA, bias_vector, make_inputs, small_case,
+                       worked_example_a)
 
 
 def test_deterministic_and_shapes():

@@ -121,6 +121,34 @@ def _backward_drops_z(x, wg, bias, k, d_w=None, d_aux=0.0, d_z=0.0, noise=None, 
     return _REAL["route_backward"](x, wg, bias, k, d_w, d_aux, 0.0, noise, temperature)
 
 
+def _near_tie_next_column(logits32, k, eps=1e-3):
+    l = np.sort(np.asarray(logits32, dtype=np.float64), axis=1)[:, ::-1]
+    if k + 1 >= l.shape[1]:
+        return np.zeros(l.shape[0], dtype=bool)
+    return (l[:, k] - l[:, k + 1]) < eps
+
+
+def _near_tie_sign(logits32, k, eps=1e-3):
+    l = np.sort(np.asarray(logits32, dtype=np.float64), axis=1)[:, ::-1]
+    if k >= l.shape[1]:
+        return np.zeros(l.shape[0], dtype=bool)
+    return (l[:, k] - l[:, k - 1]) < eps
+
+
+def _near_tie_le(logits32, k, eps=1e-3):
+    l = np.sort(np.asarray(logits32, dtype=np.float64), axis=1)[:, ::-1]
+    if k >= l.shape[1]:
+        return np.zeros(l.shape[0], dtype=bool)
+    return (l[:, k - 1] - l[:, k]) <= eps
+
+
+def _near_tie_unsorted(logits32, k, eps=1e-3):
+    l = np.asarray(logits32, dtype=np.float64)
+    if k >= l.shape[1]:
+        return np.zeros(l.shape[0], dtype=bool)
+    return np.abs(l[:, k - 1] - l[:, k]) < eps
+
+
 _REAL = {n: getattr(O, n) for n in ("combine", "expert_ffn", "permute", "permute_binned",
                                     "jitter_multipliers", "route_backward")}
 
@@ -144,6 +172,10 @@ MUTATIONS = {
     "temperature_ignored": ("tempered_logits", _temperature_ignored),
     "backward_ignores_temperature": ("route_backward", _backward_ignores_temperature),
     "backward_drops_z_loss": ("route_backward", _backward_drops_z),
+    "near_tie_next_column": ("near_tie_tokens", _near_tie_next_column),
+    "near_tie_sign_slip": ("near_tie_tokens", _near_tie_sign),
+    "near_tie_non_strict": ("near_tie_tokens", _near_tie_le),
+    "near_tie_unsorted": ("near_tie_tokens", _near_tie_unsorted),
 }
 
 

@@ -1,5 +1,9 @@
 """Seeded synthetic inputs for the MoE-layer forward.
 
+A module of its own, outside the library package: it imports torch only, so a
+process that runs the CPU oracle on these inputs (the reference arm of the
+benchmark, the calibration script) never loads the CUDA library.
+
 This module only draws random numbers and fixes tensor shapes. It holds none of
 the layer's arithmetic (no routing, no sorting, no FFN), so that the CPU oracle
 and the CUDA path can both be fed the very same bytes from here without sharing
