@@ -59,6 +59,8 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-per-config", action="store_true",
+                   help="skip the bounded runs of the other workloads (the per_config key)")
     p.add_argument("--binned", action="store_true",
                    help="padded-binned [E, C, hs] layout (capacity_factor 0: C = the largest count)")
     p.add_argument("--gather-in-gemm", action="store_true",
@@ -85,6 +87,14 @@ def shape_of(args):
     if args.k is not None and args.k != sh.k:
         sh = sh.with_(k=args.k, name=f"{sh.name}_k{args.k}")
     return sh
+
+
+def arm_config(sh, args, world):
+    """The JSON line's config, the same in both arms for the same flags."""
+    return dict(workload_config(sh), parallelism=f"replicas x{world}" if world > 1 else "1 GPU",
+                **({"gather": "in the up projection (tile::gather4)"} if args.gather_in_gemm else {}),
+                **({"layout": "binned [E, C, d]"} if args.binned else {}),
+                **({"combine": "in the down projection's epilogue"} if args.combine_in_gemm else {}))
 
 
 def workload_config(sh):
@@ -180,7 +190,7 @@ class ClockSampler:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", ",".join(str(g) for g in self.gpus)],
+                 "-lms", "20", "-i", ",".join(str(g) for g in self.gpus)],
                 stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -391,7 +401,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded)", "config": workload_config(sh),
+        "data": "synthetic (seeded)", "config": arm_config(sh, args, max(1, args.gpus)),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "cpu_model": cpu_model(),
                          "kind": "oracle",
                          "sample": f"{tokens} of the workload's {sh.T} tokens per step, whole "
@@ -493,14 +503,155 @@ def run_router_backward(args):
     return 0
 
 
+PER_CONFIG = ("tiny_fp32", "fine_grained", "capacity_skew", "long_skewed", "long_skewed_cf")
+PER_CONFIG_STEPS = 20
+
+
+def stage_roofline(sh, stage_ms, alg, peaks, tc_peak, args):
+    """Per-stage time, achieved GB/s and TFLOP/s and their fractions of the
+    measured peaks (and of the spec figures)."""
+    roof = {}
+    for s_ in STAGES:
+        t = stage_ms[s_] * 1e-3
+        a = alg[s_]
+        if s_ == "gather" and args.gather_in_gemm and sh.dtype == "bf16" and not args.combine_in_gemm:
+            roof[s_] = {"us": stage_ms[s_] * 1e3, "fused_into": "ffn_up (tile::gather4 A loads)"}
+            continue
+        if s_ == "combine" and args.combine_in_gemm:
+            roof[s_] = {"us": stage_ms[s_] * 1e3, "fused_into": "ffn_down (epilogue)"}
+            continue
+        r = {"us": stage_ms[s_] * 1e3, "GB_s": a["bytes"] / t / 1e9 if t > 0 else None}
+        r["hbm_frac"] = r["GB_s"] / peaks["hbm_gbs"] if r["GB_s"] else None
+        r["hbm_frac_spec"] = r["GB_s"] / SPEC_HBM_GBS if r["GB_s"] else None
+        if "flops" in a:
+            r["TFLOP_s"] = a["flops"] / t / 1e12 if t > 0 else None
+            r["tensor_frac"] = r["TFLOP_s"] / tc_peak if r["TFLOP_s"] and sh.dtype == "bf16" else None
+            r["tensor_frac_spec"] = r["TFLOP_s"] / SPEC_BF16_TFLOPS if r["TFLOP_s"] else None
+        roof[s_] = r
+    return roof
+
+
+def dispatch_span_of(stage_ms, alg, peaks):
+    """Route + permute + gather judged as one span against its bytes (the
+    permute alone moves < 1 MB and is latency-bound)."""
+    span_us = sum(stage_ms[s_] for s_ in ("route", "permute", "gather")) * 1e3
+    span_bytes = sum(alg[s_]["bytes"] for s_ in ("route", "permute", "gather"))
+    gbs = span_bytes / (span_us * 1e-6) / 1e9 if span_us > 0 else None
+    return {"us": span_us, "bytes": span_bytes,
+            "hbm_frac": gbs / peaks["hbm_gbs"] if gbs else None,
+            "hbm_frac_spec": gbs / SPEC_HBM_GBS if gbs else None}
+
+
+class LayerRun:
+    """One workload's layer on the device with its input, output and the L2
+    eviction buffer; timed_steps() runs the timed loop, stage_times() the
+    separate per-stage pass."""
+
+    def __init__(self, sh, inp, dev, args, flush):
+        from mixture_experts_routing_route_b200 import MoeLayer
+        self.sh, self.args = sh, args
+        self.x = inp.x.to(dev)
+        self.layer = MoeLayer(inp.wg.to(dev), inp.w1.to(dev), inp.w2.to(dev),
+                              w3=None if inp.w3 is None else inp.w3.to(dev),
+                              bias=None if inp.bias is None else inp.bias.to(dev),
+                              k=sh.k, act=sh.act, capacity_factor=sh.cf,
+                              gather_in_gemm=args.gather_in_gemm, binned=args.binned,
+                              combine_in_gemm=args.combine_in_gemm)
+        self.out = torch.empty(sh.T, sh.d, dtype=self.x.dtype, device=dev)
+        self.aux = torch.empty(1, dtype=torch.float32, device=dev)
+        self.flush = flush
+        self.sink = torch.zeros(1, dtype=torch.int64, device=dev)
+
+    def evict_l2(self):
+        torch.sum(self.flush, dim=0, dtype=torch.int64, out=self.sink[0])
+
+    def warm(self, n):
+        for _ in range(n):
+            self.layer.forward(self.x, self.out, self.aux)
+        torch.cuda.synchronize()
+        if self.layer.device_error(self.sh.T) != 0:
+            raise RuntimeError(f"device error word set during warm-up ({self.sh.name})")
+        v = self.layer.views(self.sh.T)
+        self.kept = v["kept_counts"].cpu().tolist()
+        self.bucket_rows = int(v["seg_offsets"][-1].item()) if self.args.binned else None
+
+    def timed_steps(self, steps, world=1):
+        """Timed steps record 4 events: before route, around the up projection
+        (the roofline's kernel) and after combine; the other stage boundaries
+        carry no event, so consecutive kernels overlap their launches as in
+        use. Returns [(step ms, up-projection ms)] and the launches counted."""
+        from mixture_experts_routing_route_b200 import _abi as abi
+        evs = [[torch.cuda.Event(enable_timing=True) if j in (0, 3, 4, 6) else None for j in range(7)]
+               for _ in range(steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        n0 = abi.moe_kernel_launches()
+        for i in range(steps):
+            self.evict_l2()
+            self.layer.forward(self.x, self.out, self.aux, events=evs[i])
+        n1 = abi.moe_kernel_launches()
+        torch.cuda.synchronize()
+        barrier(world)
+        per = [(evs[i][0].elapsed_time(evs[i][6]), evs[i][3].elapsed_time(evs[i][4]))
+               for i in range(steps)]
+        return per, n1 - n0
+
+    def stage_times(self, nb):
+        """Median over nb steps of each stage's time, with an event at every
+        stage boundary (the events serialise the stages). The first step
+        starts on an idle GPU, so its events also span the host's enqueue of
+        each launch: hence the median."""
+        bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(nb)]
+        for i in range(nb):
+            self.evict_l2()
+            self.layer.forward(self.x, self.out, self.aux, events=bevs[i])
+        torch.cuda.synchronize()
+        if self.layer.device_error(self.sh.T) != 0:
+            raise RuntimeError(f"device error word set during the stage pass ({self.sh.name})")
+        return {s_: statistics.median(bevs[i][j].elapsed_time(bevs[i][j + 1]) for i in range(nb))
+                for j, s_ in enumerate(STAGES)}
+
+
+def per_config_runs(dev, args, flush, peaks):
+    """Every other workload of the layer on this GPU, with a bounded step
+    count: tokens/s, ms per forward, the stages' times and fractions of the
+    measured peaks (burst GEMM figure), and the dispatch span."""
+    out = {}
+    for name in PER_CONFIG:
+        sh = CONFIGS[name]
+        if args.k is not None and args.k != sh.k:
+            continue
+        inp = make_inputs(sh)
+        run = LayerRun(sh, inp, dev, args, flush)
+        del inp
+        run.warm(3)
+        per, launches = run.timed_steps(PER_CONFIG_STEPS)
+        step_ms = [p[0] for p in per]
+        up_ms = statistics.mean(p[1] for p in per)
+        stage_ms = run.stage_times(PER_CONFIG_STEPS)
+        alg = algorithmic(sh, run.kept, run.bucket_rows, combine_in_gemm=args.combine_in_gemm)
+        ms = sum(step_ms) / len(step_ms)
+        roof = stage_roofline(sh, stage_ms, alg, peaks, peaks["bf16_tflops"], args)
+        out[name] = {
+            "workload": workload_config(sh)["workload"],
+            "tokens_per_s": sh.T / (ms * 1e-3), "ms_per_forward": ms, "steps": PER_CONFIG_STEPS,
+            "gpu_launches_per_step": launches / PER_CONFIG_STEPS,
+            "ffn_up_event_us": up_ms * 1e3,
+            "stages": roof, "dispatch_span": dispatch_span_of(stage_ms, alg, peaks),
+            "aux_loss": float(run.aux.item()), "rows": int(sum(run.kept)),
+            "imbalance_max_over_mean": (max(run.kept) / (sum(run.kept) / sh.E)) if sum(run.kept) else None,
+        }
+        del run
+        torch.cuda.empty_cache()
+    return out
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     if args.router_backward:
         return run_router_backward(args)
-    from mixture_experts_routing_route_b200 import MoeLayer
-    from mixture_experts_routing_route_b200 import _abi as abi
 
     rank, world, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
@@ -511,77 +662,41 @@ def main():
     if rank != 0:
         from workloads import make_x
         inp.x = make_x(sh.with_(seed=replica_seed(sh, rank)))
-    x = inp.x.to(dev)
-    layer = MoeLayer(inp.wg.to(dev), inp.w1.to(dev), inp.w2.to(dev),
-                     w3=None if inp.w3 is None else inp.w3.to(dev),
-                     bias=None if inp.bias is None else inp.bias.to(dev),
-                     k=sh.k, act=sh.act, capacity_factor=sh.cf, gather_in_gemm=args.gather_in_gemm,
-                     binned=args.binned, combine_in_gemm=args.combine_in_gemm)
-    out = torch.empty(sh.T, sh.d, dtype=x.dtype, device=dev)
-    aux = torch.empty(1, dtype=torch.float32, device=dev)
     flush = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
-    flush_sink = torch.zeros(1, dtype=torch.int64, device=dev)
-
-    def evict_l2():
-        torch.sum(flush, dim=0, dtype=torch.int64, out=flush_sink[0])
-    stream = torch.cuda.current_stream()
-    # Timed steps record 4 events: before route, around the up projection (the
-    # roofline's kernel) and after combine; the other stage boundaries carry
-    # no event, so consecutive kernels overlap their launches as in use.
-    evs = [[torch.cuda.Event(enable_timing=True) if j in (0, 3, 4, 6) else None for j in range(7)]
-           for _ in range(args.steps)]
-
-    for _ in range(max(3, args.warmup)):
-        layer.forward(x, out, aux)
-    torch.cuda.synchronize()
-    if layer.device_error(sh.T) != 0:
-        raise RuntimeError("device error word set during warm-up")
-    v = layer.views(sh.T)
-    kept = v["kept_counts"].cpu().tolist()
-    bucket_rows = int(v["seg_offsets"][-1].item()) if args.binned else None
-    def timed_region():
-        barrier(world)
-        torch.cuda.synchronize()
-        n0 = abi.moe_kernel_launches()
-        for i in range(args.steps):
-            evict_l2()
-            layer.forward(x, out, aux, events=evs[i])
-        n1 = abi.moe_kernel_launches()
-        torch.cuda.synchronize()
-        barrier(world)
-        per = [(evs[i][0].elapsed_time(evs[i][6]), evs[i][3].elapsed_time(evs[i][4]))
-               for i in range(args.steps)]
-        return per, n1 - n0
+    run = LayerRun(sh, inp, dev, args, flush)
+    run.warm(max(3, args.warmup))
+    kept, bucket_rows = run.kept, run.bucket_rows
 
     sampler = ClockSampler(list(range(world)) if rank == 0 else [])
     if rank == 0:
         sampler.start()
-    per, launches = timed_region()
+    per, launches = run.timed_steps(args.steps, world)
     clocks = sampler.stop() if rank == 0 else {}
-    if rank == 0 and ClockSampler.rejected(clocks):
-        sampler = ClockSampler(list(range(world)))
-        sampler.start()
-        per, launches = timed_region()
-        clocks = sampler.stop()
-        clocks["remeasured"] = True
+    remeasure = int(rank == 0 and ClockSampler.rejected(clocks))
+    if world > 1:
+        # every rank takes the same collective steps: agree on a re-measurement
+        import torch.distributed as dist
+        t = torch.tensor([remeasure], dtype=torch.int32, device=dev)
+        dist.broadcast(t, 0)
+        remeasure = int(t.item())
+    if remeasure:
+        sampler = ClockSampler(list(range(world)) if rank == 0 else [])
+        if rank == 0:
+            sampler.start()
+        per, launches = run.timed_steps(args.steps, world)
+        if rank == 0:
+            clocks = sampler.stop()
+            clocks["remeasured"] = True
     step_ms = [p[0] for p in per]
     total_ms = reduce_max(sum(step_ms), world)
     up_ms = statistics.mean(p[1] for p in per)
-    if layer.device_error(sh.T) != 0:
+    if run.layer.device_error(sh.T) != 0:
         raise RuntimeError("device error word set during the timed steps")
 
     # Stage breakdown: a separate, untimed pass with an event at every stage
     # boundary (the events serialise the stages).
     nb = min(args.steps, 20)
-    bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(nb)]
-    for i in range(nb):
-        evict_l2()
-        layer.forward(x, out, aux, events=bevs[i])
-    torch.cuda.synchronize()
-    # Median over the steps: the first one starts on an idle GPU, so its stage
-    # events also span the host's enqueue of each launch.
-    stage_ms = {s: statistics.median(bevs[i][j].elapsed_time(bevs[i][j + 1]) for i in range(nb))
-                for j, s in enumerate(STAGES)}
+    stage_ms = run.stage_times(nb)
     alg = algorithmic(sh, kept, bucket_rows, combine_in_gemm=args.combine_in_gemm)
     peaks = load_peaks()
     # A timed region long enough to hit the 1 kW power cap is compared with the
@@ -591,24 +706,7 @@ def main():
         tc_peak, tc_kind = peaks["bf16_tflops_sustained"], "sustained (sw_power_cap active while timed)"
     else:
         tc_peak, tc_kind = peaks["bf16_tflops"], "burst"
-    roof = {}
-    for s in STAGES:
-        t = stage_ms[s] * 1e-3
-        a = alg[s]
-        if s == "gather" and args.gather_in_gemm and sh.dtype == "bf16" and not args.combine_in_gemm:
-            roof[s] = {"us": stage_ms[s] * 1e3, "fused_into": "ffn_up (tile::gather4 A loads)"}
-            continue
-        if s == "combine" and args.combine_in_gemm:
-            roof[s] = {"us": stage_ms[s] * 1e3, "fused_into": "ffn_down (epilogue)"}
-            continue
-        r = {"us": stage_ms[s] * 1e3, "GB_s": a["bytes"] / t / 1e9 if t > 0 else None}
-        r["hbm_frac"] = r["GB_s"] / peaks["hbm_gbs"] if r["GB_s"] else None
-        r["hbm_frac_spec"] = r["GB_s"] / SPEC_HBM_GBS if r["GB_s"] else None
-        if "flops" in a:
-            r["TFLOP_s"] = a["flops"] / t / 1e12 if t > 0 else None
-            r["tensor_frac"] = r["TFLOP_s"] / tc_peak if r["TFLOP_s"] else None
-            r["tensor_frac_spec"] = r["TFLOP_s"] / SPEC_BF16_TFLOPS if r["TFLOP_s"] else None
-        roof[s] = r
+    roof = stage_roofline(sh, stage_ms, alg, peaks, tc_peak, args)
 
     dom = "ffn_up"
     tf = alg[dom]["flops"] / (up_ms * 1e-3) / 1e12 if up_ms > 0 else None
@@ -622,35 +720,32 @@ def main():
                 "launch_us": up_ms * 1e3,
                 "timing": "CUDA events on the launch stream around the up projection, every timed step",
                 "peak_spec": SPEC_BF16_TFLOPS, "frac_spec": tf / SPEC_BF16_TFLOPS if tf else None}
-    # Route + permute + gather judged as one span against its bytes (the
-    # permute alone moves < 1 MB and is latency-bound).
-    span_us = sum(stage_ms[s_] for s_ in ("route", "permute", "gather")) * 1e3
-    span_bytes = sum(alg[s_]["bytes"] for s_ in ("route", "permute", "gather"))
-    dispatch_span = {"us": span_us, "bytes": span_bytes,
-                     "hbm_frac": span_bytes / (span_us * 1e-6) / 1e9 / peaks["hbm_gbs"] if span_us > 0 else None,
-                     "hbm_frac_spec": span_bytes / (span_us * 1e-6) / 1e9 / SPEC_HBM_GBS if span_us > 0 else None}
+    dispatch_span = dispatch_span_of(stage_ms, alg, peaks)
 
     e2e = None
     if not args.no_e2e:
-        e2e = measure_e2e(layer, inp, sh, args, world, x.element_size())
+        e2e = measure_e2e(run.layer, inp, sh, args, world, run.x.element_size())
 
     if rank != 0:
         _finish(world)
         return 0
+    aux_value = float(run.aux.item())
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(sh, inp)
+    per_config = None
+    if world == 1 and not args.no_per_config and sh.name == "mixtral" and not args.router_backward:
+        del run
+        torch.cuda.empty_cache()
+        per_config = per_config_runs(dev, args, flush, peaks)
     value = job_value(sh.T, args.steps, world, total_ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": total_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": sh.dtype,
         "data": "synthetic (seeded; random-init weights of the layer's shape)",
-        "config": dict(workload_config(sh), parallelism=f"replicas x{world}" if world > 1 else "1 GPU",
-                       **({"gather": "in the up projection (tile::gather4)"} if args.gather_in_gemm else {}),
-                       **({"layout": f"binned [E, C, d], C = {bucket_rows // sh.E if sh.E else 0}"}
-                          if args.binned else {}),
-                       **({"combine": "in the down projection's epilogue"} if args.combine_in_gemm else {})),
+        "config": arm_config(sh, args, world),
+        **({"bin_rows_C": bucket_rows // sh.E} if args.binned and sh.E else {}),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks,
@@ -658,9 +753,14 @@ def main():
         "dispatch_span": dispatch_span,
         "stages_note": f"per-stage times: median over a separate pass of {nb} steps with an "
                        f"event at every stage boundary (events serialise the stages)",
-        "aux_loss": float(aux.item()),
+        "aux_loss": aux_value,
         "rows": int(sum(kept)), "experts_active": int(sum(1 for c in kept if c > 0)),
         "imbalance_max_over_mean": (max(kept) / (sum(kept) / sh.E)) if sum(kept) else None,
+        "per_config": per_config,
+        "per_config_note": (f"each other workload of the layer on the same GPU after the headline: "
+                            f"3 warm-up and {PER_CONFIG_STEPS} timed steps (L2 evicted between), "
+                            f"stage times from a separate {PER_CONFIG_STEPS}-step pass; GEMM "
+                            f"fractions of the burst bf16 peak") if per_config else None,
     }
     print(json.dumps(line), flush=True)
     _finish(world)

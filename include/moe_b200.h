@@ -166,8 +166,22 @@ typedef struct {
 MOE_API const char* moe_status_string(moe_status_t status);
 
 /* Zero the control block (first 256 bytes) of a workspace, asynchronously
- * on `stream`. Needed once per workspace before its first use. */
+ * on `stream`. Needed once per workspace before its first use, and again
+ * after a call reported MOE_DEVERR_TIMEOUT: a wait that gave up leaves the
+ * grid-barrier words of the control block in an unknown state, and the next
+ * call on that workspace could pass its barrier early. Zeroing also clears
+ * the error word and restores the default wait limit. */
 MOE_API moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Set how long a kernel using this workspace waits at a barrier between its
+ * CTAs (the permute's grid barrier, where every CTA waits for all others to
+ * publish their counts) before it gives up: it then sets MOE_DEVERR_TIMEOUT,
+ * skips the work that needed the barrier and returns, leaving the GPU
+ * context usable. limit_us in microseconds; 0 restores the default of 2 s.
+ * Written asynchronously on `stream` (one small kernel). The waits inside a
+ * CTA (on TMA and tensor-core completion) keep their fixed 2 s bound. */
+MOE_API moe_status_t moe_workspace_set_wait_limit(void* ws, size_t ws_bytes, uint32_t limit_us,
+                                                  moe_stream_t stream);
 
 /* Number of CUDA kernels this library has launched in this process so far
  * (all devices, all streams, every entry point), counted on the host at each
@@ -348,11 +362,15 @@ MOE_API int64_t moe_rows_max_binned(int T, int k, int E, int64_t capacity);
  *   MOE_ERR_WORKSPACE and launch nothing.
  * Its scratch is one file-scope static device array (256 bytes of control
  * block + 4 bytes per slot up to the limit, ~256 KB), which every GPU that
- * loads this library holds until the process exits. The first call on a
- * device looks up that array's device address (cudaGetSymbolAddress, with
- * that device current); make that first call before any stream capture.
- * Every call shares the array: calls that overlap on the GPU (other streams,
- * other host threads) race and give wrong results. */
+ * loads this library holds until the process exits. Each call looks up that
+ * array's device address (cudaGetSymbolAddress, with the caller's device
+ * current), so the address stays right after a cudaDeviceReset. The first
+ * call on a device may load the library's device code (the CUDA runtime
+ * loads modules lazily) and loading allocates device memory, the array
+ * included: a caller that must not allocate makes one call at start-up, and
+ * makes that first call before any stream capture. Every call shares the
+ * array and clears its control block first: calls that overlap on the GPU
+ * (other streams, other host threads) race and give wrong results. */
 #define MOE_PERMUTE_NOALLOC_MAX_SLOTS 65536
 MOE_API moe_status_t moe_permute_noalloc(const int32_t* topk_idx, int T, int k, int E,
                                          int64_t capacity, int32_t* counts, int32_t* bins,

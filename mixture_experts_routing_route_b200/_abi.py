@@ -64,6 +64,7 @@ class MoeViewsC(ctypes.Structure):
 _SIGS = {
     "moe_status_string": (ctypes.c_char_p, [c_int]),
     "moe_workspace_init": (c_int, [c_void_p, c_size_t, c_void_p]),
+    "moe_workspace_set_wait_limit": (c_int, [c_void_p, c_size_t, c_uint32, c_void_p]),
     "moe_kernel_launches": (ctypes.c_uint64, []),
     "moe_get_device_error": (c_int, [c_void_p, c_void_p, ctypes.POINTER(c_uint32), c_int]),
     "moe_capacity": (c_int64, [c_double, c_int, c_int, c_int]),
@@ -178,6 +179,11 @@ def moe_permute_workspace_size(T, k, E) -> int:
 
 def moe_workspace_init(ws: torch.Tensor, stream=None):
     _check("moe_workspace_init", _lib.moe_workspace_init(_ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_workspace_set_wait_limit(ws: torch.Tensor, limit_us: int, stream=None):
+    _check("moe_workspace_set_wait_limit",
+           _lib.moe_workspace_set_wait_limit(_ptr(ws), ws.numel(), int(limit_us), _stream(stream)))
 
 
 def moe_get_device_error(ws: torch.Tensor, stream=None, clear: bool = True) -> int:

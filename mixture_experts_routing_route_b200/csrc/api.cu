@@ -249,6 +249,14 @@ moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream) 
   return from_cuda(cudaMemsetAsync(ws, 0, sizeof(Control), reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status_t moe_workspace_set_wait_limit(void* ws, size_t ws_bytes, uint32_t limit_us,
+                                          moe_stream_t stream) {
+  MOE_NEED(ws);
+  if (ws_bytes < sizeof(Control)) return MOE_ERR_WORKSPACE;
+  return from_cuda(launch_set_wait_limit(static_cast<Control*>(ws), limit_us,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_get_device_error(void* ws, moe_stream_t stream, uint32_t* host_bits, int clear) {
   MOE_NEED(ws);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

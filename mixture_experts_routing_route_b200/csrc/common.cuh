@@ -16,7 +16,8 @@ struct Control {
   uint32_t route_ticket;  // blocks of the router that finished (reset by the last one)
   uint32_t bar_count;     // grid barrier: blocks arrived (reset by the last one)
   uint32_t bar_gen;       // grid barrier: generation, bumped when all arrived
-  uint32_t reserved[60];
+  uint32_t wait_limit_us; // limit of the waits between CTAs; 0: 2 s
+  uint32_t reserved[59];
 };
 static_assert(sizeof(Control) == 256, "control block is 256 bytes");
 
@@ -25,6 +26,12 @@ __host__ __device__ inline size_t align_up(size_t v, size_t a = kAlign) { return
 
 __device__ __forceinline__ void set_error(Control* ctl, uint32_t bits) {
   atomicOr(&ctl->err, bits);
+}
+
+// How long a wait between CTAs may last before it gives up (ns).
+__device__ __forceinline__ uint64_t wait_limit_ns(const Control* ctl) {
+  const uint32_t us = *reinterpret_cast<const volatile uint32_t*>(&ctl->wait_limit_us);
+  return us == 0 ? 2000000000ull : static_cast<uint64_t>(us) * 1000ull;
 }
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t u) {
@@ -154,6 +161,9 @@ cudaError_t launch_gather(const void* x, size_t elem, int T, int d, int k, const
                           const int32_t* seg, int E, int64_t rows_max, void* x_perm, Control* ctl,
                           cudaStream_t s, bool binned = false, const int32_t* slot_to_row = nullptr,
                           void* zero_out = nullptr);
+
+// Control block: write the wait limit (one thread).
+cudaError_t launch_set_wait_limit(Control* ctl, uint32_t limit_us, cudaStream_t s);
 
 // Grouped GEMMs. bf16: A is x_perm [rows_max, d] when row_slot is NULL, else
 // the token rows x [a_rows = T, d], gathered by the up projection itself

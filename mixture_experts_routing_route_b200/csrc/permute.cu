@@ -209,9 +209,10 @@ __device__ bool grid_barrier(Control* ctl, unsigned nblocks) {
       __threadfence();
       atomicAdd(&ctl->bar_gen, 1u);
     } else {
+      const uint64_t limit = wait_limit_ns(ctl);
       const uint64_t t0 = globaltimer_ns_p();
       while (*gen_p == gen) {
-        if (globaltimer_ns_p() - t0 > 2000000000ull) {
+        if (globaltimer_ns_p() - t0 > limit) {
           set_error(ctl, MOE_DEVERR_TIMEOUT);
           ok = 0;
           break;
@@ -376,7 +377,16 @@ permute_grid_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_
   }
 }
 
+__global__ void set_wait_limit_kernel(Control* ctl, uint32_t limit_us) {
+  pdl_begin();
+  ctl->wait_limit_us = limit_us;
+}
+
 }  // namespace
+
+cudaError_t launch_set_wait_limit(Control* ctl, uint32_t limit_us, cudaStream_t s) {
+  return launch_pdl(set_wait_limit_kernel, dim3(1), dim3(1), 0, s, false, ctl, limit_us);
+}
 
 size_t permute_scratch_bytes(int T, int k, int E) {
   // rank scratch of the single-CTA kernel, then per-CTA counts of the multi-CTA one

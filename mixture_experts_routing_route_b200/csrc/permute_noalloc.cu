@@ -9,11 +9,13 @@
 //
 // The array is shared by every call on a device and keeps the last call's
 // contents. Calls that overlap on the GPU (two streams, or two host threads)
-// race on it and give wrong results; serialise them. The error word is
-// cleared at the start of each call; the rank buffer needs no clearing
-// (every slot's rank is written before it is read).
+// race on it and give wrong results; serialise them. The control block (error
+// word and barrier words) is cleared at the start of each call; the rank
+// buffer needs no clearing (every slot's rank is written before it is read).
+// The first call on a device may load this library's device code (the CUDA
+// runtime loads modules lazily), and loading allocates device memory, this
+// array included: a caller that must not allocate makes one call at start-up.
 #include "common.cuh"
-#include <mutex>
 
 namespace moe {
 namespace {
@@ -24,26 +26,18 @@ constexpr size_t kNoallocCtlWords = sizeof(Control) / 4;
 // [control block (256 B)] [rank of each slot (kNoallocMaxSlots int32)]
 static __device__ __align__(256) int32_t g_permute_scratch[kNoallocCtlWords + kNoallocMaxSlots];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of the static scratch on the current device, looked up once
-// per device. In host code g_permute_scratch is only a host-side stand-in for
-// the symbol, never a device address, so the address must come from here.
+// Device address of the static scratch on the current device. In host code
+// g_permute_scratch is only a host-side stand-in for the symbol, never a
+// device address, so the address must come from cudaGetSymbolAddress, called
+// with the caller's device current. It is looked up on every call (a host-side
+// table lookup once the module is loaded) rather than cached: after a
+// cudaDeviceReset the module is loaded again and the array may move.
 cudaError_t scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_permute_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_permute_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  if (p == nullptr) return cudaErrorInvalidSymbol;
+  *out = p;
   return cudaSuccess;
 }
 

@@ -58,7 +58,7 @@ from scipy.special import erf as _erf
 __all__ = [
     "gate_logits", "softmax_rows", "topk_select", "renormalise", "aux_loss",
     "near_tie_tokens", "route", "capacity", "sort_end_bit", "permute", "gather",
-    "activation", "expert_ffn", "combine", "forward", "forward_tokens",
+    "activation", "expert_hidden", "expert_ffn", "combine", "forward", "forward_tokens",
     "permute_binned", "gather_binned", "expert_ffn_binned",
     "philox4x32_10", "jitter_multipliers", "apply_jitter", "bf16_round", "logit_noise", "z_loss",
 ]
@@ -524,12 +524,30 @@ def activation(z, act, z_up=None):
     raise ValueError(act)
 
 
-def _expert_mlp(xe, e, w1, w3, w2, act):
+def _expert_hidden(xe, e, w1, w3, act):
     xe = np.asarray(xe, dtype=np.float64)
     z1 = xe @ np.asarray(w1[e], dtype=np.float64)
     z3 = xe @ np.asarray(w3[e], dtype=np.float64) if act == "swiglu" else None
-    h = activation(z1, act, z3)
-    return h @ np.asarray(w2[e], dtype=np.float64)
+    return activation(z1, act, z3)
+
+
+def _expert_mlp(xe, e, w1, w3, w2, act):
+    return _expert_hidden(xe, e, w1, w3, act) @ np.asarray(w2[e], dtype=np.float64)
+
+
+def expert_hidden(x_perm, seg_offsets, w1, w3, act):
+    """The expert MLP's hidden rows h = act(x_perm W1[e]) (GELU) or
+    silu(x_perm W_gate[e]) * (x_perm W_up[e]) (SwiGLU) over each expert's
+    rows: the first bmm and the activation of the MegaBlocks page's section
+    4.3. Returns float64 [R, F]."""
+    seg = np.asarray(seg_offsets, dtype=np.int64)
+    E = len(seg) - 1
+    h = np.zeros((int(seg[-1]), np.asarray(w1[0]).shape[1]), dtype=np.float64)
+    for e in range(E):
+        a, b = int(seg[e]), int(seg[e + 1])
+        if b > a:
+            h[a:b] = _expert_hidden(x_perm[a:b], e, w1, w3, act)
+    return h
 
 
 def expert_ffn(x_perm, seg_offsets, w1, w3, w2, act):

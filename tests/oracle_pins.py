@@ -263,6 +263,33 @@ def pin_dense_mlp(o):
     assert np.allclose(os_, ref_s, rtol=1e-12, atol=1e-12)
 
 
+def pin_expert_hidden_segments(o):
+    """The hidden rows of each expert's segment are that expert's first
+    projection and activation (torch F.linear/F.gelu/F.silu, fp64); an
+    expert with an empty segment contributes no rows, and the rows of
+    expert_ffn are the hidden rows times that expert's W2."""
+    rng = _rng(42)
+    d, F, E = 10, 14, 3
+    seg = [0, 3, 3, 7]
+    x = rng.standard_normal((7, d))
+    w1 = rng.standard_normal((E, d, F)) * 0.4
+    w3 = rng.standard_normal((E, d, F)) * 0.4
+    w2 = rng.standard_normal((E, F, d)) * 0.4
+    lin = lambda a, w: Fn.linear(torch.from_numpy(a), torch.from_numpy(w.T.copy()))  # noqa: E731
+    for act in ("gelu", "swiglu"):
+        h = o.expert_hidden(x, seg, w1, w3 if act == "swiglu" else None, act)
+        assert h.shape == (7, F)
+        for e, (a, b) in enumerate(zip(seg[:-1], seg[1:])):
+            if b == a:
+                continue
+            z = lin(x[a:b], w1[e])
+            ref = Fn.gelu(z, approximate="none") if act == "gelu" else Fn.silu(z) * lin(x[a:b], w3[e])
+            assert np.allclose(h[a:b], ref.numpy(), rtol=1e-12, atol=1e-12), (act, e)
+            y = o.expert_ffn(x, seg, w1, w3 if act == "swiglu" else None, w2, act)
+            assert np.allclose(y[a:b], lin(np.ascontiguousarray(h[a:b]), w2[e]).numpy(),
+                               rtol=1e-12, atol=1e-12)
+
+
 def _dense_dispatch_reference(x, idx, w, kept_mask, w1, w3, w2, act):
     """The dispatch-mask / combine-weight formulation: every expert runs on
     every token (torch fp64), and a dense [T, E] combine weight picks and
@@ -625,5 +652,5 @@ def pin_near_tie(o):
 
 ALL_PINS.extend([pin_philox_kat, pin_jitter, pin_logit_noise, pin_z_loss, pin_route_noise,
                  pin_temperature, pin_route_backward_finite_differences,
-                 pin_route_backward_identities, pin_near_tie])
+                 pin_route_backward_identities, pin_near_tie, pin_expert_hidden_segments])
 

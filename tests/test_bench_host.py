@@ -71,3 +71,48 @@ def test_traffic_record_matches_source_hash():
     else:
         assert t is None                     # a changed kernel reports no stale traffic
     assert bench.measured_traffic("grouped_gemm_tc_swiglu", "no_such_workload") is None
+
+
+def test_reference_arm_never_loads_the_library_and_shares_the_config():
+    """The reference arm (the CPU oracle) runs in a process that maps no
+    library .so of this repository, and prints the config the GPU arm prints
+    for the same flags."""
+    import json
+    import subprocess
+    code = (
+        "import sys, json, io, contextlib\n"
+        "sys.argv = ['bench.py', '--impl', 'reference', '--config', 'tiny_fp32', '--steps', '1',"
+        " '--warmup', '0']\n"
+        "import bench\n"
+        "buf = io.StringIO()\n"
+        "with contextlib.redirect_stdout(buf):\n"
+        "    bench.main()\n"
+        "maps = open('/proc/self/maps').read()\n"
+        "print(json.dumps({'line': json.loads(buf.getvalue().strip().splitlines()[-1]),"
+        " 'pkg': 'mixture_experts_routing_route_b200' in sys.modules,"
+        " 'so': 'libmoe_b200' in maps}))\n")
+    res = subprocess.run([sys.executable, "-c", code], cwd=bench.ROOT, capture_output=True, text=True,
+                         timeout=300)
+    assert res.returncode == 0, res.stderr[-2000:]
+    got = json.loads(res.stdout.strip().splitlines()[-1])
+    assert not got["pkg"] and not got["so"]
+    line = got["line"]
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s"
+    args = _args(config="tiny_fp32")
+    assert line["config"] == json.loads(json.dumps(bench.arm_config(bench.shape_of(args), args, 1)))
+
+
+def test_stage_roofline_and_dispatch_span():
+    sh = CONFIGS["mixtral"]
+    args = _args()
+    alg = bench.algorithmic(sh, [1024] * 8)
+    stage_ms = {"route": 0.0201, "permute": 0.0103, "gather": 0.0226, "ffn_up": 1.5, "ffn_down": 0.85,
+                "combine": 0.019}
+    peaks = {"hbm_gbs": 6546.9, "bf16_tflops": 1676.5}
+    roof = bench.stage_roofline(sh, stage_ms, alg, peaks, 1676.5, args)
+    assert abs(roof["route"]["GB_s"] - alg["route"]["bytes"] / 20.1e-6 / 1e9) < 1e-6
+    assert abs(roof["ffn_up"]["tensor_frac"] - alg["ffn_up"]["flops"] / 1.5e-3 / 1e12 / 1676.5) < 1e-12
+    span = bench.dispatch_span_of(stage_ms, alg, peaks)
+    byts = alg["route"]["bytes"] + alg["permute"]["bytes"] + alg["gather"]["bytes"]
+    assert abs(span["us"] - 53.0) < 1e-9
+    assert abs(span["hbm_frac"] - byts / 53.0e-6 / 1e9 / 6546.9) < 1e-12

@@ -1,8 +1,19 @@
 """GPU parity at the workloads' full sizes, in the launch configuration
-bench.py times (MoeLayer.forward -> moe_forward). Route and permute are
-checked on every token / slot; the layer output on a seeded sample of tokens
-that the oracle evaluates one by one (each sampled token's kept slots through
-its experts' MLPs), plus every token whose slots were all dropped."""
+bench.py times (MoeLayer.forward -> moe_forward).
+
+* Route and permute on every token and slot.
+* The gathered rows x_perm: every row an exact copy of its token.
+* The layer output: every token for the T = 4096 and T = 16384 workloads; for
+  the T = 32768 workloads, 4096 seeded tokens that the oracle evaluates one by
+  one (each sampled token's kept slots through its experts' MLPs), plus every
+  token whose slots were all dropped (exact zeros).
+* The hidden rows h and the expert outputs y_perm stage-chained: for the
+  largest and the smallest non-empty expert, every row of h against the
+  oracle's hidden rows of the GPU's x_perm, and every row of y_perm against
+  the oracle's MLP of those rows.
+
+The float stages run on the GPU's routing (verified first): in a capacity
+workload one flipped near tie would shift later arrival ranks."""
 import numpy as np
 import pytest
 import torch
@@ -14,7 +25,42 @@ from tests.gpu_helpers import (check_topk_end_to_end, TOL_AUX_REL, TOL_BF16_OUT,
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
-N_SAMPLE = 48
+ALL_TOKENS = ("mixtral", "fine_grained", "capacity_skew")
+N_SAMPLE = 4096  # tokens of the T = 32768 workloads the oracle evaluates
+
+
+def _check_expert_rows(v, pm, inp, sh):
+    """h and y_perm of the largest and the smallest non-empty expert, every
+    row, from the GPU's own x_perm (stage-chained)."""
+    seg = pm["seg_offsets"].astype(np.int64)
+    sizes = np.diff(seg)
+    live = np.nonzero(sizes > 0)[0]
+    experts = sorted({int(live[np.argmax(sizes[live])]), int(live[np.argmin(sizes[live])])})
+    w1 = ExpertWeights(inp.w1)
+    w3 = None if inp.w3 is None else ExpertWeights(inp.w3)
+    w2 = ExpertWeights(inp.w2)
+    for e in experts:
+        a, b = int(seg[e]), int(seg[e + 1])
+        xe = np32(v["x_perm"][a:b])
+        one = [0, b - a]
+        pick = lambda w: None if w is None else _One(w, e)  # noqa: E731
+        h_ref = O.expert_hidden(xe, one, pick(w1), pick(w3), sh.act)
+        h_got = np32(v["h"][a:b])
+        assert max_err_ratio(h_got, h_ref) <= TOL_BF16_OUT, ("h", e)
+        y_ref = O.expert_ffn(xe, one, pick(w1), pick(w3), pick(w2), sh.act)
+        assert max_err_ratio(np32(v["y_perm"][a:b]), y_ref) <= TOL_BF16_OUT, ("y_perm", e)
+    return experts
+
+
+class _One:
+    """Expert e of an [E, r, c] weight seen as a one-expert list."""
+
+    def __init__(self, w, e):
+        self.w, self.e = w, e
+
+    def __getitem__(self, i):
+        assert i == 0
+        return self.w[self.e]
 
 
 @pytest.mark.parametrize("name", ["mixtral", "fine_grained", "capacity_skew", "long_skewed",
@@ -33,7 +79,8 @@ def test_full_size(name):
     T, k, E = sh.T, sh.k, sh.E
 
     x = np32(inp.x)
-    r = O.route(x, np32(inp.wg), None if inp.bias is None else inp.bias.numpy(), k)
+    bias = None if inp.bias is None else inp.bias.numpy()
+    r = O.route(x, np32(inp.wg), bias, k)
     g_idx = npi(v["topk_idx"]).astype(np.int64)
     check_topk_end_to_end(g_idx, r)
     w_ref = O.renormalise(r["probs64"], g_idx)
@@ -48,26 +95,31 @@ def test_full_size(name):
     assert np.array_equal(npi(v["drop"]), pm["drop"])
     assert np.array_equal(npi(v["row_slot"])[:pm["rows"]], pm["row_slot"])
 
-    rng = np.random.default_rng(sh.seed)
-    sample = np.sort(rng.choice(T, size=min(N_SAMPLE, T), replace=False))
-    all_dropped = np.nonzero(pm["drop"].reshape(T, k).all(axis=1))[0]
+    # every gathered row is an exact copy of its token's row
+    R = pm["rows"]
+    xp = np32(v["x_perm"][:R])
+    assert np.array_equal(xp, x[pm["row_slot"].astype(np.int64) // k])
+    del xp
+
     got = np32(out)
+    all_dropped = np.nonzero(pm["drop"].reshape(T, k).all(axis=1))[0]
     if len(all_dropped):
         assert np.all(got[all_dropped] == 0.0)
-    # gathered rows of the sampled tokens are exact copies (where a forward
-    # keeps x_perm; the bf16 forward gathers inside the up projection)
-    if v["x_perm"] is not None:
-        rows = pm["slot_to_row"].reshape(T, k)[sample]
-        xp = np32(v["x_perm"])
-        for i, t in enumerate(sample):
-            for rr in rows[i]:
-                if rr >= 0:
-                    assert np.array_equal(xp[rr], x[t])
-    ref = O.forward_tokens(x, sample, g_idx, w_ref, pm["slot_to_row"], ExpertWeights(inp.w1),
-                           None if inp.w3 is None else ExpertWeights(inp.w3),
-                           ExpertWeights(inp.w2), sh.act)
-    err = max_err_ratio(got[sample], ref)
+
+    W = lambda w: None if w is None else ExpertWeights(w)  # noqa: E731
+    if name in ALL_TOKENS:
+        ref = O.forward(x, np32(inp.wg), bias, W(inp.w1), W(inp.w3), W(inp.w2), k, sh.act, sh.cf,
+                        topk_idx=g_idx, topk_w=w_ref)["out"]
+        err = max_err_ratio(got, ref)
+    else:
+        rng = np.random.default_rng(sh.seed)
+        sample = np.sort(rng.choice(T, size=min(N_SAMPLE, T), replace=False))
+        ref = O.forward_tokens(x, sample, g_idx, w_ref, pm["slot_to_row"], W(inp.w1), W(inp.w3),
+                               W(inp.w2), sh.act)
+        err = max_err_ratio(got[sample], ref)
     assert err <= TOL_BF16_OUT, err
+
+    _check_expert_rows(v, pm, inp, sh)
 
 
 @pytest.mark.parametrize("name", ["mixtral", "long_skewed_cf"])
