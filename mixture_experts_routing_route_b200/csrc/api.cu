@@ -201,7 +201,8 @@ moe_status_t run_forward(const moe_layer_t* L, const void* x, int T, void* out, 
                                         g ? f.row_slot : nullptr, L->k, L->w1, L->w3, L->w2,
                                         L->act, f.rows_max, L->d, L->F, L->E, f.seg,
                                         binned(L) ? f.kept : nullptr, f.h, f.y_perm, f.ctl, s,
-                                        after_up, cig ? &co : nullptr)));
+                                        after_up, cig ? &co : nullptr,
+                                        static_cast<int64_t>(T) * L->k)));
   } else {
     MOE_CHECK(from_cuda(launch_ffn_f32(static_cast<const float*>(f.x_perm),
                                        static_cast<const float*>(L->w1),

@@ -177,11 +177,14 @@ struct CombineOut {
   void* out;                // [T, d] layer output
   int T;
 };
+// slots: rows the permute distributes over the experts (T * k), which picks
+// the single-CTA or the CTA-pair kernel; negative: rows_max.
 cudaError_t launch_ffn_bf16(const void* a, int64_t a_rows, const int32_t* row_slot, int k,
                             const void* w1, const void* w3, const void* w2, moe_act_t act,
                             int64_t rows_max, int d, int F, int E, const int32_t* seg,
                             const int32_t* kept, void* h, void* y, Control* ctl, cudaStream_t s,
-                            cudaEvent_t after_up, const CombineOut* comb = nullptr);
+                            cudaEvent_t after_up, const CombineOut* comb = nullptr,
+                            int64_t slots = -1);
 cudaError_t launch_ffn_f32(const float* x_perm, const float* w1, const float* w3, const float* w2,
                            moe_act_t act, int64_t rows_max, int d, int F, int E,
                            const int32_t* seg, float* h, float* y, Control* ctl, cudaStream_t s,

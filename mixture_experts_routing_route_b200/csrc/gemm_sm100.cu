@@ -65,7 +65,12 @@ struct GemmArgs {
   Control* ctl;
 };
 
-__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+// silu(g) = g / (1 + e^-g) with the hardware exponential and reciprocal
+// (CUDA's __expf and __fdividef intrinsics, a few ulp of fp32): the result is
+// rounded to bf16 (2^-9 relative), so their error never shows, and the
+// epilogue of the up projection runs in the tensor cores' shadow. For
+// g < -88 the exponential overflows and __fdividef returns 0, the limit.
+__device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 __device__ __forceinline__ float gelu_erf(float z) {
   return 0.5f * z * (1.0f + erff(z * 0.70710678118654752440f));
 }
@@ -530,6 +535,244 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   }
 }
 
+// ============================================================ CTA-pair kernel
+// The same grouped GEMM on tile pairs (cta_group::2): the two CTAs of a
+// cluster compute one 256-row x NMMA tile together. CTA r loads A rows
+// [row0 + 128 r, +128) and its half of the B columns (for SwiGLU: CTA 0 the
+// W_gate box(es), CTA 1 the W_up box(es) of the same output columns) into a
+// 6-stage ring of 32 KB; the even CTA issues M = 256 MMAs that read both CTAs'
+// operands and write each CTA's 128 rows (all NMMA columns) into that CTA's
+// tensor memory, so both epilogues see gate and up side by side as before.
+// Per k-block an SM moves 32 KB into shared memory instead of 48 KB for the
+// same tensor work: the fill bandwidth, not the tensor core, bounds the
+// single-CTA kernel.
+//
+// Barriers: full[s] lives in the even CTA, armed there with both CTAs' bytes;
+// both CTAs' TMA loads count their bytes on it (the cta_group::2 TMA form).
+// empty[s] and tfull[acc] live in both CTAs; the MMA commits arrive on both
+// (multicast). tempty[acc] lives in the even CTA and counts the 8 epilogue
+// warps of the pair. Every wait is bounded; a time-out sets
+// MOE_DEVERR_TIMEOUT and unwinds; the peer notices through its own bounded
+// waits. Both CTAs meet at two cluster barriers only: after set-up and before
+// tensor memory is freed, reached on every path.
+constexpr int kPairStages = 6;
+constexpr int kPairRows = 256;
+
+template <int EPI>
+struct PairCfg {
+  static constexpr int NMMA = 256;
+  static constexpr int A_BYTES = 128 * BK * 2;           // this CTA's 128 rows
+  static constexpr int B_BYTES = BK * (NMMA / 2) * 2;     // this CTA's half of the columns
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // 32 KB
+  static constexpr int OUT_N = EPI == EPI_SWIGLU ? NMMA / 2 : NMMA;
+  static constexpr int TMEM_COLS = 2 * NMMA;
+  static constexpr size_t STAGING = 4 * kStageWarpBytes;
+  static constexpr size_t SMEM = static_cast<size_t>(kPairStages) * STAGE_BYTES + STAGING + 1024;
+};
+
+// This CTA's B boxes of one stage. Full unit: SwiGLU CTA 0 loads W_gate
+// columns [n0, n0 + 128), CTA 1 the same W_up columns; otherwise CTA r loads
+// columns [n0 + 128 r, +128). Half-width unit: one 64-column box each, W_gate
+// / W_up at n0 (SwiGLU) or [n0 + 64 r, +64).
+template <int EPI>
+__device__ __forceinline__ void load_b_pair(uint8_t* sb, const CUtensorMap* b0, const CUtensorMap* b1,
+                                            uint32_t bar, int n0, int brow, uint32_t rank, bool half) {
+  if constexpr (EPI == EPI_SWIGLU) {
+    const CUtensorMap* m = rank == 0 ? b0 : b1;
+    tma_load_2d_pair(sb, m, bar, n0, brow);
+    if (!half) tma_load_2d_pair(sb + kBoxBytes, m, bar, n0 + 64, brow);
+  } else {
+    if (half) {
+      tma_load_2d_pair(sb, b0, bar, n0 + 64 * static_cast<int>(rank), brow);
+    } else {
+      const int c = n0 + 128 * static_cast<int>(rank);
+      tma_load_2d_pair(sb, b0, bar, c, brow);
+      tma_load_2d_pair(sb + kBoxBytes, b0, bar, c + 64, brow);
+    }
+  }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                  const __grid_constant__ CUtensorMap tmB1, GemmArgs args) {
+  pdl_begin();
+  using C = PairCfg<EPI>;
+  constexpr int NMMA = C::NMMA;
+  constexpr int STAGES_P = kPairStages;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[STAGES_P], empty_bar[STAGES_P];
+  __shared__ __align__(8) uint64_t tfull_bar[2], tempty_bar[2], drain_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int seg_s[kMaxE + 1];
+  __shared__ int cnt_s[kMaxE];
+  __shared__ int tile_start_s[kMaxE + 1];
+  __shared__ volatile int abort_s;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = args.E;
+  const uint32_t rank = cluster_ctarank();  // 0: the CTA that issues the MMAs
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+
+  for (int i = threadIdx.x; i <= E; i += kThreads) {
+    seg_s[i] = __ldg(args.seg + i);
+    if (i < E)
+      cnt_s[i] = args.kept != nullptr ? __ldg(args.kept + i) : __ldg(args.seg + i + 1) - __ldg(args.seg + i);
+  }
+  if (threadIdx.x == 0) abort_s = 0;
+  __syncthreads();
+  if (warp == 0) build_schedule<kPairRows>(args, args.N / C::OUT_N, seg_s, cnt_s, tile_start_s, lane);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES_P; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&tfull_bar[b], 1); mbar_init(&tempty_bar[b], 8); }
+    mbar_init(&drain_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc_pair(&tmem_base_s, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // barriers initialised and tensor memory allocated in both CTAs
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+  const int total_tiles = tile_start_s[E];
+  const int W = gridDim.x >> 1;  // pairs
+  const int pid = blockIdx.x >> 1;
+  const int total = num_units(total_tiles, W);
+  const int nkb = args.K / BK;
+  // the even CTA's full and tempty barriers, as shared::cluster addresses
+  const uint32_t full0 = mapa_shared(smem_u32(&full_bar[0]), 0);
+  const uint32_t tempty0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tmA);
+      prefetch_tmap(&tmB0);
+      prefetch_tmap(&tmB1);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0;  // stages that ever received a load
+      uint32_t last_parity = 0;  // parity of that stage's latest load
+      for (int u = pid; u < total && !abort_s; u += W) {
+        const Tile t = decode_unit<kPairRows, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, cnt_s, E);
+        const uint32_t tx = 2u * (C::A_BYTES + (t.half ? C::B_BYTES / 2 : C::B_BYTES));
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u)) {
+            set_error(args.ctl, MOE_DEVERR_TIMEOUT);
+            abort_s = 1;
+            break;
+          }
+          uint8_t* sa = smem + stage * C::STAGE_BYTES;
+          uint8_t* sb = sa + C::A_BYTES;
+          if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], tx);
+          const uint32_t fb = full0 + stage * 8u;
+          tma_load_2d_pair(sa, &tmA, fb, kb * BK, t.row0 + 128 * static_cast<int>(rank));
+          load_b_pair<EPI>(sb, &tmB0, &tmB1, fb, t.n0, t.e * args.K + kb * BK, rank, t.half);
+          issued_mask |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES_P) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // Every load issued must have been consumed by the MMAs (so it landed)
+      // before this CTA may leave: the MMA commit of each stage's last load
+      // arrives on empty[s] in both CTAs.
+      for (int s = 0; s < STAGES_P; ++s)
+        if (issued_mask & (1u << s)) (void)mbar_wait_bounded(&empty_bar[s], (last_parity >> s) & 1u);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t kIdescFull = make_idesc_bf16(kPairRows, NMMA);
+      constexpr uint32_t kIdescHalf = make_idesc_bf16(kPairRows, NMMA / 2);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool issued_any = false;
+      for (int u = pid; u < total && !abort_s; u += W) {
+        const Tile t = decode_unit<kPairRows, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, cnt_s, E);
+        const uint32_t idesc = t.half ? kIdescHalf : kIdescFull;
+        if (!mbar_wait_cluster_bounded(&tempty_bar[acc], acc_phase ^ 1u)) {
+          set_error(args.ctl, MOE_DEVERR_TIMEOUT);
+          abort_s = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * NMMA;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_cluster_bounded(&full_bar[stage], phase)) {
+            set_error(args.ctl, MOE_DEVERR_TIMEOUT);
+            abort_s = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t adesc = make_sw128_desc(a_addr + kk * 32, 16, 1024);
+            const uint64_t bdesc = make_sw128_desc(b_addr + kk * 2048, kBoxBytes, 1024);
+            umma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          issued_any = true;
+          umma_commit_pair_mc(&empty_bar[stage], 0x3);
+          if (++stage == STAGES_P) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit_pair_mc(&tfull_bar[acc], 0x3);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (issued_any) {
+        // Tensor memory is freed below: wait until every MMA issued is done.
+        umma_commit_pair_mc(&drain_bar, 0x1);
+        (void)mbar_wait_bounded(&drain_bar, 0);
+      }
+    }
+  } else {
+    // epilogue warps 2..5: TMEM lane quarter = warp % 4 of this CTA's 128 rows
+    const int q = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = pid; u < total; u += W) {
+      int ok = 0;
+      if (lane == 0) {
+        ok = !abort_s && mbar_wait_cluster_bounded(&tfull_bar[acc], acc_phase);
+        if (!ok && !abort_s) {
+          set_error(args.ctl, MOE_DEVERR_TIMEOUT);
+          abort_s = 1;
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      const Tile t = decode_unit<kPairRows, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, cnt_s, E);
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * NMMA;
+      {
+        uint8_t* buf = smem + STAGES_P * C::STAGE_BYTES + q * kStageWarpBytes;
+        const int crow = 128 * static_cast<int>(rank) + q * 32;  // first row of this warp in the tile
+        const int nrows = max(0, min(32, t.rows - crow));
+        if (t.half)
+          epilogue_staged<EPI, C::OUT_N / 2>(tbase, buf, args, t.row0 + crow, nrows, args.N, t.n0, lane);
+        else
+          epilogue_staged<EPI, C::OUT_N>(tbase, buf, args, t.row0 + crow, nrows, args.N, t.n0, lane);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty0 + acc * 8u);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no peer still reads or signals this CTA; every MMA is done
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
 // ----------------------------------------------------------------- host side
 }  // namespace
 
@@ -593,11 +836,62 @@ cudaError_t run_gemm(const void* A, int64_t a_rows, const int32_t* row_slot, int
   return launch_pdl(kern, dim3(num_sms()), dim3(kThreads), C::SMEM, s, false, ta, tb0, tb1, a);
 }
 
+// The CTA-pair kernel, for NMMA = 256. Each CTA's A box is 128 rows.
+template <int EPI>
+cudaError_t run_gemm_pair(const void* A, int64_t a_rows, const int32_t* row_slot, int k,
+                          const void* B0, const void* B1, int64_t rows_max, int K, int N, int E,
+                          const int32_t* seg, const int32_t* kept, void* out, Control* ctl,
+                          cudaStream_t s, const float* comb_w = nullptr, long long slots = 0) {
+  using C = PairCfg<EPI>;
+  CUtensorMap ta, tb0, tb1;
+  if (!make_tma_2d_bf16(&ta, A, static_cast<uint64_t>(a_rows), K, 128)) return cudaErrorInvalidValue;
+  if (!make_tma_2d_bf16(&tb0, B0, static_cast<uint64_t>(E) * K, N, BK)) return cudaErrorInvalidValue;
+  if (!make_tma_2d_bf16(&tb1, B1 ? B1 : B0, static_cast<uint64_t>(E) * K, N, BK)) return cudaErrorInvalidValue;
+  GemmArgs a;
+  a.seg = seg;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.row_slot = row_slot;
+  a.kept = kept;
+  a.k = k;
+  a.E = E;
+  a.K = K;
+  a.N = N;
+  a.rows_max = rows_max;
+  a.comb_w = comb_w;
+  a.slots = slots;
+  a.ctl = ctl;
+  auto kern = grouped_gemm_pair<EPI>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM));
+  const int pairs = num_sms() / 2;
+  return launch_pdl_cluster(kern, dim3(2 * pairs), dim3(kThreads), C::SMEM, s, 2, ta, tb0, tb1, a);
+}
+
+// Experts averaging at least this many rows run on CTA pairs (256-row tiles):
+// below it the 256-row tile's padding costs more than the pair saves. The
+// average is taken over the slots the permute distributes (T * k for a layer
+// forward, whatever the row layout), so the dense and the binned layouts pick
+// the same kernel. Measured on B200 (event medians, L2 evicted): at 1024 rows
+// per expert the pair takes the down projection from 884 to 783 us and the up
+// projection from 1528 to 1505 us; on a Zipf-skewed layer with 512 slots per
+// expert and capacity 512 it is slower (up 90 vs 70 us, down 57 vs 45 us).
+constexpr int64_t kPairMinRowsPerExpert = 768;
+
+bool use_pair(int64_t slots, int E, int out_cols) {
+  return out_cols % 256 == 0 && slots >= kPairMinRowsPerExpert * E;
+}
+
 template <bool GATHER>
 cudaError_t run_up(const void* a, int64_t a_rows, const int32_t* row_slot, int k, const void* w1,
                    const void* w3, moe_act_t act, int64_t rows_max, int d, int F, int E,
                    const int32_t* seg, const int32_t* kept, void* h, Control* ctl,
-                   cudaStream_t s) {
+                   cudaStream_t s, int64_t slots) {
+  if (!GATHER && use_pair(slots, E, F)) {
+    if (act == MOE_ACT_SWIGLU)
+      return run_gemm_pair<EPI_SWIGLU>(a, a_rows, nullptr, k, w1, w3, rows_max, d, F, E, seg, kept, h,
+                                       ctl, s);
+    return run_gemm_pair<EPI_GELU>(a, a_rows, nullptr, k, w1, nullptr, rows_max, d, F, E, seg, kept, h,
+                                   ctl, s);
+  }
   if (act == MOE_ACT_SWIGLU)
     return run_gemm<EPI_SWIGLU, 256, GATHER>(a, a_rows, row_slot, k, w1, w3, rows_max, d, F, E, seg,
                                              kept, h, ctl, s);
@@ -614,27 +908,35 @@ cudaError_t launch_ffn_bf16(const void* a, int64_t a_rows, const int32_t* row_sl
                             const void* w1, const void* w3, const void* w2, moe_act_t act,
                             int64_t rows_max, int d, int F, int E, const int32_t* seg,
                             const int32_t* kept, void* h, void* y, Control* ctl, cudaStream_t s,
-                            cudaEvent_t after_up, const CombineOut* comb) {
+                            cudaEvent_t after_up, const CombineOut* comb, int64_t slots) {
+  if (slots < 0) slots = rows_max;
   if (rows_max <= 0) {
     if (after_up) cudaEventRecord(after_up, s);
     return cudaSuccess;
   }
   cudaError_t err =
       row_slot != nullptr
-          ? run_up<true>(a, a_rows, row_slot, k, w1, w3, act, rows_max, d, F, E, seg, kept, h, ctl, s)
+          ? run_up<true>(a, a_rows, row_slot, k, w1, w3, act, rows_max, d, F, E, seg, kept, h, ctl, s,
+                         slots)
           : run_up<false>(a, rows_max, nullptr, 1, w1, w3, act, rows_max, d, F, E, seg, kept, h, ctl,
-                          s);
+                          s, slots);
   if (err != cudaSuccess) return err;
   if (after_up) cudaEventRecord(after_up, s);
   if (comb != nullptr) {  // k = 1: the combine in the down projection's epilogue
-    const long long slots = static_cast<long long>(comb->T) * k;
+    const long long comb_slots = static_cast<long long>(comb->T) * k;
+    if (use_pair(slots, E, d))
+      return run_gemm_pair<EPI_COMBINE>(h, rows_max, comb->row_slot, k, w2, nullptr, rows_max, F, d, E,
+                                        seg, kept, comb->out, ctl, s, comb->w, comb_slots);
     if (d % 256 == 0)
       return run_gemm<EPI_COMBINE, 256, false>(h, rows_max, comb->row_slot, k, w2, nullptr, rows_max, F,
-                                               d, E, seg, kept, comb->out, ctl, s, comb->w, slots);
+                                               d, E, seg, kept, comb->out, ctl, s, comb->w, comb_slots);
     return run_gemm<EPI_COMBINE, 128, false>(h, rows_max, comb->row_slot, k, w2, nullptr, rows_max, F,
-                                             d, E, seg, kept, comb->out, ctl, s, comb->w, slots);
+                                             d, E, seg, kept, comb->out, ctl, s, comb->w, comb_slots);
   }
-  if (d % 256 == 0)
+  if (use_pair(slots, E, d))
+    err = run_gemm_pair<EPI_STORE>(h, rows_max, nullptr, 1, w2, nullptr, rows_max, F, d, E, seg, kept,
+                                   y, ctl, s);
+  else if (d % 256 == 0)
     err = run_gemm<EPI_STORE, 256, false>(h, rows_max, nullptr, 1, w2, nullptr, rows_max, F, d, E,
                                           seg, kept, y, ctl, s);
   else

@@ -31,6 +31,10 @@ CASES = {
     "expert0_skew_cf": (900, 256, 8, 2, 256, "swiglu", "bf16", 1.25, "expert0"),
     "f32_swiglu": (200, 64, 6, 2, 96, "swiglu", "f32", 0.0, "none"),
     "f32_gelu_capacity": (256, 64, 4, 1, 128, "gelu", "f32", 1.25, "none"),
+    # >= 768 slots per expert: the CTA-pair grouped GEMM (256-row tiles)
+    "pair_gelu_capacity_zipf": (3200, 256, 8, 2, 512, "gelu", "bf16", 1.25, "zipf"),
+    "pair_swiglu_skew_cf": (1600, 256, 4, 2, 256, "swiglu", "bf16", 1.0, "expert0"),
+    "pair_swiglu_dropless": (1600, 512, 4, 2, 768, "swiglu", "bf16", 0.0, "none"),
 }
 
 
@@ -201,6 +205,8 @@ def test_layer_binned(T, d, E, k, F, act, dt, cf, bias):
     (1000, 256, 16, 512, "gelu", 1.0, "zipf", False, True),       # gather in the up projection too
     (333, 384, 8, 384, "gelu", 0.0, "none", False, False),        # d % 256 != 0: 128-column tiles
     (300, 256, 8, 256, "swiglu", 0.02, "none", False, False),     # C = 0: every token dropped
+    (3200, 256, 4, 256, "swiglu", 0.0, "none", False, False),     # CTA-pair GEMMs, dropless
+    (3200, 256, 4, 512, "gelu", 1.0, "expert0", True, False),     # CTA pairs, bucket layout, drops
 ])
 def test_layer_combine_in_gemm(T, d, E, F, act, cf, bias, binned, gig):
     """k = 1: the combine in the down projection's epilogue

@@ -226,6 +226,50 @@ def test_expert_ffn_segment_boundaries(act, d, F):
     assert np.all(np32(y)[seg[-1]:] == sentinel) and np.all(np32(h)[seg[-1]:] == sentinel)
 
 
+@pytest.mark.parametrize("act,d,F,m", [
+    ("swiglu", 256, 256, [0, 1, 127, 128, 129, 255, 256, 257, 383, 384, 385, 600, 1000]),
+    ("gelu", 512, 256, [0, 1, 127, 128, 129, 255, 256, 257, 383, 384, 385, 600, 1000]),
+    ("swiglu", 256, 256, [1, 200, 256, 300, 700]),   # few tiles: half-width gate/up units
+    ("gelu", 256, 512, [513, 0, 64, 1024]),
+])
+def test_expert_ffn_pair_tiles(act, d, F, m):
+    """Row counts that select the CTA-pair kernel (256-row tiles, each CTA
+    128 rows): segments on both sides of 128 (the second CTA has no valid
+    rows) and 256, empty experts, a last wave split into half-width units,
+    and slack rows past the last segment that are never written."""
+    E = len(m)
+    seg = np.concatenate([[0], np.cumsum(m)]).astype(np.int32)
+    R = max(int(seg[-1]) + 77, 768 * E + 1)  # enough rows for the pair kernel
+    g = torch.Generator().manual_seed(d + F + E)
+    x = torch.randn(R, d, generator=g).to(torch.bfloat16)
+    w1 = (torch.randn(E, d, F, generator=g) * 0.05).to(torch.bfloat16)
+    w3 = (torch.randn(E, d, F, generator=g) * 0.05).to(torch.bfloat16) if act == "swiglu" else None
+    w2 = (torch.randn(E, F, d, generator=g) * 0.05).to(torch.bfloat16)
+    sentinel = -3.0
+    h = torch.full((R, F), sentinel, dtype=torch.bfloat16, device=DEV)
+    y = torch.full((R, d), sentinel, dtype=torch.bfloat16, device=DEV)
+    ws = new_ws(256)
+    code = abi.MOE_ACT_SWIGLU if act == "swiglu" else abi.MOE_ACT_GELU
+    abi.moe_expert_ffn(x.to(DEV), w1.to(DEV), None if w3 is None else w3.to(DEV), w2.to(DEV), code,
+                       R, d, F, E, torch.from_numpy(seg).to(DEV), h, y, ws)
+    torch.cuda.synchronize()
+    assert abi.moe_get_device_error(ws) == 0
+    xs = np32(x)
+    W1, W2 = ExpertWeights(w1), ExpertWeights(w2)
+    W3 = ExpertWeights(w3) if w3 is not None else None
+    n = int(seg[-1])
+    h_ref = O.expert_hidden(xs[:n], seg, W1, W3, act)
+    assert max_err_ratio(np32(h)[:n], h_ref) <= TOL_BF16_OUT
+    y_ref = O.expert_ffn(xs[:n], seg, W1, W3, W2, act)
+    assert max_err_ratio(np32(y)[:n], y_ref) <= TOL_BF16_OUT
+    # every expert's rows, not only the largest values
+    for e in range(E):
+        a, b = int(seg[e]), int(seg[e + 1])
+        if b > a:
+            assert max_err_ratio(np32(y)[a:b], y_ref[a:b]) <= TOL_BF16_OUT, e
+    assert np.all(np32(y)[n:] == sentinel) and np.all(np32(h)[n:] == sentinel)
+
+
 @pytest.mark.parametrize("act,T,d,E,k,F,cf", [("swiglu", 700, 256, 8, 2, 512, 0.0),
                                              ("gelu", 555, 384, 16, 2, 384, 1.0),
                                              ("swiglu", 300, 256, 64, 8, 256, 0.0)])
