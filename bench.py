@@ -710,8 +710,8 @@ def main():
 
     dom = "ffn_up"
     tf = alg[dom]["flops"] / (up_ms * 1e-3) / 1e12 if up_ms > 0 else None
-    traffic = measured_traffic("grouped_gemm_tc_swiglu", sh.name)
-    roofline = {"kernel": "grouped_gemm_tc<SwiGLU> (expert up/gate projection)",
+    traffic = measured_traffic("grouped_gemm_up_swiglu", sh.name)
+    roofline = {"kernel": "grouped GEMM, SwiGLU up/gate projection (CTA pairs for experts of >= 768 rows)",
                 "bound": "tensor", "achieved": tf, "peak": tc_peak,
                 "unit": "TFLOP/s", "frac": tf / tc_peak if tf else None,
                 "traffic": traffic,

@@ -65,12 +65,12 @@ def test_traffic_record_matches_source_hash():
             parts = line.split()
             if parts and not line.startswith("#"):
                 rec[(parts[0], parts[1])] = (int(parts[2]), parts[3])
-    t = bench.measured_traffic("grouped_gemm_tc_swiglu", "mixtral")
-    if rec[("grouped_gemm_tc_swiglu", "mixtral")][1] == h:
-        assert t == rec[("grouped_gemm_tc_swiglu", "mixtral")][0]
+    t = bench.measured_traffic("grouped_gemm_up_swiglu", "mixtral")
+    if rec[("grouped_gemm_up_swiglu", "mixtral")][1] == h:
+        assert t == rec[("grouped_gemm_up_swiglu", "mixtral")][0]
     else:
         assert t is None                     # a changed kernel reports no stale traffic
-    assert bench.measured_traffic("grouped_gemm_tc_swiglu", "no_such_workload") is None
+    assert bench.measured_traffic("grouped_gemm_up_swiglu", "no_such_workload") is None
 
 
 def test_reference_arm_never_loads_the_library_and_shares_the_config():
