@@ -379,6 +379,55 @@ MOE_API moe_status_t moe_permute_noalloc(const int32_t* topk_idx, int T, int k, 
                                          int32_t* kept_counts, int32_t* seg_offsets,
                                          uint32_t* device_error, moe_stream_t stream);
 
+/* ------------------------------------------------ expert-parallel dispatch
+ * Plans for running the experts on several ranks ("MoE Router: who decides
+ * which expert a token goes to": per-device send counts with
+ * device = expert / experts_per_device, an all-to-all-v with per-pair counts
+ * and displacements, the experts computed where they live; "ops-transformer
+ * MoE operators", 坑2: tokens go to the cards holding their experts and come
+ * back after the compute; "Integrating MoE into your model with Colossal-AI",
+ * step 2: all-to-all to the expert's GPU, expert MLP, all-to-all back).
+ * Experts are owned in contiguous blocks: rank g holds experts
+ * [g*E/world, (g+1)*E/world). Each rank routes, permutes (its own capacity)
+ * and gathers its own tokens as on one GPU; because the gathered rows are
+ * sorted by expert, the rows for rank g are one contiguous range of x_perm.
+ * The exchanges are the caller's (e.g. NCCL all-to-all-v); these calls only
+ * plan them. A layer computed this way gives each rank exactly the output of
+ * moe_forward on its own tokens.
+ *
+ * Send plan: send_rows[g] = rows of x_perm for rank g (the kept counts of
+ * g's experts summed), send_offsets[g] = its first row (seg_offsets of g's
+ * first expert); send_offsets[world] = seg_offsets[E]. The per-expert counts
+ * the receiver needs are kept_counts itself: its slice
+ * [g*E/world, (g+1)*E/world) goes to rank g.
+ *   kept_counts [E], seg_offsets [E+1] (moe_permute's outputs, device)
+ *   send_rows [world], send_offsets [world+1] (device, out)
+ *   ws >= 256 bytes (control block; a negative count sets MOE_DEVERR_ROW_RANGE)
+ * E in [1, 256] and a multiple of world, else MOE_ERR_INVALID. */
+MOE_API moe_status_t moe_ep_send_plan(const int32_t* kept_counts, const int32_t* seg_offsets, int E,
+                                      int world, int32_t* send_rows, int32_t* send_offsets,
+                                      void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Receive plan. recv_counts [world][experts_per_rank] (device): from each
+ * source rank, its kept counts for this rank's experts, as received. Rows
+ * arrive source-major (source 0's rows in expert order, then source 1's ...).
+ *   recv_rows [world], recv_offsets [world+1]: rows from each source and
+ *     where they start in the received buffer
+ *   local_seg [experts_per_rank+1]: expert-major segment offsets (for local
+ *     expert e: source 0's rows, then source 1's ...), for moe_expert_ffn
+ *   local_to_recv [rows]: received row of each expert-major row (gather the
+ *     received rows into expert-major order with moe_gather, k = 1)
+ *   recv_to_local [rows]: the inverse (gather the expert outputs back into
+ *     received order before the return exchange)
+ *   rows_cap: capacity of the two maps; a total above it sets
+ *     MOE_DEVERR_ROW_RANGE in ws and writes no map
+ * world * experts_per_rank <= 256. */
+MOE_API moe_status_t moe_ep_recv_plan(const int32_t* recv_counts, int world, int experts_per_rank,
+                                      int64_t rows_cap, int32_t* recv_rows, int32_t* recv_offsets,
+                                      int32_t* local_seg, int32_t* local_to_recv,
+                                      int32_t* recv_to_local, void* ws, size_t ws_bytes,
+                                      moe_stream_t stream);
+
 /* ----------------------------------------------------------------- gather
  * x_perm[r] = x[row_slot[r] / k] for r < seg_offsets[E] ("MegaBlocks",
  * section 4.3, binned_gather in compact form), moved row by row with bulk

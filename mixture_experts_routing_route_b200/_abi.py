@@ -97,6 +97,10 @@ _SIGS = {
                                c_size_t, c_void_p]),
     "moe_combine": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int64,
                             c_void_p, c_void_p, c_size_t, c_void_p]),
+    "moe_ep_send_plan": (c_int, [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p,
+                                 c_size_t, c_void_p]),
+    "moe_ep_recv_plan": (c_int, [c_void_p, c_int, c_int, c_int64, c_void_p, c_void_p, c_void_p,
+                                 c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "moe_forward_workspace_size": (c_size_t, [ctypes.POINTER(MoeLayerC), c_int]),
     "moe_forward_host_workspace_size": (c_size_t, [ctypes.POINTER(MoeLayerC), c_int]),
     "moe_forward": (c_int, [ctypes.POINTER(MoeLayerC), c_void_p, c_int, c_void_p, c_void_p,
@@ -276,6 +280,19 @@ def moe_combine(y_perm, topk_w, slot_to_row, T, d, k, rows_max, out, ws, stream=
     _check("moe_combine", _lib.moe_combine(
         _ptr(y_perm), _ptr(topk_w), _ptr(slot_to_row), dtype_code(out.dtype), T, d, k,
         int(rows_max), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_ep_send_plan(kept_counts, seg_offsets, E, world, send_rows, send_offsets, ws, stream=None):
+    _check("moe_ep_send_plan", _lib.moe_ep_send_plan(
+        _ptr(kept_counts), _ptr(seg_offsets), E, world, _ptr(send_rows), _ptr(send_offsets), _ptr(ws),
+        ws.numel(), _stream(stream)))
+
+
+def moe_ep_recv_plan(recv_counts, world, experts_per_rank, rows_cap, recv_rows, recv_offsets, local_seg,
+                     local_to_recv, recv_to_local, ws, stream=None):
+    _check("moe_ep_recv_plan", _lib.moe_ep_recv_plan(
+        _ptr(recv_counts), world, experts_per_rank, int(rows_cap), _ptr(recv_rows), _ptr(recv_offsets),
+        _ptr(local_seg), _ptr(local_to_recv), _ptr(recv_to_local), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def layer_struct(d, E, k, F, dtype, act, cf, w_router, bias, w1, w3, w2, flags=0,

@@ -514,6 +514,44 @@ moe_status_t moe_combine(const void* y_perm, const float* topk_w, const int32_t*
                                   static_cast<Control*>(ws), reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status_t moe_ep_send_plan(const int32_t* kept_counts, const int32_t* seg_offsets, int E,
+                              int world, int32_t* send_rows, int32_t* send_offsets, void* ws,
+                              size_t ws_bytes, moe_stream_t stream) {
+  if (E < 1 || E > 256 || world < 1 || E % world != 0) return MOE_ERR_INVALID;
+  MOE_NEED(kept_counts);
+  MOE_NEED(seg_offsets);
+  MOE_NEED(send_rows);
+  MOE_NEED(send_offsets);
+  MOE_NEED(ws);
+  if (ws_bytes < sizeof(Control)) return MOE_ERR_WORKSPACE;
+  return from_cuda(launch_ep_send_plan(kept_counts, seg_offsets, world, E / world, send_rows,
+                                       send_offsets, static_cast<Control*>(ws),
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_ep_recv_plan(const int32_t* recv_counts, int world, int experts_per_rank,
+                              int64_t rows_cap, int32_t* recv_rows, int32_t* recv_offsets,
+                              int32_t* local_seg, int32_t* local_to_recv, int32_t* recv_to_local,
+                              void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (world < 1 || experts_per_rank < 1 || static_cast<long long>(world) * experts_per_rank > 256)
+    return MOE_ERR_INVALID;
+  if (rows_cap < 0 || rows_cap >= INT_MAX) return MOE_ERR_INVALID;
+  MOE_NEED(recv_counts);
+  MOE_NEED(recv_rows);
+  MOE_NEED(recv_offsets);
+  MOE_NEED(local_seg);
+  MOE_NEED(ws);
+  if (rows_cap > 0) {
+    MOE_NEED(local_to_recv);
+    MOE_NEED(recv_to_local);
+  }
+  if (ws_bytes < sizeof(Control)) return MOE_ERR_WORKSPACE;
+  return from_cuda(launch_ep_recv_plan(recv_counts, world, experts_per_rank, rows_cap, recv_rows,
+                                       recv_offsets, local_seg, local_to_recv, recv_to_local,
+                                       static_cast<Control*>(ws),
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t moe_forward_workspace_size(const moe_layer_t* layer, int T) {
   if (layer == nullptr || T < 0) return 0;
   return fwd_layout(layer, T, nullptr, false).bytes;

@@ -195,6 +195,16 @@ cudaError_t launch_combine(const void* y, const float* w, const int32_t* slot_to
                            int T, int d, int k, int64_t rows_max, void* out, Control* ctl,
                            cudaStream_t s);
 
+// Expert-parallel dispatch plans (ep.cu). Experts are owned in contiguous
+// blocks of e_loc per rank.
+cudaError_t launch_ep_send_plan(const int32_t* kept, const int32_t* seg, int world, int e_loc,
+                                int32_t* send_rows, int32_t* send_offsets, Control* ctl,
+                                cudaStream_t s);
+cudaError_t launch_ep_recv_plan(const int32_t* counts, int world, int e_loc, long long rows_cap,
+                                int32_t* recv_rows, int32_t* recv_offsets, int32_t* local_seg,
+                                int32_t* local_to_recv, int32_t* recv_to_local, Control* ctl,
+                                cudaStream_t s);
+
 int num_sms();
 
 // 2-D bf16 TMA map over [rows, cols] row-major, box [box_rows, 64 cols], 128-byte swizzle.

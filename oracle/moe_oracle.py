@@ -61,6 +61,7 @@ __all__ = [
     "activation", "expert_hidden", "expert_ffn", "combine", "forward", "forward_tokens",
     "permute_binned", "gather_binned", "expert_ffn_binned",
     "philox4x32_10", "jitter_multipliers", "apply_jitter", "bf16_round", "logit_noise", "z_loss",
+    "ep_send_plan", "ep_recv_plan", "ep_forward",
 ]
 
 
@@ -604,6 +605,116 @@ def forward(x, wg, bias, w1, w3, w2, k, act, cf=0.0, topk_idx=None, topk_w=None)
     y = expert_ffn(xp, pm["seg_offsets"], w1, w3, w2, act)
     out = combine(y, w, pm["slot_to_row"], T, k)
     return {"route": r, "permute": pm, "x_perm": xp, "y_perm": y, "out": out}
+
+
+# --------------------------------------------------------------------------
+# expert-parallel dispatch
+# --------------------------------------------------------------------------
+#
+# "MoE Router: who decides which expert a token goes to": the dispatch counts,
+# for every chosen expert of every token, one send to the device holding that
+# expert (device = expert / experts_per_device), then an all-to-all-v moves
+# the rows; "ops-transformer MoE operators", 坑2: the tokens are computed on
+# the cards that hold their experts and sent back; "Integrating MoE into your
+# model with Colossal-AI", step 2: all-to-all to the expert's GPU, expert
+# MLP, all-to-all back. Readings: experts are owned in contiguous blocks of
+# E / world; each rank applies the capacity to its own tokens before sending
+# (a dropped slot sends nothing); rows keep the permute's order (by expert,
+# then arrival) on the way out and come back to the same places.
+
+def ep_send_plan(idx, drop, E, world):
+    """Rows this rank sends to each rank, their start in the expert-sorted
+    gathered rows, and the per-expert counts each receiver needs (its slice
+    of the kept counts). Counted slot by slot, as the page's dispatch loop
+    does."""
+    idx = np.asarray(idx, dtype=np.int64).reshape(-1)
+    drop = np.asarray(drop, dtype=bool).reshape(-1)
+    if E % world != 0:
+        raise ValueError("E must be a multiple of world")
+    e_loc = E // world
+    send = np.zeros(world, dtype=np.int64)
+    per_expert = np.zeros(E, dtype=np.int64)
+    for s in range(len(idx)):
+        if drop[s]:
+            continue
+        send[idx[s] // e_loc] += 1
+        per_expert[idx[s]] += 1
+    offsets = np.concatenate([[0], np.cumsum(send)])
+    return {"send_rows": send, "send_offsets": offsets, "expert_counts": per_expert}
+
+
+def ep_recv_plan(recv_counts):
+    """recv_counts[src][e]: rows from rank src for this rank's local expert
+    e. Rows arrive source-major (all of src 0's rows, in expert order, then
+    src 1's). Returns the rows per source, where each source's rows start,
+    the expert-major segment offsets (for expert e: src 0's rows, then src
+    1's, ...) and the two row maps between the orders."""
+    c = np.asarray(recv_counts, dtype=np.int64)
+    world, e_loc = c.shape
+    recv_rows = c.sum(axis=1)
+    recv_offsets = np.concatenate([[0], np.cumsum(recv_rows)])
+    # position of each received row: (src, e, i) in source-major order
+    arrival = []
+    for src in range(world):
+        for e in range(e_loc):
+            for i in range(c[src, e]):
+                arrival.append((src, e, i))
+    expert_major = sorted(range(len(arrival)), key=lambda q: (arrival[q][1], arrival[q][0], arrival[q][2]))
+    local_to_recv = np.array(expert_major, dtype=np.int64)
+    recv_to_local = np.empty_like(local_to_recv)
+    recv_to_local[local_to_recv] = np.arange(len(local_to_recv))
+    local_counts = c.sum(axis=0)
+    local_seg = np.concatenate([[0], np.cumsum(local_counts)])
+    return {"recv_rows": recv_rows, "recv_offsets": recv_offsets, "local_seg": local_seg,
+            "local_to_recv": local_to_recv, "recv_to_local": recv_to_local}
+
+
+def ep_forward(x_ranks, wg, bias, w1, w3, w2, k, act, cf=0.0):
+    """The expert-parallel layer by plain message passing between the ranks'
+    lists (no collective library): each rank routes, permutes (its own
+    capacity) and gathers its own tokens; its rows for each destination rank
+    are sent; each rank computes its experts on what it received and sends
+    the outputs back, which land where the rows were; each rank combines.
+    w1 / w3 / w2 hold all E experts (rank g uses its block). Returns each
+    rank's output and route / permute results."""
+    world = len(x_ranks)
+    E = np.asarray(wg).shape[1]
+    e_loc = E // world
+    local = []
+    sent = [[None] * world for _ in range(world)]   # sent[src][dst] = rows
+    counts = [[None] * world for _ in range(world)]  # counts[src][dst] = per-local-expert counts
+    for src, x in enumerate(x_ranks):
+        x = np.asarray(x)
+        T = x.shape[0]
+        r = route(x, wg, bias, k)
+        pm = permute(r["topk_idx"], E, capacity(cf, k, T, E))
+        xp = gather(x, pm["row_slot"], k)
+        plan = ep_send_plan(r["topk_idx"], pm["drop"], E, world)
+        for dst in range(world):
+            a, b = plan["send_offsets"][dst], plan["send_offsets"][dst + 1]
+            sent[src][dst] = xp[a:b]
+            counts[src][dst] = plan["expert_counts"][dst * e_loc:(dst + 1) * e_loc]
+        local.append({"route": r, "permute": pm, "plan": plan, "T": T})
+    back = [[None] * world for _ in range(world)]  # back[dst][src] = outputs of src's rows
+    for dst in range(world):
+        rp = ep_recv_plan(np.stack([counts[src][dst] for src in range(world)]))
+        x_recv = np.concatenate([sent[src][dst] for src in range(world)], axis=0)
+        x_loc = x_recv[rp["local_to_recv"]]
+        y_loc = np.zeros((len(x_loc), np.asarray(w2[0]).shape[1]))
+        for e in range(e_loc):
+            a, b = rp["local_seg"][e], rp["local_seg"][e + 1]
+            if b > a:
+                y_loc[a:b] = _expert_mlp(x_loc[a:b], dst * e_loc + e, w1, w3, w2, act)
+        y_recv = y_loc[rp["recv_to_local"]]
+        for src in range(world):
+            a, b = rp["recv_offsets"][src], rp["recv_offsets"][src + 1]
+            back[dst][src] = y_recv[a:b]
+    outs = []
+    for src in range(world):
+        st = local[src]
+        y_perm = np.concatenate([back[dst][src] for dst in range(world)], axis=0)
+        outs.append(combine(y_perm, st["route"]["topk_w64"], st["permute"]["slot_to_row"], st["T"], k))
+    return {"out": outs, "local": local}
 
 
 def forward_tokens(x, tokens, topk_idx, topk_w, slot_to_row, w1, w3, w2, act):

@@ -650,7 +650,71 @@ def pin_near_tie(o):
     assert r["near_tie"].tolist() == want
 
 
+def pin_ep_forward_equals_each_rank_alone(o):
+    """Expert parallelism moves rows, not arithmetic: on every rank the
+    layer's output is the single-GPU forward of that rank's own tokens
+    (world 1, 2 and 4; SwiGLU and GELU; with and without capacity drops;
+    ranks with different token counts). A wrong destination, a wrong
+    regroup order or rows returned to the wrong place change some rank's
+    output."""
+    rng = _rng(51)
+    d, F = 8, 12
+    for world, E, k, act, cf in [(1, 4, 2, "swiglu", 0.0), (2, 8, 2, "swiglu", 1.0),
+                                 (4, 8, 3, "gelu", 0.0), (2, 4, 1, "gelu", 1.25), (4, 16, 2, "swiglu", 0.5)]:
+        xs = [rng.standard_normal((int(rng.integers(5, 40)), d)) for _ in range(world)]
+        wg = rng.standard_normal((d, E))
+        w1 = rng.standard_normal((E, d, F)) * 0.3
+        w3 = rng.standard_normal((E, d, F)) * 0.3 if act == "swiglu" else None
+        w2 = rng.standard_normal((E, F, d)) * 0.3
+        r = o.ep_forward(xs, wg, None, w1, w3, w2, k, act, cf)
+        for i, x in enumerate(xs):
+            ref = o.forward(x, wg, None, w1, w3, w2, k, act, cf)["out"]
+            assert np.allclose(r["out"][i], ref, rtol=1e-12, atol=1e-12), (world, E, k, act, cf, i)
+
+
+def pin_ep_plans_bruteforce(o):
+    """Send plan: rows per destination = kept slots whose expert lies in that
+    rank's block, counted by a mask over the slots; they start where the
+    permute's segment of the rank's first expert starts. Receive plan: the
+    maps are inverse permutations and expert-major row r holds, for its
+    expert, source 0's rows before source 1's, each in arrival order."""
+    rng = _rng(52)
+    for _ in range(30):
+        world = int(rng.choice([1, 2, 4]))
+        E = world * int(rng.integers(1, 4))
+        k = int(rng.integers(1, min(E, 3) + 1))
+        T = int(rng.integers(0, 30))
+        idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).reshape(T, k) if T else np.zeros((0, k), int)
+        cap = int(rng.integers(0, 6)) if rng.random() < 0.5 else None
+        pm = o.permute(idx, E, cap)
+        plan = o.ep_send_plan(idx, pm["drop"], E, world)
+        e_loc = E // world
+        flat = idx.reshape(-1)
+        keep = pm["drop"].astype(bool) == False  # noqa: E712
+        for g in range(world):
+            mask = keep & (flat >= g * e_loc) & (flat < (g + 1) * e_loc)
+            assert plan["send_rows"][g] == int(mask.sum())
+            assert plan["send_offsets"][g] == pm["seg_offsets"][g * e_loc]
+        assert plan["send_offsets"][world] == pm["seg_offsets"][E]
+        assert np.array_equal(plan["expert_counts"], pm["kept_counts"])
+        c = rng.integers(0, 5, size=(world, e_loc))
+        rp = o.ep_recv_plan(c)
+        n = int(c.sum())
+        assert sorted(rp["local_to_recv"].tolist()) == list(range(n))
+        assert np.array_equal(rp["recv_to_local"][rp["local_to_recv"]], np.arange(n))
+        tags = []  # (src, e, i) of each received row, source-major
+        for src in range(world):
+            for e in range(e_loc):
+                tags += [(src, e, i) for i in range(c[src, e])]
+        got = [tags[q] for q in rp["local_to_recv"]]
+        want = [(src, e, i) for e in range(e_loc) for src in range(world) for i in range(c[src, e])]
+        assert got == want
+        assert rp["local_seg"].tolist() == [0] + np.cumsum(c.sum(axis=0)).tolist()
+        assert rp["recv_offsets"].tolist() == [0] + np.cumsum(c.sum(axis=1)).tolist()
+
+
 ALL_PINS.extend([pin_philox_kat, pin_jitter, pin_logit_noise, pin_z_loss, pin_route_noise,
                  pin_temperature, pin_route_backward_finite_differences,
-                 pin_route_backward_identities, pin_near_tie, pin_expert_hidden_segments])
+                 pin_route_backward_identities, pin_near_tie, pin_expert_hidden_segments,
+                 pin_ep_forward_equals_each_rank_alone, pin_ep_plans_bruteforce])
 

@@ -149,8 +149,26 @@ def _near_tie_unsorted(logits32, k, eps=1e-3):
     return np.abs(l[:, k - 1] - l[:, k]) < eps
 
 
+def _ep_round_robin_owner(idx, drop, E, world):
+    idx = np.asarray(idx, dtype=np.int64).reshape(-1)
+    drop = np.asarray(drop, dtype=bool).reshape(-1)
+    send = np.zeros(world, dtype=np.int64)
+    for s in range(len(idx)):
+        if not drop[s]:
+            send[idx[s] % world] += 1
+    per_expert = np.bincount(idx[~drop], minlength=E)
+    return {"send_rows": send, "send_offsets": np.concatenate([[0], np.cumsum(send)]),
+            "expert_counts": per_expert}
+
+
+def _ep_recv_source_major(recv_counts):
+    r = _REAL["ep_recv_plan"](recv_counts)
+    n = len(r["local_to_recv"])
+    return dict(r, local_to_recv=np.arange(n), recv_to_local=np.arange(n))
+
+
 _REAL = {n: getattr(O, n) for n in ("combine", "expert_ffn", "permute", "permute_binned",
-                                    "jitter_multipliers", "route_backward")}
+                                    "jitter_multipliers", "route_backward", "ep_recv_plan")}
 
 MUTATIONS = {
     "topk_ties_to_higher_index": ("topk_select", _ties_to_higher),
@@ -176,6 +194,8 @@ MUTATIONS = {
     "near_tie_sign_slip": ("near_tie_tokens", _near_tie_sign),
     "near_tie_non_strict": ("near_tie_tokens", _near_tie_le),
     "near_tie_unsorted": ("near_tie_tokens", _near_tie_unsorted),
+    "ep_round_robin_expert_owner": ("ep_send_plan", _ep_round_robin_owner),
+    "ep_regroup_left_source_major": ("ep_recv_plan", _ep_recv_source_major),
 }
 
 
