@@ -17,7 +17,9 @@ struct Control {
   uint32_t bar_count;     // grid barrier: blocks arrived (reset by the last one)
   uint32_t bar_gen;       // grid barrier: generation, bumped when all arrived
   uint32_t wait_limit_us; // limit of the waits between CTAs; 0: 2 s
-  uint32_t reserved[59];
+  uint32_t gemm_next;     // CTA-pair GEMM: next work unit (reset by the last pair)
+  uint32_t gemm_done;     // CTA-pair GEMM: pairs that finished (reset by the last pair)
+  uint32_t reserved[57];
 };
 static_assert(sizeof(Control) == 256, "control block is 256 bytes");
 

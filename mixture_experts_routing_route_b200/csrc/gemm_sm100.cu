@@ -555,8 +555,21 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 // MOE_DEVERR_TIMEOUT and unwinds; the peer notices through its own bounded
 // waits. Both CTAs meet at two cluster barriers only: after set-up and before
 // tensor memory is freed, reached on every path.
+//
+// Work is handed out dynamically: the even CTA's producer takes the next unit
+// from a counter in the control block (atomicAdd) when it is ready to load
+// one and publishes it through a small ring in both CTAs' shared memory
+// (unit_full in each CTA, unit_empty in the even CTA counting the ten readers:
+// the peer's producer, the MMA thread and the pair's 8 epilogue warps); a
+// value >= the unit count ends every role's loop. The units in flight thus
+// stay a window of consecutive units, and the pairs sharing a weight block
+// read it at nearly the same time (with a fixed round-robin deal the pairs
+// drifted apart by up to a tile over a launch and re-read blocks from DRAM).
+// The last pair to finish resets the counter for the next launch.
 constexpr int kPairStages = 6;
 constexpr int kPairRows = 256;
+constexpr int kUnitSlots = 4;  // ring of work units published to the pair's roles
+constexpr uint32_t kUnitReaders = 10;  // peer producer + MMA thread + 8 epilogue warps
 
 template <int EPI>
 struct PairCfg {
@@ -608,6 +621,8 @@ grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   __shared__ int cnt_s[kMaxE];
   __shared__ int tile_start_s[kMaxE + 1];
   __shared__ volatile int abort_s;
+  __shared__ __align__(8) uint64_t unit_full[kUnitSlots], unit_empty[kUnitSlots];
+  __shared__ volatile int unit_ring[kUnitSlots];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = args.E;
@@ -626,6 +641,10 @@ grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES_P; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(&tfull_bar[b], 1); mbar_init(&tempty_bar[b], 8); }
+    for (int i = 0; i < kUnitSlots; ++i) {
+      mbar_init(&unit_full[i], 1);
+      mbar_init(&unit_empty[i], kUnitReaders);
+    }
     mbar_init(&drain_bar, 1);
     fence_mbar_init();
   }
@@ -639,12 +658,28 @@ grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   const uint32_t tmem_base = tmem_base_s;
   const int total_tiles = tile_start_s[E];
   const int W = gridDim.x >> 1;  // pairs
-  const int pid = blockIdx.x >> 1;
   const int total = num_units(total_tiles, W);
   const int nkb = args.K / BK;
-  // the even CTA's full and tempty barriers, as shared::cluster addresses
+  // the even CTA's full, tempty and unit_empty barriers, as shared::cluster addresses
   const uint32_t full0 = mapa_shared(smem_u32(&full_bar[0]), 0);
   const uint32_t tempty0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
+  const uint32_t uempty0 = mapa_shared(smem_u32(&unit_empty[0]), 0);
+
+  // A reader's next unit: wait for its slot, read it, free the slot for the
+  // producer (every reader frees every slot it reads, the end marker too).
+  // Returns total (the end) on a time-out.
+  auto next_unit = [&](int& uslot, uint32_t& uphase) -> int {
+    int u = total;
+    if (mbar_wait_cluster_bounded(&unit_full[uslot], uphase)) {
+      u = unit_ring[uslot];
+      mbar_arrive_cluster(uempty0 + uslot * 8u);
+    } else {
+      set_error(args.ctl, MOE_DEVERR_TIMEOUT);
+      abort_s = 1;
+    }
+    if (++uslot == kUnitSlots) { uslot = 0; uphase ^= 1u; }
+    return u < total ? u : total;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -655,7 +690,38 @@ grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       uint32_t phase = 0;
       uint32_t issued_mask = 0;  // stages that ever received a load
       uint32_t last_parity = 0;  // parity of that stage's latest load
-      for (int u = pid; u < total && !abort_s; u += W) {
+      int uslot = 0;
+      uint32_t uphase = 0;
+      const uint32_t ring_peer = mapa_shared(smem_u32(const_cast<int*>(&unit_ring[0])), 1);
+      const uint32_t ufull_peer = mapa_shared(smem_u32(&unit_full[0]), 1);
+      // The even CTA takes units one ahead: the counter's round trip overlaps
+      // the current unit's loads.
+      auto take = [&]() -> int {
+        return abort_s ? total
+                       : static_cast<int>(min(atomicAdd(&args.ctl->gemm_next, 1u),
+                                              static_cast<unsigned>(total)));
+      };
+      int u_next = rank == 0 ? take() : total;
+      for (;;) {
+        int u = total;
+        if (rank == 0) {
+          // publish the unit taken to both CTAs' readers
+          if (!mbar_wait_cluster_bounded(&unit_empty[uslot], uphase ^ 1u)) {
+            set_error(args.ctl, MOE_DEVERR_TIMEOUT);
+            abort_s = 1;
+            break;
+          }
+          u = abort_s ? total : u_next;
+          if (u < total) u_next = take();
+          unit_ring[uslot] = u;
+          st_shared_cluster_u32(ring_peer + uslot * 4u, static_cast<uint32_t>(u));
+          mbar_arrive(&unit_full[uslot]);
+          mbar_arrive_cluster(ufull_peer + uslot * 8u);
+          if (++uslot == kUnitSlots) { uslot = 0; uphase ^= 1u; }
+        } else {
+          u = next_unit(uslot, uphase);
+        }
+        if (u >= total || abort_s) break;
         const Tile t = decode_unit<kPairRows, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, cnt_s, E);
         const uint32_t tx = 2u * (C::A_BYTES + (t.half ? C::B_BYTES / 2 : C::B_BYTES));
         for (int kb = 0; kb < nkb; ++kb) {
@@ -680,6 +746,12 @@ grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       // arrives on empty[s] in both CTAs.
       for (int s = 0; s < STAGES_P; ++s)
         if (issued_mask & (1u << s)) (void)mbar_wait_bounded(&empty_bar[s], (last_parity >> s) & 1u);
+      // The last pair to finish resets the unit counter for the next launch
+      // (every pair's last take precedes its increment here).
+      if (rank == 0 && atomicAdd(&args.ctl->gemm_done, 1u) == static_cast<unsigned>(W) - 1u) {
+        atomicExch(&args.ctl->gemm_next, 0u);
+        atomicExch(&args.ctl->gemm_done, 0u);
+      }
     }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
@@ -690,7 +762,11 @@ grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       int acc = 0;
       uint32_t acc_phase = 0;
       bool issued_any = false;
-      for (int u = pid; u < total && !abort_s; u += W) {
+      int uslot = 0;
+      uint32_t uphase = 0;
+      for (;;) {
+        const int u = next_unit(uslot, uphase);
+        if (u >= total || abort_s) break;
         const Tile t = decode_unit<kPairRows, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, cnt_s, E);
         const uint32_t idesc = t.half ? kIdescHalf : kIdescFull;
         if (!mbar_wait_cluster_bounded(&tempty_bar[acc], acc_phase ^ 1u)) {
@@ -736,16 +812,20 @@ grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     const int q = warp & 3;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int u = pid; u < total; u += W) {
-      int ok = 0;
+    int uslot = 0;
+    uint32_t uphase = 0;
+    for (;;) {
+      int ok = 0, u = total;
       if (lane == 0) {
-        ok = !abort_s && mbar_wait_cluster_bounded(&tfull_bar[acc], acc_phase);
-        if (!ok && !abort_s) {
+        u = next_unit(uslot, uphase);
+        ok = u < total && !abort_s && mbar_wait_cluster_bounded(&tfull_bar[acc], acc_phase);
+        if (!ok && u < total && !abort_s) {
           set_error(args.ctl, MOE_DEVERR_TIMEOUT);
           abort_s = 1;
         }
       }
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      u = __shfl_sync(0xffffffffu, u, 0);
       const Tile t = decode_unit<kPairRows, C::OUT_N>(u, total_tiles, W, tile_start_s, seg_s, cnt_s, E);
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * NMMA;

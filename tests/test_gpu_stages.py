@@ -496,3 +496,23 @@ def test_route_backward(T, d, E, k, dt, tau, d_aux, d_z):
     assert max_err_ratio(np32(d_logits), ref["d_logits"]) <= 1e-5
     assert max_err_ratio(np32(d_wg), ref["dwg"]) <= 1e-4
     assert max_err_ratio(np32(dx), ref["dx"]) <= (TOL_BF16_OUT if dt == "bf16" else 1e-5)
+
+
+def test_pair_gemm_repeats_on_one_workspace():
+    """The CTA-pair GEMM hands out its tiles from a counter in the
+    workspace's control block, reset by the last pair of each launch: three
+    forwards on one workspace (six pair launches) give the same output bit
+    for bit, and both counter words are zero afterwards."""
+    from mixture_experts_routing_route_b200 import MoeLayer
+    inp = small_case("rep", T=1600, d=256, E=4, k=2, F=256, act="swiglu", seed=44)
+    layer = MoeLayer(inp.wg.to(DEV), inp.w1.to(DEV), inp.w2.to(DEV), w3=inp.w3.to(DEV), k=2, act="swiglu")
+    x = inp.x.to(DEV)
+    outs = []
+    for _ in range(3):
+        out, _ = layer.forward(x)
+        outs.append(out.clone())
+    torch.cuda.synchronize()
+    assert layer.device_error(1600) == 0
+    assert all(torch.equal(o, outs[0]) for o in outs[1:])
+    ctl = layer.workspace(1600)[:256].view(torch.int32).cpu()
+    assert int(ctl[5]) == 0 and int(ctl[6]) == 0  # next unit, pairs done
