@@ -174,16 +174,22 @@ moe_status_t run_forward(const moe_layer_t* L, const void* x, int T, void* out, 
   };
   const size_t es = esize(L->dtype);
   rec(0);
-  // the router may read its own input (a jittered x) and add logit noise
+  // the router may read its own input (a jittered x) and add logit noise; the
+  // last step of its load-balance loss may run in the multi-CTA permute
+  // kernel's tail instead of a launch of its own (launch_route decides)
+  AuxJob aux_job{};
+  AuxJob* defer = permute_uses_grid(T, L->k, L->E) ? &aux_job : nullptr;
   MOE_CHECK(from_cuda(launch_route(L->x_router != nullptr ? L->x_router : x, L->w_router,
                                    L->router_bias, L->logit_noise, L->dtype, T, L->d, L->E, L->k,
                                    f.idx, f.w, f.aux, (L->flags & MOE_LAYER_Z_LOSS) ? f.z : nullptr,
                                    nullptr, nullptr, f.logits_scratch, f.partials, f.ctl, s,
-                                   L->router_temperature > 0.0f ? L->router_temperature : 1.0f)));
+                                   L->router_temperature > 0.0f ? L->router_temperature : 1.0f,
+                                   defer)));
   rec(1);
   MOE_CHECK(from_cuda(launch_permute(f.idx, T, L->k, L->E, f.cap, f.counts, f.bins, f.sorted_slot,
                                      f.slot_to_row, f.row_slot, f.drop, f.kept, f.seg, f.rank,
-                                     f.ctl, s, binned(L))));
+                                     f.ctl, s, binned(L),
+                                     defer != nullptr && defer->pending ? defer : nullptr)));
   rec(2);
   const bool cig = combine_in_gemm(L);
   // the gather kernel also zeroes the output rows of fully dropped tokens

@@ -48,6 +48,105 @@ template <> struct Elem<__nv_bfloat16> {
   static __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
 };
 
+// The load-balance loss's last step, which a layer forward may leave to the
+// permute kernel (it runs next anyway) when the router would otherwise need a
+// launch of its own for it: aux = E * sum_e (c_e / (T k)) (p_e / T)
+// from the router's per-block partials part_p / part_c [E][ldb] (nblk
+// blocks), and the z-loss, mean over tokens of lse^2, from part_z [nblk]
+// (null: none). terms [E] is scratch.
+struct AuxJob {
+  int pending;  // 1: launch_route left the step to a later kernel
+  const float* part_p;
+  const int32_t* part_c;
+  const float* part_z;
+  double* terms;
+  float* aux;
+  float* z;
+  int ldb, nblk, E, T, k;
+};
+
+// Finish a deferred load-balance loss with the first min(gridDim.x, E) CTAs
+// of a grid (every thread of each CTA calls it; threads 0..255 do the work,
+// blockDim.x >= 256; the other CTAs return at once). CTA b takes the experts
+// b, b + gridDim.x, ...: thread i adds the partials of blocks i, i + 256, ...
+// in float64, each warp reduces with a fixed butterfly and thread 0 adds the
+// 8 warp sums in order; the last of those CTAs (ticket) adds the E terms the
+// same way and reduces the z-loss likewise. Deterministic. Uses
+// ctl->route_ticket (free during the permute).
+constexpr int kAuxFinishThreads = 256;
+
+__device__ __forceinline__ double warp_sum_f64(double v) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+__device__ __forceinline__ long long warp_sum_i64(long long v) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+// scratch: >= 2 * 8 * 8 bytes of the caller's shared memory, 8-byte aligned,
+// free from this call on (a barrier first orders it after the caller's use).
+__device__ __forceinline__ void finish_aux_job(const AuxJob& j, Control* ctl, void* scratch) {
+  constexpr int nt = kAuxFinishThreads, nw = nt / 32;
+  const int parts = min(static_cast<int>(gridDim.x), j.E);
+  if (static_cast<int>(blockIdx.x) >= parts) return;  // CTA-uniform
+  double* wp = static_cast<double*>(scratch);         // [nw]
+  long long* wc = reinterpret_cast<long long*>(wp + nw);  // [nw]
+  double* wz = wp + nw;                                   // [nw], the z-loss step (reuses wc)
+  __shared__ int fa_last;
+  const int tid = threadIdx.x, lane = tid & 31, wq = tid >> 5;
+  const bool part = tid < nt;
+  __syncthreads();
+  for (int e = blockIdx.x; e < j.E; e += gridDim.x) {
+    if (part) {
+      double ps = 0.0;
+      long long cs = 0;
+      for (int b = tid; b < j.nblk; b += nt) {
+        ps += static_cast<double>(__ldcg(j.part_p + static_cast<size_t>(e) * j.ldb + b));
+        cs += __ldcg(j.part_c + static_cast<size_t>(e) * j.ldb + b);
+      }
+      ps = warp_sum_f64(ps);
+      cs = warp_sum_i64(cs);
+      if (lane == 0) { wp[wq] = ps; wc[wq] = cs; }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      double p = 0.0;
+      long long c = 0;
+      for (int w = 0; w < nw; ++w) { p += wp[w]; c += wc[w]; }
+      j.terms[e] = j.T > 0 ? (static_cast<double>(c) / (static_cast<double>(j.T) * j.k)) * (p / j.T) : 0.0;
+    }
+    __syncthreads();
+  }
+  if (tid == 0) {
+    __threadfence();
+    fa_last = atomicAdd(&ctl->route_ticket, 1u) == static_cast<unsigned>(parts) - 1u;
+  }
+  __syncthreads();
+  if (!fa_last) return;
+  __threadfence();
+  if (part) {
+    double v = tid < j.E ? __ldcg(j.terms + tid) : 0.0;
+    v = warp_sum_f64(v);
+    double zs = 0.0;
+    if (j.part_z != nullptr)
+      for (int b = tid; b < j.nblk; b += nt) zs += static_cast<double>(__ldcg(j.part_z + b));
+    zs = warp_sum_f64(zs);
+    if (lane == 0) { wp[wq] = v; wz[wq] = zs; }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    double tot = 0.0, z = 0.0;
+    for (int w = 0; w < nw; ++w) { tot += wp[w]; z += wz[w]; }
+    *j.aux = static_cast<float>(j.E * tot);
+    if (j.part_z != nullptr) *j.z = j.T > 0 ? static_cast<float>(z / j.T) : 0.f;
+    ctl->route_ticket = 0u;
+  }
+}
+
 // ------------------------------------------- programmatic dependent launch
 // Every kernel of the library is launched with programmatic stream
 // serialisation and starts with pdl_begin(): it waits there until the
@@ -117,7 +216,7 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, const
                          moe_dtype_t dt, int T, int d, int E, int k, int32_t* idx, float* w,
                          float* aux, float* z_out, float* logits, float* probs,
                          float* logits_scratch, void* partials, Control* ctl, cudaStream_t s,
-                         float temperature = 1.0f);
+                         float temperature = 1.0f, AuxJob* defer_aux = nullptr);
 size_t route_logits_scratch_bytes(int T, int d, int E);
 // Router backward (see router_backward.cu): d_logits [T, E] fp32 (or NULL:
 // kept in scratch), dx [T, d] (dtype) or NULL, d_wg [d, E] fp32 or NULL.
@@ -137,16 +236,21 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
 // the [E, C] bucket layout (row e*C + rank; C = cap, or the largest count
 // when cap < 0; padding rows get row_slot -1).
 size_t permute_scratch_bytes(int T, int k, int E);
+// Whether launch_permute runs the multi-CTA kernel for these sizes (which
+// finishes a deferred load-balance loss cheaply across its CTAs).
+bool permute_uses_grid(int T, int k, int E);
 cudaError_t launch_permute_single(const int32_t* idx, int T, int k, int E, int64_t cap,
                                   int32_t* counts, int32_t* bins, int32_t* sorted_slot,
                                   int32_t* slot_to_row, int32_t* row_slot, uint8_t* drop,
                                   int32_t* kept, int32_t* seg, int32_t* rank_scratch, Control* ctl,
-                                  cudaStream_t s, bool binned = false);
+                                  cudaStream_t s, bool binned = false,
+                                  const AuxJob* aux_job = nullptr);
+// aux_job: a load-balance loss left by launch_route to finish (see AuxJob).
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int64_t cap, int32_t* counts,
                            int32_t* bins, int32_t* sorted_slot, int32_t* slot_to_row,
                            int32_t* row_slot, uint8_t* drop, int32_t* kept, int32_t* seg,
                            int32_t* rank_scratch, Control* ctl, cudaStream_t s,
-                           bool binned = false);
+                           bool binned = false, const AuxJob* aux_job = nullptr);
 
 // Router training inputs (noise.cu): x' = x * uniform(1 - eps, 1 + eps)
 // elementwise (n elements, dtype dt), and std * N(0, 1) logit noise (n

@@ -44,9 +44,9 @@ permute_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_mask,
                int32_t* __restrict__ sorted_slot, int32_t* __restrict__ slot_to_row,
                int32_t* __restrict__ row_slot, uint8_t* __restrict__ drop,
                int32_t* __restrict__ kept, int32_t* __restrict__ seg, int32_t* __restrict__ rank_g,
-               Control* ctl) {
+               Control* ctl, AuxJob job, int has_job) {
   pdl_begin();
-  __shared__ int hist[32][kMaxE + 1];
+  __shared__ __align__(16) int hist[32][kMaxE + 1];
   __shared__ int running[kMaxE];
   __shared__ int start_s[kMaxE];
   __shared__ int seg_s[kMaxE + 1];
@@ -180,6 +180,7 @@ permute_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_mask,
       if (!dr) row_slot[row] = s;
     }
   }
+  if (has_job) finish_aux_job(job, ctl, &hist[0][0]);  // the router's loss, left to this kernel
 }
 
 // ---------------------------------------------------------------- multi-CTA
@@ -233,9 +234,10 @@ permute_grid_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_
                     int32_t* __restrict__ bins, int32_t* __restrict__ sorted_slot,
                     int32_t* __restrict__ slot_to_row, int32_t* __restrict__ row_slot,
                     uint8_t* __restrict__ drop, int32_t* __restrict__ kept,
-                    int32_t* __restrict__ seg, int32_t* __restrict__ cta_counts, Control* ctl) {
+                    int32_t* __restrict__ seg, int32_t* __restrict__ cta_counts, Control* ctl,
+                    AuxJob job, int has_job) {
   pdl_begin();
-  __shared__ int s_e[kGMaxChunk];
+  __shared__ __align__(16) int s_e[kGMaxChunk];
   __shared__ int s_rank[kGMaxChunk];
   __shared__ int hist[8][kMaxE + 1];
   __shared__ int running[kMaxE];
@@ -375,6 +377,7 @@ permute_grid_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_
     slot_to_row[s] = row;
     if (!dr) row_slot[row] = s;
   }
+  if (has_job) finish_aux_job(job, ctl, s_e);  // the router's loss, spread over the CTAs
 }
 
 __global__ void set_wait_limit_kernel(Control* ctl, uint32_t limit_us) {
@@ -403,34 +406,45 @@ cudaError_t launch_permute_single(const int32_t* idx, int T, int k, int E, int64
                                   int32_t* counts, int32_t* bins, int32_t* sorted_slot,
                                   int32_t* slot_to_row, int32_t* row_slot, uint8_t* drop,
                                   int32_t* kept, int32_t* seg, int32_t* rank_scratch, Control* ctl,
-                                  cudaStream_t s, bool binned) {
+                                  cudaStream_t s, bool binned, const AuxJob* aux_job) {
   const unsigned mask = static_cast<unsigned>(key_mask_of(E));
   const long long c = cap < 0 ? LLONG_MAX : static_cast<long long>(cap);
+  const AuxJob job = aux_job != nullptr ? *aux_job : AuxJob{};
   return launch_pdl(permute_kernel, dim3(1), dim3(kThreads), 0, s, false, idx, T * k, E, mask, c,
                     binned ? 1 : 0, counts, bins, sorted_slot, slot_to_row, row_slot, drop, kept, seg, rank_scratch,
-                    ctl);
+                    ctl, job, aux_job != nullptr ? 1 : 0);
+}
+
+bool permute_uses_grid(int T, int k, int E) {
+  (void)E;
+  const int S = T * k;
+  const int g = std::max(1, std::min(num_sms(), (S + kGThreads - 1) / kGThreads));
+  const int chunk = S > 0 ? (S + g - 1) / g : 0;
+  return !(S == 0 || chunk > kGMaxChunk || g < 2);
 }
 
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int64_t cap, int32_t* counts,
                            int32_t* bins, int32_t* sorted_slot, int32_t* slot_to_row,
                            int32_t* row_slot, uint8_t* drop, int32_t* kept, int32_t* seg,
-                           int32_t* scratch, Control* ctl, cudaStream_t s, bool binned) {
+                           int32_t* scratch, Control* ctl, cudaStream_t s, bool binned,
+                           const AuxJob* aux_job) {
   const int S = T * k;
   const int sms = num_sms();
   // enough CTAs that each chunk fits shared memory, at most one per SM, and
-  // at least ~256 slots per CTA
+  // at least ~256 slots per CTA (the same rule as permute_uses_grid)
   const int g = std::max(1, std::min(sms, (S + kGThreads - 1) / kGThreads));
   const int chunk = S > 0 ? (S + g - 1) / g : 0;
-  if (S == 0 || chunk > kGMaxChunk || g < 2)
+  if (!permute_uses_grid(T, k, E))
     return launch_permute_single(idx, T, k, E, cap, counts, bins, sorted_slot, slot_to_row,
-                                 row_slot, drop, kept, seg, scratch, ctl, s, binned);
+                                 row_slot, drop, kept, seg, scratch, ctl, s, binned, aux_job);
   int32_t* cta_counts = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(scratch) +
                                                    align_up(static_cast<size_t>(S) * 4));
   unsigned mask = static_cast<unsigned>(key_mask_of(E));
   long long c = cap < 0 ? LLONG_MAX : static_cast<long long>(cap);
+  const AuxJob job = aux_job != nullptr ? *aux_job : AuxJob{};
   return launch_pdl(permute_grid_kernel, dim3(g), dim3(kGThreads), 0, s, true, idx, S, E, mask, c,
                     binned ? 1 : 0, chunk, counts, bins, sorted_slot, slot_to_row, row_slot, drop, kept, seg,
-                    cta_counts, ctl);
+                    cta_counts, ctl, job, aux_job != nullptr ? 1 : 0);
 }
 
 }  // namespace moe

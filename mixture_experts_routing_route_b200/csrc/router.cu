@@ -1437,7 +1437,7 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, const
                          moe_dtype_t dt, int T, int d, int E, int k, int32_t* idx, float* w,
                          float* aux, float* z_out, float* logits, float* probs,
                          float* logits_scratch, void* partials, Control* ctl, cudaStream_t s,
-                         float temperature) {
+                         float temperature, AuxJob* defer_aux) {
   const float inv_tau = 1.0f / temperature;
   const int ldb = route_max_blocks(T);
   float* part_p = static_cast<float*>(partials);
@@ -1449,6 +1449,14 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, const
                                    : reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(terms) +
                                                               align_up(256 * 8));
   int nblk = 0;
+  // With defer_aux the loss's last step is described for a later kernel
+  // instead of being run here.
+  // Only the paths that would launch aux_reduce defer (the fused tensor-core
+  // router's own last-tile step costs less than a later kernel's).
+  auto defer = [&](int blocks) {
+    *defer_aux = AuxJob{1, part_p, part_c, part_z, terms, aux, z_out, ldb, blocks, E, T, k};
+  };
+  if (defer_aux != nullptr) defer_aux->pending = 0;
   // The fp32 E <= 8 kernel has neither the noise input, the z-loss nor a temperature.
   if (use_fused(d, E, dt) && noise == nullptr && z_out == nullptr && inv_tau == 1.0f) {
     const int groups = (T + kFusedTokensPerGroup - 1) / kFusedTokensPerGroup;
@@ -1575,6 +1583,10 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, const
                                      ctl);
     if (e != cudaSuccess) return e;
     nblk = g2;
+  }
+  if (defer_aux != nullptr) {
+    defer(nblk);
+    return cudaSuccess;
   }
   return launch_pdl(aux_reduce, dim3(E), dim3(kAuxThreads), 0, s, false,
                     static_cast<const float*>(part_p), static_cast<const int32_t*>(part_c),
