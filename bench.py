@@ -483,6 +483,8 @@ def run_router_backward(args):
         b.record()
     n1 = abi.moe_kernel_launches()
     torch.cuda.synchronize()
+    if abi.moe_get_device_error(bws) != 0:
+        raise RuntimeError("device error word set during the timed calls")
     times = sorted(a.elapsed_time(b) for a, b in evs)
     ms = statistics.median(times)
     eb = x.element_size()

@@ -382,7 +382,7 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       }
       // Every load issued must have landed before the CTA may exit.
       for (int s = 0; s < STAGES; ++s)
-        if (issued_mask & (1u << s)) (void)mbar_wait_bounded(&full_bar[s], (last_parity >> s) & 1u);
+        if (issued_mask & (1u << s)) if (!mbar_wait_bounded(&full_bar[s], (last_parity >> s) & 1u)) set_error(args.ctl, MOE_DEVERR_TIMEOUT);
     }
   } else if (warp == 0) {
     // GATHER: lane 0 waits for each ring slot and arms it, then the whole
@@ -437,7 +437,7 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     }
     if (lane == 0)
       for (int s = 0; s < STAGES; ++s)
-        if (issued_mask & (1u << s)) (void)mbar_wait_bounded(&full_bar[s], (last_parity >> s) & 1u);
+        if (issued_mask & (1u << s)) if (!mbar_wait_bounded(&full_bar[s], (last_parity >> s) & 1u)) set_error(args.ctl, MOE_DEVERR_TIMEOUT);
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t kIdescFull = make_idesc_bf16(BM, NMMA);
@@ -745,7 +745,7 @@ grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       // before this CTA may leave: the MMA commit of each stage's last load
       // arrives on empty[s] in both CTAs.
       for (int s = 0; s < STAGES_P; ++s)
-        if (issued_mask & (1u << s)) (void)mbar_wait_bounded(&empty_bar[s], (last_parity >> s) & 1u);
+        if (issued_mask & (1u << s)) if (!mbar_wait_bounded(&empty_bar[s], (last_parity >> s) & 1u)) set_error(args.ctl, MOE_DEVERR_TIMEOUT);
       // The last pair to finish resets the unit counter for the next launch
       // (every pair's last take precedes its increment here).
       if (rank == 0 && atomicAdd(&args.ctl->gemm_done, 1u) == static_cast<unsigned>(W) - 1u) {

@@ -19,6 +19,7 @@
 // dWg as per-token-split partials added in split order (deterministic).
 // fp32 arithmetic throughout; dx is rounded once to the input dtype.
 #include "common.cuh"
+#include "ptx.cuh"
 
 #include <cmath>
 
@@ -345,6 +346,254 @@ bwd_dwg_part(const T* __restrict__ x, const float* __restrict__ dl, int Tn, int 
   }
 }
 
+// ------------------------------------------------ bf16, E <= 16: streaming
+// The two T x d passes of the Mixtral-sized router are pure streams (E
+// multiply-adds per element): dx writes T x d, dWg reads x once. These
+// kernels give each thread 8 consecutive columns (one 16-byte bf16 vector
+// per token row) so that every row of x or dx is touched by whole 16-byte
+// accesses, keep the per-column Wg values or accumulators in registers, and
+// stage each block's d_logits tile in shared memory once.
+constexpr int kFastThreads = 128;   // dx: 128 x 8 = 1024 columns per block
+constexpr int kFastTok = 32;        // dx: tokens per block
+constexpr int kFastDwgThreads = 128;  // dWg: 128 x 8 = 1024 columns per block
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float (&v)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+__device__ __forceinline__ uint4 f32x8_to_bf16(const float (&v)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    w[i] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// dx[t, c] = sum_e dl[t, e] Wg[c, e], e in increasing order (the order of
+// bwd_dx). EC >= E (8 or 16); d a multiple of 8. The block's Wg rows
+// [c0, c0 + 1024) are one contiguous range of memory: they are copied to
+// shared memory with 16-byte loads, then each thread keeps its 8 rows in
+// registers; the block's d_logits rows are staged once.
+template <int EC>
+__global__ void __launch_bounds__(kFastThreads)
+bwd_dx_fast(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, int Tn, int d, int E,
+            __nv_bfloat16* __restrict__ dx) {
+  pdl_begin();
+  extern __shared__ __align__(16) uint8_t dx_sm[];
+  __nv_bfloat16* wg_s = reinterpret_cast<__nv_bfloat16*>(dx_sm);                       // [2048][E]
+  float* dl_s = reinterpret_cast<float*>(dx_sm + kFastThreads * 8 * EC * 2);           // [kFastTok][EC]
+  const int c0 = blockIdx.x * kFastThreads * 8;
+  const int ncol = min(kFastThreads * 8, d - c0);
+  const int c = c0 + threadIdx.x * 8;
+  const int t0 = blockIdx.y * kFastTok;
+  {
+    const long long n16 = static_cast<long long>(ncol) * E * 2 / 16;  // a whole number: ncol % 8 == 0
+    const uint4* src = reinterpret_cast<const uint4*>(wg + static_cast<size_t>(c0) * E);
+    for (long long i = threadIdx.x; i < n16; i += kFastThreads)
+      reinterpret_cast<uint4*>(wg_s)[i] = __ldg(src + i);
+  }
+  for (int i = threadIdx.x; i < kFastTok * EC; i += kFastThreads) {
+    const int tt = i / EC, e = i - tt * EC;
+    const int t = t0 + tt;
+    dl_s[i] = (e < E && t < Tn) ? __ldg(dl + static_cast<size_t>(t) * E + e) : 0.f;
+  }
+  __syncthreads();
+  if (c >= d) return;
+  float wv[8][EC];
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+    for (int e = 0; e < EC; ++e)
+      wv[jj][e] = e < E ? __bfloat162float(wg_s[(threadIdx.x * 8 + jj) * E + e]) : 0.f;
+  const int nt = min(kFastTok, Tn - t0);
+#pragma unroll 4
+  for (int tt = 0; tt < nt; ++tt) {
+    float acc[8];
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) acc[jj] = 0.f;
+#pragma unroll
+    for (int e4 = 0; e4 < EC; e4 += 4) {
+      const float4 g4 = *reinterpret_cast<const float4*>(dl_s + tt * EC + e4);
+      const float g[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) acc[jj] = fmaf(g[q], wv[jj][e4 + q], acc[jj]);
+    }
+    *reinterpret_cast<uint4*>(dx + static_cast<size_t>(t0 + tt) * d + c) = f32x8_to_bf16(acc);
+  }
+}
+
+size_t dx_fast_smem(int ec) {
+  return static_cast<size_t>(kFastThreads) * 8 * ec * 2 + static_cast<size_t>(kFastTok) * ec * 4;
+}
+
+// dWg partial of token split s: part[s][c][e] = sum over the split's tokens
+// (increasing) of x[t, c] dl[t, e]. EC >= E (8 or 16); d a multiple of 8.
+// Block = G row groups of 128 threads, one block per SM; a group's thread
+// owns 8 columns of the block's 1024 (G = 4 for EC = 8, 2 for EC = 16, so
+// that the accumulators fit). Thread 0 streams the split's rows of that
+// column slice (2 KB per token row) with bulk copies into a 4-stage ring of
+// 16 rows (128 KB in flight per SM, the copy engine's, not registers); group
+// g adds rows g, g + G, ... of each stage. At the end groups 1..G-1 leave
+// their sums in the idle ring and group 0 adds them in group order.
+// Waits are bounded.
+constexpr int kDwgBulkStages = 4;
+constexpr int kDwgBulkRows = 16;
+constexpr int kDwgBulkRowBytes = kFastDwgThreads * 8 * 2;  // 2048
+
+template <int EC>
+struct DwgBulk {
+  static constexpr int G = EC == 8 ? 4 : 2;
+  static constexpr int kThreads = G * kFastDwgThreads;
+};
+
+size_t dwg_bulk_smem(int tps, int ec) {
+  return static_cast<size_t>(kDwgBulkStages) * kDwgBulkRows * kDwgBulkRowBytes + 128 +
+         static_cast<size_t>(tps) * ec * sizeof(float);
+}
+
+template <int EC>
+__global__ void __launch_bounds__(DwgBulk<EC>::kThreads, 1)
+bwd_dwg_bulk(const __nv_bfloat16* __restrict__ x, const float* __restrict__ dl, int Tn, int d, int E,
+             int tok_per_split, float* __restrict__ part, Control* ctl) {
+  pdl_begin();
+  constexpr int G = DwgBulk<EC>::G, NT = DwgBulk<EC>::kThreads;
+  static_assert(static_cast<size_t>(G - 1) * kFastDwgThreads * 8 * EC * 4 <=
+                    static_cast<size_t>(kDwgBulkStages) * kDwgBulkRows * kDwgBulkRowBytes,
+                "the groups' sums fit in the ring");
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ __align__(8) uint64_t full[kDwgBulkStages], empty[kDwgBulkStages];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm) + 127) & ~uintptr_t(127));
+  float* dls = reinterpret_cast<float*>(ring + kDwgBulkStages * kDwgBulkRows * kDwgBulkRowBytes);
+  const int tid = threadIdx.x;
+  const int grp = tid / kFastDwgThreads, gt = tid - grp * kFastDwgThreads;
+  const int c0 = blockIdx.x * kFastDwgThreads * 8;
+  const int ncol = min(kFastDwgThreads * 8, d - c0);
+  const uint32_t rowb = static_cast<uint32_t>(ncol) * 2;  // a multiple of 16 (d % 8 == 0)
+  const int tb = blockIdx.y * tok_per_split;
+  const int n = max(0, min(Tn, tb + tok_per_split) - tb);
+  const int nstg = (n + kDwgBulkRows - 1) / kDwgBulkRows;
+  if (tid == 0) {
+    for (int i = 0; i < kDwgBulkStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], NT);
+    }
+    fence_mbar_init();
+  }
+  for (int i = tid; i < n * EC; i += NT) {
+    const int tt = i / EC, e = i - tt * EC;
+    dls[i] = e < E ? __ldg(dl + static_cast<size_t>(tb + tt) * E + e) : 0.f;
+  }
+  __syncthreads();
+  auto issue = [&](int st) {
+    const int slot = st % kDwgBulkStages, r0 = st * kDwgBulkRows;
+    const int nr = min(kDwgBulkRows, n - r0);
+    mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nr) * rowb);
+    for (int r = 0; r < nr; ++r)
+      bulk_load(ring + (slot * kDwgBulkRows + r) * kDwgBulkRowBytes,
+                x + static_cast<size_t>(tb + r0 + r) * d + c0, rowb, &full[slot]);
+  };
+  if (tid == 0)
+    for (int st = 0; st < nstg && st < kDwgBulkStages; ++st) issue(st);
+  float acc[8][EC];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+#pragma unroll
+    for (int e = 0; e < EC; ++e) acc[j][e] = 0.f;
+  const bool mine = gt * 8 < ncol;
+  int issued = min(nstg, kDwgBulkStages);
+  bool ok = true;
+  for (int st = 0; st < nstg; ++st) {
+    const int slot = st % kDwgBulkStages;
+    if (!mbar_wait_bounded(&full[slot], static_cast<uint32_t>(st / kDwgBulkStages) & 1u)) {
+      set_error(ctl, MOE_DEVERR_TIMEOUT);
+      ok = false;
+      break;
+    }
+    const int nr = min(kDwgBulkRows, n - st * kDwgBulkRows);
+    if (mine) {
+      const uint8_t* rows = ring + slot * kDwgBulkRows * kDwgBulkRowBytes + gt * 16;
+#pragma unroll 2
+      for (int r = grp; r < nr; r += G) {
+        float xv[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(rows + r * kDwgBulkRowBytes), xv);
+        const float* g = dls + (st * kDwgBulkRows + r) * EC;
+#pragma unroll
+        for (int e = 0; e < EC; ++e) {
+          const float ge = g[e];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[j][e] = fmaf(xv[j], ge, acc[j][e]);
+        }
+      }
+    }
+    mbar_arrive(&empty[slot]);
+    if (tid == 0 && issued < nstg) {
+      // the slot is free once every thread has read this stage
+      if (!mbar_wait_bounded(&empty[slot], static_cast<uint32_t>(st / kDwgBulkStages) & 1u)) {
+        set_error(ctl, MOE_DEVERR_TIMEOUT);
+        ok = false;
+        break;
+      }
+      issue(issued);
+      ++issued;
+    }
+  }
+  if (tid == 0) {
+    // every copy issued must have landed before the ring is reused or the
+    // block leaves: wait for the last stage issued into each slot
+    for (int slot = 0; slot < kDwgBulkStages && slot < issued; ++slot) {
+      const int last = slot + ((issued - 1 - slot) / kDwgBulkStages) * kDwgBulkStages;
+      if (!mbar_wait_bounded(&full[slot], static_cast<uint32_t>(last / kDwgBulkStages) & 1u))
+        set_error(ctl, MOE_DEVERR_TIMEOUT);
+    }
+  }
+  __syncthreads();  // every thread is done with the ring: it holds the groups' sums now
+  float* red = reinterpret_cast<float*>(ring);  // [G - 1][128 threads][8][EC]
+  if (grp > 0 && mine) {
+    float* dst = red + (static_cast<size_t>(grp - 1) * kFastDwgThreads + gt) * 8 * EC;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < EC; e += 4)
+        *reinterpret_cast<float4*>(dst + j * EC + e) =
+            make_float4(acc[j][e], acc[j][e + 1], acc[j][e + 2], acc[j][e + 3]);
+  }
+  __syncthreads();
+  if (grp != 0 || !mine || !ok) return;
+#pragma unroll
+  for (int q = 1; q < G; ++q) {
+    const float* src = red + (static_cast<size_t>(q - 1) * kFastDwgThreads + gt) * 8 * EC;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < EC; ++e) acc[j][e] += src[j * EC + e];
+  }
+  // the 8 columns' E values are 8 * E consecutive floats of the partial
+  float* dst = part + (static_cast<size_t>(blockIdx.y) * d + c0 + gt * 8) * E;
+  if (E == EC) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < EC; e += 4)
+        *reinterpret_cast<float4*>(dst + j * EC + e) =
+            make_float4(acc[j][e], acc[j][e + 1], acc[j][e + 2], acc[j][e + 3]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < EC; ++e)
+        if (e < E) dst[j * E + e] = acc[j][e];
+  }
+}
+
 // d_wg[c, e] = sum_s part[s][c][e], s increasing.
 __global__ void __launch_bounds__(256)
 bwd_dwg_reduce(const float* __restrict__ part, int nsplit, long long n, float* __restrict__ d_wg) {
@@ -388,6 +637,13 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
   float* part = reinterpret_cast<float*>(sc);
   const float inv_tau = 1.0f / temperature;
   const bool aux = d_aux != 0.0f;
+  // bf16 with at most 16 experts: the streaming kernels (16-byte row access;
+  // dWg through the bulk-copy ring while a split's d_logits fit beside it)
+  const bool fast = dt == MOE_BF16 && E <= 16 && d % 8 == 0;
+  const int fxb = (d + kFastDwgThreads * 8 - 1) / (kFastDwgThreads * 8);
+  const int fns = std::max(1, std::min(dwg_splits(T, d, E), num_sms() / fxb));
+  const int ftps = T > 0 ? (T + fns - 1) / fns : 0;
+  const bool fast_dwg = fast && dwg_bulk_smem(std::max(ftps, 1), E <= 8 ? 8 : 16) <= 200 * 1024;
   cudaError_t err = cudaSuccess;
   if (T > 0) {
     if (aux) {
@@ -403,7 +659,15 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
                      d_z != 0.0f ? logits : nullptr, idx, w, d_w, aux ? counts : nullptr, d_aux,
                      d_z, inv_tau, T, E, k, dl, ctl);
     if (err != cudaSuccess) return err;
-    if (dx != nullptr) {
+    if (dx != nullptr && fast) {
+      const dim3 g((d + kFastThreads * 8 - 1) / (kFastThreads * 8), (T + kFastTok - 1) / kFastTok);
+      auto kern = E <= 8 ? bwd_dx_fast<8> : bwd_dx_fast<16>;
+      const size_t dsm = dx_fast_smem(E <= 8 ? 8 : 16);
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dsm));
+      err = launch_pdl(kern, g, dim3(kFastThreads), dsm, s, false, static_cast<const float*>(dl),
+                       static_cast<const __nv_bfloat16*>(wg), T, d, E, static_cast<__nv_bfloat16*>(dx));
+      if (err != cudaSuccess) return err;
+    } else if (dx != nullptr) {
       const int tiles = E <= kDxE ? kDxTiles : 1;
       const dim3 g((d + kDxCols - 1) / kDxCols, (T + kDxTok * tiles - 1) / (kDxTok * tiles));
       err = dt == MOE_BF16
@@ -415,7 +679,23 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
       if (err != cudaSuccess) return err;
     }
   }
-  if (d_wg != nullptr) {
+  if (d_wg != nullptr && fast_dwg) {
+    // one block per SM: the column slices times the token splits
+    const int xb = fxb, ns = fns, tps = ftps;
+    const int ec = E <= 8 ? 8 : 16;
+    const size_t smem = dwg_bulk_smem(std::max(tps, 1), ec);
+    auto kern = ec == 8 ? bwd_dwg_bulk<8> : bwd_dwg_bulk<16>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    const int nthr = ec == 8 ? DwgBulk<8>::kThreads : DwgBulk<16>::kThreads;
+    err = launch_pdl(kern, dim3(xb, ns), dim3(nthr), smem, s, false,
+                     static_cast<const __nv_bfloat16*>(x), static_cast<const float*>(dl), T, d, E, tps,
+                     part, ctl);
+    if (err != cudaSuccess) return err;
+    const long long n = static_cast<long long>(d) * E;
+    const int rg = static_cast<int>(std::min<long long>((n + 255) / 256, 8LL * num_sms()));
+    err = launch_pdl(bwd_dwg_reduce, dim3(std::max(rg, 1)), dim3(256), 0, s, false,
+                     static_cast<const float*>(part), ns, n, d_wg);
+  } else if (d_wg != nullptr) {
     const int ns = dwg_splits(T, d, E);
     const int tps = T > 0 ? (T + ns - 1) / ns : 0;
     const int ec = E <= 8 ? 8 : (E <= 16 ? 16 : 32);
