@@ -63,9 +63,12 @@ bwd_logits(const float* __restrict__ probs, const float* __restrict__ logits,
            const int32_t* __restrict__ idx, const float* __restrict__ w,
            const float* __restrict__ d_w, const int32_t* __restrict__ counts, float d_aux,
            float d_z, float inv_tau, int T, int E, int k, float* __restrict__ d_logits,
-           Control* ctl) {
+           __nv_bfloat16* __restrict__ dlT, int ec, int ldt, int* __restrict__ tickets,
+           int ntickets, Control* ctl) {
   pdl_begin();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (tickets != nullptr && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < ntickets; i += blockDim.x) tickets[i] = 0;
   // the aux term is the same for every token: d_aux * E * f_e / T
   float aux_c[EPL];
 #pragma unroll
@@ -149,6 +152,14 @@ bwd_logits(const float* __restrict__ probs, const float* __restrict__ logits,
     for (int q = 0; q < EPL; ++q) {
       const int e = lane + 32 * q;
       if (e < E) d_logits[row + e] = dl[q];
+    }
+    if (dlT != nullptr && lane < ec) {
+      // the tensor-core dWg's B operand: rows [hi 0..ec) then [lo 0..ec),
+      // tokens along the rows (E <= 16, so EPL == 1 and lane = expert)
+      const float v = lane < E ? dl[0] : 0.f;
+      const __nv_bfloat16 h = __float2bfloat16_rn(v);
+      dlT[static_cast<size_t>(lane) * ldt + t] = h;
+      dlT[static_cast<size_t>(ec + lane) * ldt + t] = __float2bfloat16_rn(v - __bfloat162float(h));
     }
   }
 }
@@ -347,250 +358,470 @@ bwd_dwg_part(const T* __restrict__ x, const float* __restrict__ dl, int Tn, int 
 }
 
 // ------------------------------------------------ bf16, E <= 16: streaming
-// The two T x d passes of the Mixtral-sized router are pure streams (E
-// multiply-adds per element): dx writes T x d, dWg reads x once. These
-// kernels give each thread 8 consecutive columns (one 16-byte bf16 vector
-// per token row) so that every row of x or dx is touched by whole 16-byte
-// accesses, keep the per-column Wg values or accumulators in registers, and
-// stage each block's d_logits tile in shared memory once.
-constexpr int kFastThreads = 128;   // dx: 128 x 8 = 1024 columns per block
-constexpr int kFastTok = 32;        // dx: tokens per block
-constexpr int kFastDwgThreads = 128;  // dWg: 128 x 8 = 1024 columns per block
-
-__device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float (&v)[8]) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    v[2 * i] = __uint_as_float(w[i] << 16);
-    v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
+// ------------------------------------------------- tensor-core passes (bf16, E <= 16)
+// The two T x d passes are contractions with a short side: dx = dL/dl Wg^T
+// (K = E) and dWg = x^T dL/dl (K = T, N = E). On the tensor cores the bf16
+// operands are exact; d_logits is fp32, so it enters as two bf16 terms,
+// hi = bf16(v) and lo = bf16(v - hi), which together keep 16 bits of it
+// (|v - hi - lo| <= 2^-17 |v|); both products are summed in the fp32
+// accumulator. EC is E rounded up to 8 or 16 (missing experts are zeros);
+// the contraction has 2 EC terms per output: [hi | lo] against [W | W].
+//
+// 128-byte swizzle, K-major (the layout of a TMA SWIZZLE_128B box of
+// 128-byte rows): the 16-byte chunk c of row r sits at
+// (r / 8) * 1024 + (r % 8) * 128 + ((c ^ (r % 8)) * 16).
+__device__ __forceinline__ uint8_t* sw128_chunk(uint8_t* base, int r, int c) {
+  return base + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4);
 }
 
-__device__ __forceinline__ uint4 f32x8_to_bf16(const float (&v)[8]) {
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-    w[i] = *reinterpret_cast<const uint32_t*>(&h);
-  }
-  return make_uint4(w[0], w[1], w[2], w[3]);
+__device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// dx[t, c] = sum_e dl[t, e] Wg[c, e], e in increasing order (the order of
-// bwd_dx). EC >= E (8 or 16); d a multiple of 8. The block's Wg rows
-// [c0, c0 + 1024) are one contiguous range of memory: they are copied to
-// shared memory with 16-byte loads, then each thread keeps its 8 rows in
-// registers; the block's d_logits rows are staged once.
+// hi and lo bf16 terms of 8 fp32 values, packed 8 per 16-byte chunk.
+__device__ __forceinline__ void split_hi_lo8(const float* v, uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float a = v[2 * i], b = v[2 * i + 1];
+    const float ah = __bfloat162float(__float2bfloat16_rn(a));
+    const float bh = __bfloat162float(__float2bfloat16_rn(b));
+    h[i] = pack2_bf16(ah, bh);
+    l[i] = pack2_bf16(a - ah, b - bh);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// EC fp32 values of row t of a [T][E] array (zeros past E or T).
 template <int EC>
-__global__ void __launch_bounds__(kFastThreads)
-bwd_dx_fast(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, int Tn, int d, int E,
-            __nv_bfloat16* __restrict__ dx) {
-  pdl_begin();
-  extern __shared__ __align__(16) uint8_t dx_sm[];
-  __nv_bfloat16* wg_s = reinterpret_cast<__nv_bfloat16*>(dx_sm);                       // [2048][E]
-  float* dl_s = reinterpret_cast<float*>(dx_sm + kFastThreads * 8 * EC * 2);           // [kFastTok][EC]
-  const int c0 = blockIdx.x * kFastThreads * 8;
-  const int ncol = min(kFastThreads * 8, d - c0);
-  const int c = c0 + threadIdx.x * 8;
-  const int t0 = blockIdx.y * kFastTok;
-  {
-    const long long n16 = static_cast<long long>(ncol) * E * 2 / 16;  // a whole number: ncol % 8 == 0
-    const uint4* src = reinterpret_cast<const uint4*>(wg + static_cast<size_t>(c0) * E);
-    for (long long i = threadIdx.x; i < n16; i += kFastThreads)
-      reinterpret_cast<uint4*>(wg_s)[i] = __ldg(src + i);
-  }
-  for (int i = threadIdx.x; i < kFastTok * EC; i += kFastThreads) {
-    const int tt = i / EC, e = i - tt * EC;
-    const int t = t0 + tt;
-    dl_s[i] = (e < E && t < Tn) ? __ldg(dl + static_cast<size_t>(t) * E + e) : 0.f;
-  }
-  __syncthreads();
-  if (c >= d) return;
-  float wv[8][EC];
+__device__ __forceinline__ void load_row(const float* __restrict__ a, int t, int T, int E,
+                                         float (&v)[EC]) {
+  if (t < T && E == EC) {
+    const float4* p = reinterpret_cast<const float4*>(a + static_cast<size_t>(t) * EC);
 #pragma unroll
-  for (int jj = 0; jj < 8; ++jj)
-#pragma unroll
-    for (int e = 0; e < EC; ++e)
-      wv[jj][e] = e < E ? __bfloat162float(wg_s[(threadIdx.x * 8 + jj) * E + e]) : 0.f;
-  const int nt = min(kFastTok, Tn - t0);
-#pragma unroll 4
-  for (int tt = 0; tt < nt; ++tt) {
-    float acc[8];
-#pragma unroll
-    for (int jj = 0; jj < 8; ++jj) acc[jj] = 0.f;
-#pragma unroll
-    for (int e4 = 0; e4 < EC; e4 += 4) {
-      const float4 g4 = *reinterpret_cast<const float4*>(dl_s + tt * EC + e4);
-      const float g[4] = {g4.x, g4.y, g4.z, g4.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) acc[jj] = fmaf(g[q], wv[jj][e4 + q], acc[jj]);
+    for (int i = 0; i < EC / 4; ++i) {
+      const float4 q = __ldg(p + i);
+      v[4 * i] = q.x; v[4 * i + 1] = q.y; v[4 * i + 2] = q.z; v[4 * i + 3] = q.w;
     }
-    *reinterpret_cast<uint4*>(dx + static_cast<size_t>(t0 + tt) * d + c) = f32x8_to_bf16(acc);
+  } else {
+#pragma unroll
+    for (int e = 0; e < EC; ++e) v[e] = (t < T && e < E) ? __ldg(a + static_cast<size_t>(t) * E + e) : 0.f;
   }
 }
 
-size_t dx_fast_smem(int ec) {
-  return static_cast<size_t>(kFastThreads) * 8 * ec * 2 + static_cast<size_t>(kFastTok) * ec * 4;
-}
-
-// dWg partial of token split s: part[s][c][e] = sum over the split's tokens
-// (increasing) of x[t, c] dl[t, e]. EC >= E (8 or 16); d a multiple of 8.
-// Block = G row groups of 128 threads, one block per SM; a group's thread
-// owns 8 columns of the block's 1024 (G = 4 for EC = 8, 2 for EC = 16, so
-// that the accumulators fit). Thread 0 streams the split's rows of that
-// column slice (2 KB per token row) with bulk copies into a 4-stage ring of
-// 16 rows (128 KB in flight per SM, the copy engine's, not registers); group
-// g adds rows g, g + G, ... of each stage. At the end groups 1..G-1 leave
-// their sums in the idle ring and group 0 adds them in group order.
-// Waits are bounded.
-constexpr int kDwgBulkStages = 4;
-constexpr int kDwgBulkRows = 16;
-constexpr int kDwgBulkRowBytes = kFastDwgThreads * 8 * 2;  // 2048
-
-template <int EC>
-struct DwgBulk {
-  static constexpr int G = EC == 8 ? 4 : 2;
-  static constexpr int kThreads = G * kFastDwgThreads;
-};
-
-size_t dwg_bulk_smem(int tps, int ec) {
-  return static_cast<size_t>(kDwgBulkStages) * kDwgBulkRows * kDwgBulkRowBytes + 128 +
-         static_cast<size_t>(tps) * ec * sizeof(float);
-}
+// dx on the tensor cores: tile = 128 tokens x 256 columns, one MMA
+// (M = 128, N = 256, K = 2 EC) per tile; A = [hi | lo] of the tile's d_logits
+// rows, B = [Wg | Wg] of its columns, both written into shared memory by the
+// block's threads (the block's 128 threads hold one token row each, loaded
+// one tile ahead). The 4 warps then read their 32-row quarter of the fp32
+// accumulator from tensor memory, round it to bf16, stage it per warp and
+// store whole 128-byte row segments. Two blocks per SM (the dynamic shared
+// memory is sized so that a third never fits: their accumulators take all
+// 512 tensor-memory columns), so one block's MMA and operand writes overlap
+// the other's stores. Waits are bounded.
+constexpr int kDxTcThreads = 128;
+constexpr int kDxTcTok = 128;
+constexpr int kDxTcCols = 256;
+constexpr int kDxTcA = kDxTcTok * 128;     // 16 KB: 128-byte rows
+constexpr int kDxTcB = kDxTcCols * 128;    // 32 KB
+constexpr int kDxStageRow = 128 + 16;      // staged output row (16-byte pad: no bank conflicts)
+constexpr int kDxStageWarp = 32 * kDxStageRow;
+constexpr size_t kDxTcSmem = 80 * 1024;
+static_assert(kDxTcA + kDxTcB + 4 * kDxStageWarp + 1024 <= static_cast<int>(kDxTcSmem), "dx smem");
+static_assert(3 * (kDxTcSmem + 1024) > 228 * 1024, "at most two dx blocks per SM");
 
 template <int EC>
-__global__ void __launch_bounds__(DwgBulk<EC>::kThreads, 1)
-bwd_dwg_bulk(const __nv_bfloat16* __restrict__ x, const float* __restrict__ dl, int Tn, int d, int E,
-             int tok_per_split, float* __restrict__ part, Control* ctl) {
+__global__ void __launch_bounds__(kDxTcThreads, 2)
+bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, int T, int d, int E,
+          __nv_bfloat16* __restrict__ dx, Control* ctl) {
   pdl_begin();
-  constexpr int G = DwgBulk<EC>::G, NT = DwgBulk<EC>::kThreads;
-  static_assert(static_cast<size_t>(G - 1) * kFastDwgThreads * 8 * EC * 4 <=
-                    static_cast<size_t>(kDwgBulkStages) * kDwgBulkRows * kDwgBulkRowBytes,
-                "the groups' sums fit in the ring");
-  extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ __align__(8) uint64_t full[kDwgBulkStages], empty[kDwgBulkStages];
-  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm) + 127) & ~uintptr_t(127));
-  float* dls = reinterpret_cast<float*>(ring + kDwgBulkStages * kDwgBulkRows * kDwgBulkRowBytes);
-  const int tid = threadIdx.x;
-  const int grp = tid / kFastDwgThreads, gt = tid - grp * kFastDwgThreads;
-  const int c0 = blockIdx.x * kFastDwgThreads * 8;
-  const int ncol = min(kFastDwgThreads * 8, d - c0);
-  const uint32_t rowb = static_cast<uint32_t>(ncol) * 2;  // a multiple of 16 (d % 8 == 0)
-  const int tb = blockIdx.y * tok_per_split;
-  const int n = max(0, min(Tn, tb + tok_per_split) - tb);
-  const int nstg = (n + kDwgBulkRows - 1) / kDwgBulkRows;
+  static_assert(EC == 8 || EC == 16, "EC");
+  extern __shared__ uint8_t dx_raw[];
+  __shared__ __align__(8) uint64_t mma_bar;
+  __shared__ uint32_t tmem_s;
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dx_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  uint8_t* sa = sm;
+  uint8_t* sb = sm + kDxTcA;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint8_t* stg = sm + kDxTcA + kDxTcB + warp * kDxStageWarp;
   if (tid == 0) {
-    for (int i = 0; i < kDwgBulkStages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], NT);
-    }
+    mbar_init(&mma_bar, 1);
     fence_mbar_init();
   }
-  for (int i = tid; i < n * EC; i += NT) {
-    const int tt = i / EC, e = i - tt * EC;
-    dls[i] = e < E ? __ldg(dl + static_cast<size_t>(tb + tt) * E + e) : 0.f;
+  if (warp == 0) {
+    tmem_alloc(&tmem_s, kDxTcCols);
+    tmem_relinquish();
   }
+  tc_fence_before();
   __syncthreads();
-  auto issue = [&](int st) {
-    const int slot = st % kDwgBulkStages, r0 = st * kDwgBulkRows;
-    const int nr = min(kDwgBulkRows, n - r0);
-    mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nr) * rowb);
-    for (int r = 0; r < nr; ++r)
-      bulk_load(ring + (slot * kDwgBulkRows + r) * kDwgBulkRowBytes,
-                x + static_cast<size_t>(tb + r0 + r) * d + c0, rowb, &full[slot]);
-  };
-  if (tid == 0)
-    for (int st = 0; st < nstg && st < kDwgBulkStages; ++st) issue(st);
-  float acc[8][EC];
+  tc_fence_after();
+  const uint32_t tmem = tmem_s;
+  const uint64_t limit = wait_limit_ns(ctl);
+  const int ntt = (T + kDxTcTok - 1) / kDxTcTok, nct = (d + kDxTcCols - 1) / kDxTcCols;
+  const int total = ntt * nct;
+  constexpr uint32_t kIdesc = make_idesc_bf16(kDxTcTok, kDxTcCols, true);
+  float g[EC];
+  if (static_cast<int>(blockIdx.x) < total) load_row<EC>(dl, (blockIdx.x % ntt) * kDxTcTok + tid, T, E, g);
+  int cur_ct = -1;
+  uint32_t phase = 0;
+  bool pending = false;  // an MMA was issued and not yet waited for
+  for (int u = blockIdx.x; u < total; u += gridDim.x) {
+    const int ct = u / ntt, tt = u - ct * ntt;
+    // A row tid: chunks [hi 0..EC) then [lo 0..EC), 8 values each
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
+    for (int h = 0; h < EC / 8; ++h) {
+      uint4 hi, lo;
+      split_hi_lo8(g + 8 * h, hi, lo);
+      *reinterpret_cast<uint4*>(sw128_chunk(sa, tid, h)) = hi;
+      *reinterpret_cast<uint4*>(sw128_chunk(sa, tid, EC / 8 + h)) = lo;
+    }
+    if (ct != cur_ct) {
+      // B rows = columns c of this tile: [Wg[c, 0..EC) | Wg[c, 0..EC)]
+      for (int r = tid; r < kDxTcCols; r += kDxTcThreads) {
+        const int c = ct * kDxTcCols + r;
+        uint4 w[EC / 8];
+        if (c < d && E == EC) {
+          const uint4* p = reinterpret_cast<const uint4*>(wg + static_cast<size_t>(c) * EC);
 #pragma unroll
-    for (int e = 0; e < EC; ++e) acc[j][e] = 0.f;
-  const bool mine = gt * 8 < ncol;
-  int issued = min(nstg, kDwgBulkStages);
-  bool ok = true;
-  for (int st = 0; st < nstg; ++st) {
-    const int slot = st % kDwgBulkStages;
-    if (!mbar_wait_bounded(&full[slot], static_cast<uint32_t>(st / kDwgBulkStages) & 1u)) {
-      set_error(ctl, MOE_DEVERR_TIMEOUT);
-      ok = false;
+          for (int h = 0; h < EC / 8; ++h) w[h] = __ldg(p + h);
+        } else {
+          uint16_t b[EC];
+#pragma unroll
+          for (int e = 0; e < EC; ++e)
+            b[e] = (c < d && e < E) ? __bfloat16_as_ushort(wg[static_cast<size_t>(c) * E + e]) : 0;
+#pragma unroll
+          for (int h = 0; h < EC / 8; ++h)
+            w[h] = make_uint4(b[8 * h] | (uint32_t(b[8 * h + 1]) << 16), b[8 * h + 2] | (uint32_t(b[8 * h + 3]) << 16),
+                              b[8 * h + 4] | (uint32_t(b[8 * h + 5]) << 16), b[8 * h + 6] | (uint32_t(b[8 * h + 7]) << 16));
+        }
+#pragma unroll
+        for (int h = 0; h < EC / 8; ++h) {
+          *reinterpret_cast<uint4*>(sw128_chunk(sb, r, h)) = w[h];
+          *reinterpret_cast<uint4*>(sw128_chunk(sb, r, EC / 8 + h)) = w[h];
+        }
+      }
+      cur_ct = ct;
+    }
+    fence_proxy_async_smem();  // the generic-proxy writes above, before the MMA reads them
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+      const uint32_t a_addr = smem_u32(sa), b_addr = smem_u32(sb);
+#pragma unroll
+      for (int kk = 0; kk < 2 * EC / 16; ++kk)
+        umma_bf16(tmem, make_sw128_desc(a_addr + kk * 32, 16, 1024),
+                  make_sw128_desc(b_addr + kk * 32, 16, 1024), kIdesc, kk > 0 ? 1u : 0u);
+      umma_commit(&mma_bar);
+    }
+    pending = true;
+    // the next tile's d_logits rows are in flight during this tile's stores
+    const int un = u + gridDim.x;
+    if (un < total) load_row<EC>(dl, (un % ntt) * kDxTcTok + tid, T, E, g);
+    int ok = 0;
+    if (lane == 0) ok = mbar_wait_bounded(&mma_bar, phase, limit);
+    ok = __shfl_sync(kFull, ok, 0);
+    if (!__syncthreads_and(ok)) {
+      if (tid == 0) set_error(ctl, MOE_DEVERR_TIMEOUT);
       break;
     }
-    const int nr = min(kDwgBulkRows, n - st * kDwgBulkRows);
-    if (mine) {
-      const uint8_t* rows = ring + slot * kDwgBulkRows * kDwgBulkRowBytes + gt * 16;
-#pragma unroll 2
-      for (int r = grp; r < nr; r += G) {
-        float xv[8];
-        bf16x8_to_f32(*reinterpret_cast<const uint4*>(rows + r * kDwgBulkRowBytes), xv);
-        const float* g = dls + (st * kDwgBulkRows + r) * EC;
+    pending = false;
+    phase ^= 1u;
+    tc_fence_after();
+    const long long t0 = static_cast<long long>(tt) * kDxTcTok + warp * 32;
+    const int nrows = static_cast<int>(max(0LL, min(32LL, T - t0)));
+    const int c0 = ct * kDxTcCols;
+    const int ncols = min(kDxTcCols, d - c0);
+    const uint32_t tq = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    if (nrows > 0) {
+      for (int gc = 0; gc < ncols; gc += 64) {
+        uint32_t v0[32], v1[32];
+        tmem_ld_32x32b_x32(tq + gc, v0);
+        tmem_ld_32x32b_x32(tq + gc + 32, v1);
+        tmem_ld_wait();
+        uint4* sp = reinterpret_cast<uint4*>(stg + lane * kDxStageRow);
 #pragma unroll
-        for (int e = 0; e < EC; ++e) {
-          const float ge = g[e];
+        for (int i = 0; i < 4; ++i) {
+          sp[i] = make_uint4(pack2_bf16(__uint_as_float(v0[8 * i]), __uint_as_float(v0[8 * i + 1])),
+                             pack2_bf16(__uint_as_float(v0[8 * i + 2]), __uint_as_float(v0[8 * i + 3])),
+                             pack2_bf16(__uint_as_float(v0[8 * i + 4]), __uint_as_float(v0[8 * i + 5])),
+                             pack2_bf16(__uint_as_float(v0[8 * i + 6]), __uint_as_float(v0[8 * i + 7])));
+          sp[4 + i] = make_uint4(pack2_bf16(__uint_as_float(v1[8 * i]), __uint_as_float(v1[8 * i + 1])),
+                                 pack2_bf16(__uint_as_float(v1[8 * i + 2]), __uint_as_float(v1[8 * i + 3])),
+                                 pack2_bf16(__uint_as_float(v1[8 * i + 4]), __uint_as_float(v1[8 * i + 5])),
+                                 pack2_bf16(__uint_as_float(v1[8 * i + 6]), __uint_as_float(v1[8 * i + 7])));
+        }
+        __syncwarp();
+        const int cq = lane & 7, rsub = lane >> 3;
+        const bool col_ok = gc + cq * 8 < ncols;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) acc[j][e] = fmaf(xv[j], ge, acc[j][e]);
+        for (int it = 0; it < 8; ++it) {
+          const int rr = it * 4 + rsub;
+          if (rr < nrows && col_ok)
+            *reinterpret_cast<uint4*>(dx + static_cast<size_t>(t0 + rr) * d + c0 + gc + cq * 8) =
+                *reinterpret_cast<const uint4*>(stg + rr * kDxStageRow + cq * 16);
+        }
+        __syncwarp();
+      }
+    }
+    tc_fence_before();  // this tile's tensor-memory reads, before the next tile's barrier and MMA
+  }
+  if (pending && tid == 0) (void)mbar_wait_bounded(&mma_bar, phase, limit);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kDxTcCols);
+  }
+}
+
+// dWg on the tensor cores, per 128-column tile of x: D[c, n] = sum_t x[t, c]
+// B[t, n] with A = x^T (M = 128 columns, MN-major: the rows of x as TMA
+// loads them) and B = the bf16 terms of d_logits, [hi | lo] (N = 2 EC,
+// K-major: the transposed copy dlT [2 EC][T] that bwd_logits writes). A unit
+// is one 128-column tile x 64 tokens (16 KB of x); units are ordered tile by
+// tile, tokens fastest, and every block takes the same number L of
+// consecutive units (the last fewer), so all SMs stream equal shares of x.
+// A block's units fall into one or more column tiles: per tile it sums its
+// units in tensor memory and writes the fp32 sum (hi + lo terms added) as
+// partial i of that tile, i = its rank among the tile's blocks. The last of
+// a tile's blocks to finish (a ticket per tile and 32-column quarter, zeroed
+// by bwd_logits) adds the tile's partials in order i = 0, 1, ... and writes
+// d_wg: the result does not depend on which block finishes last.
+//
+// Warps: 0 TMA producer (x boxes and the dlT box per unit, 8-stage ring),
+// 1 MMA issuer (4 MMAs of K = 16 per unit, double-buffered accumulator),
+// 2..5 epilogue (tensor-memory lane quarter = warp % 4). Waits are bounded.
+constexpr int kDwgTcThreads = 192;
+constexpr int kDwgTcStages = 8;
+constexpr int kDwgTcCols = 128;
+constexpr int kDwgTcTok = 64;
+constexpr int kDwgMaxContrib = 32;  // partials per column tile (the host keeps L large enough)
+
+template <int EC>
+struct DwgTc {
+  static constexpr int N = 2 * EC;
+  static constexpr int A_BYTES = kDwgTcCols * kDwgTcTok * 2;  // two 64-column boxes
+  static constexpr int B_BYTES = N * kDwgTcTok * 2;
+  static constexpr int STAGE = A_BYTES + B_BYTES;              // a multiple of 1024
+  static constexpr size_t SMEM = static_cast<size_t>(kDwgTcStages) * STAGE + 1024;
+};
+
+template <int EC>
+__global__ void __launch_bounds__(kDwgTcThreads, 1)
+bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmg, int d,
+           int E, int ntb, int total, int L, float* __restrict__ part, int* __restrict__ tickets,
+           float* __restrict__ d_wg, Control* ctl) {
+  pdl_begin();
+  using C = DwgTc<EC>;
+  static_assert(C::STAGE % 1024 == 0, "stage alignment");
+  extern __shared__ uint8_t dwg_raw[];
+  __shared__ __align__(8) uint64_t full[kDwgTcStages], empty[kDwgTcStages];
+  __shared__ __align__(8) uint64_t tfull[2], tempty[2], drain;
+  __shared__ uint32_t tmem_s;
+  __shared__ volatile int abort_s;
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dwg_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u0 = blockIdx.x * L, u1 = min(total, u0 + L);
+  const uint64_t limit = wait_limit_ns(ctl);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kDwgTcStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(&drain, 1);
+    abort_s = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_s, 64);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_s;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tmx);
+      prefetch_tmap(&tmg);
+      int stage = 0;
+      uint32_t phase = 0, issued_mask = 0, last_parity = 0;
+      for (int u = u0; u < u1 && !abort_s; ++u) {
+        const int j = u / ntb, tb = u - j * ntb;
+        if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, limit)) {
+          set_error(ctl, MOE_DEVERR_TIMEOUT);
+          abort_s = 1;
+          break;
+        }
+        uint8_t* sa = sm + stage * C::STAGE;
+        mbar_arrive_expect_tx(&full[stage], C::STAGE);
+        tma_load_2d(sa, &tmx, &full[stage], j * kDwgTcCols, tb * kDwgTcTok);
+        tma_load_2d(sa + C::A_BYTES / 2, &tmx, &full[stage], j * kDwgTcCols + 64, tb * kDwgTcTok);
+        tma_load_2d(sa + C::A_BYTES, &tmg, &full[stage], tb * kDwgTcTok, 0);
+        issued_mask |= 1u << stage;
+        last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == kDwgTcStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      for (int s = 0; s < kDwgTcStages; ++s)
+        if ((issued_mask >> s) & 1u)
+          if (!mbar_wait_bounded(&full[s], (last_parity >> s) & 1u, limit)) set_error(ctl, MOE_DEVERR_TIMEOUT);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // A MN-major (bit 15), B K-major
+      constexpr uint32_t kIdesc = make_idesc_bf16(kDwgTcCols, C::N, true) | (1u << 15);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool issued_any = false;
+      int u = u0;
+      while (u < u1 && !abort_s) {
+        const int j = u / ntb;
+        const int ue = min(u1, (j + 1) * ntb);
+        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, limit)) {
+          set_error(ctl, MOE_DEVERR_TIMEOUT);
+          abort_s = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + acc * 32;
+        const int us = u;
+        bool ok = true;
+        for (; u < ue; ++u) {
+          if (!mbar_wait_bounded(&full[stage], phase, limit)) {
+            set_error(ctl, MOE_DEVERR_TIMEOUT);
+            abort_s = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sm + stage * C::STAGE);
+          const uint32_t b_addr = a_addr + C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < kDwgTcTok / 16; ++kk)
+            umma_bf16(d_tmem, make_sw128_desc(a_addr + kk * 2048, C::A_BYTES / 2, 1024),
+                      make_sw128_desc(b_addr + kk * 32, 16, 1024), kIdesc,
+                      (u != us || kk != 0) ? 1u : 0u);
+          issued_any = true;
+          umma_commit(&empty[stage]);
+          if (++stage == kDwgTcStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (issued_any) {
+        umma_commit(&drain);
+        (void)mbar_wait_bounded(&drain, 0, limit);
+      }
+    }
+  } else {
+    // epilogue warps 2..5: columns 32 q .. 32 q + 31 of each tile
+    const int q = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int u = u0;
+    while (u < u1) {
+      const int j = u / ntb;
+      const int ue = min(u1, (j + 1) * ntb);
+      u = ue;
+      int ok = 0;
+      if (lane == 0) {
+        ok = !abort_s && mbar_wait_bounded(&tfull[acc], acc_phase, limit);
+        if (!ok && !abort_s) {
+          set_error(ctl, MOE_DEVERR_TIMEOUT);
+          abort_s = 1;
+        }
+      }
+      if (!__shfl_sync(kFull, ok, 0)) break;
+      tc_fence_after();
+      float v[EC];
+      {
+        const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * 32;
+        if constexpr (EC == 8) {
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(ta, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[e]) + __uint_as_float(r[8 + e]);
+        } else {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(ta, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(r[e]) + __uint_as_float(r[16 + e]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+      // this block's rank among the tile's blocks, and their number
+      const int first = static_cast<int>((static_cast<long long>(j) * ntb) / L);
+      const int last = static_cast<int>((static_cast<long long>(j + 1) * ntb - 1) / L);
+      const int i = blockIdx.x - first, n = last - first + 1;
+      const int r = q * 32 + lane;
+      float* mine = part + ((static_cast<size_t>(j) * kDwgMaxContrib + i) * kDwgTcCols + r) * EC;
+#pragma unroll
+      for (int e = 0; e < EC; e += 4)
+        *reinterpret_cast<float4*>(mine + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+      __threadfence();
+      __syncwarp();
+      int prev = 0;
+      if (lane == 0) prev = atomicAdd(tickets + j * 4 + q, 1);
+      prev = __shfl_sync(kFull, prev, 0);
+      if (prev == n - 1) {
+        __threadfence();
+        const int c = j * kDwgTcCols + r;
+        float sum[EC];
+#pragma unroll
+        for (int e = 0; e < EC; ++e) sum[e] = 0.f;
+        for (int k = 0; k < n; ++k) {
+          const float4* src = reinterpret_cast<const float4*>(
+              part + ((static_cast<size_t>(j) * kDwgMaxContrib + k) * kDwgTcCols + r) * EC);
+#pragma unroll
+          for (int e4 = 0; e4 < EC / 4; ++e4) {
+            const float4 t4 = __ldcg(src + e4);
+            sum[4 * e4] += t4.x;
+            sum[4 * e4 + 1] += t4.y;
+            sum[4 * e4 + 2] += t4.z;
+            sum[4 * e4 + 3] += t4.w;
+          }
+        }
+        if (c < d) {
+#pragma unroll
+          for (int e = 0; e < EC; ++e)
+            if (e < E) d_wg[static_cast<size_t>(c) * E + e] = sum[e];
         }
       }
     }
-    mbar_arrive(&empty[slot]);
-    if (tid == 0 && issued < nstg) {
-      // the slot is free once every thread has read this stage
-      if (!mbar_wait_bounded(&empty[slot], static_cast<uint32_t>(st / kDwgBulkStages) & 1u)) {
-        set_error(ctl, MOE_DEVERR_TIMEOUT);
-        ok = false;
-        break;
-      }
-      issue(issued);
-      ++issued;
-    }
   }
-  if (tid == 0) {
-    // every copy issued must have landed before the ring is reused or the
-    // block leaves: wait for the last stage issued into each slot
-    for (int slot = 0; slot < kDwgBulkStages && slot < issued; ++slot) {
-      const int last = slot + ((issued - 1 - slot) / kDwgBulkStages) * kDwgBulkStages;
-      if (!mbar_wait_bounded(&full[slot], static_cast<uint32_t>(last / kDwgBulkStages) & 1u))
-        set_error(ctl, MOE_DEVERR_TIMEOUT);
-    }
-  }
-  __syncthreads();  // every thread is done with the ring: it holds the groups' sums now
-  float* red = reinterpret_cast<float*>(ring);  // [G - 1][128 threads][8][EC]
-  if (grp > 0 && mine) {
-    float* dst = red + (static_cast<size_t>(grp - 1) * kFastDwgThreads + gt) * 8 * EC;
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int e = 0; e < EC; e += 4)
-        *reinterpret_cast<float4*>(dst + j * EC + e) =
-            make_float4(acc[j][e], acc[j][e + 1], acc[j][e + 2], acc[j][e + 3]);
-  }
+  tc_fence_before();
   __syncthreads();
-  if (grp != 0 || !mine || !ok) return;
-#pragma unroll
-  for (int q = 1; q < G; ++q) {
-    const float* src = red + (static_cast<size_t>(q - 1) * kFastDwgThreads + gt) * 8 * EC;
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int e = 0; e < EC; ++e) acc[j][e] += src[j * EC + e];
-  }
-  // the 8 columns' E values are 8 * E consecutive floats of the partial
-  float* dst = part + (static_cast<size_t>(blockIdx.y) * d + c0 + gt * 8) * E;
-  if (E == EC) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int e = 0; e < EC; e += 4)
-        *reinterpret_cast<float4*>(dst + j * EC + e) =
-            make_float4(acc[j][e], acc[j][e + 1], acc[j][e + 2], acc[j][e + 3]);
-  } else {
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int e = 0; e < EC; ++e)
-        if (e < E) dst[j * E + e] = acc[j][e];
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
   }
 }
 
@@ -616,11 +847,29 @@ int dwg_splits(int T, int d, int E) {
   return s < 1 ? 1 : s;
 }
 
+// Tensor-core dWg (E <= 16): partials [column tile][kDwgMaxContrib][128][EC],
+// the transposed bf16 terms dlT [32][ldt] and the tickets [column tile][4].
+int dwg_tc_ec(int E) { return E <= 8 ? 8 : 16; }
+long long dlt_ld(int T) { return (static_cast<long long>(T) + 7) / 8 * 8; }
+int dwg_tc_tiles(int d) { return (d + kDwgTcCols - 1) / kDwgTcCols; }
+size_t dwg_tc_part_bytes(int d, int E) {
+  return static_cast<size_t>(dwg_tc_tiles(d)) * kDwgMaxContrib * kDwgTcCols * dwg_tc_ec(E) * 4;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 }  // namespace
 
 size_t route_backward_scratch_bytes(int T, int d, int E) {
+  size_t part = static_cast<size_t>(dwg_splits(T, d, E)) * d * E * 4;
+  size_t extra = 0;
+  if (E <= 16) {
+    part = std::max(part, dwg_tc_part_bytes(d, E));
+    extra = align_up(static_cast<size_t>(32) * dlt_ld(T) * 2) +
+            align_up(static_cast<size_t>(dwg_tc_tiles(d)) * 4 * 4);
+  }
   return align_up(static_cast<size_t>(E) * 4) + align_up(static_cast<size_t>(T) * E * 4) +
-         align_up(static_cast<size_t>(dwg_splits(T, d, E)) * d * E * 4);
+         align_up(part) + extra;
 }
 
 cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt, int T, int d,
@@ -635,15 +884,23 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
   float* dl = d_logits != nullptr ? d_logits : reinterpret_cast<float*>(sc);
   sc += align_up(static_cast<size_t>(T) * E * 4);
   float* part = reinterpret_cast<float*>(sc);
+  size_t part_bytes = static_cast<size_t>(dwg_splits(T, d, E)) * d * E * 4;
+  if (E <= 16) part_bytes = std::max(part_bytes, dwg_tc_part_bytes(d, E));
+  sc += align_up(part_bytes);
+  __nv_bfloat16* dlT = nullptr;
+  int* tickets = nullptr;
+  if (E <= 16) {
+    dlT = reinterpret_cast<__nv_bfloat16*>(sc);
+    sc += align_up(static_cast<size_t>(32) * dlt_ld(T) * 2);
+    tickets = reinterpret_cast<int*>(sc);
+  }
   const float inv_tau = 1.0f / temperature;
   const bool aux = d_aux != 0.0f;
-  // bf16 with at most 16 experts: the streaming kernels (16-byte row access;
-  // dWg through the bulk-copy ring while a split's d_logits fit beside it)
-  const bool fast = dt == MOE_BF16 && E <= 16 && d % 8 == 0;
-  const int fxb = (d + kFastDwgThreads * 8 - 1) / (kFastDwgThreads * 8);
-  const int fns = std::max(1, std::min(dwg_splits(T, d, E), num_sms() / fxb));
-  const int ftps = T > 0 ? (T + fns - 1) / fns : 0;
-  const bool fast_dwg = fast && dwg_bulk_smem(std::max(ftps, 1), E <= 8 ? 8 : 16) <= 200 * 1024;
+  // bf16 with at most 16 experts: both T x d passes on the tensor cores
+  const bool tc = dt == MOE_BF16 && E <= 16 && d % 8 == 0 && T > 0 && aligned16(x) &&
+                  aligned16(wg) && aligned16(dl);
+  const int ec = dwg_tc_ec(E);
+  const bool tc_dwg = tc && d_wg != nullptr;
   cudaError_t err = cudaSuccess;
   if (T > 0) {
     if (aux) {
@@ -657,15 +914,16 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
     const int grid = std::max(1, std::min((T + kLogitWarps - 1) / kLogitWarps, 8 * num_sms()));
     err = launch_pdl(kern, dim3(grid), dim3(kLogitWarps * 32), 0, s, false, probs,
                      d_z != 0.0f ? logits : nullptr, idx, w, d_w, aux ? counts : nullptr, d_aux,
-                     d_z, inv_tau, T, E, k, dl, ctl);
+                     d_z, inv_tau, T, E, k, dl, tc_dwg ? dlT : nullptr, ec, static_cast<int>(dlt_ld(T)),
+                     tc_dwg ? tickets : nullptr, dwg_tc_tiles(d) * 4, ctl);
     if (err != cudaSuccess) return err;
-    if (dx != nullptr && fast) {
-      const dim3 g((d + kFastThreads * 8 - 1) / (kFastThreads * 8), (T + kFastTok - 1) / kFastTok);
-      auto kern = E <= 8 ? bwd_dx_fast<8> : bwd_dx_fast<16>;
-      const size_t dsm = dx_fast_smem(E <= 8 ? 8 : 16);
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dsm));
-      err = launch_pdl(kern, g, dim3(kFastThreads), dsm, s, false, static_cast<const float*>(dl),
-                       static_cast<const __nv_bfloat16*>(wg), T, d, E, static_cast<__nv_bfloat16*>(dx));
+    if (dx != nullptr && tc) {
+      const int tiles = ((T + kDxTcTok - 1) / kDxTcTok) * ((d + kDxTcCols - 1) / kDxTcCols);
+      auto kern = ec == 8 ? bwd_dx_tc<8> : bwd_dx_tc<16>;
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kDxTcSmem));
+      err = launch_pdl(kern, dim3(std::min(tiles, 2 * num_sms())), dim3(kDxTcThreads), kDxTcSmem, s, false,
+                       static_cast<const float*>(dl), static_cast<const __nv_bfloat16*>(wg), T, d, E,
+                       static_cast<__nv_bfloat16*>(dx), ctl);
       if (err != cudaSuccess) return err;
     } else if (dx != nullptr) {
       const int tiles = E <= kDxE ? kDxTiles : 1;
@@ -679,22 +937,25 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
       if (err != cudaSuccess) return err;
     }
   }
-  if (d_wg != nullptr && fast_dwg) {
-    // one block per SM: the column slices times the token splits
-    const int xb = fxb, ns = fns, tps = ftps;
-    const int ec = E <= 8 ? 8 : 16;
-    const size_t smem = dwg_bulk_smem(std::max(tps, 1), ec);
-    auto kern = ec == 8 ? bwd_dwg_bulk<8> : bwd_dwg_bulk<16>;
+  if (tc_dwg) {
+    // equal shares of 64-token x 128-column units; L keeps a tile's blocks <= kDwgMaxContrib
+    const int ntb = (T + kDwgTcTok - 1) / kDwgTcTok;
+    const int nct = dwg_tc_tiles(d);
+    const long long total = static_cast<long long>(ntb) * nct;
+    if (total > 0x7fffffffLL) return cudaErrorInvalidValue;
+    long long L = (total + num_sms() - 1) / num_sms();
+    L = std::max<long long>(L, (ntb + kDwgMaxContrib - 2) / (kDwgMaxContrib - 1));
+    const int G = static_cast<int>((total + L - 1) / L);
+    CUtensorMap tmx, tmg;
+    if (!make_tma_2d_bf16(&tmx, x, static_cast<uint64_t>(T), static_cast<uint64_t>(d), kDwgTcTok) ||
+        !make_tma_2d_bf16_ld(&tmg, dlT, static_cast<uint64_t>(2 * ec), static_cast<uint64_t>(T),
+                             static_cast<uint64_t>(dlt_ld(T)), static_cast<uint32_t>(2 * ec)))
+      return cudaErrorInvalidValue;
+    const size_t smem = ec == 8 ? DwgTc<8>::SMEM : DwgTc<16>::SMEM;
+    auto kern = ec == 8 ? bwd_dwg_tc<8> : bwd_dwg_tc<16>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    const int nthr = ec == 8 ? DwgBulk<8>::kThreads : DwgBulk<16>::kThreads;
-    err = launch_pdl(kern, dim3(xb, ns), dim3(nthr), smem, s, false,
-                     static_cast<const __nv_bfloat16*>(x), static_cast<const float*>(dl), T, d, E, tps,
-                     part, ctl);
-    if (err != cudaSuccess) return err;
-    const long long n = static_cast<long long>(d) * E;
-    const int rg = static_cast<int>(std::min<long long>((n + 255) / 256, 8LL * num_sms()));
-    err = launch_pdl(bwd_dwg_reduce, dim3(std::max(rg, 1)), dim3(256), 0, s, false,
-                     static_cast<const float*>(part), ns, n, d_wg);
+    err = launch_pdl(kern, dim3(G), dim3(kDwgTcThreads), smem, s, false, tmx, tmg, d, E, ntb,
+                     static_cast<int>(total), static_cast<int>(L), part, tickets, d_wg, ctl);
   } else if (d_wg != nullptr) {
     const int ns = dwg_splits(T, d, E);
     const int tps = T > 0 ? (T + ns - 1) / ns : 0;

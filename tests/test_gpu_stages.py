@@ -461,9 +461,11 @@ def test_route_train_at_unit_temperature_is_route(T, d, E, k, dt):
     (129, 256, 256, 8, "bf16", 1.0, 0.05, 0.01),    # E = 256, k = 8
     (300, 512, 24, 3, "bf16", 2.0, 0.0, 0.1),       # E not a multiple of 32, no aux term
     (200, 64, 40, 4, "f32", 1.0, 0.3, 0.05),        # fp32 (dx in fp32)
-    (64, 384, 16, 4, "bf16", 1.0, 0.1, 0.01),       # streaming kernels, E = 16, a partial column slice
-    (5, 256, 12, 2, "bf16", 1.0, 0.2, 0.0),         # five tokens, E = 12
-    (2500, 2048, 8, 2, "bf16", 1.3, 0.01, 0.001),   # many token splits, a partial last ring stage
+    (64, 384, 16, 4, "bf16", 1.0, 0.1, 0.01),       # tensor-core passes, E = 16, a half-width dx column tile
+    (5, 256, 12, 2, "bf16", 1.0, 0.2, 0.0),         # five tokens, E = 12 (zero expert columns)
+    (2500, 2048, 8, 2, "bf16", 1.3, 0.01, 0.001),   # dWg tiles shared by several blocks, a ragged last unit
+    (333, 128, 5, 2, "bf16", 1.0, 0.1, 0.01),       # one column tile, E = 5, a ragged last unit
+    (4100, 256, 16, 3, "bf16", 0.8, 0.05, 0.0),     # 2 column tiles x 65 units: 22 blocks per tile
 ])
 def test_route_backward(T, d, E, k, dt, tau, d_aux, d_z):
     """moe_route_backward from the GPU's own forward (moe_route_train at tau)
