@@ -161,6 +161,50 @@ __device__ __forceinline__ void pdl_begin() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+__device__ __forceinline__ uint64_t globaltimer_ns_c() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Barrier over all blocks of a cooperatively launched grid (every block is
+// resident), through bar_count / bar_gen of the control block: the last block
+// to arrive resets the count and bumps the generation. The spin is bounded by
+// the control block's wait limit; a time-out sets MOE_DEVERR_TIMEOUT and
+// returns false in every thread of the block.
+__device__ __forceinline__ bool grid_barrier(Control* ctl, unsigned nblocks) {
+  __shared__ int ok_s;
+  __threadfence();  // this thread's global writes are visible before the block arrives
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    __threadfence();
+    volatile unsigned* gen_p = &ctl->bar_gen;
+    const unsigned gen = *gen_p;
+    const unsigned arrived = atomicAdd(&ctl->bar_count, 1u);
+    if (arrived == nblocks - 1) {
+      ctl->bar_count = 0u;
+      __threadfence();
+      atomicAdd(&ctl->bar_gen, 1u);
+    } else {
+      const uint64_t limit = wait_limit_ns(ctl);
+      const uint64_t t0 = globaltimer_ns_c();
+      while (*gen_p == gen) {
+        if (globaltimer_ns_c() - t0 > limit) {
+          set_error(ctl, MOE_DEVERR_TIMEOUT);
+          ok = 0;
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __threadfence();
+    ok_s = ok;
+  }
+  __syncthreads();
+  return ok_s != 0;
+}
+
 // Counts every kernel this library launches (moe_kernel_launches reads it).
 void note_launch();
 

@@ -22,16 +22,6 @@
 #include <climits>
 
 namespace moe {
-namespace {
-__device__ __forceinline__ uint64_t globaltimer_ns_p() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-}  // namespace
-}  // namespace moe
-
-namespace moe {
 
 namespace {
 
@@ -195,38 +185,6 @@ permute_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_mask,
 constexpr int kGThreads = 256;
 constexpr int kGMaxChunk = 4096;
 
-__device__ bool grid_barrier(Control* ctl, unsigned nblocks) {
-  __shared__ int ok_s;
-  __threadfence();  // this thread's global writes are visible before the block arrives
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int ok = 1;
-    __threadfence();
-    volatile unsigned* gen_p = &ctl->bar_gen;
-    const unsigned gen = *gen_p;
-    const unsigned arrived = atomicAdd(&ctl->bar_count, 1u);
-    if (arrived == nblocks - 1) {
-      ctl->bar_count = 0u;
-      __threadfence();
-      atomicAdd(&ctl->bar_gen, 1u);
-    } else {
-      const uint64_t limit = wait_limit_ns(ctl);
-      const uint64_t t0 = globaltimer_ns_p();
-      while (*gen_p == gen) {
-        if (globaltimer_ns_p() - t0 > limit) {
-          set_error(ctl, MOE_DEVERR_TIMEOUT);
-          ok = 0;
-          break;
-        }
-        __nanosleep(64);
-      }
-    }
-    __threadfence();
-    ok_s = ok;
-  }
-  __syncthreads();
-  return ok_s != 0;
-}
 
 __global__ void __launch_bounds__(kGThreads)
 permute_grid_kernel(const int32_t* __restrict__ idx, int S, int E, unsigned key_mask,

@@ -56,7 +56,10 @@ bwd_hist(const int32_t* __restrict__ idx, long long S, int E, int32_t* __restric
 
 constexpr int kLogitWarps = 8;
 
-// Warp per token; lane holds experts lane + 32 q, q < EPL.
+// Warp per token; lane holds experts lane + 32 q, q < EPL. The short per-lane
+// chains and a grid over every SM suit small T (counts from bwd_hist first);
+// with dlT set (E <= 16) it also writes the bf16 terms of d_logits for the
+// tensor-core dWg, and block 0 zeroes dWg's tickets.
 template <int EPL>
 __global__ void __launch_bounds__(kLogitWarps * 32)
 bwd_logits(const float* __restrict__ probs, const float* __restrict__ logits,
@@ -154,13 +157,211 @@ bwd_logits(const float* __restrict__ probs, const float* __restrict__ logits,
       if (e < E) d_logits[row + e] = dl[q];
     }
     if (dlT != nullptr && lane < ec) {
-      // the tensor-core dWg's B operand: rows [hi 0..ec) then [lo 0..ec),
-      // tokens along the rows (E <= 16, so EPL == 1 and lane = expert)
+      // the tensor-core dWg's B operand (E <= 16, so EPL == 1 and lane =
+      // expert): dlT[e][t] = hi, dlT[ec + e][t] = lo
       const float v = lane < E ? dl[0] : 0.f;
       const __nv_bfloat16 h = __float2bfloat16_rn(v);
       dlT[static_cast<size_t>(lane) * ldt + t] = h;
       dlT[static_cast<size_t>(ec + lane) * ldt + t] = __float2bfloat16_rn(v - __bfloat162float(h));
     }
+  }
+}
+
+// EC fp32 values of row t of a [T][E] array (t < T), zeros past E; one or
+// more 16-byte loads when E == EC (rows 16-byte aligned).
+template <int EC>
+__device__ __forceinline__ void load_row_f32(const float* __restrict__ a, long long t, int E, float (&v)[EC]) {
+  if (E == EC) {
+    const float4* p = reinterpret_cast<const float4*>(a + t * EC);
+#pragma unroll
+    for (int i = 0; i < EC / 4; ++i) {
+      const float4 q = __ldg(p + i);
+      v[4 * i] = q.x; v[4 * i + 1] = q.y; v[4 * i + 2] = q.z; v[4 * i + 3] = q.w;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < EC; ++e) v[e] = e < E ? __ldg(a + t * E + e) : 0.f;
+  }
+}
+
+// d_logits with a thread per token, for large T (E <= 16, k <= 8; EC = 8
+// or 16 register slots, zeros past E): the token's probabilities, logits,
+// picks, weights and upstream gradients are loaded together as whole rows, so
+// a thread waits on memory once and every load of a warp is one contiguous
+// range. With the aux term (count) each block first counts its own tokens'
+// picks (per-lane 8-bit counters packed four to a word, flushed before they
+// can carry, then one warp reduction per expert) and publishes them; after
+// one grid barrier (cooperative launch: every block is resident; the wait is
+// bounded) every block adds all blocks' counts in block order, so no separate
+// histogram launch is needed. With dlT set it also writes the bf16 terms of
+// d_logits, transposed, for the tensor-core dWg: dlT[e][t] = hi,
+// dlT[EC + e][t] = lo (consecutive tokens: coalesced), and block 0 zeroes
+// dWg's tickets.
+constexpr int kTptThreads = 256;
+constexpr int kTptMaxBlocks = 1024;        // hist_part holds kTptMaxBlocks x 16 counts
+constexpr int kTptMaxK = 8;
+constexpr long long kTptMinPicks = 16384;  // below this many picks the warp kernels are faster
+
+// one lane's picks into 8-bit counters, four experts per word
+template <int EC>
+__device__ __forceinline__ void tally(int e, int E, Control* ctl, uint32_t (&pk)[EC / 4]) {
+  if (e < 0 || e >= E) {
+    set_error(ctl, MOE_DEVERR_EXPERT_RANGE);
+    return;
+  }
+  const uint32_t inc = 1u << ((e & 3) * 8);
+#pragma unroll
+  for (int q = 0; q < EC / 4; ++q) pk[q] += (e >> 2) == q ? inc : 0u;
+}
+
+template <int EC>
+__global__ void __launch_bounds__(kTptThreads)
+bwd_logits_tpt(const float* __restrict__ probs, const float* __restrict__ logits,
+               const int32_t* __restrict__ idx, const float* __restrict__ w,
+               const float* __restrict__ d_w, int count, int32_t* __restrict__ hist_part,
+               float d_aux, float d_z, float inv_tau, int T, int E, int k,
+               float* __restrict__ d_logits, __nv_bfloat16* __restrict__ dlT, int ldt,
+               int* __restrict__ tickets, int ntickets, Control* ctl) {
+  pdl_begin();
+  __shared__ int h_s[EC];
+  __shared__ float aux_s[EC];
+  const int tid = threadIdx.x, lane = tid & 31;
+  if (tickets != nullptr && blockIdx.x == 0)
+    for (int i = tid; i < ntickets; i += kTptThreads) tickets[i] = 0;
+  if (tid < EC) {
+    h_s[tid] = 0;
+    aux_s[tid] = 0.f;
+  }
+  const long long stride = static_cast<long long>(gridDim.x) * kTptThreads;
+  long long t = static_cast<long long>(blockIdx.x) * kTptThreads + tid;
+  // the current token's inputs, loaded before they are needed
+  float ip[EC], ilt[EC], ig[kTptMaxK], iw[kTptMaxK];
+  int ie[kTptMaxK];
+  auto load = [&](long long u) {
+    load_row_f32<EC>(probs, u, E, ip);
+    if (logits != nullptr) load_row_f32<EC>(logits, u, E, ilt);
+#pragma unroll
+    for (int j = 0; j < kTptMaxK; ++j) {
+      const bool on = d_w != nullptr && j < k;
+      ie[j] = on ? __ldg(idx + u * k + j) : 0;
+      ig[j] = on ? __ldg(d_w + u * k + j) : 0.f;
+      iw[j] = on ? __ldg(w + u * k + j) : 0.f;
+    }
+  };
+  if (t < T) load(t);
+  __syncthreads();
+  if (count) {
+    uint32_t pk[EC / 4];
+#pragma unroll
+    for (int q = 0; q < EC / 4; ++q) pk[q] = 0u;
+    // this block's tokens: at most 255 picks per lane between flushes
+    int n_since = 0;
+    for (long long u = t; u < T; u += stride) {
+      for (int j = 0; j < k; ++j) tally<EC>(__ldg(idx + u * k + j), E, ctl, pk);
+      n_since += k;
+      if (n_since > 255 - kTptMaxK) {
+#pragma unroll
+        for (int e = 0; e < EC; ++e) {
+          const uint32_t c = (pk[e >> 2] >> ((e & 3) * 8)) & 0xffu;
+          if (c != 0) atomicAdd(&h_s[e], static_cast<int>(c));
+        }
+#pragma unroll
+        for (int q = 0; q < EC / 4; ++q) pk[q] = 0u;
+        n_since = 0;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < EC; ++e) {
+      const unsigned c = __reduce_add_sync(kFull, (pk[e >> 2] >> ((e & 3) * 8)) & 0xffu);
+      if (lane == 0 && c != 0) atomicAdd(&h_s[e], static_cast<int>(c));
+    }
+    __syncthreads();
+    if (tid < EC) hist_part[static_cast<size_t>(blockIdx.x) * EC + tid] = h_s[tid];
+    if (!grid_barrier(ctl, gridDim.x)) return;
+    if (tid < EC) {
+      int n = 0;
+      for (unsigned b = 0; b < gridDim.x; ++b) n += __ldcg(hist_part + static_cast<size_t>(b) * EC + tid);
+      h_s[tid] = n;
+    }
+    __syncthreads();
+    // the aux term is the same for every token: d_aux * E * f_e / T
+    if (tid < EC)
+      aux_s[tid] = tid < E ? d_aux * static_cast<float>(E) *
+                                 (static_cast<float>(h_s[tid]) / (static_cast<float>(T) * k)) /
+                                 static_cast<float>(T)
+                           : 0.f;
+    __syncthreads();
+  }
+  const float zc = d_z * 2.0f / static_cast<float>(T);
+  while (t < T) {
+    float dp[EC];
+#pragma unroll
+    for (int e = 0; e < EC; ++e) dp[e] = aux_s[e];
+    if (d_w != nullptr) {
+      float s = 0.f, gw = 0.f;
+#pragma unroll
+      for (int j = 0; j < kTptMaxK; ++j) {
+        if (j < k) {
+          if (ie[j] < 0 || ie[j] >= E) {
+            set_error(ctl, MOE_DEVERR_EXPERT_RANGE);
+            ie[j] = 0;
+          }
+          float pj = 0.f;
+#pragma unroll
+          for (int ee = 0; ee < EC; ++ee) pj = ee == ie[j] ? ip[ee] : pj;
+          s += pj;
+          gw += ig[j] * iw[j];
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kTptMaxK; ++j) {
+        if (j < k) {
+          const float v = (ig[j] - gw) / s;
+#pragma unroll
+          for (int ee = 0; ee < EC; ++ee) dp[ee] += ee == ie[j] ? v : 0.f;
+        }
+      }
+    }
+    float c = 0.f;
+#pragma unroll
+    for (int e = 0; e < EC; ++e) c += ip[e] * dp[e];
+    float dl[EC];
+#pragma unroll
+    for (int e = 0; e < EC; ++e) dl[e] = ip[e] * (dp[e] - c) * inv_tau;
+    if (logits != nullptr) {  // z-loss term: lse of l / tau
+      float m = -INFINITY, lt[EC];
+#pragma unroll
+      for (int e = 0; e < EC; ++e) {
+        lt[e] = e < E ? ilt[e] * inv_tau : -INFINITY;
+        m = fmaxf(m, lt[e]);
+      }
+      float se = 0.f;
+#pragma unroll
+      for (int e = 0; e < EC; ++e) se += e < E ? expf(lt[e] - m) : 0.f;
+      const float lse = m + logf(se);
+#pragma unroll
+      for (int e = 0; e < EC; ++e) dl[e] += zc * lse * ip[e] * inv_tau;
+    }
+    if (E == EC) {
+      float4* o = reinterpret_cast<float4*>(d_logits + t * EC);
+#pragma unroll
+      for (int i = 0; i < EC / 4; ++i) o[i] = make_float4(dl[4 * i], dl[4 * i + 1], dl[4 * i + 2], dl[4 * i + 3]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < EC; ++e)
+        if (e < E) d_logits[t * E + e] = dl[e];
+    }
+    if (dlT != nullptr) {
+#pragma unroll
+      for (int e = 0; e < EC; ++e) {
+        const float v = e < E ? dl[e] : 0.f;
+        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+        dlT[static_cast<size_t>(e) * ldt + t] = h;
+        dlT[static_cast<size_t>(EC + e) * ldt + t] = __float2bfloat16_rn(v - __bfloat162float(h));
+      }
+    }
+    t += stride;
+    if (t < T) load(t);
   }
 }
 
@@ -420,7 +621,9 @@ __device__ __forceinline__ void load_row(const float* __restrict__ a, int t, int
 // store whole 128-byte row segments. Two blocks per SM (the dynamic shared
 // memory is sized so that a third never fits: their accumulators take all
 // 512 tensor-memory columns), so one block's MMA and operand writes overlap
-// the other's stores. Waits are bounded.
+// the other's stores. Tiles are numbered token tile major (u = tt * nct +
+// ct) and the grid is a multiple of nct when it can be, so a block keeps one
+// column tile and writes its B operand once. Waits are bounded.
 constexpr int kDxTcThreads = 128;
 constexpr int kDxTcTok = 128;
 constexpr int kDxTcCols = 256;
@@ -464,12 +667,12 @@ bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, in
   const int total = ntt * nct;
   constexpr uint32_t kIdesc = make_idesc_bf16(kDxTcTok, kDxTcCols, true);
   float g[EC];
-  if (static_cast<int>(blockIdx.x) < total) load_row<EC>(dl, (blockIdx.x % ntt) * kDxTcTok + tid, T, E, g);
+  if (static_cast<int>(blockIdx.x) < total) load_row<EC>(dl, (blockIdx.x / nct) * kDxTcTok + tid, T, E, g);
   int cur_ct = -1;
   uint32_t phase = 0;
   bool pending = false;  // an MMA was issued and not yet waited for
   for (int u = blockIdx.x; u < total; u += gridDim.x) {
-    const int ct = u / ntt, tt = u - ct * ntt;
+    const int tt = u / nct, ct = u - tt * nct;
     // A row tid: chunks [hi 0..EC) then [lo 0..EC), 8 values each
 #pragma unroll
     for (int h = 0; h < EC / 8; ++h) {
@@ -520,7 +723,7 @@ bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, in
     pending = true;
     // the next tile's d_logits rows are in flight during this tile's stores
     const int un = u + gridDim.x;
-    if (un < total) load_row<EC>(dl, (un % ntt) * kDxTcTok + tid, T, E, g);
+    if (un < total) load_row<EC>(dl, (un / nct) * kDxTcTok + tid, T, E, g);
     int ok = 0;
     if (lane == 0) ok = mbar_wait_bounded(&mma_bar, phase, limit);
     ok = __shfl_sync(kFull, ok, 0);
@@ -581,7 +784,7 @@ bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, in
 // dWg on the tensor cores, per 128-column tile of x: D[c, n] = sum_t x[t, c]
 // B[t, n] with A = x^T (M = 128 columns, MN-major: the rows of x as TMA
 // loads them) and B = the bf16 terms of d_logits, [hi | lo] (N = 2 EC,
-// K-major: the transposed copy dlT [2 EC][T] that bwd_logits writes). A unit
+// K-major: the transposed copy dlT [2 EC][T] that bwd_logits_tpt writes). A unit
 // is one 128-column tile x 64 tokens (16 KB of x); units are ordered tile by
 // tile, tokens fastest, and every block takes the same number L of
 // consecutive units (the last fewer), so all SMs stream equal shares of x.
@@ -589,7 +792,7 @@ bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, in
 // units in tensor memory and writes the fp32 sum (hi + lo terms added) as
 // partial i of that tile, i = its rank among the tile's blocks. The last of
 // a tile's blocks to finish (a ticket per tile and 32-column quarter, zeroed
-// by bwd_logits) adds the tile's partials in order i = 0, 1, ... and writes
+// by bwd_logits_tpt) adds the tile's partials in order i = 0, 1, ... and writes
 // d_wg: the result does not depend on which block finishes last.
 //
 // Warps: 0 TMA producer (x boxes and the dlT box per unit, 8-stage ring),
@@ -599,7 +802,9 @@ constexpr int kDwgTcThreads = 192;
 constexpr int kDwgTcStages = 8;
 constexpr int kDwgTcCols = 128;
 constexpr int kDwgTcTok = 64;
-constexpr int kDwgMaxContrib = 32;  // partials per column tile (the host keeps L large enough)
+// Partials per column tile: enough for every SM to share one tile when d is
+// small (2 x 160 SMs' worth), at least 32; the host keeps L large enough.
+__host__ __device__ inline int dwg_max_contrib(int nct) { return max(32, (320 + nct - 1) / nct + 2); }
 
 template <int EC>
 struct DwgTc {
@@ -613,8 +818,8 @@ struct DwgTc {
 template <int EC>
 __global__ void __launch_bounds__(kDwgTcThreads, 1)
 bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmg, int d,
-           int E, int ntb, int total, int L, float* __restrict__ part, int* __restrict__ tickets,
-           float* __restrict__ d_wg, Control* ctl) {
+           int E, int ntb, int total, int L, int maxc, float* __restrict__ part,
+           int* __restrict__ tickets, float* __restrict__ d_wg, Control* ctl) {
   pdl_begin();
   using C = DwgTc<EC>;
   static_assert(C::STAGE % 1024 == 0, "stage alignment");
@@ -782,7 +987,7 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
       const int last = static_cast<int>((static_cast<long long>(j + 1) * ntb - 1) / L);
       const int i = blockIdx.x - first, n = last - first + 1;
       const int r = q * 32 + lane;
-      float* mine = part + ((static_cast<size_t>(j) * kDwgMaxContrib + i) * kDwgTcCols + r) * EC;
+      float* mine = part + ((static_cast<size_t>(j) * maxc + i) * kDwgTcCols + r) * EC;
 #pragma unroll
       for (int e = 0; e < EC; e += 4)
         *reinterpret_cast<float4*>(mine + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
@@ -797,16 +1002,28 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
         float sum[EC];
 #pragma unroll
         for (int e = 0; e < EC; ++e) sum[e] = 0.f;
-        for (int k = 0; k < n; ++k) {
-          const float4* src = reinterpret_cast<const float4*>(
-              part + ((static_cast<size_t>(j) * kDwgMaxContrib + k) * kDwgTcCols + r) * EC);
+        // partials in batches whose loads are all in flight at once; added in order k
+        constexpr int kBatch = 64 / EC;
+        for (int k0 = 0; k0 < n; k0 += kBatch) {
+          float4 t4[kBatch][EC / 4];
 #pragma unroll
-          for (int e4 = 0; e4 < EC / 4; ++e4) {
-            const float4 t4 = __ldcg(src + e4);
-            sum[4 * e4] += t4.x;
-            sum[4 * e4 + 1] += t4.y;
-            sum[4 * e4 + 2] += t4.z;
-            sum[4 * e4 + 3] += t4.w;
+          for (int kb = 0; kb < kBatch; ++kb) {
+            const float4* src = reinterpret_cast<const float4*>(
+                part + ((static_cast<size_t>(j) * maxc + min(k0 + kb, n - 1)) * kDwgTcCols + r) * EC);
+#pragma unroll
+            for (int e4 = 0; e4 < EC / 4; ++e4) t4[kb][e4] = __ldcg(src + e4);
+          }
+#pragma unroll
+          for (int kb = 0; kb < kBatch; ++kb) {
+            if (k0 + kb < n) {
+#pragma unroll
+              for (int e4 = 0; e4 < EC / 4; ++e4) {
+                sum[4 * e4] += t4[kb][e4].x;
+                sum[4 * e4 + 1] += t4[kb][e4].y;
+                sum[4 * e4 + 2] += t4[kb][e4].z;
+                sum[4 * e4 + 3] += t4[kb][e4].w;
+              }
+            }
           }
         }
         if (c < d) {
@@ -847,13 +1064,14 @@ int dwg_splits(int T, int d, int E) {
   return s < 1 ? 1 : s;
 }
 
-// Tensor-core dWg (E <= 16): partials [column tile][kDwgMaxContrib][128][EC],
+// Tensor-core dWg (E <= 16): partials [column tile][dwg_max_contrib][128][EC],
 // the transposed bf16 terms dlT [32][ldt] and the tickets [column tile][4].
 int dwg_tc_ec(int E) { return E <= 8 ? 8 : 16; }
 long long dlt_ld(int T) { return (static_cast<long long>(T) + 7) / 8 * 8; }
 int dwg_tc_tiles(int d) { return (d + kDwgTcCols - 1) / kDwgTcCols; }
 size_t dwg_tc_part_bytes(int d, int E) {
-  return static_cast<size_t>(dwg_tc_tiles(d)) * kDwgMaxContrib * kDwgTcCols * dwg_tc_ec(E) * 4;
+  const int nct = dwg_tc_tiles(d);
+  return static_cast<size_t>(nct) * dwg_max_contrib(nct) * kDwgTcCols * dwg_tc_ec(E) * 4;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -866,7 +1084,8 @@ size_t route_backward_scratch_bytes(int T, int d, int E) {
   if (E <= 16) {
     part = std::max(part, dwg_tc_part_bytes(d, E));
     extra = align_up(static_cast<size_t>(32) * dlt_ld(T) * 2) +
-            align_up(static_cast<size_t>(dwg_tc_tiles(d)) * 4 * 4);
+            align_up(static_cast<size_t>(dwg_tc_tiles(d)) * 4 * 4) +
+            align_up(static_cast<size_t>(kTptMaxBlocks) * 16 * 4);
   }
   return align_up(static_cast<size_t>(E) * 4) + align_up(static_cast<size_t>(T) * E * 4) +
          align_up(part) + extra;
@@ -889,20 +1108,44 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
   sc += align_up(part_bytes);
   __nv_bfloat16* dlT = nullptr;
   int* tickets = nullptr;
+  int32_t* hist_part = nullptr;
   if (E <= 16) {
     dlT = reinterpret_cast<__nv_bfloat16*>(sc);
     sc += align_up(static_cast<size_t>(32) * dlt_ld(T) * 2);
     tickets = reinterpret_cast<int*>(sc);
+    sc += align_up(static_cast<size_t>(dwg_tc_tiles(d)) * 4 * 4);
+    hist_part = reinterpret_cast<int32_t*>(sc);
   }
   const float inv_tau = 1.0f / temperature;
   const bool aux = d_aux != 0.0f;
-  // bf16 with at most 16 experts: both T x d passes on the tensor cores
-  const bool tc = dt == MOE_BF16 && E <= 16 && d % 8 == 0 && T > 0 && aligned16(x) &&
-                  aligned16(wg) && aligned16(dl);
+  // at most 16 experts and many picks: d_logits with a thread per token
+  // (rows read and written as 16-byte vectors when E is 8 or 16); bf16 with
+  // at most 16 experts: both T x d passes on the tensor cores
+  const bool tpt = E <= 16 && k <= kTptMaxK && static_cast<long long>(T) * k >= kTptMinPicks &&
+                   aligned16(probs) && aligned16(dl) && (d_z == 0.0f || aligned16(logits));
+  const bool tc = E <= 16 && dt == MOE_BF16 && d % 8 == 0 && T > 0 && aligned16(x) && aligned16(wg) &&
+                  aligned16(dl);
   const int ec = dwg_tc_ec(E);
   const bool tc_dwg = tc && d_wg != nullptr;
   cudaError_t err = cudaSuccess;
-  if (T > 0) {
+  if (T > 0 && tpt) {
+    // large T: thread per token, the pick counts in the same launch
+    // (cooperative: at most as many blocks as are resident)
+    auto kern = ec == 8 ? bwd_logits_tpt<8> : bwd_logits_tpt<16>;
+    int g = std::min((T + kTptThreads - 1) / kTptThreads, kTptMaxBlocks);
+    if (aux) {
+      int per_sm = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kTptThreads, 0) != cudaSuccess ||
+          per_sm < 1)
+        return cudaErrorInvalidConfiguration;
+      g = std::min(g, per_sm * num_sms());
+    }
+    err = launch_pdl(kern, dim3(g), dim3(kTptThreads), 0, s, aux, probs, d_z != 0.0f ? logits : nullptr,
+                     idx, w, d_w, aux ? 1 : 0, hist_part, d_aux, d_z, inv_tau, T, E, k, dl,
+                     tc_dwg ? dlT : nullptr, static_cast<int>(dlt_ld(T)), tc_dwg ? tickets : nullptr,
+                     dwg_tc_tiles(d) * 4, ctl);
+    if (err != cudaSuccess) return err;
+  } else if (T > 0) {
     if (aux) {
       err = launch_pdl(bwd_hist, dim3(1), dim3(1024), 0, s, false, idx, static_cast<long long>(T) * k,
                        E, counts, ctl);
@@ -917,11 +1160,16 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
                      d_z, inv_tau, T, E, k, dl, tc_dwg ? dlT : nullptr, ec, static_cast<int>(dlt_ld(T)),
                      tc_dwg ? tickets : nullptr, dwg_tc_tiles(d) * 4, ctl);
     if (err != cudaSuccess) return err;
+  }
+  if (T > 0) {
     if (dx != nullptr && tc) {
-      const int tiles = ((T + kDxTcTok - 1) / kDxTcTok) * ((d + kDxTcCols - 1) / kDxTcCols);
+      const int nct = (d + kDxTcCols - 1) / kDxTcCols;
+      const int tiles = ((T + kDxTcTok - 1) / kDxTcTok) * nct;
+      const int slots = 2 * num_sms();
+      const int g = std::min(tiles, nct <= slots ? slots / nct * nct : slots);
       auto kern = ec == 8 ? bwd_dx_tc<8> : bwd_dx_tc<16>;
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kDxTcSmem));
-      err = launch_pdl(kern, dim3(std::min(tiles, 2 * num_sms())), dim3(kDxTcThreads), kDxTcSmem, s, false,
+      err = launch_pdl(kern, dim3(g), dim3(kDxTcThreads), kDxTcSmem, s, false,
                        static_cast<const float*>(dl), static_cast<const __nv_bfloat16*>(wg), T, d, E,
                        static_cast<__nv_bfloat16*>(dx), ctl);
       if (err != cudaSuccess) return err;
@@ -938,13 +1186,14 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
     }
   }
   if (tc_dwg) {
-    // equal shares of 64-token x 128-column units; L keeps a tile's blocks <= kDwgMaxContrib
+    // equal shares of 64-token x 128-column units; L keeps a tile's blocks <= maxc
     const int ntb = (T + kDwgTcTok - 1) / kDwgTcTok;
     const int nct = dwg_tc_tiles(d);
+    const int maxc = dwg_max_contrib(nct);
     const long long total = static_cast<long long>(ntb) * nct;
     if (total > 0x7fffffffLL) return cudaErrorInvalidValue;
     long long L = (total + num_sms() - 1) / num_sms();
-    L = std::max<long long>(L, (ntb + kDwgMaxContrib - 2) / (kDwgMaxContrib - 1));
+    L = std::max<long long>(L, (ntb + maxc - 2) / (maxc - 1));
     const int G = static_cast<int>((total + L - 1) / L);
     CUtensorMap tmx, tmg;
     if (!make_tma_2d_bf16(&tmx, x, static_cast<uint64_t>(T), static_cast<uint64_t>(d), kDwgTcTok) ||
@@ -955,7 +1204,7 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
     auto kern = ec == 8 ? bwd_dwg_tc<8> : bwd_dwg_tc<16>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     err = launch_pdl(kern, dim3(G), dim3(kDwgTcThreads), smem, s, false, tmx, tmg, d, E, ntb,
-                     static_cast<int>(total), static_cast<int>(L), part, tickets, d_wg, ctl);
+                     static_cast<int>(total), static_cast<int>(L), maxc, part, tickets, d_wg, ctl);
   } else if (d_wg != nullptr) {
     const int ns = dwg_splits(T, d, E);
     const int tps = T > 0 ? (T + ns - 1) / ns : 0;

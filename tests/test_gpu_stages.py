@@ -466,6 +466,10 @@ def test_route_train_at_unit_temperature_is_route(T, d, E, k, dt):
     (2500, 2048, 8, 2, "bf16", 1.3, 0.01, 0.001),   # dWg tiles shared by several blocks, a ragged last unit
     (333, 128, 5, 2, "bf16", 1.0, 0.1, 0.01),       # one column tile, E = 5, a ragged last unit
     (4100, 256, 16, 3, "bf16", 0.8, 0.05, 0.0),     # 2 column tiles x 65 units: 22 blocks per tile
+    (5462, 256, 8, 3, "bf16", 1.0, 0.2, 0.0),       # 16386 picks: thread per token, counts over a grid barrier
+    (9000, 128, 16, 2, "bf16", 1.0, 0.0, 0.01),     # thread per token without the aux term (no barrier)
+    (300, 64, 8, 2, "f32", 1.0, 0.1, 0.01),         # fp32, E = 8: CUDA-core passes
+    (270000, 128, 8, 2, "bf16", 1.0, 0.01, 0.001),  # > 1024 x 256 tokens: grid-stride d_logits, 147 blocks on one tile
 ])
 def test_route_backward(T, d, E, k, dt, tau, d_aux, d_z):
     """moe_route_backward from the GPU's own forward (moe_route_train at tau)
