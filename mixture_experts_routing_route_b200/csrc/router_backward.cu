@@ -58,12 +58,15 @@ bwd_hist(const int32_t* __restrict__ idx, long long S, int E, int32_t* __restric
   for (int e = threadIdx.x; e < E; e += blockDim.x) counts[e] = h[e];
 }
 
-constexpr int kLogitWarps = 8;
+constexpr int kLogitWarps = 16;
 
 // Warp per token; lane holds experts lane + 32 q, q < EPL. The short per-lane
 // chains and a grid over every SM suit small T (counts from bwd_hist first);
-// with dlT set (E <= 16) it also writes the bf16 terms of d_logits for the
-// tensor-core dWg, and block 0 zeroes dWg's tickets.
+// with dlT set (E <= 64) it also writes the bf16 terms of d_logits for the
+// tensor-core dWg, and block 0 zeroes dWg's tickets. A block's 16 warps take
+// 16 consecutive tokens per round, so with dlT the round's terms are staged
+// in shared memory and each dlT row gets one whole 32-byte sector per round
+// (ldt is a multiple of 16) instead of a 2-byte store per lane and row.
 template <int EPL>
 __global__ void __launch_bounds__(kLogitWarps * 32)
 bwd_logits(const float* __restrict__ probs, const float* __restrict__ logits,
@@ -88,7 +91,15 @@ bwd_logits(const float* __restrict__ probs, const float* __restrict__ logits,
                  static_cast<float>(T);
   }
   const float zc = d_z * 2.0f / static_cast<float>(T);
-  for (int t = blockIdx.x * kLogitWarps + warp; t < T; t += gridDim.x * kLogitWarps) {
+  __shared__ __align__(16) __nv_bfloat16 st_s[128][kLogitWarps];  // [hi/lo row][token of the round]
+  // block-uniform rounds (the dlT staging has barriers)
+  for (long long base = static_cast<long long>(blockIdx.x) * kLogitWarps; base < T;
+       base += static_cast<long long>(gridDim.x) * kLogitWarps) {
+    const int t = static_cast<int>(base) + warp;
+    if (t >= T) {
+      if (dlT != nullptr)
+        for (int n = lane; n < 2 * ec; n += 32) st_s[n][warp] = __float2bfloat16_rn(0.f);
+    } else {
     const size_t row = static_cast<size_t>(t) * E;
     float p[EPL], dp[EPL];
 #pragma unroll
@@ -160,13 +171,30 @@ bwd_logits(const float* __restrict__ probs, const float* __restrict__ logits,
       const int e = lane + 32 * q;
       if (e < E) d_logits[row + e] = dl[q];
     }
-    if (dlT != nullptr && lane < ec) {
-      // the tensor-core dWg's B operand (E <= 16, so EPL == 1 and lane =
-      // expert): dlT[e][t] = hi, dlT[ec + e][t] = lo
-      const float v = lane < E ? dl[0] : 0.f;
-      const __nv_bfloat16 h = __float2bfloat16_rn(v);
-      dlT[static_cast<size_t>(lane) * ldt + t] = h;
-      dlT[static_cast<size_t>(ec + lane) * ldt + t] = __float2bfloat16_rn(v - __bfloat162float(h));
+    if (dlT != nullptr) {
+      // the tensor-core dWg's B operand (E <= 64): dlT[e][t] = hi,
+      // dlT[ec + e][t] = lo for the lane's experts e = lane + 32 q < ec
+#pragma unroll
+      for (int q = 0; q < EPL; ++q) {
+        const int e = lane + 32 * q;
+        if (e < ec) {
+          const float v = e < E ? dl[q] : 0.f;
+          const __nv_bfloat16 h = __float2bfloat16_rn(v);
+          st_s[e][warp] = h;
+          st_s[ec + e][warp] = __float2bfloat16_rn(v - __bfloat162float(h));
+        }
+      }
+    }
+    }
+    if (dlT != nullptr) {
+      __syncthreads();
+      // row n, tokens base .. base + 15: two 16-byte stores
+      for (int i = threadIdx.x; i < 4 * ec; i += kLogitWarps * 32) {
+        const int n = i >> 1, h = i & 1;
+        *reinterpret_cast<uint4*>(dlT + static_cast<size_t>(n) * ldt + base + 8 * h) =
+            *reinterpret_cast<const uint4*>(&st_s[n][8 * h]);
+      }
+      __syncthreads();
     }
   }
 }
@@ -630,13 +658,23 @@ __device__ __forceinline__ void load_row(const float* __restrict__ a, int t, int
 // column tile and writes its B operand once. Waits are bounded.
 constexpr int kDxTcThreads = 128;
 constexpr int kDxTcTok = 128;
-constexpr int kDxTcCols = 256;
-constexpr int kDxTcA = kDxTcTok * 128;     // 16 KB: 128-byte rows
-constexpr int kDxTcB = kDxTcCols * 128;    // 32 KB
 constexpr int kDxStageRow = 128 + 16;      // staged output row (16-byte pad: no bank conflicts)
 constexpr int kDxStageWarp = 32 * kDxStageRow;
-constexpr size_t kDxTcSmem = 80 * 1024;
-static_assert(kDxTcA + kDxTcB + 4 * kDxStageWarp + 1024 <= static_cast<int>(kDxTcSmem), "dx smem");
+constexpr size_t kDxTcSmem = 86 * 1024;
+
+// K = 2 EC is one 128-byte swizzle atom (EC <= 32) or two (EC = 64: hi in the
+// first, lo in the second); a 64-expert tile is 128 columns wide so that two
+// blocks still share an SM.
+template <int EC>
+struct DxTc {
+  static constexpr int KB = (2 * EC + 63) / 64;        // K atoms
+  static constexpr int TN = EC <= 32 ? 256 : 128;      // columns per tile (MMA N)
+  static constexpr int A_ATOM = kDxTcTok * 128;        // 16 KB
+  static constexpr int B_ATOM = TN * 128;
+  static constexpr int A_BYTES = KB * A_ATOM;
+  static constexpr int B_BYTES = KB * B_ATOM;
+  static_assert(A_BYTES + B_BYTES + 4 * kDxStageWarp + 1024 <= static_cast<int>(kDxTcSmem), "dx smem");
+};
 static_assert(3 * (kDxTcSmem + 1024) > 228 * 1024, "at most two dx blocks per SM");
 
 template <int EC>
@@ -644,22 +682,27 @@ __global__ void __launch_bounds__(kDxTcThreads, 2)
 bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, int T, int d, int E,
           __nv_bfloat16* __restrict__ dx, Control* ctl) {
   pdl_begin();
-  static_assert(EC == 8 || EC == 16, "EC");
+  static_assert(EC == 8 || EC == 16 || EC == 32 || EC == 64, "EC");
+  using C = DxTc<EC>;
+  constexpr int TN = C::TN;
   extern __shared__ uint8_t dx_raw[];
   __shared__ __align__(8) uint64_t mma_bar;
   __shared__ uint32_t tmem_s;
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dx_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   uint8_t* sa = sm;
-  uint8_t* sb = sm + kDxTcA;
+  uint8_t* sb = sm + C::A_BYTES;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  uint8_t* stg = sm + kDxTcA + kDxTcB + warp * kDxStageWarp;
+  uint8_t* stg = sm + C::A_BYTES + C::B_BYTES + warp * kDxStageWarp;
+  // 16-byte chunk c (8 K values) of row r of an operand of KB atoms
+  auto chunk_a = [&](int r, int c) { return sw128_chunk(sa + (c >> 3) * C::A_ATOM, r, c & 7); };
+  auto chunk_b = [&](int r, int c) { return sw128_chunk(sb + (c >> 3) * C::B_ATOM, r, c & 7); };
   if (tid == 0) {
     mbar_init(&mma_bar, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(&tmem_s, kDxTcCols);
+    tmem_alloc(&tmem_s, TN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -667,9 +710,9 @@ bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, in
   tc_fence_after();
   const uint32_t tmem = tmem_s;
   const uint64_t limit = wait_limit_ns(ctl);
-  const int ntt = (T + kDxTcTok - 1) / kDxTcTok, nct = (d + kDxTcCols - 1) / kDxTcCols;
+  const int ntt = (T + kDxTcTok - 1) / kDxTcTok, nct = (d + TN - 1) / TN;
   const int total = ntt * nct;
-  constexpr uint32_t kIdesc = make_idesc_bf16(kDxTcTok, kDxTcCols, true);
+  constexpr uint32_t kIdesc = make_idesc_bf16(kDxTcTok, TN, true);
   float g[EC];
   if (static_cast<int>(blockIdx.x) < total) load_row<EC>(dl, (blockIdx.x / nct) * kDxTcTok + tid, T, E, g);
   int cur_ct = -1;
@@ -682,13 +725,13 @@ bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, in
     for (int h = 0; h < EC / 8; ++h) {
       uint4 hi, lo;
       split_hi_lo8(g + 8 * h, hi, lo);
-      *reinterpret_cast<uint4*>(sw128_chunk(sa, tid, h)) = hi;
-      *reinterpret_cast<uint4*>(sw128_chunk(sa, tid, EC / 8 + h)) = lo;
+      *reinterpret_cast<uint4*>(chunk_a(tid, h)) = hi;
+      *reinterpret_cast<uint4*>(chunk_a(tid, EC / 8 + h)) = lo;
     }
     if (ct != cur_ct) {
       // B rows = columns c of this tile: [Wg[c, 0..EC) | Wg[c, 0..EC)]
-      for (int r = tid; r < kDxTcCols; r += kDxTcThreads) {
-        const int c = ct * kDxTcCols + r;
+      for (int r = tid; r < TN; r += kDxTcThreads) {
+        const int c = ct * TN + r;
         uint4 w[EC / 8];
         if (c < d && E == EC) {
           const uint4* p = reinterpret_cast<const uint4*>(wg + static_cast<size_t>(c) * EC);
@@ -706,8 +749,8 @@ bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, in
         }
 #pragma unroll
         for (int h = 0; h < EC / 8; ++h) {
-          *reinterpret_cast<uint4*>(sw128_chunk(sb, r, h)) = w[h];
-          *reinterpret_cast<uint4*>(sw128_chunk(sb, r, EC / 8 + h)) = w[h];
+          *reinterpret_cast<uint4*>(chunk_b(r, h)) = w[h];
+          *reinterpret_cast<uint4*>(chunk_b(r, EC / 8 + h)) = w[h];
         }
       }
       cur_ct = ct;
@@ -720,8 +763,9 @@ bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, in
       const uint32_t a_addr = smem_u32(sa), b_addr = smem_u32(sb);
 #pragma unroll
       for (int kk = 0; kk < 2 * EC / 16; ++kk)
-        umma_bf16(tmem, make_sw128_desc(a_addr + kk * 32, 16, 1024),
-                  make_sw128_desc(b_addr + kk * 32, 16, 1024), kIdesc, kk > 0 ? 1u : 0u);
+        umma_bf16(tmem, make_sw128_desc(a_addr + (kk >> 2) * C::A_ATOM + (kk & 3) * 32, 16, 1024),
+                  make_sw128_desc(b_addr + (kk >> 2) * C::B_ATOM + (kk & 3) * 32, 16, 1024), kIdesc,
+                  kk > 0 ? 1u : 0u);
       umma_commit(&mma_bar);
     }
     pending = true;
@@ -740,8 +784,8 @@ bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, in
     tc_fence_after();
     const long long t0 = static_cast<long long>(tt) * kDxTcTok + warp * 32;
     const int nrows = static_cast<int>(max(0LL, min(32LL, T - t0)));
-    const int c0 = ct * kDxTcCols;
-    const int ncols = min(kDxTcCols, d - c0);
+    const int c0 = ct * TN;
+    const int ncols = min(TN, d - c0);
     const uint32_t tq = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     if (nrows > 0) {
       for (int gc = 0; gc < ncols; gc += 64) {
@@ -781,7 +825,7 @@ bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, in
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, kDxTcCols);
+    tmem_dealloc(tmem, TN);
   }
 }
 
@@ -804,6 +848,7 @@ bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, in
 // 2..5 epilogue (tensor-memory lane quarter = warp % 4). Waits are bounded.
 constexpr int kDwgTcThreads = 192;
 constexpr int kDwgTcStages = 8;
+constexpr int kMaxDwgStages = 8;
 constexpr int kDwgTcCols = 128;
 constexpr int kDwgTcTok = 64;
 // Partials per column tile: enough for every SM to share one tile when d is
@@ -816,7 +861,10 @@ struct DwgTc {
   static constexpr int A_BYTES = kDwgTcCols * kDwgTcTok * 2;  // two 64-column boxes
   static constexpr int B_BYTES = N * kDwgTcTok * 2;
   static constexpr int STAGE = A_BYTES + B_BYTES;              // a multiple of 1024
-  static constexpr size_t SMEM = static_cast<size_t>(kDwgTcStages) * STAGE + 1024;
+  static constexpr int STAGES = EC <= 32 ? kDwgTcStages : 6;
+  static constexpr int ACC = N < 32 ? 32 : N;                  // tensor-memory columns per accumulator
+  static constexpr int TMEM = 2 * ACC;                         // a power of two >= 64
+  static constexpr size_t SMEM = static_cast<size_t>(STAGES) * STAGE + 1024;
 };
 
 template <int EC>
@@ -827,8 +875,9 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
   pdl_begin();
   using C = DwgTc<EC>;
   static_assert(C::STAGE % 1024 == 0, "stage alignment");
+  static_assert(C::STAGES <= kMaxDwgStages, "ring barriers");
   extern __shared__ uint8_t dwg_raw[];
-  __shared__ __align__(8) uint64_t full[kDwgTcStages], empty[kDwgTcStages];
+  __shared__ __align__(8) uint64_t full[kMaxDwgStages], empty[kMaxDwgStages];
   __shared__ __align__(8) uint64_t tfull[2], tempty[2], drain;
   __shared__ uint32_t tmem_s;
   __shared__ volatile int abort_s;
@@ -838,7 +887,7 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
   const int u0 = blockIdx.x * L, u1 = min(total, u0 + L);
   const uint64_t limit = wait_limit_ns(ctl);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kDwgTcStages; ++i) {
+    for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
@@ -851,7 +900,7 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(&tmem_s, 64);
+    tmem_alloc(&tmem_s, C::TMEM);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -879,12 +928,12 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
         tma_load_2d(sa + C::A_BYTES, &tmg, &full[stage], tb * kDwgTcTok, 0);
         issued_mask |= 1u << stage;
         last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-        if (++stage == kDwgTcStages) {
+        if (++stage == C::STAGES) {
           stage = 0;
           phase ^= 1u;
         }
       }
-      for (int s = 0; s < kDwgTcStages; ++s)
+      for (int s = 0; s < C::STAGES; ++s)
         if ((issued_mask >> s) & 1u)
           if (!mbar_wait_bounded(&full[s], (last_parity >> s) & 1u, limit)) set_error(ctl, MOE_DEVERR_TIMEOUT);
     }
@@ -905,7 +954,7 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem + acc * 32;
+        const uint32_t d_tmem = tmem + acc * C::ACC;
         const int us = u;
         bool ok = true;
         for (; u < ue; ++u) {
@@ -925,7 +974,7 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
                       (u != us || kk != 0) ? 1u : 0u);
           issued_any = true;
           umma_commit(&empty[stage]);
-          if (++stage == kDwgTcStages) {
+          if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
@@ -964,7 +1013,7 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
       tc_fence_after();
       float v[EC];
       {
-        const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * 32;
+        const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * C::ACC;
         if constexpr (EC == 8) {
           uint32_t r[16];
           tmem_ld_32x32b_x16(ta, r);
@@ -972,11 +1021,16 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
 #pragma unroll
           for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[e]) + __uint_as_float(r[8 + e]);
         } else {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(ta, r);
-          tmem_ld_wait();
+          // hi in columns [0, EC), lo in [EC, 2 EC), 16 at a time
 #pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(r[e]) + __uint_as_float(r[16 + e]);
+          for (int h = 0; h < EC / 16; ++h) {
+            uint32_t rh[16], rl[16];
+            tmem_ld_32x32b_x16(ta + 16 * h, rh);
+            tmem_ld_32x32b_x16(ta + EC + 16 * h, rl);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[16 * h + i] = __uint_as_float(rh[i]) + __uint_as_float(rl[i]);
+          }
         }
       }
       tc_fence_before();
@@ -995,6 +1049,7 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
 #pragma unroll
       for (int e = 0; e < EC; e += 4)
         *reinterpret_cast<float4*>(mine + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+      if (tickets == nullptr) continue;  // EC >= 32: bwd_dwg_tc_reduce adds the partials
       __threadfence();
       __syncwarp();
       int prev = 0;
@@ -1007,7 +1062,7 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
 #pragma unroll
         for (int e = 0; e < EC; ++e) sum[e] = 0.f;
         // partials in batches whose loads are all in flight at once; added in order k
-        constexpr int kBatch = 64 / EC;
+        constexpr int kBatch = EC <= 64 ? 64 / EC : 1;
         for (int k0 = 0; k0 < n; k0 += kBatch) {
           float4 t4[kBatch][EC / 4];
 #pragma unroll
@@ -1042,7 +1097,7 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 64);
+    tmem_dealloc(tmem, C::TMEM);
   }
 }
 
@@ -1068,10 +1123,45 @@ int dwg_splits(int T, int d, int E) {
   return s < 1 ? 1 : s;
 }
 
-// Tensor-core dWg (E <= 16): partials [column tile][dwg_max_contrib][128][EC],
-// the transposed bf16 terms dlT [32][ldt] and the tickets [column tile][4].
-int dwg_tc_ec(int E) { return E <= 8 ? 8 : 16; }
-long long dlt_ld(int T) { return (static_cast<long long>(T) + 7) / 8 * 8; }
+// The partials of bwd_dwg_tc for EC >= 32, where one block per tile adding
+// about 150 / (d / 128) partials of 128 x EC floats would be a long serial
+// tail: d_wg[c, e] = sum over the tile's blocks i = 0, 1, ... of
+// part[tile][i][c % 128][e], a thread per 4 experts of a column (the same
+// order as the in-kernel reduction: deterministic).
+template <int EC>
+__global__ void __launch_bounds__(256)
+bwd_dwg_tc_reduce(const float* __restrict__ part, int d, int E, int ntb, int L, int maxc,
+                  float* __restrict__ d_wg) {
+  pdl_begin();
+  const long long n = static_cast<long long>(d) * (EC / 4);
+  for (long long i = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * 256) {
+    const int c = static_cast<int>(i / (EC / 4)), e4 = static_cast<int>(i - static_cast<long long>(c) * (EC / 4));
+    const int j = c / kDwgTcCols, r = c - j * kDwgTcCols;
+    const int first = static_cast<int>((static_cast<long long>(j) * ntb) / L);
+    const int last = static_cast<int>((static_cast<long long>(j + 1) * ntb - 1) / L);
+    const float4* src = reinterpret_cast<const float4*>(part) +
+                        ((static_cast<size_t>(j) * maxc) * kDwgTcCols + r) * (EC / 4) + e4;
+    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int k = 0; k < last - first + 1; ++k) {
+      const float4 t4 = __ldg(src + static_cast<size_t>(k) * kDwgTcCols * (EC / 4));
+      sum.x += t4.x;
+      sum.y += t4.y;
+      sum.z += t4.z;
+      sum.w += t4.w;
+    }
+    const float v[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (4 * e4 + q < E) d_wg[static_cast<size_t>(c) * E + 4 * e4 + q] = v[q];
+  }
+}
+
+// Tensor-core dWg (E <= 64): partials [column tile][dwg_max_contrib][128][EC],
+// the transposed bf16 terms dlT [2 EC][ldt] and the tickets [column tile][4].
+int dwg_tc_ec(int E) { return E <= 8 ? 8 : E <= 16 ? 16 : E <= 32 ? 32 : 64; }
+long long dlt_ld(int T) { return (static_cast<long long>(T) + 15) / 16 * 16; }
 int dwg_tc_tiles(int d) { return (d + kDwgTcCols - 1) / kDwgTcCols; }
 size_t dwg_tc_part_bytes(int d, int E) {
   const int nct = dwg_tc_tiles(d);
@@ -1085,9 +1175,9 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 size_t route_backward_scratch_bytes(int T, int d, int E) {
   size_t part = static_cast<size_t>(dwg_splits(T, d, E)) * d * E * 4;
   size_t extra = 0;
-  if (E <= 16) {
+  if (E <= 64) {
     part = std::max(part, dwg_tc_part_bytes(d, E));
-    extra = align_up(static_cast<size_t>(32) * dlt_ld(T) * 2) +
+    extra = align_up(static_cast<size_t>(2 * dwg_tc_ec(E)) * dlt_ld(T) * 2) +
             align_up(static_cast<size_t>(dwg_tc_tiles(d)) * 4 * 4) +
             align_up(static_cast<size_t>(kTptMaxBlocks) * 16 * 4);
   }
@@ -1108,14 +1198,14 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
   sc += align_up(static_cast<size_t>(T) * E * 4);
   float* part = reinterpret_cast<float*>(sc);
   size_t part_bytes = static_cast<size_t>(dwg_splits(T, d, E)) * d * E * 4;
-  if (E <= 16) part_bytes = std::max(part_bytes, dwg_tc_part_bytes(d, E));
+  if (E <= 64) part_bytes = std::max(part_bytes, dwg_tc_part_bytes(d, E));
   sc += align_up(part_bytes);
   __nv_bfloat16* dlT = nullptr;
   int* tickets = nullptr;
   int32_t* hist_part = nullptr;
-  if (E <= 16) {
+  if (E <= 64) {
     dlT = reinterpret_cast<__nv_bfloat16*>(sc);
-    sc += align_up(static_cast<size_t>(32) * dlt_ld(T) * 2);
+    sc += align_up(static_cast<size_t>(2 * dwg_tc_ec(E)) * dlt_ld(T) * 2);
     tickets = reinterpret_cast<int*>(sc);
     sc += align_up(static_cast<size_t>(dwg_tc_tiles(d)) * 4 * 4);
     hist_part = reinterpret_cast<int32_t*>(sc);
@@ -1124,10 +1214,10 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
   const bool aux = d_aux != 0.0f;
   // at most 16 experts and many picks: d_logits with a thread per token
   // (rows read and written as 16-byte vectors when E is 8 or 16); bf16 with
-  // at most 16 experts: both T x d passes on the tensor cores
+  // at most 64 experts: both T x d passes on the tensor cores
   const bool tpt = E <= 16 && k <= kTptMaxK && static_cast<long long>(T) * k >= kTptMinPicks &&
                    aligned16(probs) && aligned16(dl) && (d_z == 0.0f || aligned16(logits));
-  const bool tc = E <= 16 && dt == MOE_BF16 && d % 8 == 0 && T > 0 && aligned16(x) && aligned16(wg) &&
+  const bool tc = E <= 64 && dt == MOE_BF16 && d % 8 == 0 && T > 0 && aligned16(x) && aligned16(wg) &&
                   aligned16(dl);
   const int ec = dwg_tc_ec(E);
   const bool tc_dwg = tc && d_wg != nullptr;
@@ -1135,7 +1225,7 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
   if (T > 0 && tpt) {
     // large T: thread per token, the pick counts in the same launch
     // (cooperative: at most as many blocks as are resident)
-    auto kern = ec == 8 ? bwd_logits_tpt<8> : bwd_logits_tpt<16>;
+    auto kern = E <= 8 ? bwd_logits_tpt<8> : bwd_logits_tpt<16>;
     int g = std::min((T + kTptThreads - 1) / kTptThreads, kTptMaxBlocks);
     if (aux) {
       int per_sm = 0;
@@ -1146,7 +1236,7 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
     }
     err = launch_pdl(kern, dim3(g), dim3(kTptThreads), 0, s, aux, probs, d_z != 0.0f ? logits : nullptr,
                      idx, w, d_w, aux ? 1 : 0, hist_part, d_aux, d_z, inv_tau, T, E, k, dl,
-                     tc_dwg ? dlT : nullptr, static_cast<int>(dlt_ld(T)), tc_dwg ? tickets : nullptr,
+                     tc_dwg ? dlT : nullptr, static_cast<int>(dlt_ld(T)), tc_dwg && ec <= 16 ? tickets : nullptr,
                      dwg_tc_tiles(d) * 4, ctl);
     if (err != cudaSuccess) return err;
   } else if (T > 0) {
@@ -1158,20 +1248,21 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
     const int epl = (E + 31) / 32;
     auto kern = epl <= 1 ? bwd_logits<1> : epl <= 2 ? bwd_logits<2> : epl <= 4 ? bwd_logits<4>
                                                                               : bwd_logits<8>;
-    const int grid = std::max(1, std::min((T + kLogitWarps - 1) / kLogitWarps, 8 * num_sms()));
+    const int grid = std::max(1, std::min((T + kLogitWarps - 1) / kLogitWarps, 4 * num_sms()));
     err = launch_pdl(kern, dim3(grid), dim3(kLogitWarps * 32), 0, s, false, probs,
                      d_z != 0.0f ? logits : nullptr, idx, w, d_w, aux ? counts : nullptr, d_aux,
                      d_z, inv_tau, T, E, k, dl, tc_dwg ? dlT : nullptr, ec, static_cast<int>(dlt_ld(T)),
-                     tc_dwg ? tickets : nullptr, dwg_tc_tiles(d) * 4, ctl);
+                     tc_dwg && ec <= 16 ? tickets : nullptr, dwg_tc_tiles(d) * 4, ctl);
     if (err != cudaSuccess) return err;
   }
   if (T > 0) {
     if (dx != nullptr && tc) {
-      const int nct = (d + kDxTcCols - 1) / kDxTcCols;
+      const int tn = ec <= 32 ? DxTc<8>::TN : DxTc<64>::TN;
+      const int nct = (d + tn - 1) / tn;
       const int tiles = ((T + kDxTcTok - 1) / kDxTcTok) * nct;
       const int slots = 2 * num_sms();
       const int g = std::min(tiles, nct <= slots ? slots / nct * nct : slots);
-      auto kern = ec == 8 ? bwd_dx_tc<8> : bwd_dx_tc<16>;
+      auto kern = ec == 8 ? bwd_dx_tc<8> : ec == 16 ? bwd_dx_tc<16> : ec == 32 ? bwd_dx_tc<32> : bwd_dx_tc<64>;
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kDxTcSmem));
       err = launch_pdl(kern, dim3(g), dim3(kDxTcThreads), kDxTcSmem, s, false,
                        static_cast<const float*>(dl), static_cast<const __nv_bfloat16*>(wg), T, d, E,
@@ -1204,11 +1295,19 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
         !make_tma_2d_bf16_ld(&tmg, dlT, static_cast<uint64_t>(2 * ec), static_cast<uint64_t>(T),
                              static_cast<uint64_t>(dlt_ld(T)), static_cast<uint32_t>(2 * ec)))
       return cudaErrorInvalidValue;
-    const size_t smem = ec == 8 ? DwgTc<8>::SMEM : DwgTc<16>::SMEM;
-    auto kern = ec == 8 ? bwd_dwg_tc<8> : bwd_dwg_tc<16>;
+    const size_t smem = ec == 8 ? DwgTc<8>::SMEM : ec == 16 ? DwgTc<16>::SMEM
+                      : ec == 32 ? DwgTc<32>::SMEM : DwgTc<64>::SMEM;
+    auto kern = ec == 8 ? bwd_dwg_tc<8> : ec == 16 ? bwd_dwg_tc<16> : ec == 32 ? bwd_dwg_tc<32> : bwd_dwg_tc<64>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     err = launch_pdl(kern, dim3(G), dim3(kDwgTcThreads), smem, s, false, tmx, tmg, d, E, ntb,
-                     static_cast<int>(total), static_cast<int>(L), maxc, part, tickets, d_wg, ctl);
+                     static_cast<int>(total), static_cast<int>(L), maxc, part,
+                     ec <= 16 ? tickets : nullptr, d_wg, ctl);
+    if (err != cudaSuccess || ec <= 16) return err;
+    const long long nout = static_cast<long long>(d) * (ec / 4);
+    const int rg = static_cast<int>(std::min<long long>((nout + 255) / 256, 8LL * num_sms()));
+    auto red = ec == 32 ? bwd_dwg_tc_reduce<32> : bwd_dwg_tc_reduce<64>;
+    err = launch_pdl(red, dim3(std::max(rg, 1)), dim3(256), 0, s, false, static_cast<const float*>(part), d, E,
+                     ntb, static_cast<int>(L), maxc, d_wg);
   } else if (d_wg != nullptr) {
     const int ns = dwg_splits(T, d, E);
     const int tps = T > 0 ? (T + ns - 1) / ns : 0;

@@ -174,12 +174,14 @@ def test_full_size_combine_in_gemm_k1():
         torch.cuda.empty_cache()
 
 
-def test_full_size_router_backward():
-    """The router backward on the Mixtral router at full size (T = 4096,
-    d = 4096, E = 8, k = 2) from the GPU's own forward, against the oracle's
-    chain rule: d_logits, dx and dWg."""
+@pytest.mark.parametrize("name", ["mixtral", "capacity_skew"])
+def test_full_size_router_backward(name):
+    """The router backward at full size from the GPU's own forward, against
+    the oracle's chain rule (d_logits, dx and dWg): the Mixtral router (T =
+    4096, d = 4096, E = 8, k = 2) and the capacity workload's (T = 16384,
+    d = 1024, E = 64, k = 2: the tensor-core passes with K = 128)."""
     from mixture_experts_routing_route_b200 import _abi as abi
-    sh = CONFIGS["mixtral"]
+    sh = CONFIGS[name]
     inp = make_inputs(sh)
     T, d, E, k = sh.T, sh.d, sh.E, sh.k
     x, wg = inp.x.to("cuda"), inp.wg.to("cuda")

@@ -457,7 +457,7 @@ def test_route_train_at_unit_temperature_is_route(T, d, E, k, dt):
 @pytest.mark.parametrize("T,d,E,k,dt,tau,d_aux,d_z", [
     (1000, 1024, 8, 2, "bf16", 1.0, 0.01, 0.001),   # Mixtral's router shape at a reduced T
     (777, 512, 8, 2, "bf16", 0.7, 0.5, 0.0),        # temperature, no z-loss term
-    (513, 256, 64, 2, "bf16", 1.3, 0.1, 0.02),      # two 32-expert chunks
+    (513, 256, 64, 2, "bf16", 1.3, 0.1, 0.02),      # E = 64: K = 128, two swizzle atoms
     (129, 256, 256, 8, "bf16", 1.0, 0.05, 0.01),    # E = 256, k = 8
     (300, 512, 24, 3, "bf16", 2.0, 0.0, 0.1),       # E not a multiple of 32, no aux term
     (200, 64, 40, 4, "f32", 1.0, 0.3, 0.05),        # fp32 (dx in fp32)
@@ -468,6 +468,8 @@ def test_route_train_at_unit_temperature_is_route(T, d, E, k, dt):
     (4100, 256, 16, 3, "bf16", 0.8, 0.05, 0.0),     # 2 column tiles x 65 units: 22 blocks per tile
     (5462, 256, 8, 3, "bf16", 1.0, 0.2, 0.0),       # 16386 picks: thread per token, counts over a grid barrier
     (9000, 128, 16, 2, "bf16", 1.0, 0.0, 0.01),     # thread per token without the aux term (no barrier)
+    (2000, 1024, 32, 2, "bf16", 1.0, 0.05, 0.01),   # EC = 32: K = 64, one swizzle atom of [hi | lo]
+    (700, 384, 48, 4, "bf16", 0.9, 0.1, 0.0),       # EC = 64 with 16 zero columns; 128-column dx tiles
     (300, 64, 8, 2, "f32", 1.0, 0.1, 0.01),         # fp32, E = 8: CUDA-core passes
     (270000, 128, 8, 2, "bf16", 1.0, 0.01, 0.001),  # > 1024 x 256 tokens: grid-stride d_logits, 147 blocks on one tile
 ])
