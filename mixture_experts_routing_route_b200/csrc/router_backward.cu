@@ -17,7 +17,7 @@
 // Kernels: d_logits (fp32) by a warp per token after an expert histogram of
 // the picks (f, when d_aux != 0) for small T, or by a thread per token that
 // counts the picks in the same launch for large T. The two T x d passes run
-// on the tensor cores for bf16 with E <= 16 (bwd_dx_tc, bwd_dwg_tc: d_logits
+// on the tensor cores for bf16 with E <= 64 (bwd_dx_tc, bwd_dwg_tc: d_logits
 // enters as bf16 hi + lo terms, products summed in fp32), otherwise on CUDA
 // cores in fp32 (bwd_dx; bwd_dwg_part + bwd_dwg_reduce). dWg is a sum of
 // partials added in a fixed order (deterministic); dx is rounded once to the
