@@ -360,6 +360,9 @@ int num_sms();
 // 2-D bf16 TMA map over [rows, cols] row-major, box [box_rows, 64 cols], 128-byte swizzle.
 bool make_tma_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
                       uint32_t box_rows);
+// Box [box_rows, box_cols] without swizzle (rows land back to back).
+bool make_tma_2d_bf16_plain(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                            uint32_t box_cols, uint32_t box_rows);
 // The same with a row stride of ld elements (ld * 2 a multiple of 16 bytes).
 bool make_tma_2d_bf16_ld(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
                          uint32_t box_rows);

@@ -884,6 +884,23 @@ bool make_tma_2d_bf16_ld(CUtensorMap* m, const void* base, uint64_t rows, uint64
   return r == CUDA_SUCCESS;
 }
 
+// 2-D bf16 map over [rows, cols] row-major (cols * 2 a multiple of 16), box
+// [box_rows, box_cols], no swizzle: a box lands as box_rows rows of
+// box_cols * 2 bytes, back to back.
+bool make_tma_2d_bf16_plain(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                            uint32_t box_cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // 2-D bf16 map over [rows, cols] row-major, box [box_rows, 64 cols], 128-B swizzle.
 bool make_tma_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
                       uint32_t box_rows) {

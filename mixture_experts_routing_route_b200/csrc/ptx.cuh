@@ -329,6 +329,20 @@ __device__ __forceinline__ uint64_t make_sw128_desc(uint32_t smem_addr, uint32_t
   return d;
 }
 
+// Shared-memory matrix descriptor, no swizzle (layout 0), MN-major operand:
+// core matrices of 8 MN elements (16 bytes) x 8 K rows, the 8 rows 16 bytes
+// apart (one contiguous 128-byte block); LBO = byte stride between core
+// matrices along K, SBO = byte stride between 8-element MN blocks.
+__device__ __forceinline__ uint64_t make_noswz_desc(uint32_t smem_addr, uint32_t lbo_bytes,
+                                                    uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B, fp32 D, A K-major,
 // B MN-major (or K-major when b_k_major), shape M x N.
 __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool b_k_major = false) {

@@ -1135,13 +1135,22 @@ router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
 }
 
 // Persistent fused router, d unsplit (KS = 1), for more token tiles than
-// SMs: one CTA per SM stages Wg^T once and walks the tiles blockIdx.x,
-// blockIdx.x + gridDim.x, ... Six warps: warp 0 (one thread) streams x
-// k-blocks of all its tiles through the ring, warp 1 (one thread) issues the
-// MMAs of tile j into accumulator j % 2 (two of 256 tensor-memory columns),
-// warps 2-5 (thread = token row; warp w reads lane quarter w % 4) run the
-// selection and aux partials of tile j while tile j + 1 loads and multiplies.
-// Same arithmetic as router_tc's fused path with KS = 1.
+// SMs: one CTA per SM walks the tiles blockIdx.x, blockIdx.x + gridDim.x, ...
+// Six warps: warp 0 (one thread) streams x k-blocks of all its tiles through
+// the ring, warp 1 (one thread) issues the MMAs of tile j into accumulator
+// j % 2 (two of 256 tensor-memory columns), warps 2-5 (thread = token row;
+// warp w reads lane quarter w % 4) run the selection and aux partials of tile
+// j while tile j + 1 loads and multiplies. Same arithmetic as router_tc's
+// fused path with KS = 1.
+// Wg is not staged: each stage also carries its k-blocks' Wg rows, TMA-loaded
+// as E/8 boxes of 8 experts x 64 rows (1 KB each, no swizzle, packed E/8 KB
+// per k-block) that the MMA reads as its MN-major operand (8-row core
+// matrices 16 bytes wide, 128 bytes apart along K, 1 KB apart along N). An
+// MMA of N = Epad > E also reads the (Epad - E)/8 KB after its k-block's
+// boxes (the next k-block's, or the 1 KB of slack after the ring) into
+// accumulator columns that nothing reads. Without the 64 KB of staged Wg^T
+// (d = 4096, E = 8) the ring holds a third 64 KB stage, and the stream runs
+// with more bytes in flight per SM.
 constexpr int kPersistThreads = 192;
 constexpr int kPersistAccCols = 256;
 
@@ -1151,7 +1160,8 @@ __device__ __forceinline__ void epi_bar_sync() {  // the four selection warps
 
 template <int EW>
 __global__ void __launch_bounds__(kPersistThreads, 1)
-router_tc_persist(const __grid_constant__ CUtensorMap tmX, RouterTcArgs a) {
+router_tc_persist(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                  RouterTcArgs a) {
   pdl_begin();
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kTcStages], empty_bar[kTcStages];
@@ -1165,14 +1175,12 @@ router_tc_persist(const __grid_constant__ CUtensorMap tmX, RouterTcArgs a) {
   constexpr uint32_t kBoxBytes = 128 * 128;  // one k-block of 128 token rows
   const int sub = a.sub;                     // k-blocks per stage (divides nkb)
   const int nkg = nkb / sub;                 // stage loads per tile
-  const uint32_t stage_bytes = kBoxBytes * sub;
+  const uint32_t wkb_bytes = static_cast<uint32_t>(a.E / 8) * 1024;  // one k-block's Wg boxes
+  const uint32_t xs_bytes = kBoxBytes * sub;
+  const uint32_t stage_bytes = xs_bytes + wkb_bytes * sub;           // a multiple of 1024
   const int nst = a.stages;
   uint8_t* ring = smem;
-  uint8_t* wgt = smem + nst * stage_bytes;
-  // k-block kb's E rows at kb * E * 128 bytes; the padding rows E..Epad-1 the
-  // MMA also reads are the next block's (or the 1 KB slack), as in router_tc.
-  const uint32_t wgt_kb_bytes = static_cast<uint32_t>(a.E) * 128;
-  uint8_t* scratch = wgt + static_cast<size_t>(a.d) * a.E * 2 + 1024;
+  uint8_t* scratch = smem + nst * stage_bytes + 1024;  // after 1 KB of slack
   const int nslot_cap = kPersistAccCols / a.Epad;
   const int G = (nkb + nslot_cap - 1) / nslot_cap;  // k-blocks per accumulator slot
   const int nslot = (nkb + G - 1) / G;
@@ -1187,10 +1195,14 @@ router_tc_persist(const __grid_constant__ CUtensorMap tmX, RouterTcArgs a) {
   auto issue = [&](int i) {
     const int j = i / nkg, kg = i - j * nkg, st = i % nst;
     const int tile = static_cast<int>(blockIdx.x) + j * static_cast<int>(gridDim.x);
+    uint8_t* sa = ring + st * stage_bytes;
     mbar_arrive_expect_tx(&full_bar[st], stage_bytes);
     for (int u = 0; u < sub; ++u)
-      tma_load_2d(ring + st * stage_bytes + u * kBoxBytes, &tmX, &full_bar[st], (kg * sub + u) * 64,
-                  tile * 128);
+      tma_load_2d(sa + u * kBoxBytes, &tmX, &full_bar[st], (kg * sub + u) * 64, tile * 128);
+    for (int u = 0; u < sub; ++u)
+      for (int n8 = 0; n8 < a.E / 8; ++n8)
+        tma_load_2d(sa + xs_bytes + u * wkb_bytes + n8 * 1024, &tmW, &full_bar[st], n8 * 8,
+                    (kg * sub + u) * 64);
   };
   if (threadIdx.x == 0) {
     for (int s = 0; s < nst; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
@@ -1198,41 +1210,13 @@ router_tc_persist(const __grid_constant__ CUtensorMap tmX, RouterTcArgs a) {
     mbar_init(&done_bar, 1);
     fence_mbar_init();
     prefetch_tmap(&tmX);
-    for (int i = 0; i < pre; ++i) issue(i);  // the ring's first round, before the staging
+    prefetch_tmap(&tmW);
+    for (int i = 0; i < pre; ++i) issue(i);  // the ring's first round
   }
   if (warp == 1) {
     tmem_alloc(&tmem_base_s, 2 * kPersistAccCols);
     tmem_relinquish();
   }
-  // Wg^T staging by all threads: task = 8 d-rows x 8 experts, transposed with
-  // byte permutes into the K-major 128-byte-swizzled rows (see router_tc).
-  {
-    const int nchunk = a.d / 8, groups = a.E / 8, ntask = nchunk * groups;
-    for (int i = threadIdx.x; i < ntask; i += kPersistThreads) {
-      const int g = i / nchunk, ch = i - g * nchunk;
-      uint32_t in[8][4];
-#pragma unroll
-      for (int rr = 0; rr < 8; ++rr) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(a.wg + static_cast<size_t>(ch * 8 + rr) * a.E) + g);
-        in[rr][0] = u.x;
-        in[rr][1] = u.y;
-        in[rr][2] = u.z;
-        in[rr][3] = u.w;
-      }
-      const int kb = ch >> 3, c = ch & 7;
-#pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        const int e = g * 8 + jj;
-        uint32_t o[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          o[q] = __byte_perm(in[2 * q][jj >> 1], in[2 * q + 1][jj >> 1], (jj & 1) ? 0x7632 : 0x5410);
-        const uint32_t off = kb * wgt_kb_bytes + e * 128 + (((c ^ e) & 7) << 4);
-        *reinterpret_cast<uint4*>(wgt + off) = make_uint4(o[0], o[1], o[2], o[3]);
-      }
-    }
-  }
-  fence_proxy_async_smem();  // generic-proxy writes, read by the tensor core
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1257,7 +1241,7 @@ router_tc_persist(const __grid_constant__ CUtensorMap tmX, RouterTcArgs a) {
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = make_idesc_bf16(128, a.Epad, true);  // staged Wg^T is K-major
+      const uint32_t idesc = make_idesc_bf16(128, a.Epad, false);  // Wg rows: MN-major
       bool issued = false, ok = true;
       int i = 0;
       for (int j = 0; j < my_tiles && ok; ++j) {
@@ -1276,14 +1260,16 @@ router_tc_persist(const __grid_constant__ CUtensorMap tmX, RouterTcArgs a) {
             break;
           }
           tc_fence_after();
+          const uint32_t s_addr = smem_u32(ring + st * stage_bytes);
           for (int u = 0; u < sub; ++u) {
             const int kb = kg * sub + u;
-            const uint32_t a_addr = smem_u32(ring + st * stage_bytes + u * kBoxBytes);
+            const uint32_t a_addr = s_addr + u * kBoxBytes;
+            const uint32_t b_addr = s_addr + xs_bytes + u * wkb_bytes;
             const uint32_t d_tmem = dbase + static_cast<uint32_t>((kb / G) * a.Epad);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t adesc = make_sw128_desc(a_addr + kk * 32, 16, 1024);
-              const uint64_t bdesc = make_sw128_desc(smem_u32(wgt) + kb * wgt_kb_bytes + kk * 32, 16, 1024);
+              const uint64_t bdesc = make_noswz_desc(b_addr + kk * 256, 128, 1024);
               umma_bf16(d_tmem, adesc, bdesc, idesc, ((kb % G) | kk) != 0 ? 1u : 0u);
             }
           }
@@ -1497,19 +1483,22 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, const
         a.part_p = part_p; a.part_c = part_c; a.aux = aux;
         a.noise = noise; a.part_z = part_z; a.z_out = z_out;
         if (tp.KS == 1 && tp.ntile > num_sms()) {
-          // persistent: one CTA per SM stages Wg^T once and walks the tiles
-          const size_t fixed = 1024 + static_cast<size_t>(d) * E * 2 + 1024 + tp.scratch;
+          // persistent: one CTA per SM walks the tiles
+          const size_t fixed = 1024 + 1024 + tp.scratch;  // alignment, slack, selection buffers
           const size_t budget = 227 * 1024 - 2048;  // dynamic shared memory next to the static
           // k-blocks per stage: 4 (each token row's 512 consecutive bytes requested
           // together, measured 14-20% faster than one k-block per stage at T =
           // 32768-65536), fewer if two such stages do not fit
+          const size_t kbytes = 16384 + static_cast<size_t>(E / 8) * 1024;  // x and Wg of one k-block
           int sub = 4;
-          while (sub > 1 && ((d / 64) % sub != 0 || fixed + 2 * 16384 * static_cast<size_t>(sub) > budget)) sub >>= 1;
-          const size_t sbytes = 16384 * static_cast<size_t>(sub);
+          while (sub > 1 && ((d / 64) % sub != 0 || fixed + 2 * kbytes * static_cast<size_t>(sub) > budget)) sub >>= 1;
+          const size_t sbytes = kbytes * static_cast<size_t>(sub);
+          CUtensorMap tw2;
           const int st = fixed + 2 * sbytes <= budget
                              ? static_cast<int>(std::min<size_t>(kTcStages, (budget - fixed) / sbytes))
                              : 0;
-          if (st >= 2) {
+          if (st >= 2 && (reinterpret_cast<uintptr_t>(wg) & 15u) == 0 &&
+              make_tma_2d_bf16_plain(&tw2, wg, static_cast<uint64_t>(d), E, 8, 64)) {
             // at least 120 KB, so that no two CTAs share an SM (each takes all
             // 512 tensor-memory columns)
             const size_t smem = std::max<size_t>(fixed + static_cast<size_t>(st) * sbytes, 120 * 1024);
@@ -1519,7 +1508,7 @@ cudaError_t launch_route(const void* x, const void* wg, const float* bias, const
                     : tp.fuse_e == 16 ? router_tc_persist<16> : router_tc_persist<32>;
             cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
             return launch_pdl(pk, dim3(std::min(tp.ntile, num_sms())), dim3(kPersistThreads), smem, s,
-                              false, tx, a);
+                              false, tx, tw2, a);
           }
         }
         auto kern = tp.fuse_e == 8 ? router_tc<false, 8>
