@@ -677,19 +677,29 @@ struct DxTc {
 };
 static_assert(3 * (kDxTcSmem + 1024) > 228 * 1024, "at most two dx blocks per SM");
 
+// Barrier over the 128 threads of a dx group (named barrier 1), and the same
+// with an AND of a per-thread flag.
+__device__ __forceinline__ void dx_group_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ int dx_group_and(int v) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, 128, q;\n\tselp.s32 %0, 1, 0, p;\n\t}"
+      : "=r"(r) : "r"(v) : "memory");
+  return r;
+}
+
+// The body of bwd_dx_tc, run by threads 0..127 of a block (block bid of nblk
+// dx blocks; sm: the block's dynamic shared memory, 1024-aligned).
 template <int EC>
-__global__ void __launch_bounds__(kDxTcThreads, 2)
-bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, int T, int d, int E,
-          __nv_bfloat16* __restrict__ dx, Control* ctl) {
-  pdl_begin();
+__device__ __forceinline__ void dx_tc_body(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg,
+                                           int T, int d, int E, __nv_bfloat16* __restrict__ dx, Control* ctl,
+                                           uint8_t* sm, int bid, int nblk) {
   static_assert(EC == 8 || EC == 16 || EC == 32 || EC == 64, "EC");
   using C = DxTc<EC>;
   constexpr int TN = C::TN;
-  extern __shared__ uint8_t dx_raw[];
   __shared__ __align__(8) uint64_t mma_bar;
   __shared__ uint32_t tmem_s;
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dx_raw) + 1023) &
-                                           ~static_cast<uintptr_t>(1023));
   uint8_t* sa = sm;
   uint8_t* sb = sm + C::A_BYTES;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -706,7 +716,7 @@ bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, in
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  dx_group_sync();
   tc_fence_after();
   const uint32_t tmem = tmem_s;
   const uint64_t limit = wait_limit_ns(ctl);
@@ -714,11 +724,11 @@ bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, in
   const int total = ntt * nct;
   constexpr uint32_t kIdesc = make_idesc_bf16(kDxTcTok, TN, true);
   float g[EC];
-  if (static_cast<int>(blockIdx.x) < total) load_row<EC>(dl, (blockIdx.x / nct) * kDxTcTok + tid, T, E, g);
+  if (bid < total) load_row<EC>(dl, (bid / nct) * kDxTcTok + tid, T, E, g);
   int cur_ct = -1;
   uint32_t phase = 0;
   bool pending = false;  // an MMA was issued and not yet waited for
-  for (int u = blockIdx.x; u < total; u += gridDim.x) {
+  for (int u = bid; u < total; u += nblk) {
     const int tt = u / nct, ct = u - tt * nct;
     // A row tid: chunks [hi 0..EC) then [lo 0..EC), 8 values each
 #pragma unroll
@@ -757,7 +767,7 @@ bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, in
     }
     fence_proxy_async_smem();  // the generic-proxy writes above, before the MMA reads them
     tc_fence_before();
-    __syncthreads();
+    dx_group_sync();
     tc_fence_after();
     if (tid == 0) {
       const uint32_t a_addr = smem_u32(sa), b_addr = smem_u32(sb);
@@ -770,12 +780,12 @@ bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, in
     }
     pending = true;
     // the next tile's d_logits rows are in flight during this tile's stores
-    const int un = u + gridDim.x;
+    const int un = u + nblk;
     if (un < total) load_row<EC>(dl, (un / nct) * kDxTcTok + tid, T, E, g);
     int ok = 0;
     if (lane == 0) ok = mbar_wait_bounded(&mma_bar, phase, limit);
     ok = __shfl_sync(kFull, ok, 0);
-    if (!__syncthreads_and(ok)) {
+    if (!dx_group_and(ok)) {
       if (tid == 0) set_error(ctl, MOE_DEVERR_TIMEOUT);
       break;
     }
@@ -822,11 +832,22 @@ bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, in
   }
   if (pending && tid == 0) (void)mbar_wait_bounded(&mma_bar, phase, limit);
   tc_fence_before();
-  __syncthreads();
+  dx_group_sync();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, TN);
   }
+}
+
+template <int EC>
+__global__ void __launch_bounds__(kDxTcThreads, 2)
+bwd_dx_tc(const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, int T, int d, int E,
+          __nv_bfloat16* __restrict__ dx, Control* ctl) {
+  pdl_begin();
+  extern __shared__ uint8_t dx_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dx_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  dx_tc_body<EC>(dl, wg, T, d, E, dx, ctl, sm, blockIdx.x, gridDim.x);
 }
 
 // dWg on the tensor cores, per 128-column tile of x: D[c, n] = sum_t x[t, c]
@@ -867,16 +888,18 @@ struct DwgTc {
   static constexpr size_t SMEM = static_cast<size_t>(STAGES) * STAGE + 1024;
 };
 
-template <int EC>
-__global__ void __launch_bounds__(kDwgTcThreads, 1)
-bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmg, int d,
-           int E, int ntb, int total, int L, int maxc, float* __restrict__ part,
-           int* __restrict__ tickets, float* __restrict__ d_wg, Control* ctl) {
-  pdl_begin();
+// The body of bwd_dwg_tc for block bid with an NST-stage ring, run by all
+// kDwgTcThreads threads of a block (dwg_raw: its dynamic shared memory,
+// before alignment).
+template <int EC, int NST>
+__device__ __forceinline__ void dwg_tc_body(const CUtensorMap* tmx_p, const CUtensorMap* tmg_p, int d,
+                                            int E, int ntb, int total, int L, int maxc,
+                                            float* __restrict__ part, int* __restrict__ tickets,
+                                            float* __restrict__ d_wg, Control* ctl, uint8_t* dwg_raw,
+                                            int bid) {
   using C = DwgTc<EC>;
   static_assert(C::STAGE % 1024 == 0, "stage alignment");
-  static_assert(C::STAGES <= kMaxDwgStages, "ring barriers");
-  extern __shared__ uint8_t dwg_raw[];
+  static_assert(NST <= kMaxDwgStages, "ring barriers");
   __shared__ __align__(8) uint64_t full[kMaxDwgStages], empty[kMaxDwgStages];
   __shared__ __align__(8) uint64_t tfull[2], tempty[2], drain;
   __shared__ uint32_t tmem_s;
@@ -884,10 +907,10 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dwg_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int u0 = blockIdx.x * L, u1 = min(total, u0 + L);
+  const int u0 = bid * L, u1 = min(total, u0 + L);
   const uint64_t limit = wait_limit_ns(ctl);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::STAGES; ++i) {
+    for (int i = 0; i < NST; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
@@ -910,8 +933,8 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
 
   if (warp == 0) {
     if (lane == 0) {
-      prefetch_tmap(&tmx);
-      prefetch_tmap(&tmg);
+      prefetch_tmap(tmx_p);
+      prefetch_tmap(tmg_p);
       int stage = 0;
       uint32_t phase = 0, issued_mask = 0, last_parity = 0;
       for (int u = u0; u < u1 && !abort_s; ++u) {
@@ -923,17 +946,17 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
         }
         uint8_t* sa = sm + stage * C::STAGE;
         mbar_arrive_expect_tx(&full[stage], C::STAGE);
-        tma_load_2d(sa, &tmx, &full[stage], j * kDwgTcCols, tb * kDwgTcTok);
-        tma_load_2d(sa + C::A_BYTES / 2, &tmx, &full[stage], j * kDwgTcCols + 64, tb * kDwgTcTok);
-        tma_load_2d(sa + C::A_BYTES, &tmg, &full[stage], tb * kDwgTcTok, 0);
+        tma_load_2d(sa, tmx_p, &full[stage], j * kDwgTcCols, tb * kDwgTcTok);
+        tma_load_2d(sa + C::A_BYTES / 2, tmx_p, &full[stage], j * kDwgTcCols + 64, tb * kDwgTcTok);
+        tma_load_2d(sa + C::A_BYTES, tmg_p, &full[stage], tb * kDwgTcTok, 0);
         issued_mask |= 1u << stage;
         last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-        if (++stage == C::STAGES) {
+        if (++stage == NST) {
           stage = 0;
           phase ^= 1u;
         }
       }
-      for (int s = 0; s < C::STAGES; ++s)
+      for (int s = 0; s < NST; ++s)
         if ((issued_mask >> s) & 1u)
           if (!mbar_wait_bounded(&full[s], (last_parity >> s) & 1u, limit)) set_error(ctl, MOE_DEVERR_TIMEOUT);
     }
@@ -974,7 +997,7 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
                       (u != us || kk != 0) ? 1u : 0u);
           issued_any = true;
           umma_commit(&empty[stage]);
-          if (++stage == C::STAGES) {
+          if (++stage == NST) {
             stage = 0;
             phase ^= 1u;
           }
@@ -1043,7 +1066,7 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
       // this block's rank among the tile's blocks, and their number
       const int first = static_cast<int>((static_cast<long long>(j) * ntb) / L);
       const int last = static_cast<int>((static_cast<long long>(j + 1) * ntb - 1) / L);
-      const int i = blockIdx.x - first, n = last - first + 1;
+      const int i = bid - first, n = last - first + 1;
       const int r = q * 32 + lane;
       float* mine = part + ((static_cast<size_t>(j) * maxc + i) * kDwgTcCols + r) * EC;
 #pragma unroll
@@ -1098,6 +1121,46 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM);
+  }
+}
+
+template <int EC>
+__global__ void __launch_bounds__(kDwgTcThreads, 1)
+bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmg, int d,
+           int E, int ntb, int total, int L, int maxc, float* __restrict__ part,
+           int* __restrict__ tickets, float* __restrict__ d_wg, Control* ctl) {
+  pdl_begin();
+  extern __shared__ uint8_t dwg_smem[];
+  dwg_tc_body<EC, DwgTc<EC>::STAGES>(&tmx, &tmg, d, E, ntb, total, L, maxc, part, tickets, d_wg, ctl,
+                                      dwg_smem, blockIdx.x);
+}
+
+// dx and dWg in one launch (bf16, EC <= 16, both requested): blocks
+// [0, ndwg) run the dWg body with a 4-stage ring, the rest the dx body on
+// threads 0..127 (threads 128.. of those blocks have nothing to do). The
+// shared memory (kDxTcSmem) and tensor memory (256 + 64 columns) of one block
+// of each kind fit one SM together, so every SM streams x for dWg and writes
+// dx at the same time; at small T each pass alone is latency-bound.
+constexpr int kFusedDwgStages = 4;
+
+template <int EC>
+__global__ void __launch_bounds__(kDwgTcThreads, 2)
+bwd_dxdwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmg, int d,
+             int E, int ntb, int total, int L, int maxc, float* __restrict__ part,
+             int* __restrict__ tickets, float* __restrict__ d_wg, int ndwg,
+             const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, int T,
+             __nv_bfloat16* __restrict__ dx, Control* ctl) {
+  pdl_begin();
+  static_assert(kFusedDwgStages * DwgTc<EC>::STAGE + 1024 <= static_cast<int>(kDxTcSmem), "fused smem");
+  extern __shared__ uint8_t both_smem[];
+  if (static_cast<int>(blockIdx.x) < ndwg) {
+    dwg_tc_body<EC, kFusedDwgStages>(&tmx, &tmg, d, E, ntb, total, L, maxc, part, tickets, d_wg, ctl,
+                                     both_smem, blockIdx.x);
+  } else if (threadIdx.x < kDxTcThreads) {
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(both_smem) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    dx_tc_body<EC>(dl, wg, T, d, E, dx, ctl, sm, static_cast<int>(blockIdx.x) - ndwg,
+                   static_cast<int>(gridDim.x) - ndwg);
   }
 }
 
@@ -1255,7 +1318,9 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
                      tc_dwg && ec <= 16 ? tickets : nullptr, dwg_tc_tiles(d) * 4, ctl);
     if (err != cudaSuccess) return err;
   }
-  if (T > 0) {
+  // both passes requested, EC <= 16: one launch runs them side by side
+  const bool fuse = tc && dx != nullptr && d_wg != nullptr && ec <= 16;
+  if (T > 0 && !fuse) {
     if (dx != nullptr && tc) {
       const int tn = ec <= 32 ? DxTc<8>::TN : DxTc<64>::TN;
       const int nct = (d + tn - 1) / tn;
@@ -1282,6 +1347,7 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
   }
   if (tc_dwg) {
     // equal shares of 64-token x 128-column units; L keeps a tile's blocks <= maxc
+    // (with the fused launch: of one block per SM beside the dx blocks)
     const int ntb = (T + kDwgTcTok - 1) / kDwgTcTok;
     const int nct = dwg_tc_tiles(d);
     const int maxc = dwg_max_contrib(nct);
@@ -1295,6 +1361,19 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
         !make_tma_2d_bf16_ld(&tmg, dlT, static_cast<uint64_t>(2 * ec), static_cast<uint64_t>(T),
                              static_cast<uint64_t>(dlt_ld(T)), static_cast<uint32_t>(2 * ec)))
       return cudaErrorInvalidValue;
+    if (fuse) {
+      const int tn = DxTc<8>::TN;
+      const int nct_x = (d + tn - 1) / tn;
+      const int tiles = ((T + kDxTcTok - 1) / kDxTcTok) * nct_x;
+      const int sms = num_sms();
+      const int gx = std::max(1, std::min(tiles, nct_x <= sms ? sms / nct_x * nct_x : sms));
+      auto kf = ec == 8 ? bwd_dxdwg_tc<8> : bwd_dxdwg_tc<16>;
+      cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kDxTcSmem));
+      return launch_pdl(kf, dim3(G + gx), dim3(kDwgTcThreads), kDxTcSmem, s, false, tmx, tmg, d, E, ntb,
+                        static_cast<int>(total), static_cast<int>(L), maxc, part, tickets, d_wg, G,
+                        static_cast<const float*>(dl), static_cast<const __nv_bfloat16*>(wg), T,
+                        static_cast<__nv_bfloat16*>(dx), ctl);
+    }
     const size_t smem = ec == 8 ? DwgTc<8>::SMEM : ec == 16 ? DwgTc<16>::SMEM
                       : ec == 32 ? DwgTc<32>::SMEM : DwgTc<64>::SMEM;
     auto kern = ec == 8 ? bwd_dwg_tc<8> : ec == 16 ? bwd_dwg_tc<16> : ec == 32 ? bwd_dwg_tc<32> : bwd_dwg_tc<64>;

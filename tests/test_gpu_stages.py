@@ -509,6 +509,42 @@ def test_route_backward(T, d, E, k, dt, tau, d_aux, d_z):
     assert max_err_ratio(np32(dx), ref["dx"]) <= (TOL_BF16_OUT if dt == "bf16" else 1e-5)
 
 
+@pytest.mark.parametrize("T,d,E", [(3000, 1024, 8), (777, 512, 16)])
+def test_route_backward_one_output(T, d, E):
+    """With both dx and d_wg requested (bf16, E <= 16) the two tensor-core
+    passes run in one launch; asked for one of them, each runs alone. Same
+    arithmetic and the same dWg split, so the results are bit-identical."""
+    k = 2
+    inp = small_case("rb1", T=T, d=d, E=E, k=k, F=128, act="gelu", dtype="bf16", bias="zipf", seed=T + E)
+    x, wg, b = inp.x.to(DEV), inp.wg.to(DEV), inp.bias.to(DEV)
+    idx = torch.empty(T, k, dtype=torch.int32, device=DEV)
+    w = torch.empty(T, k, dtype=torch.float32, device=DEV)
+    aux = torch.empty(1, dtype=torch.float32, device=DEV)
+    logits = torch.empty(T, E, dtype=torch.float32, device=DEV)
+    probs = torch.empty(T, E, dtype=torch.float32, device=DEV)
+    ws = new_ws(abi.moe_route_workspace_size(T, d, E))
+    abi.moe_route_train(x, wg, b, None, T, d, E, k, idx, w, aux, None, logits, probs, ws)
+    g = torch.from_numpy(np.random.default_rng(T).standard_normal((T, k)).astype(np.float32)).to(DEV)
+    bws = new_ws(abi.moe_route_backward_workspace_size(T, d, E))
+    res = {}
+    for name, want_dx, want_wg in (("both", True, True), ("dx", True, False), ("wg", False, True)):
+        dl = torch.empty(T, E, dtype=torch.float32, device=DEV)
+        dx = torch.full((T, d), 7.0, dtype=x.dtype, device=DEV) if want_dx else None
+        d_wg = torch.full((d, E), 7.0, dtype=torch.float32, device=DEV) if want_wg else None
+        abi.moe_route_backward(x, wg, T, d, E, k, probs, logits, idx, w, g, 0.05, 0.01, 1.0, dl, dx, d_wg, bws)
+        torch.cuda.synchronize()
+        assert abi.moe_get_device_error(bws) == 0
+        res[name] = (dl, dx, d_wg)
+    assert torch.equal(res["both"][0], res["dx"][0]) and torch.equal(res["both"][0], res["wg"][0])
+    assert torch.equal(res["both"][1], res["dx"][1])
+    assert torch.equal(res["both"][2], res["wg"][2])
+    ref = O.route_backward_from(np32(probs).astype(np.float64), npi(idx), np32(w).astype(np.float64),
+                                np32(logits).astype(np.float64), np32(inp.x), np32(inp.wg),
+                                d_w=np32(g).astype(np.float64), d_aux=0.05, d_z=0.01)
+    assert max_err_ratio(np32(res["both"][2]), ref["dwg"]) <= 1e-4
+    assert max_err_ratio(np32(res["both"][1]), ref["dx"]) <= TOL_BF16_OUT
+
+
 def test_pair_gemm_repeats_on_one_workspace():
     """The CTA-pair GEMM hands out its tiles from a counter in the
     workspace's control block, reset by the last pair of each launch: three
