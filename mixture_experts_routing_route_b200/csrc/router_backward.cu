@@ -883,6 +883,8 @@ struct DwgTc {
   static constexpr int B_BYTES = N * kDwgTcTok * 2;
   static constexpr int STAGE = A_BYTES + B_BYTES;              // a multiple of 1024
   static constexpr int STAGES = EC <= 32 ? kDwgTcStages : 6;
+  // beside a dx block (bwd_dxdwg_tc): what fits in kDxTcSmem
+  static constexpr int FUSED_STAGES = EC <= 16 ? 4 : (EC == 32 ? 3 : 2);
   static constexpr int ACC = N < 32 ? 32 : N;                  // tensor-memory columns per accumulator
   static constexpr int TMEM = 2 * ACC;                         // a power of two >= 64
   static constexpr size_t SMEM = static_cast<size_t>(STAGES) * STAGE + 1024;
@@ -1135,13 +1137,13 @@ bwd_dwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUte
                                       dwg_smem, blockIdx.x);
 }
 
-// dx and dWg in one launch (bf16, EC <= 16, both requested): blocks
-// [0, ndwg) run the dWg body with a 4-stage ring, the rest the dx body on
-// threads 0..127 (threads 128.. of those blocks have nothing to do). The
-// shared memory (kDxTcSmem) and tensor memory (256 + 64 columns) of one block
-// of each kind fit one SM together, so every SM streams x for dWg and writes
-// dx at the same time; at small T each pass alone is latency-bound.
-constexpr int kFusedDwgStages = 4;
+// dx and dWg in one launch (bf16, both requested): blocks [0, ndwg) run the
+// dWg body with a shorter ring (DwgTc<EC>::FUSED_STAGES), the rest the dx
+// body on threads 0..127 (threads 128.. of those blocks have nothing to do).
+// The shared memory (kDxTcSmem) and tensor memory (at most 384 columns) of
+// one block of each kind fit one SM together, so every SM streams x for dWg
+// and writes dx at the same time; at small T each pass alone is
+// latency-bound.
 
 template <int EC>
 __global__ void __launch_bounds__(kDwgTcThreads, 2)
@@ -1151,10 +1153,11 @@ bwd_dxdwg_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
              const float* __restrict__ dl, const __nv_bfloat16* __restrict__ wg, int T,
              __nv_bfloat16* __restrict__ dx, Control* ctl) {
   pdl_begin();
-  static_assert(kFusedDwgStages * DwgTc<EC>::STAGE + 1024 <= static_cast<int>(kDxTcSmem), "fused smem");
+  static_assert(DwgTc<EC>::FUSED_STAGES * DwgTc<EC>::STAGE + 1024 <= static_cast<int>(kDxTcSmem), "fused smem");
+  static_assert(DxTc<EC>::TN + DwgTc<EC>::TMEM <= 512, "fused tensor memory");
   extern __shared__ uint8_t both_smem[];
   if (static_cast<int>(blockIdx.x) < ndwg) {
-    dwg_tc_body<EC, kFusedDwgStages>(&tmx, &tmg, d, E, ntb, total, L, maxc, part, tickets, d_wg, ctl,
+    dwg_tc_body<EC, DwgTc<EC>::FUSED_STAGES>(&tmx, &tmg, d, E, ntb, total, L, maxc, part, tickets, d_wg, ctl,
                                      both_smem, blockIdx.x);
   } else if (threadIdx.x < kDxTcThreads) {
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(both_smem) + 1023) &
@@ -1318,7 +1321,9 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
                      tc_dwg && ec <= 16 ? tickets : nullptr, dwg_tc_tiles(d) * 4, ctl);
     if (err != cudaSuccess) return err;
   }
-  // both passes requested, EC <= 16: one launch runs them side by side
+  // both passes requested, EC <= 16: one launch runs them side by side (for
+  // EC = 64 the 2-stage dWg ring that fits beside a dx block measured slower
+  // than the two launches: 70.8 against 63.5 us on the capacity workload)
   const bool fuse = tc && dx != nullptr && d_wg != nullptr && ec <= 16;
   if (T > 0 && !fuse) {
     if (dx != nullptr && tc) {
@@ -1361,18 +1366,27 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
         !make_tma_2d_bf16_ld(&tmg, dlT, static_cast<uint64_t>(2 * ec), static_cast<uint64_t>(T),
                              static_cast<uint64_t>(dlt_ld(T)), static_cast<uint32_t>(2 * ec)))
       return cudaErrorInvalidValue;
+    auto launch_reduce = [&]() -> cudaError_t {
+      const long long nout = static_cast<long long>(d) * (ec / 4);
+      const int rg = static_cast<int>(std::min<long long>((nout + 255) / 256, 8LL * num_sms()));
+      auto red = ec == 32 ? bwd_dwg_tc_reduce<32> : bwd_dwg_tc_reduce<64>;
+      return launch_pdl(red, dim3(std::max(rg, 1)), dim3(256), 0, s, false, static_cast<const float*>(part), d, E,
+                        ntb, static_cast<int>(L), maxc, d_wg);
+    };
     if (fuse) {
-      const int tn = DxTc<8>::TN;
+      const int tn = ec <= 32 ? DxTc<8>::TN : DxTc<64>::TN;
       const int nct_x = (d + tn - 1) / tn;
       const int tiles = ((T + kDxTcTok - 1) / kDxTcTok) * nct_x;
       const int sms = num_sms();
       const int gx = std::max(1, std::min(tiles, nct_x <= sms ? sms / nct_x * nct_x : sms));
-      auto kf = ec == 8 ? bwd_dxdwg_tc<8> : bwd_dxdwg_tc<16>;
+      auto kf = ec == 8 ? bwd_dxdwg_tc<8> : ec == 16 ? bwd_dxdwg_tc<16> : ec == 32 ? bwd_dxdwg_tc<32> : bwd_dxdwg_tc<64>;
       cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kDxTcSmem));
-      return launch_pdl(kf, dim3(G + gx), dim3(kDwgTcThreads), kDxTcSmem, s, false, tmx, tmg, d, E, ntb,
-                        static_cast<int>(total), static_cast<int>(L), maxc, part, tickets, d_wg, G,
-                        static_cast<const float*>(dl), static_cast<const __nv_bfloat16*>(wg), T,
-                        static_cast<__nv_bfloat16*>(dx), ctl);
+      err = launch_pdl(kf, dim3(G + gx), dim3(kDwgTcThreads), kDxTcSmem, s, false, tmx, tmg, d, E, ntb,
+                       static_cast<int>(total), static_cast<int>(L), maxc, part, ec <= 16 ? tickets : nullptr,
+                       d_wg, G, static_cast<const float*>(dl), static_cast<const __nv_bfloat16*>(wg), T,
+                       static_cast<__nv_bfloat16*>(dx), ctl);
+      if (err != cudaSuccess || ec <= 16) return err;
+      return launch_reduce();
     }
     const size_t smem = ec == 8 ? DwgTc<8>::SMEM : ec == 16 ? DwgTc<16>::SMEM
                       : ec == 32 ? DwgTc<32>::SMEM : DwgTc<64>::SMEM;
@@ -1382,11 +1396,7 @@ cudaError_t launch_route_backward(const void* x, const void* wg, moe_dtype_t dt,
                      static_cast<int>(total), static_cast<int>(L), maxc, part,
                      ec <= 16 ? tickets : nullptr, d_wg, ctl);
     if (err != cudaSuccess || ec <= 16) return err;
-    const long long nout = static_cast<long long>(d) * (ec / 4);
-    const int rg = static_cast<int>(std::min<long long>((nout + 255) / 256, 8LL * num_sms()));
-    auto red = ec == 32 ? bwd_dwg_tc_reduce<32> : bwd_dwg_tc_reduce<64>;
-    err = launch_pdl(red, dim3(std::max(rg, 1)), dim3(256), 0, s, false, static_cast<const float*>(part), d, E,
-                     ntb, static_cast<int>(L), maxc, d_wg);
+    err = launch_reduce();
   } else if (d_wg != nullptr) {
     const int ns = dwg_splits(T, d, E);
     const int tps = T > 0 ? (T + ns - 1) / ns : 0;

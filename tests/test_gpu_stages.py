@@ -509,7 +509,7 @@ def test_route_backward(T, d, E, k, dt, tau, d_aux, d_z):
     assert max_err_ratio(np32(dx), ref["dx"]) <= (TOL_BF16_OUT if dt == "bf16" else 1e-5)
 
 
-@pytest.mark.parametrize("T,d,E", [(3000, 1024, 8), (777, 512, 16)])
+@pytest.mark.parametrize("T,d,E", [(3000, 1024, 8), (777, 512, 16), (700, 384, 48), (900, 256, 32)])
 def test_route_backward_one_output(T, d, E):
     """With both dx and d_wg requested (bf16, E <= 16) the two tensor-core
     passes run in one launch; asked for one of them, each runs alone. Same
