@@ -39,7 +39,7 @@ def route_on_gpu(x, wg, bias, T, d, E, k):
     (2000, 1024, 64, 2, "bf16", "zipf"),   # tensor cores, TMA Wg, one tile per CTA
     (97, 128, 128, 3, "bf16", "none"),     # tensor cores, 4 experts per lane
     (10000, 4096, 8, 2, "bf16", "expert0"),  # tensor cores, no d split: 64 k-blocks in 32 slots
-    (20000, 1024, 8, 2, "bf16", "zipf"),   # more tiles than SMs: persistent, Wg^T staged once per SM
+    (20000, 1024, 8, 2, "bf16", "zipf"),   # more tiles than SMs: the persistent kernel
     (24000, 512, 24, 3, "bf16", "none"),   # persistent, E = 24 (Epad 32: padding rows from the next k-block)
     (19000, 256, 16, 2, "bf16", "expert0"),  # persistent, E = 16, 149 tiles (one SM takes two)
     (1000, 1024, 24, 2, "bf16", "expert0"),  # E = 24, split over d in a cluster
