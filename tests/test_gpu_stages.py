@@ -469,6 +469,8 @@ def test_route_train_at_unit_temperature_is_route(T, d, E, k, dt):
     (5462, 256, 8, 3, "bf16", 1.0, 0.2, 0.0),       # 16386 picks: thread per token, counts over a grid barrier
     (9000, 128, 16, 2, "bf16", 1.0, 0.0, 0.01),     # thread per token without the aux term (no barrier)
     (2000, 1024, 32, 2, "bf16", 1.0, 0.05, 0.01),   # EC = 32: K = 64, one swizzle atom of [hi | lo]
+    (1, 128, 8, 2, "bf16", 1.0, 0.1, 0.01),         # one token: one dx tile, one dWg unit, mostly padding
+    (64, 256, 16, 1, "bf16", 1.0, 0.1, 0.0),        # exactly one 64-token dWg unit per column tile, k = 1
     (700, 384, 48, 4, "bf16", 0.9, 0.1, 0.0),       # EC = 64 with 16 zero columns; 128-column dx tiles
     (300, 64, 8, 2, "f32", 1.0, 0.1, 0.01),         # fp32, E = 8: CUDA-core passes
     (270000, 128, 8, 2, "bf16", 1.0, 0.01, 0.001),  # > 1024 x 256 tokens: grid-stride d_logits, 147 blocks on one tile
