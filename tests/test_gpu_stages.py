@@ -474,6 +474,8 @@ def test_route_train_at_unit_temperature_is_route(T, d, E, k, dt):
     (700, 384, 48, 4, "bf16", 0.9, 0.1, 0.0),       # EC = 64 with 16 zero columns; 128-column dx tiles
     (300, 64, 8, 2, "f32", 1.0, 0.1, 0.01),         # fp32, E = 8: CUDA-core passes
     (270000, 128, 8, 2, "bf16", 1.0, 0.01, 0.001),  # > 1024 x 256 tokens: grid-stride d_logits, 147 blocks on one tile
+    (7001, 128, 24, 2, "bf16", 1.0, 0.2, 0.0),      # 14002 picks, E = 24: one counting block, warp-per-token d_logits
+    (8192, 128, 20, 2, "bf16", 1.0, 0.1, 0.01),     # 16384 picks: the largest count taken by one block
 ])
 def test_route_backward(T, d, E, k, dt, tau, d_aux, d_z):
     """moe_route_backward from the GPU's own forward (moe_route_train at tau)
