@@ -32,7 +32,10 @@ def route_on_gpu(x, wg, bias, T, d, E, k):
     (1000, 512, 8, 2, "bf16", "none"),     # fused E <= 8 path
     (77, 4096, 8, 2, "bf16", "expert0"),   # fused, d = 4096, ragged quad
     (300, 256, 5, 3, "bf16", "none"),      # fused with E < 8 (padded experts)
-    (513, 256, 64, 2, "bf16", "zipf"),     # tiled GEMM + select, 2 experts per lane
+    (513, 256, 64, 2, "bf16", "zipf"),     # tensor cores, TMA Wg + router_select, 2 experts per lane
+    (700, 256, 64, 8, "bf16", "none"),     # E = 64, k = 8: eight warp arg-max rounds
+    (300, 4096, 64, 2, "bf16", "zipf"),    # E = 64, d = 4096 split over KS CTAs (partials added in ks order)
+    (20000, 512, 64, 2, "bf16", "expert0"),  # E = 64, more token tiles than SMs
     (129, 256, 256, 8, "bf16", "none"),    # tensor cores, TMA Wg, 8 experts per lane, k = 8
     (300, 512, 16, 2, "bf16", "zipf"),     # tensor cores, staged Wg^T (E <= 32)
     (1000, 1024, 32, 4, "bf16", "none"),   # tensor cores, staged Wg^T, split over d
@@ -399,6 +402,7 @@ def test_router_noise_matches_oracle(T, E):
     (300, 512, 32, 4, "bf16", 3.0),
     (513, 256, 64, 2, "bf16", 1.0),     # tensor cores (TMA Wg) + router_select + aux_reduce
     (513, 256, 64, 2, "bf16", 0.5),
+    (300, 256, 128, 2, "bf16", 0.8),    # the same at E = 128 (4 experts per lane)
     (90, 64, 40, 4, "f32", 1.5),        # CUDA-core gate + router_select
     (200, 64, 4, 1, "f32", 1.0),        # fp32 E <= 8: the general path when noise / z-loss are asked
     (200, 64, 4, 1, "f32", 2.5),
