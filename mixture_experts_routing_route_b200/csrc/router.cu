@@ -420,10 +420,25 @@ router_gemm_tiled(const Tin* __restrict__ x, const Tin* __restrict__ wg, int T, 
   }
 }
 
+// An unsigned key with the order of the float v: sign-magnitude to offset
+// binary. -0 is taken as +0 first, so keys are equal exactly when the floats
+// compare equal; NaN gets key 0, below every number (never selected, as a
+// comparison would not select it).
+__device__ __forceinline__ uint32_t order_key(float v) {
+  if (v != v) return 0u;
+  const uint32_t u = v == 0.0f ? 0u : __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
 // One token's routing by one warp: lane l holds the logits (bias included) of
 // experts l + 32q, q < EPL (-inf for e >= E). Softmax over E, top-k by k
 // rounds of a warp arg-max (ties to the lower expert), renormalised weights;
 // accumulates the token's probabilities and choices into the lane's aux sums.
+// A round's arg-max is two warp reductions: the largest key of the lanes'
+// best untaken logits, then the lowest expert among the lanes that hold it.
 template <int EPL>
 __device__ __forceinline__ float warp_route_token(const float (&v)[EPL], int E, int k, int lane,
                                                  size_t t, int32_t* __restrict__ idx_out,
@@ -437,11 +452,10 @@ __device__ __forceinline__ float warp_route_token(const float (&v)[EPL], int E, 
     const int e = lane + 32 * q;
     if (logits_out != nullptr && e < E) logits_out[t * E + e] = v[q];
   }
-  float m = -INFINITY;
+  uint32_t mk = 0;
 #pragma unroll
-  for (int q = 0; q < EPL; ++q) m = fmaxf(m, v[q]);
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+  for (int q = 0; q < EPL; ++q) mk = max(mk, order_key(v[q]));
+  const float m = key_value(__reduce_max_sync(kFull, mk));
   float ex[EPL], s = 0.f;
 #pragma unroll
   for (int q = 0; q < EPL; ++q) {
@@ -467,19 +481,18 @@ __device__ __forceinline__ float warp_route_token(const float (&v)[EPL], int E, 
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     if (j < k) {
-      float bv = -INFINITY;
+      // the lane's best untaken expert (q ascending, strict >: ties keep the
+      // lower expert); key 0 is below every logit's key and means none
+      uint32_t bk = 0;
       int be = 0x7fffffff;
 #pragma unroll
       for (int q = 0; q < EPL; ++q) {
         const int e = lane + 32 * q;
-        if (e < E && !((taken >> q) & 1u) && better(v[q], e, bv, be)) { bv = v[q]; be = e; }
+        const uint32_t key = order_key(v[q]);
+        if (e < E && !((taken >> q) & 1u) && key > bk) { bk = key; be = e; }
       }
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) {
-        const float ov = __shfl_xor_sync(kFull, bv, off);
-        const int oe = __shfl_xor_sync(kFull, be, off);
-        if (better(ov, oe, bv, be)) { bv = ov; be = oe; }
-      }
+      const uint32_t wk = __reduce_max_sync(kFull, bk);
+      be = static_cast<int>(__reduce_min_sync(kFull, bk == wk ? static_cast<uint32_t>(be) : 0xffffffffu));
       if (be >= E || be < 0) {
         if (lane == 0) set_error(ctl, MOE_DEVERR_EXPERT_RANGE);
         be = 0;
