@@ -80,7 +80,10 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
 typedef enum { MOE_ACT_GELU = 0, MOE_ACT_SWIGLU = 1 } moe_act_t;
 
 /* Bits of the device error word. */
-#define MOE_DEVERR_EXPERT_RANGE 0x1u /* a top-k expert id outside [0, E) */
+#define MOE_DEVERR_EXPERT_RANGE 0x1u /* a top-k expert id outside [0, E), or a router
+                                        row with fewer than k selectable logits
+                                        (NaN is never selected); expert 0 is
+                                        written in that pick's place */
 #define MOE_DEVERR_ROW_RANGE 0x2u    /* a slot/row index outside its buffer */
 #define MOE_DEVERR_TIMEOUT 0x4u      /* a bounded on-chip wait gave up */
 
