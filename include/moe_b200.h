@@ -281,8 +281,9 @@ MOE_API moe_status_t moe_route_train(const void* x, const void* w_router, const 
  * d must be a multiple of 4 (MOE_ERR_UNSUPPORTED otherwise). d_logits is
  * computed in fp32. dx and d_wg: for bf16 with E <= 64 (16-byte aligned x,
  * w_router and d_logits) on the tensor cores, d_logits entering as two bf16
- * terms hi = bf16(v), lo = bf16(v - hi) (|v - hi - lo| <= 2^-17 |v|) and the
- * products summed in fp32; otherwise fp32 on CUDA cores. d_wg adds its
+ * terms hi = bf16(v), lo = bf16(v - hi) (|v - hi - lo| <= 2^-17 |v| for
+ * |v| >= 2^-117, <= 2^-134 below, where v - hi leaves bf16's normal range)
+ * and the products summed in fp32; otherwise fp32 on CUDA cores. d_wg adds its
  * partial sums in a fixed order (deterministic). */
 MOE_API size_t moe_route_backward_workspace_size(int T, int d, int E);
 MOE_API moe_status_t moe_route_backward(const void* x, const void* w_router, moe_dtype_t dtype,

@@ -626,7 +626,8 @@ bwd_dwg_part(const T* __restrict__ x, const float* __restrict__ dl, int Tn, int 
 // (K = E) and dWg = x^T dL/dl (K = T, N = E). On the tensor cores the bf16
 // operands are exact; d_logits is fp32, so it enters as two bf16 terms,
 // hi = bf16(v) and lo = bf16(v - hi), which together keep 16 bits of it
-// (|v - hi - lo| <= 2^-17 |v|); both products are summed in the fp32
+// (|v - hi - lo| <= 2^-17 |v| for |v| >= 2^-117, <= 2^-134 below); both
+// products are summed in the fp32
 // accumulator. EC is E rounded up to 8 or 16 (missing experts are zeros);
 // the contraction has 2 EC terms per output: [hi | lo] against [W | W].
 //
