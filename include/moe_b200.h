@@ -278,7 +278,8 @@ MOE_API moe_status_t moe_route_train(const void* x, const void* w_router, const 
  *   dx            out [T, d] (dtype, rounded once), or NULL
  *   d_wg          out [d, E] fp32, or NULL
  *   ws            >= moe_route_backward_workspace_size(T, d, E) bytes
- * d must be a multiple of 4 (MOE_ERR_UNSUPPORTED otherwise). d_logits is
+ * d follows the general limits above (a multiple of 128 for bf16, of 4 for
+ * fp32; MOE_ERR_UNSUPPORTED otherwise). d_logits is
  * computed in fp32. dx and d_wg: for bf16 with E <= 64 (16-byte aligned x,
  * w_router and d_logits) on the tensor cores, d_logits entering as two bf16
  * terms hi = bf16(v), lo = bf16(v - hi) (|v - hi - lo| <= 2^-17 |v| for
