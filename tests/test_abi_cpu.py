@@ -122,6 +122,11 @@ def test_argument_checks_return_before_launch(abi):
                                        1.0, 1.0, None, None, None, 16, 1 << 30, None) == 1  # d_z needs logits
     assert abi._lib.moe_route_backward(16, 16, abi.MOE_BF16, 8, 128, 8, 2, 16, None, 16, 16, None, 0.0,
                                        0.0, 1.0, None, None, None, 16, 16, None) == 4
+    # router backward: d limits as everywhere (bf16 d % 128, fp32 d % 4)
+    assert abi._lib.moe_route_backward(16, 16, abi.MOE_BF16, 8, 96, 8, 2, 16, None, 16, 16, None, 0.0,
+                                       0.0, 1.0, None, None, None, 16, 1 << 30, None) == 3
+    assert abi._lib.moe_route_backward(16, 16, abi.MOE_F32, 8, 66, 8, 2, 16, None, 16, 16, None, 0.0,
+                                       0.0, 1.0, None, None, None, 16, 1 << 30, None) == 3
     assert abi.moe_route_backward_workspace_size(4096, 4096, 8) >= 4096 * 8 * 4
     assert abi.moe_kernel_launches() == n0
 
